@@ -1,0 +1,199 @@
+/*
+ * lf_attention.h -- C ABI of the B200 Longformer self-attention library.
+ *
+ * The library computes the Longformer attention forward on one GPU:
+ * each non-global query attends to a sliding window of keys (w/2 taps per
+ * side, or w taps to the left when causal), the taps spaced by a per-head
+ * dilation, plus every global token; each global query attends to the whole
+ * sequence through its own projections Qg, Kg, Vg; padded query rows are zero.
+ *
+ * Sources:
+ *   "LongFormer: The Long-Document Transformer" (reading notes), sections
+ *     "Sliding Window", "Dilated Sliding Window", "Global Attention", and the
+ *     part on autoregressive language models;
+ *   FasterTransformer Longformer Encoder guide, sections "four hard
+ *     constraints" (head size 64) and "Longformer Encoder compute flow"
+ *     (global-index extraction, local/global softmax, zeroed masked rows).
+ *
+ * Conventions for every entry point:
+ *   - Device pointers point to memory of the current CUDA device; host
+ *     pointers are marked "host".  The caller owns every buffer; the library
+ *     allocates no memory and keeps no pointer after a call returns.
+ *   - Tensors are contiguous and row-major.  Inputs are never modified.
+ *   - Work is queued asynchronously on `stream` (a cudaStream_t passed as a
+ *     void*, NULL = the legacy default stream).  No entry point synchronises
+ *     the stream except lf_workspace_status and lf_attention_forward_host.
+ *   - Host-detectable errors return a negative lf_status before anything is
+ *     launched.  No C++ exception crosses this interface.
+ *   - Errors found on the device (a count of global tokens above max_global,
+ *     a bounded wait that ran out) are recorded in a status word inside the
+ *     workspace; the output is then undefined.  Read it with
+ *     lf_workspace_status.
+ *   - All calls are thread-compatible: concurrent calls must use distinct
+ *     workspaces and outputs.
+ */
+#ifndef LF_ATTENTION_H
+#define LF_ATTENTION_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LF_API __attribute__((visibility("default")))
+#else
+#define LF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, passed untyped so this header needs no CUDA header. */
+typedef void *lf_stream_t;
+
+typedef enum {
+    LF_F32 = 0,   /* fp32 in, fp32 arithmetic, fp32 out */
+    LF_F16 = 1,   /* fp16 in, fp32 accumulation, fp16 out */
+    LF_BF16 = 2   /* bf16 in, fp32 accumulation, bf16 out */
+} lf_dtype;
+
+typedef enum {
+    LF_OK = 0,
+    LF_ERR_INVALID_ARG = -1,      /* bad size, pointer, window or dilation */
+    LF_ERR_UNSUPPORTED = -2,      /* d_head != 64; causal with global tokens */
+    LF_ERR_WORKSPACE = -3,        /* workspace NULL, misaligned or too small */
+    LF_ERR_CUDA = -4,             /* a CUDA runtime call failed */
+    LF_ERR_DEVICE_TIMEOUT = -5,   /* a bounded device-side wait ran out */
+    LF_ERR_GLOBAL_OVERFLOW = -6,  /* a batch has more global tokens than max_global */
+    LF_ERR_NO_DEVICE = -7         /* no sm_100 device is current */
+} lf_status;
+
+/* Library version, major*10000 + minor*100 + patch. */
+LF_API int lf_version(void);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+LF_API const char *lf_status_string(int status);
+
+/*
+ * Global-token index extraction (FasterTransformer Longformer Encoder guide,
+ * compute flow: the global mask of each batch is compacted into the list of
+ * its global positions and their count).
+ *
+ *   global_mask  device uint8 [B, n]; nonzero marks a global token.
+ *   global_idx   device int32 [B, n]; out: row b holds the global positions of
+ *                batch b in ascending order, then -1 up to n.
+ *   counts       device int32 [B]; out: number of global tokens per batch.
+ *
+ * Returns LF_ERR_INVALID_ARG for B < 1, n < 1 or a NULL pointer.
+ */
+LF_API int lf_global_index(const uint8_t *global_mask, int B, int n,
+                    int32_t *global_idx, int32_t *counts, lf_stream_t stream);
+
+/*
+ * Workspace bytes needed by lf_attention_prepare / lf_attention_run /
+ * lf_attention_forward for these sizes (0 on invalid sizes).  The workspace
+ * must be 256-byte aligned device memory; it needs no initialisation.
+ * It holds the compacted global indices, per-batch validity and global
+ * bitmaps, the fp32 partial results of the global rows, and a status word.
+ */
+LF_API size_t lf_workspace_size(int B, int H, int n, int d_head, int max_global);
+
+/*
+ * Mask preprocessing, once per set of masks (shared by every layer that uses
+ * the same masks).  Compacts the global mask (as lf_global_index), builds the
+ * per-batch bitmaps of valid keys and of global tokens, clears the status
+ * word.
+ *
+ *   local_mask   device uint8 [B, n]; 1 (nonzero) = valid token, 0 = padding.
+ *                NULL: every token valid.
+ *   global_mask  device uint8 [B, n]; nonzero = global token.  NULL: none.
+ *   max_global   host upper bound on the global tokens of any batch (sizes
+ *                grids without a device-to-host copy); 0 when there are none.
+ *                A batch above it sets LF_ERR_GLOBAL_OVERFLOW in the status word.
+ */
+LF_API int lf_attention_prepare(int B, int H, int n, int d_head,
+                         const uint8_t *local_mask, const uint8_t *global_mask,
+                         int max_global, void *workspace, size_t workspace_bytes,
+                         lf_stream_t stream);
+
+/*
+ * The attention itself, on a workspace prepared by lf_attention_prepare with
+ * the same B, H, n, d_head, max_global and masks.
+ *
+ *   dtype        element type of all seven tensors.
+ *   q, k, v      device [B, H, n, d_head]: the sliding-window projections.
+ *   qg, kg, vg   device [B, H, n, d_head]: the global projections; qg is read
+ *                only at global rows.  May alias q, k, v.
+ *   window       w.  Non-causal: even, >= 2; taps i + t*dil[h] for
+ *                t in [-w/2, w/2].  Causal: >= 1; taps i - t*dil[h] for
+ *                t in [0, w-1].  Taps outside [0, n) are dropped.
+ *   dilation     host int32 [H], every entry >= 1.  NULL: all 1.
+ *   causal       0 or 1.  Causal attention with global tokens is
+ *                LF_ERR_UNSUPPORTED (rejected by lf_attention_prepare's
+ *                caller-visible max_global: pass max_global = 0 and a NULL
+ *                global mask).
+ *   out          device [B, H, n, d_head], same dtype.  Every row is written:
+ *                padded rows with zeros.  Must not alias an input.
+ *
+ * Key set of a valid, non-global row i of head h in batch b:
+ *   (window taps of i  UNION  global tokens of b)  INTERSECT  valid tokens of b
+ * with softmax over s * <q_i, k_j>, s = 1/sqrt(d_head), applied to v_j.
+ * A valid global row attends to every valid token with qg, kg, vg.
+ * Inputs must be finite everywhere, padded positions included.
+ */
+LF_API int lf_attention_run(lf_dtype dtype, int B, int H, int n, int d_head,
+                     const void *q, const void *k, const void *v,
+                     const void *qg, const void *kg, const void *vg,
+                     int max_global, int window, const int32_t *dilation, int causal,
+                     void *out, void *workspace, size_t workspace_bytes,
+                     lf_stream_t stream);
+
+/*
+ * lf_attention_prepare followed by lf_attention_run: the whole forward.
+ */
+LF_API int lf_attention_forward(lf_dtype dtype, int B, int H, int n, int d_head,
+                         const void *q, const void *k, const void *v,
+                         const void *qg, const void *kg, const void *vg,
+                         const uint8_t *local_mask, const uint8_t *global_mask,
+                         int max_global, int window, const int32_t *dilation, int causal,
+                         void *out, void *workspace, size_t workspace_bytes,
+                         lf_stream_t stream);
+
+/*
+ * The whole forward from HOST buffers: copies the six projections and the
+ * masks from host memory (pinned memory makes the copies asynchronous) into
+ * caller-provided device staging buffers, runs lf_attention_forward, copies
+ * the output back to host memory and synchronises the stream.
+ *
+ *   h_q ... h_vg    host [B, H, n, d_head] of dtype.
+ *   h_local_mask, h_global_mask   host uint8 [B, n] or NULL.
+ *   h_out           host [B, H, n, d_head] of dtype; out.
+ *   d_staging       device buffer of lf_host_staging_size(...) bytes,
+ *                   256-byte aligned, which receives the copies.
+ *   workspace       as for lf_attention_forward.
+ *
+ * Returns the status of the run or, after the synchronisation, the status
+ * word of the workspace.
+ */
+LF_API size_t lf_host_staging_size(lf_dtype dtype, int B, int H, int n, int d_head);
+LF_API int lf_attention_forward_host(lf_dtype dtype, int B, int H, int n, int d_head,
+                              const void *h_q, const void *h_k, const void *h_v,
+                              const void *h_qg, const void *h_kg, const void *h_vg,
+                              const uint8_t *h_local_mask, const uint8_t *h_global_mask,
+                              int max_global, int window, const int32_t *dilation,
+                              int causal, void *h_out, void *d_staging,
+                              size_t staging_bytes, void *workspace,
+                              size_t workspace_bytes, lf_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns the device status word of `workspace`
+ * (LF_OK, LF_ERR_GLOBAL_OVERFLOW or LF_ERR_DEVICE_TIMEOUT), or LF_ERR_CUDA if
+ * the synchronisation or the copy failed.
+ */
+LF_API int lf_workspace_status(const void *workspace, lf_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LF_ATTENTION_H */

@@ -1,0 +1,15 @@
+"""Longformer self-attention forward on B200 (sm_100a).
+
+The compute path is the CUDA library under ``csrc/`` behind the C ABI
+``include/lf_attention.h``; ``api`` is its thin Python binding.  Importing this
+package loads nothing; the first API call loads the library and raises if it
+is missing.
+"""
+from .api import (attention_forward, attention_forward_host, attention_prepare, attention_run,
+                  global_index, host_staging_size, new_workspace, workspace_size,
+                  workspace_status)
+from ._lib import LfError
+
+__all__ = ["attention_forward", "attention_forward_host", "attention_prepare", "attention_run",
+           "global_index", "host_staging_size", "new_workspace", "workspace_size",
+           "workspace_status", "LfError"]

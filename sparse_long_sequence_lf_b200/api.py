@@ -1,0 +1,175 @@
+"""Python binding of the C ABI in include/lf_attention.h.
+
+Argument marshalling only: shapes and dtypes are checked, pointers and the
+current CUDA stream are handed to the library, and every step of the
+attention runs in the library's CUDA kernels.  PyTorch provides device memory
+and streams.  There is no CPU fallback: without the built library (or
+without an sm_100 GPU) every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import LF_BF16, LF_F16, LF_F32, LfError
+
+D_HEAD = 64
+_DTYPES = {torch.float32: LF_F32, torch.float16: LF_F16, torch.bfloat16: LF_BF16}
+
+
+def _stream_ptr(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _mask(m, B, n, name):
+    if m is None:
+        return None
+    if m.dtype == torch.bool:
+        m = m.view(torch.uint8)
+    if m.dtype != torch.uint8:
+        raise TypeError(f"{name} must be uint8 or bool")
+    if tuple(m.shape) != (B, n) or not m.is_contiguous() or not m.is_cuda:
+        raise ValueError(f"{name} must be a contiguous CUDA tensor of shape [B, n]")
+    return m
+
+
+def _dilation(dilation, H):
+    if dilation is None:
+        return None
+    vals = [int(x) for x in (dilation.tolist() if hasattr(dilation, "tolist") else dilation)]
+    if len(vals) != H:
+        raise ValueError("dilation must have one entry per head")
+    return (ctypes.c_int32 * H)(*vals)
+
+
+def _check_projections(tensors):
+    q = tensors[0]
+    if q.dtype not in _DTYPES:
+        raise TypeError("projections must be float32, float16 or bfloat16")
+    if q.dim() != 4 or q.shape[-1] != D_HEAD:
+        raise ValueError("projections must have shape [B, H, n, 64]")
+    for t in tensors:
+        if t.dtype != q.dtype or t.shape != q.shape:
+            raise ValueError("all projections must share dtype and shape")
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("projections must be contiguous CUDA tensors")
+    return _DTYPES[q.dtype], q.shape
+
+
+def workspace_size(B: int, H: int, n: int, max_global: int) -> int:
+    size = _lib.lib().lf_workspace_size(B, H, n, D_HEAD, max_global)
+    if size == 0:
+        raise LfError(-1, "lf_workspace_size")
+    return int(size)
+
+
+def new_workspace(B: int, H: int, n: int, max_global: int, device=None) -> torch.Tensor:
+    return torch.empty(workspace_size(B, H, n, max_global), dtype=torch.uint8,
+                       device=device or "cuda")
+
+
+def global_index(global_mask: torch.Tensor, stream=None):
+    """Compacted global positions per batch (ascending, -1 padded) and counts."""
+    B, n = global_mask.shape
+    gm = _mask(global_mask, B, n, "global_mask")
+    gidx = torch.empty((B, n), dtype=torch.int32, device=gm.device)
+    counts = torch.empty((B,), dtype=torch.int32, device=gm.device)
+    _lib.check(_lib.lib().lf_global_index(_ptr(gm), B, n, _ptr(gidx), _ptr(counts),
+                                          _stream_ptr(stream)), "lf_global_index")
+    return gidx, counts
+
+
+def default_max_global(global_mask) -> int:
+    """Upper bound of global tokens per batch read from the mask (syncs)."""
+    if global_mask is None:
+        return 0
+    return int((global_mask != 0).sum(dim=1).max().item())
+
+
+def attention_prepare(local_mask, global_mask, *, B, H, n, max_global, workspace, stream=None):
+    lm = _mask(local_mask, B, n, "local_mask")
+    gm = _mask(global_mask, B, n, "global_mask")
+    _lib.check(_lib.lib().lf_attention_prepare(B, H, n, D_HEAD, _ptr(lm), _ptr(gm), max_global,
+                                               _ptr(workspace), workspace.numel(),
+                                               _stream_ptr(stream)), "lf_attention_prepare")
+
+
+def attention_run(q, k, v, qg, kg, vg, *, window, dilation=None, causal=False, max_global,
+                  workspace, out=None, stream=None):
+    dt, (B, H, n, _) = _check_projections([q, k, v, qg, kg, vg])
+    if out is None:
+        out = torch.empty_like(q)
+    _check_projections([q, out])
+    _lib.check(_lib.lib().lf_attention_run(dt, B, H, n, D_HEAD, _ptr(q), _ptr(k), _ptr(v),
+                                           _ptr(qg), _ptr(kg), _ptr(vg), max_global, int(window),
+                                           _dilation(dilation, H), int(bool(causal)), _ptr(out),
+                                           _ptr(workspace), workspace.numel(),
+                                           _stream_ptr(stream)), "lf_attention_run")
+    return out
+
+
+def attention_forward(q, k, v, qg, kg, vg, local_mask=None, global_mask=None, *, window,
+                      dilation=None, causal=False, max_global=None, out=None, workspace=None,
+                      stream=None):
+    """Longformer attention forward; returns out [B, H, n, 64] in the input dtype.
+
+    max_global: host upper bound on the global tokens of any batch; when None
+    it is read from global_mask (one device-to-host sync).
+    """
+    dt, (B, H, n, _) = _check_projections([q, k, v, qg, kg, vg])
+    lm = _mask(local_mask, B, n, "local_mask")
+    gm = _mask(global_mask, B, n, "global_mask")
+    if max_global is None:
+        max_global = default_max_global(gm)
+    if workspace is None:
+        workspace = new_workspace(B, H, n, max_global, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_projections([q, out])
+    _lib.check(_lib.lib().lf_attention_forward(
+        dt, B, H, n, D_HEAD, _ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg), _ptr(vg), _ptr(lm),
+        _ptr(gm), int(max_global), int(window), _dilation(dilation, H), int(bool(causal)),
+        _ptr(out), _ptr(workspace), workspace.numel(), _stream_ptr(stream)),
+        "lf_attention_forward")
+    return out
+
+
+def host_staging_size(dtype: torch.dtype, B: int, H: int, n: int) -> int:
+    return int(_lib.lib().lf_host_staging_size(_DTYPES[dtype], B, H, n, D_HEAD))
+
+
+def attention_forward_host(q, k, v, qg, kg, vg, local_mask=None, global_mask=None, *, window,
+                           dilation=None, causal=False, max_global, out, staging, workspace,
+                           stream=None):
+    """The whole forward from host (ideally pinned) tensors: copies in, runs,
+    copies the output back into the host tensor ``out`` and synchronises."""
+    q0 = q
+    if q0.dtype not in _DTYPES or q0.dim() != 4 or q0.shape[-1] != D_HEAD:
+        raise ValueError("projections must be [B, H, n, 64] of a supported dtype")
+    B, H, n, _ = q0.shape
+    for t in (k, v, qg, kg, vg, out):
+        if t.is_cuda or t.shape != q0.shape or t.dtype != q0.dtype or not t.is_contiguous():
+            raise ValueError("host tensors must be contiguous CPU tensors of one shape/dtype")
+    for m in (local_mask, global_mask):
+        if m is not None and (m.is_cuda or m.dtype not in (torch.uint8, torch.bool)
+                              or tuple(m.shape) != (B, n) or not m.is_contiguous()):
+            raise ValueError("host masks must be contiguous uint8 CPU tensors of shape [B, n]")
+    rc = _lib.lib().lf_attention_forward_host(
+        _DTYPES[q0.dtype], B, H, n, D_HEAD, _ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg),
+        _ptr(vg), _ptr(local_mask), _ptr(global_mask), int(max_global), int(window),
+        _dilation(dilation, H), int(bool(causal)), _ptr(out), _ptr(staging), staging.numel(),
+        _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _lib.check(rc, "lf_attention_forward_host")
+    return out
+
+
+def workspace_status(workspace, stream=None) -> int:
+    """Synchronises the stream and returns the device status word."""
+    return int(_lib.lib().lf_workspace_status(_ptr(workspace), _stream_ptr(stream)))

@@ -1,0 +1,248 @@
+// C ABI of the Longformer attention library: argument checks, workspace
+// layout, kernel dispatch.  Declared in include/lf_attention.h.
+#include <cmath>
+#include <cstring>
+
+#include "../../include/lf_attention.h"
+#include "lf_device.cuh"
+
+namespace lf {
+int launch_prepare(const uint8_t *local_mask, const uint8_t *global_mask, int B, int n,
+                   int max_global, int32_t *gidx, int32_t *counts, int *flags, uint32_t *vbits,
+                   uint32_t *gbits, int *status, int *counters, int counters_per_batch,
+                   cudaStream_t stream);
+template <typename T> int launch_simt(const AttnArgs &a, cudaStream_t stream);
+int launch_tc(lf_dtype dtype, const AttnArgs &a, cudaStream_t stream);
+}  // namespace lf
+
+using namespace lf;
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+int device_ok()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return kErrNoDevice;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return kErrNoDevice;
+    return major == 10 ? kOk : kErrNoDevice;
+}
+
+bool sizes_ok(int B, int H, int n)
+{
+    if (B < 1 || H < 1 || n < 1 || H > kMaxHeads) return false;
+    // Offsets inside one tensor are computed in 64-bit, positions in 32-bit.
+    return double(B) * H * n * kDHead < 9.0e18 && n < (1 << 30);
+}
+
+size_t elem_size(lf_dtype dt)
+{
+    switch (dt) {
+        case LF_F32: return 4;
+        case LF_F16: return 2;
+        case LF_BF16: return 2;
+    }
+    return 0;
+}
+
+int check_workspace(const void *ws, size_t bytes, const WsLayout &L)
+{
+    if (ws == nullptr) return kErrWorkspace;
+    if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return kErrWorkspace;
+    if (bytes < L.total) return kErrWorkspace;
+    return kOk;
+}
+
+}  // namespace
+
+extern "C" {
+
+int lf_version(void) { return kVersion; }
+
+const char *lf_status_string(int status)
+{
+    switch (status) {
+        case LF_OK: return "ok";
+        case LF_ERR_INVALID_ARG: return "invalid argument";
+        case LF_ERR_UNSUPPORTED: return "unsupported configuration";
+        case LF_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case LF_ERR_CUDA: return "CUDA runtime error";
+        case LF_ERR_DEVICE_TIMEOUT: return "bounded device-side wait ran out";
+        case LF_ERR_GLOBAL_OVERFLOW: return "more global tokens than max_global";
+        case LF_ERR_NO_DEVICE: return "no sm_100 device is current";
+    }
+    return "unknown status";
+}
+
+int lf_global_index(const uint8_t *global_mask, int B, int n, int32_t *global_idx,
+                    int32_t *counts, lf_stream_t stream)
+{
+    if (B < 1 || n < 1 || !global_mask || !global_idx || !counts) return LF_ERR_INVALID_ARG;
+    if (int rc = device_ok()) return rc;
+    return launch_prepare(nullptr, global_mask, B, n, n, global_idx, counts, nullptr, nullptr,
+                          nullptr, nullptr, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
+size_t lf_workspace_size(int B, int H, int n, int d_head, int max_global)
+{
+    if (!sizes_ok(B, H, n) || d_head != kDHead || max_global < 0 || max_global > n) return 0;
+    return ws_layout(B, H, n, max_global).total;
+}
+
+int lf_attention_prepare(int B, int H, int n, int d_head, const uint8_t *local_mask,
+                         const uint8_t *global_mask, int max_global, void *workspace,
+                         size_t workspace_bytes, lf_stream_t stream)
+{
+    if (d_head != kDHead) return LF_ERR_UNSUPPORTED;
+    if (!sizes_ok(B, H, n) || max_global < 0 || max_global > n) return LF_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(B, H, n, max_global);
+    if (int rc = check_workspace(workspace, workspace_bytes, L)) return rc;
+    if (int rc = device_ok()) return rc;
+    WsPtrs p = ws_ptrs(workspace, L);
+    return launch_prepare(local_mask, global_mask, B, n, max_global, p.gidx, p.counts, p.flags,
+                          p.vbits, p.gbits, p.status, p.counters, H * (L.ngroups + 1),
+                          static_cast<cudaStream_t>(stream));
+}
+
+int lf_attention_run(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
+                     const void *k, const void *v, const void *qg, const void *kg, const void *vg,
+                     int max_global, int window, const int32_t *dilation, int causal, void *out,
+                     void *workspace, size_t workspace_bytes, lf_stream_t stream)
+{
+    if (d_head != kDHead) return LF_ERR_UNSUPPORTED;
+    if (elem_size(dtype) == 0) return LF_ERR_INVALID_ARG;
+    if (!sizes_ok(B, H, n) || max_global < 0 || max_global > n) return LF_ERR_INVALID_ARG;
+    if (!q || !k || !v || !qg || !kg || !vg || !out) return LF_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return LF_ERR_INVALID_ARG;
+    if (causal) {
+        if (window < 1) return LF_ERR_INVALID_ARG;
+        if (max_global != 0) return LF_ERR_UNSUPPORTED;
+    } else if (window < 2 || (window % 2) != 0) {
+        return LF_ERR_INVALID_ARG;
+    }
+    if (dilation)
+        for (int h = 0; h < H; ++h)
+            if (dilation[h] < 1) return LF_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(B, H, n, max_global);
+    if (int rc = check_workspace(workspace, workspace_bytes, L)) return rc;
+    if (int rc = device_ok()) return rc;
+
+    AttnArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = q; a.k = k; a.v = v; a.qg = qg; a.kg = kg; a.vg = vg;
+    a.out = out;
+    a.L = L;
+    a.ws = ws_ptrs(workspace, L);
+    a.B = B; a.H = H; a.n = n;
+    a.window = window;
+    a.half = window / 2;
+    a.causal = causal;
+    a.max_global = max_global;
+    a.scale_log2 = float(1.4426950408889634 / std::sqrt(double(kDHead)));
+    int items = 0;
+    for (int h = 0; h < H; ++h) {
+        const int dil = dilation ? dilation[h] : 1;
+        a.dil[h] = dil;
+        a.head_prefix[h] = items;
+        for (int r = 0; r < dil && r < n; ++r) {
+            const int n_r = (n - r + dil - 1) / dil;
+            items += (n_r + 127) / 128;
+        }
+    }
+    a.head_prefix[H] = items;
+    a.band_items_per_batch = items;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    switch (dtype) {
+        case LF_F32: return launch_simt<float>(a, s);
+        case LF_F16: return launch_tc(LF_F16, a, s);
+        case LF_BF16: return launch_tc(LF_BF16, a, s);
+    }
+    return LF_ERR_INVALID_ARG;
+}
+
+int lf_attention_forward(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
+                         const void *k, const void *v, const void *qg, const void *kg,
+                         const void *vg, const uint8_t *local_mask, const uint8_t *global_mask,
+                         int max_global, int window, const int32_t *dilation, int causal,
+                         void *out, void *workspace, size_t workspace_bytes, lf_stream_t stream)
+{
+    // Argument checks of the run come first so nothing is launched on error.
+    if (d_head != kDHead) return LF_ERR_UNSUPPORTED;
+    if (causal && max_global != 0) return LF_ERR_UNSUPPORTED;
+    int rc = lf_attention_prepare(B, H, n, d_head, local_mask, global_mask, max_global,
+                                  workspace, workspace_bytes, stream);
+    if (rc != LF_OK) return rc;
+    return lf_attention_run(dtype, B, H, n, d_head, q, k, v, qg, kg, vg, max_global, window,
+                            dilation, causal, out, workspace, workspace_bytes, stream);
+}
+
+size_t lf_host_staging_size(lf_dtype dtype, int B, int H, int n, int d_head)
+{
+    if (!sizes_ok(B, H, n) || d_head != kDHead || elem_size(dtype) == 0) return 0;
+    const size_t t = lf_align256(size_t(B) * H * n * kDHead * elem_size(dtype));
+    const size_t m = lf_align256(size_t(B) * n);
+    return 7 * t + 2 * m;
+}
+
+int lf_attention_forward_host(lf_dtype dtype, int B, int H, int n, int d_head, const void *h_q,
+                              const void *h_k, const void *h_v, const void *h_qg,
+                              const void *h_kg, const void *h_vg, const uint8_t *h_local_mask,
+                              const uint8_t *h_global_mask, int max_global, int window,
+                              const int32_t *dilation, int causal, void *h_out, void *d_staging,
+                              size_t staging_bytes, void *workspace, size_t workspace_bytes,
+                              lf_stream_t stream)
+{
+    const size_t need = lf_host_staging_size(dtype, B, H, n, d_head);
+    if (need == 0) return d_head != kDHead ? LF_ERR_UNSUPPORTED : LF_ERR_INVALID_ARG;
+    if (!h_q || !h_k || !h_v || !h_qg || !h_kg || !h_vg || !h_out) return LF_ERR_INVALID_ARG;
+    if (!d_staging || staging_bytes < need || reinterpret_cast<uintptr_t>(d_staging) % 256)
+        return LF_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t tb = size_t(B) * H * n * kDHead * elem_size(dtype);
+    const size_t t = lf_align256(tb);
+    const size_t mb = size_t(B) * n;
+    const size_t m = lf_align256(mb);
+    char *base = static_cast<char *>(d_staging);
+    const void *src[6] = {h_q, h_k, h_v, h_qg, h_kg, h_vg};
+    for (int i = 0; i < 6; ++i)
+        if (cudaMemcpyAsync(base + i * t, src[i], tb, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return LF_ERR_CUDA;
+    uint8_t *d_lm = nullptr, *d_gm = nullptr;
+    if (h_local_mask) {
+        d_lm = reinterpret_cast<uint8_t *>(base + 7 * t);
+        if (cudaMemcpyAsync(d_lm, h_local_mask, mb, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return LF_ERR_CUDA;
+    }
+    if (h_global_mask) {
+        d_gm = reinterpret_cast<uint8_t *>(base + 7 * t + m);
+        if (cudaMemcpyAsync(d_gm, h_global_mask, mb, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return LF_ERR_CUDA;
+    }
+    void *d_out = base + 6 * t;
+    int rc = lf_attention_forward(dtype, B, H, n, d_head, base, base + t, base + 2 * t,
+                                  base + 3 * t, base + 4 * t, base + 5 * t, d_lm, d_gm, max_global,
+                                  window, dilation, causal, d_out, workspace, workspace_bytes,
+                                  stream);
+    if (rc != LF_OK) return rc;
+    if (cudaMemcpyAsync(h_out, d_out, tb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return LF_ERR_CUDA;
+    return lf_workspace_status(workspace, stream);
+}
+
+int lf_workspace_status(const void *workspace, lf_stream_t stream)
+{
+    if (!workspace) return LF_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return LF_ERR_CUDA;
+    int status = 0;
+    // The status word sits at offset 0 of every workspace layout.
+    if (cudaMemcpy(&status, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return LF_ERR_CUDA;
+    return status;
+}
+
+}  // extern "C"
