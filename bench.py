@@ -1,0 +1,481 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the Longformer attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl b200|reference]
+
+One step is one pass of the whole hot path (global-index compaction and mask
+bitmaps, then band + global-column + global-row attention) over one batch of
+synthetic inputs already resident in HBM, launched through the C ABI.  Steps
+rotate over enough input sets that their total exceeds twice the L2 cache, and
+run from a CUDA graph so the host does not limit the launch rate.  K timed
+steps sit between a barrier plus device synchronisation on both sides; times
+come from CUDA events, the maximum over ranks.  Under torchrun every rank runs
+the same workload on its own GPU (independent (batch, head) work, no
+collective on the data path: weak scaling).
+
+Printed (rank 0, one JSON line): useful band+global TFLOP/s of the whole job,
+tokens/s, the roofline of the attention kernel against the measured HBM peak,
+the CPU oracle timed on this host, an end-to-end figure through the host-buffer
+entry point, clocks sampled around the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "useful band+global attention TFLOP/s & tokens/s at n=4096,w=512 bf16, 1 B200"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def reduce_max(value: float, device) -> float:
+    """Maximum of a float over all ranks (identity on one process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_step_per_rank: float, steps: int, world: int, max_ms: float) -> float:
+    """Units per second of the whole job: every rank's units over the slowest rank's time."""
+    return units_per_step_per_rank * steps * world / (max_ms * 1e-3)
+
+
+class ClockSampler:
+    """Samples SM clock, max clock and clock-event reasons through NVML."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.error = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.h = None
+            try:
+                props = torch.cuda.get_device_properties(device_index)
+                bus = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0),
+                                             props.pci_bus_id, props.pci_device_id)
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+                self.bus = bus
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+                self.bus = f"index {device_index}"
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        except Exception as e:  # NVML missing: report, do not guess
+            self.error = f"nvml unavailable: {e.__class__.__name__}"
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                sm = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = int(self._reasons(self.h))
+                self.samples.append((sm, rs))
+            except Exception as e:
+                self.error = f"nvml sample failed: {e.__class__.__name__}"
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.error is None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self, window: str):
+        if self.error is not None and not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "error": self.error}
+        loaded = [s for s in self.samples if not (s[1] & 0x1)] or self.samples
+        reasons = set()
+        for _, rs in loaded:
+            for bit, name in self.REASONS.items():
+                if rs & bit and bit != 0x1:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[0] for s in loaded), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(loaded), "window": window}
+
+
+# --------------------------------------------------------------- GPU arm
+def make_device_sets(wl, nsets, device):
+    import torch
+    from sparse_long_sequence_lf_b200.workloads import make_inputs
+    sets = []
+    for s in range(nsets):
+        x = make_inputs(wl, seed=wl.seed + 7919 * s)
+        sets.append({k: (v.to(device) if torch.is_tensor(v) else v) for k, v in x.items()})
+    return sets
+
+
+def launches_per_step(wl, max_global):
+    # prepare kernel + attention kernel, plus the global-row kernel (fp32) or
+    # the global-row combine kernel (bf16/fp16) when there are global tokens
+    return 2 + (1 if max_global > 0 else 0)
+
+
+def run_gpu_arm(args, wl, world, rank, local):
+    import torch
+    import sparse_long_sequence_lf_b200 as lf
+    from sparse_long_sequence_lf_b200 import accounting
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist(world, "nccl")
+
+    x0 = make_device_sets(wl, 1, device)[0]
+    per_set = sum(t.numel() * t.element_size() for t in x0.values() if torch.is_tensor(t))
+    per_set += x0["q"].numel() * x0["q"].element_size()          # output
+    nsets = max(2, -(-2 * L2_BYTES // per_set))
+    sets = [x0] + make_device_sets(wl.with_(seed=wl.seed + 1), nsets - 1, device)
+    outs = [torch.empty_like(s["q"]) for s in sets]
+    max_global = max(int((s["global_mask"] != 0).sum(1).max()) if s["global_mask"] is not None
+                     else 0 for s in sets)
+    ws = lf.new_workspace(wl.B, wl.H, wl.n, max_global, device)
+    stream = torch.cuda.Stream(device)
+
+    def step(i):
+        s = sets[i % nsets]
+        lf.attention_forward(s["q"], s["k"], s["v"], s["qg"], s["kg"], s["vg"],
+                             s["local_mask"], s["global_mask"], window=wl.window,
+                             dilation=s["dilation"], causal=wl.causal, max_global=max_global,
+                             out=outs[i % nsets], workspace=ws)
+
+    def run_only(i):
+        s = sets[i % nsets]
+        lf.attention_run(s["q"], s["k"], s["v"], s["qg"], s["kg"], s["vg"], window=wl.window,
+                         dilation=s["dilation"], causal=wl.causal, max_global=max_global,
+                         out=outs[i % nsets], workspace=ws)
+
+    def capture(fn, count, offset=0):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(count):
+                fn(offset + i)
+        return g
+
+    # Eager warm-up (also builds the tensor-map cache), then the graphs.
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 1)):
+            step(i)
+    stream.synchronize()
+    status = lf.workspace_status(ws, stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    chunk = nsets * max(1, 64 // nsets)
+    g_chunk = capture(step, min(chunk, args.steps))
+    full, rem = divmod(args.steps, chunk) if args.steps >= chunk else (0, args.steps)
+    g_rem = capture(step, rem) if (rem and full) else None
+    if full == 0:
+        g_chunk, full, g_rem = g_chunk, 1, None
+
+    # Graphs replay on `stream`, the stream the CUDA events are recorded on.
+    def replay(g):
+        with torch.cuda.stream(stream):
+            g.replay()
+
+    def timed_steps():
+        for _ in range(full):
+            replay(g_chunk)
+        if g_rem is not None:
+            replay(g_rem)
+
+    # Graph warm-up (W steps' worth, at least one replay).
+    for _ in range(max(1, -(-args.warmup // chunk))):
+        replay(g_chunk)
+    stream.synchronize()
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        t_pad = time.time()
+        while time.time() - t_pad < 0.5:           # same work before the timed region
+            replay(g_chunk)
+            stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+        start.record(stream)
+        timed_steps()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+        if world > 1:
+            dist.barrier()
+        t_pad = time.time()
+        while time.time() - t_pad < 0.5:           # and after it
+            replay(g_chunk)
+            stream.synchronize()
+    local_ms = start.elapsed_time(end)
+    max_ms = reduce_max(local_ms, device)
+    clocks = sampler.summary("timed region plus 0.5 s of the same graph on each side")
+
+    status = lf.workspace_status(ws, stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    # Attention kernel alone (the dominant kernel), same rotation, graph replay.
+    g_run = capture(run_only, chunk)
+    for _ in range(2):
+        replay(g_run)
+    stream.synchronize()
+    reps = max(1, -(-args.steps // chunk))
+    ks, ke = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ks.record(stream)
+    for _ in range(reps):
+        replay(g_run)
+    ke.record(stream)
+    torch.cuda.synchronize(device)
+    kernel_ms = ks.elapsed_time(ke) / (reps * chunk)
+
+    flops = accounting.useful_flops(wl)
+    bytes_ = accounting.algorithmic_bytes(wl)
+    ms_per_step = max_ms / args.steps
+    value = whole_job_rate(flops, args.steps, world, max_ms) / 1e12
+    tokens_per_s = whole_job_rate(accounting.tokens(wl), args.steps, world, max_ms)
+
+    peaks, peak_kind = load_peaks()
+    achieved_gbs = bytes_ / (kernel_ms * 1e-3) / 1e9
+    kernel_tflops = flops / (kernel_ms * 1e-3) / 1e12
+    roofline = {
+        "kernel": "attn_tc_kernel" if wl.dtype != "f32" else "band_simt_kernel",
+        "bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
+        "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
+        "traffic": None, "peak_source": peak_kind,
+        "kernel_us": round(kernel_ms * 1e3, 3), "algorithmic_bytes": bytes_,
+        "useful_tflops": round(kernel_tflops, 1),
+        "tensor_frac_of_measured_bf16": round(kernel_tflops / peaks["bf16_tflops"], 4),
+    }
+
+    if world > 1:
+        dist.barrier()
+    e2e = run_e2e(args, wl, device, stream, max_global)
+    e2e_max_ms = reduce_max(e2e["ms_per_step"], device)
+    e2e["value"] = round(whole_job_rate(flops, 1, world, e2e_max_ms) / 1e12, 4)
+    e2e["ms_per_step"] = round(e2e_max_ms, 4)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = run_cpu_baseline(wl, budget_s=args.cpu_seconds)
+
+    result = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic",
+        "tokens_per_s": round(tokens_per_s, 1),
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "n": wl.n, "d_head": wl.d,
+                   "window": wl.window, "dilation": wl.dilation_list(), "causal": wl.causal,
+                   "globals": wl.globals_kind, "pad_tail": list(wl.pad_tail),
+                   "global_batch": wl.B * world, "seq_len": wl.n,
+                   "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"{nsets} rotating input sets, {nsets * per_set / 2**20:.0f} MiB > 2x L2",
+                   "launch": "CUDA graph of C-ABI calls",
+                   "useful_gflop_per_step": round(flops / 1e9, 4),
+                   "algorithmic_mb_per_step": round(bytes_ / 1e6, 3)},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step(wl, max_global) * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        del g_chunk, g_rem, g_run
+        dist.destroy_process_group()
+
+
+def run_e2e(args, wl, device, stream, max_global):
+    """Same metric through lf_attention_forward_host: pinned host inputs are
+    copied in, the forward runs, the output is copied back, every step."""
+    import torch
+    import sparse_long_sequence_lf_b200 as lf
+    from sparse_long_sequence_lf_b200 import accounting
+    from sparse_long_sequence_lf_b200.workloads import make_inputs
+
+    x = make_inputs(wl)
+    pin = {k: (v.pin_memory() if torch.is_tensor(v) else v) for k, v in x.items()}
+    out = torch.empty_like(pin["q"]).pin_memory()
+    staging = torch.empty(lf.host_staging_size(pin["q"].dtype, wl.B, wl.H, wl.n),
+                          dtype=torch.uint8, device=device)
+    ws = lf.new_workspace(wl.B, wl.H, wl.n, max_global, device)
+
+    def once():
+        lf.attention_forward_host(pin["q"], pin["k"], pin["v"], pin["qg"], pin["kg"], pin["vg"],
+                                  pin["local_mask"], pin["global_mask"], window=wl.window,
+                                  dilation=pin["dilation"], causal=wl.causal,
+                                  max_global=max_global, out=out, staging=staging,
+                                  workspace=ws, stream=stream)
+
+    for _ in range(3):
+        once()
+    steps = max(3, min(args.steps, args.e2e_steps))
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        once()
+    e.record(stream)
+    torch.cuda.synchronize(device)
+    ms = s.elapsed_time(e) / steps
+    h2d = sum(t.numel() * t.element_size() for t in pin.values() if torch.is_tensor(t))
+    d2h = out.numel() * out.element_size()
+    return {"value": round(accounting.useful_flops(wl) / (ms * 1e-3) / 1e12, 4), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(ms, 4), "steps": steps,
+            "path": "lf_attention_forward_host (pinned host buffers)"}
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_sample_plan(wl, budget_s):
+    """Head count and repetitions of the oracle sample for a time budget."""
+    import oracle
+    from sparse_long_sequence_lf_b200 import accounting
+    from sparse_long_sequence_lf_b200.workloads import make_inputs
+
+    x = make_inputs(wl)
+    # Calibrate on one head of every batch.
+    t0 = time.perf_counter()
+    run_oracle_heads(oracle, x, wl, 1)
+    t1 = time.perf_counter() - t0
+    heads = max(1, min(wl.H, int(budget_s / max(t1, 1e-3))))
+    reps = 1
+    if heads == wl.H:
+        reps = max(1, int(budget_s / max(t1 * wl.H, 1e-3)))
+    sub = wl.with_(H=heads, dilation=tuple(wl.dilation_list()[:heads]))
+    return x, heads, reps, accounting.useful_flops(sub)
+
+
+def run_oracle_heads(oracle, x, wl, heads):
+    for b in range(wl.B):
+        oracle.forward(x["q"], x["k"], x["v"], x["qg"], x["kg"], x["vg"], x["local_mask"],
+                       x["global_mask"], window=wl.window, dilation=x["dilation"],
+                       causal=wl.causal, bh_range=(b * wl.H, b * wl.H + heads))
+
+
+def run_cpu_baseline(wl, budget_s=10.0):
+    import oracle
+    x, heads, reps, flops = oracle_sample_plan(wl, budget_s)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        run_oracle_heads(oracle, x, wl, heads)
+    dt = time.perf_counter() - t0
+    return {"value": round(flops * reps / dt / 1e12, 6), "unit": UNIT,
+            "cores": oracle.default().max_threads(), "kind": "oracle",
+            "sample": f"{heads} of {wl.H} heads x {wl.B} batches, {reps} repetition(s), "
+                      f"{dt:.1f} s, fp64 C oracle with OpenMP",
+            "seconds": round(dt, 2)}
+
+
+def run_reference_arm(args, wl, world, rank):
+    """The oracle as the reference arm: each step a bounded sample (one or more
+    heads) of the same workload on the host cores.  Rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    budget_per_step = max(0.05, min(2.0, args.reference_seconds / max(1, args.steps + args.warmup)))
+    x, heads, _, flops = oracle_sample_plan(wl, budget_per_step)
+    for _ in range(args.warmup):
+        run_oracle_heads(oracle, x, wl, heads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run_oracle_heads(oracle, x, wl, heads)
+    dt = time.perf_counter() - t0
+    value = flops * args.steps / dt / 1e12
+    sample = f"{heads} of {wl.H} heads x {wl.B} batches per step, fp64 C oracle with OpenMP"
+    cores = oracle.default().max_threads()
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "n": wl.n, "window": wl.window},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    from sparse_long_sequence_lf_b200.workloads import HEADLINE, WORKLOADS
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=HEADLINE)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--reference-seconds", type=float, default=60.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus N > 1 needs torchrun with N processes")
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference_arm(args, wl, world, rank)
+        return
+    run_gpu_arm(args, wl, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

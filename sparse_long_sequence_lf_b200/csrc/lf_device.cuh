@@ -181,27 +181,34 @@ __device__ __forceinline__ void band_item(const AttnArgs &a, int item, int &b, i
     tile = rem;
 }
 
-// Merges the chunk partials of one global row and writes its output row.
-// Partial layout: [bh][chunk][slot][m, l, acc[64]], m in log2 units.
+// Partial results of the global rows, per (bh, chunk): field-major
+// [m (log2 units), l, acc[64]] x max_global slots.
+__device__ __forceinline__ float *partial_base(const AttnArgs &a, int bh, int chunk)
+{
+    return a.ws.partials + (size_t(bh) * a.L.nchunks + chunk) * kPartialFloats * size_t(a.max_global);
+}
+
+// Merges the chunk partials of one global row and writes its output row;
+// lane l of the calling warp handles dimensions 2l and 2l+1.
 template <typename T>
 __device__ __forceinline__ void combine_row_partials(const AttnArgs &a, int bh, int slot,
                                                      int nchunks_used, int lane, T *orow)
 {
-    const float *P = a.ws.partials +
-                     (size_t(bh) * a.L.nchunks * a.max_global + slot) * kPartialFloats;
-    const size_t cstride = size_t(a.max_global) * kPartialFloats;
+    const size_t mg = size_t(a.max_global);
+    const float *P = partial_base(a, bh, 0) + slot;
+    const size_t cstride = kPartialFloats * mg;
     float M = -INFINITY;
     for (int c = 0; c < nchunks_used; ++c) M = fmaxf(M, P[c * cstride]);
     float Lsum = 0.f, acc0 = 0.f, acc1 = 0.f;
     for (int c = 0; c < nchunks_used; ++c) {
         const float *pc = P + c * cstride;
-        float mc = pc[0];
-        float f = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
-        Lsum += f * pc[1];
-        acc0 += f * pc[2 + 2 * lane];
-        acc1 += f * pc[3 + 2 * lane];
+        const float mc = pc[0];
+        const float f = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+        Lsum += f * pc[mg];
+        acc0 += f * pc[(2 + 2 * lane) * mg];
+        acc1 += f * pc[(3 + 2 * lane) * mg];
     }
-    float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
     orow[2 * lane] = from_f32<T>(acc0 * inv);
     orow[2 * lane + 1] = from_f32<T>(acc1 * inv);
 }

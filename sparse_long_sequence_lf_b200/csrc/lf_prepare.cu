@@ -4,16 +4,44 @@
 // once before the layer loop, the positions of the global tokens of each batch
 // and their count from the global mask, and turns the local mask into an
 // additive -10000 bias.  Here one CTA per batch does a stable ascending
-// compaction with warp ballots and a block-wide prefix sum, and the local mask
-// becomes a bitmap of valid keys (exclusion, not a bias).  The same pass
-// builds a bitmap of global tokens, a has-padding flag, and clears the
-// arrival counters of the global-row combine.
+// compaction in a single pass: every thread owns a run of whole 32-position
+// words, loads all of its mask bytes at once, counts its global tokens, and one
+// block-wide exclusive scan gives each thread its output offset.  The local
+// mask becomes a bitmap of valid keys (exclusion, not a bias).  The same pass
+// builds a bitmap of global tokens, a has-padding flag, and clears the arrival
+// counters of the global-row combine.
 #include "lf_device.cuh"
 
 namespace lf {
 
 constexpr int kPrepThreads = 1024;
 constexpr int kPrepWarps = kPrepThreads / 32;
+constexpr int kPrepMaxWordsPerThread = 8;    // n up to 1024 * 8 * 32 = 262144 in one pass
+
+// Bit i of the result is set when byte p0 + i of the mask is nonzero (bits past
+// n are 0).  A NULL mask reads as all default_value.
+__device__ __forceinline__ uint32_t word_bits(const uint8_t *m, int p0, int n, bool present,
+                                              bool default_value)
+{
+    const int left = n - p0;
+    const uint32_t inrange = left >= 32 ? 0xffffffffu : (left <= 0 ? 0u : ((1u << left) - 1u));
+    if (!present) return default_value ? inrange : 0u;
+    uint32_t w = 0;
+    if (left >= 32 && (reinterpret_cast<uintptr_t>(m + p0) & 15u) == 0) {
+        const uint4 *v = reinterpret_cast<const uint4 *>(m + p0);
+        const uint4 a = v[0], b = v[1];
+        const uint32_t x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if ((x[q] >> (8 * k)) & 0xffu) w |= 1u << (4 * q + k);
+        return w;
+    }
+    for (int i = 0; i < 32 && i < left; ++i)
+        if (m[p0 + i] != 0) w |= 1u << i;
+    return w;
+}
 
 // One CTA per batch.  Any output pointer may be NULL (not written).
 __global__ void __launch_bounds__(kPrepThreads)
@@ -21,9 +49,11 @@ prepare_kernel(const uint8_t *__restrict__ local_mask, const uint8_t *__restrict
                int B, int n, int max_global, int32_t *gidx, int32_t *counts, int *flags,
                uint32_t *vbits, uint32_t *gbits, int *status, int *counters, int counters_per_batch)
 {
-    __shared__ int warp_tot[kPrepWarps];
-    __shared__ int s_base;
-    __shared__ int s_pad;
+    // The attention kernel may start its prologue now; it waits for this
+    // grid's results before reading them.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    __shared__ int warp_sum[kPrepWarps];
 
     const int b = blockIdx.x;
     const int tid = threadIdx.x;
@@ -32,58 +62,64 @@ prepare_kernel(const uint8_t *__restrict__ local_mask, const uint8_t *__restrict
     const uint8_t *lm = local_mask ? local_mask + size_t(b) * n : nullptr;
     const uint8_t *gm = global_mask ? global_mask + size_t(b) * n : nullptr;
     const int nwords = (n + 31) / 32;
+    const int wpt = (nwords + kPrepThreads - 1) / kPrepThreads;   // words per thread (<= 8)
+    const int w0 = tid * wpt;
 
-    if (tid == 0) {
-        s_base = 0;
-        s_pad = 0;
-        if (b == 0 && status) *status = 0;
-    }
+    if (tid == 0 && b == 0 && status) *status = 0;
     if (counters)
         for (int c = tid; c < counters_per_batch; c += kPrepThreads)
             counters[size_t(b) * counters_per_batch + c] = 0;
-    __syncthreads();
 
-    int any_pad = 0;
-    for (int start = 0; start < n; start += kPrepThreads) {
-        const int p = start + tid;
-        const bool in = p < n;
-        const bool is_g = in && gm && gm[p] != 0;
-        const bool valid = in && (lm == nullptr || lm[p] != 0);
-        any_pad |= (in && !valid);
-        const unsigned gball = __ballot_sync(0xffffffffu, is_g);
-        const unsigned vball = __ballot_sync(0xffffffffu, valid);
-        if (lane == 0) {
-            const int word = p >> 5;
-            if (word < nwords) {
-                if (vbits) vbits[size_t(b) * nwords + word] = vball;
-                if (gbits) gbits[size_t(b) * nwords + word] = gball;
-            }
-            warp_tot[warp] = __popc(gball);
+    uint32_t gw[kPrepMaxWordsPerThread];
+    int mine = 0, pad = 0;
+#pragma unroll
+    for (int k = 0; k < kPrepMaxWordsPerThread; ++k) {
+        gw[k] = 0u;
+        const int w = w0 + k;
+        if (k < wpt && w < nwords) {
+            const uint32_t g = word_bits(gm, 32 * w, n, gm != nullptr, false);
+            const uint32_t v = word_bits(lm, 32 * w, n, lm != nullptr, true);
+            gw[k] = g;
+            mine += __popc(g);
+            const int left = n - 32 * w;
+            const uint32_t inrange = left >= 32 ? 0xffffffffu : ((1u << left) - 1u);
+            pad |= (v != inrange);
+            if (vbits) vbits[size_t(b) * nwords + w] = v;
+            if (gbits) gbits[size_t(b) * nwords + w] = g;
         }
-        __syncthreads();
-        // Exclusive prefix over the warps of this chunk (warp totals are small).
-        int before = 0, total = 0;
-        for (int w = 0; w < kPrepWarps; ++w) {
-            const int t = warp_tot[w];
-            before += (w < warp) ? t : 0;
-            total += t;
-        }
-        if (is_g && gidx) {
-            const int rank = before + __popc(gball & ((1u << lane) - 1u));
-            gidx[size_t(b) * n + s_base + rank] = p;
-        }
-        __syncthreads();
-        if (tid == 0) s_base += total;
-        __syncthreads();
     }
-    const int count = s_base;
-    if (gidx)
-        for (int p = count + tid; p < n; p += kPrepThreads) gidx[size_t(b) * n + p] = -1;
-    any_pad = __syncthreads_or(any_pad);
+    // Block-wide exclusive scan of the per-thread global counts.
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    const int any_pad = __syncthreads_or(pad);
+    int before = 0, total = 0;
+    for (int w = 0; w < kPrepWarps; ++w) {
+        const int t = warp_sum[w];
+        before += (w < warp) ? t : 0;
+        total += t;
+    }
+    int off = before + incl - mine;
+    if (gidx) {
+#pragma unroll
+        for (int k = 0; k < kPrepMaxWordsPerThread; ++k) {
+            uint32_t g = gw[k];
+            while (g) {
+                const int i = __ffs(g) - 1;
+                g &= g - 1u;
+                gidx[size_t(b) * n + off++] = 32 * (w0 + k) + i;
+            }
+        }
+        for (int p = total + tid; p < n; p += kPrepThreads) gidx[size_t(b) * n + p] = -1;
+    }
     if (tid == 0) {
-        if (counts) counts[b] = count;
+        if (counts) counts[b] = total;
         if (flags)
-            flags[b] = (any_pad ? kFlagHasPadding : 0) | (count > max_global ? kFlagOverflow : 0);
+            flags[b] = (any_pad ? kFlagHasPadding : 0) | (total > max_global ? kFlagOverflow : 0);
     }
 }
 
@@ -92,6 +128,7 @@ int launch_prepare(const uint8_t *local_mask, const uint8_t *global_mask, int B,
                    uint32_t *gbits, int *status, int *counters, int counters_per_batch,
                    cudaStream_t stream)
 {
+    if ((n + 31) / 32 > kPrepThreads * kPrepMaxWordsPerThread) return kErrUnsupported;
     prepare_kernel<<<B, kPrepThreads, 0, stream>>>(local_mask, global_mask, B, n, max_global, gidx,
                                                    counts, flags, vbits, gbits, status, counters,
                                                    counters_per_batch);

@@ -261,14 +261,14 @@ global_simt_kernel(const AttnArgs a)
     for (int t = 0; t < kGlobSlotsPerWarp; ++t) {
         const int slot = slot0 + warp * kGlobSlotsPerWarp + t;
         if (slot >= g) break;
-        float *P = a.ws.partials +
-                   ((size_t(bh) * a.L.nchunks + chunk) * a.max_global + slot) * kPartialFloats;
+        float *P = partial_base(a, bh, chunk) + slot;
+        const size_t mg = size_t(a.max_global);
         if (lane == 0) {
             P[0] = m[t];
-            P[1] = l[t];
+            P[mg] = l[t];
         }
-        P[2 + 2 * lane] = acc0[t];
-        P[3 + 2 * lane] = acc1[t];
+        P[(2 + 2 * lane) * mg] = acc0[t];
+        P[(3 + 2 * lane) * mg] = acc1[t];
     }
 
     // The last CTA of this (bh, group) to finish merges every chunk.

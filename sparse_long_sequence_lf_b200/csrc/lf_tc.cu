@@ -21,24 +21,24 @@
 // Layout of one CTA (384 threads, one CTA per SM, persistent over items):
 //   warps 0-3   softmax warpgroup of lane 0   (one thread per query row)
 //   warps 4-7   softmax warpgroup of lane 1
-//   warp  8     TMA producer of lane 0
-//   warp  9     TMA producer of lane 1
-//   warp 10     TMEM allocator and MMA issuer for both lanes
-//   warp 11     idle (completes the third warpgroup for the register split)
-// The two lanes are independent item streams; the MMA warp alternates
-// between them so one lane's QK^T / PV runs while the other lane's softmax
-// does its exponentials.
+//   warps 8-9   TMA producers of lanes 0 and 1
+//   warps 10-11 MMA issuers of lanes 0 and 1 (warp 10 also owns TMEM)
+// The two lanes are independent item streams sharing the SM's tensor core,
+// SFU and FMA pipes.
 //
-// TMEM (512 columns): S/P of lane X at columns [128X, 128X+128) (fp32 scores,
-// overwritten in place by the 16-bit probabilities P in the first 64
-// columns), O of lane X at [256+64X, 320+64X).
+// TMEM (512 columns; lane X uses [192X, 192X+192)): two 64-key score
+// buffers S0, S1 (fp32, overwritten in place by the 16-bit probabilities P in
+// their first 32 columns) and the 64-column output accumulator O.  While the
+// softmax works on S(j), the tensor core already computes S(j+1) into the
+// other buffer.
 //   S = Q K^T      tcgen05.mma kind::f16, A = Q (smem, K-major),
-//                  B = K tile (smem, K-major), 128x128 fp32 in TMEM
+//                  B = K tile (smem, K-major), 128x64 fp32 in TMEM
 //   O += P V       tcgen05.mma kind::f16, A = P (TMEM), B = V tile
 //                  (smem, MN-major), 128x64 fp32 in TMEM
-// Shared-memory tiles are 128 rows x 128 bytes with the 128-byte swizzle,
-// written by TMA: whole tiles for undilated rows, single-row loads for dilated
-// rows, global tokens and gathered Qg rows.  Every wait on an mbarrier is
+// Shared-memory tiles have 128-byte rows with the 128-byte swizzle, written
+// by TMA: whole tiles for undilated rows, single-row loads for dilated rows,
+// global tokens and gathered Qg rows.  Q is double-buffered per lane, K/V
+// run through a 4-stage ring of 64-key tiles per lane.  Every wait on an mbarrier is
 // bounded; on expiry the kernel records LF_ERR_DEVICE_TIMEOUT, drains its own
 // copies and MMAs, frees its TMEM and returns.
 #include <algorithm>
@@ -55,23 +55,29 @@ namespace lf {
 
 using namespace sm100;
 
-constexpr int kRows = 128;
-constexpr int kKeys = 128;
-constexpr int kStages = 2;
+constexpr int kRows = 128;                        // query rows per tile (M)
+constexpr int kKeys = 64;                         // keys per S tile / K-V stage
+constexpr int kStages = 4;                        // K/V ring depth per lane
 constexpr int kLanes = 2;
-constexpr int kTileBytes = kRows * kDHead * 2;   // 16 KB of 16-bit elements
-constexpr int kRowBytes = kDHead * 2;            // 128 B
-constexpr int kThreads = 384;        // 3 warpgroups
-constexpr int kWarpProducer = 8;
-constexpr int kWarpMma = 10;
+constexpr int kQBytes = kRows * kDHead * 2;       // 16 KB of 16-bit elements
+constexpr int kKvBytes = kKeys * kDHead * 2;      // 8 KB
+constexpr int kRowBytes = kDHead * 2;             // 128 B
+constexpr int kThreads = 384;                     // 3 warpgroups
+constexpr int kWarpProducer = 8;                  // warps 8, 9: TMA producers of lanes 0, 1
+constexpr int kWarpMma = 10;                      // warps 10, 11: MMA issuers of lanes 0, 1
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemLaneCols = 192;           // S0 (64) | S1 (64) | O (64) per lane
+constexpr float kRescaleLog2 = 8.f;               // lazy rescale: P stays below 2^8
 // Register split: the softmax warpgroups take registers from the producer /
 // MMA warpgroup.  The launch must hold at least kRegsNeeded registers
 // (checked on the host against the compiled register count).
-constexpr int kRegsSoftmax = 216;
-constexpr int kRegsControl = 64;
+constexpr int kRegsSoftmax = 176;
+constexpr int kRegsControl = 144;
 constexpr int kRegsNeeded = 2 * 128 * kRegsSoftmax + 128 * kRegsControl;
-constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleLog2 = 8.f;   // lazy rescale: P stays below 2^8
+// Of every 8 column pairs of a score tile, the pairs whose bit is set here
+// take 2^x from a cubic on the FMA pipe, the others from the SFU; the two
+// units then share the exponentials.
+constexpr uint32_t kPolyPairs = 0x49u;            // pairs 0, 3, 6 of each 8
 
 enum MapId {
     kMapQTile, kMapKTile, kMapVTile, kMapKgTile, kMapVgTile,
@@ -91,13 +97,14 @@ static_assert(sizeof(AttnArgs) + kMapCount * sizeof(CUtensorMap) + 64 <= 4096,
               "kernel arguments must fit the classic 4 KB parameter space");
 
 struct __align__(1024) TcSmem {
-    uint8_t q[kLanes][kTileBytes];
-    uint8_t k[kLanes][kStages][kTileBytes];
-    uint8_t v[kLanes][kStages][kTileBytes];
-    uint64_t q_full[kLanes], q_empty[kLanes];
+    uint8_t q[kLanes][2][kQBytes];
+    uint8_t k[kLanes][kStages][kKvBytes];
+    uint8_t v[kLanes][kStages][kKvBytes];
+    uint64_t q_full[kLanes][2], q_empty[kLanes][2];
     uint64_t kv_full[kLanes][kStages], kv_empty[kLanes][kStages];
-    uint64_t s_full[kLanes], p_full[kLanes], o_full[kLanes], o_free[kLanes];
-    uint64_t drain;
+    uint64_t s_full[kLanes][2], p_full[kLanes][2], pv_done[kLanes][2];
+    uint64_t o_free[kLanes];
+    uint64_t drain[kLanes];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -160,10 +167,12 @@ __device__ __forceinline__ Geom decode_item(const TcParams &p, int item)
     return G;
 }
 
-// Walks the tiles of the items of one lane: items lane, lane + stride, ...
+// Walks the 64-key tiles of the items of one lane: items lane, lane + stride,
+// ...  `j` counts the lane's tiles and `k` its items (both from 0); they pick
+// the double buffers and the barrier parities.
 struct Cursor {
     int item, stride, total;
-    int t;
+    int t, j, k;
     Geom G;
     bool valid;
 
@@ -185,16 +194,22 @@ struct Cursor {
         item = first;
         stride = stride_;
         total = p.total_items;
+        j = 0;
+        k = 0;
         seek(p);
     }
     __device__ __forceinline__ void advance(const TcParams &p)
     {
+        ++j;
         if (++t < G.ntiles) return;
+        ++k;
         item += stride;
         seek(p);
     }
+    __device__ __forceinline__ bool first() const { return t == 0; }
+    __device__ __forceinline__ bool last() const { return t == G.ntiles - 1; }
     __device__ __forceinline__ bool is_global_col_tile() const { return G.kind == 1 && t >= G.nkv; }
-    // Keys in this tile (N of QK^T, K of PV): 128, or the global tokens of a
+    // Keys in this tile (N of QK^T, K of PV): 64, or the global tokens of a
     // global-column tile rounded up to a multiple of 16.
     __device__ __forceinline__ int tile_n() const
     {
@@ -224,31 +239,45 @@ __device__ __forceinline__ void advance_ring(int &stage, uint32_t &phase)
     }
 }
 
-// TMA producer of one lane.
-__device__ void producer_role(const TcParams &p, TcSmem &sm, int X, int lane)
+// Waits (bounded, ignoring the abort flag) for a copy this CTA started, so
+// that nothing lands in shared memory after the CTA has exited.
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < kWaitLimitNs) {
+    }
+}
+
+// TMA producer of one lane: Q (double-buffered) and the 64-key K/V ring.
+__device__ __forceinline__ void producer_role(const TcParams &p, TcSmem &sm, int X, int lane)
 {
     const AttnArgs &a = p.a;
     Cursor cur;
     cur.init(p, blockIdx.x * kLanes + X, gridDim.x * kLanes);
     int stage = 0;
-    uint32_t phase = 0, qe_phase = 1;
+    uint32_t phase = 0;
     bool armed[kStages] = {};
     uint32_t armed_phase[kStages] = {};
-    bool q_armed = false;
-    uint32_t q_armed_phase = 0, qf_count = 0;
+    bool q_armed[2] = {false, false};
+    uint32_t q_armed_phase[2] = {0u, 0u};
     const int n = a.n;
     bool ok = true;
 
     while (cur.valid && ok) {
         const Geom &G = cur.G;
-        if (cur.t == 0) {
-            if (!warp_wait(&sm.q_empty[X], qe_phase, &sm.abort_flag, a.ws.status)) { ok = false; break; }
-            qe_phase ^= 1u;
-            const bool tile_load = (G.kind == 1 && G.dil == 1);
-            if (lane == 0) mbar_arrive_expect_tx(&sm.q_full[X], kTileBytes);
+        if (cur.first()) {
+            const int qb = cur.k & 1;
+            const uint32_t use = uint32_t(cur.k >> 1);
+            if (!warp_wait(&sm.q_empty[X][qb], (use & 1u) ^ 1u, &sm.abort_flag, a.ws.status)) {
+                ok = false;
+                break;
+            }
+            uint8_t *qd = sm.q[X][qb];
+            uint64_t *qbar = &sm.q_full[X][qb];
+            if (lane == 0) mbar_arrive_expect_tx(qbar, kQBytes);
             __syncwarp();
-            if (tile_load) {
-                if (lane == 0) tma_load_3d(sm.q[X], &p.maps[kMapQTile], &sm.q_full[X], 0, G.q0, G.bh);
+            if (G.kind == 1 && G.dil == 1) {
+                if (lane == 0) tma_load_3d(qd, &p.maps[kMapQTile], qbar, 0, G.q0, G.bh);
             } else {
                 const CUtensorMap *map = G.kind == 1 ? &p.maps[kMapQRow] : &p.maps[kMapQgRow];
                 for (int rr = lane; rr < kRows; rr += 32) {
@@ -260,28 +289,26 @@ __device__ void producer_role(const TcParams &p, TcSmem &sm, int X, int lane)
                         const int slot = G.q0 + rr;
                         if (slot < G.g) y = G.bh * n + a.ws.gidx[size_t(G.b) * n + slot];
                     }
-                    tma_load_2d(sm.q[X] + rr * kRowBytes, map, &sm.q_full[X], 0, y);
+                    tma_load_2d(qd + rr * kRowBytes, map, qbar, 0, y);
                 }
             }
-            q_armed = true;
-            q_armed_phase = qf_count & 1u;
-            ++qf_count;
+            q_armed[qb] = true;
+            q_armed_phase[qb] = use & 1u;
         }
-        if (!warp_wait(&sm.kv_empty[X][stage], phase ^ 1u, &sm.abort_flag, a.ws.status)) { ok = false; break; }
+        if (!warp_wait(&sm.kv_empty[X][stage], phase ^ 1u, &sm.abort_flag, a.ws.status)) {
+            ok = false;
+            break;
+        }
         uint8_t *kd = sm.k[X][stage];
         uint8_t *vd = sm.v[X][stage];
         uint64_t *bar = &sm.kv_full[X][stage];
-        if (G.kind == 2) {
+        if (G.kind == 2 || (!cur.is_global_col_tile() && G.dil == 1)) {
+            const CUtensorMap *km = G.kind == 2 ? &p.maps[kMapKgTile] : &p.maps[kMapKTile];
+            const CUtensorMap *vm = G.kind == 2 ? &p.maps[kMapVgTile] : &p.maps[kMapVTile];
             if (lane == 0) {
-                mbar_arrive_expect_tx(bar, 2 * kTileBytes);
-                tma_load_3d(kd, &p.maps[kMapKgTile], bar, 0, cur.k0(), G.bh);
-                tma_load_3d(vd, &p.maps[kMapVgTile], bar, 0, cur.k0(), G.bh);
-            }
-        } else if (!cur.is_global_col_tile() && G.dil == 1) {
-            if (lane == 0) {
-                mbar_arrive_expect_tx(bar, 2 * kTileBytes);
-                tma_load_3d(kd, &p.maps[kMapKTile], bar, 0, cur.k0(), G.bh);
-                tma_load_3d(vd, &p.maps[kMapVTile], bar, 0, cur.k0(), G.bh);
+                mbar_arrive_expect_tx(bar, 2 * kKvBytes);
+                tma_load_3d(kd, km, bar, 0, cur.k0(), G.bh);
+                tma_load_3d(vd, vm, bar, 0, cur.k0(), G.bh);
             }
         } else {
             const bool gcol = cur.is_global_col_tile();
@@ -307,118 +334,96 @@ __device__ void producer_role(const TcParams &p, TcSmem &sm, int X, int lane)
         cur.advance(p);
     }
     if (!ok || sm.abort_flag) {
-        // Let every copy this warp started land before the CTA exits.
         for (int s = 0; s < kStages; ++s)
-            if (armed[s]) {
-                const uint64_t t0 = global_timer_ns();
-                while (!mbar_try_wait(&sm.kv_full[X][s], armed_phase[s]) &&
-                       global_timer_ns() - t0 < kWaitLimitNs) {
-                }
-            }
-        if (q_armed) {
-            const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(&sm.q_full[X], q_armed_phase) &&
-                   global_timer_ns() - t0 < kWaitLimitNs) {
-            }
-        }
+            if (armed[s]) drain_wait(&sm.kv_full[X][s], armed_phase[s]);
+        for (int b = 0; b < 2; ++b)
+            if (q_armed[b]) drain_wait(&sm.q_full[X][b], q_armed_phase[b]);
     }
 }
 
-struct MmaLane {
-    Cursor cur;
-    int stage;
-    uint32_t phase, qf_phase, pf_phase, of_phase;
-    bool pend;
-    int pend_stage, pend_n;
-    bool pend_first, pend_last;
+struct TileInfo {
+    int stage, n, j, k;
+    bool first, last;
 };
 
-// One step of the MMA schedule of lane X: the PV of the previous tile, then
-// the QK^T of the next one.  Returns false on abort.
-__device__ __forceinline__ bool mma_step(const TcParams &p, TcSmem &sm, MmaLane &L, int X,
-                                         uint32_t tmem, bool leader, uint32_t id_s,
-                                         uint32_t id_pv)
+// MMA issuer of one lane.  Order: S(0); then for every tile j:
+// S(j+1) into the other S buffer (look-ahead), then PV(j) once P(j) is ready.
+// S(j+2) reuses the buffer of P(j) and is issued after PV(j), and the tensor
+// pipe executes in issue order.
+__device__ __forceinline__ void mma_role(const TcParams &p, TcSmem &sm, uint32_t tmem, int X,
+                                         bool bf16)
 {
     const AttnArgs &a = p.a;
-    const uint32_t tS = tmem + X * 128;
-    const uint32_t tO = tmem + 256 + X * 64;
-    if (L.pend) {
-        if (!warp_wait(&sm.p_full[X], L.pf_phase, &sm.abort_flag, a.ws.status)) return false;
-        L.pf_phase ^= 1u;
-        if (L.pend_first) {
-            if (!warp_wait(&sm.o_free[X], L.of_phase, &sm.abort_flag, a.ws.status)) return false;
-            L.of_phase ^= 1u;
-        }
-        tc_fence_after();
-        if (leader) {
-            const uint32_t vbase = smem_u32(sm.v[X][L.pend_stage]);
-            for (int kk = 0; kk < L.pend_n / 16; ++kk) {
-                const uint64_t bdesc = make_sdesc(vbase + kk * 2048, 16, 1024);
-                mma_ts(tO, tS + kk * 8, bdesc, id_pv, (kk > 0 || !L.pend_first) ? 1u : 0u);
-            }
-            tc_commit(&sm.kv_empty[X][L.pend_stage]);
-            if (L.pend_last) tc_commit(&sm.o_full[X]);
-        }
-        __syncwarp();
-        L.pend = false;
-    }
-    if (L.cur.valid) {
-        if (L.cur.t == 0) {
-            if (!warp_wait(&sm.q_full[X], L.qf_phase, &sm.abort_flag, a.ws.status)) return false;
-            L.qf_phase ^= 1u;
-        }
-        if (!warp_wait(&sm.kv_full[X][L.stage], L.phase, &sm.abort_flag, a.ws.status)) return false;
-        tc_fence_after();
-        const int N = L.cur.tile_n();
-        if (leader) {
-            const uint32_t qbase = smem_u32(sm.q[X]);
-            const uint32_t kbase = smem_u32(sm.k[X][L.stage]);
-            const uint32_t idesc = id_s | (uint32_t(N >> 3) << 17);
-#pragma unroll
-            for (int kk = 0; kk < kDHead / 16; ++kk) {
-                const uint64_t adesc = make_sdesc(qbase + kk * 32, 16, 1024);
-                const uint64_t bdesc = make_sdesc(kbase + kk * 32, 16, 1024);
-                mma_ss(tS, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(&sm.s_full[X]);
-            if (L.cur.t == L.cur.G.ntiles - 1) tc_commit(&sm.q_empty[X]);
-        }
-        __syncwarp();
-        L.pend = true;
-        L.pend_stage = L.stage;
-        L.pend_n = N;
-        L.pend_first = (L.cur.t == 0);
-        L.pend_last = (L.cur.t == L.cur.G.ntiles - 1);
-        advance_ring(L.stage, L.phase);
-        L.cur.advance(p);
-    }
-    return true;
-}
-
-__device__ void mma_role(const TcParams &p, TcSmem &sm, uint32_t tmem, int lane, bool bf16)
-{
-    // S tiles: M = 128, N set per tile; PV: M = 128, N = 64, B MN-major.
     const uint32_t id_s = make_idesc(128, 0, bf16, false);
     const uint32_t id_pv = make_idesc(128, 64, bf16, true);
-    MmaLane L[kLanes];
-    for (int X = 0; X < kLanes; ++X) {
-        L[X].cur.init(p, blockIdx.x * kLanes + X, gridDim.x * kLanes);
-        L[X].stage = 0;
-        L[X].phase = 0;
-        L[X].qf_phase = 0;
-        L[X].pf_phase = 0;
-        L[X].of_phase = 1;   // the first item has no previous epilogue to wait for
-        L[X].pend = false;
-    }
-    const bool leader = (lane == 0);
-    for (;;) {
-        bool any = false;
-        for (int X = 0; X < kLanes; ++X) {
-            if (!L[X].cur.valid && !L[X].pend) continue;
-            any = true;
-            if (!mma_step(p, sm, L[X], X, tmem, leader, id_s, id_pv)) return;
+    const uint32_t tbase = tmem + X * kTmemLaneCols;
+    const uint32_t tO = tbase + 128;
+    Cursor cur;
+    cur.init(p, blockIdx.x * kLanes + X, gridDim.x * kLanes);
+    int stage = 0;
+    uint32_t phase = 0;
+
+    // Issues S(j) for the tile under the cursor; returns false on abort.
+    auto issue_s = [&](TileInfo &info) -> bool {
+        if (cur.first()) {
+            const uint32_t use = uint32_t(cur.k >> 1);
+            if (!warp_wait(&sm.q_full[X][cur.k & 1], use & 1u, &sm.abort_flag, a.ws.status))
+                return false;
         }
-        if (!any) break;
+        if (!warp_wait(&sm.kv_full[X][stage], phase, &sm.abort_flag, a.ws.status)) return false;
+        tc_fence_after();
+        const int N = cur.tile_n();
+        const uint32_t tS = tbase + (cur.j & 1) * 64;
+        const uint64_t qdesc = make_sdesc(smem_u32(sm.q[X][cur.k & 1]), 16, 1024);
+        const uint64_t kdesc = make_sdesc(smem_u32(sm.k[X][stage]), 16, 1024);
+        const uint32_t idesc = id_s | (uint32_t(N >> 3) << 17);
+#pragma unroll
+        for (int kk = 0; kk < kDHead / 16; ++kk)
+            mma_ss_elect(tS, qdesc + uint64_t((kk * 32) >> 4), kdesc + uint64_t((kk * 32) >> 4),
+                         idesc, kk > 0 ? 1u : 0u);
+        tc_commit_elect(&sm.s_full[X][cur.j & 1]);
+        if (cur.last()) tc_commit_elect(&sm.q_empty[X][cur.k & 1]);
+        __syncwarp();
+        info.stage = stage;
+        info.n = N;
+        info.j = cur.j;
+        info.k = cur.k;
+        info.first = cur.first();
+        info.last = cur.last();
+        advance_ring(stage, phase);
+        cur.advance(p);
+        return true;
+    };
+
+    if (!cur.valid) return;
+    TileInfo pend;
+    if (!issue_s(pend)) return;
+    for (;;) {
+        TileInfo next;
+        const bool have_next = cur.valid;
+        if (have_next && !issue_s(next)) return;
+        // PV of the pending tile.
+        const int b = pend.j & 1;
+        if (!warp_wait(&sm.p_full[X][b], uint32_t(pend.j >> 1) & 1u, &sm.abort_flag, a.ws.status))
+            return;
+        if (pend.first && pend.k > 0) {
+            if (!warp_wait(&sm.o_free[X], uint32_t(pend.k - 1) & 1u, &sm.abort_flag, a.ws.status))
+                return;
+        }
+        tc_fence_after();
+        {
+            const uint32_t tP = tbase + b * 64;
+            const uint64_t vdesc = make_sdesc(smem_u32(sm.v[X][pend.stage]), 16, 1024);
+            const int ksteps = pend.n >> 4;
+            for (int kk = 0; kk < ksteps; ++kk)
+                mma_ts_elect(tO, tP + kk * 8, vdesc + uint64_t((kk * 2048) >> 4), id_pv,
+                             (kk > 0 || !pend.first) ? 1u : 0u);
+            tc_commit_elect(&sm.kv_empty[X][pend.stage]);
+            tc_commit_elect(&sm.pv_done[X][b]);
+        }
+        __syncwarp();
+        if (!have_next) break;
+        pend = next;
     }
 }
 
@@ -434,15 +439,15 @@ template <> __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Bits of the 128 key columns of a tile that hold real, unpadded keys, built
-// by each warp on its own (4 lookups per lane and 4 ballots).
+// Bits of the 64 key columns of a tile that hold real, unpadded keys, built
+// by each warp on its own (2 lookups per lane and 2 ballots).
 __device__ __forceinline__ void column_bits(const AttnArgs &a, const Cursor &cur, int lane,
-                                            uint32_t (&bits)[4])
+                                            uint32_t (&bits)[2])
 {
     const Geom &G = cur.G;
     const uint32_t *vb = a.ws.vbits + size_t(G.b) * a.L.nwords;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < 2; ++w) {
         const int c = w * 32 + lane;
         bool ok;
         if (cur.is_global_col_tile()) {
@@ -463,101 +468,74 @@ struct RowState {
     float m, l;
 };
 
-// Softmax of one full 128-key tile for this thread's row.  clo/chi bound the
-// columns of the row's key range; cbits (when use_bits) marks real keys.
-template <typename T>
-__device__ __forceinline__ void softmax_tile128(uint32_t tS, uint32_t tO, RowState &st,
-                                                bool first, int clo, int chi, bool use_bits,
-                                                const uint32_t (&cbits)[4], float sl2)
+// Bits of the columns [32q, 32q + 32) that lie inside [clo, chi].
+__device__ __forceinline__ uint32_t range_bits(int q, int clo, int chi)
 {
-    float s[128];
-    tmem_ld128(tS, s);
-    const bool need_mask = (clo > 0) || (chi < 127) || use_bits;
-    if (__any_sync(0xffffffffu, need_mask)) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-            bool ok = (c >= clo) && (c <= chi);
-            if (use_bits) ok = ok && ((cbits[c >> 5] >> (c & 31)) & 1u);
-            s[c] = ok ? s[c] : -INFINITY;
-        }
-    }
-    float mx = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < 128; ++c) mx = fmaxf(mx, s[c]);
-    const float mt = mx * sl2;
-    float alpha = 1.f;
-    bool rescale = false;
-    if (first) {
-        st.m = mt;
-        st.l = 0.f;
-    } else if (mt > st.m + kRescaleLog2) {
-        alpha = ex2(st.m - mt);
-        st.m = mt;
-        rescale = true;
-    }
-    const float base = (st.m == -INFINITY) ? 0.f : st.m;
-    float sum = 0.f;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            const float p0 = ex2(fmaf(s[32 * q + 2 * c], sl2, -base));
-            const float p1 = ex2(fmaf(s[32 * q + 2 * c + 1], sl2, -base));
-            sum += p0 + p1;
-            pk[c] = pack2<T>(p0, p1);
-        }
-        tmem_st16(tS + 16 * q, pk);
-    }
-    if (__any_sync(0xffffffffu, rescale)) {
-        // O of the previous tiles is complete: its PV was issued before this S.
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float o[32];
-            tmem_ld32(tO + half * 32, o);
-            uint32_t ob[32];
-#pragma unroll
-            for (int x = 0; x < 32; ++x) ob[x] = __float_as_uint(o[x] * alpha);
-            tmem_st32(tO + half * 32, ob);
-        }
-    }
-    st.l = st.l * alpha + sum;
-    tmem_st_wait();
+    const int lo = min(max(clo - 32 * q, 0), 32);
+    const int hi = min(max(chi - 32 * q + 1, 0), 32);
+    const uint32_t below_hi = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+    const uint32_t below_lo = lo >= 32 ? 0xffffffffu : ((1u << lo) - 1u);
+    return below_hi & ~below_lo;
 }
 
-// Softmax of a global-token column tile with N (multiple of 16) columns.
-// Unrolled over the 8 possible 16-column chunks so every mask bit stays in a
-// register (N is the same for the whole warp).
-template <typename T>
-__device__ __forceinline__ void softmax_tile_global_cols(const AttnArgs &a, const Cursor &cur,
-                                                         uint32_t tS, uint32_t tO, RowState &st,
-                                                         bool first, int i, int dil,
-                                                         const uint32_t (&cbits)[4], float sl2)
+// Maximum of 32 values as a shallow tree of 3-input maxima.
+__device__ __forceinline__ float max32(const float *s)
 {
-    const Geom &G = cur.G;
-    const int N = cur.tile_n();
-    const int *gl = a.ws.gidx + size_t(G.b) * a.n + cur.slot0();
-    uint32_t okb[4] = {0u, 0u, 0u, 0u};
-    float mx = -INFINITY;
+    float t[11];
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-        if (ch * 16 < N) {
-            float s[16];
-            tmem_ld16(tS + ch * 16, s);
+    for (int i = 0; i < 10; ++i) t[i] = max3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
+    t[10] = fmaxf(s[30], s[31]);
+    const float u0 = max3(t[0], t[1], t[2]);
+    const float u1 = max3(t[3], t[4], t[5]);
+    const float u2 = max3(t[6], t[7], t[8]);
+    return max3(u0, u1, max3(u2, t[9], t[10]));
+}
+
+// 2^x for a pair of arguments on the FMA pipe.  x = j + f with j = round(x)
+// (the 1.5*2^23 addition rounds to an integer in the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f is a cubic fitted to minimise the maximum relative
+// error on [-1/2, 1/2] (Remez exchange, error below 7.5e-5); 2^j is added to
+// the exponent field.  Arguments below -126 are clamped (the result is then
+// at most 2^-126, which is zero for every use here).
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float &y0, float &y1)
+{
+    constexpr float kRound = 12582912.f;     // 1.5 * 2^23
+    constexpr float c0 = 0.999928074f, c1 = 0.693260985f, c2 = 0.242611122f,
+                    c3 = 0.0551716691f;
+    x0 = fmaxf(x0, -126.f);
+    x1 = fmaxf(x1, -126.f);
+    float t0, t1, j0, j1, f0, f1, p0, p1;
+    add2(t0, t1, x0, x1, kRound, kRound);
+    add2(j0, j1, t0, t1, -kRound, -kRound);
+    fma2(f0, f1, j0, j1, -1.f, -1.f, x0, x1);
+    fma2(p0, p1, f0, f1, c3, c3, c2, c2);
+    fma2(p0, p1, p0, p1, f0, f1, c1, c1);
+    fma2(p0, p1, p0, p1, f0, f1, c0, c0);
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// Online softmax of one 64-key score tile for this thread's row.  mw marks
+// the columns that are keys of this row.  Writes P = 2^(S*scale*log2e - m)
+// as 16-bit pairs over the first 32 columns of the tile and adds the row sum.
+// O is rescaled in TMEM only when the running maximum grows by more than 2^8
+// (after the previous PV has completed).  Returns false on abort.
+template <typename T>
+__device__ __forceinline__ bool softmax_tile(TcSmem &sm, const AttnArgs &a, int X, uint32_t tS,
+                                             uint32_t tO, RowState &st, const Cursor &cur,
+                                             const uint32_t (&mw)[2], bool need_mask, float sl2)
+{
+    float s[64];
+    tmem_ld32(tS, *reinterpret_cast<float(*)[32]>(&s[0]));
+    tmem_ld32(tS + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+    if (need_mask) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const int col = ch * 16 + c;
-                bool ok = (cbits[col >> 5] >> (col & 31)) & 1u;
-                if (ok) ok = !is_tap(i, __ldg(gl + col), a.window, a.half, dil, a.causal);
-                okb[col >> 5] |= (ok ? 1u : 0u) << (col & 31);
-                mx = ok ? fmaxf(mx, s[c]) : mx;
-            }
-        }
+        for (int c = 0; c < 64; ++c) s[c] = ((mw[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
     }
-    const float mt = mx * sl2;
+    const float mt = fmaxf(max32(&s[0]), max32(&s[32])) * sl2;
     float alpha = 1.f;
     bool rescale = false;
-    if (first) {
+    if (cur.first()) {
         st.m = mt;
         st.l = 0.f;
     } else if (mt > st.m + kRescaleLog2) {
@@ -565,28 +543,32 @@ __device__ __forceinline__ void softmax_tile_global_cols(const AttnArgs &a, cons
         st.m = mt;
         rescale = true;
     }
-    const float base = (st.m == -INFINITY) ? 0.f : st.m;
-    float sum = 0.f;
+    const float nb = (st.m == -INFINITY) ? 0.f : -st.m;
+    float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
+    uint32_t pk[32];
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-        if (ch * 16 < N) {
-            float s[16];
-            tmem_ld16(tS + ch * 16, s);
-            uint32_t pk[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const int col = ch * 16 + 2 * c;
-                const bool ok0 = (okb[col >> 5] >> (col & 31)) & 1u;
-                const bool ok1 = (okb[(col + 1) >> 5] >> ((col + 1) & 31)) & 1u;
-                const float p0 = ok0 ? ex2(fmaf(s[2 * c], sl2, -base)) : 0.f;
-                const float p1 = ok1 ? ex2(fmaf(s[2 * c + 1], sl2, -base)) : 0.f;
-                sum += p0 + p1;
-                pk[c] = pack2<T>(p0, p1);
-            }
-            tmem_st8(tS + ch * 8, pk);
+    for (int c = 0; c < 32; ++c) {
+        float x0, x1, p0, p1;
+        fma2(x0, x1, s[2 * c], s[2 * c + 1], sl2, sl2, nb, nb);
+        if ((kPolyPairs >> (c & 7)) & 1u) {
+            exp2_poly2(x0, x1, p0, p1);
+        } else {
+            p0 = ex2(x0);
+            p1 = ex2(x1);
         }
+        if (c & 1)
+            add2(sb0, sb1, sb0, sb1, p0, p1);
+        else
+            add2(sa0, sa1, sa0, sa1, p0, p1);
+        pk[c] = pack2<T>(p0, p1);
     }
     if (__any_sync(0xffffffffu, rescale)) {
+        // O must hold every PV before this tile: the previous one may still run.
+        const int jp = cur.j - 1;
+        if (!warp_wait(&sm.pv_done[X][jp & 1], uint32_t(jp >> 1) & 1u, &sm.abort_flag,
+                       a.ws.status))
+            return false;
+        tc_fence_after();
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             float o[32];
@@ -597,8 +579,10 @@ __device__ __forceinline__ void softmax_tile_global_cols(const AttnArgs &a, cons
             tmem_st32(tO + half * 32, ob);
         }
     }
-    st.l = st.l * alpha + sum;
+    tmem_st32(tS, pk);
+    st.l = st.l * alpha + ((sa0 + sa1) + (sb0 + sb1));
     tmem_st_wait();
+    return true;
 }
 
 template <typename T>
@@ -631,91 +615,80 @@ __device__ __forceinline__ void store_row(T *dst, const float (&o)[64], float in
     }
 }
 
-// Merges the chunk partials of the global rows of one (bh, 128-row tile); run
-// by the warp that arrived last.  Lane l handles rows l, l+32, l+64, l+96.
 template <typename T>
-__device__ void combine_global_tile(const AttnArgs &a, const Geom &G, int lane)
-{
-    const int nch = a.L.nchunks;
-    const size_t cstride = size_t(a.max_global) * kPartialFloats;
-    const uint32_t *vb = a.ws.vbits + size_t(G.b) * a.L.nwords;
-    T *Out = static_cast<T *>(a.out) + size_t(G.bh) * a.n * kDHead;
-    for (int rr = lane; rr < kRows; rr += 32) {
-        const int slot = G.q0 + rr;
-        if (slot >= G.g) break;
-        const int pos = a.ws.gidx[size_t(G.b) * a.n + slot];
-        if (!bit_at(vb, pos)) continue;   // padded global position: written as zeros elsewhere
-        const float *P = a.ws.partials + (size_t(G.bh) * nch * a.max_global + slot) * kPartialFloats;
-        float M = -INFINITY;
-        for (int c = 0; c < nch; ++c) M = fmaxf(M, __ldcg(P + c * cstride));
-        float Lsum = 0.f;
-        float o[64];
-#pragma unroll
-        for (int x = 0; x < 64; ++x) o[x] = 0.f;
-        for (int c = 0; c < nch; ++c) {
-            const float *pc = P + c * cstride;
-            const float mc = __ldcg(pc);
-            const float f = (mc == -INFINITY) ? 0.f : ex2(mc - M);
-            Lsum += f * __ldcg(pc + 1);
-#pragma unroll
-            for (int x = 0; x < 64; ++x) o[x] = fmaf(f, __ldcg(pc + 2 + x), o[x]);
-        }
-        store_row<T>(Out + size_t(pos) * kDHead, o, Lsum > 0.f ? 1.f / Lsum : 0.f);
-    }
-}
-
-template <typename T>
-__device__ void softmax_role(const TcParams &p, TcSmem &sm, uint32_t tmem, int X, int tid)
+__device__ __forceinline__ void softmax_role(const TcParams &p, TcSmem &sm, uint32_t tmem, int X,
+                                             int tid)
 {
     const AttnArgs &a = p.a;
     const int warp = tid >> 5, lane = tid & 31;
     const uint32_t lane_off = uint32_t(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_off + X * 128;
-    const uint32_t tO = tmem + lane_off + 256 + X * 64;
+    const uint32_t tbase = tmem + lane_off + X * kTmemLaneCols;
+    const uint32_t tO = tbase + 128;
     const float sl2 = a.scale_log2;
     Cursor cur;
     cur.init(p, blockIdx.x * kLanes + X, gridDim.x * kLanes);
-    uint32_t sf_phase = 0, of_phase = 0;
     RowState st{-INFINITY, 0.f};
 
     while (cur.valid) {
         const Geom &G = cur.G;
-        const bool first = (cur.t == 0);
-        const bool last = (cur.t == G.ntiles - 1);
-        if (first && tid == 0 && a.ws.counts[G.b] > a.max_global)
+        if (cur.first() && tid == 0 && a.ws.counts[G.b] > a.max_global)
             set_status(a.ws.status, kErrGlobalOverflow);
         const int row = G.q0 + tid;     // residue-space row (band) or global slot
-        uint32_t cbits[4] = {~0u, ~0u, ~0u, ~0u};
+        const int bsel = cur.j & 1;
+        const uint32_t tS = tbase + bsel * 64;
         const bool gcol = cur.is_global_col_tile();
-        const bool use_bits = gcol || G.has_pad;
-        if (use_bits) column_bits(a, cur, lane, cbits);
-
-        if (!warp_wait(&sm.s_full[X], sf_phase, &sm.abort_flag, a.ws.status)) return;
-        sf_phase ^= 1u;
-        tc_fence_after();
+        uint32_t cbits[2] = {~0u, ~0u};
+        if (gcol || G.has_pad) column_bits(a, cur, lane, cbits);
+        uint32_t mw[2];
+        bool need_mask;
         if (gcol) {
-            softmax_tile_global_cols<T>(a, cur, tS, tO, st, first, row * G.dil + G.r, G.dil,
-                                        cbits, sl2);
+            // Global-token columns: real, unpadded tokens that are not already
+            // window taps of this row.
+            const int i = row * G.dil + G.r;
+            const int *gl = a.ws.gidx + size_t(G.b) * a.n + cur.slot0();
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                uint32_t m = cbits[q];
+                uint32_t rest = m;
+                while (rest) {
+                    const int c = __ffs(rest) - 1;
+                    rest &= rest - 1u;
+                    if (is_tap(i, __ldg(gl + 32 * q + c), a.window, a.half, G.dil, a.causal))
+                        m &= ~(1u << c);
+                }
+                mw[q] = m;
+            }
+            need_mask = true;
         } else {
             int clo, chi;
             const int k0 = cur.k0();
             if (G.kind == 2) {
                 clo = 0;
-                chi = min(127, G.key_end - 1 - k0);
+                chi = min(kKeys - 1, G.key_end - 1 - k0);
             } else {
                 const int lo = max(row - (a.causal ? a.window - 1 : a.half), 0);
                 const int hi = min(row + (a.causal ? 0 : a.half), G.n_r - 1);
                 clo = lo - k0;
                 chi = hi - k0;
             }
-            softmax_tile128<T>(tS, tO, st, first, clo, chi, use_bits, cbits, sl2);
+            mw[0] = range_bits(0, clo, chi) & cbits[0];
+            mw[1] = range_bits(1, clo, chi) & cbits[1];
+            need_mask = __any_sync(0xffffffffu, (mw[0] & mw[1]) != 0xffffffffu);
         }
-        tc_fence_before();
-        mbar_arrive(&sm.p_full[X]);
 
-        if (last) {
-            if (!warp_wait(&sm.o_full[X], of_phase, &sm.abort_flag, a.ws.status)) return;
-            of_phase ^= 1u;
+        if (!warp_wait(&sm.s_full[X][bsel], uint32_t(cur.j >> 1) & 1u, &sm.abort_flag,
+                       a.ws.status))
+            return;
+        tc_fence_after();
+        if (!softmax_tile<T>(sm, a, X, tS, tO, st, cur, mw, need_mask, sl2)) return;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_full[X][bsel]);
+
+        if (cur.last()) {
+            if (!warp_wait(&sm.pv_done[X][bsel], uint32_t(cur.j >> 1) & 1u, &sm.abort_flag,
+                           a.ws.status))
+                return;
             tc_fence_after();
             if (G.kind == 1) {
                 const bool row_in = row < G.n_r;
@@ -734,12 +707,14 @@ __device__ void softmax_role(const TcParams &p, TcSmem &sm, uint32_t tmem, int X
                     if (write) store_half_row<T>(dst + half * 32, o, inv);
                 }
                 tc_fence_before();
-                mbar_arrive(&sm.o_free[X]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.o_free[X]);
             } else {
                 const int slot = row;
+                const size_t mg = size_t(a.max_global);
                 float *P = a.ws.partials +
-                           ((size_t(G.bh) * a.L.nchunks + G.chunk) * a.max_global +
-                            min(slot, a.max_global - 1)) * kPartialFloats;
+                           (size_t(G.bh) * a.L.nchunks + G.chunk) * kPartialFloats * mg +
+                           min(slot, a.max_global - 1);
                 const bool write = slot < G.g;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -747,29 +722,15 @@ __device__ void softmax_role(const TcParams &p, TcSmem &sm, uint32_t tmem, int X
                     tmem_ld32(tO + half * 32, o);
                     if (write) {
 #pragma unroll
-                        for (int x = 0; x < 32; ++x) P[2 + half * 32 + x] = o[x];
+                        for (int x = 0; x < 32; ++x) P[(2 + half * 32 + x) * mg] = o[x];
                     }
                 }
                 tc_fence_before();
-                mbar_arrive(&sm.o_free[X]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.o_free[X]);
                 if (write) {
                     P[0] = st.m;
-                    P[1] = st.l;
-                }
-                __threadfence();
-                __syncwarp();
-                int last_warp = 0;
-                if (lane == 0) {
-                    int *ctr = a.ws.counters + size_t(G.bh) * (a.L.ngroups + 1) + G.gtile;
-                    const int target = 4 * a.L.nchunks;
-                    const int prev = atomicAdd(ctr, 1);
-                    last_warp = (prev == target - 1);
-                    if (last_warp) *ctr = 0;
-                }
-                last_warp = __shfl_sync(0xffffffffu, last_warp, 0);
-                if (last_warp) {
-                    __threadfence();
-                    combine_global_tile<T>(a, G, lane);
+                    P[mg] = st.l;
                 }
             }
         }
@@ -788,18 +749,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
     if (threadIdx.x == 0) {
         for (int X = 0; X < kLanes; ++X) {
-            mbar_init(&sm.q_full[X], 1);
-            mbar_init(&sm.q_empty[X], 1);
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&sm.q_full[X][b], 1);
+                mbar_init(&sm.q_empty[X][b], 1);
+                mbar_init(&sm.s_full[X][b], 1);
+                mbar_init(&sm.p_full[X][b], 4);     // one arrival per softmax warp
+                mbar_init(&sm.pv_done[X][b], 1);
+            }
             for (int s = 0; s < kStages; ++s) {
                 mbar_init(&sm.kv_full[X][s], 1);
                 mbar_init(&sm.kv_empty[X][s], 1);
             }
-            mbar_init(&sm.s_full[X], 1);
-            mbar_init(&sm.p_full[X], kRows);
-            mbar_init(&sm.o_full[X], 1);
-            mbar_init(&sm.o_free[X], kRows);
+            mbar_init(&sm.o_free[X], 4);
+            mbar_init(&sm.drain[X], 1);
         }
-        mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
         mbar_fence_init();
     }
@@ -813,23 +776,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    // Everything above overlaps the previous kernel in the stream; the
+    // workspace it writes (compacted indices, bitmaps) is read only below.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp < 8) {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         softmax_role<T>(p, sm, tmem, warp >> 2, threadIdx.x & 127);
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
-    }
-    if (warp < 8) {
-    } else if (warp < kWarpMma) {
-        producer_role(p, sm, warp - kWarpProducer, lane);
-    } else if (warp == kWarpMma) {
-        mma_role(p, sm, tmem, lane, std::is_same<T, __nv_bfloat16>::value);
-        // Every MMA of this CTA has completed once this commit lands.
-        if (lane == 0) tc_commit(&sm.drain);
-        __syncwarp();
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(&sm.drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+        if (warp < kWarpMma) {
+            producer_role(p, sm, warp - kWarpProducer, lane);
+        } else {
+            const int X = warp - kWarpMma;
+            mma_role(p, sm, tmem, X, std::is_same<T, __nv_bfloat16>::value);
+            // Every MMA this warp issued has completed once this commit lands.
+            tc_commit_elect(&sm.drain[X]);
+            __syncwarp();
+            drain_wait(&sm.drain[X], 0);
         }
     }
     tc_fence_before();
@@ -837,6 +802,49 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Merges the chunk partials of every global row into its output row: one
+// warp per (batch*head, global slot); lane l handles dimensions 2l, 2l+1.
+// Launched after the attention kernel (programmatic dependent launch: its
+// prologue overlaps the attention kernel's tail, the wait below orders it).
+template <typename T>
+__global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a)
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int lane = threadIdx.x & 31;
+    const int bh = blockIdx.x;
+    const int slot = blockIdx.y * 4 + (threadIdx.x >> 5);
+    const int b = bh / a.H;
+    const int g = min(a.ws.counts[b], a.max_global);
+    if (slot >= g) return;
+    const int pos = a.ws.gidx[size_t(b) * a.n + slot];
+    if (!bit_at(a.ws.vbits + size_t(b) * a.L.nwords, pos)) return;   // padded: zeros elsewhere
+    const int nch = a.L.nchunks;
+    const size_t mg = size_t(a.max_global);
+    const size_t cstride = kPartialFloats * mg;
+    const float *P = partial_base(a, bh, 0) + slot;
+    float M = -INFINITY;
+    for (int c = lane; c < nch; c += 32) M = fmaxf(M, P[c * cstride]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f, a0 = 0.f, a1 = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < nch; ++c) {
+        const float *pc = P + c * cstride;
+        const float mc = pc[0];
+        const float f = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+        L = fmaf(f, pc[mg], L);
+        a0 = fmaf(f, pc[(2 + 2 * lane) * mg], a0);
+        a1 = fmaf(f, pc[(3 + 2 * lane) * mg], a1);
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    T *dst = static_cast<T *>(a.out) + (size_t(bh) * a.n + pos) * kDHead;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        reinterpret_cast<__nv_bfloat162 *>(dst)[lane] = __floats2bfloat162_rn(a0 * inv, a1 * inv);
+    } else {
+        reinterpret_cast<__half2 *>(dst)[lane] = __floats2half2_rn(a0 * inv, a1 * inv);
     }
 }
 
@@ -858,14 +866,15 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder()
     return fn;
 }
 
-// Whole 128-row tiles of one (batch*head) slice: dims {64, n, B*H}.
-bool encode_tile_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int n, int BH)
+// Whole tiles of box_rows rows of one (batch*head) slice: dims {64, n, B*H}.
+bool encode_tile_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int n, int BH,
+                     int box_rows)
 {
     auto enc = get_encoder();
     if (!enc) return false;
     cuuint64_t dims[3] = {cuuint64_t(kDHead), cuuint64_t(n), cuuint64_t(BH)};
     cuuint64_t strides[2] = {cuuint64_t(kRowBytes), cuuint64_t(n) * kRowBytes};
-    cuuint32_t box[3] = {kDHead, kRows, 1};
+    cuuint32_t box[3] = {kDHead, cuuint32_t(box_rows), 1};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -896,6 +905,7 @@ struct MapCacheEntry {
 };
 
 // Encoded tensor maps, reused while the same buffer and shape come back.
+// kind: 0 = tiles of 128 rows, 1 = single rows, 2 = tiles of kKeys rows.
 bool cached_map(CUtensorMap *out, int kind, const void *base, CUtensorMapDataType dt, int n, int BH)
 {
     static std::mutex mu;
@@ -908,8 +918,8 @@ bool cached_map(CUtensorMap *out, int kind, const void *base, CUtensorMapDataTyp
             return true;
         }
     CUtensorMap m;
-    const bool ok = kind == 0 ? encode_tile_map(&m, base, dt, n, BH)
-                              : encode_row_map(&m, base, dt, long(n) * BH);
+    const bool ok = kind == 1 ? encode_row_map(&m, base, dt, long(n) * BH)
+                              : encode_tile_map(&m, base, dt, n, BH, kind == 0 ? kRows : kKeys);
     if (!ok) return false;
     MapCacheEntry &e = cache[next++ % 64];
     e = MapCacheEntry{base, kind, int(dt), n, BH, m, true};
@@ -934,10 +944,10 @@ int launch_typed(const AttnArgs &a, CUtensorMapDataType dt, cudaStream_t stream)
     const int BH = a.B * a.H;
     bool ok = true;
     ok = ok && cached_map(&p.maps[kMapQTile], 0, a.q, dt, a.n, BH);
-    ok = ok && cached_map(&p.maps[kMapKTile], 0, a.k, dt, a.n, BH);
-    ok = ok && cached_map(&p.maps[kMapVTile], 0, a.v, dt, a.n, BH);
-    ok = ok && cached_map(&p.maps[kMapKgTile], 0, a.kg, dt, a.n, BH);
-    ok = ok && cached_map(&p.maps[kMapVgTile], 0, a.vg, dt, a.n, BH);
+    ok = ok && cached_map(&p.maps[kMapKTile], 2, a.k, dt, a.n, BH);
+    ok = ok && cached_map(&p.maps[kMapVTile], 2, a.v, dt, a.n, BH);
+    ok = ok && cached_map(&p.maps[kMapKgTile], 2, a.kg, dt, a.n, BH);
+    ok = ok && cached_map(&p.maps[kMapVgTile], 2, a.vg, dt, a.n, BH);
     ok = ok && cached_map(&p.maps[kMapQRow], 1, a.q, dt, a.n, BH);
     ok = ok && cached_map(&p.maps[kMapKRow], 1, a.k, dt, a.n, BH);
     ok = ok && cached_map(&p.maps[kMapVRow], 1, a.v, dt, a.n, BH);
@@ -964,7 +974,28 @@ int launch_typed(const AttnArgs &a, CUtensorMapDataType dt, cudaStream_t stream)
     }
     const int want = (p.total_items + kLanes - 1) / kLanes;
     const int grid = std::max(1, std::min(num_sms(), want));
-    attn_tc_kernel<T><<<grid, kThreads, smem, stream>>>(p);
+    // Programmatic dependent launch: the kernel's prologue (barriers, TMEM,
+    // tensor-map prefetch) overlaps the kernel before it in the stream.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, attn_tc_kernel<T>, p) != cudaSuccess) return kErrCuda;
+    if (a.max_global > 0) {
+        cudaLaunchConfig_t cc = {};
+        cc.gridDim = dim3(a.B * a.H, (a.max_global + 3) / 4);
+        cc.blockDim = dim3(128);
+        cc.stream = stream;
+        cc.attrs = attr;
+        cc.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cc, combine_kernel<T>, a) != cudaSuccess) return kErrCuda;
+    }
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 
