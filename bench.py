@@ -22,6 +22,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import os
 import statistics
@@ -47,6 +48,35 @@ def load_peaks():
             return json.load(f), "measured"
     except (OSError, ValueError):
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+# Kernel sources whose change invalidates a stored DRAM-traffic figure.
+TRAFFIC_SOURCES = {
+    "attn_tc_kernel": ("lf_tc.cu", "lf_sm100.cuh", "lf_device.cuh"),
+    "band_simt_kernel": ("lf_simt.cu", "lf_device.cuh"),
+}
+
+
+def kernel_source_digest(kernel: str) -> str:
+    h = hashlib.sha256()
+    for name in TRAFFIC_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "sparse_long_sequence_lf_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def stored_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from a committed ncu
+    capture (profiles/dram_traffic.json), or None when there is none or the
+    kernel sources changed since it was taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            rec = json.load(f).get(kernel, {}).get(workload)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("sources_sha256") != kernel_source_digest(kernel):
+        return None
+    return int(rec["dram_bytes_per_launch"])
 
 
 def dist_env():
@@ -290,11 +320,12 @@ def run_gpu_arm(args, wl, world, rank, local):
     peaks, peak_kind = load_peaks()
     achieved_gbs = bytes_ / (kernel_ms * 1e-3) / 1e9
     kernel_tflops = flops / (kernel_ms * 1e-3) / 1e12
+    kname = "attn_tc_kernel" if wl.dtype != "f32" else "band_simt_kernel"
     roofline = {
-        "kernel": "attn_tc_kernel" if wl.dtype != "f32" else "band_simt_kernel",
+        "kernel": kname,
         "bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
         "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
-        "traffic": None, "peak_source": peak_kind,
+        "traffic": stored_traffic(kname, wl.name), "peak_source": peak_kind,
         "kernel_us": round(kernel_ms * 1e3, 3), "algorithmic_bytes": bytes_,
         "useful_tflops": round(kernel_tflops, 1),
         "tensor_frac_of_measured_bf16": round(kernel_tflops / peaks["bf16_tflops"], 4),

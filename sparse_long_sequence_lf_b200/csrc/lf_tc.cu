@@ -79,22 +79,31 @@ constexpr int kRegsNeeded = 2 * 128 * kRegsSoftmax + 128 * kRegsControl;
 // units then share the exponentials.
 constexpr uint32_t kPolyPairs = 0x49u;            // pairs 0, 3, 6 of each 8
 
-enum MapId {
-    kMapQTile, kMapKTile, kMapVTile, kMapKgTile, kMapVgTile,
-    kMapQRow, kMapKRow, kMapVRow, kMapQgRow, kMapCount
-};
+enum MapId { kMapKgTile, kMapVgTile, kMapQRow, kMapKRow, kMapVRow, kMapQgRow, kMapCount };
+
+// Residue-class tensor maps: for a head with dilation d, the rows r, r+d,
+// r+2d, ... of each (batch, head) slice form a plain sequence (row stride
+// d*128 B, first row r), so whole tiles of a dilated window load with one TMA
+// copy.  Up to kMaxResidues (dilation, residue) pairs per call; heads beyond
+// that load their rows one by one.
+constexpr int kMaxResidues = 24;
 
 struct TcParams {
-    CUtensorMap maps[kMapCount];   // first: 64-byte aligned
+    CUtensorMap maps[kMapCount];              // first: 64-byte aligned
+    CUtensorMap res_q[kMaxResidues];          // Q tiles of 128 rows
+    CUtensorMap res_k[kMaxResidues];          // K tiles of 64 rows
+    CUtensorMap res_v[kMaxResidues];          // V tiles of 64 rows
     AttnArgs a;
+    int res_base[kMaxHeads];  // residue map of (head h, residue 0); -1: load rows one by one
     int global_items;     // B*H*gtiles*nchunks, ordered before the band items
     int total_items;
     int gtiles;           // ceil(max_global / 128)
     int oob_row;          // a row coordinate past the end of the row maps (reads zeros)
+    int n_res;            // residue maps in use
 };
 
-static_assert(sizeof(AttnArgs) + kMapCount * sizeof(CUtensorMap) + 64 <= 4096,
-              "kernel arguments must fit the classic 4 KB parameter space");
+// Kernel arguments above 4 KB need CUDA 12.1 or newer (up to 32764 bytes).
+static_assert(sizeof(TcParams) <= 32000, "kernel arguments exceed the parameter space");
 
 struct __align__(1024) TcSmem {
     uint8_t q[kLanes][2][kQBytes];
@@ -274,22 +283,29 @@ __device__ __forceinline__ void producer_role(const TcParams &p, TcSmem &sm, int
             }
             uint8_t *qd = sm.q[X][qb];
             uint64_t *qbar = &sm.q_full[X][qb];
-            if (lane == 0) mbar_arrive_expect_tx(qbar, kQBytes);
-            __syncwarp();
-            if (G.kind == 1 && G.dil == 1) {
-                if (lane == 0) tma_load_3d(qd, &p.maps[kMapQTile], qbar, 0, G.q0, G.bh);
-            } else {
-                const CUtensorMap *map = G.kind == 1 ? &p.maps[kMapQRow] : &p.maps[kMapQgRow];
+            const int rb = G.kind == 1 ? p.res_base[G.h] : -1;
+            if (rb >= 0) {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(qbar, kQBytes);
+                    tma_load_3d(qd, &p.res_q[rb + G.r], qbar, 0, G.q0, G.bh);
+                }
+            } else if (G.kind == 1) {
+                if (lane == 0) mbar_arrive_expect_tx(qbar, kQBytes);
+                __syncwarp();
                 for (int rr = lane; rr < kRows; rr += 32) {
-                    int y = p.oob_row;
-                    if (G.kind == 1) {
-                        const int ir = G.q0 + rr;
-                        if (ir < G.n_r) y = G.bh * n + ir * G.dil + G.r;
-                    } else {
-                        const int slot = G.q0 + rr;
-                        if (slot < G.g) y = G.bh * n + a.ws.gidx[size_t(G.b) * n + slot];
-                    }
-                    tma_load_2d(qd + rr * kRowBytes, map, qbar, 0, y);
+                    const int ir = G.q0 + rr;
+                    const int y = ir < G.n_r ? G.bh * n + ir * G.dil + G.r : p.oob_row;
+                    tma_load_2d(qd + rr * kRowBytes, &p.maps[kMapQRow], qbar, 0, y);
+                }
+            } else {
+                // Only the rows of real global tokens: a query row only feeds
+                // its own output row, and rows past the count are never stored.
+                const int rows = min(kRows, G.g - G.q0);
+                if (lane == 0) mbar_arrive_expect_tx(qbar, rows * kRowBytes);
+                __syncwarp();
+                for (int rr = lane; rr < rows; rr += 32) {
+                    const int y = G.bh * n + a.ws.gidx[size_t(G.b) * n + G.q0 + rr];
+                    tma_load_2d(qd + rr * kRowBytes, &p.maps[kMapQgRow], qbar, 0, y);
                 }
             }
             q_armed[qb] = true;
@@ -302,9 +318,10 @@ __device__ __forceinline__ void producer_role(const TcParams &p, TcSmem &sm, int
         uint8_t *kd = sm.k[X][stage];
         uint8_t *vd = sm.v[X][stage];
         uint64_t *bar = &sm.kv_full[X][stage];
-        if (G.kind == 2 || (!cur.is_global_col_tile() && G.dil == 1)) {
-            const CUtensorMap *km = G.kind == 2 ? &p.maps[kMapKgTile] : &p.maps[kMapKTile];
-            const CUtensorMap *vm = G.kind == 2 ? &p.maps[kMapVgTile] : &p.maps[kMapVTile];
+        const int rb = G.kind == 1 ? p.res_base[G.h] : -1;
+        if (G.kind == 2 || (!cur.is_global_col_tile() && rb >= 0)) {
+            const CUtensorMap *km = G.kind == 2 ? &p.maps[kMapKgTile] : &p.res_k[rb + G.r];
+            const CUtensorMap *vm = G.kind == 2 ? &p.maps[kMapVgTile] : &p.res_v[rb + G.r];
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar, 2 * kKvBytes);
                 tma_load_3d(kd, km, bar, 0, cur.k0(), G.bh);
@@ -440,9 +457,13 @@ template <> __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi
 }
 
 // Bits of the 64 key columns of a tile that hold real, unpadded keys, built
-// by each warp on its own (2 lookups per lane and 2 ballots).
+// by each warp on its own (2 lookups per lane and 2 ballots).  For a
+// global-column tile also the token position of column 32w + lane (jpos[w])
+// and the columns whose token lies in the row's residue class (res[w]): a
+// window tap of row i = ir*dil + r always does.
 __device__ __forceinline__ void column_bits(const AttnArgs &a, const Cursor &cur, int lane,
-                                            uint32_t (&bits)[2])
+                                            uint32_t (&bits)[2], int (&jpos)[2],
+                                            uint32_t (&res)[2])
 {
     const Geom &G = cur.G;
     const uint32_t *vb = a.ws.vbits + size_t(G.b) * a.L.nwords;
@@ -452,7 +473,10 @@ __device__ __forceinline__ void column_bits(const AttnArgs &a, const Cursor &cur
         bool ok;
         if (cur.is_global_col_tile()) {
             const int slot = cur.slot0() + c;
-            ok = slot < G.g && bit_at(vb, a.ws.gidx[size_t(G.b) * a.n + slot]);
+            const int j = slot < G.g ? a.ws.gidx[size_t(G.b) * a.n + slot] : -1;
+            ok = j >= 0 && bit_at(vb, j);
+            jpos[w] = j;
+            res[w] = __ballot_sync(0xffffffffu, ok && (j % G.dil) == G.r);
         } else if (G.kind == 2) {
             const int j = cur.k0() + c;
             ok = j < G.key_end && bit_at(vb, j);
@@ -637,26 +661,29 @@ __device__ __forceinline__ void softmax_role(const TcParams &p, TcSmem &sm, uint
         const int bsel = cur.j & 1;
         const uint32_t tS = tbase + bsel * 64;
         const bool gcol = cur.is_global_col_tile();
-        uint32_t cbits[2] = {~0u, ~0u};
-        if (gcol || G.has_pad) column_bits(a, cur, lane, cbits);
+        uint32_t cbits[2] = {~0u, ~0u}, res[2] = {0u, 0u};
+        int jpos[2] = {-1, -1};
+        if (gcol || G.has_pad) column_bits(a, cur, lane, cbits, jpos, res);
         uint32_t mw[2];
         bool need_mask;
         if (gcol) {
             // Global-token columns: real, unpadded tokens that are not already
-            // window taps of this row.
+            // window taps of this row.  A tap shares the row's residue class
+            // and lies within the (dilated) window span.
             const int i = row * G.dil + G.r;
-            const int *gl = a.ws.gidx + size_t(G.b) * a.n + cur.slot0();
+            const int span_lo = a.causal ? (a.window - 1) * G.dil : a.half * G.dil;
+            const int span_hi = a.causal ? 0 : a.half * G.dil;
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                uint32_t m = cbits[q];
-                uint32_t rest = m;
+            for (int w = 0; w < 2; ++w) {
+                uint32_t m = cbits[w];
+                uint32_t rest = res[w];
                 while (rest) {
                     const int c = __ffs(rest) - 1;
                     rest &= rest - 1u;
-                    if (is_tap(i, __ldg(gl + 32 * q + c), a.window, a.half, G.dil, a.causal))
-                        m &= ~(1u << c);
+                    const int d = __shfl_sync(0xffffffffu, jpos[w], c) - i;
+                    if (d >= -span_lo && d <= span_hi) m &= ~(1u << c);
                 }
-                mw[q] = m;
+                mw[w] = m;
             }
             need_mask = true;
         } else {
@@ -767,7 +794,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         mbar_fence_init();
     }
     if (warp == kWarpProducer && lane == 0)
+    {
         for (int m = 0; m < kMapCount; ++m) tma_prefetch_map(&p.maps[m]);
+        for (int m = 0; m < p.n_res; ++m) {
+            tma_prefetch_map(&p.res_q[m]);
+            tma_prefetch_map(&p.res_k[m]);
+            tma_prefetch_map(&p.res_v[m]);
+        }
+    }
     if (warp == kWarpMma) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
         tmem_relinquish();
@@ -866,14 +900,17 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder()
     return fn;
 }
 
-// Whole tiles of box_rows rows of one (batch*head) slice: dims {64, n, B*H}.
+// Whole tiles of box_rows rows of the residue class r of dilation dil of each
+// (batch*head) slice: rows r, r+dil, ... ; dims {64, ceil((n-r)/dil), B*H}.
 bool encode_tile_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int n, int BH,
-                     int box_rows)
+                     int box_rows, int dil, int r)
 {
     auto enc = get_encoder();
     if (!enc) return false;
-    cuuint64_t dims[3] = {cuuint64_t(kDHead), cuuint64_t(n), cuuint64_t(BH)};
-    cuuint64_t strides[2] = {cuuint64_t(kRowBytes), cuuint64_t(n) * kRowBytes};
+    const int n_r = (n - r + dil - 1) / dil;
+    base = static_cast<const char *>(base) + size_t(r) * kRowBytes;
+    cuuint64_t dims[3] = {cuuint64_t(kDHead), cuuint64_t(n_r), cuuint64_t(BH)};
+    cuuint64_t strides[2] = {cuuint64_t(dil) * kRowBytes, cuuint64_t(n) * kRowBytes};
     cuuint32_t box[3] = {kDHead, cuuint32_t(box_rows), 1};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, es,
@@ -899,30 +936,34 @@ bool encode_row_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, lo
 
 struct MapCacheEntry {
     const void *base;
-    int kind, dt, n, BH;
+    int kind, dt, n, BH, dil, r;
     CUtensorMap map;
     bool used;
 };
 
 // Encoded tensor maps, reused while the same buffer and shape come back.
 // kind: 0 = tiles of 128 rows, 1 = single rows, 2 = tiles of kKeys rows.
-bool cached_map(CUtensorMap *out, int kind, const void *base, CUtensorMapDataType dt, int n, int BH)
+bool cached_map(CUtensorMap *out, int kind, const void *base, CUtensorMapDataType dt, int n, int BH,
+                int dil = 1, int r = 0)
 {
+    constexpr int kCache = 256;
     static std::mutex mu;
-    static MapCacheEntry cache[64];
+    static MapCacheEntry cache[kCache];
     static unsigned next = 0;
     std::lock_guard<std::mutex> lock(mu);
     for (auto &e : cache)
-        if (e.used && e.base == base && e.kind == kind && e.dt == int(dt) && e.n == n && e.BH == BH) {
+        if (e.used && e.base == base && e.kind == kind && e.dt == int(dt) && e.n == n &&
+            e.BH == BH && e.dil == dil && e.r == r) {
             *out = e.map;
             return true;
         }
     CUtensorMap m;
     const bool ok = kind == 1 ? encode_row_map(&m, base, dt, long(n) * BH)
-                              : encode_tile_map(&m, base, dt, n, BH, kind == 0 ? kRows : kKeys);
+                              : encode_tile_map(&m, base, dt, n, BH, kind == 0 ? kRows : kKeys,
+                                                dil, r);
     if (!ok) return false;
-    MapCacheEntry &e = cache[next++ % 64];
-    e = MapCacheEntry{base, kind, int(dt), n, BH, m, true};
+    MapCacheEntry &e = cache[next++ % kCache];
+    e = MapCacheEntry{base, kind, int(dt), n, BH, dil, r, m, true};
     *out = m;
     return true;
 }
@@ -943,9 +984,24 @@ int launch_typed(const AttnArgs &a, CUtensorMapDataType dt, cudaStream_t stream)
     p.a = a;
     const int BH = a.B * a.H;
     bool ok = true;
-    ok = ok && cached_map(&p.maps[kMapQTile], 0, a.q, dt, a.n, BH);
-    ok = ok && cached_map(&p.maps[kMapKTile], 2, a.k, dt, a.n, BH);
-    ok = ok && cached_map(&p.maps[kMapVTile], 2, a.v, dt, a.n, BH);
+    // Residue maps of every distinct dilation, while they fit.
+    for (int h = 0; h < a.H; ++h) p.res_base[h] = -1;
+    p.n_res = 0;
+    for (int h = 0; h < a.H; ++h) {
+        if (p.res_base[h] >= 0) continue;
+        const int dil = a.dil[h];
+        const int nres = std::min(dil, a.n);
+        if (p.n_res + nres > kMaxResidues) continue;
+        const int base = p.n_res;
+        for (int r = 0; r < nres && ok; ++r) {
+            ok = ok && cached_map(&p.res_q[base + r], 0, a.q, dt, a.n, BH, dil, r);
+            ok = ok && cached_map(&p.res_k[base + r], 2, a.k, dt, a.n, BH, dil, r);
+            ok = ok && cached_map(&p.res_v[base + r], 2, a.v, dt, a.n, BH, dil, r);
+        }
+        p.n_res += nres;
+        for (int h2 = h; h2 < a.H; ++h2)
+            if (a.dil[h2] == dil) p.res_base[h2] = base;
+    }
     ok = ok && cached_map(&p.maps[kMapKgTile], 2, a.kg, dt, a.n, BH);
     ok = ok && cached_map(&p.maps[kMapVgTile], 2, a.vg, dt, a.n, BH);
     ok = ok && cached_map(&p.maps[kMapQRow], 1, a.q, dt, a.n, BH);
