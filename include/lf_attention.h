@@ -59,7 +59,7 @@ typedef enum {
 
 typedef enum {
     LF_OK = 0,
-    LF_ERR_INVALID_ARG = -1,      /* bad size, pointer, window or dilation */
+    LF_ERR_INVALID_ARG = -1,      /* bad size, pointer, alignment, window or dilation */
     LF_ERR_UNSUPPORTED = -2,      /* d_head != 64; causal with global tokens */
     LF_ERR_WORKSPACE = -3,        /* workspace NULL, misaligned or too small */
     LF_ERR_CUDA = -4,             /* a CUDA runtime call failed */
@@ -120,7 +120,8 @@ LF_API int lf_attention_prepare(int B, int H, int n, int d_head,
  * The attention itself, on a workspace prepared by lf_attention_prepare with
  * the same B, H, n, d_head, max_global and masks.
  *
- *   dtype        element type of all seven tensors.
+ *   dtype        element type of all seven tensors.  Each of the seven
+ *                pointers must be 16-byte aligned (LF_ERR_INVALID_ARG).
  *   q, k, v      device [B, H, n, d_head]: the sliding-window projections.
  *   qg, kg, vg   device [B, H, n, d_head]: the global projections; qg is read
  *                only at global rows.  May alias q, k, v.
@@ -128,10 +129,9 @@ LF_API int lf_attention_prepare(int B, int H, int n, int d_head,
  *                t in [-w/2, w/2].  Causal: >= 1; taps i - t*dil[h] for
  *                t in [0, w-1].  Taps outside [0, n) are dropped.
  *   dilation     host int32 [H], every entry >= 1.  NULL: all 1.
- *   causal       0 or 1.  Causal attention with global tokens is
- *                LF_ERR_UNSUPPORTED (rejected by lf_attention_prepare's
- *                caller-visible max_global: pass max_global = 0 and a NULL
- *                global mask).
+ *   causal       0 or 1.  Causal attention takes no global tokens: with
+ *                causal = 1 a max_global other than 0 is LF_ERR_UNSUPPORTED
+ *                (prepare with max_global = 0 and a NULL global mask).
  *   out          device [B, H, n, d_head], same dtype.  Every row is written:
  *                padded rows with zeros.  Must not alias an input.
  *

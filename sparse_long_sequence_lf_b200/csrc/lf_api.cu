@@ -116,6 +116,9 @@ int lf_attention_run(lf_dtype dtype, int B, int H, int n, int d_head, const void
     if (elem_size(dtype) == 0) return LF_ERR_INVALID_ARG;
     if (!sizes_ok(B, H, n) || max_global < 0 || max_global > n) return LF_ERR_INVALID_ARG;
     if (!q || !k || !v || !qg || !kg || !vg || !out) return LF_ERR_INVALID_ARG;
+    // Tiles move as 16-byte pieces (TMA boxes, vector loads).
+    for (const void *ptr : {q, k, v, qg, kg, vg, static_cast<const void *>(out)})
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return LF_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return LF_ERR_INVALID_ARG;
     if (causal) {
         if (window < 1) return LF_ERR_INVALID_ARG;

@@ -26,12 +26,65 @@ namespace lf {
 constexpr int kSimtRows = 128;
 constexpr int kSimtKeys = 32;
 
+// Four consecutive elements of a 16-byte (fp32) or 8-byte (fp16/bf16)
+// aligned address, as floats.
+template <typename T> __device__ __forceinline__ float4 load4(const T *p);
+template <> __device__ __forceinline__ float4 load4<float>(const float *p)
+{
+    return __ldg(reinterpret_cast<const float4 *>(p));
+}
+template <> __device__ __forceinline__ float4 load4<__half>(const __half *p)
+{
+    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&u.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16 *p)
+{
+    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+template <typename T> __device__ __forceinline__ void store4(T *p, float4 v);
+template <> __device__ __forceinline__ void store4<float>(float *p, float4 v)
+{
+    *reinterpret_cast<float4 *>(p) = v;
+}
+template <> __device__ __forceinline__ void store4<__half>(__half *p, float4 v)
+{
+    __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t *>(&a);
+    u.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = u;
+}
+template <> __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, float4 v)
+{
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t *>(&a);
+    u.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = u;
+}
+
+// One staged tile of 32 keys: each thread holds 4 of the 512 four-element
+// pieces of K and of V (key c = tid/16 + 8u, dims 4*(tid%16) .. +3), loaded
+// into registers while the previous tile is being consumed.
+struct KvStage {
+    float4 k[4], v[4];
+    int pos[4];
+};
+
 template <typename T>
 __global__ void __launch_bounds__(kSimtRows)
 band_simt_kernel(const AttnArgs a)
 {
-    __shared__ float ks[kSimtKeys][kDHead];
-    __shared__ float vs[kSimtKeys][kDHead];
+    __shared__ __align__(16) float ks[kSimtKeys][kDHead];
+    __shared__ __align__(16) float vs[kSimtKeys][kDHead];
+    __shared__ float ss[kSimtKeys][kSimtRows];   // scores, column = thread
     __shared__ int kpos[kSimtKeys];    // sequence position of each staged key, -1 = not a key
 
     int b, h, r, tile;
@@ -53,9 +106,13 @@ band_simt_kernel(const AttnArgs a)
 
     float q[kDHead], acc[kDHead];
 #pragma unroll
-    for (int x = 0; x < kDHead; ++x) {
-        q[x] = row_in ? to_f32(Q[size_t(i) * kDHead + x]) * a.scale_log2 : 0.f;
-        acc[x] = 0.f;
+    for (int x = 0; x < kDHead; x += 4) {
+        const float4 t = row_in ? load4(Q + size_t(i) * kDHead + x) : make_float4(0.f, 0.f, 0.f, 0.f);
+        q[x] = t.x * a.scale_log2;
+        q[x + 1] = t.y * a.scale_log2;
+        q[x + 2] = t.z * a.scale_log2;
+        q[x + 3] = t.w * a.scale_log2;
+        acc[x] = acc[x + 1] = acc[x + 2] = acc[x + 3] = 0.f;
     }
     float m = -INFINITY, l = 0.f;
 
@@ -72,27 +129,46 @@ band_simt_kernel(const AttnArgs a)
     lo = max(lo, 0);
     hi = min(hi, n_r - 1);
 
-    auto consume = [&](bool band_tile) {
-        float s[kSimtKeys];
+    // Scores of the staged keys go through shared memory (one column per
+    // thread), so the key loops stay rolled: fully unrolled 32-key x 64-dim
+    // loops are too large for the instruction cache.
+    auto consume = [&](int k0, bool band_tile) {
         float tmax = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < kSimtKeys; c += 2) {
+            float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < kSimtKeys; ++c) {
-            const int j = kpos[c];
-            bool ok = row_in && j >= 0;
-            if (ok) {
-                if (band_tile) {
-                    const int jr = (j - r) / dil;
-                    ok = a.causal ? (jr <= ir && ir - jr <= a.window - 1)
-                                  : (jr - ir <= a.half && ir - jr <= a.half);
-                } else {
-                    ok = !is_tap(i, j, a.window, a.half, dil, a.causal);
-                }
+            for (int x = 0; x < kDHead; x += 4) {
+                const float4 ka = *reinterpret_cast<const float4 *>(&ks[c][x]);
+                const float4 kb = *reinterpret_cast<const float4 *>(&ks[c + 1][x]);
+                d0[0] = fmaf(q[x], ka.x, d0[0]);
+                d0[1] = fmaf(q[x + 1], ka.y, d0[1]);
+                d0[2] = fmaf(q[x + 2], ka.z, d0[2]);
+                d0[3] = fmaf(q[x + 3], ka.w, d0[3]);
+                d1[0] = fmaf(q[x], kb.x, d1[0]);
+                d1[1] = fmaf(q[x + 1], kb.y, d1[1]);
+                d1[2] = fmaf(q[x + 2], kb.z, d1[2]);
+                d1[3] = fmaf(q[x + 3], kb.w, d1[3]);
             }
-            float dot = 0.f;
 #pragma unroll
-            for (int x = 0; x < kDHead; ++x) dot = fmaf(q[x], ks[c][x], dot);
-            s[c] = ok ? dot : -INFINITY;
-            tmax = fmaxf(tmax, s[c]);
+            for (int u = 0; u < 2; ++u) {
+                const int j = kpos[c + u];
+                bool ok = row_in && j >= 0;
+                if (ok) {
+                    if (band_tile) {
+                        const int jr = k0 + c + u;
+                        ok = a.causal ? (jr <= ir && ir - jr <= a.window - 1)
+                                      : (jr - ir <= a.half && ir - jr <= a.half);
+                    } else {
+                        ok = !is_tap(i, j, a.window, a.half, dil, a.causal);
+                    }
+                }
+                const float *d = u ? d1 : d0;
+                const float dot = (d[0] + d[1]) + (d[2] + d[3]);
+                const float sc = ok ? dot : -INFINITY;
+                ss[c + u][tid] = sc;
+                tmax = fmaxf(tmax, sc);
+            }
         }
         const float mnew = fmaxf(m, tmax);
         const float base = (mnew == -INFINITY) ? 0.f : mnew;
@@ -100,61 +176,77 @@ band_simt_kernel(const AttnArgs a)
         l *= corr;
 #pragma unroll
         for (int x = 0; x < kDHead; ++x) acc[x] *= corr;
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < kSimtKeys; ++c) {
-            const float p = exp2f(s[c] - base);
+            const float p = exp2f(ss[c][tid] - base);
             l += p;
 #pragma unroll
-            for (int x = 0; x < kDHead; ++x) acc[x] = fmaf(p, vs[c][x], acc[x]);
+            for (int x = 0; x < kDHead; x += 4) {
+                const float4 vv = *reinterpret_cast<const float4 *>(&vs[c][x]);
+                acc[x] = fmaf(p, vv.x, acc[x]);
+                acc[x + 1] = fmaf(p, vv.y, acc[x + 1]);
+                acc[x + 2] = fmaf(p, vv.z, acc[x + 2]);
+                acc[x + 3] = fmaf(p, vv.w, acc[x + 3]);
+            }
         }
         m = mnew;
     };
 
-    // Window taps, 32 residue-space keys at a time.
-    for (int k0 = lo; k0 <= hi; k0 += kSimtKeys) {
-        __syncthreads();
-        for (int e = tid; e < kSimtKeys * kDHead; e += kSimtRows) {
-            const int c = e / kDHead, x = e % kDHead;
-            const int jr = k0 + c;
-            const int j = jr * dil + r;
-            const bool in = jr <= hi && j < n;
-            ks[c][x] = in ? to_f32(K[size_t(j) * kDHead + x]) : 0.f;
-            vs[c][x] = in ? to_f32(V[size_t(j) * kDHead + x]) : 0.f;
-            if (x == 0) kpos[c] = (in && bit_at(vb, j)) ? j : -1;
-        }
-        __syncthreads();
-        consume(true);
-    }
-
-    // Global-token columns (keys that are not already window taps).
+    // Key tiles: the window taps, 32 residue-space keys at a time, then the
+    // global-token columns (keys that are not already window taps), 32 slots
+    // at a time.  The next tile's loads are in flight during each consume.
     int g = a.ws.counts[b];
     g = min(g, a.max_global);
     const int *gl = a.ws.gidx + size_t(b) * n;
-    for (int s0 = 0; s0 < g; s0 += kSimtKeys) {
+    const int nband = hi >= lo ? (hi - lo) / kSimtKeys + 1 : 0;
+    const int ntiles = nband + (g + kSimtKeys - 1) / kSimtKeys;
+    const int x4 = 4 * (tid & 15);
+    auto fetch = [&](int t, KvStage &st) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = (tid >> 4) + 8 * u;
+            int j;
+            if (t < nband) {
+                const int jr = lo + kSimtKeys * t + c;
+                j = (jr <= hi && jr * dil + r < n) ? jr * dil + r : -1;
+            } else {
+                const int slot = kSimtKeys * (t - nband) + c;
+                j = slot < g ? gl[slot] : -1;
+            }
+            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+            st.k[u] = j >= 0 ? load4(K + size_t(j) * kDHead + x4) : z;
+            st.v[u] = j >= 0 ? load4(V + size_t(j) * kDHead + x4) : z;
+            st.pos[u] = (j >= 0 && bit_at(vb, j)) ? j : -1;
+        }
+    };
+    KvStage st;
+    if (ntiles > 0) fetch(0, st);
+    for (int t = 0; t < ntiles; ++t) {
         __syncthreads();
-        for (int e = tid; e < kSimtKeys * kDHead; e += kSimtRows) {
-            const int c = e / kDHead, x = e % kDHead;
-            const int slot = s0 + c;
-            const int j = slot < g ? gl[slot] : -1;
-            ks[c][x] = j >= 0 ? to_f32(K[size_t(j) * kDHead + x]) : 0.f;
-            vs[c][x] = j >= 0 ? to_f32(V[size_t(j) * kDHead + x]) : 0.f;
-            if (x == 0) kpos[c] = (j >= 0 && bit_at(vb, j)) ? j : -1;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = (tid >> 4) + 8 * u;
+            *reinterpret_cast<float4 *>(&ks[c][x4]) = st.k[u];
+            *reinterpret_cast<float4 *>(&vs[c][x4]) = st.v[u];
+            if (x4 == 0) kpos[c] = st.pos[u];
         }
         __syncthreads();
-        consume(false);
+        if (t + 1 < ntiles) fetch(t + 1, st);
+        consume(lo + kSimtKeys * t, t < nband);
     }
 
     if (!row_in) return;
     T *O = static_cast<T *>(a.out) + bh * n * kDHead + size_t(i) * kDHead;
     if (!bit_at(vb, i)) {
 #pragma unroll
-        for (int x = 0; x < kDHead; ++x) O[x] = from_f32<T>(0.f);
+        for (int x = 0; x < kDHead; x += 4) store4(O + x, make_float4(0.f, 0.f, 0.f, 0.f));
         return;
     }
     if (bit_at(gb, i)) return;     // written by the global-row kernel
     const float inv = 1.f / l;
 #pragma unroll
-    for (int x = 0; x < kDHead; ++x) O[x] = from_f32<T>(acc[x] * inv);
+    for (int x = 0; x < kDHead; x += 4)
+        store4(O + x, make_float4(acc[x] * inv, acc[x + 1] * inv, acc[x + 2] * inv, acc[x + 3] * inv));
 }
 
 constexpr int kGlobWarps = 4;
@@ -165,9 +257,9 @@ template <typename T>
 __global__ void __launch_bounds__(kGlobWarps * 32)
 global_simt_kernel(const AttnArgs a)
 {
-    __shared__ float qs[kSlotGroup][kDHead];
+    __shared__ __align__(16) float qs[kSlotGroup][kDHead];
     __shared__ float ks[kGlobKeys][kDHead + 1];
-    __shared__ float vs[kGlobKeys][kDHead];
+    __shared__ __align__(16) float vs[kGlobKeys][kDHead];
     __shared__ int kok[kGlobKeys];
     __shared__ int s_last;
 
@@ -188,10 +280,16 @@ global_simt_kernel(const AttnArgs a)
     const T *Kg = static_cast<const T *>(a.kg) + size_t(bh) * n * kDHead;
     const T *Vg = static_cast<const T *>(a.vg) + size_t(bh) * n * kDHead;
 
-    for (int e = tid; e < kSlotGroup * kDHead; e += blockDim.x) {
-        const int s = e / kDHead, x = e % kDHead;
+    const int x4 = 4 * (tid & 15);
+#pragma unroll
+    for (int u = 0; u < kSlotGroup / 8; ++u) {
+        const int s = (tid >> 4) + 8 * u;
         const int slot = slot0 + s;
-        qs[s][x] = slot < g ? to_f32(Qg[size_t(gl[slot]) * kDHead + x]) * a.scale_log2 : 0.f;
+        const float4 t = slot < g ? load4(Qg + size_t(gl[slot]) * kDHead + x4)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(&qs[s][x4]) =
+            make_float4(t.x * a.scale_log2, t.y * a.scale_log2, t.z * a.scale_log2,
+                        t.w * a.scale_log2);
     }
 
     float m[kGlobSlotsPerWarp], l[kGlobSlotsPerWarp], acc0[kGlobSlotsPerWarp],
@@ -204,19 +302,37 @@ global_simt_kernel(const AttnArgs a)
         acc1[t] = 0.f;
     }
 
+    // Key tiles of 64: each thread holds 8 of the 1024 four-element pieces of
+    // Kg and of Vg (key c = tid/16 + 8u), loaded while the previous tile is
+    // being consumed.
     const int key_begin = chunk * kChunkKeys;
     const int key_end = min(n, key_begin + kChunkKeys);
+    constexpr int kPieces = kGlobKeys / 8;
+    float4 kr[kPieces], vr[kPieces];
+    auto fetch = [&](int k0) {
+#pragma unroll
+        for (int u = 0; u < kPieces; ++u) {
+            const int j = k0 + (tid >> 4) + 8 * u;
+            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+            kr[u] = j < key_end ? load4(Kg + size_t(j) * kDHead + x4) : z;
+            vr[u] = j < key_end ? load4(Vg + size_t(j) * kDHead + x4) : z;
+        }
+    };
+    fetch(key_begin);
     for (int k0 = key_begin; k0 < key_end; k0 += kGlobKeys) {
         __syncthreads();
-        for (int e = tid; e < kGlobKeys * kDHead; e += blockDim.x) {
-            const int c = e / kDHead, x = e % kDHead;
-            const int j = k0 + c;
-            const bool in = j < key_end;
-            ks[c][x] = in ? to_f32(Kg[size_t(j) * kDHead + x]) : 0.f;
-            vs[c][x] = in ? to_f32(Vg[size_t(j) * kDHead + x]) : 0.f;
-            if (x == 0) kok[c] = in && bit_at(vb, j);
+#pragma unroll
+        for (int u = 0; u < kPieces; ++u) {
+            const int c = (tid >> 4) + 8 * u;
+            ks[c][x4] = kr[u].x;
+            ks[c][x4 + 1] = kr[u].y;
+            ks[c][x4 + 2] = kr[u].z;
+            ks[c][x4 + 3] = kr[u].w;
+            *reinterpret_cast<float4 *>(&vs[c][x4]) = vr[u];
         }
+        if (tid < kGlobKeys) kok[tid] = k0 + tid < key_end && bit_at(vb, k0 + tid);
         __syncthreads();
+        if (k0 + kGlobKeys < key_end) fetch(k0 + kGlobKeys);
 #pragma unroll
         for (int t = 0; t < kGlobSlotsPerWarp; ++t) {
             const int s = warp * kGlobSlotsPerWarp + t;

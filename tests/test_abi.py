@@ -40,8 +40,10 @@ def test_workspace_size(L):
 
 
 def _run(L, **over):
-    a = dict(dtype=2, B=1, H=2, n=64, d=64, q=1, k=1, v=1, qg=1, kg=1, vg=1, max_global=0,
-             window=8, dil=None, causal=0, out=1, ws=256, wsb=1 << 20)
+    # Fake, 256-byte aligned addresses: every call below fails a host-side
+    # check or finds no device before anything is dereferenced.
+    a = dict(dtype=2, B=1, H=2, n=64, d=64, q=256, k=256, v=256, qg=256, kg=256, vg=256,
+             max_global=0, window=8, dil=None, causal=0, out=512, ws=256, wsb=1 << 20)
     a.update(over)
     P = ctypes.c_void_p
     return L.lf_attention_run(a["dtype"], a["B"], a["H"], a["n"], a["d"], P(a["q"]), P(a["k"]),
@@ -58,6 +60,8 @@ def test_argument_checks_before_any_launch(L):
     assert _run(L, causal=1, window=0) == -1
     assert _run(L, causal=1, max_global=2) == -2
     assert _run(L, q=0) == -1
+    assert _run(L, q=264) == -1                       # not 16-byte aligned
+    assert _run(L, out=520) == -1
     assert _run(L, n=0) == -1
     assert _run(L, ws=0) == -3
     assert _run(L, ws=255) == -3                      # misaligned workspace

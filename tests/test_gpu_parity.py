@@ -220,3 +220,18 @@ def test_invalid_arguments(kw, code):
         lf.attention_forward(g["q"], g["k"], g["v"], g["qg"], g["kg"], g["vg"], None,
                              g["global_mask"], **args)
     assert e.value.code == code
+
+
+def test_misaligned_tensor_rejected():
+    # A tensor that starts 4 bytes past a 16-byte boundary is refused before
+    # any launch.
+    wl = Workload("misaligned", "bf16", 1, 2, 256, 16, globals_kind="first:1")
+    g = to_dev(make_inputs(wl))
+    q = g["q"]
+    buf = torch.zeros(q.numel() + 8, dtype=q.dtype, device=q.device)
+    q_off = buf[2:2 + q.numel()].view(q.shape)
+    q_off.copy_(q)
+    with pytest.raises(lf.LfError) as e:
+        lf.attention_forward(q_off, g["k"], g["v"], g["qg"], g["kg"], g["vg"], None,
+                             g["global_mask"], window=16, max_global=1)
+    assert e.value.code == -1
