@@ -65,7 +65,8 @@ typedef enum {
     LF_ERR_CUDA = -4,             /* a CUDA runtime call failed */
     LF_ERR_DEVICE_TIMEOUT = -5,   /* a bounded device-side wait ran out */
     LF_ERR_GLOBAL_OVERFLOW = -6,  /* a batch has more global tokens than max_global */
-    LF_ERR_NO_DEVICE = -7         /* no sm_100 device is current */
+    LF_ERR_NO_DEVICE = -7,        /* no sm_100 device is current */
+    LF_ERR_SCRATCH_LIMIT = -8     /* too large for the fixed scratch (lf_attention_forward_static) */
 } lf_status;
 
 /* Library version, major*10000 + minor*100 + patch. */
@@ -191,6 +192,47 @@ LF_API int lf_attention_forward_host(lf_dtype dtype, int B, int H, int n, int d_
  * the synchronisation or the copy failed.
  */
 LF_API int lf_workspace_status(const void *workspace, lf_stream_t stream);
+
+/* Size of the fixed scratch of lf_attention_forward_static: 16 MiB. */
+#define LF_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/*
+ * lf_attention_forward with its workspace in a fixed scratch array of
+ * LF_STATIC_SCRATCH_BYTES per device, held in the library's own device
+ * global memory.  The pages describe nothing like it: it has no counterpart
+ * in the method and computes exactly what lf_attention_forward computes; only
+ * the place of the workspace differs.
+ *
+ * It is for callers that cannot allocate device memory when they call: a
+ * host program or plugin that receives device tensors and a stream but owns
+ * no device allocator, or a latency-bound loop where cudaMalloc / cudaFree
+ * are off limits because they can synchronise the device.  It allocates
+ * nothing itself.
+ *
+ *   arguments    as lf_attention_forward, without workspace and
+ *                workspace_bytes.
+ *   scratch      optional (may be NULL); out: the device address of the
+ *                scratch used, to pass to lf_workspace_status to read the
+ *                device-side status word of the call.
+ *
+ * Limit: a problem with lf_workspace_size(B, H, n, d_head, max_global) above
+ * LF_STATIC_SCRATCH_BYTES returns LF_ERR_SCRATCH_LIMIT before anything
+ * touches the device (for example B = 1, H = 16, n = 16384 with 32 global
+ * tokens needs about 4.5 MB).
+ * Set-up: the first call on a device looks up the scratch address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.
+ * Concurrency: there is one scratch per device, so calls on the same device
+ * that overlap in time (several streams or host threads) race on it; callers
+ * serialise them.  Nothing must be cleared beforehand: each call's
+ * mask-preparation step clears what has to start at zero.
+ */
+LF_API int lf_attention_forward_static(lf_dtype dtype, int B, int H, int n, int d_head,
+                         const void *q, const void *k, const void *v,
+                         const void *qg, const void *kg, const void *vg,
+                         const uint8_t *local_mask, const uint8_t *global_mask,
+                         int max_global, int window, const int32_t *dilation, int causal,
+                         void *out, lf_stream_t stream, void **scratch);
 
 #ifdef __cplusplus
 }

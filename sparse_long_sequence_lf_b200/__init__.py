@@ -5,11 +5,11 @@ The compute path is the CUDA library under ``csrc/`` behind the C ABI
 package loads nothing; the first API call loads the library and raises if it
 is missing.
 """
-from .api import (attention_forward, attention_forward_host, attention_prepare, attention_run,
-                  global_index, host_staging_size, new_workspace, workspace_size,
-                  workspace_status)
+from .api import (attention_forward, attention_forward_host, attention_forward_static,
+                  attention_prepare, attention_run, global_index, host_staging_size,
+                  new_workspace, scratch_status, workspace_size, workspace_status)
 from ._lib import LfError
 
-__all__ = ["attention_forward", "attention_forward_host", "attention_prepare", "attention_run",
-           "global_index", "host_staging_size", "new_workspace", "workspace_size",
-           "workspace_status", "LfError"]
+__all__ = ["attention_forward", "attention_forward_host", "attention_forward_static",
+           "attention_prepare", "attention_run", "global_index", "host_staging_size",
+           "new_workspace", "scratch_status", "workspace_size", "workspace_status", "LfError"]

@@ -24,7 +24,9 @@ STATUS = {
     -5: "LF_ERR_DEVICE_TIMEOUT",
     -6: "LF_ERR_GLOBAL_OVERFLOW",
     -7: "LF_ERR_NO_DEVICE",
+    -8: "LF_ERR_SCRATCH_LIMIT",
 }
+STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 _lock = threading.Lock()
 _lib: ctypes.CDLL | None = None
@@ -59,6 +61,8 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         "lf_attention_forward_host": (I, [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P, I, P,
                                           P, Z, P, Z, P]),
         "lf_workspace_status": (I, [P, P]),
+        "lf_attention_forward_static": (I, [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P, I, P,
+                                            P, ctypes.POINTER(P)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

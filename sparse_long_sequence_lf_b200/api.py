@@ -173,3 +173,31 @@ def attention_forward_host(q, k, v, qg, kg, vg, local_mask=None, global_mask=Non
 def workspace_status(workspace, stream=None) -> int:
     """Synchronises the stream and returns the device status word."""
     return int(_lib.lib().lf_workspace_status(_ptr(workspace), _stream_ptr(stream)))
+
+
+def attention_forward_static(q, k, v, qg, kg, vg, local_mask=None, global_mask=None, *, window,
+                             dilation=None, causal=False, max_global, out, stream=None) -> int:
+    """``lf_attention_forward_static``: the forward with its workspace in the
+    library's fixed per-device scratch (no device allocation by the call).
+
+    ``out`` and ``max_global`` are required, so the binding allocates nothing
+    either.  Returns the device address of the scratch, for
+    ``scratch_status``.  Calls on one device must not overlap in time.
+    """
+    dt, (B, H, n, _) = _check_projections([q, k, v, qg, kg, vg])
+    _check_projections([q, out])
+    lm = _mask(local_mask, B, n, "local_mask")
+    gm = _mask(global_mask, B, n, "global_mask")
+    scratch = ctypes.c_void_p()
+    _lib.check(_lib.lib().lf_attention_forward_static(
+        dt, B, H, n, D_HEAD, _ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg), _ptr(vg), _ptr(lm),
+        _ptr(gm), int(max_global), int(window), _dilation(dilation, H), int(bool(causal)),
+        _ptr(out), _stream_ptr(stream), ctypes.byref(scratch)),
+        "lf_attention_forward_static")
+    return int(scratch.value)
+
+
+def scratch_status(scratch: int, stream=None) -> int:
+    """Synchronises the stream and returns the status word of the last
+    ``attention_forward_static`` call that used ``scratch``."""
+    return int(_lib.lib().lf_workspace_status(ctypes.c_void_p(scratch), _stream_ptr(stream)))

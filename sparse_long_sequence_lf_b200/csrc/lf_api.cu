@@ -73,6 +73,8 @@ const char *lf_status_string(int status)
         case LF_ERR_DEVICE_TIMEOUT: return "bounded device-side wait ran out";
         case LF_ERR_GLOBAL_OVERFLOW: return "more global tokens than max_global";
         case LF_ERR_NO_DEVICE: return "no sm_100 device is current";
+        case LF_ERR_SCRATCH_LIMIT:
+            return "workspace would exceed the fixed 16 MiB scratch of lf_attention_forward_static";
     }
     return "unknown status";
 }
