@@ -192,9 +192,14 @@ def make_device_sets(wl, nsets, device):
 
 
 def launches_per_step(wl, max_global):
-    # prepare kernel + attention kernel, plus the global-row kernel (fp32) or
-    # the global-row combine kernel (bf16/fp16) when there are global tokens
-    return 2 + (1 if max_global > 0 else 0)
+    # prepare kernel + attention kernel; with global tokens fp32 adds its
+    # global-row kernel, bf16/fp16 merge them inside the attention kernel up to
+    # 8 chunks of 512 keys and add the merge kernel beyond
+    if max_global == 0:
+        return 2
+    if wl.dtype == "f32":
+        return 3
+    return 2 if -(-wl.n // 512) <= 8 else 3
 
 
 def run_gpu_arm(args, wl, world, rank, local):

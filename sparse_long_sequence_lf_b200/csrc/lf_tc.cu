@@ -87,6 +87,7 @@ enum MapId { kMapKgTile, kMapVgTile, kMapQRow, kMapKRow, kMapVRow, kMapQgRow, kM
 // copy.  Up to kMaxResidues (dilation, residue) pairs per call; heads beyond
 // that load their rows one by one.
 constexpr int kMaxResidues = 24;
+constexpr int kMergeInKernelChunks = 8;           // longest sequence merged in-kernel: 4096
 
 struct TcParams {
     CUtensorMap maps[kMapCount];              // first: 64-byte aligned
@@ -100,6 +101,7 @@ struct TcParams {
     int gtiles;           // ceil(max_global / 128)
     int oob_row;          // a row coordinate past the end of the row maps (reads zeros)
     int n_res;            // residue maps in use
+    int merge_in_kernel;  // global rows merged by the last chunk (else by combine_kernel)
 };
 
 // Kernel arguments above 4 KB need CUDA 12.1 or newer (up to 32764 bytes).
@@ -639,6 +641,39 @@ __device__ __forceinline__ void store_row(T *dst, const float (&o)[64], float in
     }
 }
 
+// Merges the chunk partials of the global rows slot0 .. slot0 + 31 (lane =
+// row) by log-sum-exp and writes their output rows.  Called by the warp that
+// wrote the last chunk of the group; the partials of the other chunks come
+// from other CTAs, so they are read past L1.
+template <typename T>
+__device__ __noinline__ void merge_global_rows(const AttnArgs &a, int b, int bh, int g, int slot0,
+                                               int lane)
+{
+    const int slot = slot0 + lane;
+    if (slot >= g) return;
+    const int pos = a.ws.gidx[size_t(b) * a.n + slot];
+    if (!bit_at(a.ws.vbits + size_t(b) * a.L.nwords, pos)) return;   // padded: zeros elsewhere
+    const size_t mg = size_t(a.max_global);
+    const size_t cstride = kPartialFloats * mg;
+    const float *P = partial_base(a, bh, 0) + slot;
+    const int nch = a.L.nchunks;
+    float M = -INFINITY;
+    for (int c = 0; c < nch; ++c) M = fmaxf(M, __ldcg(P + c * cstride));
+    float L = 0.f, acc[kDHead];
+#pragma unroll
+    for (int x = 0; x < kDHead; ++x) acc[x] = 0.f;
+    for (int c = 0; c < nch; ++c) {
+        const float *pc = P + c * cstride;
+        const float mc = __ldcg(pc);
+        const float f = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+        L = fmaf(f, __ldcg(pc + mg), L);
+#pragma unroll
+        for (int x = 0; x < kDHead; ++x) acc[x] = fmaf(f, __ldcg(pc + (2 + x) * mg), acc[x]);
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    store_row<T>(static_cast<T *>(a.out) + (size_t(bh) * a.n + pos) * kDHead, acc, inv);
+}
+
 template <typename T>
 __device__ __forceinline__ void softmax_role(const TcParams &p, TcSmem &sm, uint32_t tmem, int X,
                                              int tid)
@@ -758,6 +793,24 @@ __device__ __forceinline__ void softmax_role(const TcParams &p, TcSmem &sm, uint
                 if (write) {
                     P[0] = st.m;
                     P[mg] = st.l;
+                }
+                // The last chunk to finish this warp's group of 32 global rows
+                // merges them and resets the group's arrival counter for the
+                // next call on the same workspace.
+                const int group = (G.q0 >> 5) + warp;
+                if (p.merge_in_kernel && group * 32 < G.g) {
+                    __threadfence();
+                    __syncwarp();
+                    int last = 0;
+                    if (lane == 0) {
+                        int *ctr = a.ws.counters + size_t(G.bh) * (a.L.ngroups + 1) + group;
+                        last = atomicAdd(ctr, 1) == a.L.nchunks - 1;
+                        if (last) atomicExch(ctr, 0);
+                    }
+                    if (__shfl_sync(0xffffffffu, last, 0)) {
+                        __threadfence();
+                        merge_global_rows<T>(a, G.b, G.bh, G.g, group * 32, lane);
+                    }
                 }
             }
         }
@@ -1013,6 +1066,9 @@ int launch_typed(const AttnArgs &a, CUtensorMapDataType dt, cudaStream_t stream)
     p.global_items = BH * p.gtiles * a.L.nchunks;
     p.total_items = p.global_items + a.B * a.band_items_per_batch;
     p.oob_row = BH * a.n;
+    // One warp merges 32 global rows over every chunk: cheap for a few chunks,
+    // a separate wide kernel beyond that.
+    p.merge_in_kernel = a.L.nchunks <= kMergeInKernelChunks;
     const size_t smem = sizeof(TcSmem) + 1024;
     static bool attr_set[64] = {};
     int dev = 0;
@@ -1043,7 +1099,7 @@ int launch_typed(const AttnArgs &a, CUtensorMapDataType dt, cudaStream_t stream)
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, attn_tc_kernel<T>, p) != cudaSuccess) return kErrCuda;
-    if (a.max_global > 0) {
+    if (a.max_global > 0 && !p.merge_in_kernel) {
         cudaLaunchConfig_t cc = {};
         cc.gridDim = dim3(a.B * a.H, (a.max_global + 3) / 4);
         cc.blockDim = dim3(128);

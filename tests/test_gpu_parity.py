@@ -54,6 +54,12 @@ EDGE = [
              pad_tail=(0, 41), seed=10),
     Workload("fp32-causal", "f32", 1, 2, 513, 33, dilation=(1, 3), causal=True, seed=11),
     Workload("fp16-w2", "f16", 1, 2, 257, 2, globals_kind="first:3", seed=12),
+    # global rows merged by the last chunk (8 chunks of 512 keys) ...
+    Workload("merge-8-chunks", "bf16", 1, 2, 4096, 16, globals_kind="random:40",
+             pad_tail=(5,), seed=13),
+    # ... and by the separate merge kernel (9 chunks)
+    Workload("merge-9-chunks", "f16", 1, 2, 4097, 16, globals_kind="random:40",
+             pad_tail=(5,), seed=14),
 ]
 
 
