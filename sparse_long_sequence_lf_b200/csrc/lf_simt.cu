@@ -1,14 +1,14 @@
 // CUDA-core kernels of the attention: the fp32 path.
 //
 // fp32 inputs are computed in fp32 on the FMA pipes end to end (the tensor
-// cores' tf32 mode keeps 10 mantissa bits, too few for fp32 parity), with
-// one thread per query row:
+// cores' tf32 mode keeps 10 mantissa bits, too few for fp32 parity):
 //
-//   band kernel     one CTA per 128 query rows of one (batch, head, residue
-//                   class of the dilation); keys stream through shared memory
-//                   32 at a time; an online softmax in registers covers the
-//                   window taps and then the global-token columns.  Writes
-//                   every row except valid global rows (zeros for padding).
+//   band kernel     one CTA per 32 query rows of one (batch, head, residue
+//                   class of the dilation), four threads per row; keys stream
+//                   through shared memory 32 at a time; an online softmax
+//                   covers the window taps and then the global-token columns.
+//                   Writes every row except valid global rows (zeros for
+//                   padding).
 //   global kernel   one CTA per (batch*head, chunk of 512 keys, group of 32
 //                   global rows); a warp owns 8 global rows, lanes split the
 //                   keys for the scores and the head dimension for Vg; writes
@@ -23,7 +23,9 @@
 
 namespace lf {
 
-constexpr int kSimtRows = 128;
+constexpr int kSimtRows = 32;                     // query rows per band CTA
+constexpr int kSimtThreads = 4 * kSimtRows;       // four threads per row
+constexpr int kSimtParts = 128 / kSimtRows;       // band CTAs per 128-row band item
 constexpr int kSimtKeys = 32;
 
 // Four consecutive elements of a 16-byte (fp32) or 8-byte (fp16/bf16)
@@ -78,22 +80,28 @@ struct KvStage {
     int pos[4];
 };
 
+// One CTA per 32 query rows (a quarter of a 128-row band item); four threads
+// per row, each holding a quarter of the head dimension of q and of the
+// accumulator.  Scores are reduced over the four threads with two shuffles.
 template <typename T>
-__global__ void __launch_bounds__(kSimtRows)
+__global__ void __launch_bounds__(kSimtThreads)
 band_simt_kernel(const AttnArgs a)
 {
     __shared__ __align__(16) float ks[kSimtKeys][kDHead];
     __shared__ __align__(16) float vs[kSimtKeys][kDHead];
-    __shared__ float ss[kSimtKeys][kSimtRows];   // scores, column = thread
+    __shared__ float ss[kSimtKeys][kSimtRows];   // scores, column = row of this CTA
     __shared__ int kpos[kSimtKeys];    // sequence position of each staged key, -1 = not a key
 
     int b, h, r, tile;
-    band_item(a, blockIdx.x, b, h, r, tile);
+    band_item(a, blockIdx.x / kSimtParts, b, h, r, tile);
     const int dil = a.dil[h];
     const int n = a.n;
     const int n_r = (n - r + dil - 1) / dil;
     const int tid = threadIdx.x;
-    const int ir = tile * kSimtRows + tid;          // row in residue space
+    const int rl = tid >> 2;                        // row of this CTA
+    const int qd = tid & 3;                         // quarter of the head dimension
+    const int r0 = tile * 128 + (blockIdx.x % kSimtParts) * kSimtRows;   // first residue-space row
+    const int ir = r0 + rl;                         // row in residue space
     const bool row_in = ir < n_r;
     const int i = ir * dil + r;                     // sequence position
     const size_t bh = size_t(b) * a.H + h;
@@ -102,12 +110,16 @@ band_simt_kernel(const AttnArgs a)
     const T *V = static_cast<const T *>(a.v) + bh * n * kDHead;
     const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
     const uint32_t *gb = a.ws.gbits + size_t(b) * a.L.nwords;
-    if (tid == 0 && a.ws.counts[b] > a.max_global) set_status(a.ws.status, kErrGlobalOverflow);
+    if (tid == 0 && blockIdx.x % kSimtParts == 0 && a.ws.counts[b] > a.max_global)
+        set_status(a.ws.status, kErrGlobalOverflow);
+    if (r0 >= n_r) return;                          // no rows in this quarter
 
-    float q[kDHead], acc[kDHead];
+    constexpr int kQ = kDHead / 4;                  // 16 dimensions per thread
+    float q[kQ], acc[kQ];
 #pragma unroll
-    for (int x = 0; x < kDHead; x += 4) {
-        const float4 t = row_in ? load4(Q + size_t(i) * kDHead + x) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int x = 0; x < kQ; x += 4) {
+        const float4 t = row_in ? load4(Q + size_t(i) * kDHead + kQ * qd + x)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
         q[x] = t.x * a.scale_log2;
         q[x + 1] = t.y * a.scale_log2;
         q[x + 2] = t.z * a.scale_log2;
@@ -117,78 +129,72 @@ band_simt_kernel(const AttnArgs a)
     float m = -INFINITY, l = 0.f;
 
     // Residue-space key range covered by the rows of this CTA.
-    const int r0 = tile * kSimtRows;
+    const int rows_hi = min(r0 + kSimtRows - 1, n_r - 1);
     int lo, hi;
     if (a.causal) {
         lo = r0 - (a.window - 1);
-        hi = r0 + kSimtRows - 1;
+        hi = rows_hi;
     } else {
         lo = r0 - a.half;
-        hi = r0 + kSimtRows - 1 + a.half;
+        hi = rows_hi + a.half;
     }
     lo = max(lo, 0);
     hi = min(hi, n_r - 1);
 
-    // Scores of the staged keys go through shared memory (one column per
-    // thread), so the key loops stay rolled: fully unrolled 32-key x 64-dim
-    // loops are too large for the instruction cache.
+    // Pass 1 puts the scores of the staged keys in shared memory, pass 2
+    // takes the exponentials and accumulates P V.
     auto consume = [&](int k0, bool band_tile) {
         float tmax = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < kSimtKeys; c += 2) {
-            float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+        for (int c = 0; c < kSimtKeys; ++c) {
+            float d0 = 0.f, d1 = 0.f;
 #pragma unroll
-            for (int x = 0; x < kDHead; x += 4) {
-                const float4 ka = *reinterpret_cast<const float4 *>(&ks[c][x]);
-                const float4 kb = *reinterpret_cast<const float4 *>(&ks[c + 1][x]);
-                d0[0] = fmaf(q[x], ka.x, d0[0]);
-                d0[1] = fmaf(q[x + 1], ka.y, d0[1]);
-                d0[2] = fmaf(q[x + 2], ka.z, d0[2]);
-                d0[3] = fmaf(q[x + 3], ka.w, d0[3]);
-                d1[0] = fmaf(q[x], kb.x, d1[0]);
-                d1[1] = fmaf(q[x + 1], kb.y, d1[1]);
-                d1[2] = fmaf(q[x + 2], kb.z, d1[2]);
-                d1[3] = fmaf(q[x + 3], kb.w, d1[3]);
+            for (int x = 0; x < kQ; x += 4) {
+                const float4 kv = *reinterpret_cast<const float4 *>(&ks[c][kQ * qd + x]);
+                d0 = fmaf(q[x], kv.x, d0);
+                d1 = fmaf(q[x + 1], kv.y, d1);
+                d0 = fmaf(q[x + 2], kv.z, d0);
+                d1 = fmaf(q[x + 3], kv.w, d1);
             }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int j = kpos[c + u];
-                bool ok = row_in && j >= 0;
-                if (ok) {
-                    if (band_tile) {
-                        const int jr = k0 + c + u;
-                        ok = a.causal ? (jr <= ir && ir - jr <= a.window - 1)
-                                      : (jr - ir <= a.half && ir - jr <= a.half);
-                    } else {
-                        ok = !is_tap(i, j, a.window, a.half, dil, a.causal);
-                    }
+            float dot = d0 + d1;
+            dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+            dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+            const int j = kpos[c];
+            bool ok = row_in && j >= 0;
+            if (ok) {
+                if (band_tile) {
+                    const int jr = k0 + c;
+                    ok = a.causal ? (jr <= ir && ir - jr <= a.window - 1)
+                                  : (jr - ir <= a.half && ir - jr <= a.half);
+                } else {
+                    ok = !is_tap(i, j, a.window, a.half, dil, a.causal);
                 }
-                const float *d = u ? d1 : d0;
-                const float dot = (d[0] + d[1]) + (d[2] + d[3]);
-                const float sc = ok ? dot : -INFINITY;
-                ss[c + u][tid] = sc;
-                tmax = fmaxf(tmax, sc);
             }
+            const float sc = ok ? dot : -INFINITY;
+            if (qd == 0) ss[c][rl] = sc;
+            tmax = fmaxf(tmax, sc);
         }
+        __syncwarp();
         const float mnew = fmaxf(m, tmax);
         const float base = (mnew == -INFINITY) ? 0.f : mnew;
         const float corr = exp2f(m - base);
         l *= corr;
 #pragma unroll
-        for (int x = 0; x < kDHead; ++x) acc[x] *= corr;
-#pragma unroll 1
+        for (int x = 0; x < kQ; ++x) acc[x] *= corr;
+#pragma unroll 2
         for (int c = 0; c < kSimtKeys; ++c) {
-            const float p = exp2f(ss[c][tid] - base);
+            const float p = exp2f(ss[c][rl] - base);
             l += p;
 #pragma unroll
-            for (int x = 0; x < kDHead; x += 4) {
-                const float4 vv = *reinterpret_cast<const float4 *>(&vs[c][x]);
+            for (int x = 0; x < kQ; x += 4) {
+                const float4 vv = *reinterpret_cast<const float4 *>(&vs[c][kQ * qd + x]);
                 acc[x] = fmaf(p, vv.x, acc[x]);
                 acc[x + 1] = fmaf(p, vv.y, acc[x + 1]);
                 acc[x + 2] = fmaf(p, vv.z, acc[x + 2]);
                 acc[x + 3] = fmaf(p, vv.w, acc[x + 3]);
             }
         }
+        __syncwarp();
         m = mnew;
     };
 
@@ -236,16 +242,16 @@ band_simt_kernel(const AttnArgs a)
     }
 
     if (!row_in) return;
-    T *O = static_cast<T *>(a.out) + bh * n * kDHead + size_t(i) * kDHead;
+    T *O = static_cast<T *>(a.out) + bh * n * kDHead + size_t(i) * kDHead + kQ * qd;
     if (!bit_at(vb, i)) {
 #pragma unroll
-        for (int x = 0; x < kDHead; x += 4) store4(O + x, make_float4(0.f, 0.f, 0.f, 0.f));
+        for (int x = 0; x < kQ; x += 4) store4(O + x, make_float4(0.f, 0.f, 0.f, 0.f));
         return;
     }
     if (bit_at(gb, i)) return;     // written by the global-row kernel
     const float inv = 1.f / l;
 #pragma unroll
-    for (int x = 0; x < kDHead; x += 4)
+    for (int x = 0; x < kQ; x += 4)
         store4(O + x, make_float4(acc[x] * inv, acc[x + 1] * inv, acc[x + 2] * inv, acc[x + 3] * inv));
 }
 
@@ -413,7 +419,7 @@ template <typename T>
 int launch_simt(const AttnArgs &a, cudaStream_t stream)
 {
     const int band_items = a.B * a.band_items_per_batch;
-    if (band_items > 0) band_simt_kernel<T><<<band_items, kSimtRows, 0, stream>>>(a);
+    if (band_items > 0) band_simt_kernel<T><<<band_items * kSimtParts, kSimtThreads, 0, stream>>>(a);
     if (a.max_global > 0) {
         dim3 grid(a.L.nchunks, a.B * a.H, a.L.ngroups);
         global_simt_kernel<T><<<grid, kGlobWarps * 32, 0, stream>>>(a);
