@@ -38,7 +38,7 @@
 // Shared-memory tiles have 128-byte rows with the 128-byte swizzle, written
 // by TMA: whole tiles for undilated rows, single-row loads for dilated rows,
 // global tokens and gathered Qg rows.  Q is double-buffered per lane, K/V
-// run through a 4-stage ring of 64-key tiles per lane.  Every wait on an mbarrier is
+// run through a 3-stage ring of 64-key tiles per lane.  Every wait on an mbarrier is
 // bounded; on expiry the kernel records LF_ERR_DEVICE_TIMEOUT, drains its own
 // copies and MMAs, frees its TMEM and returns.
 #include <algorithm>
@@ -57,7 +57,7 @@ using namespace sm100;
 
 constexpr int kRows = 128;                        // query rows per tile (M)
 constexpr int kKeys = 64;                         // keys per S tile / K-V stage
-constexpr int kStages = 4;                        // K/V ring depth per lane
+constexpr int kStages = 3;                        // K/V ring depth per lane
 constexpr int kLanes = 2;
 constexpr int kQBytes = kRows * kDHead * 2;       // 16 KB of 16-bit elements
 constexpr int kKvBytes = kKeys * kDHead * 2;      // 8 KB
