@@ -1,0 +1,82 @@
+"""Pins of the projection oracle (oracle/projection.py) to closed forms:
+identity and scaled-identity weights, one-hot tokens, bias only, and the
+global-row gather.  Each pin fails for a transposed weight, a wrong head
+split, a wrong block order or a Qg row written at the wrong position."""
+import numpy as np
+
+from oracle.projection import PROJECTIONS, projection_forward
+
+H, D = 3, 64
+HID = H * D
+
+
+def _gidx(B, n, lists):
+    gidx = -np.ones((B, n), dtype=np.int32)
+    counts = np.zeros(B, dtype=np.int32)
+    for b, pos in enumerate(lists):
+        gidx[b, :len(pos)] = sorted(pos)
+        counts[b] = len(pos)
+    return gidx, counts
+
+
+def test_scaled_identity_blocks_give_the_input_split_into_heads():
+    rng = np.random.default_rng(1)
+    B, n = 2, 5
+    x = rng.standard_normal((B, n, HID))
+    scales = [1.0, 2.0, -1.0, 0.0, 0.5]
+    w = np.concatenate([s * np.eye(HID) for s in scales])
+    gidx, counts = _gidx(B, n, [[], []])
+    out = projection_forward(x, w, None, np.eye(HID), None, gidx, counts, H=H)
+    for s, name in zip(scales, PROJECTIONS):
+        for b in range(B):
+            for h in range(H):
+                for i in range(n):
+                    np.testing.assert_array_equal(out[name][b, h, i], s * x[b, i, h * D:(h + 1) * D])
+
+
+def test_one_hot_token_picks_a_weight_column():
+    rng = np.random.default_rng(2)
+    B, n = 1, 4
+    w = rng.standard_normal((5 * HID, HID))
+    bias = rng.standard_normal(5 * HID)
+    x = np.zeros((B, n, HID))
+    x[0, 2, 7] = 1.0                          # token 2 is the unit vector e_7
+    gidx, counts = _gidx(B, n, [[]])
+    out = projection_forward(x, w, bias, np.eye(HID), None, gidx, counts, H=H)
+    for p, name in enumerate(PROJECTIONS):
+        col = w[p * HID:(p + 1) * HID, 7] + bias[p * HID:(p + 1) * HID]
+        got = out[name][0, :, 2, :].reshape(HID)          # heads in order
+        np.testing.assert_allclose(got, col, rtol=0, atol=1e-12)
+        other = out[name][0, :, 1, :].reshape(HID)        # a zero token gives the bias
+        np.testing.assert_allclose(other, bias[p * HID:(p + 1) * HID], rtol=0, atol=0)
+
+
+def test_qg_only_at_global_rows_and_equal_to_q_with_the_same_weights():
+    rng = np.random.default_rng(3)
+    B, n = 2, 9
+    x = rng.standard_normal((B, n, HID))
+    w = rng.standard_normal((5 * HID, HID)) / np.sqrt(HID)
+    bias = rng.standard_normal(5 * HID)
+    gidx, counts = _gidx(B, n, [[0, 4, 8], [6]])
+    sentinel = np.full((B, H, n, D), 7.0)
+    out = projection_forward(x, w, bias, w[:HID], bias[:HID], gidx, counts, H=H,
+                             qg_init=sentinel)
+    for b, pos in enumerate([[0, 4, 8], [6]]):
+        for i in range(n):
+            if i in pos:
+                np.testing.assert_allclose(out["qg"][b, :, i], out["q"][b, :, i], atol=1e-12)
+            else:
+                np.testing.assert_array_equal(out["qg"][b, :, i], sentinel[b, :, i])
+
+
+def test_linearity_in_the_input():
+    rng = np.random.default_rng(4)
+    B, n = 1, 6
+    w = rng.standard_normal((5 * HID, HID))
+    x1, x2 = rng.standard_normal((2, B, n, HID))
+    gidx, counts = _gidx(B, n, [[1]])
+    o1 = projection_forward(x1, w, None, w[:HID], None, gidx, counts, H=H)
+    o2 = projection_forward(x2, w, None, w[:HID], None, gidx, counts, H=H)
+    o12 = projection_forward(2 * x1 - x2, w, None, w[:HID], None, gidx, counts, H=H)
+    for name in PROJECTIONS + ("qg",):
+        np.testing.assert_allclose(o12[name], 2 * o1[name] - o2[name], atol=1e-9)
