@@ -193,6 +193,41 @@ LF_API int lf_attention_forward_host(lf_dtype dtype, int B, int H, int n, int d_
  */
 LF_API int lf_workspace_status(const void *workspace, lf_stream_t stream);
 
+/*
+ * Projection prologue (FasterTransformer Longformer Encoder guide, "compute
+ * flow": the Q, K, V, Kg, Vg products over every token, the Qg product over
+ * the global tokens only, then bias add and the split into heads).  Produces
+ * the six inputs of lf_attention_run / lf_attention_forward.
+ *
+ *   dtype        LF_BF16 or LF_F16 (fp32 accumulation, outputs rounded to the
+ *                input type); LF_F32 is LF_ERR_UNSUPPORTED.
+ *   x            device [B, n, H*d_head]: hidden states.
+ *   w            device [5*H*d_head, H*d_head]: the Q, K, V, Kg, Vg weight
+ *                matrices stacked in that order, each [out, in] (row o holds
+ *                the weights of output feature o = h*d_head + e).
+ *   bias         device [5*H*d_head] in the same order, or NULL (no bias).
+ *   wqg, bqg     device [H*d_head, H*d_head] and [H*d_head] (bqg may be
+ *                NULL): the global-query projection.  wqg = NULL or
+ *                max_global = 0 skips Qg.
+ *   global_idx,  device int32 [B, n] and [B] as written by lf_global_index:
+ *   counts       the rows that get Qg (at most max_global per batch).
+ *   q, k, v,     device [B, H, n, d_head] outputs: out[b, h, i, e] =
+ *   kg, vg       sum_c x[b, i, c] * w[o, c] + bias[o], o = h*d_head + e of
+ *                the projection's block.
+ *   qg           device [B, H, n, d_head]: written at global positions only;
+ *                other rows keep their contents.
+ *   status       optional device int32: receives LF_ERR_DEVICE_TIMEOUT if a
+ *                bounded device-side wait ran out (left untouched otherwise).
+ * Every pointer must be 16-byte aligned.  d_head must be 64.  Outputs must
+ * not alias the inputs.
+ */
+LF_API int lf_qkv_projection(lf_dtype dtype, int B, int n, int H, int d_head,
+                      const void *x, const void *w, const void *bias,
+                      const void *wqg, const void *bqg,
+                      const int32_t *global_idx, const int32_t *counts, int max_global,
+                      void *q, void *k, void *v, void *qg, void *kg, void *vg,
+                      int32_t *status, lf_stream_t stream);
+
 /* Size of the fixed scratch of lf_attention_forward_static: 16 MiB. */
 #define LF_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 

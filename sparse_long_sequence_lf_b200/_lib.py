@@ -63,6 +63,7 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         "lf_workspace_status": (I, [P, P]),
         "lf_attention_forward_static": (I, [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P, I, P,
                                             P, ctypes.POINTER(P)]),
+        "lf_qkv_projection": (I, [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

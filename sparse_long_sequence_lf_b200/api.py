@@ -201,3 +201,38 @@ def scratch_status(scratch: int, stream=None) -> int:
     """Synchronises the stream and returns the status word of the last
     ``attention_forward_static`` call that used ``scratch``."""
     return int(_lib.lib().lf_workspace_status(ctypes.c_void_p(scratch), _stream_ptr(stream)))
+
+
+def qkv_projection(x, w, bias=None, wqg=None, bqg=None, global_idx=None, counts=None, *,
+                   H: int, max_global: int = 0, out=None, status=None, stream=None):
+    """``lf_qkv_projection``: Q, K, V, Kg, Vg of every token and Qg of the
+    global tokens, each [B, H, n, 64] in x's dtype.
+
+    x [B, n, H*64]; w [5*H*64, H*64] (Q, K, V, Kg, Vg stacked, rows = output
+    features); bias [5*H*64] or None; wqg [H*64, H*64] and bqg [H*64] for Qg
+    (skipped when wqg is None or max_global is 0); global_idx [B, n] and
+    counts [B] int32 as from ``global_index``.  ``out`` may hold preallocated
+    tensors under the keys q, k, v, qg, kg, vg.  Qg rows at non-global
+    positions are left as they are (zeros when this call allocates qg).
+    """
+    if x.dtype not in (torch.bfloat16, torch.float16) or x.dim() != 3:
+        raise ValueError("x must be a [B, n, H*64] bf16 or fp16 CUDA tensor")
+    B, n, hid = x.shape
+    if hid != H * D_HEAD:
+        raise ValueError("x's last dimension must be H * 64")
+    for t in (x, w, bias, wqg, bqg):
+        if t is not None and (not t.is_cuda or not t.is_contiguous() or t.dtype != x.dtype):
+            raise ValueError("x, w, bias, wqg, bqg must be contiguous CUDA tensors of one dtype")
+    outs = dict(out or {})
+    for name in ("q", "k", "v", "kg", "vg"):
+        if name not in outs:
+            outs[name] = torch.empty((B, H, n, D_HEAD), dtype=x.dtype, device=x.device)
+    if "qg" not in outs:
+        outs["qg"] = torch.zeros((B, H, n, D_HEAD), dtype=x.dtype, device=x.device)
+    _check_projections([outs[k] for k in ("q", "k", "v", "qg", "kg", "vg")])
+    _lib.check(_lib.lib().lf_qkv_projection(
+        _DTYPES[x.dtype], B, n, H, D_HEAD, _ptr(x), _ptr(w), _ptr(bias), _ptr(wqg), _ptr(bqg),
+        _ptr(global_idx), _ptr(counts), int(max_global), _ptr(outs["q"]), _ptr(outs["k"]),
+        _ptr(outs["v"]), _ptr(outs["qg"]), _ptr(outs["kg"]), _ptr(outs["vg"]), _ptr(status),
+        _stream_ptr(stream)), "lf_qkv_projection")
+    return outs

@@ -13,6 +13,10 @@ int launch_prepare(const uint8_t *local_mask, const uint8_t *global_mask, int B,
                    cudaStream_t stream);
 template <typename T> int launch_simt(const AttnArgs &a, cudaStream_t stream);
 int launch_tc(lf_dtype dtype, const AttnArgs &a, cudaStream_t stream);
+int launch_projection(lf_dtype dtype, int B, int n, int H, const void *x, const void *w,
+                      const void *bias, const void *wqg, const void *bqg, const int32_t *gidx,
+                      const int32_t *counts, int max_global, void *const out[6], int32_t *status,
+                      cudaStream_t stream);
 }  // namespace lf
 
 using namespace lf;
@@ -248,6 +252,31 @@ int lf_workspace_status(const void *workspace, lf_stream_t stream)
     if (cudaMemcpy(&status, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
         return LF_ERR_CUDA;
     return status;
+}
+
+int lf_qkv_projection(lf_dtype dtype, int B, int n, int H, int d_head, const void *x,
+                      const void *w, const void *bias, const void *wqg, const void *bqg,
+                      const int32_t *global_idx, const int32_t *counts, int max_global, void *q,
+                      void *k, void *v, void *qg, void *kg, void *vg, int32_t *status,
+                      lf_stream_t stream)
+{
+    if (d_head != kDHead) return LF_ERR_UNSUPPORTED;
+    if (dtype != LF_BF16 && dtype != LF_F16) return elem_size(dtype) ? LF_ERR_UNSUPPORTED
+                                                                   : LF_ERR_INVALID_ARG;
+    if (!sizes_ok(B, H, n) || max_global < 0 || max_global > n) return LF_ERR_INVALID_ARG;
+    if (!x || !w || !q || !k || !v || !kg || !vg) return LF_ERR_INVALID_ARG;
+    const bool with_qg = wqg != nullptr && max_global > 0;
+    if (with_qg && (!qg || !global_idx || !counts)) return LF_ERR_INVALID_ARG;
+    for (const void *ptr : {x, w, bias, wqg, bqg, static_cast<const void *>(q),
+                            static_cast<const void *>(k), static_cast<const void *>(v),
+                            static_cast<const void *>(qg), static_cast<const void *>(kg),
+                            static_cast<const void *>(vg)})
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return LF_ERR_INVALID_ARG;
+    if (int rc = device_ok()) return rc;
+    void *const out[6] = {q, k, v, kg, vg, qg};
+    return launch_projection(dtype, B, n, H, x, w, bias, with_qg ? wqg : nullptr, bqg, global_idx,
+                             counts, with_qg ? max_global : 0, out, status,
+                             static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -1,0 +1,355 @@
+// Projection prologue of the attention: Q, K, V, Kg, Vg of every token and
+// Qg of the global tokens, as tcgen05 GEMMs with a bias-and-split-heads
+// epilogue (FasterTransformer Longformer Encoder guide, "compute flow": five
+// products of the hidden states with the weight matrices over all tokens, a
+// batched product for the global rows only, then bias add and transpose to
+// [B, H, n, d]).
+//
+//   C[m, o] = sum_k X[m, k] W[o, k] + bias[o]
+//   m = b*n + i (token), o = p*H*d + h*d + e (projection p, head h, dim e)
+//   out_p[b, h, i, e] = C[m, o] rounded to the input type.
+// The global-query product gathers the rows X[b, global_idx[b, s]] for
+// s < counts[b] and writes Qg at those positions only.
+//
+// One CTA per 128 x 128 tile of C (non-persistent, two CTAs per SM):
+//   warps 0-3  epilogue: TMEM -> registers, + bias, round, store rows
+//   warp 4     TMA producer: 64-wide K slices of X and W through a 3-stage ring
+//              (row by row for the gathered global rows)
+//   warp 5     MMA issuer (one thread): tcgen05.mma kind::f16, 128x128x16,
+//              both operands K-major in shared memory (128-byte swizzle),
+//              fp32 accumulator in 128 TMEM columns.
+// Every mbarrier wait is bounded; on expiry the kernel records
+// LF_ERR_DEVICE_TIMEOUT in the optional status word, drains its copies and
+// MMAs, frees its TMEM and returns.
+#include <cstring>
+#include <mutex>
+#include <type_traits>
+
+#include <cudaTypedefs.h>
+
+#include "../../include/lf_attention.h"
+#include "lf_sm100.cuh"
+
+namespace lf {
+namespace proj {
+
+using namespace sm100;
+
+constexpr int kTileM = 128;
+constexpr int kTileN = 128;
+constexpr int kTileK = 64;                      // 128-byte rows of 16-bit elements
+constexpr int kStages = 3;
+constexpr int kThreads = 192;
+constexpr int kWarpProducer = 4;
+constexpr int kWarpMma = 5;
+constexpr uint32_t kTmemCols = 128;
+constexpr int kSliceBytes = kTileM * kTileK * 2;   // 16 KB per operand slice
+
+struct ProjParams {
+    CUtensorMap a_tile;      // X as {K, M} tiles of 64 x 128
+    CUtensorMap a_row;       // X as {K, B*n} single rows (gathered global rows)
+    CUtensorMap b_tile;      // W as {K, N} tiles of 64 x 128
+    const void *bias;        // [N] in the input type, or NULL
+    void *out[5];            // outputs of the column blocks of width H*d
+    const int32_t *gidx;     // gather mode: [B, n] compacted global positions
+    const int32_t *counts;   // gather mode: [B]
+    int32_t *status;         // optional device status word
+    int M, N, K, B, H, n, max_global, gather;
+};
+
+struct __align__(1024) ProjSmem {
+    uint8_t a[kStages][kSliceBytes];
+    uint8_t b[kStages][kSliceBytes];
+    float bias[kTileN];
+    uint64_t full[kStages], empty[kStages], acc_full, drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+// Bounded wait (1 s); on expiry records the timeout and raises the abort flag.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                         int32_t *status)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t spins = 1;; ++spins) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((spins & 31u) == 0u) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                if (status) atomicCAS(status, 0, kErrDeviceTimeout);
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// Waits (bounded, ignoring the abort flag) for work this CTA started.
+__device__ __forceinline__ void drain_bar(uint64_t *bar, uint32_t parity)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < kWaitLimitNs) {
+    }
+}
+
+// Token row of output row m of the tile (gather mode: -1 for a slot past the
+// batch's count), and its batch.
+__device__ __forceinline__ int token_of(const ProjParams &p, int m, int &b)
+{
+    if (!p.gather) {
+        b = m / p.n;
+        return m < p.M ? m - b * p.n : -1;
+    }
+    b = m / p.max_global;
+    const int s = m - b * p.max_global;
+    if (b >= p.B || s >= min(p.counts[b], p.max_global)) return -1;
+    return p.gidx[size_t(b) * p.n + s];
+}
+
+template <typename T> __device__ __forceinline__ uint32_t pack2(float lo, float hi);
+template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+template <> __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi)
+{
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ ProjParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    ProjSmem &sm = *reinterpret_cast<ProjSmem *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.y * kTileM, n0 = blockIdx.x * kTileN;
+    const int ktiles = p.K / kTileK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.acc_full, 1);
+        mbar_init(&sm.drain, 1);
+        sm.abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (threadIdx.x < kTileN) {
+        const int o = n0 + threadIdx.x;
+        float bv = 0.f;
+        if (p.bias && o < p.N) bv = to_f32(static_cast<const T *>(p.bias)[o]);
+        sm.bias[threadIdx.x] = bv;
+    }
+    if (warp == kWarpProducer && lane == 0) {
+        tma_prefetch_map(p.gather ? &p.a_row : &p.a_tile);
+        tma_prefetch_map(&p.b_tile);
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    volatile int *abort_flag = &sm.abort_flag;
+
+    if (warp == kWarpProducer) {
+        int issued = 0;
+        bool ok = true;
+        for (int kt = 0; kt < ktiles && ok; ++kt) {
+            const int s = kt % kStages;
+            const uint32_t ph = uint32_t(kt / kStages) & 1u;
+            bool w = true;
+            if (lane == 0) w = wait_bar(&sm.empty[s], ph ^ 1u, abort_flag, p.status);
+            ok = __shfl_sync(0xffffffffu, w, 0);
+            if (!ok) break;
+            if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], 2 * kSliceBytes);
+            __syncwarp();
+            if (!p.gather) {
+                if (lane == 0) tma_load_2d(sm.a[s], &p.a_tile, &sm.full[s], kt * kTileK, m0);
+            } else {
+                for (int r = lane; r < kTileM; r += 32) {
+                    int b;
+                    const int i = token_of(p, m0 + r, b);
+                    const int y = i >= 0 ? b * p.n + i : p.B * p.n;   // past the end: zeros
+                    tma_load_2d(sm.a[s] + r * (kTileK * 2), &p.a_row, &sm.full[s], kt * kTileK, y);
+                }
+            }
+            if (lane == 0) tma_load_2d(sm.b[s], &p.b_tile, &sm.full[s], kt * kTileK, n0);
+            __syncwarp();
+            issued = kt + 1;
+        }
+        if (*abort_flag && lane == 0) {
+            // Copies still in flight land before the CTA exits.
+            for (int kt = max(0, issued - kStages); kt < issued; ++kt)
+                drain_bar(&sm.full[kt % kStages], uint32_t(kt / kStages) & 1u);
+        }
+        __syncwarp();
+    } else if (warp == kWarpMma) {
+        if (lane == 0) {
+            constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+            const uint32_t idesc = make_idesc(kTileM, kTileN, kBf16, false);
+            bool ok = true;
+            for (int kt = 0; kt < ktiles && ok; ++kt) {
+                const int s = kt % kStages;
+                ok = wait_bar(&sm.full[s], uint32_t(kt / kStages) & 1u, abort_flag, p.status);
+                if (!ok) break;
+                tc_fence_after();
+                const uint64_t ad = make_sdesc(smem_u32(sm.a[s]), 16, 1024);
+                const uint64_t bd = make_sdesc(smem_u32(sm.b[s]), 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < kTileK / 16; ++kk)
+                    mma_ss(tmem, ad + uint64_t((kk * 32) >> 4), bd + uint64_t((kk * 32) >> 4), idesc,
+                           (kt > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&sm.empty[s]);
+            }
+            if (ok) tc_commit(&sm.acc_full);
+            // Every MMA issued here has completed once this commit lands.
+            tc_commit(&sm.drain);
+            drain_bar(&sm.drain, 0);
+        }
+        __syncwarp();
+    } else {
+        // Epilogue: thread t owns output row m0 + t (TMEM lane t).
+        bool ok = true;
+        if (lane == 0) ok = wait_bar(&sm.acc_full, 0, abort_flag, p.status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (ok) {
+            tc_fence_after();
+            int b;
+            const int i = token_of(p, m0 + threadIdx.x, b);
+            const int hid = p.H * kDHead;
+            const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
+#pragma unroll
+            for (int c = 0; c < kTileN / 32; ++c) {
+                float acc[32];
+                tmem_ld32(taddr + 32 * c, acc);
+                const int o = n0 + 32 * c;                 // 32 columns within one head
+                if (i < 0 || o >= p.N) continue;
+                const int blk = o / hid, rem = o - blk * hid;
+                const int h = rem / kDHead, e0 = rem - h * kDHead;
+                T *dst = static_cast<T *>(p.out[blk]) +
+                         ((size_t(b) * p.H + h) * p.n + i) * kDHead + e0;
+                uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float *v = acc + 8 * q;
+                    const float *bv = sm.bias + 32 * c + 8 * q;
+                    uint4 u;
+                    u.x = pack2<T>(v[0] + bv[0], v[1] + bv[1]);
+                    u.y = pack2<T>(v[2] + bv[2], v[3] + bv[3]);
+                    u.z = pack2<T>(v[4] + bv[4], v[5] + bv[5]);
+                    u.w = pack2<T>(v[6] + bv[6], v[7] + bv[7]);
+                    d4[q] = u;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ host
+PFN_cuTensorMapEncodeTiled_v12000 encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// A row-major [rows, K] matrix of 16-bit elements as boxes of 64 x box_rows.
+bool encode_matrix(CUtensorMap *m, const void *base, CUtensorMapDataType dt, long rows, int K,
+                   int box_rows)
+{
+    auto enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(K) * 2};
+    cuuint32_t box[2] = {kTileK, cuuint32_t(box_rows)};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+template <typename T>
+int launch(const ProjParams &p, cudaStream_t stream)
+{
+    const size_t smem = sizeof(ProjSmem) + 1024;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(proj_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem)) != cudaSuccess)
+            return kErrCuda;
+        attr_set[dev] = true;
+    }
+    dim3 grid((p.N + kTileN - 1) / kTileN, (p.M + kTileM - 1) / kTileM);
+    proj_kernel<T><<<grid, kThreads, smem, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+}
+
+}  // namespace proj
+
+int launch_projection(lf_dtype dtype, int B, int n, int H, const void *x, const void *w,
+                      const void *bias, const void *wqg, const void *bqg, const int32_t *gidx,
+                      const int32_t *counts, int max_global, void *const out[6], int32_t *status,
+                      cudaStream_t stream)
+{
+    using namespace proj;
+    const CUtensorMapDataType dt =
+        dtype == LF_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const int hid = H * kDHead;
+    ProjParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.K = hid;
+    p.B = B;
+    p.H = H;
+    p.n = n;
+    p.status = status;
+    // Q, K, V, Kg, Vg over every token.
+    p.M = B * n;
+    p.N = 5 * hid;
+    p.bias = bias;
+    for (int j = 0; j < 5; ++j) p.out[j] = out[j];
+    if (!encode_matrix(&p.a_tile, x, dt, long(B) * n, hid, kTileM)) return kErrCuda;
+    if (!encode_matrix(&p.b_tile, w, dt, 5L * hid, hid, kTileN)) return kErrCuda;
+    int rc = dtype == LF_BF16 ? launch<__nv_bfloat16>(p, stream) : launch<__half>(p, stream);
+    if (rc != kOk || max_global == 0 || wqg == nullptr) return rc;
+    // Qg over the gathered global rows.
+    ProjParams g = p;
+    g.gather = 1;
+    g.max_global = max_global;
+    g.gidx = gidx;
+    g.counts = counts;
+    g.M = B * max_global;
+    g.N = hid;
+    g.bias = bqg;
+    for (int j = 0; j < 5; ++j) g.out[j] = out[5];
+    if (!encode_matrix(&g.a_row, x, dt, long(B) * n, hid, 1)) return kErrCuda;
+    if (!encode_matrix(&g.b_tile, wqg, dt, hid, hid, kTileN)) return kErrCuda;
+    return dtype == LF_BF16 ? launch<__nv_bfloat16>(g, stream) : launch<__half>(g, stream);
+}
+
+}  // namespace lf

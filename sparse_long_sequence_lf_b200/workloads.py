@@ -165,3 +165,24 @@ def random_workload(rng: np.random.Generator, *, dtype: str = "bf16", max_n: int
     pad = tuple(int(rng.integers(0, n // 2 + 1)) if rng.random() < 0.5 else 0 for _ in range(B))
     return Workload(name, dtype, B, H, n, window, dilation=dil, causal=causal,
                     globals_kind=gk, pad_tail=pad, seed=int(rng.integers(0, 2**31 - 1)))
+
+
+def make_layer_inputs(wl: Workload, seed: int | None = None) -> dict:
+    """Inputs of the projection prologue for the workload's shape: hidden
+    states x [B, n, H*d] ~ N(0, 1); stacked weights w [5*H*d, H*d] and the
+    global-query weights wqg [H*d, H*d] ~ N(0, 1/(H*d)) (unit-scale outputs);
+    biases ~ N(0, 0.1^2); plus the workload's masks.  CPU tensors of the
+    workload dtype, drawn in that order from one seeded generator."""
+    gen = torch.Generator("cpu")
+    gen.manual_seed((wl.seed if seed is None else seed) + 500009)
+    hid = wl.H * wl.d
+    scale = 1.0 / np.sqrt(hid)
+    x = torch.randn((wl.B, wl.n, hid), generator=gen)
+    w = torch.randn((5 * hid, hid), generator=gen) * scale
+    bias = torch.randn((5 * hid,), generator=gen) * 0.1
+    wqg = torch.randn((hid, hid), generator=gen) * scale
+    bqg = torch.randn((hid,), generator=gen) * 0.1
+    local, glob = make_masks(wl)
+    dt = wl.torch_dtype
+    return dict(x=x.to(dt), w=w.to(dt), bias=bias.to(dt), wqg=wqg.to(dt), bqg=bqg.to(dt),
+                local_mask=local, global_mask=glob)
