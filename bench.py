@@ -416,6 +416,188 @@ def run_e2e(args, wl, device, stream, max_global):
             "path": "lf_attention_forward_host (pinned host buffers)"}
 
 
+# ------------------------------------------------------ projection prologue
+PROJ_METRIC = "projection prologue TFLOP/s (Q,K,V,Kg,Vg over all tokens, Qg over global tokens), 1 B200"
+
+
+def projection_flops(wl, counts, max_global):
+    hid = wl.H * wl.d
+    g = sum(min(int(c), max_global) for c in counts)
+    return 2.0 * wl.B * wl.n * hid * 5 * hid + 2.0 * g * hid * hid
+
+
+def run_projection_arm(args, wl, world, rank, local):
+    """One step = lf_qkv_projection on one batch of hidden states (the global
+    index is computed once beforehand, as it is once per batch before the
+    layer loop).  Tensor-bound: roofline against the measured dense peak."""
+    import torch
+    import sparse_long_sequence_lf_b200 as lf
+    from sparse_long_sequence_lf_b200.workloads import make_layer_inputs
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist(world, "nccl")
+    stream = torch.cuda.Stream(device)
+    x0 = make_layer_inputs(wl)
+    hid = wl.H * wl.d
+    gm = x0["global_mask"]
+    gm = (gm if gm is not None else torch.zeros((wl.B, wl.n), dtype=torch.uint8)).to(device)
+    with torch.cuda.stream(stream):
+        gidx, counts = lf.global_index(gm, stream=stream)
+    stream.synchronize()
+    max_global = int(counts.max().item())
+    per_set = sum(t.numel() * t.element_size() for k, t in x0.items()
+                  if torch.is_tensor(t) and k in ("x", "w", "bias", "wqg", "bqg"))
+    per_set += 6 * wl.B * wl.H * wl.n * wl.d * x0["x"].element_size()
+    nsets = max(2, -(-2 * L2_BYTES // per_set))
+    sets = []
+    for s_ in range(nsets):
+        xs = make_layer_inputs(wl, seed=wl.seed + 7919 * s_) if s_ else x0
+        d = {k: xs[k].to(device) for k in ("x", "w", "bias", "wqg", "bqg")}
+        d["out"] = {k: torch.empty((wl.B, wl.H, wl.n, wl.d), dtype=xs["x"].dtype, device=device)
+                    for k in ("q", "k", "v", "qg", "kg", "vg")}
+        sets.append(d)
+
+    def step(i):
+        d = sets[i % nsets]
+        lf.qkv_projection(d["x"], d["w"], d["bias"], d["wqg"], d["bqg"], gidx, counts, H=wl.H,
+                          max_global=max_global, out=d["out"], stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    stream.synchronize()
+    chunk = nsets * max(1, 32 // nsets)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(chunk):
+            step(i)
+    reps = max(1, -(-args.steps // chunk))
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        t_pad = time.time()
+        while time.time() - t_pad < 0.5:
+            with torch.cuda.stream(stream):
+                g.replay()
+            stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+        start.record(stream)
+        for _ in range(reps):
+            with torch.cuda.stream(stream):
+                g.replay()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+        if world > 1:
+            dist.barrier()
+    steps = reps * chunk
+    max_ms = reduce_max(start.elapsed_time(end), device)
+    clocks = sampler.summary("timed region plus 0.5 s of the same graph before it")
+    flops = projection_flops(wl, counts.cpu().tolist(), max_global)
+    ms_per_step = max_ms / steps
+    value = whole_job_rate(flops, steps, world, max_ms) / 1e12
+    peaks, peak_kind = load_peaks()
+    kernel_tflops = flops / (ms_per_step * 1e-3) / 1e12
+    roofline = {"kernel": "proj_kernel", "bound": "tensor", "achieved": round(kernel_tflops, 1),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(kernel_tflops / peaks["bf16_tflops"], 4), "traffic": None,
+                "peak_source": peak_kind + " (bf16 dense; fp16 has the same nominal rate)"}
+
+    # End to end: hidden states from pinned host memory in, six outputs back.
+    pin_x = x0["x"].pin_memory()
+    dev = sets[0]
+    host_out = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in dev["out"].items()}
+    xd = torch.empty_like(dev["x"])
+
+    def e2e_once():
+        with torch.cuda.stream(stream):
+            xd.copy_(pin_x, non_blocking=True)
+            lf.qkv_projection(xd, dev["w"], dev["bias"], dev["wqg"], dev["bqg"], gidx, counts,
+                              H=wl.H, max_global=max_global, out=dev["out"], stream=stream)
+            for k in host_out:
+                host_out[k].copy_(dev["out"][k], non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(3):
+        e2e_once()
+    e_steps = max(3, min(args.steps, args.e2e_steps))
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    es.record(stream)
+    for _ in range(e_steps):
+        e2e_once()
+    ee.record(stream)
+    torch.cuda.synchronize(device)
+    e_ms = reduce_max(es.elapsed_time(ee) / e_steps, device)
+    e2e = {"value": round(whole_job_rate(flops, 1, world, e_ms) / 1e12, 4), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(pin_x.numel() * pin_x.element_size()),
+           "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in host_out.values())),
+           "ms_per_step": round(e_ms, 4), "steps": e_steps,
+           "path": "lf_qkv_projection with pinned host copies of x and the six outputs"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = run_projection_cpu_baseline(wl, counts.cpu().numpy(), gidx.cpu().numpy(),
+                                          max_global, args.cpu_seconds)
+    result = {
+        "metric": PROJ_METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "op": "projection", "B": wl.B, "H": wl.H, "n": wl.n,
+                   "hidden": hid, "global_rows": int(sum(min(int(c), max_global)
+                                                         for c in counts.cpu().tolist())),
+                   "global_batch": wl.B * world, "seq_len": wl.n,
+                   "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"{nsets} rotating input sets, {nsets * per_set / 2**20:.0f} MiB > 2x L2",
+                   "launch": "CUDA graph of C-ABI calls",
+                   "useful_gflop_per_step": round(flops / 1e9, 4)},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": (2 if max_global > 0 else 1) * steps, "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        del g
+        dist.destroy_process_group()
+
+
+def run_projection_cpu_baseline(wl, counts, gidx, max_global, budget_s):
+    """The fp64 projection oracle on the first tokens of batch 0 (a bounded
+    sample), scaled to the metric's unit."""
+    import numpy as np
+    from oracle.projection import projection_forward
+    from sparse_long_sequence_lf_b200.workloads import make_layer_inputs
+    x = make_layer_inputs(wl)
+    f = lambda t: t.double().numpy()
+    X, W, Bi, Wg, Bg = f(x["x"]), f(x["w"]), f(x["bias"]), f(x["wqg"]), f(x["bqg"])
+    hid = wl.H * wl.d
+    rows = min(wl.n, 256)
+    g0 = -np.ones((1, rows), dtype=np.int32)
+    sel = [int(p) for p in gidx[0, :min(int(counts[0]), max_global)] if p < rows]
+    g0[0, :len(sel)] = sel
+    c0 = np.array([len(sel)], dtype=np.int32)
+    flops = 2.0 * rows * hid * 5 * hid + 2.0 * len(sel) * hid * hid
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        projection_forward(X[:1, :rows], W, Bi, Wg, Bg, g0, c0, H=wl.H)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt > budget_s or reps >= 1000:
+            break
+    import os
+    return {"value": round(flops * reps / dt / 1e12, 6), "unit": "TFLOP/s",
+            "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"first {rows} tokens of batch 0, {reps} repetition(s), {dt:.1f} s, "
+                      "fp64 numpy oracle (BLAS threads)",
+            "seconds": round(dt, 2)}
+
+
 # ------------------------------------------------------------- CPU oracle
 def oracle_sample_plan(wl, budget_s):
     """Head count and repetitions of the oracle sample for a time budget."""
@@ -499,6 +681,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=["attention", "projection"], default="attention",
+                    help="attention: the hot path (default); projection: the Q/K/V/Kg/Vg/Qg "
+                         "prologue on the workload's shape")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -509,6 +694,11 @@ def main(argv=None):
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference_arm(args, wl, world, rank)
+        return
+    if args.op == "projection":
+        if wl.dtype == "f32":
+            ap.error("the projection prologue runs on bf16 / fp16 workloads")
+        run_projection_arm(args, wl, world, rank, local)
         return
     run_gpu_arm(args, wl, world, rank, local)
 

@@ -45,16 +45,23 @@ constexpr int kWarpMma = 5;
 constexpr uint32_t kTmemCols = 128;
 constexpr int kSliceBytes = kTileM * kTileK * 2;   // 16 KB per operand slice
 
-struct ProjParams {
-    CUtensorMap a_tile;      // X as {K, M} tiles of 64 x 128
-    CUtensorMap a_row;       // X as {K, B*n} single rows (gathered global rows)
+// One product C = A W^T + bias.
+struct ProjJob {
+    CUtensorMap a_map;       // X as {K, M} tiles of 64 x 128, or {K, B*n} single rows
     CUtensorMap b_tile;      // W as {K, N} tiles of 64 x 128
     const void *bias;        // [N] in the input type, or NULL
     void *out[5];            // outputs of the column blocks of width H*d
-    const int32_t *gidx;     // gather mode: [B, n] compacted global positions
-    const int32_t *counts;   // gather mode: [B]
+    int M, N, gather;        // gather: A rows are the global tokens' rows of X
+};
+
+// Both products in one launch: grid rows [0, mtiles0) take job 0 (Q, K, V,
+// Kg, Vg), the rest job 1 (Qg over the gathered global rows).
+struct ProjParams {
+    ProjJob job[2];
+    const int32_t *gidx;     // [B, n] compacted global positions
+    const int32_t *counts;   // [B]
     int32_t *status;         // optional device status word
-    int M, N, K, B, H, n, max_global, gather;
+    int K, B, H, n, max_global, mtiles0;
 };
 
 struct __align__(1024) ProjSmem {
@@ -95,11 +102,11 @@ __device__ __forceinline__ void drain_bar(uint64_t *bar, uint32_t parity)
 
 // Token row of output row m of the tile (gather mode: -1 for a slot past the
 // batch's count), and its batch.
-__device__ __forceinline__ int token_of(const ProjParams &p, int m, int &b)
+__device__ __forceinline__ int token_of(const ProjParams &p, const ProjJob &J, int m, int &b)
 {
-    if (!p.gather) {
+    if (!J.gather) {
         b = m / p.n;
-        return m < p.M ? m - b * p.n : -1;
+        return m < J.M ? m - b * p.n : -1;
     }
     b = m / p.max_global;
     const int s = m - b * p.max_global;
@@ -126,7 +133,11 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
     ProjSmem &sm = *reinterpret_cast<ProjSmem *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * kTileM, n0 = blockIdx.x * kTileN;
+    const int jid = int(blockIdx.y) < p.mtiles0 ? 0 : 1;
+    const ProjJob &J = p.job[jid];
+    const int m0 = (jid == 0 ? blockIdx.y : blockIdx.y - p.mtiles0) * kTileM;
+    const int n0 = blockIdx.x * kTileN;
+    if (n0 >= J.N) return;                      // the Qg product is narrower
     const int ktiles = p.K / kTileK;
 
     if (threadIdx.x == 0) {
@@ -142,12 +153,12 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
     if (threadIdx.x < kTileN) {
         const int o = n0 + threadIdx.x;
         float bv = 0.f;
-        if (p.bias && o < p.N) bv = to_f32(static_cast<const T *>(p.bias)[o]);
+        if (J.bias && o < J.N) bv = to_f32(static_cast<const T *>(J.bias)[o]);
         sm.bias[threadIdx.x] = bv;
     }
     if (warp == kWarpProducer && lane == 0) {
-        tma_prefetch_map(p.gather ? &p.a_row : &p.a_tile);
-        tma_prefetch_map(&p.b_tile);
+        tma_prefetch_map(&J.a_map);
+        tma_prefetch_map(&J.b_tile);
     }
     if (warp == 0) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -160,6 +171,21 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
     volatile int *abort_flag = &sm.abort_flag;
 
     if (warp == kWarpProducer) {
+        // Gathered rows: only the real global tokens are loaded (the other
+        // rows of the tile feed output rows that are never stored).
+        int arow[kTileM / 32];
+        int a_bytes = kSliceBytes;
+        if (J.gather) {
+            int valid = 0;
+#pragma unroll
+            for (int q = 0; q < kTileM / 32; ++q) {
+                int b;
+                const int i = token_of(p, J, m0 + 32 * q + lane, b);
+                arow[q] = i >= 0 ? b * p.n + i : -1;
+                valid += __popc(__ballot_sync(0xffffffffu, i >= 0));
+            }
+            a_bytes = valid * (kTileK * 2);
+        }
         int issued = 0;
         bool ok = true;
         for (int kt = 0; kt < ktiles && ok; ++kt) {
@@ -169,19 +195,18 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
             if (lane == 0) w = wait_bar(&sm.empty[s], ph ^ 1u, abort_flag, p.status);
             ok = __shfl_sync(0xffffffffu, w, 0);
             if (!ok) break;
-            if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], 2 * kSliceBytes);
+            if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], a_bytes + kSliceBytes);
             __syncwarp();
-            if (!p.gather) {
-                if (lane == 0) tma_load_2d(sm.a[s], &p.a_tile, &sm.full[s], kt * kTileK, m0);
+            if (!J.gather) {
+                if (lane == 0) tma_load_2d(sm.a[s], &J.a_map, &sm.full[s], kt * kTileK, m0);
             } else {
-                for (int r = lane; r < kTileM; r += 32) {
-                    int b;
-                    const int i = token_of(p, m0 + r, b);
-                    const int y = i >= 0 ? b * p.n + i : p.B * p.n;   // past the end: zeros
-                    tma_load_2d(sm.a[s] + r * (kTileK * 2), &p.a_row, &sm.full[s], kt * kTileK, y);
-                }
+#pragma unroll
+                for (int q = 0; q < kTileM / 32; ++q)
+                    if (arow[q] >= 0)
+                        tma_load_2d(sm.a[s] + (32 * q + lane) * (kTileK * 2), &J.a_map,
+                                    &sm.full[s], kt * kTileK, arow[q]);
             }
-            if (lane == 0) tma_load_2d(sm.b[s], &p.b_tile, &sm.full[s], kt * kTileK, n0);
+            if (lane == 0) tma_load_2d(sm.b[s], &J.b_tile, &sm.full[s], kt * kTileK, n0);
             __syncwarp();
             issued = kt + 1;
         }
@@ -223,7 +248,7 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
         if (ok) {
             tc_fence_after();
             int b;
-            const int i = token_of(p, m0 + threadIdx.x, b);
+            const int i = token_of(p, J, m0 + threadIdx.x, b);
             const int hid = p.H * kDHead;
             const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
 #pragma unroll
@@ -231,10 +256,10 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
                 float acc[32];
                 tmem_ld32(taddr + 32 * c, acc);
                 const int o = n0 + 32 * c;                 // 32 columns within one head
-                if (i < 0 || o >= p.N) continue;
+                if (i < 0 || o >= J.N) continue;
                 const int blk = o / hid, rem = o - blk * hid;
                 const int h = rem / kDHead, e0 = rem - h * kDHead;
-                T *dst = static_cast<T *>(p.out[blk]) +
+                T *dst = static_cast<T *>(J.out[blk]) +
                          ((size_t(b) * p.H + h) * p.n + i) * kDHead + e0;
                 uint4 *d4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
@@ -305,7 +330,8 @@ int launch(const ProjParams &p, cudaStream_t stream)
             return kErrCuda;
         attr_set[dev] = true;
     }
-    dim3 grid((p.N + kTileN - 1) / kTileN, (p.M + kTileM - 1) / kTileM);
+    const int mtiles1 = (p.job[1].M + kTileM - 1) / kTileM;
+    dim3 grid((p.job[0].N + kTileN - 1) / kTileN, p.mtiles0 + mtiles1);
     proj_kernel<T><<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
@@ -328,28 +354,30 @@ int launch_projection(lf_dtype dtype, int B, int n, int H, const void *x, const 
     p.H = H;
     p.n = n;
     p.status = status;
-    // Q, K, V, Kg, Vg over every token.
-    p.M = B * n;
-    p.N = 5 * hid;
-    p.bias = bias;
-    for (int j = 0; j < 5; ++j) p.out[j] = out[j];
-    if (!encode_matrix(&p.a_tile, x, dt, long(B) * n, hid, kTileM)) return kErrCuda;
-    if (!encode_matrix(&p.b_tile, w, dt, 5L * hid, hid, kTileN)) return kErrCuda;
-    int rc = dtype == LF_BF16 ? launch<__nv_bfloat16>(p, stream) : launch<__half>(p, stream);
-    if (rc != kOk || max_global == 0 || wqg == nullptr) return rc;
-    // Qg over the gathered global rows.
-    ProjParams g = p;
-    g.gather = 1;
-    g.max_global = max_global;
-    g.gidx = gidx;
-    g.counts = counts;
-    g.M = B * max_global;
-    g.N = hid;
-    g.bias = bqg;
-    for (int j = 0; j < 5; ++j) g.out[j] = out[5];
-    if (!encode_matrix(&g.a_row, x, dt, long(B) * n, hid, 1)) return kErrCuda;
-    if (!encode_matrix(&g.b_tile, wqg, dt, hid, hid, kTileN)) return kErrCuda;
-    return dtype == LF_BF16 ? launch<__nv_bfloat16>(g, stream) : launch<__half>(g, stream);
+    p.gidx = gidx;
+    p.counts = counts;
+    p.max_global = max_global;
+    // Job 0: Q, K, V, Kg, Vg over every token.
+    ProjJob &J0 = p.job[0];
+    J0.M = B * n;
+    J0.N = 5 * hid;
+    J0.bias = bias;
+    for (int j = 0; j < 5; ++j) J0.out[j] = out[j];
+    if (!encode_matrix(&J0.a_map, x, dt, long(B) * n, hid, kTileM)) return kErrCuda;
+    if (!encode_matrix(&J0.b_tile, w, dt, 5L * hid, hid, kTileN)) return kErrCuda;
+    p.mtiles0 = (J0.M + kTileM - 1) / kTileM;
+    // Job 1: Qg over the gathered global rows (none when max_global is 0).
+    ProjJob &J1 = p.job[1];
+    J1.gather = 1;
+    J1.M = (max_global > 0 && wqg) ? B * max_global : 0;
+    J1.N = hid;
+    J1.bias = bqg;
+    for (int j = 0; j < 5; ++j) J1.out[j] = out[5];
+    if (J1.M > 0) {
+        if (!encode_matrix(&J1.a_map, x, dt, long(B) * n, hid, 1)) return kErrCuda;
+        if (!encode_matrix(&J1.b_tile, wqg, dt, hid, hid, kTileN)) return kErrCuda;
+    }
+    return dtype == LF_BF16 ? launch<__nv_bfloat16>(p, stream) : launch<__half>(p, stream);
 }
 
 }  // namespace lf

@@ -84,3 +84,15 @@ def test_reference_arm_other_ranks_do_no_work():
 def test_warmup_below_three_is_rejected():
     r = _run_bench(["--warmup", "2"])
     assert r.returncode != 0
+
+
+def test_projection_cpu_baseline_line_is_well_formed():
+    import numpy as np
+    import bench
+    from sparse_long_sequence_lf_b200.workloads import Workload
+    wl = Workload("proj-host", "bf16", 1, 2, 40, 8, globals_kind="list:3,17", seed=5)
+    gidx = -np.ones((1, 40), dtype=np.int32)
+    gidx[0, :2] = [3, 17]
+    cpu = bench.run_projection_cpu_baseline(wl, np.array([2]), gidx, 2, budget_s=0.05)
+    assert cpu["kind"] == "oracle" and cpu["unit"] == "TFLOP/s" and cpu["value"] > 0
+    assert bench.projection_flops(wl, [2], 2) == 2.0 * 40 * 128 * 640 + 2.0 * 2 * 128 * 128
