@@ -72,3 +72,30 @@ def projection_forward(x, w, bias, wqg, bqg, global_idx, counts, *, H: int, d: i
         qg[b][:, rows, :] = y.reshape(g, H, d).transpose(1, 0, 2)
     out["qg"] = qg
     return out
+
+
+def output_layer(attn, wo, bo, residual, gamma, beta, *, eps: float = 1e-5):
+    """fp64 output layer of the attention block (FasterTransformer Longformer
+    Encoder guide, "compute flow": the heads are concatenated back into one
+    [B, n, H*d] tensor, multiplied by the output weight matrix plus bias, the
+    layer input is added back and the sum layer-normalised with its own
+    scale and shift).
+
+    attn     [B, H, n, d] attention output.
+    wo, bo   [H*d, H*d] (rows = output features) and [H*d] or None.
+    residual [B, n, H*d] the layer input.
+    gamma, beta [H*d]; eps added to the variance (the population variance
+    over the H*d features of a token).
+    Returns [B, n, H*d] fp64.
+    """
+    a = np.asarray(attn, dtype=np.float64)
+    B, H, n, d = a.shape
+    merged = a.transpose(0, 2, 1, 3).reshape(B, n, H * d)
+    y = np.einsum("bni,oi->bno", merged, np.asarray(wo, dtype=np.float64))
+    if bo is not None:
+        y = y + np.asarray(bo, dtype=np.float64)
+    y = y + np.asarray(residual, dtype=np.float64)
+    mean = y.mean(axis=-1, keepdims=True)
+    var = ((y - mean) ** 2).mean(axis=-1, keepdims=True)
+    z = (y - mean) / np.sqrt(var + eps)
+    return z * np.asarray(gamma, dtype=np.float64) + np.asarray(beta, dtype=np.float64)

@@ -80,3 +80,48 @@ def test_linearity_in_the_input():
     o12 = projection_forward(2 * x1 - x2, w, None, w[:HID], None, gidx, counts, H=H)
     for name in PROJECTIONS + ("qg",):
         np.testing.assert_allclose(o12[name], 2 * o1[name] - o2[name], atol=1e-9)
+
+
+# ------------------------------------------------------------ output layer
+from oracle.projection import output_layer  # noqa: E402
+
+
+def test_output_layer_alternating_row_normalises_to_plus_minus_one():
+    B, n = 1, 2
+    attn = np.zeros((B, H, n, D))
+    row = np.array([1.0, -1.0] * (HID // 2))            # mean 0, population variance 1
+    attn[0, :, 1, :] = row.reshape(H, D)
+    z = output_layer(attn, np.eye(HID), None, np.zeros((B, n, HID)), np.ones(HID),
+                     np.zeros(HID), eps=1e-5)
+    np.testing.assert_allclose(z[0, 1], row / np.sqrt(1.0 + 1e-5), rtol=0, atol=1e-12)
+
+
+def test_output_layer_concatenates_heads_in_order():
+    # A ramp over the features of a token, spread across heads: with identity
+    # weights the normalised row is the normalised ramp only if head h lands
+    # at features [h*d, (h+1)*d).
+    B, n = 1, 1
+    ramp = np.arange(HID, dtype=np.float64)
+    attn = ramp.reshape(1, H, 1, D)
+    z = output_layer(attn, np.eye(HID), None, np.zeros((B, n, HID)), np.ones(HID),
+                     np.zeros(HID), eps=0.0)
+    want = (ramp - ramp.mean()) / ramp.std()
+    np.testing.assert_allclose(z[0, 0], want, atol=1e-12)
+
+
+def test_output_layer_bias_residual_and_affine():
+    rng = np.random.default_rng(7)
+    B, n = 2, 3
+    attn = rng.standard_normal((B, H, n, D))
+    wo = rng.standard_normal((HID, HID)) / np.sqrt(HID)
+    bo = rng.standard_normal(HID)
+    res = rng.standard_normal((B, n, HID))
+    g, b = rng.standard_normal(HID), rng.standard_normal(HID)
+    z = output_layer(attn, wo, bo, res, g, b)
+    unit = output_layer(attn, wo, bo, res, np.ones(HID), np.zeros(HID))
+    np.testing.assert_allclose(z, unit * g + b, atol=1e-12)
+    # unit-scale rows: mean 0 and variance 1 / (1 + eps / var)
+    np.testing.assert_allclose(unit.mean(axis=-1), 0.0, atol=1e-12)
+    # adding a constant to every feature of the pre-norm sum changes nothing
+    z2 = output_layer(attn, wo, bo + 5.0, res, g, b)
+    np.testing.assert_allclose(z2, z, atol=1e-9)
