@@ -228,6 +228,35 @@ LF_API int lf_qkv_projection(lf_dtype dtype, int B, int n, int H, int d_head,
                       void *q, void *k, void *v, void *qg, void *kg, void *vg,
                       int32_t *status, lf_stream_t stream);
 
+/*
+ * Output layer of the attention block (FasterTransformer Longformer Encoder
+ * guide, "compute flow": the heads concatenated back into [B, n, H*d_head],
+ * the output projection plus bias, the layer input added back, then layer
+ * normalisation):
+ *   y[b, i, :] = LayerNorm(concat_h attn[b, h, i, :] . wo^T + bo + residual[b, i, :])
+ * with LayerNorm(s) = (s - mean(s)) / sqrt(var(s) + eps) * gamma + beta over
+ * the H*d_head features (population variance).
+ *
+ *   dtype        LF_BF16 or LF_F16 (fp32 accumulation and normalisation).
+ *   attn         device [B, H, n, d_head]: the attention output.
+ *   wo, bo       device [H*d_head, H*d_head] (rows = output features) and
+ *                [H*d_head] or NULL.
+ *   residual     device [B, n, H*d_head]: the layer input.
+ *   gamma, beta  device [H*d_head].
+ *   eps          >= 0, finite.
+ *   out          device [B, n, H*d_head].
+ *   workspace    device, 256-byte aligned, lf_output_workspace_size bytes:
+ *                the fp32 pre-normalisation sums.
+ *   status       optional device int32 (see lf_qkv_projection).
+ * Every pointer must be 16-byte aligned; d_head must be 64.
+ */
+LF_API size_t lf_output_workspace_size(int B, int n, int H, int d_head);
+LF_API int lf_output_layer(lf_dtype dtype, int B, int n, int H, int d_head,
+                    const void *attn, const void *wo, const void *bo, const void *residual,
+                    const void *gamma, const void *beta, float eps, void *out,
+                    void *workspace, size_t workspace_bytes, int32_t *status,
+                    lf_stream_t stream);
+
 /* Size of the fixed scratch of lf_attention_forward_static: 16 MiB. */
 #define LF_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 

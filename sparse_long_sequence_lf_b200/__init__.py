@@ -7,11 +7,11 @@ is missing.
 """
 from .api import (attention_forward, attention_forward_host, attention_forward_static,
                   attention_prepare, attention_run, global_index, host_staging_size,
-                  new_workspace, qkv_projection, scratch_status, workspace_size,
-                  workspace_status)
+                  new_workspace, output_layer, output_workspace_size, qkv_projection,
+                  scratch_status, workspace_size, workspace_status)
 from ._lib import LfError
 
 __all__ = ["attention_forward", "attention_forward_host", "attention_forward_static",
            "attention_prepare", "attention_run", "global_index", "host_staging_size",
-           "new_workspace", "qkv_projection", "scratch_status", "workspace_size",
-           "workspace_status", "LfError"]
+           "new_workspace", "output_layer", "output_workspace_size", "qkv_projection",
+           "scratch_status", "workspace_size", "workspace_status", "LfError"]

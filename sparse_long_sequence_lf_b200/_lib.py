@@ -64,6 +64,8 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         "lf_attention_forward_static": (I, [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P, I, P,
                                             P, ctypes.POINTER(P)]),
         "lf_qkv_projection": (I, [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, P, P, P, P, P]),
+        "lf_output_workspace_size": (Z, [I, I, I, I]),
+        "lf_output_layer": (I, [I, I, I, I, I, P, P, P, P, P, P, ctypes.c_float, P, P, Z, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

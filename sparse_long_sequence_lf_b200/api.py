@@ -236,3 +236,30 @@ def qkv_projection(x, w, bias=None, wqg=None, bqg=None, global_idx=None, counts=
         _ptr(outs["v"]), _ptr(outs["qg"]), _ptr(outs["kg"]), _ptr(outs["vg"]), _ptr(status),
         _stream_ptr(stream)), "lf_qkv_projection")
     return outs
+
+
+def output_workspace_size(B: int, n: int, H: int) -> int:
+    return int(_lib.lib().lf_output_workspace_size(B, n, H, D_HEAD))
+
+
+def output_layer(attn, wo, bo, residual, gamma, beta, *, eps: float = 1e-5, out=None,
+                 workspace=None, status=None, stream=None):
+    """``lf_output_layer``: LayerNorm(concat_heads(attn) . wo^T + bo + residual)
+    with gamma, beta; returns out [B, n, H*64] in attn's dtype."""
+    if attn.dtype not in (torch.bfloat16, torch.float16) or attn.dim() != 4 \
+            or attn.shape[-1] != D_HEAD:
+        raise ValueError("attn must be a [B, H, n, 64] bf16 or fp16 CUDA tensor")
+    B, H, n, _ = attn.shape
+    for t in (attn, wo, bo, residual, gamma, beta):
+        if t is not None and (not t.is_cuda or not t.is_contiguous() or t.dtype != attn.dtype):
+            raise ValueError("all inputs must be contiguous CUDA tensors of attn's dtype")
+    if out is None:
+        out = torch.empty_like(residual)
+    if workspace is None:
+        workspace = torch.empty(output_workspace_size(B, n, H), dtype=torch.uint8,
+                                device=attn.device)
+    _lib.check(_lib.lib().lf_output_layer(
+        _DTYPES[attn.dtype], B, n, H, D_HEAD, _ptr(attn), _ptr(wo), _ptr(bo), _ptr(residual),
+        _ptr(gamma), _ptr(beta), float(eps), _ptr(out), _ptr(workspace), workspace.numel(),
+        _ptr(status), _stream_ptr(stream)), "lf_output_layer")
+    return out

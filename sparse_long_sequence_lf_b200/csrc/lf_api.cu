@@ -17,6 +17,10 @@ int launch_projection(lf_dtype dtype, int B, int n, int H, const void *x, const 
                       const void *bias, const void *wqg, const void *bqg, const int32_t *gidx,
                       const int32_t *counts, int max_global, void *const out[6], int32_t *status,
                       cudaStream_t stream);
+int launch_output_layer(lf_dtype dtype, int B, int n, int H, const void *attn, const void *wo,
+                        const void *bo, const void *residual, const void *gamma,
+                        const void *beta, float eps, void *out, float *sum, int32_t *status,
+                        cudaStream_t stream);
 }  // namespace lf
 
 using namespace lf;
@@ -277,6 +281,34 @@ int lf_qkv_projection(lf_dtype dtype, int B, int n, int H, int d_head, const voi
     return launch_projection(dtype, B, n, H, x, w, bias, with_qg ? wqg : nullptr, bqg, global_idx,
                              counts, with_qg ? max_global : 0, out, status,
                              static_cast<cudaStream_t>(stream));
+}
+
+size_t lf_output_workspace_size(int B, int n, int H, int d_head)
+{
+    if (!sizes_ok(B, H, n) || d_head != kDHead) return 0;
+    return lf_align256(sizeof(float) * size_t(B) * n * H * kDHead);
+}
+
+int lf_output_layer(lf_dtype dtype, int B, int n, int H, int d_head, const void *attn,
+                    const void *wo, const void *bo, const void *residual, const void *gamma,
+                    const void *beta, float eps, void *out, void *workspace,
+                    size_t workspace_bytes, int32_t *status, lf_stream_t stream)
+{
+    if (d_head != kDHead) return LF_ERR_UNSUPPORTED;
+    if (dtype != LF_BF16 && dtype != LF_F16) return elem_size(dtype) ? LF_ERR_UNSUPPORTED
+                                                                   : LF_ERR_INVALID_ARG;
+    if (!sizes_ok(B, H, n)) return LF_ERR_INVALID_ARG;
+    if (!attn || !wo || !residual || !gamma || !beta || !out) return LF_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return LF_ERR_INVALID_ARG;
+    for (const void *ptr : {attn, wo, bo, residual, gamma, beta, static_cast<const void *>(out)})
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return LF_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+        workspace_bytes < lf_output_workspace_size(B, n, H, d_head))
+        return LF_ERR_WORKSPACE;
+    if (int rc = device_ok()) return rc;
+    return launch_output_layer(dtype, B, n, H, attn, wo, bo, residual, gamma, beta, eps, out,
+                               static_cast<float *>(workspace), status,
+                               static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

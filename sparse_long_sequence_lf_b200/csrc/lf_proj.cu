@@ -46,12 +46,18 @@ constexpr uint32_t kTmemCols = 128;
 constexpr int kSliceBytes = kTileM * kTileK * 2;   // 16 KB per operand slice
 
 // One product C = A W^T + bias.
+enum JobMode { kModeHeads = 0, kModeGather = 1, kModeResidual = 2 };
 struct ProjJob {
-    CUtensorMap a_map;       // X as {K, M} tiles of 64 x 128, or {K, B*n} single rows
+    CUtensorMap a_map;       // heads: X as {K, M} tiles of 64 x 128; gather: X as
+                             // {K, B*n} single rows; residual: the attention output
+                             // as {d, n, B*H} tiles of 64 x 128 x 1 (one head per K slice)
     CUtensorMap b_tile;      // W as {K, N} tiles of 64 x 128
     const void *bias;        // [N] in the input type, or NULL
-    void *out[5];            // outputs of the column blocks of width H*d
-    int M, N, gather;        // gather: A rows are the global tokens' rows of X
+    void *out[5];            // heads / gather: outputs of the column blocks of width H*d
+    const void *residual;    // residual: [B, n, N] in the input type
+    float *sum;              // residual: [B, n, N] fp32, C + bias + residual
+    int M, N, mode;
+    int tiles_per_batch;     // residual: M tiles of 128 tokens per batch
 };
 
 // Both products in one launch: grid rows [0, mtiles0) take job 0 (Q, K, V,
@@ -104,7 +110,13 @@ __device__ __forceinline__ void drain_bar(uint64_t *bar, uint32_t parity)
 // batch's count), and its batch.
 __device__ __forceinline__ int token_of(const ProjParams &p, const ProjJob &J, int m, int &b)
 {
-    if (!J.gather) {
+    if (J.mode == kModeResidual) {          // m = tile row: b * tiles_per_batch * 128 + i
+        const int per = J.tiles_per_batch * kTileM;
+        b = m / per;
+        const int i = m - b * per;
+        return i < p.n ? i : -1;
+    }
+    if (J.mode == kModeHeads) {
         b = m / p.n;
         return m < J.M ? m - b * p.n : -1;
     }
@@ -175,7 +187,7 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
         // rows of the tile feed output rows that are never stored).
         int arow[kTileM / 32];
         int a_bytes = kSliceBytes;
-        if (J.gather) {
+        if (J.mode == kModeGather) {
             int valid = 0;
 #pragma unroll
             for (int q = 0; q < kTileM / 32; ++q) {
@@ -197,8 +209,14 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
             if (!ok) break;
             if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], a_bytes + kSliceBytes);
             __syncwarp();
-            if (!J.gather) {
+            if (J.mode == kModeHeads) {
                 if (lane == 0) tma_load_2d(sm.a[s], &J.a_map, &sm.full[s], kt * kTileK, m0);
+            } else if (J.mode == kModeResidual) {
+                // K slice kt is head kt of the attention output: rows i0 .. i0+127
+                // of batch b (rows past n read as zeros).
+                const int b = m0 / (J.tiles_per_batch * kTileM);
+                const int i0 = m0 - b * J.tiles_per_batch * kTileM;
+                if (lane == 0) tma_load_3d(sm.a[s], &J.a_map, &sm.full[s], 0, i0, b * p.H + kt);
             } else {
 #pragma unroll
                 for (int q = 0; q < kTileM / 32; ++q)
@@ -257,6 +275,21 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
                 tmem_ld32(taddr + 32 * c, acc);
                 const int o = n0 + 32 * c;                 // 32 columns within one head
                 if (i < 0 || o >= J.N) continue;
+                if (J.mode == kModeResidual) {
+                    const size_t row = (size_t(b) * p.n + i) * J.N + o;
+                    const T *res = static_cast<const T *>(J.residual) + row;
+                    float4 *dst = reinterpret_cast<float4 *>(J.sum + row);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float4 v;
+                        v.x = acc[4 * q + 0] + sm.bias[32 * c + 4 * q + 0] + to_f32(res[4 * q + 0]);
+                        v.y = acc[4 * q + 1] + sm.bias[32 * c + 4 * q + 1] + to_f32(res[4 * q + 1]);
+                        v.z = acc[4 * q + 2] + sm.bias[32 * c + 4 * q + 2] + to_f32(res[4 * q + 2]);
+                        v.w = acc[4 * q + 3] + sm.bias[32 * c + 4 * q + 3] + to_f32(res[4 * q + 3]);
+                        dst[q] = v;
+                    }
+                    continue;
+                }
                 const int blk = o / hid, rem = o - blk * hid;
                 const int h = rem / kDHead, e0 = rem - h * kDHead;
                 T *dst = static_cast<T *>(J.out[blk]) +
@@ -282,6 +315,52 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// LayerNorm of each row of the fp32 sums: one warp per row.  Mean first, then
+// the mean square deviation (two passes over the row, which stays in L1/L2),
+// then out = (s - mean) / sqrt(var + eps) * gamma + beta in the output type.
+template <typename T>
+__global__ void __launch_bounds__(256) layernorm_kernel(const float *__restrict__ sum,
+                                                        const T *__restrict__ gamma,
+                                                        const T *__restrict__ beta, float eps,
+                                                        int rows, int N, T *__restrict__ out)
+{
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= rows) return;
+    const float4 *r4 = reinterpret_cast<const float4 *>(sum + size_t(warp) * N);
+    const int n4 = N / 4;
+    float s = 0.f;
+    for (int c = lane; c < n4; c += 32) {
+        const float4 v = r4[c];
+        s += (v.x + v.y) + (v.z + v.w);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mean = s / float(N);
+    float q = 0.f;
+    for (int c = lane; c < n4; c += 32) {
+        const float4 v = r4[c];
+        const float a = v.x - mean, b = v.y - mean, e = v.z - mean, f = v.w - mean;
+        q += (a * a + b * b) + (e * e + f * f);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    const float inv = rsqrtf(q / float(N) + eps);
+    T *dst = out + size_t(warp) * N;
+    for (int c = lane; c < n4; c += 32) {
+        const float4 v = r4[c];
+        const int o = 4 * c;
+        const float y0 = (v.x - mean) * inv * to_f32(gamma[o]) + to_f32(beta[o]);
+        const float y1 = (v.y - mean) * inv * to_f32(gamma[o + 1]) + to_f32(beta[o + 1]);
+        const float y2 = (v.z - mean) * inv * to_f32(gamma[o + 2]) + to_f32(beta[o + 2]);
+        const float y3 = (v.w - mean) * inv * to_f32(gamma[o + 3]) + to_f32(beta[o + 3]);
+        uint2 u;
+        u.x = pack2<T>(y0, y1);
+        u.y = pack2<T>(y2, y3);
+        *reinterpret_cast<uint2 *>(dst + o) = u;
     }
 }
 
@@ -312,6 +391,21 @@ bool encode_matrix(CUtensorMap *m, const void *base, CUtensorMapDataType dt, lon
     cuuint32_t box[2] = {kTileK, cuuint32_t(box_rows)};
     cuuint32_t es[2] = {1, 1};
     return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// The attention output [B, H, n, d] as {d, n, B*H} tiles of 64 x 128 x 1.
+bool encode_heads(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int B, int H, int n)
+{
+    auto enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {cuuint64_t(kDHead), cuuint64_t(n), cuuint64_t(B) * H};
+    cuuint64_t strides[2] = {cuuint64_t(kDHead) * 2, cuuint64_t(n) * kDHead * 2};
+    cuuint32_t box[3] = {kTileK, kTileM, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
@@ -368,7 +462,7 @@ int launch_projection(lf_dtype dtype, int B, int n, int H, const void *x, const 
     p.mtiles0 = (J0.M + kTileM - 1) / kTileM;
     // Job 1: Qg over the gathered global rows (none when max_global is 0).
     ProjJob &J1 = p.job[1];
-    J1.gather = 1;
+    J1.mode = kModeGather;
     J1.M = (max_global > 0 && wqg) ? B * max_global : 0;
     J1.N = hid;
     J1.bias = bqg;
@@ -378,6 +472,50 @@ int launch_projection(lf_dtype dtype, int B, int n, int H, const void *x, const 
         if (!encode_matrix(&J1.b_tile, wqg, dt, hid, hid, kTileN)) return kErrCuda;
     }
     return dtype == LF_BF16 ? launch<__nv_bfloat16>(p, stream) : launch<__half>(p, stream);
+}
+
+int launch_output_layer(lf_dtype dtype, int B, int n, int H, const void *attn, const void *wo,
+                        const void *bo, const void *residual, const void *gamma,
+                        const void *beta, float eps, void *out, float *sum, int32_t *status,
+                        cudaStream_t stream)
+{
+    using namespace proj;
+    const CUtensorMapDataType dt =
+        dtype == LF_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const int hid = H * kDHead;
+    ProjParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.K = hid;
+    p.B = B;
+    p.H = H;
+    p.n = n;
+    p.status = status;
+    ProjJob &J = p.job[0];
+    J.mode = kModeResidual;
+    J.tiles_per_batch = (n + kTileM - 1) / kTileM;
+    J.M = B * J.tiles_per_batch * kTileM;
+    J.N = hid;
+    J.bias = bo;
+    J.residual = residual;
+    J.sum = sum;
+    if (!encode_heads(&J.a_map, attn, dt, B, H, n)) return kErrCuda;
+    if (!encode_matrix(&J.b_tile, wo, dt, hid, hid, kTileN)) return kErrCuda;
+    p.mtiles0 = J.M / kTileM;
+    p.job[1].M = 0;
+    p.job[1].N = 0;
+    int rc = dtype == LF_BF16 ? launch<__nv_bfloat16>(p, stream) : launch<__half>(p, stream);
+    if (rc != kOk) return rc;
+    const int rows = B * n;
+    const int blocks = (rows + 7) / 8;
+    if (dtype == LF_BF16)
+        layernorm_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>(
+            sum, static_cast<const __nv_bfloat16 *>(gamma), static_cast<const __nv_bfloat16 *>(beta),
+            eps, rows, hid, static_cast<__nv_bfloat16 *>(out));
+    else
+        layernorm_kernel<__half><<<blocks, 256, 0, stream>>>(
+            sum, static_cast<const __half *>(gamma), static_cast<const __half *>(beta), eps, rows,
+            hid, static_cast<__half *>(out));
+    return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 
 }  // namespace lf

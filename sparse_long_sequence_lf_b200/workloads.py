@@ -186,3 +186,22 @@ def make_layer_inputs(wl: Workload, seed: int | None = None) -> dict:
     dt = wl.torch_dtype
     return dict(x=x.to(dt), w=w.to(dt), bias=bias.to(dt), wqg=wqg.to(dt), bqg=bqg.to(dt),
                 local_mask=local, global_mask=glob)
+
+
+def make_output_inputs(wl: Workload, seed: int | None = None) -> dict:
+    """Inputs of the output layer for the workload's shape: attention output
+    attn [B, H, n, d] ~ N(0, 1); wo [H*d, H*d] ~ N(0, 1/(H*d)); bo ~ N(0, 0.1^2);
+    residual [B, n, H*d] ~ N(0, 1); gamma ~ 1 + N(0, 0.1^2); beta ~ N(0, 0.1^2).
+    CPU tensors of the workload dtype, drawn in that order."""
+    gen = torch.Generator("cpu")
+    gen.manual_seed((wl.seed if seed is None else seed) + 700001)
+    hid = wl.H * wl.d
+    attn = torch.randn((wl.B, wl.H, wl.n, wl.d), generator=gen)
+    wo = torch.randn((hid, hid), generator=gen) / np.sqrt(hid)
+    bo = torch.randn((hid,), generator=gen) * 0.1
+    residual = torch.randn((wl.B, wl.n, hid), generator=gen)
+    gamma = 1.0 + torch.randn((hid,), generator=gen) * 0.1
+    beta = torch.randn((hid,), generator=gen) * 0.1
+    dt = wl.torch_dtype
+    return dict(attn=attn.to(dt), wo=wo.to(dt), bo=bo.to(dt), residual=residual.to(dt),
+                gamma=gamma.to(dt), beta=beta.to(dt))
