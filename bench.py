@@ -567,6 +567,160 @@ def run_projection_arm(args, wl, world, rank, local):
         dist.destroy_process_group()
 
 
+OUT_METRIC = "output layer TFLOP/s (heads concatenated, output projection, bias, residual, LayerNorm), 1 B200"
+
+
+def run_output_arm(args, wl, world, rank, local):
+    """One step = lf_output_layer on one batch (GEMM 2 B n (H d)^2 FLOPs on the
+    tensor cores, then a memory-bound LayerNorm).  Roofline: the step against
+    the measured dense peak."""
+    import torch
+    import sparse_long_sequence_lf_b200 as lf
+    from sparse_long_sequence_lf_b200.workloads import make_output_inputs
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist(world, "nccl")
+    stream = torch.cuda.Stream(device)
+    hid = wl.H * wl.d
+    x0 = make_output_inputs(wl)
+    per_set = sum(t.numel() * t.element_size() for t in x0.values())
+    per_set += wl.B * wl.n * hid * (x0["attn"].element_size() + 4)
+    nsets = max(2, -(-2 * L2_BYTES // per_set))
+    ws = torch.empty(lf.output_workspace_size(wl.B, wl.n, wl.H), dtype=torch.uint8,
+                     device=device)
+    sets = []
+    for s_ in range(nsets):
+        xs = make_output_inputs(wl, seed=wl.seed + 7919 * s_) if s_ else x0
+        d = {k: v.to(device) for k, v in xs.items()}
+        d["out"] = torch.empty_like(d["residual"])
+        sets.append(d)
+
+    def step(i):
+        d = sets[i % nsets]
+        lf.output_layer(d["attn"], d["wo"], d["bo"], d["residual"], d["gamma"], d["beta"],
+                        out=d["out"], workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    stream.synchronize()
+    chunk = nsets * max(1, 32 // nsets)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(chunk):
+            step(i)
+    reps = max(1, -(-args.steps // chunk))
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        t_pad = time.time()
+        while time.time() - t_pad < 0.5:
+            with torch.cuda.stream(stream):
+                g.replay()
+            stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+        start.record(stream)
+        for _ in range(reps):
+            with torch.cuda.stream(stream):
+                g.replay()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+        if world > 1:
+            dist.barrier()
+    steps = reps * chunk
+    max_ms = reduce_max(start.elapsed_time(end), device)
+    clocks = sampler.summary("timed region plus 0.5 s of the same graph before it")
+    flops = 2.0 * wl.B * wl.n * hid * hid
+    ms_per_step = max_ms / steps
+    value = whole_job_rate(flops, steps, world, max_ms) / 1e12
+    peaks, peak_kind = load_peaks()
+    tflops = flops / (ms_per_step * 1e-3) / 1e12
+    roofline = {"kernel": "proj_kernel (residual mode) + layernorm_kernel", "bound": "tensor",
+                "achieved": round(tflops, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(tflops / peaks["bf16_tflops"], 4), "traffic": None,
+                "peak_source": peak_kind + " (bf16 dense; fp16 has the same nominal rate)"}
+
+    # End to end: attention output and residual from pinned host memory in, the
+    # normalised rows back.
+    dev = sets[0]
+    pin = {k: x0[k].pin_memory() for k in ("attn", "residual")}
+    host_out = torch.empty_like(x0["residual"]).pin_memory()
+    da, dr = torch.empty_like(dev["attn"]), torch.empty_like(dev["residual"])
+
+    def e2e_once():
+        with torch.cuda.stream(stream):
+            da.copy_(pin["attn"], non_blocking=True)
+            dr.copy_(pin["residual"], non_blocking=True)
+            lf.output_layer(da, dev["wo"], dev["bo"], dr, dev["gamma"], dev["beta"],
+                            out=dev["out"], workspace=ws, stream=stream)
+            host_out.copy_(dev["out"], non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(3):
+        e2e_once()
+    e_steps = max(3, min(args.steps, args.e2e_steps))
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    es.record(stream)
+    for _ in range(e_steps):
+        e2e_once()
+    ee.record(stream)
+    torch.cuda.synchronize(device)
+    e_ms = reduce_max(es.elapsed_time(ee) / e_steps, device)
+    e2e = {"value": round(whole_job_rate(flops, 1, world, e_ms) / 1e12, 4), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in pin.values())),
+           "d2h_bytes_per_step": int(host_out.numel() * host_out.element_size()),
+           "ms_per_step": round(e_ms, 4), "steps": e_steps,
+           "path": "lf_output_layer with pinned host copies of attn, residual and the output"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import os
+        import numpy as np
+        from oracle.projection import output_layer as oracle_output_layer
+        f = lambda t: t.double().numpy()
+        rows = min(wl.n, 256)
+        X = {k: f(v) for k, v in x0.items()}
+        reps_, t0 = 0, time.perf_counter()
+        while True:
+            oracle_output_layer(X["attn"][:1, :, :rows], X["wo"], X["bo"], X["residual"][:1, :rows],
+                                X["gamma"], X["beta"])
+            reps_ += 1
+            dt = time.perf_counter() - t0
+            if dt > args.cpu_seconds or reps_ >= 1000:
+                break
+        cflops = 2.0 * rows * hid * hid
+        cpu = {"value": round(cflops * reps_ / dt / 1e12, 6), "unit": "TFLOP/s",
+               "cores": os.cpu_count(), "kind": "oracle",
+               "sample": f"first {rows} tokens of batch 0, {reps_} repetition(s), {dt:.1f} s, "
+                         "fp64 numpy oracle (BLAS threads)", "seconds": round(dt, 2)}
+    result = {
+        "metric": OUT_METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.name, "op": "output", "B": wl.B, "H": wl.H, "n": wl.n,
+                   "hidden": hid, "eps": 1e-5, "global_batch": wl.B * world, "seq_len": wl.n,
+                   "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"{nsets} rotating input sets, {nsets * per_set / 2**20:.0f} MiB > 2x L2",
+                   "launch": "CUDA graph of C-ABI calls",
+                   "useful_gflop_per_step": round(flops / 1e9, 4)},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": 2 * steps, "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        del g
+        dist.destroy_process_group()
+
+
 def run_projection_cpu_baseline(wl, counts, gidx, max_global, budget_s):
     """The fp64 projection oracle on the first tokens of batch 0 (a bounded
     sample), scaled to the metric's unit."""
@@ -681,9 +835,10 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["attention", "projection"], default="attention",
+    ap.add_argument("--op", choices=["attention", "projection", "output"], default="attention",
                     help="attention: the hot path (default); projection: the Q/K/V/Kg/Vg/Qg "
-                         "prologue on the workload's shape")
+                         "prologue; output: the output projection + LayerNorm, on the "
+                         "workload's shape")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -695,10 +850,11 @@ def main(argv=None):
     if args.impl == "reference":
         run_reference_arm(args, wl, world, rank)
         return
-    if args.op == "projection":
+    if args.op in ("projection", "output"):
         if wl.dtype == "f32":
-            ap.error("the projection prologue runs on bf16 / fp16 workloads")
-        run_projection_arm(args, wl, world, rank, local)
+            ap.error("the projection and output layers run on bf16 / fp16 workloads")
+        (run_projection_arm if args.op == "projection" else run_output_arm)(
+            args, wl, world, rank, local)
         return
     run_gpu_arm(args, wl, world, rank, local)
 
