@@ -21,6 +21,7 @@
 // Every mbarrier wait is bounded; on expiry the kernel records
 // LF_ERR_DEVICE_TIMEOUT in the optional status word, drains its copies and
 // MMAs, frees its TMEM and returns.
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <type_traits>
@@ -36,14 +37,16 @@ namespace proj {
 using namespace sm100;
 
 constexpr int kTileM = 128;
-constexpr int kTileN = 128;
+constexpr int kTileN = 256;
 constexpr int kTileK = 64;                      // 128-byte rows of 16-bit elements
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kThreads = 192;
 constexpr int kWarpProducer = 4;
 constexpr int kWarpMma = 5;
-constexpr uint32_t kTmemCols = 128;
-constexpr int kSliceBytes = kTileM * kTileK * 2;   // 16 KB per operand slice
+constexpr uint32_t kTmemCols = 2 * kTileN;        // two accumulators: epilogue of one
+                                                  // tile overlaps the MMAs of the next
+constexpr int kSliceBytes = kTileM * kTileK * 2;   // 16 KB slice of A
+constexpr int kBSliceBytes = kTileN * kTileK * 2;  // 32 KB slice of W
 
 // One product C = A W^T + bias.
 enum JobMode { kModeHeads = 0, kModeGather = 1, kModeResidual = 2 };
@@ -68,13 +71,28 @@ struct ProjParams {
     const int32_t *counts;   // [B]
     int32_t *status;         // optional device status word
     int K, B, H, n, max_global, mtiles0;
+    int ntiles0, ntiles1, tiles0, tiles;   // column tiles per row of tiles; tile counts
 };
+
+// Tile t of the persistent schedule: job, first row, first column (column
+// tiles fastest, so consecutive tiles share their rows of A).
+__device__ __forceinline__ const ProjJob &tile_of(const ProjParams &p, int t, int &m0, int &n0)
+{
+    if (t < p.tiles0) {
+        m0 = (t / p.ntiles0) * kTileM;
+        n0 = (t % p.ntiles0) * kTileN;
+        return p.job[0];
+    }
+    t -= p.tiles0;
+    m0 = (t / p.ntiles1) * kTileM;
+    n0 = (t % p.ntiles1) * kTileN;
+    return p.job[1];
+}
 
 struct __align__(1024) ProjSmem {
     uint8_t a[kStages][kSliceBytes];
-    uint8_t b[kStages][kSliceBytes];
-    float bias[kTileN];
-    uint64_t full[kStages], empty[kStages], acc_full, drain;
+    uint8_t b[kStages][kBSliceBytes];
+    uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -138,18 +156,16 @@ template <> __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Persistent: CTA c takes tiles c, c + gridDim.x, ...  The producer and the
+// MMA thread run through the K slices of consecutive tiles without a break;
+// the epilogue drains accumulator buffer t & 1 while the MMAs fill the other.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ ProjParams p)
+__global__ void __launch_bounds__(kThreads, 1) proj_kernel(const __grid_constant__ ProjParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     ProjSmem &sm = *reinterpret_cast<ProjSmem *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int jid = int(blockIdx.y) < p.mtiles0 ? 0 : 1;
-    const ProjJob &J = p.job[jid];
-    const int m0 = (jid == 0 ? blockIdx.y : blockIdx.y - p.mtiles0) * kTileM;
-    const int n0 = blockIdx.x * kTileN;
-    if (n0 >= J.N) return;                      // the Qg product is narrower
     const int ktiles = p.K / kTileK;
 
     if (threadIdx.x == 0) {
@@ -157,20 +173,19 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
-        mbar_init(&sm.acc_full, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_empty[b], 4);     // one arrival per epilogue warp
+        }
         mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
         mbar_fence_init();
     }
-    if (threadIdx.x < kTileN) {
-        const int o = n0 + threadIdx.x;
-        float bv = 0.f;
-        if (J.bias && o < J.N) bv = to_f32(static_cast<const T *>(J.bias)[o]);
-        sm.bias[threadIdx.x] = bv;
-    }
     if (warp == kWarpProducer && lane == 0) {
-        tma_prefetch_map(&J.a_map);
-        tma_prefetch_map(&J.b_tile);
+        for (int j = 0; j < 2; ++j) {
+            tma_prefetch_map(&p.job[j].a_map);
+            tma_prefetch_map(&p.job[j].b_tile);
+        }
     }
     if (warp == 0) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -183,55 +198,59 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
     volatile int *abort_flag = &sm.abort_flag;
 
     if (warp == kWarpProducer) {
-        // Gathered rows: only the real global tokens are loaded (the other
-        // rows of the tile feed output rows that are never stored).
-        int arow[kTileM / 32];
-        int a_bytes = kSliceBytes;
-        if (J.mode == kModeGather) {
-            int valid = 0;
-#pragma unroll
-            for (int q = 0; q < kTileM / 32; ++q) {
-                int b;
-                const int i = token_of(p, J, m0 + 32 * q + lane, b);
-                arow[q] = i >= 0 ? b * p.n + i : -1;
-                valid += __popc(__ballot_sync(0xffffffffu, i >= 0));
-            }
-            a_bytes = valid * (kTileK * 2);
-        }
-        int issued = 0;
+        int it = 0;          // K slices issued by this CTA
         bool ok = true;
-        for (int kt = 0; kt < ktiles && ok; ++kt) {
-            const int s = kt % kStages;
-            const uint32_t ph = uint32_t(kt / kStages) & 1u;
-            bool w = true;
-            if (lane == 0) w = wait_bar(&sm.empty[s], ph ^ 1u, abort_flag, p.status);
-            ok = __shfl_sync(0xffffffffu, w, 0);
-            if (!ok) break;
-            if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], a_bytes + kSliceBytes);
-            __syncwarp();
-            if (J.mode == kModeHeads) {
-                if (lane == 0) tma_load_2d(sm.a[s], &J.a_map, &sm.full[s], kt * kTileK, m0);
-            } else if (J.mode == kModeResidual) {
-                // K slice kt is head kt of the attention output: rows i0 .. i0+127
-                // of batch b (rows past n read as zeros).
-                const int b = m0 / (J.tiles_per_batch * kTileM);
-                const int i0 = m0 - b * J.tiles_per_batch * kTileM;
-                if (lane == 0) tma_load_3d(sm.a[s], &J.a_map, &sm.full[s], 0, i0, b * p.H + kt);
-            } else {
+        for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
+            int m0, n0;
+            const ProjJob &J = tile_of(p, t, m0, n0);
+            // Gathered rows: only the real global tokens are loaded (the other
+            // rows of the tile feed output rows that are never stored).
+            int arow[kTileM / 32];
+            int a_bytes = kSliceBytes;
+            if (J.mode == kModeGather) {
+                int valid = 0;
 #pragma unroll
-                for (int q = 0; q < kTileM / 32; ++q)
-                    if (arow[q] >= 0)
-                        tma_load_2d(sm.a[s] + (32 * q + lane) * (kTileK * 2), &J.a_map,
-                                    &sm.full[s], kt * kTileK, arow[q]);
+                for (int q = 0; q < kTileM / 32; ++q) {
+                    int b;
+                    const int i = token_of(p, J, m0 + 32 * q + lane, b);
+                    arow[q] = i >= 0 ? b * p.n + i : -1;
+                    valid += __popc(__ballot_sync(0xffffffffu, i >= 0));
+                }
+                a_bytes = valid * (kTileK * 2);
             }
-            if (lane == 0) tma_load_2d(sm.b[s], &J.b_tile, &sm.full[s], kt * kTileK, n0);
-            __syncwarp();
-            issued = kt + 1;
+            for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                const int s = it % kStages;
+                const uint32_t ph = uint32_t(it / kStages) & 1u;
+                bool w = true;
+                if (lane == 0) w = wait_bar(&sm.empty[s], ph ^ 1u, abort_flag, p.status);
+                ok = __shfl_sync(0xffffffffu, w, 0);
+                if (!ok) break;
+                if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], a_bytes + kBSliceBytes);
+                __syncwarp();
+                if (J.mode == kModeHeads) {
+                    if (lane == 0) tma_load_2d(sm.a[s], &J.a_map, &sm.full[s], kt * kTileK, m0);
+                } else if (J.mode == kModeResidual) {
+                    // K slice kt is head kt of the attention output: rows i0 ..
+                    // i0+127 of batch b (rows past n read as zeros).
+                    const int b = m0 / (J.tiles_per_batch * kTileM);
+                    const int i0 = m0 - b * J.tiles_per_batch * kTileM;
+                    if (lane == 0)
+                        tma_load_3d(sm.a[s], &J.a_map, &sm.full[s], 0, i0, b * p.H + kt);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < kTileM / 32; ++q)
+                        if (arow[q] >= 0)
+                            tma_load_2d(sm.a[s] + (32 * q + lane) * (kTileK * 2), &J.a_map,
+                                        &sm.full[s], kt * kTileK, arow[q]);
+                }
+                if (lane == 0) tma_load_2d(sm.b[s], &J.b_tile, &sm.full[s], kt * kTileK, n0);
+                __syncwarp();
+            }
         }
         if (*abort_flag && lane == 0) {
             // Copies still in flight land before the CTA exits.
-            for (int kt = max(0, issued - kStages); kt < issued; ++kt)
-                drain_bar(&sm.full[kt % kStages], uint32_t(kt / kStages) & 1u);
+            for (int k = max(0, it - kStages); k < it; ++k)
+                drain_bar(&sm.full[k % kStages], uint32_t(k / kStages) & 1u);
         }
         __syncwarp();
     } else if (warp == kWarpMma) {
@@ -239,53 +258,88 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
             constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
             const uint32_t idesc = make_idesc(kTileM, kTileN, kBf16, false);
             bool ok = true;
-            for (int kt = 0; kt < ktiles && ok; ++kt) {
-                const int s = kt % kStages;
-                ok = wait_bar(&sm.full[s], uint32_t(kt / kStages) & 1u, abort_flag, p.status);
+            int it = 0, tc = 0;
+            for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++tc) {
+                const int buf = tc & 1;
+                ok = wait_bar(&sm.acc_empty[buf], (uint32_t(tc >> 1) & 1u) ^ 1u, abort_flag,
+                              p.status);
                 if (!ok) break;
                 tc_fence_after();
-                const uint64_t ad = make_sdesc(smem_u32(sm.a[s]), 16, 1024);
-                const uint64_t bd = make_sdesc(smem_u32(sm.b[s]), 16, 1024);
+                const uint32_t acc = tmem + buf * kTileN;
+                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                    const int s = it % kStages;
+                    ok = wait_bar(&sm.full[s], uint32_t(it / kStages) & 1u, abort_flag, p.status);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint64_t ad = make_sdesc(smem_u32(sm.a[s]), 16, 1024);
+                    const uint64_t bd = make_sdesc(smem_u32(sm.b[s]), 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < kTileK / 16; ++kk)
-                    mma_ss(tmem, ad + uint64_t((kk * 32) >> 4), bd + uint64_t((kk * 32) >> 4), idesc,
-                           (kt > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(&sm.empty[s]);
+                    for (int kk = 0; kk < kTileK / 16; ++kk)
+                        mma_ss(acc, ad + uint64_t((kk * 32) >> 4), bd + uint64_t((kk * 32) >> 4),
+                               idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&sm.empty[s]);
+                }
+                if (ok) tc_commit(&sm.acc_full[buf]);
             }
-            if (ok) tc_commit(&sm.acc_full);
             // Every MMA issued here has completed once this commit lands.
             tc_commit(&sm.drain);
             drain_bar(&sm.drain, 0);
         }
         __syncwarp();
     } else {
-        // Epilogue: thread t owns output row m0 + t (TMEM lane t).
+        // Epilogue: thread t owns row m0 + t of each tile (TMEM lane t).
         bool ok = true;
-        if (lane == 0) ok = wait_bar(&sm.acc_full, 0, abort_flag, p.status);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (ok) {
+        int tc = 0;
+        for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++tc) {
+            int m0, n0;
+            const ProjJob &J = tile_of(p, t, m0, n0);
+            const int buf = tc & 1;
+            bool w = true;
+            if (lane == 0) w = wait_bar(&sm.acc_full[buf], uint32_t(tc >> 1) & 1u, abort_flag,
+                                        p.status);
+            ok = __shfl_sync(0xffffffffu, w, 0);
+            if (!ok) break;
             tc_fence_after();
             int b;
             const int i = token_of(p, J, m0 + threadIdx.x, b);
             const int hid = p.H * kDHead;
-            const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
+            const uint32_t taddr = tmem + buf * kTileN + (uint32_t(warp * 32) << 16);
 #pragma unroll
             for (int c = 0; c < kTileN / 32; ++c) {
                 float acc[32];
                 tmem_ld32(taddr + 32 * c, acc);
                 const int o = n0 + 32 * c;                 // 32 columns within one head
                 if (i < 0 || o >= J.N) continue;
+                float bias[32];
+                if (J.bias) {
+                    const uint4 *b4 = reinterpret_cast<const uint4 *>(static_cast<const T *>(J.bias) + o);
+                    uint4 bv[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) bv[q] = __ldg(b4 + q);
+                    const T *bt = reinterpret_cast<const T *>(bv);
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) bias[x] = to_f32(bt[x]);
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) bias[x] = 0.f;
+                }
                 if (J.mode == kModeResidual) {
                     const size_t row = (size_t(b) * p.n + i) * J.N + o;
-                    const T *res = static_cast<const T *>(J.residual) + row;
+                    // 32 residual values as four 16-byte loads.
+                    const uint4 *res4 = reinterpret_cast<const uint4 *>(
+                        static_cast<const T *>(J.residual) + row);
+                    uint4 rv[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) rv[q] = __ldg(res4 + q);
+                    const T *res = reinterpret_cast<const T *>(rv);
                     float4 *dst = reinterpret_cast<float4 *>(J.sum + row);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         float4 v;
-                        v.x = acc[4 * q + 0] + sm.bias[32 * c + 4 * q + 0] + to_f32(res[4 * q + 0]);
-                        v.y = acc[4 * q + 1] + sm.bias[32 * c + 4 * q + 1] + to_f32(res[4 * q + 1]);
-                        v.z = acc[4 * q + 2] + sm.bias[32 * c + 4 * q + 2] + to_f32(res[4 * q + 2]);
-                        v.w = acc[4 * q + 3] + sm.bias[32 * c + 4 * q + 3] + to_f32(res[4 * q + 3]);
+                        v.x = acc[4 * q + 0] + bias[4 * q + 0] + to_f32(res[4 * q + 0]);
+                        v.y = acc[4 * q + 1] + bias[4 * q + 1] + to_f32(res[4 * q + 1]);
+                        v.z = acc[4 * q + 2] + bias[4 * q + 2] + to_f32(res[4 * q + 2]);
+                        v.w = acc[4 * q + 3] + bias[4 * q + 3] + to_f32(res[4 * q + 3]);
                         dst[q] = v;
                     }
                     continue;
@@ -298,7 +352,7 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const float *v = acc + 8 * q;
-                    const float *bv = sm.bias + 32 * c + 8 * q;
+                    const float *bv = bias + 8 * q;
                     uint4 u;
                     u.x = pack2<T>(v[0] + bv[0], v[1] + bv[1]);
                     u.y = pack2<T>(v[2] + bv[2], v[3] + bv[3]);
@@ -307,6 +361,11 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
                     d4[q] = u;
                 }
             }
+            // This warp's rows of the accumulator are read: the buffer may be
+            // refilled.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
         }
     }
 
@@ -318,9 +377,26 @@ __global__ void __launch_bounds__(kThreads) proj_kernel(const __grid_constant__ 
     }
 }
 
-// LayerNorm of each row of the fp32 sums: one warp per row.  Mean first, then
-// the mean square deviation (two passes over the row, which stays in L1/L2),
-// then out = (s - mean) / sqrt(var + eps) * gamma + beta in the output type.
+// LayerNorm of each row of the fp32 sums: one warp per row.  Rows of up to
+// 32 * 4 * kLnRegs features are read once into registers; longer rows are
+// read again for each pass.  Mean first, then the mean square deviation, then
+// out = (s - mean) / sqrt(var + eps) * gamma + beta in the output type.
+constexpr int kLnRegs = 8;      // float4 per lane kept in registers (rows <= 1024)
+
+template <typename T>
+__device__ __forceinline__ void ln_store(T *dst, int o, float4 v, float mean, float inv,
+                                         const T *__restrict__ gamma, const T *__restrict__ beta)
+{
+    const float y0 = (v.x - mean) * inv * to_f32(gamma[o]) + to_f32(beta[o]);
+    const float y1 = (v.y - mean) * inv * to_f32(gamma[o + 1]) + to_f32(beta[o + 1]);
+    const float y2 = (v.z - mean) * inv * to_f32(gamma[o + 2]) + to_f32(beta[o + 2]);
+    const float y3 = (v.w - mean) * inv * to_f32(gamma[o + 3]) + to_f32(beta[o + 3]);
+    uint2 u;
+    u.x = pack2<T>(y0, y1);
+    u.y = pack2<T>(y2, y3);
+    *reinterpret_cast<uint2 *>(dst + o) = u;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) layernorm_kernel(const float *__restrict__ sum,
                                                         const T *__restrict__ gamma,
@@ -331,7 +407,39 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float *__restrict_
     const int lane = threadIdx.x & 31;
     if (warp >= rows) return;
     const float4 *r4 = reinterpret_cast<const float4 *>(sum + size_t(warp) * N);
+    T *dst = out + size_t(warp) * N;
     const int n4 = N / 4;
+    if (n4 <= 32 * kLnRegs) {
+        float4 v[kLnRegs];
+        float s = 0.f;
+#pragma unroll
+        for (int u = 0; u < kLnRegs; ++u) {
+            const int c = lane + 32 * u;
+            v[u] = c < n4 ? __ldcs(r4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+            s += (v[u].x + v[u].y) + (v[u].z + v[u].w);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        const float mean = s / float(N);
+        float q = 0.f;
+#pragma unroll
+        for (int u = 0; u < kLnRegs; ++u) {
+            if (lane + 32 * u < n4) {
+                const float a = v[u].x - mean, b = v[u].y - mean, e = v[u].z - mean,
+                            f = v[u].w - mean;
+                q += (a * a + b * b) + (e * e + f * f);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+        const float inv = rsqrtf(q / float(N) + eps);
+#pragma unroll
+        for (int u = 0; u < kLnRegs; ++u) {
+            const int c = lane + 32 * u;
+            if (c < n4) ln_store(dst, 4 * c, v[u], mean, inv, gamma, beta);
+        }
+        return;
+    }
     float s = 0.f;
     for (int c = lane; c < n4; c += 32) {
         const float4 v = r4[c];
@@ -349,19 +457,7 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const float *__restrict_
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
     const float inv = rsqrtf(q / float(N) + eps);
-    T *dst = out + size_t(warp) * N;
-    for (int c = lane; c < n4; c += 32) {
-        const float4 v = r4[c];
-        const int o = 4 * c;
-        const float y0 = (v.x - mean) * inv * to_f32(gamma[o]) + to_f32(beta[o]);
-        const float y1 = (v.y - mean) * inv * to_f32(gamma[o + 1]) + to_f32(beta[o + 1]);
-        const float y2 = (v.z - mean) * inv * to_f32(gamma[o + 2]) + to_f32(beta[o + 2]);
-        const float y3 = (v.w - mean) * inv * to_f32(gamma[o + 3]) + to_f32(beta[o + 3]);
-        uint2 u;
-        u.x = pack2<T>(y0, y1);
-        u.y = pack2<T>(y2, y3);
-        *reinterpret_cast<uint2 *>(dst + o) = u;
-    }
+    for (int c = lane; c < n4; c += 32) ln_store(dst, 4 * c, r4[c], mean, inv, gamma, beta);
 }
 
 // ------------------------------------------------------------------ host
@@ -424,9 +520,15 @@ int launch(const ProjParams &p, cudaStream_t stream)
             return kErrCuda;
         attr_set[dev] = true;
     }
-    const int mtiles1 = (p.job[1].M + kTileM - 1) / kTileM;
-    dim3 grid((p.job[0].N + kTileN - 1) / kTileN, p.mtiles0 + mtiles1);
-    proj_kernel<T><<<grid, kThreads, smem, stream>>>(p);
+    ProjParams q = p;
+    q.ntiles0 = (p.job[0].N + kTileN - 1) / kTileN;
+    q.ntiles1 = p.job[1].N > 0 ? (p.job[1].N + kTileN - 1) / kTileN : 1;
+    q.tiles0 = p.mtiles0 * q.ntiles0;
+    q.tiles = q.tiles0 + ((p.job[1].M + kTileM - 1) / kTileM) * (p.job[1].M > 0 ? q.ntiles1 : 0);
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = std::max(1, std::min(q.tiles, sms > 0 ? sms : 1));
+    proj_kernel<T><<<grid, kThreads, smem, stream>>>(q);
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 

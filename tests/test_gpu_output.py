@@ -20,6 +20,7 @@ CASES = [
     Workload("out-b1-n1000-h3", "f16", 1, 3, 1000, 16, seed=32),    # odd head count
     Workload("out-b1-n128-h16", "bf16", 1, 16, 128, 16, seed=33),   # one row tile, hidden 1024
     Workload("out-b1-n4096-h12", "bf16", 1, 12, 4096, 512, seed=34),  # Longformer-base shape
+    Workload("out-b1-n70-h20", "f16", 1, 20, 70, 16, seed=35),      # rows longer than 1024
 ]
 
 
