@@ -54,6 +54,7 @@ def load_peaks():
 TRAFFIC_SOURCES = {
     "attn_tc_kernel": ("lf_tc.cu", "lf_sm100.cuh", "lf_device.cuh"),
     "band_simt_kernel": ("lf_simt.cu", "lf_device.cuh"),
+    "proj_kernel": ("lf_proj.cu", "lf_sm100.cuh", "lf_device.cuh"),
 }
 
 
@@ -505,7 +506,8 @@ def run_projection_arm(args, wl, world, rank, local):
     kernel_tflops = flops / (ms_per_step * 1e-3) / 1e12
     roofline = {"kernel": "proj_kernel", "bound": "tensor", "achieved": round(kernel_tflops, 1),
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(kernel_tflops / peaks["bf16_tflops"], 4), "traffic": None,
+                "frac": round(kernel_tflops / peaks["bf16_tflops"], 4),
+                "traffic": stored_traffic("proj_kernel", wl.name),
                 "peak_source": peak_kind + " (bf16 dense; fp16 has the same nominal rate)"}
 
     # End to end: hidden states from pinned host memory in, six outputs back.
