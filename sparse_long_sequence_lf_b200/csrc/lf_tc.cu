@@ -10,13 +10,15 @@
 //   band items    128 query rows of one (batch, head, residue class of the
 //                 head's dilation).  A dilated head is a plain band over each
 //                 residue subsequence x[r::dil], so the same tile loop serves
-//                 every dilation.  The keys stream as 128-key tiles over the
+//                 every dilation.  The keys stream as 64-key tiles over the
 //                 band's diagonals, then as tiles of the (deduplicated) global
 //                 tokens; an online softmax runs over all of them.
 //   global items  up to 128 global rows of one (batch, head) against one
 //                 512-key chunk of Kg/Vg; each writes fp32 partials (max, sum,
-//                 unnormalised output) and the last chunk to finish merges
-//                 them by log-sum-exp into the output rows.
+//                 unnormalised output).  While a row spans at most 8 chunks,
+//                 the warp that finishes the last chunk of a group of 32 rows
+//                 merges them by log-sum-exp into the output rows; beyond
+//                 that combine_kernel does, after this kernel.
 //
 // Layout of one CTA (384 threads, one CTA per SM, persistent over items):
 //   warps 0-3   softmax warpgroup of lane 0   (one thread per query row)
@@ -36,9 +38,10 @@
 //   O += P V       tcgen05.mma kind::f16, A = P (TMEM), B = V tile
 //                  (smem, MN-major), 128x64 fp32 in TMEM
 // Shared-memory tiles have 128-byte rows with the 128-byte swizzle, written
-// by TMA: whole tiles for undilated rows, single-row loads for dilated rows,
-// global tokens and gathered Qg rows.  Q is double-buffered per lane, K/V
-// run through a 3-stage ring of 64-key tiles per lane.  Every wait on an mbarrier is
+// by TMA: whole tiles from residue-class tensor maps (rows r, r+dil, ...),
+// single-row loads for global tokens, gathered Qg rows and heads beyond the
+// residue-map budget.  Q is double-buffered per lane, K/V run through a
+// 3-stage ring of 64-key tiles per lane.  Every wait on an mbarrier is
 // bounded; on expiry the kernel records LF_ERR_DEVICE_TIMEOUT, drains its own
 // copies and MMAs, frees its TMEM and returns.
 #include <algorithm>
