@@ -354,11 +354,7 @@ def run_gpu_arm(args, wl, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic",
         "tokens_per_s": round(tokens_per_s, 1),
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "n": wl.n, "d_head": wl.d,
-                   "window": wl.window, "dilation": wl.dilation_list(), "causal": wl.causal,
-                   "globals": wl.globals_kind, "pad_tail": list(wl.pad_tail),
-                   "global_batch": wl.B * world, "seq_len": wl.n,
-                   "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU",
+        "config": {**workload_config(wl, world),
                    "l2": f"{nsets} rotating input sets, {nsets * per_set / 2**20:.0f} MiB > 2x L2",
                    "launch": "CUDA graph of C-ABI calls",
                    "useful_gflop_per_step": round(flops / 1e9, 4),
@@ -795,6 +791,15 @@ def run_cpu_baseline(wl, budget_s=10.0):
             "seconds": round(dt, 2)}
 
 
+def workload_config(wl, world):
+    """The workload part of a bench line's config (both arms)."""
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "n": wl.n, "d_head": wl.d,
+            "window": wl.window, "dilation": wl.dilation_list(), "causal": wl.causal,
+            "globals": wl.globals_kind, "pad_tail": list(wl.pad_tail),
+            "global_batch": wl.B * world, "seq_len": wl.n,
+            "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU"}
+
+
 def run_reference_arm(args, wl, world, rank):
     """The oracle as the reference arm: each step a bounded sample (one or more
     heads) of the same workload on the host cores.  Rank 0 only."""
@@ -817,7 +822,8 @@ def run_reference_arm(args, wl, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "n": wl.n, "window": wl.window},
+        "config": {**workload_config(wl, world),
+                   "sample": "a bounded number of heads per step (see cpu_baseline)"},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
