@@ -298,6 +298,51 @@ LF_API int lf_attention_forward_static(lf_dtype dtype, int B, int H, int n, int 
                          int max_global, int window, const int32_t *dilation, int causal,
                          void *out, lf_stream_t stream, void **scratch);
 
+/*
+ * Backward pass of the attention: the gradients of a scalar loss with
+ * respect to the six projections, given dO = dLoss/dO of the forward output.
+ * ("LongFormer: The Long-Document Transformer" notes, "Sliding Window",
+ * "Dilated Sliding Window", "Global Attention" define the attention; its
+ * derivative is the softmax-attention chain rule.  The pages print no
+ * backward of their own.)
+ *
+ * With s_ij = <q_i, k_j> / sqrt(d_head), p_ij = softmax over the keys of row
+ * i, and D_i = <dO_i, O_i>:
+ *   dv_j = sum_i p_ij dO_i,   dS_ij = p_ij (<dO_i, v_j> - D_i),
+ *   dq_i = sum_j dS_ij k_j / sqrt(d_head),  dk_j = sum_i dS_ij q_i / sqrt(d_head),
+ * where rows and keys run over the same sets as the forward: a valid
+ * non-global row i uses Q, K, V over its window taps and the global tokens,
+ * a valid global row uses Qg, Kg, Vg over every valid token.  Gradients of
+ * rows and keys that take part in nothing (padded tokens; Qg rows of
+ * non-global tokens; Q rows of global tokens) are written as zeros.
+ *
+ *   q ... vg, max_global, window, dilation, causal
+ *                as passed to the forward.
+ *   out          device [B, H, n, d_head]: the forward's output for these
+ *                inputs (the library's, or any O within rounding of it).
+ *   dout         device [B, H, n, d_head]: dLoss/dO.
+ *   dq ... dvg   device [B, H, n, d_head], out: every element is written.
+ *   workspace    the workspace of the forward, prepared for the same masks
+ *                and max_global (lf_attention_prepare or
+ *                lf_attention_forward); read only.
+ *   scratch      device, 256-byte aligned, lf_backward_scratch_size bytes:
+ *                per-row log-sum-exp and D between the kernels.
+ * Arithmetic in fp32 for every dtype; results are rounded to dtype once.
+ * Every tensor pointer must be 16-byte aligned.  Errors are returned before
+ * anything is launched, as for lf_attention_run.  More global tokens than
+ * max_global is recorded by the preparation in the workspace status word
+ * (lf_workspace_status), as for the forward.
+ */
+LF_API size_t lf_backward_scratch_size(int B, int H, int n, int d_head, int max_global);
+LF_API int lf_attention_backward(lf_dtype dtype, int B, int H, int n, int d_head,
+                         const void *q, const void *k, const void *v,
+                         const void *qg, const void *kg, const void *vg,
+                         const void *out, const void *dout,
+                         int max_global, int window, const int32_t *dilation, int causal,
+                         void *dq, void *dk, void *dv, void *dqg, void *dkg, void *dvg,
+                         const void *workspace, size_t workspace_bytes,
+                         void *scratch, size_t scratch_bytes, lf_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -66,6 +66,9 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         "lf_qkv_projection": (I, [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, P, P, P, P, P]),
         "lf_output_workspace_size": (Z, [I, I, I, I]),
         "lf_output_layer": (I, [I, I, I, I, I, P, P, P, P, P, P, ctypes.c_float, P, P, Z, P, P]),
+        "lf_backward_scratch_size": (Z, [I, I, I, I, I]),
+        "lf_attention_backward": (I, [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P, I, P, P, P,
+                                      P, P, P, P, Z, P, Z, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

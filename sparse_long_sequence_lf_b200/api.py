@@ -263,3 +263,33 @@ def output_layer(attn, wo, bo, residual, gamma, beta, *, eps: float = 1e-5, out=
         _ptr(gamma), _ptr(beta), float(eps), _ptr(out), _ptr(workspace), workspace.numel(),
         _ptr(status), _stream_ptr(stream)), "lf_output_layer")
     return out
+
+
+def backward_scratch_size(B: int, H: int, n: int, max_global: int) -> int:
+    return int(_lib.lib().lf_backward_scratch_size(B, H, n, D_HEAD, max_global))
+
+
+def attention_backward(q, k, v, qg, kg, vg, out, dout, *, window, dilation=None, causal=False,
+                       max_global, workspace, grads=None, scratch=None, stream=None):
+    """``lf_attention_backward``: gradients of the attention with respect to
+    q, k, v, qg, kg, vg given the forward output ``out`` and dLoss/dout.
+
+    ``workspace`` is the forward's prepared workspace (same masks and
+    max_global).  Returns a dict of the six gradients (``grads`` may supply
+    them, keyed q, k, v, qg, kg, vg).
+    """
+    dt, (B, H, n, _) = _check_projections([q, k, v, qg, kg, vg])
+    _check_projections([q, out, dout])
+    names = ("q", "k", "v", "qg", "kg", "vg")
+    if grads is None:
+        grads = {nm: torch.empty_like(q) for nm in names}
+    _check_projections([q] + [grads[nm] for nm in names])
+    if scratch is None:
+        scratch = torch.empty(backward_scratch_size(B, H, n, max_global), dtype=torch.uint8,
+                              device=q.device)
+    _lib.check(_lib.lib().lf_attention_backward(
+        dt, B, H, n, D_HEAD, _ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg), _ptr(vg), _ptr(out),
+        _ptr(dout), int(max_global), int(window), _dilation(dilation, H), int(bool(causal)),
+        *[_ptr(grads[nm]) for nm in names], _ptr(workspace), workspace.numel(), _ptr(scratch),
+        scratch.numel(), _stream_ptr(stream)), "lf_attention_backward")
+    return grads

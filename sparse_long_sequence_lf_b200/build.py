@@ -19,7 +19,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(BUILD, "liblf_attention.so")
-SOURCES = ["lf_api.cu", "lf_prepare.cu", "lf_simt.cu", "lf_tc.cu", "lf_static.cu", "lf_proj.cu"]
+SOURCES = ["lf_api.cu", "lf_prepare.cu", "lf_simt.cu", "lf_tc.cu", "lf_static.cu", "lf_proj.cu",
+           "lf_bwd.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -2,9 +2,11 @@
 // layout, kernel dispatch.  Declared in include/lf_attention.h.
 #include <cmath>
 #include <cstring>
+#include <initializer_list>
 
 #include "../../include/lf_attention.h"
 #include "lf_device.cuh"
+#include "lf_bwd.cuh"
 
 namespace lf {
 int launch_prepare(const uint8_t *local_mask, const uint8_t *global_mask, int B, int n,
@@ -61,6 +63,61 @@ int check_workspace(const void *ws, size_t bytes, const WsLayout &L)
     if (ws == nullptr) return kErrWorkspace;
     if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return kErrWorkspace;
     if (bytes < L.total) return kErrWorkspace;
+    return kOk;
+}
+
+// Checks the arguments shared by the forward run and the backward pass and
+// fills the kernel arguments; nothing is launched and the device is not
+// queried.
+int make_args(lf_dtype dtype, int B, int H, int n, int d_head, const void *q, const void *k,
+              const void *v, const void *qg, const void *kg, const void *vg, int max_global,
+              int window, const int32_t *dilation, int causal, void *workspace,
+              size_t workspace_bytes, std::initializer_list<const void *> outputs, AttnArgs &a)
+{
+    if (d_head != kDHead) return LF_ERR_UNSUPPORTED;
+    if (elem_size(dtype) == 0) return LF_ERR_INVALID_ARG;
+    if (!sizes_ok(B, H, n) || max_global < 0 || max_global > n) return LF_ERR_INVALID_ARG;
+    if (!q || !k || !v || !qg || !kg || !vg) return LF_ERR_INVALID_ARG;
+    // Tiles move as 16-byte pieces (TMA boxes, vector loads).
+    for (const void *ptr : {q, k, v, qg, kg, vg})
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return LF_ERR_INVALID_ARG;
+    for (const void *ptr : outputs)
+        if (!ptr || (reinterpret_cast<uintptr_t>(ptr) & 15u)) return LF_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return LF_ERR_INVALID_ARG;
+    if (causal) {
+        if (window < 1) return LF_ERR_INVALID_ARG;
+        if (max_global != 0) return LF_ERR_UNSUPPORTED;
+    } else if (window < 2 || (window % 2) != 0) {
+        return LF_ERR_INVALID_ARG;
+    }
+    if (dilation)
+        for (int h = 0; h < H; ++h)
+            if (dilation[h] < 1) return LF_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(B, H, n, max_global);
+    if (int rc = check_workspace(workspace, workspace_bytes, L)) return rc;
+
+    std::memset(&a, 0, sizeof(a));
+    a.q = q; a.k = k; a.v = v; a.qg = qg; a.kg = kg; a.vg = vg;
+    a.L = L;
+    a.ws = ws_ptrs(workspace, L);
+    a.B = B; a.H = H; a.n = n;
+    a.window = window;
+    a.half = window / 2;
+    a.causal = causal;
+    a.max_global = max_global;
+    a.scale_log2 = float(1.4426950408889634 / std::sqrt(double(kDHead)));
+    int items = 0;
+    for (int h = 0; h < H; ++h) {
+        const int dil = dilation ? dilation[h] : 1;
+        a.dil[h] = dil;
+        a.head_prefix[h] = items;
+        for (int r = 0; r < dil && r < n; ++r) {
+            const int n_r = (n - r + dil - 1) / dil;
+            items += (n_r + 127) / 128;
+        }
+    }
+    a.head_prefix[H] = items;
+    a.band_items_per_batch = items;
     return kOk;
 }
 
@@ -122,52 +179,12 @@ int lf_attention_run(lf_dtype dtype, int B, int H, int n, int d_head, const void
                      int max_global, int window, const int32_t *dilation, int causal, void *out,
                      void *workspace, size_t workspace_bytes, lf_stream_t stream)
 {
-    if (d_head != kDHead) return LF_ERR_UNSUPPORTED;
-    if (elem_size(dtype) == 0) return LF_ERR_INVALID_ARG;
-    if (!sizes_ok(B, H, n) || max_global < 0 || max_global > n) return LF_ERR_INVALID_ARG;
-    if (!q || !k || !v || !qg || !kg || !vg || !out) return LF_ERR_INVALID_ARG;
-    // Tiles move as 16-byte pieces (TMA boxes, vector loads).
-    for (const void *ptr : {q, k, v, qg, kg, vg, static_cast<const void *>(out)})
-        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return LF_ERR_INVALID_ARG;
-    if (causal != 0 && causal != 1) return LF_ERR_INVALID_ARG;
-    if (causal) {
-        if (window < 1) return LF_ERR_INVALID_ARG;
-        if (max_global != 0) return LF_ERR_UNSUPPORTED;
-    } else if (window < 2 || (window % 2) != 0) {
-        return LF_ERR_INVALID_ARG;
-    }
-    if (dilation)
-        for (int h = 0; h < H; ++h)
-            if (dilation[h] < 1) return LF_ERR_INVALID_ARG;
-    const WsLayout L = ws_layout(B, H, n, max_global);
-    if (int rc = check_workspace(workspace, workspace_bytes, L)) return rc;
-    if (int rc = device_ok()) return rc;
-
     AttnArgs a;
-    std::memset(&a, 0, sizeof(a));
-    a.q = q; a.k = k; a.v = v; a.qg = qg; a.kg = kg; a.vg = vg;
+    if (int rc = make_args(dtype, B, H, n, d_head, q, k, v, qg, kg, vg, max_global, window,
+                           dilation, causal, workspace, workspace_bytes, {out}, a))
+        return rc;
+    if (int rc = device_ok()) return rc;
     a.out = out;
-    a.L = L;
-    a.ws = ws_ptrs(workspace, L);
-    a.B = B; a.H = H; a.n = n;
-    a.window = window;
-    a.half = window / 2;
-    a.causal = causal;
-    a.max_global = max_global;
-    a.scale_log2 = float(1.4426950408889634 / std::sqrt(double(kDHead)));
-    int items = 0;
-    for (int h = 0; h < H; ++h) {
-        const int dil = dilation ? dilation[h] : 1;
-        a.dil[h] = dil;
-        a.head_prefix[h] = items;
-        for (int r = 0; r < dil && r < n; ++r) {
-            const int n_r = (n - r + dil - 1) / dil;
-            items += (n_r + 127) / 128;
-        }
-    }
-    a.head_prefix[H] = items;
-    a.band_items_per_batch = items;
-
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (dtype) {
         case LF_F32: return launch_simt<float>(a, s);
@@ -309,6 +326,48 @@ int lf_output_layer(lf_dtype dtype, int B, int n, int H, int d_head, const void 
     return launch_output_layer(dtype, B, n, H, attn, wo, bo, residual, gamma, beta, eps, out,
                                static_cast<float *>(workspace), status,
                                static_cast<cudaStream_t>(stream));
+}
+
+size_t lf_backward_scratch_size(int B, int H, int n, int d_head, int max_global)
+{
+    if (!sizes_ok(B, H, n) || d_head != kDHead || max_global < 0 || max_global > n) return 0;
+    return lf_align256(2 * sizeof(float) * size_t(B) * H * n) +
+           lf_align256(2 * sizeof(float) * size_t(B) * H * (max_global > 0 ? max_global : 1));
+}
+
+int lf_attention_backward(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
+                          const void *k, const void *v, const void *qg, const void *kg,
+                          const void *vg, const void *out, const void *dout, int max_global,
+                          int window, const int32_t *dilation, int causal, void *dq, void *dk,
+                          void *dv, void *dqg, void *dkg, void *dvg, const void *workspace,
+                          size_t workspace_bytes, void *scratch, size_t scratch_bytes,
+                          lf_stream_t stream)
+{
+    BwdArgs A;
+    if (int rc = make_args(dtype, B, H, n, d_head, q, k, v, qg, kg, vg, max_global, window,
+                           dilation, causal, const_cast<void *>(workspace), workspace_bytes,
+                           {out, dout, dq, dk, dv, dqg, dkg, dvg}, A.a))
+        return rc;
+    const size_t need = lf_backward_scratch_size(B, H, n, d_head, max_global);
+    if (!scratch || scratch_bytes < need || reinterpret_cast<uintptr_t>(scratch) % 256)
+        return LF_ERR_WORKSPACE;
+    if (int rc = device_ok()) return rc;
+    A.out = out;
+    A.dout = dout;
+    A.dq = dq; A.dk = dk; A.dv = dv; A.dqg = dqg; A.dkg = dkg; A.dvg = dvg;
+    const size_t rows = size_t(B) * H * n;
+    char *base = static_cast<char *>(scratch);
+    A.lse = reinterpret_cast<float *>(base);
+    A.dsum = A.lse + rows;
+    A.lse_g = reinterpret_cast<float *>(base + lf_align256(2 * sizeof(float) * rows));
+    A.dsum_g = A.lse_g + size_t(B) * H * (max_global > 0 ? max_global : 1);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    switch (dtype) {
+        case LF_F32: return launch_backward<float>(A, 4, s);
+        case LF_F16: return launch_backward<__half>(A, 2, s);
+        case LF_BF16: return launch_backward<__nv_bfloat16>(A, 2, s);
+    }
+    return LF_ERR_INVALID_ARG;
 }
 
 }  // extern "C"

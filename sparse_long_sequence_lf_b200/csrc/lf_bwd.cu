@@ -1,0 +1,551 @@
+// Backward pass of the attention on the CUDA cores (fp32 arithmetic for
+// every input type).
+//
+// With s_ij = <q_i, k_j> / sqrt(d), p_ij = exp(s_ij - lse_i) over the key set
+// of row i (the same sets as the forward: window taps and global tokens for a
+// valid non-global row through Q, K, V; every valid token for a valid global
+// row through Qg, Kg, Vg) and D_i = <dO_i, O_i>:
+//   dP_ij = <dO_i, v_j>,  dS_ij = p_ij (dP_ij - D_i)
+//   dq_i = sum_j dS_ij k_j / sqrt(d),  dk_j = sum_i dS_ij q_i / sqrt(d),
+//   dv_j = sum_i p_ij dO_i.
+// ("LongFormer: The Long-Document Transformer" notes, "Sliding Window",
+// "Dilated Sliding Window", "Global Attention": the attention these rows
+// differentiate.)
+//
+// Four kernels, no atomics: every output row is owned by one thread quad.
+//   rows    32 query rows of one (batch, head, residue class) per CTA, four
+//           threads per row (a quarter of the head dimension each): pass 1
+//           recomputes the row's log-sum-exp over its keys, pass 2 sums dq;
+//           writes lse and D per row for the key kernel.
+//   keys    32 keys of one (batch, head, residue class) per CTA: dk, dv over
+//           the window rows that reach the key, plus, for a global token,
+//           every other valid non-global row of the head.
+//   grows   the global rows (Qg): lse, D and dqg over every valid key.
+//   gkeys   dkg, dvg of every key over the global rows.
+#include "lf_bwd.cuh"
+#include "lf_vec.cuh"
+
+namespace lf {
+
+namespace bwd {
+
+constexpr int kRows = 32;               // rows (or keys) per CTA
+constexpr int kThreads = 4 * kRows;     // four threads per row
+constexpr int kParts = 128 / kRows;     // CTAs per 128-row band item
+constexpr int kTile = 32;               // keys (or rows) staged at a time
+constexpr int kQ = kDHead / 4;          // dimensions per thread
+
+__device__ __forceinline__ float quad_sum(float x)
+{
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    return x;
+}
+
+// 32 rows of 64 values staged in shared memory by 128 threads: thread t loads
+// row t/16 + 8u, dims 4*(t%16) .. +3, for u = 0..3.
+template <typename T>
+__device__ __forceinline__ void stage_rows(float (*dst)[kDHead], const T *base, const int (&pos)[4],
+                                           int tid)
+{
+    const int x4 = 4 * (tid & 15);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int c = (tid >> 4) + 8 * u;
+        const float4 v = pos[u] >= 0 ? load4(base + size_t(pos[u]) * kDHead + x4)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(&dst[c][x4]) = v;
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void load_quarter(float (&r)[kQ], const T *row, int qd, float scale)
+{
+#pragma unroll
+    for (int x = 0; x < kQ; x += 4) {
+        const float4 t = load4(row + kQ * qd + x);
+        r[x] = t.x * scale;
+        r[x + 1] = t.y * scale;
+        r[x + 2] = t.z * scale;
+        r[x + 3] = t.w * scale;
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void store_quarter(T *row, const float (&r)[kQ], int qd, float scale)
+{
+#pragma unroll
+    for (int x = 0; x < kQ; x += 4)
+        store4(row + kQ * qd + x,
+               make_float4(r[x] * scale, r[x + 1] * scale, r[x + 2] * scale, r[x + 3] * scale));
+}
+
+__device__ __forceinline__ float dot_quarter(const float (&r)[kQ], const float *s, int qd)
+{
+    float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+    for (int x = 0; x < kQ; x += 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(s + kQ * qd + x);
+        d0 = fmaf(r[x], v.x, d0);
+        d1 = fmaf(r[x + 1], v.y, d1);
+        d0 = fmaf(r[x + 2], v.z, d0);
+        d1 = fmaf(r[x + 3], v.w, d1);
+    }
+    return quad_sum(d0 + d1);
+}
+
+__device__ __forceinline__ void axpy_quarter(float (&r)[kQ], float a, const float *s, int qd)
+{
+#pragma unroll
+    for (int x = 0; x < kQ; x += 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(s + kQ * qd + x);
+        r[x] = fmaf(a, v.x, r[x]);
+        r[x + 1] = fmaf(a, v.y, r[x + 1]);
+        r[x + 2] = fmaf(a, v.z, r[x + 2]);
+        r[x + 3] = fmaf(a, v.w, r[x + 3]);
+    }
+}
+
+// ------------------------------------------------------------------ rows
+template <typename T>
+__global__ void __launch_bounds__(kThreads) rows_kernel(const BwdArgs A)
+{
+    const AttnArgs &a = A.a;
+    __shared__ __align__(16) float ks[kTile][kDHead];
+    __shared__ __align__(16) float vs[kTile][kDHead];
+    __shared__ int kpos[kTile];
+
+    int b, h, r, tile;
+    band_item(a, blockIdx.x / kParts, b, h, r, tile);
+    const int dil = a.dil[h];
+    const int n = a.n;
+    const int n_r = (n - r + dil - 1) / dil;
+    const int tid = threadIdx.x, rl = tid >> 2, qd = tid & 3;
+    const int r0 = tile * 128 + (blockIdx.x % kParts) * kRows;
+    if (r0 >= n_r) return;
+    const int ir = r0 + rl;
+    const bool row_in = ir < n_r;
+    const int i = ir * dil + r;
+    const size_t bh = size_t(b) * a.H + h;
+    const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
+    const uint32_t *gb = a.ws.gbits + size_t(b) * a.L.nwords;
+    const bool active = row_in && bit_at(vb, i) && !bit_at(gb, i);
+    const T *K = static_cast<const T *>(a.k) + bh * n * kDHead;
+    const T *V = static_cast<const T *>(a.v) + bh * n * kDHead;
+    const size_t rowoff = (bh * n + (row_in ? i : 0)) * kDHead;
+
+    float q[kQ], dO[kQ], dq[kQ];
+    float D = 0.f;
+    {
+        float o[kQ];
+        if (active) {
+            load_quarter(q, static_cast<const T *>(a.q) + rowoff, qd, a.scale_log2);
+            load_quarter(dO, static_cast<const T *>(A.dout) + rowoff, qd, 1.f);
+            load_quarter(o, static_cast<const T *>(A.out) + rowoff, qd, 1.f);
+        } else {
+#pragma unroll
+            for (int x = 0; x < kQ; ++x) q[x] = dO[x] = o[x] = 0.f;
+        }
+        float d = 0.f;
+#pragma unroll
+        for (int x = 0; x < kQ; ++x) d = fmaf(dO[x], o[x], d);
+        D = quad_sum(d);
+#pragma unroll
+        for (int x = 0; x < kQ; ++x) dq[x] = 0.f;
+    }
+
+    const int rows_hi = min(r0 + kRows - 1, n_r - 1);
+    int lo = max(r0 - (a.causal ? a.window - 1 : a.half), 0);
+    int hi = min(rows_hi + (a.causal ? 0 : a.half), n_r - 1);
+    const int g = min(a.ws.counts[b], a.max_global);
+    const int *gl = a.ws.gidx + size_t(b) * n;
+    const int nband = hi >= lo ? (hi - lo) / kTile + 1 : 0;
+    const int ntiles = nband + (g + kTile - 1) / kTile;
+
+    // Key position of column c of tile t, or -1.
+    auto key_at = [&](int t, int c) -> int {
+        if (t < nband) {
+            const int jr = lo + kTile * t + c;
+            return (jr <= hi && jr * dil + r < n) ? jr * dil + r : -1;
+        }
+        const int slot = kTile * (t - nband) + c;
+        return slot < g ? gl[slot] : -1;
+    };
+    // Is key column c of tile t a key of this row?
+    auto is_key = [&](int t, int c) -> bool {
+        const int j = kpos[c];
+        if (!active || j < 0) return false;
+        if (t < nband) {
+            const int jr = lo + kTile * t + c;
+            return a.causal ? (jr <= ir && ir - jr <= a.window - 1)
+                            : (jr - ir <= a.half && ir - jr <= a.half);
+        }
+        return !is_tap(i, j, a.window, a.half, dil, a.causal);
+    };
+    auto stage = [&](int t, bool with_v) {
+        __syncthreads();
+        int pos[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = (tid >> 4) + 8 * u;
+            const int j = key_at(t, c);
+            pos[u] = j;
+            if ((tid & 15) == 0) kpos[c] = (j >= 0 && bit_at(vb, j)) ? j : -1;
+        }
+        stage_rows(ks, K, pos, tid);
+        if (with_v) stage_rows(vs, V, pos, tid);
+        __syncthreads();
+    };
+
+    // Pass 1: log-sum-exp (log2 domain) of the row's scores.
+    float m = -INFINITY, l = 0.f;
+    for (int t = 0; t < ntiles; ++t) {
+        stage(t, false);
+        for (int c = 0; c < kTile; ++c) {
+            const float s = dot_quarter(q, ks[c], qd);
+            if (!is_key(t, c)) continue;
+            const float mn = fmaxf(m, s);
+            l = l * exp2f(m - mn) + exp2f(s - mn);
+            m = mn;
+        }
+    }
+    const float lse = l > 0.f ? m + log2f(l) : INFINITY;
+
+    // Pass 2: dq.
+    for (int t = 0; t < ntiles; ++t) {
+        stage(t, true);
+        for (int c = 0; c < kTile; ++c) {
+            const float s = dot_quarter(q, ks[c], qd);
+            const float dp = dot_quarter(dO, vs[c], qd);
+            if (!is_key(t, c)) continue;
+            const float p = exp2f(s - lse);
+            axpy_quarter(dq, p * (dp - D), ks[c], qd);
+        }
+    }
+
+    if (!row_in) return;
+    // dq = sum dS k / sqrt(d); scale_log2 = log2(e) / sqrt(d).
+    const float inv_sqrt_d = a.scale_log2 * 0.69314718055994531f;
+    store_quarter(static_cast<T *>(A.dq) + rowoff, dq, qd, inv_sqrt_d);
+    if (qd == 0) {
+        A.lse[bh * n + i] = active ? lse : INFINITY;
+        A.dsum[bh * n + i] = D;
+    }
+}
+
+// ------------------------------------------------------------------ keys
+template <typename T>
+__global__ void __launch_bounds__(kThreads) keys_kernel(const BwdArgs A)
+{
+    const AttnArgs &a = A.a;
+    __shared__ __align__(16) float qs[kTile][kDHead];
+    __shared__ __align__(16) float ds[kTile][kDHead];
+    __shared__ float lse_s[kTile], d_s[kTile];
+    __shared__ int rpos[kTile];
+    __shared__ int any_global;
+
+    int b, h, r, tile;
+    band_item(a, blockIdx.x / kParts, b, h, r, tile);
+    const int dil = a.dil[h];
+    const int n = a.n;
+    const int n_r = (n - r + dil - 1) / dil;
+    const int tid = threadIdx.x, rl = tid >> 2, qd = tid & 3;
+    const int k0 = tile * 128 + (blockIdx.x % kParts) * kRows;
+    if (k0 >= n_r) return;
+    const int jr = k0 + rl;
+    const bool key_in = jr < n_r;
+    const int j = jr * dil + r;
+    const size_t bh = size_t(b) * a.H + h;
+    const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
+    const uint32_t *gb = a.ws.gbits + size_t(b) * a.L.nwords;
+    const bool kvalid = key_in && bit_at(vb, j);
+    const bool kglobal = kvalid && bit_at(gb, j);
+    const size_t keyoff = (bh * n + (key_in ? j : 0)) * kDHead;
+    const T *Q = static_cast<const T *>(a.q) + bh * n * kDHead;
+    const T *dO = static_cast<const T *>(A.dout) + bh * n * kDHead;
+    const float *lse = A.lse + bh * n;
+    const float *dsum = A.dsum + bh * n;
+
+    float k[kQ], v[kQ], dk[kQ], dv[kQ];
+    if (kvalid) {
+        load_quarter(k, static_cast<const T *>(a.k) + keyoff, qd, a.scale_log2);
+        load_quarter(v, static_cast<const T *>(a.v) + keyoff, qd, 1.f);
+    } else {
+#pragma unroll
+        for (int x = 0; x < kQ; ++x) k[x] = v[x] = 0.f;
+    }
+#pragma unroll
+    for (int x = 0; x < kQ; ++x) dk[x] = dv[x] = 0.f;
+    if (tid == 0) any_global = 0;
+    __syncthreads();
+    if (kglobal && qd == 0) atomicOr(&any_global, 1);
+
+    // Stage rows at positions pos (band or any), then accumulate.
+    auto stage = [&](const int (&pos)[4]) {
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = (tid >> 4) + 8 * u;
+            if ((tid & 15) == 0) {
+                const int i = pos[u];
+                const bool act = i >= 0 && bit_at(vb, i) && !bit_at(gb, i);
+                rpos[c] = act ? i : -1;
+                lse_s[c] = act ? lse[i] : INFINITY;
+                d_s[c] = act ? dsum[i] : 0.f;
+            }
+        }
+        stage_rows(qs, Q, pos, tid);
+        stage_rows(ds, dO, pos, tid);
+        __syncthreads();
+    };
+    auto accumulate = [&](int c) {
+        const float s = dot_quarter(k, qs[c], qd);
+        const float dp = dot_quarter(v, ds[c], qd);
+        return make_float2(s, dp);
+    };
+
+    // Window rows: residue rows within reach of these keys.
+    const int keys_hi = min(k0 + kRows - 1, n_r - 1);
+    const int lo = max(a.causal ? k0 : k0 - a.half, 0);
+    const int hi = min(a.causal ? keys_hi + a.window - 1 : keys_hi + a.half, n_r - 1);
+    for (int t0 = lo; t0 <= hi; t0 += kTile) {
+        int pos[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int ir = t0 + (tid >> 4) + 8 * u;
+            pos[u] = (ir <= hi && ir * dil + r < n) ? ir * dil + r : -1;
+        }
+        stage(pos);
+        for (int c = 0; c < kTile; ++c) {
+            const float2 sd = accumulate(c);
+            const int ir = t0 + c;
+            const bool tap = a.causal ? (jr <= ir && ir - jr <= a.window - 1)
+                                      : (jr - ir <= a.half && ir - jr <= a.half);
+            if (!kvalid || rpos[c] < 0 || !tap) continue;
+            const float p = exp2f(sd.x - lse_s[c]);
+            axpy_quarter(dv, p, ds[c], qd);
+            axpy_quarter(dk, p * (sd.y - d_s[c]), qs[c], qd);
+        }
+    }
+    // A global token is a key of every valid non-global row of the head; the
+    // rows already counted as window taps are skipped.
+    __syncthreads();
+    if (any_global) {
+        for (int t0 = 0; t0 < n; t0 += kTile) {
+            int pos[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = t0 + (tid >> 4) + 8 * u;
+                pos[u] = i < n ? i : -1;
+            }
+            stage(pos);
+            for (int c = 0; c < kTile; ++c) {
+                const float2 sd = accumulate(c);
+                const int i = rpos[c];
+                if (!kglobal || i < 0 || is_tap(i, j, a.window, a.half, dil, a.causal)) continue;
+                const float p = exp2f(sd.x - lse_s[c]);
+                axpy_quarter(dv, p, ds[c], qd);
+                axpy_quarter(dk, p * (sd.y - d_s[c]), qs[c], qd);
+            }
+        }
+    }
+
+    if (!key_in) return;
+    const float inv_sqrt_d = a.scale_log2 * 0.69314718055994531f;
+    store_quarter(static_cast<T *>(A.dk) + keyoff, dk, qd, inv_sqrt_d);
+    store_quarter(static_cast<T *>(A.dv) + keyoff, dv, qd, 1.f);
+}
+
+// ------------------------------------------------------------ global rows
+template <typename T>
+__global__ void __launch_bounds__(kThreads) grows_kernel(const BwdArgs A)
+{
+    const AttnArgs &a = A.a;
+    __shared__ __align__(16) float ks[kTile][kDHead];
+    __shared__ __align__(16) float vs[kTile][kDHead];
+    __shared__ int kok[kTile];
+
+    // One CTA per (batch*head, 32 global slots), flattened.
+    const int gparts = (a.max_global + kRows - 1) / kRows;
+    const int bh = blockIdx.x / gparts;
+    const int s0 = (blockIdx.x % gparts) * kRows;
+    const int b = bh / a.H;
+    const int n = a.n;
+    const int tid = threadIdx.x, rl = tid >> 2, qd = tid & 3;
+    const int g = min(a.ws.counts[b], a.max_global);
+    const int slot = s0 + rl;
+    if (s0 >= g) return;
+    const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
+    const int i = slot < g ? a.ws.gidx[size_t(b) * n + slot] : -1;
+    const bool active = i >= 0 && bit_at(vb, i);
+    const size_t rowoff = (size_t(bh) * n + (active ? i : 0)) * kDHead;
+    const T *Kg = static_cast<const T *>(a.kg) + size_t(bh) * n * kDHead;
+    const T *Vg = static_cast<const T *>(a.vg) + size_t(bh) * n * kDHead;
+
+    float q[kQ], dO[kQ], dq[kQ];
+    float D = 0.f;
+    {
+        float o[kQ];
+        if (active) {
+            load_quarter(q, static_cast<const T *>(a.qg) + rowoff, qd, a.scale_log2);
+            load_quarter(dO, static_cast<const T *>(A.dout) + rowoff, qd, 1.f);
+            load_quarter(o, static_cast<const T *>(A.out) + rowoff, qd, 1.f);
+        } else {
+#pragma unroll
+            for (int x = 0; x < kQ; ++x) q[x] = dO[x] = o[x] = 0.f;
+        }
+        float d = 0.f;
+#pragma unroll
+        for (int x = 0; x < kQ; ++x) d = fmaf(dO[x], o[x], d);
+        D = quad_sum(d);
+#pragma unroll
+        for (int x = 0; x < kQ; ++x) dq[x] = 0.f;
+    }
+    auto stage = [&](int t0, bool with_v) {
+        __syncthreads();
+        int pos[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = (tid >> 4) + 8 * u;
+            const int jj = t0 + c;
+            pos[u] = jj < n ? jj : -1;
+            if ((tid & 15) == 0) kok[c] = jj < n && bit_at(vb, jj);
+        }
+        stage_rows(ks, Kg, pos, tid);
+        if (with_v) stage_rows(vs, Vg, pos, tid);
+        __syncthreads();
+    };
+    float m = -INFINITY, l = 0.f;
+    for (int t0 = 0; t0 < n; t0 += kTile) {
+        stage(t0, false);
+        for (int c = 0; c < kTile; ++c) {
+            const float s = dot_quarter(q, ks[c], qd);
+            if (!active || !kok[c]) continue;
+            const float mn = fmaxf(m, s);
+            l = l * exp2f(m - mn) + exp2f(s - mn);
+            m = mn;
+        }
+    }
+    const float lse = l > 0.f ? m + log2f(l) : INFINITY;
+    for (int t0 = 0; t0 < n; t0 += kTile) {
+        stage(t0, true);
+        for (int c = 0; c < kTile; ++c) {
+            const float s = dot_quarter(q, ks[c], qd);
+            const float dp = dot_quarter(dO, vs[c], qd);
+            if (!active || !kok[c]) continue;
+            const float p = exp2f(s - lse);
+            axpy_quarter(dq, p * (dp - D), ks[c], qd);
+        }
+    }
+    if (slot >= g) return;
+    if (qd == 0) {
+        A.lse_g[size_t(bh) * a.max_global + slot] = active ? lse : INFINITY;
+        A.dsum_g[size_t(bh) * a.max_global + slot] = D;
+    }
+    if (!active) return;
+    const float inv_sqrt_d = a.scale_log2 * 0.69314718055994531f;
+    store_quarter(static_cast<T *>(A.dqg) + rowoff, dq, qd, inv_sqrt_d);
+}
+
+// ------------------------------------------------------------ global keys
+template <typename T>
+__global__ void __launch_bounds__(kThreads) gkeys_kernel(const BwdArgs A)
+{
+    const AttnArgs &a = A.a;
+    __shared__ __align__(16) float qs[kTile][kDHead];
+    __shared__ __align__(16) float ds[kTile][kDHead];
+    __shared__ float lse_s[kTile], d_s[kTile];
+    __shared__ int rok[kTile];
+
+    // One CTA per (batch*head, 32 keys), flattened.
+    const int kparts = (a.n + kRows - 1) / kRows;
+    const int bh = blockIdx.x / kparts;
+    const int b = bh / a.H;
+    const int n = a.n;
+    const int tid = threadIdx.x, rl = tid >> 2, qd = tid & 3;
+    const int j = (blockIdx.x % kparts) * kRows + rl;
+    const bool key_in = j < n;
+    const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
+    const bool kvalid = key_in && bit_at(vb, j);
+    const size_t keyoff = (size_t(bh) * n + (key_in ? j : 0)) * kDHead;
+    const int g = min(a.ws.counts[b], a.max_global);
+    const int *gl = a.ws.gidx + size_t(b) * n;
+    const T *Qg = static_cast<const T *>(a.qg) + size_t(bh) * n * kDHead;
+    const T *dO = static_cast<const T *>(A.dout) + size_t(bh) * n * kDHead;
+
+    float k[kQ], v[kQ], dk[kQ], dv[kQ];
+    if (kvalid) {
+        load_quarter(k, static_cast<const T *>(a.kg) + keyoff, qd, a.scale_log2);
+        load_quarter(v, static_cast<const T *>(a.vg) + keyoff, qd, 1.f);
+    } else {
+#pragma unroll
+        for (int x = 0; x < kQ; ++x) k[x] = v[x] = 0.f;
+    }
+#pragma unroll
+    for (int x = 0; x < kQ; ++x) dk[x] = dv[x] = 0.f;
+
+    for (int s0 = 0; s0 < g; s0 += kTile) {
+        __syncthreads();
+        int pos[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = (tid >> 4) + 8 * u;
+            const int slot = s0 + c;
+            const int i = slot < g ? gl[slot] : -1;
+            const bool act = i >= 0 && bit_at(vb, i);
+            pos[u] = act ? i : -1;
+            if ((tid & 15) == 0) {
+                rok[c] = act;
+                lse_s[c] = act ? A.lse_g[size_t(bh) * a.max_global + slot] : INFINITY;
+                d_s[c] = act ? A.dsum_g[size_t(bh) * a.max_global + slot] : 0.f;
+            }
+        }
+        stage_rows(qs, Qg, pos, tid);
+        stage_rows(ds, dO, pos, tid);
+        __syncthreads();
+        for (int c = 0; c < kTile; ++c) {
+            const float s = dot_quarter(k, qs[c], qd);
+            const float dp = dot_quarter(v, ds[c], qd);
+            if (!kvalid || !rok[c]) continue;
+            const float p = exp2f(s - lse_s[c]);
+            axpy_quarter(dv, p, ds[c], qd);
+            axpy_quarter(dk, p * (dp - d_s[c]), qs[c], qd);
+        }
+    }
+    if (!key_in) return;
+    const float inv_sqrt_d = a.scale_log2 * 0.69314718055994531f;
+    store_quarter(static_cast<T *>(A.dkg) + keyoff, dk, qd, inv_sqrt_d);
+    store_quarter(static_cast<T *>(A.dvg) + keyoff, dv, qd, 1.f);
+}
+
+}  // namespace bwd
+
+template <typename T>
+int launch_backward(const BwdArgs &A, size_t elem, cudaStream_t stream)
+{
+    using namespace bwd;
+    const AttnArgs &a = A.a;
+    const size_t bytes = size_t(a.B) * a.H * a.n * kDHead * elem;
+    // Qg gets gradient rows only at global positions.
+    if (cudaMemsetAsync(A.dqg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
+    const int band_ctas = a.B * a.band_items_per_batch * kParts;
+    if (band_ctas > 0) {
+        rows_kernel<T><<<band_ctas, kThreads, 0, stream>>>(A);
+        keys_kernel<T><<<band_ctas, kThreads, 0, stream>>>(A);
+    }
+    if (a.max_global > 0) {
+        const int bh = a.B * a.H;
+        grows_kernel<T><<<bh * ((a.max_global + kRows - 1) / kRows), kThreads, 0, stream>>>(A);
+        gkeys_kernel<T><<<bh * ((a.n + kRows - 1) / kRows), kThreads, 0, stream>>>(A);
+    } else {
+        if (cudaMemsetAsync(A.dkg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
+        if (cudaMemsetAsync(A.dvg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
+    }
+    return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+}
+
+template int launch_backward<float>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_backward<__half>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_backward<__nv_bfloat16>(const BwdArgs &, size_t, cudaStream_t);
+
+}  // namespace lf

@@ -20,6 +20,7 @@
 // Encoder guide, "compute flow": softmax of local rows over window + global
 // tokens, of global rows over the whole sequence, masked rows zeroed.)
 #include "lf_device.cuh"
+#include "lf_vec.cuh"
 
 namespace lf {
 
@@ -27,50 +28,6 @@ constexpr int kSimtRows = 32;                     // query rows per band CTA
 constexpr int kSimtThreads = 4 * kSimtRows;       // four threads per row
 constexpr int kSimtParts = 128 / kSimtRows;       // band CTAs per 128-row band item
 constexpr int kSimtKeys = 32;
-
-// Four consecutive elements of a 16-byte (fp32) or 8-byte (fp16/bf16)
-// aligned address, as floats.
-template <typename T> __device__ __forceinline__ float4 load4(const T *p);
-template <> __device__ __forceinline__ float4 load4<float>(const float *p)
-{
-    return __ldg(reinterpret_cast<const float4 *>(p));
-}
-template <> __device__ __forceinline__ float4 load4<__half>(const __half *p)
-{
-    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
-    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&u.x));
-    const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&u.y));
-    return make_float4(a.x, a.y, b.x, b.y);
-}
-template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16 *p)
-{
-    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-    return make_float4(a.x, a.y, b.x, b.y);
-}
-
-template <typename T> __device__ __forceinline__ void store4(T *p, float4 v);
-template <> __device__ __forceinline__ void store4<float>(float *p, float4 v)
-{
-    *reinterpret_cast<float4 *>(p) = v;
-}
-template <> __device__ __forceinline__ void store4<__half>(__half *p, float4 v)
-{
-    __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
-    uint2 u;
-    u.x = *reinterpret_cast<uint32_t *>(&a);
-    u.y = *reinterpret_cast<uint32_t *>(&b);
-    *reinterpret_cast<uint2 *>(p) = u;
-}
-template <> __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, float4 v)
-{
-    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
-    uint2 u;
-    u.x = *reinterpret_cast<uint32_t *>(&a);
-    u.y = *reinterpret_cast<uint32_t *>(&b);
-    *reinterpret_cast<uint2 *>(p) = u;
-}
 
 // One staged tile of 32 keys: each thread holds 4 of the 512 four-element
 // pieces of K and of V (key c = tid/16 + 8u, dims 4*(tid%16) .. +3), loaded

@@ -205,3 +205,11 @@ def make_output_inputs(wl: Workload, seed: int | None = None) -> dict:
     dt = wl.torch_dtype
     return dict(attn=attn.to(dt), wo=wo.to(dt), bo=bo.to(dt), residual=residual.to(dt),
                 gamma=gamma.to(dt), beta=beta.to(dt))
+
+
+def make_output_grad(wl: Workload, seed: int | None = None) -> torch.Tensor:
+    """dLoss/dO [B, H, n, d] ~ N(0, 1) for the backward pass, a CPU tensor of
+    the workload dtype."""
+    gen = torch.Generator("cpu")
+    gen.manual_seed((wl.seed if seed is None else seed) + 900007)
+    return torch.randn((wl.B, wl.H, wl.n, wl.d), generator=gen).to(wl.torch_dtype)

@@ -77,3 +77,32 @@ def test_valid_call_without_gpu_reports_no_device(L):
     assert _run(L) == -7
     assert L.lf_global_index(ctypes.c_void_p(1), 1, 8, ctypes.c_void_p(1), ctypes.c_void_p(1),
                              None) == -7
+
+
+def test_backward_argument_checks(L):
+    import torch
+    P = ctypes.c_void_p
+
+    def bwd(**over):
+        a = dict(dtype=2, B=1, H=2, n=64, d=64, t=256, out=512, dout=512, g=768,
+                 max_global=0, window=8, causal=0, ws=256, wsb=1 << 20, sc=256, scb=1 << 20)
+        a.update(over)
+        t = P(a["t"])
+        return L.lf_attention_backward(
+            a["dtype"], a["B"], a["H"], a["n"], a["d"], t, t, t, t, t, t, P(a["out"]),
+            P(a["dout"]), a["max_global"], a["window"], None, a["causal"], P(a["g"]), P(a["g"]),
+            P(a["g"]), P(a["g"]), P(a["g"]), P(a["g"]), P(a["ws"]), a["wsb"], P(a["sc"]),
+            a["scb"], None)
+
+    assert L.lf_backward_scratch_size(1, 2, 64, 64, 0) >= 2 * 4 * 2 * 64
+    assert L.lf_backward_scratch_size(1, 2, 64, 32, 0) == 0
+    assert bwd(d=32) == -2
+    assert bwd(window=3) == -1
+    assert bwd(dout=0) == -1
+    assert bwd(g=520) == -1                             # misaligned gradient
+    assert bwd(ws=0) == -3
+    assert bwd(sc=0) == -3
+    assert bwd(sc=264) == -3                            # misaligned scratch
+    assert bwd(scb=8) == -3                             # scratch too small
+    if not torch.cuda.is_available():
+        assert bwd() == -7
