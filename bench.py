@@ -719,6 +719,350 @@ def run_output_arm(args, wl, world, rank, local):
         dist.destroy_process_group()
 
 
+BWD_METRIC = ("attention backward TFLOP/s (dq, dk, dv, dqg, dkg, dvg; 10*d flops per "
+              "attended pair), 1 B200")
+
+
+def run_backward_arm(args, wl, world, rank, local):
+    """One step = lf_attention_backward over one batch (the forward's output
+    and workspace prepared once beforehand).  The kernels run on the CUDA
+    cores in fp32: the roofline is the fp32 FMA rate of the SMs at the
+    sampled clock."""
+    import torch
+    import sparse_long_sequence_lf_b200 as lf
+    from sparse_long_sequence_lf_b200 import accounting
+    from sparse_long_sequence_lf_b200.workloads import make_inputs, make_output_grad
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist(world, "nccl")
+    stream = torch.cuda.Stream(device)
+    names = ("q", "k", "v", "qg", "kg", "vg")
+    x0 = make_inputs(wl)
+    mg = 0 if x0["global_mask"] is None else int((x0["global_mask"] != 0).sum(1).max())
+    t_bytes = wl.B * wl.H * wl.n * wl.d * x0["q"].element_size()
+    per_set = 14 * t_bytes
+    nsets = max(2, -(-2 * L2_BYTES // per_set))
+    sets = []
+    with torch.cuda.stream(stream):
+        for s_ in range(nsets):
+            xs = make_inputs(wl, seed=wl.seed + 7919 * s_) if s_ else x0
+            d = {k: (v.to(device) if torch.is_tensor(v) else v) for k, v in xs.items()}
+            d["ws"] = lf.new_workspace(wl.B, wl.H, wl.n, mg, device)
+            kw = dict(window=wl.window, dilation=xs["dilation"], causal=wl.causal,
+                      max_global=mg)
+            d["out"] = lf.attention_forward(*[d[nm] for nm in names], d["local_mask"],
+                                            d["global_mask"], workspace=d["ws"], stream=stream,
+                                            **kw)
+            d["dout"] = make_output_grad(wl, seed=wl.seed + 7919 * s_).to(device)
+            d["grads"] = {nm: torch.empty_like(d["q"]) for nm in names}
+            d["kw"] = kw
+            sets.append(d)
+    scratch = torch.empty(lf.backward_scratch_size(wl.B, wl.H, wl.n, mg), dtype=torch.uint8,
+                          device=device)
+    stream.synchronize()
+    for d in sets:
+        if lf.workspace_status(d["ws"]) != 0:
+            raise RuntimeError("forward status not ok")
+
+    def step(i):
+        d = sets[i % nsets]
+        lf.attention_backward(*[d[nm] for nm in names], d["out"], d["dout"],
+                              workspace=d["ws"], grads=d["grads"], scratch=scratch,
+                              stream=stream, **d["kw"])
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    stream.synchronize()
+    chunk = nsets * max(1, 8 // nsets)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(chunk):
+            step(i)
+    reps = max(1, -(-args.steps // chunk))
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        t_pad = time.time()
+        while time.time() - t_pad < 0.5:
+            with torch.cuda.stream(stream):
+                g.replay()
+            stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+        start.record(stream)
+        for _ in range(reps):
+            with torch.cuda.stream(stream):
+                g.replay()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+        if world > 1:
+            dist.barrier()
+    steps = reps * chunk
+    max_ms = reduce_max(start.elapsed_time(end), device)
+    clocks = sampler.summary("timed region plus 0.5 s of the same graph before it")
+    flops = accounting.backward_flops(wl)
+    ms_per_step = max_ms / steps
+    value = whole_job_rate(flops, steps, world, max_ms) / 1e12
+    tflops = flops / (ms_per_step * 1e-3) / 1e12
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965
+    peak = accounting.FP32_FLOPS_PER_CLOCK * mhz * 1e6 / 1e12
+    roofline = {"kernel": "bwd rows_kernel + keys_kernel (+ global rows / keys)",
+                "bound": "alu", "achieved": round(tflops, 2), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
+                "peak_source": f"derived: 148 SMs x 128 fp32 lanes x 2 flops x {mhz} MHz "
+                               "(median sampled SM clock)"}
+
+    # End to end through the host-buffer path: the eight inputs from pinned
+    # host memory in, the six gradients back.
+    dev = sets[0]
+    ins = list(names) + ["out", "dout"]
+    pin = {nm: (x0[nm] if nm in names else dev[nm].cpu()).pin_memory() for nm in ins}
+    host_g = {nm: torch.empty_like(x0["q"]).pin_memory() for nm in names}
+    stage = {nm: torch.empty_like(dev["q"]) for nm in ins}
+
+    def e2e_once():
+        with torch.cuda.stream(stream):
+            for nm in ins:
+                stage[nm].copy_(pin[nm], non_blocking=True)
+            lf.attention_backward(*[stage[nm] for nm in names], stage["out"], stage["dout"],
+                                  workspace=dev["ws"], grads=dev["grads"], scratch=scratch,
+                                  stream=stream, **dev["kw"])
+            for nm in names:
+                host_g[nm].copy_(dev["grads"][nm], non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(3):
+        e2e_once()
+    e_steps = max(3, min(args.steps, args.e2e_steps))
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    es.record(stream)
+    for _ in range(e_steps):
+        e2e_once()
+    ee.record(stream)
+    torch.cuda.synchronize(device)
+    e_ms = reduce_max(es.elapsed_time(ee) / e_steps, device)
+    e2e = {"value": round(whole_job_rate(flops, 1, world, e_ms) / 1e12, 4), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": 8 * t_bytes, "d2h_bytes_per_step": 6 * t_bytes,
+           "ms_per_step": round(e_ms, 4), "steps": e_steps,
+           "path": "lf_attention_backward with pinned host copies of the eight inputs and "
+                   "the six gradients (masks prepared once)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import os
+        from oracle import backward as obw
+        sub = wl.with_(B=1, H=1, n=min(wl.n, 1024), pad_tail=())
+        xs = make_inputs(sub)
+        dsub = make_output_grad(sub)
+        reps_, t0 = 0, time.perf_counter()
+        while True:
+            obw.backward(*[xs[nm] for nm in names], xs["local_mask"], xs["global_mask"], dsub,
+                         window=sub.window, dilation=xs["dilation"], causal=sub.causal)
+            reps_ += 1
+            dt = time.perf_counter() - t0
+            if dt > args.cpu_seconds or reps_ >= 100:
+                break
+        cflops = accounting.backward_flops(sub)
+        cpu = {"value": round(cflops * reps_ / dt / 1e12, 6), "unit": "TFLOP/s",
+               "cores": torch.get_num_threads(), "kind": "oracle",
+               "sample": f"batch 0, head 0, first {sub.n} tokens, {reps_} repetition(s), "
+                         f"{dt:.1f} s, fp64 dense-mask autograd oracle (torch CPU threads)",
+               "seconds": round(dt, 2)}
+    launches = 4 if mg > 0 else 2
+    result = {
+        "metric": BWD_METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic",
+        "config": {**workload_config(wl, world), "op": "backward",
+                   "l2": f"{nsets} rotating input sets, {nsets * per_set / 2**20:.0f} MiB > 2x L2",
+                   "launch": "CUDA graph of C-ABI calls",
+                   "useful_gflop_per_step": round(flops / 1e9, 4)},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches * steps, "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        del g
+        dist.destroy_process_group()
+
+
+ENC_METRIC = ("Longformer encoder stack latency, ms per forward (projections, attention, "
+              "output LayerNorm, GELU FFN per layer), 1 B200")
+# FasterTransformer's fp16 encoder latencies on A100-80GB for this model
+# (guide's benchmark table), keyed by (batch, seq_len): context, other hardware.
+FT_A100_FP16_MS = {(1, 1024): 14, (1, 2048): 31, (1, 4096): 50, (8, 1024): 79, (8, 2048): 208,
+                   (8, 4096): 369, (32, 1024): 305, (32, 2048): 820, (32, 4096): 823}
+
+
+def encoder_flops(ew, counts):
+    """Useful FLOPs of one stack forward: per layer the five projections over
+    all tokens and Qg over the global rows, the attention, the output
+    product and the two feed-forward products."""
+    from sparse_long_sequence_lf_b200 import accounting
+    wl = ew.attn
+    hid = wl.H * wl.d
+    tok = wl.B * wl.n
+    per_layer = (2.0 * tok * hid * 5 * hid + 2.0 * sum(counts) * hid * hid
+                 + accounting.useful_flops(wl) + 2.0 * tok * hid * hid
+                 + 2 * 2.0 * tok * hid * ew.inter)
+    return per_layer * ew.layers
+
+
+def run_encoder_arm(args, ew, world, rank, local):
+    """One step = one forward of the whole stack through lf_encoder_forward
+    (masks prepared inside the call).  Roofline: the stack's useful FLOPs
+    against the measured dense peak (its GEMMs dominate)."""
+    import torch
+    import sparse_long_sequence_lf_b200 as lf
+    from sparse_long_sequence_lf_b200.workloads import make_encoder_inputs, make_masks
+
+    wl = ew.attn
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist(world, "nccl")
+    stream = torch.cuda.Stream(device)
+    x0, layers = make_encoder_inputs(wl, ew.layers, ew.inter)
+    local_m, glob_m = make_masks(wl)
+    counts = [0] * wl.B if glob_m is None else [int(c) for c in (glob_m != 0).sum(1)]
+    mg = max(counts)
+    dev_layers = [{k: v.to(device) for k, v in lw.items()} for lw in layers]
+    x = x0.to(device)
+    lm = None if local_m is None else local_m.to(device)
+    gm = None if glob_m is None else glob_m.to(device)
+    out = torch.empty_like(x)
+    ws = torch.empty(lf.encoder_workspace_size(wl.B, wl.n, wl.H, ew.inter, mg),
+                     dtype=torch.uint8, device=device)
+    weight_bytes = sum(t.numel() * t.element_size() for lw in dev_layers for t in lw.values())
+    windows = [wl.window] * ew.layers
+
+    def step():
+        lf.encoder_forward(x, dev_layers, lm, gm, H=wl.H, windows=windows, max_global=mg,
+                           out=out, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    if lf.workspace_status(ws) != 0:
+        raise RuntimeError("encoder status not ok")
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        step()
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    steps = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+        start.record(stream)
+        for _ in range(steps):
+            with torch.cuda.stream(stream):
+                g.replay()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+        if world > 1:
+            dist.barrier()
+    max_ms = reduce_max(start.elapsed_time(end), device)
+    clocks = sampler.summary("timed region")
+    ms = max_ms / steps
+    flops = encoder_flops(ew, counts)
+    tflops = flops / (ms * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"kernel": "whole stack (proj_kernel GEMMs dominate)", "bound": "tensor",
+                "achieved": round(tflops, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(tflops / peak, 4), "traffic": None,
+                "peak_source": peak_kind + " sustained (bf16 dense; fp16 has the same nominal "
+                               "rate; the step runs for milliseconds)"}
+
+    pin_x = x0.pin_memory()
+    host_out = torch.empty_like(x0).pin_memory()
+    xd = torch.empty_like(x)
+
+    def e2e_once():
+        with torch.cuda.stream(stream):
+            xd.copy_(pin_x, non_blocking=True)
+            lf.encoder_forward(xd, dev_layers, lm, gm, H=wl.H, windows=windows, max_global=mg,
+                               out=out, workspace=ws, stream=stream)
+            host_out.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    e2e_once()
+    e_steps = max(3, min(steps, args.e2e_steps))
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    es.record(stream)
+    for _ in range(e_steps):
+        e2e_once()
+    ee.record(stream)
+    torch.cuda.synchronize(device)
+    e_ms = reduce_max(es.elapsed_time(ee) / e_steps, device)
+    e2e = {"value": round(e_ms, 4), "unit": "ms", "h2d_bytes_per_step":
+           int(x0.numel() * x0.element_size()),
+           "d2h_bytes_per_step": int(x0.numel() * x0.element_size()), "steps": e_steps,
+           "path": "lf_encoder_forward with the input copied from pinned host memory and the "
+                   "output copied back (weights resident)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import encoder as oenc
+        w0 = {k: v.double().numpy() for k, v in layers[0].items()}
+        # Sample: layer 0 over batch 0's first rows (every per-token cost is
+        # linear in the tokens at a fixed window), scaled to the whole stack.
+        rows = min(wl.n, 1024)
+        sl = lambda m: None if m is None else m[:1, :rows].contiguous()
+        t0 = time.perf_counter()
+        oenc.encoder_layer(x0[:1, :rows].double().numpy(), w0, sl(local_m), sl(glob_m), H=wl.H,
+                           window=wl.window)
+        dt = time.perf_counter() - t0
+        scale = ew.layers * wl.B * wl.n / rows
+        cpu = {"value": round(dt * 1e3 * scale, 1), "unit": "ms", "cores": os.cpu_count(),
+               "kind": "oracle",
+               "sample": f"layer 0 on the first {rows} tokens of batch 0 timed once "
+                         f"({dt:.1f} s, fp64 numpy products and the C attention oracle), "
+                         f"scaled by {scale:g} to the whole stack"}
+    ft = FT_A100_FP16_MS.get((wl.B, wl.n)) if wl.dtype == "f16" and ew.inter == 4096 \
+        and wl.H == 16 and ew.layers == 24 and wl.window == 512 else None
+    result = {
+        "metric": ENC_METRIC, "value": round(ms, 4), "unit": "ms", "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None if ft is None else round(ms / ft, 4),
+        "dtype": wl.dtype, "data": "synthetic (random-init weights)",
+        "config": {**workload_config(wl, world), "workload": ew.name, "op": "encoder",
+                   "layers": ew.layers, "inter": ew.inter, "hidden": wl.H * wl.d,
+                   "l2": f"weights {weight_bytes / 2**20:.0f} MiB per step > L2",
+                   "launch": "CUDA graph of one lf_encoder_forward call",
+                   "useful_tflop_per_step": round(flops / 1e12, 4),
+                   "tflops": round(tflops, 1),
+                   "vs_baseline_note": None if ft is None else
+                   f"ms / FasterTransformer's {ft} ms on A100-80GB (guide's table; other "
+                   "hardware, context only)"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": None, "clocks": clocks,
+    }
+    attn_launches = launches_per_step(wl, mg) - 1
+    result["gpu_launches"] = steps * (1 + ew.layers * (1 + attn_launches + 2 + 3))
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        del g
+        dist.destroy_process_group()
+
+
 def run_projection_cpu_baseline(wl, counts, gidx, max_global, budget_s):
     """The fp64 projection oracle on the first tokens of batch 0 (a bounded
     sample), scaled to the metric's unit."""
@@ -843,10 +1187,14 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["attention", "projection", "output"], default="attention",
+    ap.add_argument("--encoder", default=None,
+                    help="encoder stack of --op encoder (default: the 24-layer fp16 model)")
+    ap.add_argument("--op", choices=["attention", "projection", "output", "backward", "encoder"],
+                    default="attention",
                     help="attention: the hot path (default); projection: the Q/K/V/Kg/Vg/Qg "
-                         "prologue; output: the output projection + LayerNorm, on the "
-                         "workload's shape")
+                         "prologue; output: the output projection + LayerNorm; backward: the "
+                         "attention backward, on the workload's shape; encoder: a whole "
+                         "encoder stack (--encoder)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -863,6 +1211,14 @@ def main(argv=None):
             ap.error("the projection and output layers run on bf16 / fp16 workloads")
         (run_projection_arm if args.op == "projection" else run_output_arm)(
             args, wl, world, rank, local)
+        return
+    if args.op == "backward":
+        run_backward_arm(args, wl, world, rank, local)
+        return
+    if args.op == "encoder":
+        from sparse_long_sequence_lf_b200.workloads import ENCODER_HEADLINE, ENCODER_WORKLOADS
+        run_encoder_arm(args, ENCODER_WORKLOADS[args.encoder or ENCODER_HEADLINE], world, rank,
+                        local)
         return
     run_gpu_arm(args, wl, world, rank, local)
 

@@ -343,6 +343,89 @@ LF_API int lf_attention_backward(lf_dtype dtype, int B, int H, int n, int d_head
                          const void *workspace, size_t workspace_bytes,
                          void *scratch, size_t scratch_bytes, lf_stream_t stream);
 
+/*
+ * Feed-forward block of an encoder layer (FasterTransformer Longformer
+ * Encoder guide, "compute flow": intermediate product plus bias, GELU,
+ * output product, then bias, residual and LayerNorm once more):
+ *   act = GELU(h W1^T + b1),        GELU(x) = x * Phi(x) (the erf form)
+ *   out = LayerNorm(act W2^T + b2 + h) * gamma + beta
+ * Both products run on the tensor cores with fp32 accumulation; act is
+ * stored in dtype, the pre-normalisation sum in fp32.
+ *
+ *   dtype        LF_BF16 or LF_F16 (LF_F32: LF_ERR_UNSUPPORTED).
+ *   hidden       features per token; a multiple of 64.
+ *   inter        intermediate features; a multiple of 64.
+ *   h            device [B, n, hidden]: the block input (also the residual).
+ *   w1, b1       device [inter, hidden] (rows = output features), [inter] or NULL.
+ *   w2, b2       device [hidden, inter], [hidden] or NULL.
+ *   gamma, beta  device [hidden]; eps >= 0 is added to the variance.
+ *   out          device [B, n, hidden]; must not overlap h.
+ *   workspace    device, 256-byte aligned, lf_ffn_workspace_size bytes.
+ *   status       optional device int32 (see lf_qkv_projection).
+ * Every pointer must be 16-byte aligned.
+ */
+LF_API size_t lf_ffn_workspace_size(int B, int n, int hidden, int inter);
+LF_API int lf_ffn_block(lf_dtype dtype, int B, int n, int hidden, int inter, const void *h,
+                        const void *w1, const void *b1, const void *w2, const void *b2,
+                        const void *gamma, const void *beta, float eps, void *out,
+                        void *workspace, size_t workspace_bytes, int32_t *status,
+                        lf_stream_t stream);
+
+/*
+ * Device pointers of one encoder layer's weights (rows = output features,
+ * hid = H * d_head).  Biases may be NULL (zero).
+ */
+typedef struct lf_layer_weights {
+    const void *w_qkv;      /* [5*hid, hid]: Q, K, V, Kg, Vg stacked, as lf_qkv_projection */
+    const void *b_qkv;      /* [5*hid] */
+    const void *w_qg;       /* [hid, hid]: global queries; may be NULL when max_global = 0 */
+    const void *b_qg;       /* [hid] */
+    const void *w_o;        /* [hid, hid]: attention output projection */
+    const void *b_o;        /* [hid] */
+    const void *ln1_gamma;  /* [hid]: LayerNorm after the attention block */
+    const void *ln1_beta;   /* [hid] */
+    const void *w_1;        /* [inter, hid]: intermediate product */
+    const void *b_1;        /* [inter] */
+    const void *w_2;        /* [hid, inter]: feed-forward output product */
+    const void *b_2;        /* [hid] */
+    const void *ln2_gamma;  /* [hid]: LayerNorm after the feed-forward block */
+    const void *ln2_beta;   /* [hid] */
+} lf_layer_weights;
+
+/*
+ * A stack of Longformer encoder layers (FasterTransformer Longformer Encoder
+ * guide, "compute flow"; "LongFormer: The Long-Document Transformer" notes,
+ * "Sliding Window", for a window per layer).  Per layer: lf_qkv_projection,
+ * lf_attention_run (non-causal), lf_output_layer with the layer input as
+ * residual, lf_ffn_block.  The masks are prepared once (lf_attention_prepare)
+ * for all layers.
+ *
+ *   dtype        LF_BF16 or LF_F16.
+ *   inter        intermediate features of the feed-forward block (multiple of 64).
+ *   layers       >= 1.
+ *   weights      host [layers] of device pointers.
+ *   windows      host [layers]: window of each layer (even, >= 2).
+ *   dilations    host [layers * H] (layer-major) or NULL for all 1.
+ *   x            device [B, n, H*d_head]: the stack input.
+ *   local_mask, global_mask, max_global  as lf_attention_forward.
+ *   eps          of both LayerNorms.
+ *   out          device [B, n, H*d_head]: the last layer's output; must not
+ *                overlap x.
+ *   workspace    device, 256-byte aligned, lf_encoder_workspace_size bytes.
+ *                It begins with the attention workspace, so
+ *                lf_workspace_status(workspace) reads the one status word
+ *                every step of the stack records into.
+ * Errors in the arguments of any layer return before anything is launched.
+ */
+LF_API size_t lf_encoder_workspace_size(int B, int n, int H, int d_head, int inter,
+                                        int max_global);
+LF_API int lf_encoder_forward(lf_dtype dtype, int B, int n, int H, int d_head, int inter,
+                              int layers, const lf_layer_weights *weights,
+                              const int32_t *windows, const int32_t *dilations, const void *x,
+                              const uint8_t *local_mask, const uint8_t *global_mask,
+                              int max_global, float eps, void *out, void *workspace,
+                              size_t workspace_bytes, lf_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -46,6 +46,15 @@ def header_symbols() -> list[str]:
     return re.findall(r"^LF_API\s+[\w\s\*]+?\b(lf_\w+)\s*\(", text, flags=re.M)
 
 
+LAYER_FIELDS = ("w_qkv", "b_qkv", "w_qg", "b_qg", "w_o", "b_o", "ln1_gamma", "ln1_beta",
+                "w_1", "b_1", "w_2", "b_2", "ln2_gamma", "ln2_beta")
+
+
+class LayerWeights(ctypes.Structure):
+    """``lf_layer_weights``: device pointers of one encoder layer."""
+    _fields_ = [(f, ctypes.c_void_p) for f in LAYER_FIELDS]
+
+
 def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     sig = {
@@ -66,6 +75,11 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         "lf_qkv_projection": (I, [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, P, P, P, P, P]),
         "lf_output_workspace_size": (Z, [I, I, I, I]),
         "lf_output_layer": (I, [I, I, I, I, I, P, P, P, P, P, P, ctypes.c_float, P, P, Z, P, P]),
+        "lf_ffn_workspace_size": (Z, [I, I, I, I]),
+        "lf_ffn_block": (I, [I, I, I, I, I, P, P, P, P, P, P, P, ctypes.c_float, P, P, Z, P, P]),
+        "lf_encoder_workspace_size": (Z, [I, I, I, I, I, I]),
+        "lf_encoder_forward": (I, [I, I, I, I, I, I, I, ctypes.POINTER(LayerWeights), P, P, P, P,
+                                   P, I, ctypes.c_float, P, P, Z, P]),
         "lf_backward_scratch_size": (Z, [I, I, I, I, I]),
         "lf_attention_backward": (I, [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P, I, P, P, P,
                                       P, P, P, P, Z, P, Z, P]),

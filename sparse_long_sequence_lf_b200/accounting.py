@@ -99,3 +99,14 @@ def algorithmic_bytes(wl: Workload) -> int:
 
 def tokens(wl: Workload) -> int:
     return wl.B * wl.n
+
+
+def backward_flops(wl: Workload) -> int:
+    """FLOPs of one backward over the same pairs: five products of 2*d flops
+    per pair (the recomputed score, dP = dO.v, and the dq, dk, dv sums)."""
+    return 10 * wl.d * useful_pairs(wl)
+
+
+# CUDA-core fp32 peak of a B200: 148 SMs x 128 fp32 lanes x 2 flops (FMA)
+# per clock; multiplied by the SM clock in MHz it gives MFLOP/s.
+FP32_FLOPS_PER_CLOCK = 148 * 128 * 2

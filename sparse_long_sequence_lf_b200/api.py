@@ -293,3 +293,93 @@ def attention_backward(q, k, v, qg, kg, vg, out, dout, *, window, dilation=None,
         *[_ptr(grads[nm]) for nm in names], _ptr(workspace), workspace.numel(), _ptr(scratch),
         scratch.numel(), _stream_ptr(stream)), "lf_attention_backward")
     return grads
+
+
+def ffn_workspace_size(B: int, n: int, hidden: int, inter: int) -> int:
+    return int(_lib.lib().lf_ffn_workspace_size(B, n, hidden, inter))
+
+
+def ffn_block(h, w1, b1, w2, b2, gamma, beta, *, eps: float = 1e-5, out=None, workspace=None,
+              status=None, stream=None):
+    """``lf_ffn_block``: LayerNorm(GELU(h w1^T + b1) w2^T + b2 + h) with gamma,
+    beta; h [B, n, hidden] bf16 / fp16; returns out [B, n, hidden]."""
+    if h.dtype not in (torch.bfloat16, torch.float16) or h.dim() != 3:
+        raise ValueError("h must be a [B, n, hidden] bf16 or fp16 CUDA tensor")
+    B, n, hidden = h.shape
+    inter = w1.shape[0]
+    for t in (h, w1, b1, w2, b2, gamma, beta):
+        if t is not None and (not t.is_cuda or not t.is_contiguous() or t.dtype != h.dtype):
+            raise ValueError("all inputs must be contiguous CUDA tensors of h's dtype")
+    if tuple(w1.shape) != (inter, hidden) or tuple(w2.shape) != (hidden, inter):
+        raise ValueError("w1 must be [inter, hidden] and w2 [hidden, inter]")
+    if out is None:
+        out = torch.empty_like(h)
+    if workspace is None:
+        workspace = torch.empty(max(1, ffn_workspace_size(B, n, hidden, inter)),
+                                dtype=torch.uint8, device=h.device)
+    _lib.check(_lib.lib().lf_ffn_block(
+        _DTYPES[h.dtype], B, n, hidden, inter, _ptr(h), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2),
+        _ptr(gamma), _ptr(beta), float(eps), _ptr(out), _ptr(workspace), workspace.numel(),
+        _ptr(status), _stream_ptr(stream)), "lf_ffn_block")
+    return out
+
+
+def encoder_workspace_size(B: int, n: int, H: int, inter: int, max_global: int) -> int:
+    return int(_lib.lib().lf_encoder_workspace_size(B, n, H, D_HEAD, inter, max_global))
+
+
+def encoder_forward(x, layers, local_mask=None, global_mask=None, *, H: int, windows,
+                    dilations=None, max_global=None, eps: float = 1e-5, out=None,
+                    workspace=None, stream=None):
+    """``lf_encoder_forward``: a stack of Longformer encoder layers.
+
+    x [B, n, H*64] bf16 / fp16; layers: a list of dicts of CUDA tensors keyed
+    like ``lf_layer_weights`` (w_qkv, b_qkv, w_qg, b_qg, w_o, b_o, ln1_gamma,
+    ln1_beta, w_1, b_1, w_2, b_2, ln2_gamma, ln2_beta; biases and w_qg may be
+    missing or None); windows: one per layer; dilations: None or one list of H
+    values per layer.
+    """
+    if x.dtype not in (torch.bfloat16, torch.float16) or x.dim() != 3:
+        raise ValueError("x must be a [B, n, H*64] bf16 or fp16 CUDA tensor")
+    B, n, hid = x.shape
+    if hid != H * D_HEAD:
+        raise ValueError("x's last dimension must be H*64")
+    L = len(layers)
+    if len(windows) != L or (dilations is not None and len(dilations) != L):
+        raise ValueError("windows (and dilations) need one entry per layer")
+    inter = layers[0]["w_1"].shape[0]
+    arr = (_lib.LayerWeights * L)()
+    for i, lw in enumerate(layers):
+        for f in _lib.LAYER_FIELDS:
+            t = lw.get(f)
+            if t is not None:
+                if not t.is_cuda or not t.is_contiguous() or t.dtype != x.dtype:
+                    raise ValueError(f"layer {i} {f}: must be a contiguous CUDA tensor of "
+                                     "x's dtype")
+                setattr(arr[i], f, t.data_ptr())
+        if lw["w_1"].shape[0] != inter:
+            raise ValueError("all layers must share the intermediate size")
+    lm = _mask(local_mask, B, n, "local_mask")
+    gm = _mask(global_mask, B, n, "global_mask")
+    if max_global is None:
+        max_global = default_max_global(gm)
+    win = (ctypes.c_int32 * L)(*[int(w) for w in windows])
+    dil = None
+    if dilations is not None:
+        flat = []
+        for dl in dilations:
+            vals = [1] * H if dl is None else [int(v) for v in dl]
+            if len(vals) != H:
+                raise ValueError("each layer's dilation needs H entries")
+            flat += vals
+        dil = (ctypes.c_int32 * (L * H))(*flat)
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        workspace = torch.empty(max(1, encoder_workspace_size(B, n, H, inter, max_global)),
+                                dtype=torch.uint8, device=x.device)
+    _lib.check(_lib.lib().lf_encoder_forward(
+        _DTYPES[x.dtype], B, n, H, D_HEAD, inter, L, arr, win, dil, _ptr(x), _ptr(lm), _ptr(gm),
+        int(max_global), float(eps), _ptr(out), _ptr(workspace), workspace.numel(),
+        _stream_ptr(stream)), "lf_encoder_forward")
+    return out

@@ -23,6 +23,10 @@ int launch_output_layer(lf_dtype dtype, int B, int n, int H, const void *attn, c
                         const void *bo, const void *residual, const void *gamma,
                         const void *beta, float eps, void *out, float *sum, int32_t *status,
                         cudaStream_t stream);
+int launch_ffn(lf_dtype dtype, int B, int n, int hidden, int inter, const void *h,
+               const void *w1, const void *b1, const void *w2, const void *b2,
+               const void *gamma, const void *beta, float eps, void *out, void *act, float *sum,
+               int32_t *status, cudaStream_t stream);
 }  // namespace lf
 
 using namespace lf;
@@ -368,6 +372,38 @@ int lf_attention_backward(lf_dtype dtype, int B, int H, int n, int d_head, const
         case LF_BF16: return launch_backward<__nv_bfloat16>(A, 2, s);
     }
     return LF_ERR_INVALID_ARG;
+}
+
+size_t lf_ffn_workspace_size(int B, int n, int hidden, int inter)
+{
+    if (B < 1 || n < 1 || hidden < 64 || inter < 64 || hidden % 64 || inter % 64) return 0;
+    const size_t rows = size_t(B) * n;
+    return lf_align256(2 * rows * inter) + lf_align256(sizeof(float) * rows * hidden);
+}
+
+int lf_ffn_block(lf_dtype dtype, int B, int n, int hidden, int inter, const void *h,
+                 const void *w1, const void *b1, const void *w2, const void *b2,
+                 const void *gamma, const void *beta, float eps, void *out, void *workspace,
+                 size_t workspace_bytes, int32_t *status, lf_stream_t stream)
+{
+    if (dtype != LF_BF16 && dtype != LF_F16) return elem_size(dtype) ? LF_ERR_UNSUPPORTED
+                                                                   : LF_ERR_INVALID_ARG;
+    if (B < 1 || n < 1 || hidden < 64 || inter < 64) return LF_ERR_INVALID_ARG;
+    if (hidden % 64 || inter % 64) return LF_ERR_UNSUPPORTED;
+    if (double(B) * n * (inter > hidden ? inter : hidden) > 9.0e18 || double(B) * n >= 2.0e9)
+        return LF_ERR_INVALID_ARG;
+    if (!h || !w1 || !w2 || !gamma || !beta || !out) return LF_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || !std::isfinite(eps)) return LF_ERR_INVALID_ARG;
+    for (const void *ptr : {h, w1, b1, w2, b2, gamma, beta, static_cast<const void *>(out)})
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return LF_ERR_INVALID_ARG;
+    const size_t need = lf_ffn_workspace_size(B, n, hidden, inter);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+        return LF_ERR_WORKSPACE;
+    if (int rc = device_ok()) return rc;
+    char *base = static_cast<char *>(workspace);
+    float *sum = reinterpret_cast<float *>(base + lf_align256(2 * size_t(B) * n * inter));
+    return launch_ffn(dtype, B, n, hidden, inter, h, w1, b1, w2, b2, gamma, beta, eps, out, base,
+                      sum, status, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -49,7 +49,19 @@ constexpr int kSliceBytes = kTileM * kTileK * 2;   // 16 KB slice of A
 constexpr int kBSliceBytes = kTileN * kTileK * 2;  // 32 KB slice of W
 
 // One product C = A W^T + bias.
-enum JobMode { kModeHeads = 0, kModeGather = 1, kModeResidual = 2 };
+//   heads     A = X [M, K] row-major; C split into the [B, H, n, d] outputs
+//   gather    A = the gathered global rows of X; C into out[0] at those rows
+//   residual  A = the attention output [B, H, n, d] (one head per K slice);
+//             sum = C + bias + residual in fp32
+//   rows_res  A = [M, K] row-major; sum = C + bias + residual in fp32
+//   gelu      A = [M, K] row-major; out[0] [M, N] = GELU(C + bias)
+enum JobMode {
+    kModeHeads = 0, kModeGather = 1, kModeResidual = 2, kModeRowsResidual = 3, kModeGelu = 4
+};
+__host__ __device__ constexpr bool rows_a(int mode)
+{
+    return mode == kModeHeads || mode == kModeRowsResidual || mode == kModeGelu;
+}
 struct ProjJob {
     CUtensorMap a_map;       // heads: X as {K, M} tiles of 64 x 128; gather: X as
                              // {K, B*n} single rows; residual: the attention output
@@ -134,7 +146,7 @@ __device__ __forceinline__ int token_of(const ProjParams &p, const ProjJob &J, i
         const int i = m - b * per;
         return i < p.n ? i : -1;
     }
-    if (J.mode == kModeHeads) {
+    if (rows_a(J.mode)) {
         b = m / p.n;
         return m < J.M ? m - b * p.n : -1;
     }
@@ -227,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(const __grid_constant
                 if (!ok) break;
                 if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], a_bytes + kBSliceBytes);
                 __syncwarp();
-                if (J.mode == kModeHeads) {
+                if (rows_a(J.mode)) {
                     if (lane == 0) tma_load_2d(sm.a[s], &J.a_map, &sm.full[s], kt * kTileK, m0);
                 } else if (J.mode == kModeResidual) {
                     // K slice kt is head kt of the attention output: rows i0 ..
@@ -323,7 +335,28 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(const __grid_constant
 #pragma unroll
                     for (int x = 0; x < 32; ++x) bias[x] = 0.f;
                 }
-                if (J.mode == kModeResidual) {
+                if (J.mode == kModeGelu) {
+                    // GELU(x) = x * Phi(x), Phi written through erf.
+                    T *dst = static_cast<T *>(J.out[0]) + (size_t(b) * p.n + i) * J.N + o;
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float g[8];
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) {
+                            const float v = acc[8 * q + x] + bias[8 * q + x];
+                            g[x] = 0.5f * v * (1.f + erff(v * 0.70710678118654752f));
+                        }
+                        uint4 u;
+                        u.x = pack2<T>(g[0], g[1]);
+                        u.y = pack2<T>(g[2], g[3]);
+                        u.z = pack2<T>(g[4], g[5]);
+                        u.w = pack2<T>(g[6], g[7]);
+                        d4[q] = u;
+                    }
+                    continue;
+                }
+                if (J.mode == kModeResidual || J.mode == kModeRowsResidual) {
                     const size_t row = (size_t(b) * p.n + i) * J.N + o;
                     // 32 residual values as four 16-byte loads.
                     const uint4 *res4 = reinterpret_cast<const uint4 *>(
@@ -618,6 +651,65 @@ int launch_output_layer(lf_dtype dtype, int B, int n, int H, const void *attn, c
             sum, static_cast<const __half *>(gamma), static_cast<const __half *>(beta), eps, rows,
             hid, static_cast<__half *>(out));
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+}
+
+// C = A W^T (+ bias) over row-major A [M, K] in one persistent launch, with
+// the GELU-store or the residual-sum epilogue.  M = B * n tokens.
+int launch_rows_gemm(lf_dtype dtype, int mode, int B, int n, int K, int N, const void *a,
+                     const void *w, const void *bias, void *out, const void *residual,
+                     float *sum, int32_t *status, cudaStream_t stream)
+{
+    using namespace proj;
+    const CUtensorMapDataType dt =
+        dtype == LF_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    ProjParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.K = K;
+    p.B = B;
+    p.H = 1;
+    p.n = n;
+    p.status = status;
+    ProjJob &J = p.job[0];
+    J.mode = mode;
+    J.M = B * n;
+    J.N = N;
+    J.bias = bias;
+    J.out[0] = out;
+    J.residual = residual;
+    J.sum = sum;
+    if (!encode_matrix(&J.a_map, a, dt, long(B) * n, K, kTileM)) return kErrCuda;
+    if (!encode_matrix(&J.b_tile, w, dt, N, K, kTileN)) return kErrCuda;
+    p.mtiles0 = (J.M + kTileM - 1) / kTileM;
+    return dtype == LF_BF16 ? launch<__nv_bfloat16>(p, stream) : launch<__half>(p, stream);
+}
+
+template <typename T>
+static int layer_norm(const float *sum, const void *gamma, const void *beta, float eps, int rows,
+                      int N, void *out, cudaStream_t stream)
+{
+    proj::layernorm_kernel<T><<<(rows + 7) / 8, 256, 0, stream>>>(
+        sum, static_cast<const T *>(gamma), static_cast<const T *>(beta), eps, rows, N,
+        static_cast<T *>(out));
+    return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+}
+
+// Feed-forward block: act = GELU(h W1^T + b1) [B*n, inter]; sum = act W2^T +
+// b2 + h (fp32); out = LayerNorm(sum) with gamma, beta.
+int launch_ffn(lf_dtype dtype, int B, int n, int hidden, int inter, const void *h,
+               const void *w1, const void *b1, const void *w2, const void *b2,
+               const void *gamma, const void *beta, float eps, void *out, void *act, float *sum,
+               int32_t *status, cudaStream_t stream)
+{
+    using namespace proj;
+    int rc = launch_rows_gemm(dtype, kModeGelu, B, n, hidden, inter, h, w1, b1, act, nullptr,
+                              nullptr, status, stream);
+    if (rc != kOk) return rc;
+    rc = launch_rows_gemm(dtype, kModeRowsResidual, B, n, inter, hidden, act, w2, b2, nullptr, h,
+                          sum, status, stream);
+    if (rc != kOk) return rc;
+    return dtype == LF_BF16
+               ? layer_norm<__nv_bfloat16>(sum, gamma, beta, eps, B * n, hidden, out, stream)
+               : layer_norm<__half>(sum, gamma, beta, eps, B * n, hidden, out, stream);
 }
 
 }  // namespace lf

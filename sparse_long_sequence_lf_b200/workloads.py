@@ -213,3 +213,66 @@ def make_output_grad(wl: Workload, seed: int | None = None) -> torch.Tensor:
     gen = torch.Generator("cpu")
     gen.manual_seed((wl.seed if seed is None else seed) + 900007)
     return torch.randn((wl.B, wl.H, wl.n, wl.d), generator=gen).to(wl.torch_dtype)
+
+
+LAYER_FIELDS = ("w_qkv", "b_qkv", "w_qg", "b_qg", "w_o", "b_o", "ln1_gamma", "ln1_beta",
+                "w_1", "b_1", "w_2", "b_2", "ln2_gamma", "ln2_beta")
+
+
+def make_encoder_inputs(wl: Workload, layers: int, inter: int, seed: int | None = None):
+    """Random-init weights of an encoder stack for the workload's shape and
+    its input x [B, n, H*d] ~ N(0, 1): weight matrices ~ N(0, 1/fan_in),
+    biases and LayerNorm shifts ~ N(0, 0.1^2), LayerNorm scales ~ 1 + N(0, 0.1^2).
+    Returns (x, [dict per layer]) as CPU tensors of the workload dtype."""
+    gen = torch.Generator("cpu")
+    gen.manual_seed((wl.seed if seed is None else seed) + 1100009)
+    hid = wl.H * wl.d
+    dt = wl.torch_dtype
+    rn = lambda *shape: torch.randn(shape, generator=gen)
+    shapes = {"w_qkv": (5 * hid, hid), "b_qkv": (5 * hid,), "w_qg": (hid, hid), "b_qg": (hid,),
+              "w_o": (hid, hid), "b_o": (hid,), "ln1_gamma": (hid,), "ln1_beta": (hid,),
+              "w_1": (inter, hid), "b_1": (inter,), "w_2": (hid, inter), "b_2": (hid,),
+              "ln2_gamma": (hid,), "ln2_beta": (hid,)}
+    out = []
+    for _ in range(layers):
+        lw = {}
+        for f in LAYER_FIELDS:
+            t = rn(*shapes[f])
+            if f.startswith("w_"):
+                t = t / np.sqrt(shapes[f][1])
+            elif f.endswith("gamma"):
+                t = 1.0 + 0.1 * t
+            else:
+                t = 0.1 * t
+            lw[f] = t.to(dt)
+        out.append(lw)
+    x = rn(wl.B, wl.n, hid).to(dt)
+    return x, out
+
+
+@dataclass(frozen=True)
+class EncoderWorkload:
+    """A stack of encoder layers on the attention workload ``attn`` (its B, H,
+    n, window, globals and padding; every layer takes that window)."""
+    name: str
+    attn: Workload
+    inter: int
+    layers: int
+
+
+# The model of the encoder latency table in the FasterTransformer Longformer
+# Encoder guide ("performance benchmark": 16 heads of 64, intermediate 4096,
+# window 512, 24 layers), at batch 1 and 4096 tokens in fp16.  The guide's
+# inputs are random; the global tokens here follow its QA demo (the question
+# tokens, global, at the front): 64 of them.
+ENCODER_WORKLOADS = {
+    e.name: e for e in [
+        EncoderWorkload("fp16-b1h16-n4096-w512-i4096-l24",
+                        Workload("fp16-b1h16-n4096-w512-g64", "f16", 1, 16, 4096, 512,
+                                 globals_kind="first:64", seed=31), 4096, 24),
+        EncoderWorkload("fp16-b8h16-n4096-w512-i4096-l24",
+                        Workload("fp16-b8h16-n4096-w512-g64", "f16", 8, 16, 4096, 512,
+                                 globals_kind="first:64", seed=32), 4096, 24),
+    ]
+}
+ENCODER_HEADLINE = "fp16-b1h16-n4096-w512-i4096-l24"
