@@ -810,13 +810,24 @@ def run_backward_arm(args, wl, world, rank, local):
     ms_per_step = max_ms / steps
     value = whole_job_rate(flops, steps, world, max_ms) / 1e12
     tflops = flops / (ms_per_step * 1e-3) / 1e12
-    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965
-    peak = accounting.FP32_FLOPS_PER_CLOCK * mhz * 1e6 / 1e12
-    roofline = {"kernel": "bwd rows_kernel + keys_kernel (+ global rows / keys)",
-                "bound": "alu", "achieved": round(tflops, 2), "peak": round(peak, 1),
-                "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
-                "peak_source": f"derived: 148 SMs x 128 fp32 lanes x 2 flops x {mhz} MHz "
-                               "(median sampled SM clock)"}
+    if wl.dtype == "f32":
+        # fp32: the CUDA-core kernels, bound by the fp32 FMA rate.
+        mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965
+        peak = accounting.FP32_FLOPS_PER_CLOCK * mhz * 1e6 / 1e12
+        roofline = {"kernel": "bwd rows_kernel + keys_kernel (+ global-token kernels)",
+                    "bound": "alu", "achieved": round(tflops, 2), "peak": round(peak, 1),
+                    "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
+                    "peak_source": f"derived: 148 SMs x 128 fp32 lanes x 2 flops x {mhz} MHz "
+                                   "(median sampled SM clock)"}
+    else:
+        # bf16 / fp16: the tcgen05 band kernels (plus the CUDA-core global-token
+        # kernels), against the measured dense tensor peak.
+        peaks, peak_kind = load_peaks()
+        roofline = {"kernel": "bwd_tc_kernel rows + keys sides (+ global-token kernels)",
+                    "bound": "tensor", "achieved": round(tflops, 2),
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": round(tflops / peaks["bf16_tflops"], 4), "traffic": None,
+                    "peak_source": peak_kind + " (bf16 dense; fp16 has the same nominal rate)"}
 
     # End to end through the host-buffer path: the eight inputs from pinned
     # host memory in, the six gradients back.
@@ -874,7 +885,9 @@ def run_backward_arm(args, wl, world, rank, local):
                "sample": f"batch 0, head 0, first {sub.n} tokens, {reps_} repetition(s), "
                          f"{dt:.1f} s, fp64 dense-mask autograd oracle (torch CPU threads)",
                "seconds": round(dt, 2)}
-    launches = 4 if mg > 0 else 2
+    # rows + keys sides; with global tokens gcols, two global-row passes,
+    # gfinal and gkeys
+    launches = 7 if mg > 0 else 2
     result = {
         "metric": BWD_METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),

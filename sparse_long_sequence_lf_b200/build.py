@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(BUILD, "liblf_attention.so")
 SOURCES = ["lf_api.cu", "lf_prepare.cu", "lf_simt.cu", "lf_tc.cu", "lf_static.cu", "lf_proj.cu",
-           "lf_bwd.cu", "lf_encoder.cu"]
+           "lf_bwd.cu", "lf_bwd_tc.cu", "lf_encoder.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -335,8 +335,7 @@ int lf_output_layer(lf_dtype dtype, int B, int n, int H, int d_head, const void 
 size_t lf_backward_scratch_size(int B, int H, int n, int d_head, int max_global)
 {
     if (!sizes_ok(B, H, n) || d_head != kDHead || max_global < 0 || max_global > n) return 0;
-    return lf_align256(2 * sizeof(float) * size_t(B) * H * n) +
-           lf_align256(2 * sizeof(float) * size_t(B) * H * (max_global > 0 ? max_global : 1));
+    return backward_scratch_bytes(B, H, n, max_global);
 }
 
 int lf_attention_backward(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
@@ -359,17 +358,17 @@ int lf_attention_backward(lf_dtype dtype, int B, int H, int n, int d_head, const
     A.out = out;
     A.dout = dout;
     A.dq = dq; A.dk = dk; A.dv = dv; A.dqg = dqg; A.dkg = dkg; A.dvg = dvg;
-    const size_t rows = size_t(B) * H * n;
-    char *base = static_cast<char *>(scratch);
-    A.lse = reinterpret_cast<float *>(base);
-    A.dsum = A.lse + rows;
-    A.lse_g = reinterpret_cast<float *>(base + lf_align256(2 * sizeof(float) * rows));
-    A.dsum_g = A.lse_g + size_t(B) * H * (max_global > 0 ? max_global : 1);
+    backward_scratch_ptrs(A, scratch, B, H, n, max_global);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (dtype) {
-        case LF_F32: return launch_backward<float>(A, 4, s);
-        case LF_F16: return launch_backward<__half>(A, 2, s);
-        case LF_BF16: return launch_backward<__nv_bfloat16>(A, 2, s);
+        case LF_F32: return launch_backward_simt<float>(A, 4, s);
+        case LF_F16:
+        case LF_BF16: {
+            const int rc = launch_backward_tc(dtype, A, s);
+            if (rc != kErrUnsupported) return rc;
+            return dtype == LF_F16 ? launch_backward_simt<__half>(A, 2, s)
+                                   : launch_backward_simt<__nv_bfloat16>(A, 2, s);
+        }
     }
     return LF_ERR_INVALID_ARG;
 }

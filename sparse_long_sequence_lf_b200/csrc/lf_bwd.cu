@@ -233,6 +233,32 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(const BwdArgs A)
     }
 }
 
+// Slot of global token j in the batch's ascending global index (binary search).
+__device__ __forceinline__ int global_slot(const AttnArgs &a, int b, int j)
+{
+    const int *gl = a.ws.gidx + size_t(b) * a.n;
+    int lo = 0, hi = min(a.ws.counts[b], a.max_global) - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (gl[mid] < j) lo = mid + 1; else hi = mid;
+    }
+    return (hi >= 0 && gl[lo] == j) ? lo : -1;
+}
+
+// Adds the non-window contributions to global key j (this thread's quarter).
+__device__ __forceinline__ void add_global_key_sums(const BwdArgs &A, int b, size_t bh, int j,
+                                                    int qd, float (&dk)[kQ], float (&dv)[kQ])
+{
+    const int slot = global_slot(A.a, b, j);
+    if (slot < 0) return;
+    const float *src = A.gkv + (bh * A.a.max_global + slot) * (2 * kDHead);
+#pragma unroll
+    for (int x = 0; x < kQ; ++x) {
+        dk[x] += src[kQ * qd + x];
+        dv[x] += src[kDHead + kQ * qd + x];
+    }
+}
+
 // ------------------------------------------------------------------ keys
 template <typename T>
 __global__ void __launch_bounds__(kThreads) keys_kernel(const BwdArgs A)
@@ -242,7 +268,6 @@ __global__ void __launch_bounds__(kThreads) keys_kernel(const BwdArgs A)
     __shared__ __align__(16) float ds[kTile][kDHead];
     __shared__ float lse_s[kTile], d_s[kTile];
     __shared__ int rpos[kTile];
-    __shared__ int any_global;
 
     int b, h, r, tile;
     band_item(a, blockIdx.x / kParts, b, h, r, tile);
@@ -276,9 +301,6 @@ __global__ void __launch_bounds__(kThreads) keys_kernel(const BwdArgs A)
     }
 #pragma unroll
     for (int x = 0; x < kQ; ++x) dk[x] = dv[x] = 0.f;
-    if (tid == 0) any_global = 0;
-    __syncthreads();
-    if (kglobal && qd == 0) atomicOr(&any_global, 1);
 
     // Stage rows at positions pos (band or any), then accumulate.
     auto stage = [&](const int (&pos)[4]) {
@@ -327,28 +349,9 @@ __global__ void __launch_bounds__(kThreads) keys_kernel(const BwdArgs A)
             axpy_quarter(dk, p * (sd.y - d_s[c]), qs[c], qd);
         }
     }
-    // A global token is a key of every valid non-global row of the head; the
-    // rows already counted as window taps are skipped.
-    __syncthreads();
-    if (any_global) {
-        for (int t0 = 0; t0 < n; t0 += kTile) {
-            int pos[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = t0 + (tid >> 4) + 8 * u;
-                pos[u] = i < n ? i : -1;
-            }
-            stage(pos);
-            for (int c = 0; c < kTile; ++c) {
-                const float2 sd = accumulate(c);
-                const int i = rpos[c];
-                if (!kglobal || i < 0 || is_tap(i, j, a.window, a.half, dil, a.causal)) continue;
-                const float p = exp2f(sd.x - lse_s[c]);
-                axpy_quarter(dv, p, ds[c], qd);
-                axpy_quarter(dk, p * (sd.y - d_s[c]), qs[c], qd);
-            }
-        }
-    }
+    // A global token is also a key of every other valid non-global row of the
+    // head: those sums come from gcols_kernel.
+    if (kglobal) add_global_key_sums(A, b, bh, j, qd, dk, dv);
 
     if (!key_in) return;
     const float inv_sqrt_d = a.scale_log2 * 0.69314718055994531f;
@@ -356,95 +359,228 @@ __global__ void __launch_bounds__(kThreads) keys_kernel(const BwdArgs A)
     store_quarter(static_cast<T *>(A.dv) + keyoff, dv, qd, 1.f);
 }
 
-// ------------------------------------------------------------ global rows
+// ------------------------------------------------- global tokens as keys
+// Contributions of the rows that reach a global token only as a global key
+// (valid non-global rows that are not its window taps): one CTA per
+// (batch*head, 32 global slots, kGChunk rows), fp32 sums added atomically to
+// A.gkv.  Needs the rows' lse and D.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) grows_kernel(const BwdArgs A)
+__global__ void __launch_bounds__(kThreads) gcols_kernel(const BwdArgs A)
+{
+    const AttnArgs &a = A.a;
+    __shared__ __align__(16) float qs[kTile][kDHead];
+    __shared__ __align__(16) float ds[kTile][kDHead];
+    __shared__ float lse_s[kTile], d_s[kTile];
+    __shared__ int rpos[kTile];
+
+    const int n = a.n;
+    const int sparts = (a.max_global + kRows - 1) / kRows;
+    const int rchunks = (n + kGChunk - 1) / kGChunk;
+    const int bh = blockIdx.x / (sparts * rchunks);
+    const int rem = blockIdx.x - bh * sparts * rchunks;
+    const int s0 = (rem / rchunks) * kRows;
+    const int i0 = (rem % rchunks) * kGChunk;
+    const int b = bh / a.H, h = bh - b * a.H;
+    const int g = min(a.ws.counts[b], a.max_global);
+    if (s0 >= g) return;
+    const int tid = threadIdx.x, rl = tid >> 2, qd = tid & 3;
+    const int slot = s0 + rl;
+    const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
+    const uint32_t *gb = a.ws.gbits + size_t(b) * a.L.nwords;
+    const int j = slot < g ? a.ws.gidx[size_t(b) * n + slot] : -1;
+    const bool kvalid = j >= 0 && bit_at(vb, j);
+    const int dil = a.dil[h];
+    const size_t keyoff = (size_t(bh) * n + (kvalid ? j : 0)) * kDHead;
+    const T *Q = static_cast<const T *>(a.q) + size_t(bh) * n * kDHead;
+    const T *dO = static_cast<const T *>(A.dout) + size_t(bh) * n * kDHead;
+    const float *lse = A.lse + size_t(bh) * n;
+    const float *dsum = A.dsum + size_t(bh) * n;
+
+    float k[kQ], v[kQ], dk[kQ], dv[kQ];
+    if (kvalid) {
+        load_quarter(k, static_cast<const T *>(a.k) + keyoff, qd, a.scale_log2);
+        load_quarter(v, static_cast<const T *>(a.v) + keyoff, qd, 1.f);
+    } else {
+#pragma unroll
+        for (int x = 0; x < kQ; ++x) k[x] = v[x] = 0.f;
+    }
+#pragma unroll
+    for (int x = 0; x < kQ; ++x) dk[x] = dv[x] = 0.f;
+
+    for (int t0 = i0; t0 < min(i0 + kGChunk, n); t0 += kTile) {
+        __syncthreads();
+        int pos[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = (tid >> 4) + 8 * u;
+            const int i = t0 + c;
+            const bool act = i < n && bit_at(vb, i) && !bit_at(gb, i);
+            pos[u] = act ? i : -1;
+            if ((tid & 15) == 0) {
+                rpos[c] = act ? i : -1;
+                lse_s[c] = act ? lse[i] : INFINITY;
+                d_s[c] = act ? dsum[i] : 0.f;
+            }
+        }
+        stage_rows(qs, Q, pos, tid);
+        stage_rows(ds, dO, pos, tid);
+        __syncthreads();
+        for (int c = 0; c < kTile; ++c) {
+            const float sc = dot_quarter(k, qs[c], qd);
+            const float dp = dot_quarter(v, ds[c], qd);
+            const int i = rpos[c];
+            if (!kvalid || i < 0 || is_tap(i, j, a.window, a.half, dil, a.causal)) continue;
+            const float pr = exp2f(sc - lse_s[c]);
+            axpy_quarter(dv, pr, ds[c], qd);
+            axpy_quarter(dk, pr * (dp - d_s[c]), qs[c], qd);
+        }
+    }
+    if (!kvalid) return;
+    float *dst = A.gkv + (size_t(bh) * a.max_global + slot) * (2 * kDHead);
+#pragma unroll
+    for (int x = 0; x < kQ; ++x) {
+        atomicAdd(dst + kQ * qd + x, dk[x]);
+        atomicAdd(dst + kDHead + kQ * qd + x, dv[x]);
+    }
+}
+
+// ------------------------------------------------------------ global rows
+// Global rows against every valid key through Qg, Kg, Vg, split into chunks
+// of kGChunk keys: gstats_kernel writes each chunk's (max, sum) of the row's
+// scores; ggrad_kernel merges them into the row's log-sum-exp, then sums the
+// chunk's dqg terms into A.dqg_acc; gfinal_kernel scales and stores dqg.
+// One CTA per (batch*head, 32 global slots, chunk).
+template <typename T, bool kGrad>
+__global__ void __launch_bounds__(kThreads) grows_chunk_kernel(const BwdArgs A)
 {
     const AttnArgs &a = A.a;
     __shared__ __align__(16) float ks[kTile][kDHead];
     __shared__ __align__(16) float vs[kTile][kDHead];
     __shared__ int kok[kTile];
 
-    // One CTA per (batch*head, 32 global slots), flattened.
-    const int gparts = (a.max_global + kRows - 1) / kRows;
-    const int bh = blockIdx.x / gparts;
-    const int s0 = (blockIdx.x % gparts) * kRows;
-    const int b = bh / a.H;
     const int n = a.n;
-    const int tid = threadIdx.x, rl = tid >> 2, qd = tid & 3;
+    const int sparts = (a.max_global + kRows - 1) / kRows;
+    const int nch = A.nchg;
+    const int bh = blockIdx.x / (sparts * nch);
+    const int rem = blockIdx.x - bh * sparts * nch;
+    const int s0 = (rem / nch) * kRows;
+    const int chunk = rem % nch;
+    const int b = bh / a.H;
     const int g = min(a.ws.counts[b], a.max_global);
-    const int slot = s0 + rl;
     if (s0 >= g) return;
+    const int tid = threadIdx.x, rl = tid >> 2, qd = tid & 3;
+    const int slot = s0 + rl;
     const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
     const int i = slot < g ? a.ws.gidx[size_t(b) * n + slot] : -1;
     const bool active = i >= 0 && bit_at(vb, i);
     const size_t rowoff = (size_t(bh) * n + (active ? i : 0)) * kDHead;
     const T *Kg = static_cast<const T *>(a.kg) + size_t(bh) * n * kDHead;
     const T *Vg = static_cast<const T *>(a.vg) + size_t(bh) * n * kDHead;
+    const size_t mg = size_t(a.max_global);
+    float2 *part = A.gpart + size_t(bh) * nch * mg;
 
     float q[kQ], dO[kQ], dq[kQ];
-    float D = 0.f;
-    {
+    float D = 0.f, lse = INFINITY;
+    if (active) {
+        load_quarter(q, static_cast<const T *>(a.qg) + rowoff, qd, a.scale_log2);
+    } else {
+#pragma unroll
+        for (int x = 0; x < kQ; ++x) q[x] = 0.f;
+    }
+    if (kGrad) {
         float o[kQ];
         if (active) {
-            load_quarter(q, static_cast<const T *>(a.qg) + rowoff, qd, a.scale_log2);
             load_quarter(dO, static_cast<const T *>(A.dout) + rowoff, qd, 1.f);
             load_quarter(o, static_cast<const T *>(A.out) + rowoff, qd, 1.f);
         } else {
 #pragma unroll
-            for (int x = 0; x < kQ; ++x) q[x] = dO[x] = o[x] = 0.f;
+            for (int x = 0; x < kQ; ++x) dO[x] = o[x] = 0.f;
         }
         float d = 0.f;
 #pragma unroll
         for (int x = 0; x < kQ; ++x) d = fmaf(dO[x], o[x], d);
         D = quad_sum(d);
+        // Merge the chunks' (max, sum) into the row's log-sum-exp.
+        if (active) {
+            float M = -INFINITY;
+            for (int c = 0; c < nch; ++c) M = fmaxf(M, part[c * mg + slot].x);
+            float L = 0.f;
+            for (int c = 0; c < nch; ++c) {
+                const float2 ml = part[c * mg + slot];
+                if (ml.x != -INFINITY) L += ml.y * exp2f(ml.x - M);
+            }
+            lse = L > 0.f ? M + log2f(L) : INFINITY;
+        }
 #pragma unroll
         for (int x = 0; x < kQ; ++x) dq[x] = 0.f;
     }
-    auto stage = [&](int t0, bool with_v) {
+
+    float m = -INFINITY, l = 0.f;
+    const int kend = min(n, (chunk + 1) * kGChunk);
+    for (int t0 = chunk * kGChunk; t0 < kend; t0 += kTile) {
         __syncthreads();
         int pos[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int c = (tid >> 4) + 8 * u;
             const int jj = t0 + c;
-            pos[u] = jj < n ? jj : -1;
-            if ((tid & 15) == 0) kok[c] = jj < n && bit_at(vb, jj);
+            pos[u] = jj < kend ? jj : -1;
+            if ((tid & 15) == 0) kok[c] = jj < kend && bit_at(vb, jj);
         }
         stage_rows(ks, Kg, pos, tid);
-        if (with_v) stage_rows(vs, Vg, pos, tid);
+        if (kGrad) stage_rows(vs, Vg, pos, tid);
         __syncthreads();
-    };
-    float m = -INFINITY, l = 0.f;
-    for (int t0 = 0; t0 < n; t0 += kTile) {
-        stage(t0, false);
         for (int c = 0; c < kTile; ++c) {
-            const float s = dot_quarter(q, ks[c], qd);
-            if (!active || !kok[c]) continue;
-            const float mn = fmaxf(m, s);
-            l = l * exp2f(m - mn) + exp2f(s - mn);
-            m = mn;
-        }
-    }
-    const float lse = l > 0.f ? m + log2f(l) : INFINITY;
-    for (int t0 = 0; t0 < n; t0 += kTile) {
-        stage(t0, true);
-        for (int c = 0; c < kTile; ++c) {
-            const float s = dot_quarter(q, ks[c], qd);
-            const float dp = dot_quarter(dO, vs[c], qd);
-            if (!active || !kok[c]) continue;
-            const float p = exp2f(s - lse);
-            axpy_quarter(dq, p * (dp - D), ks[c], qd);
+            const float sc = dot_quarter(q, ks[c], qd);
+            if (kGrad) {
+                const float dp = dot_quarter(dO, vs[c], qd);
+                if (!active || !kok[c]) continue;
+                const float pr = exp2f(sc - lse);
+                axpy_quarter(dq, pr * (dp - D), ks[c], qd);
+            } else {
+                if (!active || !kok[c]) continue;
+                const float mn = fmaxf(m, sc);
+                l = l * exp2f(m - mn) + exp2f(sc - mn);
+                m = mn;
+            }
         }
     }
     if (slot >= g) return;
-    if (qd == 0) {
-        A.lse_g[size_t(bh) * a.max_global + slot] = active ? lse : INFINITY;
-        A.dsum_g[size_t(bh) * a.max_global + slot] = D;
+    if (!kGrad) {
+        if (qd == 0) part[size_t(chunk) * mg + slot] = make_float2(m, l);
+        return;
+    }
+    if (chunk == 0 && qd == 0) {
+        A.lse_g[size_t(bh) * mg + slot] = lse;
+        A.dsum_g[size_t(bh) * mg + slot] = D;
     }
     if (!active) return;
-    const float inv_sqrt_d = a.scale_log2 * 0.69314718055994531f;
-    store_quarter(static_cast<T *>(A.dqg) + rowoff, dq, qd, inv_sqrt_d);
+    float *dst = A.dqg_acc + (size_t(bh) * mg + slot) * kDHead + kQ * qd;
+#pragma unroll
+    for (int x = 0; x < kQ; ++x) atomicAdd(dst + x, dq[x]);
+}
+
+// dqg of each valid global row: the fp32 sums scaled by 1/sqrt(d), in T.
+// One thread per (batch*head, slot, 4 dimensions).
+template <typename T>
+__global__ void __launch_bounds__(256) gfinal_kernel(const BwdArgs A)
+{
+    const AttnArgs &a = A.a;
+    const size_t t = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    const size_t mg = size_t(a.max_global);
+    if (t >= size_t(a.B) * a.H * mg * (kDHead / 4)) return;
+    const int x4 = int(t % (kDHead / 4)) * 4;
+    const size_t rs = t / (kDHead / 4);
+    const int slot = int(rs % mg);
+    const int bh = int(rs / mg);
+    const int b = bh / a.H;
+    if (slot >= min(a.ws.counts[b], a.max_global)) return;
+    const int i = a.ws.gidx[size_t(b) * a.n + slot];
+    if (!bit_at(a.ws.vbits + size_t(b) * a.L.nwords, i)) return;
+    const float s = a.scale_log2 * 0.69314718055994531f;
+    const float4 v = *reinterpret_cast<const float4 *>(A.dqg_acc + rs * kDHead + x4);
+    store4(static_cast<T *>(A.dqg) + (size_t(bh) * a.n + i) * kDHead + x4,
+           make_float4(v.x * s, v.y * s, v.z * s, v.w * s));
 }
 
 // ------------------------------------------------------------ global keys
@@ -520,8 +656,36 @@ __global__ void __launch_bounds__(kThreads) gkeys_kernel(const BwdArgs A)
 
 }  // namespace bwd
 
+// Launches of the global-token parts, shared by both band paths: they run
+// after the band rows (which write lse and D of the local rows).
 template <typename T>
-int launch_backward(const BwdArgs &A, size_t elem, cudaStream_t stream)
+int launch_global_parts(const BwdArgs &A, size_t elem, cudaStream_t stream)
+{
+    using namespace bwd;
+    const AttnArgs &a = A.a;
+    const size_t bytes = size_t(a.B) * a.H * a.n * kDHead * elem;
+    if (a.max_global == 0) {
+        if (cudaMemsetAsync(A.dkg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
+        if (cudaMemsetAsync(A.dvg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
+        return kOk;
+    }
+    const int bh = a.B * a.H;
+    const int sparts = (a.max_global + kRows - 1) / kRows;
+    const size_t mg = size_t(a.max_global);
+    if (cudaMemsetAsync(A.gkv, 0, sizeof(float) * bh * mg * 2 * kDHead, stream) != cudaSuccess ||
+        cudaMemsetAsync(A.dqg_acc, 0, sizeof(float) * bh * mg * kDHead, stream) != cudaSuccess)
+        return kErrCuda;
+    gcols_kernel<T><<<bh * sparts * ((a.n + kGChunk - 1) / kGChunk), kThreads, 0, stream>>>(A);
+    grows_chunk_kernel<T, false><<<bh * sparts * A.nchg, kThreads, 0, stream>>>(A);
+    grows_chunk_kernel<T, true><<<bh * sparts * A.nchg, kThreads, 0, stream>>>(A);
+    const size_t nfin = size_t(bh) * mg * (kDHead / 4);
+    gfinal_kernel<T><<<unsigned((nfin + 255) / 256), 256, 0, stream>>>(A);
+    gkeys_kernel<T><<<bh * ((a.n + kRows - 1) / kRows), kThreads, 0, stream>>>(A);
+    return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+}
+
+template <typename T>
+int launch_backward_simt(const BwdArgs &A, size_t elem, cudaStream_t stream)
 {
     using namespace bwd;
     const AttnArgs &a = A.a;
@@ -529,23 +693,17 @@ int launch_backward(const BwdArgs &A, size_t elem, cudaStream_t stream)
     // Qg gets gradient rows only at global positions.
     if (cudaMemsetAsync(A.dqg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
     const int band_ctas = a.B * a.band_items_per_batch * kParts;
-    if (band_ctas > 0) {
-        rows_kernel<T><<<band_ctas, kThreads, 0, stream>>>(A);
-        keys_kernel<T><<<band_ctas, kThreads, 0, stream>>>(A);
-    }
-    if (a.max_global > 0) {
-        const int bh = a.B * a.H;
-        grows_kernel<T><<<bh * ((a.max_global + kRows - 1) / kRows), kThreads, 0, stream>>>(A);
-        gkeys_kernel<T><<<bh * ((a.n + kRows - 1) / kRows), kThreads, 0, stream>>>(A);
-    } else {
-        if (cudaMemsetAsync(A.dkg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
-        if (cudaMemsetAsync(A.dvg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
-    }
+    if (band_ctas > 0) rows_kernel<T><<<band_ctas, kThreads, 0, stream>>>(A);
+    // The keys kernel adds the global-key sums of gcols_kernel.
+    if (int rc = launch_global_parts<T>(A, elem, stream)) return rc;
+    if (band_ctas > 0) keys_kernel<T><<<band_ctas, kThreads, 0, stream>>>(A);
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 
-template int launch_backward<float>(const BwdArgs &, size_t, cudaStream_t);
-template int launch_backward<__half>(const BwdArgs &, size_t, cudaStream_t);
-template int launch_backward<__nv_bfloat16>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_global_parts<__half>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_global_parts<__nv_bfloat16>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_backward_simt<float>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_backward_simt<__half>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_backward_simt<__nv_bfloat16>(const BwdArgs &, size_t, cudaStream_t);
 
 }  // namespace lf

@@ -1,6 +1,7 @@
 // Arguments of the attention backward kernels (lf_bwd.cu).
 #pragma once
 
+#include "../../include/lf_attention.h"
 #include "lf_device.cuh"
 
 namespace lf {
@@ -11,8 +12,56 @@ struct BwdArgs {
     void *dq, *dk, *dv, *dqg, *dkg, *dvg;
     float *lse, *dsum;          // [B*H*n] per band row: log2-domain lse, D
     float *lse_g, *dsum_g;      // [B*H*max_global] per global slot
+    // Global tokens as keys of the rows that do not reach them through the
+    // window: [B*H*max_global][dk (64, unscaled) | dv (64)] fp32 sums.
+    float *gkv;
+    // Global rows: (max, sum) per chunk of kGChunk keys
+    // [B*H][nchg][max_global] and the fp32 dqg sums [B*H*max_global][64].
+    float2 *gpart;
+    float *dqg_acc;
+    int nchg;
 };
 
-template <typename T> int launch_backward(const BwdArgs &A, size_t elem, cudaStream_t stream);
+constexpr int kGChunk = 128;    // keys per partial of a global row; rows per
+                                // chunk of the global-key column pass
+
+// Bytes of the caller scratch of the backward.
+inline size_t backward_scratch_bytes(int B, int H, int n, int max_global)
+{
+    const size_t bh = size_t(B) * H, mg = max_global > 0 ? max_global : 1;
+    const size_t nchg = (size_t(n) + kGChunk - 1) / kGChunk;
+    return lf_align256(2 * sizeof(float) * bh * n) + lf_align256(2 * sizeof(float) * bh * mg) +
+           lf_align256(sizeof(float) * bh * mg * 2 * kDHead) +
+           lf_align256(sizeof(float2) * bh * nchg * mg) +
+           lf_align256(sizeof(float) * bh * mg * kDHead);
+}
+
+// Carves the scratch (256-byte aligned) into the pointers above.
+inline void backward_scratch_ptrs(BwdArgs &A, void *scratch, int B, int H, int n, int max_global)
+{
+    const size_t bh = size_t(B) * H, mg = max_global > 0 ? max_global : 1;
+    const size_t nchg = (size_t(n) + kGChunk - 1) / kGChunk;
+    char *p = static_cast<char *>(scratch);
+    A.lse = reinterpret_cast<float *>(p);
+    A.dsum = A.lse + bh * n;
+    p += lf_align256(2 * sizeof(float) * bh * n);
+    A.lse_g = reinterpret_cast<float *>(p);
+    A.dsum_g = A.lse_g + bh * mg;
+    p += lf_align256(2 * sizeof(float) * bh * mg);
+    A.gkv = reinterpret_cast<float *>(p);
+    p += lf_align256(sizeof(float) * bh * mg * 2 * kDHead);
+    A.gpart = reinterpret_cast<float2 *>(p);
+    p += lf_align256(sizeof(float2) * bh * nchg * mg);
+    A.dqg_acc = reinterpret_cast<float *>(p);
+    A.nchg = int(nchg);
+}
+
+// CUDA-core path: every dtype, any dilations.
+template <typename T> int launch_backward_simt(const BwdArgs &A, size_t elem, cudaStream_t stream);
+// Global-token parts (after the band rows, before the band keys).
+template <typename T> int launch_global_parts(const BwdArgs &A, size_t elem, cudaStream_t stream);
+// Tensor-core path for bf16 / fp16; kErrUnsupported (nothing launched) when
+// the heads' residue classes exceed its tensor-map budget.
+int launch_backward_tc(lf_dtype dtype, const BwdArgs &A, cudaStream_t stream);
 
 }  // namespace lf
