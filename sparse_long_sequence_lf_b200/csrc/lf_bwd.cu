@@ -359,6 +359,23 @@ __global__ void __launch_bounds__(kThreads) keys_kernel(const BwdArgs A)
     store_quarter(static_cast<T *>(A.dv) + keyoff, dv, qd, 1.f);
 }
 
+// Few global tokens leave most thread quads of a CTA without a slot: the CTA's
+// gv valid slots (1..32) take G2 = the next power of two quads each, and the
+// 32 / G2 groups of quads share out the streamed rows or keys of each tile.
+struct SlotGroups {
+    int G2, R, sl, grp;
+};
+__device__ __forceinline__ SlotGroups slot_groups(int gv, int rl)
+{
+    SlotGroups q;
+    q.G2 = 1;
+    while (q.G2 < gv) q.G2 <<= 1;
+    q.R = kRows / q.G2;
+    q.sl = rl & (q.G2 - 1);
+    q.grp = rl / q.G2;
+    return q;
+}
+
 // ------------------------------------------------- global tokens as keys
 // Contributions of the rows that reach a global token only as a global key
 // (valid non-global rows that are not its window taps): one CTA per
@@ -372,6 +389,7 @@ __global__ void __launch_bounds__(kThreads) gcols_kernel(const BwdArgs A)
     __shared__ __align__(16) float ds[kTile][kDHead];
     __shared__ float lse_s[kTile], d_s[kTile];
     __shared__ int rpos[kTile];
+    __shared__ __align__(16) float red[kRows][2 * kDHead];
 
     const int n = a.n;
     const int sparts = (a.max_global + kRows - 1) / kRows;
@@ -384,10 +402,13 @@ __global__ void __launch_bounds__(kThreads) gcols_kernel(const BwdArgs A)
     const int g = min(a.ws.counts[b], a.max_global);
     if (s0 >= g) return;
     const int tid = threadIdx.x, rl = tid >> 2, qd = tid & 3;
-    const int slot = s0 + rl;
+    const int gv = min(g - s0, kRows);
+    const SlotGroups sg = slot_groups(gv, rl);
+    const int slot = s0 + sg.sl;
     const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
     const uint32_t *gb = a.ws.gbits + size_t(b) * a.L.nwords;
-    const int j = slot < g ? a.ws.gidx[size_t(b) * n + slot] : -1;
+    const int j = sg.sl < gv ? a.ws.gidx[size_t(b) * n + slot] : -1;
+    for (int e = tid; e < kRows * 2 * kDHead; e += kThreads) (&red[0][0])[e] = 0.f;
     const bool kvalid = j >= 0 && bit_at(vb, j);
     const int dil = a.dil[h];
     const size_t keyoff = (size_t(bh) * n + (kvalid ? j : 0)) * kDHead;
@@ -425,7 +446,8 @@ __global__ void __launch_bounds__(kThreads) gcols_kernel(const BwdArgs A)
         stage_rows(qs, Q, pos, tid);
         stage_rows(ds, dO, pos, tid);
         __syncthreads();
-        for (int c = 0; c < kTile; ++c) {
+#pragma unroll 2
+        for (int c = sg.grp; c < kTile; c += sg.R) {
             const float sc = dot_quarter(k, qs[c], qd);
             const float dp = dot_quarter(v, ds[c], qd);
             const int i = rpos[c];
@@ -435,12 +457,19 @@ __global__ void __launch_bounds__(kThreads) gcols_kernel(const BwdArgs A)
             axpy_quarter(dk, pr * (dp - d_s[c]), qs[c], qd);
         }
     }
-    if (!kvalid) return;
-    float *dst = A.gkv + (size_t(bh) * a.max_global + slot) * (2 * kDHead);
+    // Groups of the same slot meet in shared memory; one global add per value.
+    if (kvalid) {
 #pragma unroll
-    for (int x = 0; x < kQ; ++x) {
-        atomicAdd(dst + kQ * qd + x, dk[x]);
-        atomicAdd(dst + kDHead + kQ * qd + x, dv[x]);
+        for (int x = 0; x < kQ; ++x) {
+            atomicAdd(&red[sg.sl][kQ * qd + x], dk[x]);
+            atomicAdd(&red[sg.sl][kDHead + kQ * qd + x], dv[x]);
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < gv * 2 * kDHead; e += kThreads) {
+        const int s_ = e / (2 * kDHead), x = e - s_ * (2 * kDHead);
+        if (!bit_at(vb, a.ws.gidx[size_t(b) * n + s0 + s_])) continue;
+        atomicAdd(A.gkv + (size_t(bh) * a.max_global + s0 + s_) * (2 * kDHead) + x, red[s_][x]);
     }
 }
 
@@ -457,6 +486,8 @@ __global__ void __launch_bounds__(kThreads) grows_chunk_kernel(const BwdArgs A)
     __shared__ __align__(16) float ks[kTile][kDHead];
     __shared__ __align__(16) float vs[kTile][kDHead];
     __shared__ int kok[kTile];
+    __shared__ float2 ml_s[kRows];
+    __shared__ __align__(16) float red[kRows][kDHead];
 
     const int n = a.n;
     const int sparts = (a.max_global + kRows - 1) / kRows;
@@ -469,10 +500,14 @@ __global__ void __launch_bounds__(kThreads) grows_chunk_kernel(const BwdArgs A)
     const int g = min(a.ws.counts[b], a.max_global);
     if (s0 >= g) return;
     const int tid = threadIdx.x, rl = tid >> 2, qd = tid & 3;
-    const int slot = s0 + rl;
+    const int gv = min(g - s0, kRows);
+    const SlotGroups sg = slot_groups(gv, rl);
+    const int slot = s0 + sg.sl;
     const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
-    const int i = slot < g ? a.ws.gidx[size_t(b) * n + slot] : -1;
+    const int i = sg.sl < gv ? a.ws.gidx[size_t(b) * n + slot] : -1;
     const bool active = i >= 0 && bit_at(vb, i);
+    if (kGrad)
+        for (int e = tid; e < kRows * kDHead; e += kThreads) (&red[0][0])[e] = 0.f;
     const size_t rowoff = (size_t(bh) * n + (active ? i : 0)) * kDHead;
     const T *Kg = static_cast<const T *>(a.kg) + size_t(bh) * n * kDHead;
     const T *Vg = static_cast<const T *>(a.vg) + size_t(bh) * n * kDHead;
@@ -530,7 +565,8 @@ __global__ void __launch_bounds__(kThreads) grows_chunk_kernel(const BwdArgs A)
         stage_rows(ks, Kg, pos, tid);
         if (kGrad) stage_rows(vs, Vg, pos, tid);
         __syncthreads();
-        for (int c = 0; c < kTile; ++c) {
+#pragma unroll 2
+        for (int c = sg.grp; c < kTile; c += sg.R) {
             const float sc = dot_quarter(q, ks[c], qd);
             if (kGrad) {
                 const float dp = dot_quarter(dO, vs[c], qd);
@@ -545,19 +581,36 @@ __global__ void __launch_bounds__(kThreads) grows_chunk_kernel(const BwdArgs A)
             }
         }
     }
-    if (slot >= g) return;
     if (!kGrad) {
-        if (qd == 0) part[size_t(chunk) * mg + slot] = make_float2(m, l);
+        // Merge the groups' (max, sum) of each slot.
+        if (qd == 0) ml_s[rl] = make_float2(m, l);
+        __syncthreads();
+        if (tid < gv) {
+            float M = -INFINITY, L = 0.f;
+            for (int q2 = 0; q2 < sg.R; ++q2) M = fmaxf(M, ml_s[q2 * sg.G2 + tid].x);
+            if (M != -INFINITY)
+                for (int q2 = 0; q2 < sg.R; ++q2) {
+                    const float2 v = ml_s[q2 * sg.G2 + tid];
+                    if (v.x != -INFINITY) L += v.y * exp2f(v.x - M);
+                }
+            part[size_t(chunk) * mg + s0 + tid] = make_float2(M, L);
+        }
         return;
     }
-    if (chunk == 0 && qd == 0) {
+    if (chunk == 0 && sg.grp == 0 && qd == 0 && sg.sl < gv) {
         A.lse_g[size_t(bh) * mg + slot] = lse;
         A.dsum_g[size_t(bh) * mg + slot] = D;
     }
-    if (!active) return;
-    float *dst = A.dqg_acc + (size_t(bh) * mg + slot) * kDHead + kQ * qd;
+    if (active) {
 #pragma unroll
-    for (int x = 0; x < kQ; ++x) atomicAdd(dst + x, dq[x]);
+        for (int x = 0; x < kQ; ++x) atomicAdd(&red[sg.sl][kQ * qd + x], dq[x]);
+    }
+    __syncthreads();
+    for (int e = tid; e < gv * kDHead; e += kThreads) {
+        const int s_ = e / kDHead, x = e - s_ * kDHead;
+        if (!bit_at(vb, a.ws.gidx[size_t(b) * n + s0 + s_])) continue;
+        atomicAdd(A.dqg_acc + (size_t(bh) * mg + s0 + s_) * kDHead + x, red[s_][x]);
+    }
 }
 
 // dqg of each valid global row: the fp32 sums scaled by 1/sqrt(d), in T.
@@ -639,7 +692,9 @@ __global__ void __launch_bounds__(kThreads) gkeys_kernel(const BwdArgs A)
         stage_rows(qs, Qg, pos, tid);
         stage_rows(ds, dO, pos, tid);
         __syncthreads();
-        for (int c = 0; c < kTile; ++c) {
+        const int cn = min(kTile, g - s0);       // real slots of this tile
+#pragma unroll 2
+        for (int c = 0; c < cn; ++c) {
             const float s = dot_quarter(k, qs[c], qd);
             const float dp = dot_quarter(v, ds[c], qd);
             if (!kvalid || !rok[c]) continue;
