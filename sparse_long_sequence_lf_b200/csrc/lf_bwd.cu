@@ -711,10 +711,10 @@ __global__ void __launch_bounds__(kThreads) gkeys_kernel(const BwdArgs A)
 
 }  // namespace bwd
 
-// Launches of the global-token parts, shared by both band paths: they run
-// after the band rows (which write lse and D of the local rows).
+// Global rows (Qg against Kg, Vg) and the Kg/Vg keys: needs only the inputs
+// and the prepared workspace, so it runs beside the band rows.
 template <typename T>
-int launch_global_parts(const BwdArgs &A, size_t elem, cudaStream_t stream)
+int launch_global_rows(const BwdArgs &A, size_t elem, cudaStream_t stream)
 {
     using namespace bwd;
     const AttnArgs &a = A.a;
@@ -727,10 +727,8 @@ int launch_global_parts(const BwdArgs &A, size_t elem, cudaStream_t stream)
     const int bh = a.B * a.H;
     const int sparts = (a.max_global + kRows - 1) / kRows;
     const size_t mg = size_t(a.max_global);
-    if (cudaMemsetAsync(A.gkv, 0, sizeof(float) * bh * mg * 2 * kDHead, stream) != cudaSuccess ||
-        cudaMemsetAsync(A.dqg_acc, 0, sizeof(float) * bh * mg * kDHead, stream) != cudaSuccess)
+    if (cudaMemsetAsync(A.dqg_acc, 0, sizeof(float) * bh * mg * kDHead, stream) != cudaSuccess)
         return kErrCuda;
-    gcols_kernel<T><<<bh * sparts * ((a.n + kGChunk - 1) / kGChunk), kThreads, 0, stream>>>(A);
     grows_chunk_kernel<T, false><<<bh * sparts * A.nchg, kThreads, 0, stream>>>(A);
     grows_chunk_kernel<T, true><<<bh * sparts * A.nchg, kThreads, 0, stream>>>(A);
     const size_t nfin = size_t(bh) * mg * (kDHead / 4);
@@ -739,24 +737,67 @@ int launch_global_parts(const BwdArgs &A, size_t elem, cudaStream_t stream)
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 
+// Global tokens as keys of the rows outside their window: needs the band
+// rows' lse and D; the band keys read its sums.
+template <typename T>
+int launch_global_cols(const BwdArgs &A, cudaStream_t stream)
+{
+    using namespace bwd;
+    const AttnArgs &a = A.a;
+    if (a.max_global == 0) return kOk;
+    const int bh = a.B * a.H;
+    const int sparts = (a.max_global + kRows - 1) / kRows;
+    const size_t mg = size_t(a.max_global);
+    if (cudaMemsetAsync(A.gkv, 0, sizeof(float) * bh * mg * 2 * kDHead, stream) != cudaSuccess)
+        return kErrCuda;
+    gcols_kernel<T><<<bh * sparts * ((a.n + kGChunk - 1) / kGChunk), kThreads, 0, stream>>>(A);
+    return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+}
+
+std::unique_lock<std::mutex> side_stream(SideStream *&out)
+{
+    static std::mutex mu;
+    static SideStream side[64];
+    static bool made[64] = {};
+    std::unique_lock<std::mutex> lock(mu);
+    out = nullptr;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return lock;
+    if (!made[dev]) {
+        SideStream &s = side[dev];
+        if (cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess)
+            return lock;
+        made[dev] = true;
+    }
+    out = &side[dev];
+    return lock;
+}
+
 template <typename T>
 int launch_backward_simt(const BwdArgs &A, size_t elem, cudaStream_t stream)
 {
     using namespace bwd;
-    const AttnArgs &a = A.a;
-    const size_t bytes = size_t(a.B) * a.H * a.n * kDHead * elem;
-    // Qg gets gradient rows only at global positions.
-    if (cudaMemsetAsync(A.dqg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
-    const int band_ctas = a.B * a.band_items_per_batch * kParts;
-    if (band_ctas > 0) rows_kernel<T><<<band_ctas, kThreads, 0, stream>>>(A);
-    // The keys kernel adds the global-key sums of gcols_kernel.
-    if (int rc = launch_global_parts<T>(A, elem, stream)) return rc;
-    if (band_ctas > 0) keys_kernel<T><<<band_ctas, kThreads, 0, stream>>>(A);
-    return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+    const int band_ctas = A.a.B * A.a.band_items_per_batch * kParts;
+    return backward_schedule<T>(
+        A, elem, stream,
+        [&]() {
+            if (band_ctas > 0) rows_kernel<T><<<band_ctas, kThreads, 0, stream>>>(A);
+            return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+        },
+        [&]() {
+            if (band_ctas > 0) keys_kernel<T><<<band_ctas, kThreads, 0, stream>>>(A);
+            return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+        });
 }
 
-template int launch_global_parts<__half>(const BwdArgs &, size_t, cudaStream_t);
-template int launch_global_parts<__nv_bfloat16>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_global_rows<__half>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_global_rows<__nv_bfloat16>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_global_rows<float>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_global_cols<__half>(const BwdArgs &, cudaStream_t);
+template int launch_global_cols<__nv_bfloat16>(const BwdArgs &, cudaStream_t);
+template int launch_global_cols<float>(const BwdArgs &, cudaStream_t);
 template int launch_backward_simt<float>(const BwdArgs &, size_t, cudaStream_t);
 template int launch_backward_simt<__half>(const BwdArgs &, size_t, cudaStream_t);
 template int launch_backward_simt<__nv_bfloat16>(const BwdArgs &, size_t, cudaStream_t);

@@ -1,6 +1,8 @@
 // Arguments of the attention backward kernels (lf_bwd.cu).
 #pragma once
 
+#include <mutex>
+
 #include "../../include/lf_attention.h"
 #include "lf_device.cuh"
 
@@ -58,8 +60,46 @@ inline void backward_scratch_ptrs(BwdArgs &A, void *scratch, int B, int H, int n
 
 // CUDA-core path: every dtype, any dilations.
 template <typename T> int launch_backward_simt(const BwdArgs &A, size_t elem, cudaStream_t stream);
-// Global-token parts (after the band rows, before the band keys).
-template <typename T> int launch_global_parts(const BwdArgs &A, size_t elem, cudaStream_t stream);
+// Global rows and Kg/Vg keys (independent of the band), and global tokens as
+// keys of the rows outside their window (after the band rows, before the band
+// keys).
+template <typename T> int launch_global_rows(const BwdArgs &A, size_t elem, cudaStream_t stream);
+template <typename T> int launch_global_cols(const BwdArgs &A, cudaStream_t stream);
+
+// A second stream of the current device, with the events that fork work onto
+// it and join it back; the returned lock serialises its use across host
+// threads (out = nullptr when it cannot be created).
+struct SideStream {
+    cudaStream_t stream;
+    cudaEvent_t fork, join;
+};
+std::unique_lock<std::mutex> side_stream(SideStream *&out);
+
+// The backward's order on `stream`: zero dqg; fork the global-row chain onto
+// the side stream; band rows; global-token columns; band keys; join.  Works
+// under stream capture (the side stream joins and leaves with the events).
+template <typename T, typename RowsFn, typename KeysFn>
+int backward_schedule(const BwdArgs &A, size_t elem, cudaStream_t stream, RowsFn &&band_rows,
+                      KeysFn &&band_keys)
+{
+    const size_t bytes = size_t(A.a.B) * A.a.H * A.a.n * kDHead * elem;
+    // Qg gets gradient rows only at global positions.
+    if (cudaMemsetAsync(A.dqg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
+    SideStream *side = nullptr;
+    auto lock = side_stream(side);
+    if (!side) return kErrCuda;
+    if (cudaEventRecord(side->fork, stream) != cudaSuccess ||
+        cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess)
+        return kErrCuda;
+    int rc = launch_global_rows<T>(A, elem, side->stream);
+    const bool joined = cudaEventRecord(side->join, side->stream) == cudaSuccess;
+    if (rc == kOk) rc = band_rows();
+    if (rc == kOk) rc = launch_global_cols<T>(A, stream);
+    if (rc == kOk) rc = band_keys();
+    // Joined on every path, so a capture of `stream` stays well formed.
+    if (!joined || cudaStreamWaitEvent(stream, side->join, 0) != cudaSuccess) return kErrCuda;
+    return rc;
+}
 // Tensor-core path for bf16 / fp16; kErrUnsupported (nothing launched) when
 // the heads' residue classes exceed its tensor-map budget.
 int launch_backward_tc(lf_dtype dtype, const BwdArgs &A, cudaStream_t stream);

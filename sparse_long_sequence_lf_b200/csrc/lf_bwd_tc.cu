@@ -729,12 +729,9 @@ int launch_typed(const BwdArgs &A, CUtensorMapDataType dt, cudaStream_t stream)
     if (!cached(&p.krow, a.k, dt, a.n, BH, false) || !cached(&p.vrow, a.v, dt, a.n, BH, false))
         return kErrCuda;
     p.oob_row = BH * a.n;
-    const size_t bytes = size_t(BH) * a.n * kDHead * sizeof(T);
-    // Qg gets gradient rows only at global positions.
-    if (cudaMemsetAsync(A.dqg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
-    if (int rc = launch_side<T, false>(p, stream)) return rc;
-    if (int rc = launch_global_parts<T>(A, sizeof(T), stream)) return rc;
-    return launch_side<T, true>(p, stream);
+    return backward_schedule<T>(A, sizeof(T), stream,
+                                [&]() { return launch_side<T, false>(p, stream); },
+                                [&]() { return launch_side<T, true>(p, stream); });
 }
 
 }  // namespace bwdtc

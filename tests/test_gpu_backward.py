@@ -42,6 +42,10 @@ CASES = [
     Workload("fp32-causal", "f32", 1, 2, 513, 33, dilation=(1, 3), causal=True, seed=11),
     Workload("g40-n1500", "bf16", 1, 2, 1500, 64, globals_kind="random:40", pad_tail=(5,),
              seed=12),
+    # 7 + 8 + 9 + 10 residue classes exceed the tensor-core path's 24 tensor
+    # maps: the whole call takes the CUDA-core kernels
+    Workload("residue-budget", "bf16", 1, 4, 300, 8, dilation=(7, 8, 9, 10),
+             globals_kind="random:3", seed=14),
 ]
 
 
