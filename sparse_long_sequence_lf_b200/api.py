@@ -49,6 +49,20 @@ def _dilation(dilation, H):
     return (ctypes.c_int32 * H)(*vals)
 
 
+def _dev(t, name, dtype=None, shape=None):
+    """A buffer handed to the library: a contiguous CUDA tensor (host memory
+    would reach the kernels as a device address); None passes through."""
+    if t is None:
+        return None
+    if not torch.is_tensor(t) or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}")
+    return t
+
+
 def _check_projections(tensors):
     q = tensors[0]
     if q.dtype not in _DTYPES:
@@ -96,6 +110,7 @@ def default_max_global(global_mask) -> int:
 def attention_prepare(local_mask, global_mask, *, B, H, n, max_global, workspace, stream=None):
     lm = _mask(local_mask, B, n, "local_mask")
     gm = _mask(global_mask, B, n, "global_mask")
+    _dev(workspace, "workspace")
     _lib.check(_lib.lib().lf_attention_prepare(B, H, n, D_HEAD, _ptr(lm), _ptr(gm), max_global,
                                                _ptr(workspace), workspace.numel(),
                                                _stream_ptr(stream)), "lf_attention_prepare")
@@ -107,6 +122,7 @@ def attention_run(q, k, v, qg, kg, vg, *, window, dilation=None, causal=False, m
     if out is None:
         out = torch.empty_like(q)
     _check_projections([q, out])
+    _dev(workspace, "workspace")
     _lib.check(_lib.lib().lf_attention_run(dt, B, H, n, D_HEAD, _ptr(q), _ptr(k), _ptr(v),
                                            _ptr(qg), _ptr(kg), _ptr(vg), max_global, int(window),
                                            _dilation(dilation, H), int(bool(causal)), _ptr(out),
@@ -133,6 +149,7 @@ def attention_forward(q, k, v, qg, kg, vg, local_mask=None, global_mask=None, *,
     if out is None:
         out = torch.empty_like(q)
     _check_projections([q, out])
+    _dev(workspace, "workspace")
     _lib.check(_lib.lib().lf_attention_forward(
         dt, B, H, n, D_HEAD, _ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg), _ptr(vg), _ptr(lm),
         _ptr(gm), int(max_global), int(window), _dilation(dilation, H), int(bool(causal)),
@@ -161,6 +178,8 @@ def attention_forward_host(q, k, v, qg, kg, vg, local_mask=None, global_mask=Non
         if m is not None and (m.is_cuda or m.dtype not in (torch.uint8, torch.bool)
                               or tuple(m.shape) != (B, n) or not m.is_contiguous()):
             raise ValueError("host masks must be contiguous uint8 CPU tensors of shape [B, n]")
+    _dev(staging, "staging")
+    _dev(workspace, "workspace")
     rc = _lib.lib().lf_attention_forward_host(
         _DTYPES[q0.dtype], B, H, n, D_HEAD, _ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg),
         _ptr(vg), _ptr(local_mask), _ptr(global_mask), int(max_global), int(window),
@@ -172,6 +191,7 @@ def attention_forward_host(q, k, v, qg, kg, vg, local_mask=None, global_mask=Non
 
 def workspace_status(workspace, stream=None) -> int:
     """Synchronises the stream and returns the device status word."""
+    _dev(workspace, "workspace")
     return int(_lib.lib().lf_workspace_status(_ptr(workspace), _stream_ptr(stream)))
 
 
@@ -223,6 +243,10 @@ def qkv_projection(x, w, bias=None, wqg=None, bqg=None, global_idx=None, counts=
     for t in (x, w, bias, wqg, bqg):
         if t is not None and (not t.is_cuda or not t.is_contiguous() or t.dtype != x.dtype):
             raise ValueError("x, w, bias, wqg, bqg must be contiguous CUDA tensors of one dtype")
+    _dev(w, "w", x.dtype, (5 * hid, hid))
+    _dev(bias, "bias", x.dtype, (5 * hid,))
+    _dev(wqg, "wqg", x.dtype, (hid, hid))
+    _dev(bqg, "bqg", x.dtype, (hid,))
     outs = dict(out or {})
     for name in ("q", "k", "v", "kg", "vg"):
         if name not in outs:
@@ -230,6 +254,11 @@ def qkv_projection(x, w, bias=None, wqg=None, bqg=None, global_idx=None, counts=
     if "qg" not in outs:
         outs["qg"] = torch.zeros((B, H, n, D_HEAD), dtype=x.dtype, device=x.device)
     _check_projections([outs[k] for k in ("q", "k", "v", "qg", "kg", "vg")])
+    if tuple(outs["q"].shape) != (B, H, n, D_HEAD) or outs["q"].dtype != x.dtype:
+        raise ValueError("outputs must be [B, H, n, 64] in x's dtype")
+    _dev(global_idx, "global_idx", torch.int32, (B, n))
+    _dev(counts, "counts", torch.int32, (B,))
+    _dev(status, "status", torch.int32)
     _lib.check(_lib.lib().lf_qkv_projection(
         _DTYPES[x.dtype], B, n, H, D_HEAD, _ptr(x), _ptr(w), _ptr(bias), _ptr(wqg), _ptr(bqg),
         _ptr(global_idx), _ptr(counts), int(max_global), _ptr(outs["q"]), _ptr(outs["k"]),
@@ -253,11 +282,20 @@ def output_layer(attn, wo, bo, residual, gamma, beta, *, eps: float = 1e-5, out=
     for t in (attn, wo, bo, residual, gamma, beta):
         if t is not None and (not t.is_cuda or not t.is_contiguous() or t.dtype != attn.dtype):
             raise ValueError("all inputs must be contiguous CUDA tensors of attn's dtype")
+    hid = H * D_HEAD
+    _dev(wo, "wo", attn.dtype, (hid, hid))
+    _dev(bo, "bo", attn.dtype, (hid,))
+    _dev(residual, "residual", attn.dtype, (B, n, hid))
+    _dev(gamma, "gamma", attn.dtype, (hid,))
+    _dev(beta, "beta", attn.dtype, (hid,))
     if out is None:
         out = torch.empty_like(residual)
+    _dev(out, "out", attn.dtype, (B, n, hid))
     if workspace is None:
         workspace = torch.empty(output_workspace_size(B, n, H), dtype=torch.uint8,
                                 device=attn.device)
+    _dev(workspace, "workspace")
+    _dev(status, "status", torch.int32)
     _lib.check(_lib.lib().lf_output_layer(
         _DTYPES[attn.dtype], B, n, H, D_HEAD, _ptr(attn), _ptr(wo), _ptr(bo), _ptr(residual),
         _ptr(gamma), _ptr(beta), float(eps), _ptr(out), _ptr(workspace), workspace.numel(),
@@ -287,6 +325,8 @@ def attention_backward(q, k, v, qg, kg, vg, out, dout, *, window, dilation=None,
     if scratch is None:
         scratch = torch.empty(backward_scratch_size(B, H, n, max_global), dtype=torch.uint8,
                               device=q.device)
+    _dev(workspace, "workspace")
+    _dev(scratch, "scratch")
     _lib.check(_lib.lib().lf_attention_backward(
         dt, B, H, n, D_HEAD, _ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg), _ptr(vg), _ptr(out),
         _ptr(dout), int(max_global), int(window), _dilation(dilation, H), int(bool(causal)),
@@ -312,11 +352,18 @@ def ffn_block(h, w1, b1, w2, b2, gamma, beta, *, eps: float = 1e-5, out=None, wo
             raise ValueError("all inputs must be contiguous CUDA tensors of h's dtype")
     if tuple(w1.shape) != (inter, hidden) or tuple(w2.shape) != (hidden, inter):
         raise ValueError("w1 must be [inter, hidden] and w2 [hidden, inter]")
+    _dev(b1, "b1", h.dtype, (inter,))
+    _dev(b2, "b2", h.dtype, (hidden,))
+    _dev(gamma, "gamma", h.dtype, (hidden,))
+    _dev(beta, "beta", h.dtype, (hidden,))
     if out is None:
         out = torch.empty_like(h)
+    _dev(out, "out", h.dtype, (B, n, hidden))
     if workspace is None:
         workspace = torch.empty(max(1, ffn_workspace_size(B, n, hidden, inter)),
                                 dtype=torch.uint8, device=h.device)
+    _dev(workspace, "workspace")
+    _dev(status, "status", torch.int32)
     _lib.check(_lib.lib().lf_ffn_block(
         _DTYPES[h.dtype], B, n, hidden, inter, _ptr(h), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2),
         _ptr(gamma), _ptr(beta), float(eps), _ptr(out), _ptr(workspace), workspace.numel(),
@@ -344,6 +391,7 @@ def encoder_forward(x, layers, local_mask=None, global_mask=None, *, H: int, win
     B, n, hid = x.shape
     if hid != H * D_HEAD:
         raise ValueError("x's last dimension must be H*64")
+    _dev(x, "x")
     L = len(layers)
     if len(windows) != L or (dilations is not None and len(dilations) != L):
         raise ValueError("windows (and dilations) need one entry per layer")
@@ -359,6 +407,12 @@ def encoder_forward(x, layers, local_mask=None, global_mask=None, *, H: int, win
                 setattr(arr[i], f, t.data_ptr())
         if lw["w_1"].shape[0] != inter:
             raise ValueError("all layers must share the intermediate size")
+        shapes = {"w_qkv": (5 * hid, hid), "b_qkv": (5 * hid,), "w_qg": (hid, hid),
+                  "b_qg": (hid,), "w_o": (hid, hid), "b_o": (hid,), "ln1_gamma": (hid,),
+                  "ln1_beta": (hid,), "w_1": (inter, hid), "b_1": (inter,), "w_2": (hid, inter),
+                  "b_2": (hid,), "ln2_gamma": (hid,), "ln2_beta": (hid,)}
+        for f, shp in shapes.items():
+            _dev(lw.get(f), f"layer {i} {f}", x.dtype, shp)
     lm = _mask(local_mask, B, n, "local_mask")
     gm = _mask(global_mask, B, n, "global_mask")
     if max_global is None:
@@ -375,9 +429,11 @@ def encoder_forward(x, layers, local_mask=None, global_mask=None, *, H: int, win
         dil = (ctypes.c_int32 * (L * H))(*flat)
     if out is None:
         out = torch.empty_like(x)
+    _dev(out, "out", x.dtype, (B, n, hid))
     if workspace is None:
         workspace = torch.empty(max(1, encoder_workspace_size(B, n, H, inter, max_global)),
                                 dtype=torch.uint8, device=x.device)
+    _dev(workspace, "workspace")
     _lib.check(_lib.lib().lf_encoder_forward(
         _DTYPES[x.dtype], B, n, H, D_HEAD, inter, L, arr, win, dil, _ptr(x), _ptr(lm), _ptr(gm),
         int(max_global), float(eps), _ptr(out), _ptr(workspace), workspace.numel(),

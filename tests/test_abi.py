@@ -106,3 +106,66 @@ def test_backward_argument_checks(L):
     assert bwd(scb=8) == -3                             # scratch too small
     if not torch.cuda.is_available():
         assert bwd() == -7
+
+
+def test_ffn_and_encoder_argument_checks(L):
+    import torch
+    P = ctypes.c_void_p
+    assert L.lf_ffn_workspace_size(1, 64, 128, 512) >= 64 * 512 * 2 + 64 * 128 * 4
+    assert L.lf_ffn_workspace_size(1, 64, 100, 512) == 0        # hidden not a multiple of 64
+    assert L.lf_ffn_workspace_size(1, 64, 128, 0) == 0
+
+    def ffn(**over):
+        a = dict(dtype=2, B=1, n=64, hid=128, inter=256, h=256, w=512, out=768, eps=1e-5,
+                 ws=1024, wsb=1 << 20)
+        a.update(over)
+        return L.lf_ffn_block(a["dtype"], a["B"], a["n"], a["hid"], a["inter"], P(a["h"]),
+                              P(a["w"]), None, P(a["w"]), None, P(a["w"]), P(a["w"]),
+                              ctypes.c_float(a["eps"]), P(a["out"]), P(a["ws"]), a["wsb"],
+                              None, None)
+
+    assert ffn(dtype=0) == -2                                    # fp32: unsupported
+    assert ffn(dtype=9) == -1
+    assert ffn(hid=96) == -2                                     # not a multiple of 64
+    assert ffn(h=0) == -1
+    assert ffn(out=520) == -1                                    # misaligned
+    assert ffn(eps=-1.0) == -1
+    assert ffn(ws=0) == -3
+    assert ffn(wsb=16) == -3
+    if not torch.cuda.is_available():
+        assert ffn() == -7
+
+    from sparse_long_sequence_lf_b200._lib import LAYER_FIELDS, LayerWeights
+    assert L.lf_encoder_workspace_size(1, 64, 2, 64, 256, 0) > 0
+    assert L.lf_encoder_workspace_size(1, 64, 2, 32, 256, 0) == 0   # head size other than 64
+    assert L.lf_encoder_workspace_size(1, 64, 2, 64, 100, 0) == 0   # inter not a multiple of 64
+
+    def enc(layers=2, windows=(8, 16), **over):
+        a = dict(dtype=2, B=1, n=64, H=2, d=64, inter=256, x=256, out=512, mg=0, eps=1e-5,
+                 ws=1024, wsb=1 << 24, skip=None, misalign=None)
+        a.update(over)
+        arr = (LayerWeights * layers)()
+        for i in range(layers):
+            for f in LAYER_FIELDS:
+                setattr(arr[i], f, 4096)
+        if a["skip"]:
+            setattr(arr[layers - 1], a["skip"], None)
+        if a["misalign"]:
+            setattr(arr[layers - 1], a["misalign"], 4104)
+        win = (ctypes.c_int32 * layers)(*windows)
+        return L.lf_encoder_forward(a["dtype"], a["B"], a["n"], a["H"], a["d"], a["inter"], layers,
+                                    arr, win, None, P(a["x"]), None, None, a["mg"],
+                                    ctypes.c_float(a["eps"]), P(a["out"]), P(a["ws"]), a["wsb"],
+                                    None)
+
+    assert enc(d=32) == -2
+    assert enc(dtype=0) == -2
+    assert enc(inter=100) == -2
+    assert enc(layers=2, windows=(8, 7)) == -1                   # odd window in the last layer
+    assert enc(skip="w_2") == -1                                 # missing weight
+    assert enc(misalign="b_1") == -1                             # misaligned bias
+    assert enc(mg=2, skip="w_qg") == -1                          # global queries need w_qg
+    assert enc(ws=0) == -3
+    assert enc(wsb=16) == -3
+    if not torch.cuda.is_available():
+        assert enc() == -7
