@@ -72,3 +72,41 @@ def test_padded_rows_and_unused_projections_get_no_gradient():
     # Qg is used only at the global row, Q only at the others
     assert np.all(g["qg"][0, 0, [i for i in range(20) if i != 5]] == 0)
     assert np.all(g["q"][0, 0, 5] == 0)
+
+
+def test_full_window_gradients_equal_sdpa_autograd():
+    # With the window covering the sequence, no global token and no padding,
+    # the attention is textbook full attention: its gradients are those of
+    # torch's scaled_dot_product_attention (fp64, CPU autograd).
+    wl, x = _case(B=1, H=2, n=24, window=64, seed=45)
+    rng = np.random.default_rng(46)
+    dout = rng.standard_normal((1, 2, 24, 64))
+    names = ("q", "k", "v", "qg", "kg", "vg")
+    arrs = {k: x[k].double().numpy() for k in names}
+    got = bwd.backward(*(arrs[k] for k in names), None, None, dout, window=wl.window)
+    q, k, v = (torch.from_numpy(arrs[n].copy()).requires_grad_(True) for n in ("q", "k", "v"))
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v)
+    (o * torch.from_numpy(dout)).sum().backward()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        np.testing.assert_allclose(got[name], t.grad.numpy(), atol=1e-10)
+    for name in ("qg", "kg", "vg"):                       # no global rows
+        assert not np.any(got[name])
+
+
+def test_all_global_gradients_equal_sdpa_autograd_on_global_projections():
+    # Every token global: every row attends to all tokens through Qg, Kg, Vg.
+    wl, x = _case(B=1, H=1, n=20, window=4, globals_kind="first:20", seed=47)
+    rng = np.random.default_rng(48)
+    dout = rng.standard_normal((1, 1, 20, 64))
+    names = ("q", "k", "v", "qg", "kg", "vg")
+    arrs = {k: x[k].double().numpy() for k in names}
+    got = bwd.backward(*(arrs[k] for k in names), None, x["global_mask"], dout,
+                       window=wl.window)
+    qg, kg, vg = (torch.from_numpy(arrs[n].copy()).requires_grad_(True)
+                  for n in ("qg", "kg", "vg"))
+    o = torch.nn.functional.scaled_dot_product_attention(qg, kg, vg)
+    (o * torch.from_numpy(dout)).sum().backward()
+    for name, t in (("qg", qg), ("kg", kg), ("vg", vg)):
+        np.testing.assert_allclose(got[name], t.grad.numpy(), atol=1e-10)
+    for name in ("q", "k", "v"):                          # no local rows
+        assert not np.any(got[name])
