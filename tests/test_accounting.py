@@ -47,3 +47,24 @@ def test_headline_workload_figures():
     flops = accounting.useful_flops(wl)
     assert 6.2e9 < flops < 6.4e9
     assert accounting.algorithmic_bytes(wl) == 6 * 12 * 4096 * 64 * 2 + 12 * 64 * 2
+
+
+def test_backward_flops_are_ten_d_per_pair():
+    wl = CASES[0]
+    assert accounting.backward_flops(wl) == 10 * wl.d * accounting.useful_pairs(wl)
+    assert accounting.backward_flops(wl) == 2.5 * accounting.useful_flops(wl)
+
+
+def test_encoder_flops_count_every_product_of_a_layer():
+    import bench
+    from sparse_long_sequence_lf_b200.workloads import EncoderWorkload
+    wl = Workload("e", "f16", 1, 2, 40, 8, globals_kind="list:0,17")
+    ew = EncoderWorkload("enc", wl, inter=256, layers=3)
+    hid, tok, g = 128, 40, 2
+    per_layer = (2 * tok * hid * 5 * hid          # Q, K, V, Kg, Vg
+                 + 2 * g * hid * hid              # Qg of the global rows
+                 + accounting.useful_flops(wl)    # the attention
+                 + 2 * tok * hid * hid            # output projection
+                 + 2 * tok * hid * 256            # FFN intermediate
+                 + 2 * tok * 256 * hid)           # FFN output
+    assert bench.encoder_flops(ew, [g]) == 3 * per_layer
