@@ -115,3 +115,38 @@ def test_backward_rejects_bad_scratch():
     with pytest.raises(lf.LfError):
         lf.attention_backward(x["q"], x["k"], x["v"], x["qg"], x["kg"], x["vg"], out, out,
                               window=8, max_global=0, workspace=ws, scratch=small)
+
+
+@pytest.mark.parametrize("name", ["bf16-b1h12-n4096-w512-g1", "fp16-b2h16-n4096-w512-g64-pad300"])
+def test_backward_full_size_sampled_heads(name):
+    # The benchmark's workloads at full size through the same call; heads are
+    # independent, so the oracle checks heads 0 and H-1 of every batch element
+    # by element (a few seconds of fp64 each).
+    from sparse_long_sequence_lf_b200.workloads import WORKLOADS
+    wl = WORKLOADS[name]
+    x = make_inputs(wl)
+    dout = make_output_grad(wl)
+    g = to_dev(x)
+    mg = max_global_of(x)
+    ws = lf.new_workspace(wl.B, wl.H, wl.n, mg, "cuda")
+    kw = dict(window=wl.window, dilation=x["dilation"], causal=wl.causal, max_global=mg)
+    out = lf.attention_forward(g["q"], g["k"], g["v"], g["qg"], g["kg"], g["vg"],
+                               g["local_mask"], g["global_mask"], workspace=ws, **kw)
+    grads = lf.attention_backward(g["q"], g["k"], g["v"], g["qg"], g["kg"], g["vg"], out,
+                                  dout.cuda(), workspace=ws, **kw)
+    torch.cuda.synchronize()
+    assert lf.workspace_status(ws) == 0
+    tol = TOL[wl.dtype]
+    for h in (0, wl.H - 1):
+        sl = lambda t: t[:, h:h + 1].contiguous()
+        ref = obw.backward(*(sl(x[k]) for k in NAMES), x["local_mask"], x["global_mask"],
+                           sl(dout), window=wl.window, dilation=[x["dilation"][h]],
+                           causal=wl.causal)
+        for nm in NAMES:
+            got = grads[nm][:, h:h + 1].float().cpu().numpy().astype(np.float64)
+            want = ref[nm]
+            assert np.all(np.isfinite(got)), f"{name} head {h} d{nm}: non-finite"
+            excess = np.abs(got - want) - tol * np.abs(want)
+            worst = np.unravel_index(int(np.argmax(excess)), excess.shape)
+            assert excess.max() <= tol, (f"{name} head {h} d{nm}: err "
+                                         f"{abs(got[worst] - want[worst]):.3e} at {worst}")
