@@ -72,6 +72,10 @@ ENC_CASES = [
     (Workload("enc-nog", "bf16", 1, 4, 384, 32, seed=22), 1, 1024, [32], [[1, 2, 1, 3]]),
     (Workload("enc-3layers", "f16", 1, 2, 700, 16, globals_kind="random:5", seed=23), 3, 256,
      [16, 64, 128], [[1, 1], [2, 1], [1, 3]]),
+    # one layer of the benchmark model at full width (16 heads, hidden 1024,
+    # intermediate 4096, window 512, 64 global tokens at the front), 1024 tokens
+    (Workload("enc-full-width", "f16", 1, 16, 1024, 512, globals_kind="first:64", seed=25), 1,
+     4096, [512], None),
 ]
 
 
