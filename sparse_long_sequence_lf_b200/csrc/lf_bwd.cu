@@ -1,5 +1,7 @@
 // Backward pass of the attention on the CUDA cores (fp32 arithmetic for
-// every input type).
+// every input type): the band kernels of the fp32 path (and of bf16 / fp16
+// calls whose dilations exceed the tensor-core path's tensor maps), and the
+// global-token kernels of every path.
 //
 // With s_ij = <q_i, k_j> / sqrt(d), p_ij = exp(s_ij - lse_i) over the key set
 // of row i (the same sets as the forward: window taps and global tokens for a
@@ -12,16 +14,23 @@
 // "Dilated Sliding Window", "Global Attention": the attention these rows
 // differentiate.)
 //
-// Four kernels, no atomics: every output row is owned by one thread quad.
-//   rows    32 query rows of one (batch, head, residue class) per CTA, four
-//           threads per row (a quarter of the head dimension each): pass 1
-//           recomputes the row's log-sum-exp over its keys, pass 2 sums dq;
-//           writes lse and D per row for the key kernel.
-//   keys    32 keys of one (batch, head, residue class) per CTA: dk, dv over
-//           the window rows that reach the key, plus, for a global token,
-//           every other valid non-global row of the head.
-//   grows   the global rows (Qg): lse, D and dqg over every valid key.
-//   gkeys   dkg, dvg of every key over the global rows.
+// Threads work in quads, each thread a quarter of the head dimension.
+//   rows_kernel    32 query rows of one (batch, head, residue class) per CTA:
+//                  pass 1 recomputes each row's log-sum-exp, pass 2 sums dq;
+//                  writes lse and D per row.
+//   keys_kernel    32 keys of one (batch, head, residue class) per CTA: dk, dv
+//                  over the window rows that reach them, plus (for a global
+//                  token) the sums gcols_kernel left in the scratch.
+//   gcols_kernel   a global token as the key of the valid non-global rows that
+//                  do not reach it through the window: chunks of 128 rows,
+//                  fp32 atomic sums per slot.
+//   grows_chunk_kernel  global rows (Qg) against 128-key chunks of Kg, Vg:
+//                  pass 1 the chunk's (max, sum), pass 2 the merged
+//                  log-sum-exp and the chunk's dqg terms (fp32 atomics);
+//                  gfinal_kernel scales and stores dqg.
+//   gkeys_kernel   dkg, dvg of every key over the global rows.
+// Order (backward_schedule): band rows; global-token columns; band keys on
+// the caller's stream, the global rows and gkeys on a side stream.
 #include "lf_bwd.cuh"
 #include "lf_vec.cuh"
 
