@@ -326,8 +326,16 @@ LF_API int lf_attention_forward_static(lf_dtype dtype, int B, int H, int n, int 
  *                and max_global (lf_attention_prepare or
  *                lf_attention_forward); read only.
  *   scratch      device, 256-byte aligned, lf_backward_scratch_size bytes:
- *                per-row log-sum-exp and D between the kernels.
- * Arithmetic in fp32 for every dtype; results are rounded to dtype once.
+ *                per-row log-sum-exp and D between the kernels, and the fp32
+ *                partial sums of the global-token parts.  Overwritten by
+ *                every call; nothing needs clearing beforehand.
+ * fp32 inputs: CUDA-core kernels, fp32 arithmetic.  bf16 / fp16 inputs:
+ * tcgen05 kernels for the window band (P and dS rounded to the input type
+ * before their products, fp32 accumulation), CUDA-core fp32 kernels for the
+ * global-token parts; more than 24 (dilation, residue) classes over the heads
+ * send the whole call to the CUDA-core kernels.  Part of the work runs on a
+ * second, library-owned stream of the device, forked from and joined back to
+ * `stream` with events (stream capture included).
  * Every tensor pointer must be 16-byte aligned.  Errors are returned before
  * anything is launched, as for lf_attention_run.  More global tokens than
  * max_global is recorded by the preparation in the workspace status word
