@@ -134,3 +134,17 @@ def test_small_window_differs_from_full_attention():
     pr /= pr.sum()
     attn = enc.encoder_layer(x, w, H=H, window=4)[1]["attn"][0, 0, i]
     assert np.allclose(attn, pr @ v[js], atol=1e-12)
+
+
+def test_stack_gives_each_layer_its_own_window():
+    # Layer 0 with a narrow window, layer 1 covering the sequence: the stack
+    # equals that narrow layer followed by a full-attention transformer layer.
+    rng = np.random.default_rng(6)
+    H, n, inter = 1, 32, 128
+    ws = [_weights(rng, H, inter) for _ in range(2)]
+    x = rng.normal(size=(1, n, 64))
+    got = enc.encoder_forward(x, ws, H=H, windows=[4, 2 * n])
+    first, _ = enc.encoder_layer(x, ws[0], H=H, window=4)
+    with torch.no_grad():
+        want = _torch_layer(ws[1], H, inter)(torch.from_numpy(first)).numpy()
+    assert np.allclose(got, want, atol=1e-10)
