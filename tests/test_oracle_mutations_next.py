@@ -116,3 +116,58 @@ def test_unmutated_copies_pass_every_pin():
                    BWD_PINS) == []
     assert _caught(te, "enc", _mutant(oenc, "import numpy as np", "import numpy as np"),
                    ENC_PINS) == []
+
+
+# ----------------------------------------------- projection / output oracle
+import test_projection_oracle as tp  # noqa: E402
+from oracle import projection as oproj  # noqa: E402
+
+PROJ_PINS = [(getattr(tp, n), ()) for n in dir(tp) if n.startswith("test_")]
+
+PROJ_MUTATIONS = [
+    ("heads split in the wrong order", "return y.reshape(B, n, H, d).transpose(0, 2, 1, 3)",
+     "return y.reshape(B, H, n, d)"),
+    ("weight blocks used transposed", 'y = np.einsum("bni,oi->bno", x, wp)',
+     'y = np.einsum("bni,io->bno", x, wp)'),
+    ("every block takes the first block's bias",
+     "[p * hid:(p + 1) * hid]\n        out[name]", "[0:hid]\n        out[name]"),
+    ("projection blocks in reverse order", "wp = w[p * hid:(p + 1) * hid]",
+     "wp = w[(4 - p) * hid:(5 - p) * hid]"),
+    ("Qg through the stacked Q weights", "y = x[b, rows] @ wqg.T", "y = x[b, rows] @ w[:hid].T"),
+    ("heads concatenated in the wrong order",
+     "merged = a.transpose(0, 2, 1, 3).reshape(B, n, H * d)",
+     "merged = a.reshape(B, n, H * d)"),
+    ("output weights used transposed",
+     'y = np.einsum("bni,oi->bno", merged, np.asarray(wo, dtype=np.float64))',
+     'y = np.einsum("bni,io->bno", merged, np.asarray(wo, dtype=np.float64))'),
+    ("residual dropped", "y = y + np.asarray(residual, dtype=np.float64)", "y = y"),
+    ("eps outside the square root", "z = (y - mean) / np.sqrt(var + eps)",
+     "z = (y - mean) / (np.sqrt(var) + eps)"),
+    ("gamma and beta swapped",
+     "return z * np.asarray(gamma, dtype=np.float64) + np.asarray(beta, dtype=np.float64)",
+     "return z * np.asarray(beta, dtype=np.float64) + np.asarray(gamma, dtype=np.float64)"),
+]
+
+
+def _caught_proj(mutant):
+    saved = (tp.projection_forward, tp.output_layer)
+    tp.projection_forward, tp.output_layer = mutant.projection_forward, mutant.output_layer
+    caught = []
+    try:
+        for fn, args in PROJ_PINS:
+            try:
+                fn(*args)
+            except Exception as e:
+                caught.append((fn.__name__, type(e).__name__))
+    finally:
+        tp.projection_forward, tp.output_layer = saved
+    return caught
+
+
+@pytest.mark.parametrize("label,old,new", PROJ_MUTATIONS, ids=[m[0] for m in PROJ_MUTATIONS])
+def test_projection_pins_catch_mutation(label, old, new):
+    assert _caught_proj(_mutant(oproj, old, new)), f"no pin caught the planted mistake: {label}"
+
+
+def test_unmutated_projection_copy_passes_every_pin():
+    assert _caught_proj(_mutant(oproj, "import numpy as np", "import numpy as np")) == []

@@ -125,3 +125,42 @@ def test_output_layer_bias_residual_and_affine():
     # adding a constant to every feature of the pre-norm sum changes nothing
     z2 = output_layer(attn, wo, bo + 5.0, res, g, b)
     np.testing.assert_allclose(z2, z, atol=1e-9)
+
+
+def test_qg_takes_its_own_weights_one_hot():
+    # A one-hot token at a global row picks column c of wqg (plus bqg); the
+    # stacked Q block is a different matrix, so using it instead would show.
+    rng = np.random.default_rng(8)
+    B, n, c = 1, 4, 77
+    x = np.zeros((B, n, HID))
+    x[0, 2, c] = 1.0
+    w = rng.standard_normal((5 * HID, HID))
+    wqg = rng.standard_normal((HID, HID))
+    bqg = rng.standard_normal(HID)
+    gidx, counts = _gidx(B, n, [[2]])
+    out = projection_forward(x, w, None, wqg, bqg, gidx, counts, H=H)
+    np.testing.assert_array_equal(out["qg"][0, :, 2, :].reshape(HID), wqg[:, c] + bqg)
+
+
+def test_output_layer_weight_orientation():
+    # attention output one-hot in feature c: the pre-norm sum is column c of
+    # wo. Column c alternates +-1 (normalises to +-1/sqrt(1+eps)); row c is a
+    # ramp, so a transposed wo gives a different row.
+    B, n, c = 1, 1, 5
+    wo = np.tile(np.arange(HID, dtype=np.float64), (HID, 1))      # row r = ramp
+    wo[:, c] = np.array([1.0, -1.0] * (HID // 2))                  # column c alternates
+    attn = np.zeros((B, H, n, D))
+    attn[0, c // D, 0, c % D] = 1.0
+    z = output_layer(attn, wo, None, np.zeros((B, n, HID)), np.ones(HID), np.zeros(HID),
+                     eps=1e-5)
+    np.testing.assert_allclose(z[0, 0], wo[:, c] / np.sqrt(1.0 + 1e-5), rtol=0, atol=1e-12)
+
+
+def test_output_layer_adds_the_residual():
+    # Zero attention output and bias: the row is the normalised residual.
+    B, n = 1, 2
+    res = np.zeros((B, n, HID))
+    res[0, 1] = np.array([1.0, -1.0] * (HID // 2))
+    z = output_layer(np.zeros((B, H, n, D)), np.eye(HID), None, res, np.ones(HID),
+                     np.zeros(HID), eps=1e-5)
+    np.testing.assert_allclose(z[0, 1], res[0, 1] / np.sqrt(1.0 + 1e-5), rtol=0, atol=1e-12)
