@@ -144,6 +144,22 @@ def pin_full_with_globals(orc):
         _close(out[0, :, i], ref, f"full+globals row {i}")
 
 
+def pin_per_head_dilation(orc):
+    """Each head takes its own dilation (LF-notes, Dilated Sliding Window:
+    different dilations per head): every (batch, head) equals attention with
+    an explicit tap mask of that head's dilation."""
+    B, H, n, d = 2, 3, 37, 8
+    q, k, v, qg, kg, vg = _six(B, H, n, d, 350)
+    dils = [1, 3, 2]
+    for (w, causal) in [(6, False), (5, True)]:
+        out = orc.forward(q, k, v, qg, kg, vg, window=w, dilation=dils, causal=causal)
+        for b in range(B):
+            for h in range(H):
+                ref = _sdpa(q[b, h], k[b, h], v[b, h],
+                            mask=_tap_mask(n, w, dils[h], causal)).numpy()
+                _close(out[b, h], ref, f"per-head dilation w={w} b={b} h={h} causal={causal}")
+
+
 # ------------------------------------------------------ structural identities
 def pin_dilation_residue(orc):
     """A head with dilation dil equals dil independent undilated windows over
@@ -311,6 +327,6 @@ def pin_rejects_causal_globals(orc):
 
 
 ALL_PINS = [pin_global_index, pin_full_attention, pin_causal_full, pin_band_masked,
-            pin_globals_masked, pin_full_with_globals, pin_dilation_residue,
+            pin_per_head_dilation, pin_globals_masked, pin_full_with_globals, pin_dilation_residue,
             pin_padding_truncation, pin_row_sums, pin_golden_key_sets,
             pin_uniform_closed_form, pin_closed_form_examples, pin_rejects_causal_globals]

@@ -39,6 +39,23 @@ MUTATIONS = [
     ("last global dropped", "counts[b] = cnt;", "counts[b] = cnt > 0 ? cnt - 1 : 0;"),
     ("dot product drops a term", "for (int x = 0; x < d; ++x) dot += qrow[x] * krow[x];",
      "for (int x = 1; x < d; ++x) dot += qrow[x] * krow[x];"),
+    ("padded global keys used by local rows",
+     "        if (!is_valid_key(local_mask_b, j)) continue;\n        if (in_window",
+     "        if (in_window"),
+    ("dedupe window too wide", "return a / dil <= w / 2;", "return a / dil <= w;"),
+    ("batch 0's global index for every batch", "gidx + (size_t)b * n, cnts[b]", "gidx, cnts[0]"),
+    ("batch 0's global mask for every batch",
+     "const uint8_t *gm_b = global_mask ? global_mask + (size_t)b * n : NULL;",
+     "const uint8_t *gm_b = global_mask ? global_mask : NULL;"),
+    ("batch 0's local mask for every batch",
+     "const uint8_t *lm_b = local_mask ? local_mask + (size_t)b * n : NULL;",
+     "const uint8_t *lm_b = local_mask ? local_mask : NULL;"),
+    ("dilation indexed by batch", "int dil = dilation ? dilation[h] : 1;",
+     "int dil = dilation ? dilation[b] : 1;"),
+    ("one dilation for every head", "int dil = dilation ? dilation[h] : 1;",
+     "int dil = dilation ? dilation[0] : 1;"),
+    ("tensor base ignores the batch", "size_t base = (size_t)bh * n * d;",
+     "size_t base = (size_t)h * n * d;"),
 ]
 
 
