@@ -20,6 +20,10 @@ def _case(**kw):
     dict(B=1, H=2, n=40, window=8, dilation=(1, 2), globals_kind="list:3,31", pad_tail=(5,),
          seed=41),
     dict(B=2, H=1, n=33, window=5, causal=True, seed=42),
+    # two batches with their own padding and global tokens, heads with their
+    # own dilations
+    dict(B=2, H=2, n=36, window=6, dilation=(1, 3), globals_kind="list:2,30;7",
+         pad_tail=(0, 9), seed=49),
 ])
 def test_forward_agrees_with_the_c_oracle(kw):
     wl, x = _case(**kw)

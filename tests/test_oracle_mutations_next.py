@@ -69,6 +69,12 @@ BWD_MUTATIONS = [
     ("gradients returned under swapped names",
      'names = ("q", "k", "v", "qg", "kg", "vg")\n    return',
      'names = ("q", "k", "v", "kg", "qg", "vg")\n    return'),
+    ("one dilation for every head", "_is_tap(i, j, window, dil[h], causal)",
+     "_is_tap(i, j, window, dil[0], causal)"),
+    ("batch 0's padding for every batch", "local[b, h, i] &= valid[b]",
+     "local[b, h, i] &= valid[0]"),
+    ("batch 0's global tokens for every batch", "gpos = [j for j in range(n) if isg[b, j]]",
+     "gpos = [j for j in range(n) if isg[0, j]]"),
 ]
 
 
