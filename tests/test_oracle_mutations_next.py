@@ -149,6 +149,9 @@ PROJ_MUTATIONS = [
     ("residual dropped", "y = y + np.asarray(residual, dtype=np.float64)", "y = y"),
     ("eps outside the square root", "z = (y - mean) / np.sqrt(var + eps)",
      "z = (y - mean) / (np.sqrt(var) + eps)"),
+    ("batch 0's global count for every batch", "g = int(counts[b])", "g = int(counts[0])"),
+    ("batch 0's hidden states for every global row", "y = x[b, rows] @ wqg.T",
+     "y = x[0, rows] @ wqg.T"),
     ("gamma and beta swapped",
      "return z * np.asarray(gamma, dtype=np.float64) + np.asarray(beta, dtype=np.float64)",
      "return z * np.asarray(beta, dtype=np.float64) + np.asarray(gamma, dtype=np.float64)"),
