@@ -148,3 +148,38 @@ def test_stack_gives_each_layer_its_own_window():
     with torch.no_grad():
         want = _torch_layer(ws[1], H, inter)(torch.from_numpy(first)).numpy()
     assert np.allclose(got, want, atol=1e-10)
+
+
+def test_padding_equals_truncation_through_the_stack():
+    # Padded tokens are no keys of any row and every other step is per token,
+    # so the valid rows of a padded sequence equal the stack on the truncated
+    # sequence.
+    rng = np.random.default_rng(7)
+    H, n, t, inter = 1, 30, 6, 128
+    ws = [_weights(rng, H, inter) for _ in range(2)]
+    x = rng.normal(size=(1, n, 64))
+    lm = np.ones((1, n), np.uint8)
+    lm[0, n - t:] = 0
+    gm = np.zeros((1, n), np.uint8)
+    gm[0, 2] = 1
+    got = enc.encoder_forward(x, ws, lm, gm, H=H, windows=[8, 8])
+    want = enc.encoder_forward(x[:, :n - t], ws, None, gm[:, :n - t].copy(), H=H,
+                               windows=[8, 8])
+    assert np.allclose(got[:, :n - t], want, atol=1e-10)
+    # and the padding does change the valid rows near the tail
+    full = enc.encoder_forward(x, ws, None, gm, H=H, windows=[8, 8])
+    assert np.abs(full[:, :n - t] - want).max() > 1e-6
+
+
+def test_stack_gives_each_layer_its_own_dilations():
+    rng = np.random.default_rng(8)
+    H, n, inter = 2, 28, 128
+    ws = [_weights(rng, H, inter) for _ in range(2)]
+    x = rng.normal(size=(1, n, 128))
+    dils = [[1, 2], [3, 1]]
+    got = enc.encoder_forward(x, ws, H=H, windows=[6, 6], dilations=dils)
+    h, _ = enc.encoder_layer(x, ws[0], H=H, window=6, dilation=dils[0])
+    want, _ = enc.encoder_layer(h, ws[1], H=H, window=6, dilation=dils[1])
+    assert np.allclose(got, want, atol=1e-12)
+    other, _ = enc.encoder_layer(h, ws[1], H=H, window=6, dilation=dils[0])
+    assert np.abs(other - want).max() > 1e-6

@@ -106,6 +106,11 @@ ENC_MUTATIONS = [
      'wqg = w["w_qkv"][:hid]'),
     ("every layer takes the first layer's window", "window=windows[l],",
      "window=windows[0],"),
+    ("attention ignores the padding", 'p["vg"], local_mask,\n                          global_mask,',
+     'p["vg"], None,\n                          global_mask,'),
+    ("every layer takes the first layer's dilations",
+     "dil = None if dilations is None else dilations[l]",
+     "dil = None if dilations is None else dilations[0]"),
 ]
 
 
