@@ -52,7 +52,7 @@ def load_peaks():
 
 # Kernel sources whose change invalidates a stored DRAM-traffic figure.
 TRAFFIC_SOURCES = {
-    "attn_tc_kernel": ("lf_tc.cu", "lf_sm100.cuh", "lf_device.cuh"),
+    "attn_fwd_kernel": ("lf_fwd.cu", "lf_sm100.cuh", "lf_device.cuh"),
     "band_simt_kernel": ("lf_simt.cu", "lf_device.cuh"),
     "proj_kernel": ("lf_proj.cu", "lf_sm100.cuh", "lf_device.cuh"),
 }
@@ -299,6 +299,10 @@ def run_gpu_arm(args, wl, world, rank, local):
     max_ms = reduce_max(local_ms, device)
     clocks = sampler.summary("timed region plus 0.5 s of the same graph on each side")
 
+    # Distribution of the step time: every replay of the graph timed on its
+    # own (events on the launching stream), at least 50 replays.
+    step_dist = replay_distribution(replay, g_chunk, chunk, stream, device, samples=50)
+
     status = lf.workspace_status(ws, stream)
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -316,6 +320,7 @@ def run_gpu_arm(args, wl, world, rank, local):
     ke.record(stream)
     torch.cuda.synchronize(device)
     kernel_ms = ks.elapsed_time(ke) / (reps * chunk)
+    kernel_dist = replay_distribution(replay, g_run, chunk, stream, device, samples=50)
 
     flops = accounting.useful_flops(wl)
     bytes_ = accounting.algorithmic_bytes(wl)
@@ -326,7 +331,7 @@ def run_gpu_arm(args, wl, world, rank, local):
     peaks, peak_kind = load_peaks()
     achieved_gbs = bytes_ / (kernel_ms * 1e-3) / 1e9
     kernel_tflops = flops / (kernel_ms * 1e-3) / 1e12
-    kname = "attn_tc_kernel" if wl.dtype != "f32" else "band_simt_kernel"
+    kname = "attn_fwd_kernel" if wl.dtype != "f32" else "band_simt_kernel"
     roofline = {
         "kernel": kname,
         "bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
@@ -335,6 +340,8 @@ def run_gpu_arm(args, wl, world, rank, local):
         "kernel_us": round(kernel_ms * 1e3, 3), "algorithmic_bytes": bytes_,
         "useful_tflops": round(kernel_tflops, 1),
         "tensor_frac_of_measured_bf16": round(kernel_tflops / peaks["bf16_tflops"], 4),
+        "kernel_us_dist": {k: (round(v * 1e3, 3) if k != "samples" else v)
+                           for k, v in kernel_dist.items()},
     }
 
     if world > 1:
@@ -354,11 +361,12 @@ def run_gpu_arm(args, wl, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic",
         "tokens_per_s": round(tokens_per_s, 1),
-        "config": {**workload_config(wl, world),
-                   "l2": f"{nsets} rotating input sets, {nsets * per_set / 2**20:.0f} MiB > 2x L2",
+        "config": workload_config(wl, world),
+        "timing": {"l2": f"{nsets} rotating input sets, {nsets * per_set / 2**20:.0f} MiB > 2x L2",
                    "launch": "CUDA graph of C-ABI calls",
                    "useful_gflop_per_step": round(flops / 1e9, 4),
-                   "algorithmic_mb_per_step": round(bytes_ / 1e6, 3)},
+                   "algorithmic_mb_per_step": round(bytes_ / 1e6, 3),
+                   "step_ms_dist": step_dist},
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -371,6 +379,23 @@ def run_gpu_arm(args, wl, world, rank, local):
         dist.barrier()
         del g_chunk, g_rem, g_run
         dist.destroy_process_group()
+
+
+def replay_distribution(replay, graph, steps_per_replay, stream, device, samples=50):
+    """Per-step time of `samples` replays of `graph`, each timed alone with
+    CUDA events on `stream`: median, min and 90th percentile in ms."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(samples)]
+    for a, b in evs:
+        a.record(stream)
+        replay(graph)
+        b.record(stream)
+    torch.cuda.synchronize(device)
+    per_step = sorted(a.elapsed_time(b) / steps_per_replay for a, b in evs)
+    p90 = per_step[min(len(per_step) - 1, int(round(0.9 * (len(per_step) - 1))))]
+    return {"median": round(statistics.median(per_step), 6), "min": round(per_step[0], 6),
+            "p90": round(p90, 6), "samples": samples}
 
 
 def run_e2e(args, wl, device, stream, max_global):
@@ -1141,11 +1166,34 @@ def run_cpu_baseline(wl, budget_s=10.0):
     for _ in range(reps):
         run_oracle_heads(oracle, x, wl, heads)
     dt = time.perf_counter() - t0
+    single = run_cpu_single_thread(wl, x, budget_s=max(1.0, budget_s / 4))
     return {"value": round(flops * reps / dt / 1e12, 6), "unit": UNIT,
             "cores": oracle.default().max_threads(), "kind": "oracle",
             "sample": f"{heads} of {wl.H} heads x {wl.B} batches, {reps} repetition(s), "
                       f"{dt:.1f} s, fp64 C oracle with OpenMP",
-            "seconds": round(dt, 2)}
+            "seconds": round(dt, 2), "single_thread": single}
+
+
+def run_cpu_single_thread(wl, x, budget_s=2.5):
+    """The oracle on one host thread, best of 3, on a block of rows of one
+    head sized to about budget_s / 3 per run."""
+    import oracle
+    from sparse_long_sequence_lf_b200 import accounting
+
+    def once(rows):
+        t0 = time.perf_counter()
+        oracle.forward(x["q"], x["k"], x["v"], x["qg"], x["kg"], x["vg"], x["local_mask"],
+                       x["global_mask"], window=wl.window, dilation=x["dilation"],
+                       causal=wl.causal, bh_range=(0, 1), row_range=(0, rows), threads=1)
+        return time.perf_counter() - t0
+
+    rows = min(wl.n, 256)
+    t = once(rows)
+    rows = max(1, min(wl.n, int(rows * (budget_s / 3) / max(t, 1e-4))))
+    best = min(once(rows) for _ in range(3))
+    flops = accounting.useful_flops_rows(wl, head=0, rows=(0, rows))
+    return {"value": round(flops / best / 1e12, 6), "unit": UNIT, "cores": 1,
+            "sample": f"rows 0..{rows} of batch 0 head 0, best of 3 ({best:.2f} s)"}
 
 
 def workload_config(wl, world):
@@ -1179,8 +1227,7 @@ def run_reference_arm(args, wl, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3 / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {**workload_config(wl, world),
-                   "sample": "a bounded number of heads per step (see cpu_baseline)"},
+        "config": workload_config(wl, world),
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,

@@ -194,6 +194,39 @@ LF_API int lf_attention_forward_host(lf_dtype dtype, int B, int H, int n, int d_
 LF_API int lf_workspace_status(const void *workspace, lf_stream_t stream);
 
 /*
+ * Test hooks of the bf16/fp16 attention kernel's bounded waits (failure
+ * detection; no counterpart in the method).  Every wait of the kernel on a
+ * shared-memory barrier gives up after a time limit, records
+ * LF_ERR_DEVICE_TIMEOUT in the workspace status word, lets the CTA's other
+ * roles stop, waits (bounded) for its own copies and products in flight,
+ * frees its tensor memory and returns.
+ *
+ *   wait_limit_ns   limit of every such wait, for the launches that follow
+ *                   (default 1 s; 0 is refused with LF_ERR_INVALID_ARG).
+ *   stall_first_q   nonzero: in later launches CTA 0 never loads the query
+ *                   tile of its first item and never signals it, so the wait
+ *                   for it runs out (no copy is started for it, nothing is
+ *                   left in flight).  0 restores normal launches.
+ *
+ * Process-wide settings read at each launch; not for concurrent use.  After a
+ * device-detected error the workspace must be prepared again
+ * (lf_attention_prepare or lf_attention_forward) before lf_attention_run.
+ */
+LF_API int lf_test_forward_hooks(unsigned long long wait_limit_ns, int stall_first_q);
+
+/*
+ * Evaluates, on the device, the 2^x approximation the bf16/fp16 attention
+ * kernel uses for part of its exponentials: x = j + f with j the nearest
+ * integer and f in [-1/2, 1/2], 2^f from a cubic fitted for minimum maximum
+ * relative error on that interval (Remez exchange), 2^j added to the
+ * exponent.  Relative error below 7.5e-5 for x >= -125.5; below that the
+ * result is a number in [0, 2^-124] (arguments below -126 are clamped).
+ *   x, y   device [n] fp32 (y = 2^x).  stream: as elsewhere.
+ * For testing the approximation against the SFU exponential and its bound.
+ */
+LF_API int lf_exp2_poly_eval(const float *x, float *y, int n, lf_stream_t stream);
+
+/*
  * Projection prologue (FasterTransformer Longformer Encoder guide, "compute
  * flow": the Q, K, V, Kg, Vg products over every token, the Qg product over
  * the global tokens only, then bias add and the split into heads).  Produces
@@ -283,9 +316,14 @@ LF_API int lf_output_layer(lf_dtype dtype, int B, int n, int H, int d_head,
  * LF_STATIC_SCRATCH_BYTES returns LF_ERR_SCRATCH_LIMIT before anything
  * touches the device (for example B = 1, H = 16, n = 16384 with 32 global
  * tokens needs about 4.5 MB).
+ * Invalid sizes (those for which lf_workspace_size returns 0) return
+ * LF_ERR_INVALID_ARG, and d_head != 64 LF_ERR_UNSUPPORTED, also before
+ * anything touches the device.
  * Set-up: the first call on a device looks up the scratch address
  * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture.
+ * first call before any stream capture.  The cached address does not survive
+ * cudaDeviceReset: a process that resets a device must not call this entry
+ * point on that device again.
  * Concurrency: there is one scratch per device, so calls on the same device
  * that overlap in time (several streams or host threads) race on it; callers
  * serialise them.  Nothing must be cleared beforehand: each call's

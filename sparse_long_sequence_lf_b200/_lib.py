@@ -70,6 +70,8 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         "lf_attention_forward_host": (I, [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P, I, P,
                                           P, Z, P, Z, P]),
         "lf_workspace_status": (I, [P, P]),
+        "lf_test_forward_hooks": (I, [ctypes.c_ulonglong, I]),
+        "lf_exp2_poly_eval": (I, [P, P, I, P]),
         "lf_attention_forward_static": (I, [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P, I, P,
                                             P, ctypes.POINTER(P)]),
         "lf_qkv_projection": (I, [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, P, P, P, P, P]),

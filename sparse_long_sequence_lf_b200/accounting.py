@@ -86,6 +86,22 @@ def useful_flops(wl: Workload) -> int:
     return 4 * wl.d * useful_pairs(wl)
 
 
+def useful_flops_rows(wl: Workload, head: int, rows: tuple, batch: int = 0) -> int:
+    """FLOPs of the attended pairs of rows [rows[0], rows[1]) of one (batch,
+    head): the same count as useful_flops, restricted to those rows."""
+    lm, gm = _masks_np(wl)
+    valid = lm[batch]
+    d = wl.dilation_list()[head]
+    per_row = _tap_counts(valid, wl.window, d, wl.causal)
+    per_row = per_row + _global_extra(valid, global_positions(wl)[batch], wl.window, d, wl.causal)
+    sel = np.zeros(wl.n, dtype=bool)
+    sel[rows[0]:rows[1]] = True
+    local_rows = sel & valid & ~gm[batch]
+    global_rows = sel & valid & gm[batch]
+    pairs = int(per_row[local_rows].sum()) + int(global_rows.sum()) * int(valid.sum())
+    return 4 * wl.d * pairs
+
+
 def algorithmic_bytes(wl: Workload) -> int:
     e = ELEM_BYTES[wl.dtype]
     full = wl.B * wl.H * wl.n * wl.d * e

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(BUILD, "liblf_attention.so")
-SOURCES = ["lf_api.cu", "lf_prepare.cu", "lf_simt.cu", "lf_tc.cu", "lf_static.cu", "lf_proj.cu",
+SOURCES = ["lf_api.cu", "lf_prepare.cu", "lf_simt.cu", "lf_fwd.cu", "lf_static.cu", "lf_proj.cu",
            "lf_bwd.cu", "lf_bwd_tc.cu", "lf_encoder.cu"]
 
 NVCC_FLAGS = [
@@ -56,8 +56,16 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     os.makedirs(BUILD, exist_ok=True)
     objs = []
     extra = ["-Xptxas", "-v"] if ptxas_verbose else []
+    headers = glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(ROOT, "include", "lf_attention.h")]
+    newest_header = max(os.path.getmtime(h) for h in headers)
     for src in SOURCES:
         obj = os.path.join(BUILD, os.path.splitext(src)[0] + ".o")
+        objs.append(obj)
+        # An object is rebuilt when its source or any shared header is newer.
+        if (not force and not ptxas_verbose and os.path.exists(obj)
+                and os.path.getmtime(obj) >= max(newest_header,
+                                                 os.path.getmtime(os.path.join(CSRC, src)))):
+            continue
         cmd = [nvcc(), *NVCC_FLAGS, *extra, "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
@@ -66,7 +74,6 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
             raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
         if ptxas_verbose or verbose:
             sys.stdout.write(r.stdout + r.stderr)
-        objs.append(obj)
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)

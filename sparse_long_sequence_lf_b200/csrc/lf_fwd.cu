@@ -1,0 +1,1373 @@
+// Tensor-core (tcgen05) attention forward for bf16 / fp16 inputs on sm_100a.
+//
+// What it computes ("LongFormer: The Long-Document Transformer" notes,
+// "Sliding Window", "Dilated Sliding Window", "Global Attention"; the notes
+// say the costly part is QK^T and that Longformer only computes a fixed
+// number of its diagonals with a banded product; FasterTransformer Longformer
+// Encoder guide, "compute flow": local rows softmax over window + global
+// tokens, global rows over the whole sequence, masked rows zeroed):
+//
+//   band items    128 query rows of one (batch, head, residue class of the
+//                 head's dilation).  A dilated head is a plain band over each
+//                 residue subsequence x[r::dil], so the same tile loop serves
+//                 every dilation.  The keys stream as 128-key tiles over the
+//                 band's diagonals, then as tiles of the (deduplicated) global
+//                 tokens; an online softmax runs over all of them.
+//   global items  up to 128 global rows of one (batch, head) against one
+//                 512-key chunk of Kg/Vg; each writes fp32 partials (max, sum,
+//                 unnormalised output).  While a row spans at most 8 chunks,
+//                 the warp that finishes the last chunk of a group of 32 rows
+//                 merges them by log-sum-exp into the output rows; beyond
+//                 that combine_kernel does, after this kernel.
+//
+// Schedule.  A persistent grid, one CTA per SM.  Items are handed out by a
+// device-wide atomic counter (band items first, the cheaper global items
+// last), so CTAs that finish early take more work.  Each CTA runs two item
+// "slots" at once; their softmax warpgroups alternate with the tensor core:
+// while slot 0 turns its scores into probabilities, the tensor core runs
+// slot 1's PV and next QK^T, and the other way round.
+//
+// Layout of one CTA (384 threads = 3 warpgroups):
+//   warps 0-3    softmax warpgroup of slot 0 (thread t owns query row t)
+//   warps 4-7    softmax warpgroup of slot 1
+//   warp  8      TMA producer of both slots: fetches items, decodes them,
+//                loads Q, K, V tiles, and precomputes each key tile's column
+//                masks (padding bits, global-token positions) in shared memory
+//   warp  9      MMA issuer of both slots (one elected thread), owns TMEM
+//   warps 10-11  idle (registers go to the softmax warpgroups)
+//
+// TMEM (512 columns, slot X uses [256X, 256X+256)): the 128-key score tile S
+// (fp32; the 16-bit probabilities P overwrite its first 64 columns as pairs)
+// and two 64-column output accumulators O, used by alternate items so that
+// the epilogue of item k (done by the softmax warps after the first tile of
+// item k+1) overlaps item k+1's products.
+//   S = Q K^T      tcgen05.mma kind::f16, A = Q (smem, K-major),
+//                  B = K tile (smem, K-major), 128x128 fp32 in TMEM
+//   O += P V       tcgen05.mma kind::f16, A = P (TMEM), B = V tile
+//                  (smem, MN-major), 128x64 fp32 in TMEM
+// Per slot and tile the MMA warp issues PV(j) then S(j+1): when the softmax
+// sees S(j+1) ready, every product before it (PV(j) included) is complete.
+// Shared-memory tiles have 128-byte rows with the 128-byte swizzle, written
+// by TMA: whole tiles from residue-class tensor maps (rows r, r+dil, ...),
+// single-row loads for global tokens, gathered Qg rows and heads beyond the
+// residue-map budget.  K/V tiles run through a 4-stage ring shared by the two
+// slots (filled and drained in the same alternating order).  Every wait on an
+// mbarrier is bounded; on expiry the kernel records LF_ERR_DEVICE_TIMEOUT,
+// drains its own copies and MMAs, frees its TMEM and returns.
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <type_traits>
+
+#include <cudaTypedefs.h>
+
+#include "../../include/lf_attention.h"
+#include "lf_sm100.cuh"
+
+namespace lf {
+
+using namespace sm100;
+
+constexpr int kRows = 128;                        // query rows per tile (M)
+constexpr int kTileKeys = 128;                    // keys per S tile (N) / K-V stage
+constexpr int kStages = 4;                        // K/V ring depth (shared by the slots)
+constexpr int kSlots = 2;
+constexpr int kRing = 4;                          // item and tile-info rings per slot
+constexpr int kQBytes = kRows * kDHead * 2;       // 16 KB of 16-bit elements
+constexpr int kKvBytes = kTileKeys * kDHead * 2;  // 16 KB
+constexpr int kRowBytes = kDHead * 2;             // 128 B
+constexpr int kThreads = 384;
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSlotCols = 256;               // S (128) | O0 (64) | O1 (64)
+constexpr float kRescaleLog2 = 8.f;               // lazy rescale: P stays below 2^8
+// Register split: the two softmax warpgroups take registers from the control
+// warpgroup: 256 * 208 + 128 * 80 = 63488 registers, which the launch (384
+// threads at the compiled count) must hold (checked on the host).
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsControl = 80;
+constexpr int kRegsNeeded = 2 * 128 * kRegsSoftmax + 128 * kRegsControl;
+// Of every 8 column pairs of a score tile, the pairs whose bit is set here
+// take 2^x from a cubic on the FMA pipe, the others from the SFU; the two
+// units then share the exponentials.
+constexpr uint32_t kPolyPairs = 0x49u;            // pairs 0, 3, 6 of each 8
+
+enum MapId { kMapKgTile, kMapVgTile, kMapQRow, kMapKRow, kMapVRow, kMapQgRow, kMapCount };
+
+// Residue-class tensor maps: for a head with dilation d, the rows r, r+d,
+// r+2d, ... of each (batch, head) slice form a plain sequence (row stride
+// d*128 B, first row r), so whole tiles of a dilated window load with one TMA
+// copy.  Up to kMaxResidues (dilation, residue) pairs per call; heads beyond
+// that load their rows one by one.
+constexpr int kMaxResidues = 24;
+constexpr int kMergeInKernelChunks = 8;           // longest sequence merged in-kernel: 4096
+constexpr int kBatchCache = 64;                   // per-batch counts / flags kept in smem
+
+struct FwdParams {
+    CUtensorMap maps[kMapCount];              // first: 64-byte aligned
+    CUtensorMap res_q[kMaxResidues];          // Q tiles of 128 rows
+    CUtensorMap res_k[kMaxResidues];          // K tiles of 128 rows
+    CUtensorMap res_v[kMaxResidues];          // V tiles of 128 rows
+    AttnArgs a;
+    int res_base[kMaxHeads];  // residue map of (head h, residue 0); -1: load rows one by one
+    int band_items;       // B * band_items_per_batch, numbered first
+    int total_items;      // + B*H*gtiles*nchunks global items
+    int gtiles;           // ceil(max_global / 128)
+    int oob_row;          // a row coordinate past the end of the row maps (reads zeros)
+    int n_res;            // residue maps in use
+    int merge_in_kernel;  // global rows merged by the last chunk (else by combine_kernel)
+    unsigned long long wait_ns;   // limit of every bounded wait
+    int stall_first_q;    // test hook: CTA 0 never loads slot 0's first Q tile
+};
+
+// Kernel arguments above 4 KB need CUDA 12.1 or newer (up to 32764 bytes).
+static_assert(sizeof(FwdParams) <= 32000, "kernel arguments exceed the parameter space");
+
+// An item as the producer decodes it; read by the MMA warp and the softmax
+// warpgroup of the slot.
+struct ItemInfo {
+    int kind;       // 0: no more items, 1 band, 2 global rows
+    int b, h, bh, dil, r, n_r;
+    int q0;         // band: first residue-space row; global: first global slot
+    int klo;        // first key of tile 0 (residue space for band items)
+    int nkv;        // key tiles before the global-column tiles
+    int ntiles;
+    int key_end;    // global items: end of the key chunk
+    int g;          // global tokens of the batch (clamped to max_global)
+    int chunk;
+    int has_pad;
+    int pad_[1];
+};
+static_assert(sizeof(ItemInfo) == 64, "item record size");
+
+// Column masks of one key tile, written by the producer: bits of the keys
+// that exist and are not padding; for a global-column tile also the token
+// position of each column (-1 past the count).
+struct TileMask {
+    uint32_t bits[4];
+    int jpos[kTileKeys];
+};
+
+struct __align__(1024) FwdSmem {
+    uint8_t q[kSlots][2][kQBytes];
+    uint8_t k[kStages][kKvBytes];
+    uint8_t v[kStages][kKvBytes];
+    TileMask tmask[kSlots][kRing];
+    ItemInfo items[kSlots][kRing];
+    uint64_t q_full[kSlots][2], q_empty[kSlots][2];
+    uint64_t kv_full[kStages], kv_empty[kStages];
+    uint64_t item_full[kSlots][kRing], item_empty[kSlots][kRing];
+    uint64_t tm_full[kSlots][kRing];
+    uint64_t s_full[kSlots], p_full[kSlots], o_full[kSlots][2], o_empty[kSlots][2];
+    uint64_t drain;
+    int batch_count[kBatchCache];
+    int batch_flags[kBatchCache];
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+constexpr size_t kFwdSmemBytes = sizeof(FwdSmem) + 1024;
+static_assert(kFwdSmemBytes <= 232448, "shared memory per CTA");
+
+// ------------------------------------------------------------ small helpers
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                             int *status, uint64_t limit_ns)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    uint32_t spins = 0;
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((++spins & 31u) == 0u) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > limit_ns) {
+                set_status(status, kErrDeviceTimeout);
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// Bounded wait taken by a whole warp: either every lane goes on or every lane
+// gives up, so no warp-collective instruction runs with a partial warp.
+__device__ __forceinline__ bool warp_wait(const FwdParams &p, FwdSmem &sm, uint64_t *bar,
+                                          uint32_t parity)
+{
+    const bool ok = wait_bounded(bar, parity, &sm.abort_flag, p.a.ws.status, p.wait_ns);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Waits (bounded, ignoring the abort flag) for a copy this CTA started, so
+// that nothing lands in shared memory after the CTA has exited.
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < limit_ns) {
+    }
+}
+
+__device__ __forceinline__ void advance_ring(int &stage, uint32_t &phase)
+{
+    if (++stage == kStages) {
+        stage = 0;
+        phase ^= 1u;
+    }
+}
+
+// Keys of the tile (N of QK^T, K of PV): 128, or the global tokens of a
+// global-column tile rounded up to a multiple of 16.
+__device__ __forceinline__ int tile_cols(const ItemInfo &I, int t)
+{
+    if (I.kind != 1 || t < I.nkv) return kTileKeys;
+    const int left = min(kTileKeys, I.g - (t - I.nkv) * kTileKeys);
+    return (left + 15) & ~15;
+}
+
+__device__ __forceinline__ int batch_count(const FwdSmem &sm, const AttnArgs &a, int b)
+{
+    return b < kBatchCache ? sm.batch_count[b] : a.ws.counts[b];
+}
+
+__device__ __forceinline__ int batch_flags(const FwdSmem &sm, const AttnArgs &a, int b)
+{
+    return b < kBatchCache ? sm.batch_flags[b] : a.ws.flags[b];
+}
+
+__device__ __forceinline__ ItemInfo decode_item(const FwdParams &p, const FwdSmem &sm, int item)
+{
+    const AttnArgs &a = p.a;
+    ItemInfo I;
+    I.pad_[0] = 0;
+    if (item < p.band_items) {
+        int tile;
+        band_item(a, item, I.b, I.h, I.r, tile);
+        I.kind = 1;
+        I.bh = I.b * a.H + I.h;
+        I.dil = a.dil[I.h];
+        I.n_r = (a.n - I.r + I.dil - 1) / I.dil;
+        I.q0 = tile * kRows;
+        const int rows_hi = min(I.q0 + kRows - 1, I.n_r - 1);
+        const int lo = max(I.q0 - (a.causal ? a.window - 1 : a.half), 0);
+        const int hi = min(rows_hi + (a.causal ? 0 : a.half), I.n_r - 1);
+        I.klo = lo;
+        I.nkv = (hi - lo + kTileKeys) / kTileKeys;
+        I.key_end = 0;
+        I.g = min(batch_count(sm, a, I.b), a.max_global);
+        I.chunk = 0;
+        I.ntiles = I.nkv + (I.g + kTileKeys - 1) / kTileKeys;
+    } else {
+        const int gi = item - p.band_items;
+        const int per_bh = p.gtiles * a.L.nchunks;
+        I.bh = gi / per_bh;
+        const int rem = gi - I.bh * per_bh;
+        const int gtile = rem / a.L.nchunks;
+        I.chunk = rem - gtile * a.L.nchunks;
+        I.b = I.bh / a.H;
+        I.h = I.bh - I.b * a.H;
+        I.kind = 2;
+        I.dil = 1;
+        I.r = 0;
+        I.n_r = a.n;
+        I.g = min(batch_count(sm, a, I.b), a.max_global);
+        I.q0 = gtile * kRows;
+        I.klo = I.chunk * kChunkKeys;
+        I.key_end = min(a.n, I.klo + kChunkKeys);
+        I.nkv = (I.key_end - I.klo + kTileKeys - 1) / kTileKeys;
+        I.ntiles = (I.g > I.q0) ? I.nkv : 0;   // 0: no global row in this tile: skipped
+    }
+    I.has_pad = batch_flags(sm, a, I.b) & kFlagHasPadding;
+    return I;
+}
+
+// ------------------------------------------------------------ producer
+struct ProducerSlot {
+    ItemInfo I;
+    int t;          // next tile of the item
+    int k;          // items fetched so far (ring position of the next one)
+    int jt;         // tiles produced so far
+    bool active;
+};
+
+// Fetches the next item of slot X from the device-wide counter, writes its
+// record to the slot's item ring and loads its Q tile.  Returns false on abort.
+__device__ __forceinline__ bool producer_fetch(const FwdParams &p, FwdSmem &sm, ProducerSlot &S, int X,
+                                            int lane, int *sched, int *finished, uint32_t &q_armed,
+                                            uint32_t &q_par)
+{
+    const AttnArgs &a = p.a;
+    ItemInfo I;
+    I.kind = 0;
+    for (;;) {
+        int idx = 0;
+        if (lane == 0) idx = atomicAdd(sched, 1);
+        idx = __shfl_sync(0xffffffffu, idx, 0);
+        if (idx >= p.total_items) {
+            // Every producer meets the end once per slot; the last one resets
+            // the counters for the next launch on this workspace.
+            if (lane == 0) {
+                __threadfence();
+                if (atomicAdd(finished, 1) == int(2 * gridDim.x) - 1) {
+                    atomicExch(sched, 0);
+                    atomicExch(finished, 0);
+                }
+            }
+            I.kind = 0;
+            break;
+        }
+        I = decode_item(p, sm, idx);
+        if (I.ntiles > 0) break;
+    }
+    const int k = S.k;
+    const int rs = k % kRing;
+    if (!warp_wait(p, sm, &sm.item_empty[X][rs], (uint32_t(k / kRing) & 1u) ^ 1u)) return false;
+    if (I.kind != 0) {
+        const int qb = k & 1;
+        const uint32_t use = uint32_t(k >> 1);
+        if (!warp_wait(p, sm, &sm.q_empty[X][qb], (use & 1u) ^ 1u)) return false;
+        uint8_t *qd = sm.q[X][qb];
+        uint64_t *qbar = &sm.q_full[X][qb];
+        const bool stall = p.stall_first_q && blockIdx.x == 0 && X == 0 && k == 0;
+        if (!stall) {
+            const int rb = I.kind == 1 ? p.res_base[I.h] : -1;
+            if (rb >= 0) {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(qbar, kQBytes);
+                    tma_load_3d(qd, &p.res_q[rb + I.r], qbar, 0, I.q0, I.bh);
+                }
+            } else if (I.kind == 1) {
+                if (lane == 0) mbar_arrive_expect_tx(qbar, kQBytes);
+                __syncwarp();
+                for (int rr = lane; rr < kRows; rr += 32) {
+                    const int ir = I.q0 + rr;
+                    const int y = ir < I.n_r ? I.bh * a.n + ir * I.dil + I.r : p.oob_row;
+                    tma_load_2d(qd + rr * kRowBytes, &p.maps[kMapQRow], qbar, 0, y);
+                }
+            } else {
+                // Only the rows of real global tokens: a query row only feeds
+                // its own output row, and rows past the count are never stored.
+                const int rows = min(kRows, I.g - I.q0);
+                if (lane == 0) mbar_arrive_expect_tx(qbar, rows * kRowBytes);
+                __syncwarp();
+                for (int rr = lane; rr < rows; rr += 32) {
+                    const int y = I.bh * a.n + a.ws.gidx[size_t(I.b) * a.n + I.q0 + rr];
+                    tma_load_2d(qd + rr * kRowBytes, &p.maps[kMapQgRow], qbar, 0, y);
+                }
+            }
+            // Bit 2X + qb: a Q copy of that buffer was started; its parity.
+            const uint32_t bit = 1u << (2 * X + qb);
+            q_armed |= bit;
+            q_par = (use & 1u) ? (q_par | bit) : (q_par & ~bit);
+        }
+    }
+    if (lane == 0) sm.items[X][rs] = I;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.item_full[X][rs]);
+    S.I = I;
+    S.t = 0;
+    S.k = k + 1;
+    S.active = I.kind != 0;
+    return true;
+}
+
+// Loads tile S.t of the slot's item into ring stage `stage` and writes its
+// column masks to the slot's tile-mask ring.
+__device__ __forceinline__ void producer_tile(const FwdParams &p, FwdSmem &sm, ProducerSlot &S,
+                                              int X, int lane, int stage)
+{
+    const AttnArgs &a = p.a;
+    const ItemInfo &I = S.I;
+    const int t = S.t;
+    uint8_t *kd = sm.k[stage];
+    uint8_t *vd = sm.v[stage];
+    uint64_t *bar = &sm.kv_full[stage];
+    TileMask &tm = sm.tmask[X][S.jt % kRing];
+    const uint32_t *vb = a.ws.vbits + size_t(I.b) * a.L.nwords;
+    if (I.kind == 2) {
+        const int k0 = I.klo + t * kTileKeys;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int j = k0 + 32 * w + lane;
+            const bool ok = j < I.key_end && (!I.has_pad || bit_at(vb, j));
+            const uint32_t bits = __ballot_sync(0xffffffffu, ok);
+            if (lane == 0) tm.bits[w] = bits;
+        }
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar, 2 * kKvBytes);
+            tma_load_3d(kd, &p.maps[kMapKgTile], bar, 0, k0, I.bh);
+            tma_load_3d(vd, &p.maps[kMapVgTile], bar, 0, k0, I.bh);
+        }
+    } else if (t < I.nkv) {
+        const int k0 = I.klo + t * kTileKeys;
+        if (I.has_pad) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const int jr = k0 + 32 * w + lane;
+                const bool ok = jr < I.n_r && bit_at(vb, jr * I.dil + I.r);
+                const uint32_t bits = __ballot_sync(0xffffffffu, ok);
+                if (lane == 0) tm.bits[w] = bits;
+            }
+        } else if (lane < 4) {
+            tm.bits[lane] = 0xffffffffu;
+        }
+        const int rb = p.res_base[I.h];
+        if (rb >= 0) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar, 2 * kKvBytes);
+                tma_load_3d(kd, &p.res_k[rb + I.r], bar, 0, k0, I.bh);
+                tma_load_3d(vd, &p.res_v[rb + I.r], bar, 0, k0, I.bh);
+            }
+        } else {
+            if (lane == 0) mbar_arrive_expect_tx(bar, 2 * kKvBytes);
+            __syncwarp();
+            for (int rr = lane; rr < kTileKeys; rr += 32) {
+                const int jr = k0 + rr;
+                const int y = jr < I.n_r ? I.bh * a.n + jr * I.dil + I.r : p.oob_row;
+                tma_load_2d(kd + rr * kRowBytes, &p.maps[kMapKRow], bar, 0, y);
+                tma_load_2d(vd + rr * kRowBytes, &p.maps[kMapVRow], bar, 0, y);
+            }
+        }
+    } else {
+        // Global-token columns: the K/V rows of the global tokens, gathered.
+        const int s0 = (t - I.nkv) * kTileKeys;
+        const int rows = tile_cols(I, t);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const int c = 32 * w + lane;
+            const int slot = s0 + c;
+            const int j = slot < I.g ? a.ws.gidx[size_t(I.b) * a.n + slot] : -1;
+            tm.jpos[c] = j;
+            const bool ok = j >= 0 && bit_at(vb, j);
+            const uint32_t bits = __ballot_sync(0xffffffffu, ok);
+            if (lane == 0) tm.bits[w] = bits;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(bar, 2 * rows * kRowBytes);
+        __syncwarp();
+        for (int rr = lane; rr < rows; rr += 32) {
+            const int slot = s0 + rr;
+            const int y = slot < I.g ? I.bh * a.n + a.ws.gidx[size_t(I.b) * a.n + slot]
+                                     : p.oob_row;
+            tma_load_2d(kd + rr * kRowBytes, &p.maps[kMapKRow], bar, 0, y);
+            tma_load_2d(vd + rr * kRowBytes, &p.maps[kMapVRow], bar, 0, y);
+        }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.tm_full[X][S.jt % kRing]);
+}
+
+__device__ __forceinline__ void producer_role(const FwdParams &p, FwdSmem &sm, int lane)
+{
+    int *sched = p.a.ws.status + 16;
+    int *finished = p.a.ws.status + 32;
+    ProducerSlot S[kSlots];
+    uint32_t kv_armed = 0, kv_par = 0;   // bit s: stage s was filled; its parity
+    uint32_t qa = 0, qp = 0;             // bit 2X+b: Q buffer b of slot X was filled
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+#pragma unroll
+    for (int X = 0; X < kSlots; ++X) {
+        S[X].k = 0;
+        S[X].jt = 0;
+        S[X].active = false;
+        if (ok) ok = producer_fetch(p, sm, S[X], X, lane, sched, finished, qa, qp);
+    }
+    while (ok && (S[0].active || S[1].active)) {
+#pragma unroll
+        for (int X = 0; X < kSlots; ++X) {
+            if (!ok || !S[X].active) continue;
+            if (!warp_wait(p, sm, &sm.kv_empty[stage], phase ^ 1u)) {
+                ok = false;
+                break;
+            }
+            producer_tile(p, sm, S[X], X, lane, stage);
+            kv_armed |= 1u << stage;
+            kv_par = phase ? (kv_par | (1u << stage)) : (kv_par & ~(1u << stage));
+            advance_ring(stage, phase);
+            ++S[X].jt;
+            if (++S[X].t == S[X].I.ntiles)
+                ok = producer_fetch(p, sm, S[X], X, lane, sched, finished, qa, qp);
+        }
+    }
+    if (!ok || sm.abort_flag) {
+        for (int s = 0; s < kStages; ++s)
+            if ((kv_armed >> s) & 1u) drain_wait(&sm.kv_full[s], (kv_par >> s) & 1u, p.wait_ns);
+        for (int X = 0; X < kSlots; ++X)
+            for (int b = 0; b < 2; ++b)
+                if ((qa >> (2 * X + b)) & 1u)
+                    drain_wait(&sm.q_full[X][b], (qp >> (2 * X + b)) & 1u, p.wait_ns);
+    }
+}
+
+// ------------------------------------------------------------ MMA issuer
+struct MmaSlot {
+    ItemInfo I;
+    int t, k, j;    // tile of the item, items taken, tiles issued
+    int stage;      // ring stage of the tile whose S was issued last
+    bool active;
+};
+
+__device__ __forceinline__ bool mma_next_item(const FwdParams &p, FwdSmem &sm, MmaSlot &S, int X)
+{
+    const int rs = S.k % kRing;
+    if (!warp_wait(p, sm, &sm.item_full[X][rs], uint32_t(S.k / kRing) & 1u)) return false;
+    S.I = sm.items[X][rs];
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.item_empty[X][rs]);
+    S.active = S.I.kind != 0;
+    S.t = 0;
+    return true;
+}
+
+// Issues S = Q K^T of the slot's current tile; returns false on abort.
+__device__ __forceinline__ bool mma_issue_s(const FwdParams &p, FwdSmem &sm, MmaSlot &S, int X,
+                                            uint32_t tmem, uint32_t id_s, int &stage,
+                                            uint32_t &phase)
+{
+    const int kq = S.k - 1;   // index of the current item
+    if (S.t == 0 &&
+        !warp_wait(p, sm, &sm.q_full[X][kq & 1], uint32_t(kq >> 1) & 1u))
+        return false;
+    if (!warp_wait(p, sm, &sm.kv_full[stage], phase)) return false;
+    tc_fence_after();
+    const int N = tile_cols(S.I, S.t);
+    const uint32_t tS = tmem + X * kSlotCols;
+    const uint64_t qdesc = make_sdesc(smem_u32(sm.q[X][kq & 1]), 16, 1024);
+    const uint64_t kdesc = make_sdesc(smem_u32(sm.k[stage]), 16, 1024);
+    const uint32_t idesc = id_s | (uint32_t(N >> 3) << 17);
+#pragma unroll
+    for (int kk = 0; kk < kDHead / 16; ++kk)
+        mma_ss_elect(tS, qdesc + uint64_t((kk * 32) >> 4), kdesc + uint64_t((kk * 32) >> 4), idesc,
+                     kk > 0 ? 1u : 0u);
+    tc_commit_elect(&sm.s_full[X]);
+    if (S.t == S.I.ntiles - 1) tc_commit_elect(&sm.q_empty[X][kq & 1]);
+    __syncwarp();
+    S.stage = stage;
+    advance_ring(stage, phase);
+    return true;
+}
+
+__device__ __forceinline__ void mma_role(const FwdParams &p, FwdSmem &sm, uint32_t tmem, bool bf16)
+{
+    const uint32_t id_s = make_idesc(128, 0, bf16, false);
+    const uint32_t id_pv = make_idesc(128, 64, bf16, true);
+    MmaSlot S[kSlots];
+    int stage = 0;
+    uint32_t phase = 0;
+#pragma unroll
+    for (int X = 0; X < kSlots; ++X) {
+        S[X].k = 0;
+        S[X].j = 0;
+        S[X].active = false;
+        if (!mma_next_item(p, sm, S[X], X)) return;
+        ++S[X].k;
+    }
+#pragma unroll
+    for (int X = 0; X < kSlots; ++X)
+        if (S[X].active && !mma_issue_s(p, sm, S[X], X, tmem, id_s, stage, phase)) return;
+    for (;;) {
+        bool any = false;
+#pragma unroll
+        for (int X = 0; X < kSlots; ++X) {
+            MmaSlot &s = S[X];
+            if (!s.active) continue;
+            any = true;
+            const int kq = s.k - 1;
+            const int ob = kq & 1;
+            if (!warp_wait(p, sm, &sm.p_full[X], uint32_t(s.j) & 1u)) return;
+            // The first PV of an item overwrites its O buffer: the epilogue of
+            // the item two before must have read it.
+            if (s.t == 0 && kq >= 2 &&
+                !warp_wait(p, sm, &sm.o_empty[X][ob], uint32_t((kq >> 1) - 1) & 1u))
+                return;
+            tc_fence_after();
+            {
+                const uint32_t tP = tmem + X * kSlotCols;
+                const uint32_t tO = tP + 128 + ob * 64;
+                const uint64_t vdesc = make_sdesc(smem_u32(sm.v[s.stage]), 16, 1024);
+                const int ksteps = tile_cols(s.I, s.t) >> 4;
+                for (int kk = 0; kk < ksteps; ++kk)
+                    mma_ts_elect(tO, tP + kk * 8, vdesc + uint64_t((kk * 2048) >> 4), id_pv,
+                                 (kk > 0 || s.t > 0) ? 1u : 0u);
+                tc_commit_elect(&sm.kv_empty[s.stage]);
+                if (s.t == s.I.ntiles - 1) tc_commit_elect(&sm.o_full[X][ob]);
+            }
+            __syncwarp();
+            ++s.j;
+            if (++s.t == s.I.ntiles) {
+                if (!mma_next_item(p, sm, s, X)) return;
+                ++s.k;
+                if (!s.active) continue;
+            }
+            if (!mma_issue_s(p, sm, s, X, tmem, id_s, stage, phase)) return;
+        }
+        if (!any) break;
+    }
+}
+
+// ------------------------------------------------------------ softmax
+template <typename T> __device__ __forceinline__ uint32_t pack2(float lo, float hi);
+template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+template <> __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi)
+{
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Bits of the columns [32q, 32q + 32) that lie inside [clo, chi].
+__device__ __forceinline__ uint32_t range_bits(int q, int clo, int chi)
+{
+    const int lo = min(max(clo - 32 * q, 0), 32);
+    const int hi = min(max(chi - 32 * q + 1, 0), 32);
+    const uint32_t below_hi = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+    const uint32_t below_lo = lo >= 32 ? 0xffffffffu : ((1u << lo) - 1u);
+    return below_hi & ~below_lo;
+}
+
+// Maximum of 32 values as a shallow tree of 3-input maxima.
+__device__ __forceinline__ float max32(const float *s)
+{
+    float t[11];
+#pragma unroll
+    for (int i = 0; i < 10; ++i) t[i] = max3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
+    t[10] = fmaxf(s[30], s[31]);
+    const float u0 = max3(t[0], t[1], t[2]);
+    const float u1 = max3(t[3], t[4], t[5]);
+    const float u2 = max3(t[6], t[7], t[8]);
+    return max3(u0, u1, max3(u2, t[9], t[10]));
+}
+
+// 2^x for a pair of arguments on the FMA pipe.  x = j + f with j = round(x)
+// (the 1.5*2^23 addition rounds to an integer in the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f is a cubic fitted to minimise the maximum relative
+// error on [-1/2, 1/2] (Remez exchange, error below 7.5e-5); 2^j is added to
+// the exponent field.  That holds for x >= -125.5; below, the exponent field
+// leaves the normal range and the result is only a number in [0, 2^-124]
+// (arguments below -126 are clamped), which is zero for every use here.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float &y0, float &y1)
+{
+    constexpr float kRound = 12582912.f;     // 1.5 * 2^23
+    constexpr float c0 = 0.999928074f, c1 = 0.693260985f, c2 = 0.242611122f,
+                    c3 = 0.0551716691f;
+    x0 = fmaxf(x0, -126.f);
+    x1 = fmaxf(x1, -126.f);
+    float t0, t1, j0, j1, f0, f1, p0, p1;
+    add2(t0, t1, x0, x1, kRound, kRound);
+    add2(j0, j1, t0, t1, -kRound, -kRound);
+    fma2(f0, f1, j0, j1, -1.f, -1.f, x0, x1);
+    fma2(p0, p1, f0, f1, c3, c3, c2, c2);
+    fma2(p0, p1, p0, p1, f0, f1, c1, c1);
+    fma2(p0, p1, p0, p1, f0, f1, c0, c0);
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+__global__ void exp2_poly_kernel(const float *x, float *y, int n)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (2 * i + 1 < n) {
+        exp2_poly2(x[2 * i], x[2 * i + 1], y[2 * i], y[2 * i + 1]);
+    } else if (2 * i < n) {
+        float y1;
+        exp2_poly2(x[2 * i], 0.f, y[2 * i], y1);
+    }
+}
+
+struct RowState {
+    float m, l;
+};
+
+// Online softmax of one 128-key score tile for this thread's row.  mw[c]
+// marks the keys of this row among columns [32c, 32c+32); a chunk that is
+// empty for every row of the warp is skipped (its probabilities are zero)
+// and a chunk that is full for every row is not masked.  Writes P =
+// 2^(S*scale*log2e - m) as 16-bit pairs over the first 64 columns of the tile
+// and adds the row sum.  O is rescaled in TMEM only when the running maximum
+// grows by more than 2^8; every PV before this tile has completed then.
+template <typename T>
+__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, RowState &st, bool first,
+                                             const uint32_t (&mw)[4], float sl2)
+{
+    uint32_t any_m = 0, full_m = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        any_m |= (__any_sync(0xffffffffu, mw[c] != 0u) ? 1u : 0u) << c;
+        full_m |= (__all_sync(0xffffffffu, mw[c] == 0xffffffffu) ? 1u : 0u) << c;
+    }
+    float s[128];
+    tmem_ld128(tS, s);
+    float mc[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        mc[c] = -INFINITY;
+        if ((any_m >> c) & 1u) {
+            if (!((full_m >> c) & 1u)) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    s[32 * c + i] = ((mw[c] >> i) & 1u) ? s[32 * c + i] : -INFINITY;
+            }
+            mc[c] = max32(&s[32 * c]);
+        }
+    }
+    const float mt = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])) * sl2;
+    float alpha = 1.f;
+    bool rescale = false;
+    if (first) {
+        st.m = mt;
+        st.l = 0.f;
+    } else if (mt > st.m + kRescaleLog2) {
+        alpha = ex2(st.m - mt);
+        st.m = mt;
+        rescale = true;
+    }
+    const float nb = (st.m == -INFINITY) ? 0.f : -st.m;
+    float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
+    // Two halves of 64 keys: each half's 32 packed columns are stored as soon
+    // as they are ready, which bounds the registers held at once.
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * h + cc;
+            if ((any_m >> c) & 1u) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int q = 16 * c + i;
+                    float x0, x1, p0, p1;
+                    fma2(x0, x1, s[2 * q], s[2 * q + 1], sl2, sl2, nb, nb);
+                    if ((kPolyPairs >> (q & 7)) & 1u) {
+                        exp2_poly2(x0, x1, p0, p1);
+                    } else {
+                        p0 = ex2(x0);
+                        p1 = ex2(x1);
+                    }
+                    if (i & 1)
+                        add2(sb0, sb1, sb0, sb1, p0, p1);
+                    else
+                        add2(sa0, sa1, sa0, sa1, p0, p1);
+                    pk[16 * cc + i] = pack2<T>(p0, p1);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[16 * cc + i] = 0u;
+            }
+        }
+        tmem_st32(tS + 32 * h, pk);
+    }
+    if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float o[32];
+            tmem_ld32(tO + half * 32, o);
+            uint32_t ob[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) ob[x] = __float_as_uint(o[x] * alpha);
+            tmem_st32(tO + half * 32, ob);
+        }
+    }
+    st.l = st.l * alpha + ((sa0 + sa1) + (sb0 + sb1));
+    tmem_st_wait();
+}
+
+template <typename T>
+__device__ __forceinline__ void store_half_row(T *dst, const float (&o)[32], float inv)
+{
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 v;
+        v.x = pack2<T>(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
+        v.y = pack2<T>(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
+        v.z = pack2<T>(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
+        v.w = pack2<T>(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+        d4[q] = v;
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void store_row(T *dst, const float (&o)[64], float inv)
+{
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        uint4 v;
+        v.x = pack2<T>(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
+        v.y = pack2<T>(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
+        v.z = pack2<T>(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
+        v.w = pack2<T>(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+        d4[q] = v;
+    }
+}
+
+// Merges the chunk partials of the global rows slot0 .. slot0 + 31 (lane =
+// row) by log-sum-exp and writes their output rows.  Called by the warp that
+// wrote the last chunk of the group; the partials of the other chunks come
+// from other CTAs, so they are read past L1.
+template <typename T>
+__device__ __noinline__ void merge_global_rows(const AttnArgs &a, int b, int bh, int g, int slot0,
+                                               int lane)
+{
+    const int slot = slot0 + lane;
+    if (slot >= g) return;
+    const int pos = a.ws.gidx[size_t(b) * a.n + slot];
+    if (!bit_at(a.ws.vbits + size_t(b) * a.L.nwords, pos)) return;   // padded: zeros elsewhere
+    const size_t mg = size_t(a.max_global);
+    const size_t cstride = kPartialFloats * mg;
+    const float *P = partial_base(a, bh, 0) + slot;
+    const int nch = a.L.nchunks;
+    float M = -INFINITY;
+    for (int c = 0; c < nch; ++c) M = fmaxf(M, __ldcg(P + c * cstride));
+    float L = 0.f, acc[kDHead];
+#pragma unroll
+    for (int x = 0; x < kDHead; ++x) acc[x] = 0.f;
+    for (int c = 0; c < nch; ++c) {
+        const float *pc = P + c * cstride;
+        const float mc = __ldcg(pc);
+        const float f = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+        L = fmaf(f, __ldcg(pc + mg), L);
+#pragma unroll
+        for (int x = 0; x < kDHead; ++x) acc[x] = fmaf(f, __ldcg(pc + (2 + x) * mg), acc[x]);
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    store_row<T>(static_cast<T *>(a.out) + (size_t(bh) * a.n + pos) * kDHead, acc, inv);
+}
+
+// Per-row results an item's epilogue needs after the softmax has moved on;
+// the item's record stays in the slot's item ring until the epilogue is done.
+struct RowOut {
+    float m, l;
+    bool write;     // band: the row exists and is not a valid global row
+    bool valid;     // band: the row is not padding
+};
+
+// Writes the output of item `ke` of slot X: band rows O / l (zeros for padded
+// rows); for global rows the chunk partials, and the merge when this is the
+// last chunk of a group.  O is complete (o_full); the O buffer and the item's
+// ring entry are released afterwards.
+template <typename T>
+__device__ __forceinline__ void epilogue(const FwdParams &p, FwdSmem &sm, uint32_t tmem_row, int X,
+                                         int ke, const RowOut &ro, int tid)
+{
+    const AttnArgs &a = p.a;
+    const int warp = tid >> 5, lane = tid & 31;
+    const ItemInfo &I = sm.items[X][ke % kRing];
+    const int kind = I.kind, bh = I.bh, q0 = I.q0;
+    const int ob = ke & 1;
+    const uint32_t tO = tmem_row + X * kSlotCols + 128 + ob * 64;
+    const int row = q0 + tid;
+    const bool active = kind == 2 ? q0 + warp * 32 < I.g : q0 + warp * 32 < I.n_r;
+    if (active) {
+        if (kind == 1) {
+            const int pos = ro.write ? row * I.dil + I.r : 0;
+            T *dst = static_cast<T *>(a.out) + (size_t(bh) * a.n + pos) * kDHead;
+            const float inv = ro.valid ? 1.f / ro.l : 0.f;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float o[32];
+                tmem_ld32(tO + half * 32, o);
+                if (ro.write) store_half_row<T>(dst + half * 32, o, inv);
+            }
+        } else {
+            const int slot = row;
+            const size_t mg = size_t(a.max_global);
+            float *P = a.ws.partials + (size_t(bh) * a.L.nchunks + I.chunk) * kPartialFloats * mg +
+                       min(slot, a.max_global - 1);
+            const bool write = slot < I.g;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float o[32];
+                tmem_ld32(tO + half * 32, o);
+                if (write) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) P[(2 + half * 32 + x) * mg] = o[x];
+                }
+            }
+            if (write) {
+                P[0] = ro.m;
+                P[mg] = ro.l;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.o_empty[X][ob]);
+    if (kind == 2 && active && p.merge_in_kernel) {
+        // The last chunk to finish this warp's group of 32 global rows merges
+        // them and resets the group's arrival counter for the next call on the
+        // same workspace.
+        const int group = (q0 >> 5) + warp;
+        const int b = I.b, g = I.g;
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+            int *ctr = a.ws.counters + size_t(bh) * (a.L.ngroups + 1) + group;
+            last = atomicAdd(ctr, 1) == a.L.nchunks - 1;
+            if (last) atomicExch(ctr, 0);
+        }
+        if (__shfl_sync(0xffffffffu, last, 0)) {
+            __threadfence();
+            merge_global_rows<T>(a, b, bh, g, group * 32, lane);
+        }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.item_empty[X][ke % kRing]);
+}
+
+// Column masks of this thread's row for one tile: mw[c] marks the keys of
+// the row among columns [32c, 32c + 32).
+__device__ __forceinline__ void tile_row_mask(const AttnArgs &a, const ItemInfo &I, const TileMask &tm,
+                                              int t, int row, int lane, uint32_t (&mw)[4])
+{
+    if (I.kind == 2) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) mw[c] = tm.bits[c];
+    } else if (t < I.nkv) {
+        const int k0 = I.klo + t * kTileKeys;
+        const int lo = max(row - (a.causal ? a.window - 1 : a.half), 0);
+        const int hi = min(row + (a.causal ? 0 : a.half), I.n_r - 1);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) mw[c] = range_bits(c, lo - k0, hi - k0) & tm.bits[c];
+    } else {
+        // Global-token columns: real, unpadded tokens that are not already
+        // window taps of this row.  A tap shares the row's residue class and
+        // lies within the (dilated) window span; only tokens near the warp's
+        // rows are tested.
+        const int i = row * I.dil + I.r;
+        const int span = a.half * I.dil;
+        const int i_lo = __shfl_sync(0xffffffffu, i, 0) - span;
+        const int i_hi = __shfl_sync(0xffffffffu, i, 31) + span;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t m = tm.bits[c];
+            const int jl = tm.jpos[32 * c + lane];
+            const bool near = jl >= i_lo && jl <= i_hi && (jl % I.dil) == I.r;
+            uint32_t cand = __ballot_sync(0xffffffffu, near) & m;
+            while (cand) {
+                const int col = __ffs(cand) - 1;
+                cand &= cand - 1u;
+                const int d = __shfl_sync(0xffffffffu, jl, col) - i;
+                if (d >= -span && d <= span) m &= ~(1u << col);
+            }
+            mw[c] = m;
+        }
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, uint32_t tmem, int X,
+                                             int tid)
+{
+    const AttnArgs &a = p.a;
+    const int warp = tid >> 5, lane = tid & 31;
+    const uint32_t tmem_row = tmem + (uint32_t(warp * 32) << 16);
+    const uint32_t tS = tmem_row + X * kSlotCols;
+    const float sl2 = a.scale_log2;
+    int k = 0;      // items taken
+    int jt = 0;     // tiles taken
+    RowOut pend;
+    bool pending = false;
+
+    for (;;) {
+        const int rs = k % kRing;
+        if (!warp_wait(p, sm, &sm.item_full[X][rs], uint32_t(k / kRing) & 1u)) return;
+        const ItemInfo I = sm.items[X][rs];
+        if (I.kind == 0) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.item_empty[X][rs]);
+            break;
+        }
+        const uint32_t tO = tS + 128 + (k & 1) * 64;
+        const int row = I.q0 + tid;
+        const int wrow0 = I.q0 + warp * 32;
+        const bool active = I.kind == 2 ? wrow0 < I.g : wrow0 < I.n_r;
+        RowOut ro;
+        ro.write = false;
+        ro.valid = false;
+        if (I.kind == 1 && active) {
+            const bool row_in = row < I.n_r;
+            const int i = row * I.dil + I.r;
+            const uint32_t *vb = a.ws.vbits + size_t(I.b) * a.L.nwords;
+            const uint32_t *gb = a.ws.gbits + size_t(I.b) * a.L.nwords;
+            ro.valid = row_in && bit_at(vb, i);
+            ro.write = row_in && (!ro.valid || !bit_at(gb, i));
+        }
+        RowState st{-INFINITY, 0.f};
+        for (int t = 0; t < I.ntiles; ++t) {
+            const int rt = jt % kRing;
+            if (!warp_wait(p, sm, &sm.tm_full[X][rt], uint32_t(jt / kRing) & 1u)) return;
+            uint32_t mw[4];
+            if (active) tile_row_mask(a, I, sm.tmask[X][rt], t, row, lane, mw);
+            if (!warp_wait(p, sm, &sm.s_full[X], uint32_t(jt) & 1u)) return;
+            tc_fence_after();
+            if (active) softmax_tile<T>(tS, tO, st, t == 0, mw, sl2);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.p_full[X]);
+            ++jt;
+            if (t == 0 && pending) {
+                // The previous item's products finished before this tile's S.
+                const int ke = k - 1;
+                if (!warp_wait(p, sm, &sm.o_full[X][ke & 1], uint32_t(ke >> 1) & 1u)) return;
+                tc_fence_after();
+                epilogue<T>(p, sm, tmem_row, X, ke, pend, tid);
+                pending = false;
+            }
+        }
+        ro.m = st.m;
+        ro.l = st.l;
+        pend = ro;
+        pending = true;
+        ++k;
+    }
+    if (pending) {
+        const int ke = k - 1;
+        if (!warp_wait(p, sm, &sm.o_full[X][ke & 1], uint32_t(ke >> 1) & 1u)) return;
+        tc_fence_after();
+        epilogue<T>(p, sm, tmem_row, X, ke, pend, tid);
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    FwdSmem &sm = *reinterpret_cast<FwdSmem *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int X = 0; X < kSlots; ++X) {
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&sm.q_full[X][b], 1);
+                mbar_init(&sm.q_empty[X][b], 1);
+                mbar_init(&sm.o_empty[X][b], 4);      // one arrival per softmax warp
+                mbar_init(&sm.o_full[X][b], 1);
+            }
+            for (int r = 0; r < kRing; ++r) {
+                mbar_init(&sm.item_full[X][r], 1);
+                mbar_init(&sm.item_empty[X][r], 5);   // four softmax warps + the MMA warp
+                mbar_init(&sm.tm_full[X][r], 1);
+            }
+            mbar_init(&sm.s_full[X], 1);
+            mbar_init(&sm.p_full[X], 4);
+        }
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.kv_full[s], 1);
+            mbar_init(&sm.kv_empty[s], 1);
+        }
+        mbar_init(&sm.drain, 1);
+        sm.abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == kWarpProducer && lane == 0) {
+        for (int m = 0; m < kMapCount; ++m) tma_prefetch_map(&p.maps[m]);
+        for (int m = 0; m < p.n_res; ++m) {
+            tma_prefetch_map(&p.res_q[m]);
+            tma_prefetch_map(&p.res_k[m]);
+            tma_prefetch_map(&p.res_v[m]);
+        }
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    // Everything above overlaps the previous kernel in the stream; the
+    // workspace it writes (compacted indices, bitmaps, counters) is read
+    // only below.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    for (int b = threadIdx.x; b < kBatchCache && b < p.a.B; b += kThreads) {
+        sm.batch_count[b] = p.a.ws.counts[b];
+        sm.batch_flags[b] = p.a.ws.flags[b];
+    }
+    if (blockIdx.x == 0)
+        for (int b = threadIdx.x; b < p.a.B; b += kThreads)
+            if (p.a.ws.counts[b] > p.a.max_global) set_status(p.a.ws.status, kErrGlobalOverflow);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    if (warp < 8) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+        softmax_role<T>(p, sm, tmem, warp >> 2, threadIdx.x & 127);
+    } else {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
+        if (warp == kWarpProducer) {
+            producer_role(p, sm, lane);
+        } else if (warp == kWarpMma) {
+            mma_role(p, sm, tmem, std::is_same<T, __nv_bfloat16>::value);
+            // Every MMA this warp issued has completed once this commit lands.
+            tc_commit_elect(&sm.drain);
+            __syncwarp();
+            drain_wait(&sm.drain, 0, p.wait_ns);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Merges the chunk partials of every global row into its output row: one
+// warp per (batch*head, global slot); lane l handles dimensions 2l, 2l+1.
+// Launched after the attention kernel (programmatic dependent launch: its
+// prologue overlaps the attention kernel's tail, the wait below orders it).
+template <typename T>
+__global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a)
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int lane = threadIdx.x & 31;
+    const int bh = blockIdx.x;
+    const int slot = blockIdx.y * 4 + (threadIdx.x >> 5);
+    const int b = bh / a.H;
+    const int g = min(a.ws.counts[b], a.max_global);
+    if (slot >= g) return;
+    const int pos = a.ws.gidx[size_t(b) * a.n + slot];
+    if (!bit_at(a.ws.vbits + size_t(b) * a.L.nwords, pos)) return;   // padded: zeros elsewhere
+    const int nch = a.L.nchunks;
+    const size_t mg = size_t(a.max_global);
+    const size_t cstride = kPartialFloats * mg;
+    const float *P = partial_base(a, bh, 0) + slot;
+    float M = -INFINITY;
+    for (int c = lane; c < nch; c += 32) M = fmaxf(M, P[c * cstride]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f, a0 = 0.f, a1 = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < nch; ++c) {
+        const float *pc = P + c * cstride;
+        const float mc = pc[0];
+        const float f = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+        L = fmaf(f, pc[mg], L);
+        a0 = fmaf(f, pc[(2 + 2 * lane) * mg], a0);
+        a1 = fmaf(f, pc[(3 + 2 * lane) * mg], a1);
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    T *dst = static_cast<T *>(a.out) + (size_t(bh) * a.n + pos) * kDHead;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        reinterpret_cast<__nv_bfloat162 *>(dst)[lane] = __floats2bfloat162_rn(a0 * inv, a1 * inv);
+    } else {
+        reinterpret_cast<__half2 *>(dst)[lane] = __floats2half2_rn(a0 * inv, a1 * inv);
+    }
+}
+
+// ------------------------------------------------------------------ host
+namespace {
+
+// Test hooks (lf_test_forward_hooks): the limit of the bounded waits and a
+// planted stall; read at every launch.
+std::atomic<unsigned long long> g_wait_ns{1000ull * 1000ull * 1000ull};
+std::atomic<int> g_stall_first_q{0};
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// Whole tiles of 128 rows of the residue class r of dilation dil of each
+// (batch*head) slice: rows r, r+dil, ... ; dims {64, ceil((n-r)/dil), B*H}.
+bool encode_tile_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int n, int BH,
+                     int dil, int r)
+{
+    auto enc = get_encoder();
+    if (!enc) return false;
+    const int n_r = (n - r + dil - 1) / dil;
+    base = static_cast<const char *>(base) + size_t(r) * kRowBytes;
+    cuuint64_t dims[3] = {cuuint64_t(kDHead), cuuint64_t(n_r), cuuint64_t(BH)};
+    cuuint64_t strides[2] = {cuuint64_t(dil) * kRowBytes, cuuint64_t(n) * kRowBytes};
+    cuuint32_t box[3] = {kDHead, cuuint32_t(kRows), 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// Single rows of the flattened tensor: dims {64, B*H*n}.
+bool encode_row_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, long rows)
+{
+    auto enc = get_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cuuint64_t(kDHead), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(kRowBytes)};
+    cuuint32_t box[2] = {kDHead, 1};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+struct MapCacheEntry {
+    const void *base;
+    int kind, dt, n, BH, dil, r;
+    CUtensorMap map;
+    bool used;
+};
+
+// Encoded tensor maps, reused while the same buffer and shape come back.
+// kind: 0 = tiles of 128 rows, 1 = single rows.
+bool cached_map(CUtensorMap *out, int kind, const void *base, CUtensorMapDataType dt, int n, int BH,
+                int dil = 1, int r = 0)
+{
+    constexpr int kCache = 256;
+    static std::mutex mu;
+    static MapCacheEntry cache[kCache];
+    static unsigned next = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (auto &e : cache)
+        if (e.used && e.base == base && e.kind == kind && e.dt == int(dt) && e.n == n &&
+            e.BH == BH && e.dil == dil && e.r == r) {
+            *out = e.map;
+            return true;
+        }
+    CUtensorMap m;
+    const bool ok = kind == 1 ? encode_row_map(&m, base, dt, long(n) * BH)
+                              : encode_tile_map(&m, base, dt, n, BH, dil, r);
+    if (!ok) return false;
+    MapCacheEntry &e = cache[next++ % kCache];
+    e = MapCacheEntry{base, kind, int(dt), n, BH, dil, r, m, true};
+    *out = m;
+    return true;
+}
+
+int num_sms()
+{
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 1;
+}
+
+template <typename T>
+int launch_typed(const AttnArgs &a, CUtensorMapDataType dt, cudaStream_t stream)
+{
+    FwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.a = a;
+    const int BH = a.B * a.H;
+    bool ok = true;
+    // Residue maps of every distinct dilation, while they fit.
+    for (int h = 0; h < a.H; ++h) p.res_base[h] = -1;
+    p.n_res = 0;
+    for (int h = 0; h < a.H; ++h) {
+        if (p.res_base[h] >= 0) continue;
+        const int dil = a.dil[h];
+        const int nres = std::min(dil, a.n);
+        if (p.n_res + nres > kMaxResidues) continue;
+        const int base = p.n_res;
+        for (int r = 0; r < nres && ok; ++r) {
+            ok = ok && cached_map(&p.res_q[base + r], 0, a.q, dt, a.n, BH, dil, r);
+            ok = ok && cached_map(&p.res_k[base + r], 0, a.k, dt, a.n, BH, dil, r);
+            ok = ok && cached_map(&p.res_v[base + r], 0, a.v, dt, a.n, BH, dil, r);
+        }
+        p.n_res += nres;
+        for (int h2 = h; h2 < a.H; ++h2)
+            if (a.dil[h2] == dil) p.res_base[h2] = base;
+    }
+    ok = ok && cached_map(&p.maps[kMapKgTile], 0, a.kg, dt, a.n, BH);
+    ok = ok && cached_map(&p.maps[kMapVgTile], 0, a.vg, dt, a.n, BH);
+    ok = ok && cached_map(&p.maps[kMapQRow], 1, a.q, dt, a.n, BH);
+    ok = ok && cached_map(&p.maps[kMapKRow], 1, a.k, dt, a.n, BH);
+    ok = ok && cached_map(&p.maps[kMapVRow], 1, a.v, dt, a.n, BH);
+    ok = ok && cached_map(&p.maps[kMapQgRow], 1, a.qg, dt, a.n, BH);
+    if (!ok) return kErrCuda;
+    p.gtiles = (a.max_global + kRows - 1) / kRows;
+    p.band_items = a.B * a.band_items_per_batch;
+    p.total_items = p.band_items + BH * p.gtiles * a.L.nchunks;
+    p.oob_row = BH * a.n;
+    // One warp merges 32 global rows over every chunk: cheap for a few chunks,
+    // a separate wide kernel beyond that.
+    p.merge_in_kernel = a.L.nchunks <= kMergeInKernelChunks;
+    p.wait_ns = g_wait_ns.load();
+    p.stall_first_q = g_stall_first_q.load();
+    const size_t smem = kFwdSmemBytes;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(attn_fwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem)) != cudaSuccess)
+            return kErrCuda;
+        // setmaxnreg.inc waits until the registers it asks for are free; refuse
+        // to launch if the compiled register count cannot cover the split.
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<T>) != cudaSuccess) return kErrCuda;
+        if (fa.numRegs * kThreads < kRegsNeeded) return kErrUnsupported;
+        attr_set[dev] = true;
+    }
+    const int want = (p.total_items + kSlots - 1) / kSlots;
+    const int grid = std::max(1, std::min(num_sms(), want));
+    // Programmatic dependent launch: the kernel's prologue (barriers, TMEM,
+    // tensor-map prefetch) overlaps the kernel before it in the stream.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, attn_fwd_kernel<T>, p) != cudaSuccess) return kErrCuda;
+    if (a.max_global > 0 && !p.merge_in_kernel) {
+        cudaLaunchConfig_t cc = {};
+        cc.gridDim = dim3(a.B * a.H, (a.max_global + 3) / 4);
+        cc.blockDim = dim3(128);
+        cc.stream = stream;
+        cc.attrs = attr;
+        cc.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cc, combine_kernel<T>, a) != cudaSuccess) return kErrCuda;
+    }
+    return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+}
+
+}  // namespace
+
+int launch_tc(lf_dtype dtype, const AttnArgs &a, cudaStream_t stream)
+{
+    if (dtype == LF_BF16) return launch_typed<__nv_bfloat16>(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, stream);
+    return launch_typed<__half>(a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, stream);
+}
+
+}  // namespace lf
+
+extern "C" int lf_test_forward_hooks(unsigned long long wait_limit_ns, int stall_first_q)
+{
+    if (wait_limit_ns == 0) return LF_ERR_INVALID_ARG;
+    lf::g_wait_ns.store(wait_limit_ns);
+    lf::g_stall_first_q.store(stall_first_q ? 1 : 0);
+    return LF_OK;
+}
+
+extern "C" int lf_exp2_poly_eval(const float *x, float *y, int n, lf_stream_t stream)
+{
+    if (n < 0 || (n > 0 && (!x || !y))) return LF_ERR_INVALID_ARG;
+    if (n == 0) return LF_OK;
+    const int pairs = (n + 1) / 2;
+    lf::exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+}

@@ -65,7 +65,13 @@ prepare_kernel(const uint8_t *__restrict__ local_mask, const uint8_t *__restrict
     const int wpt = (nwords + kPrepThreads - 1) / kPrepThreads;   // words per thread (<= 8)
     const int w0 = tid * wpt;
 
-    if (tid == 0 && b == 0 && status) *status = 0;
+    // The status word, and the attention kernel's item counter and finished
+    // count (words 16 and 32 of the status region), start at zero.
+    if (tid == 0 && b == 0 && status) {
+        status[0] = 0;
+        status[16] = 0;
+        status[32] = 0;
+    }
     if (counters)
         for (int c = tid; c < counters_per_batch; c += kPrepThreads)
             counters[size_t(b) * counters_per_batch + c] = 0;

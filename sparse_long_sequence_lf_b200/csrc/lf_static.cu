@@ -8,7 +8,8 @@
 // The scratch is one file-scope array per device (the CUDA module's own
 // global memory), of kStaticScratchBytes.  The first call on a device looks
 // up its address with cudaGetSymbolAddress while that device is current and
-// caches it; later calls on that device reuse the cached address.  Because
+// caches it; later calls on that device reuse the cached address (after a
+// cudaDeviceReset the cached address is stale: reload the library).  Because
 // there is one scratch per device, calls on one device must not overlap in
 // time (two streams, two host threads): overlapping calls race on it.
 //
@@ -67,10 +68,12 @@ extern "C" int lf_attention_forward_static(lf_dtype dtype, int B, int H, int n, 
                                            int causal, void *out, lf_stream_t stream,
                                            void **scratch)
 {
-    // A problem whose workspace does not fit is refused before the device is
-    // touched.  Invalid sizes (workspace size 0) are left to the checks of
-    // lf_attention_forward.
+    // Sizes that have no workspace (lf_workspace_size returns 0) and problems
+    // whose workspace does not fit are refused before the device is touched:
+    // no context is created and no module is loaded for them.
+    if (d_head != lf::kDHead) return LF_ERR_UNSUPPORTED;
     const size_t need = lf_workspace_size(B, H, n, d_head, max_global);
+    if (need == 0) return LF_ERR_INVALID_ARG;
     if (need > kStaticScratchBytes) return LF_ERR_SCRATCH_LIMIT;
     void *ws = nullptr;
     if (int rc = current_scratch(&ws)) return rc;

@@ -149,7 +149,10 @@ def random_workload(rng: np.random.Generator, *, dtype: str = "bf16", max_n: int
         window = int(rng.integers(1, 300))
     else:
         window = 2 * int(rng.integers(1, 300))
-    dil = tuple(int(x) for x in rng.integers(1, 4, size=H))
+    # Mostly small dilations; one draw in four takes them up to 12, so that the
+    # heads' (dilation, residue) classes can outgrow the residue tensor maps.
+    dil_hi = 13 if rng.random() < 0.25 else 4
+    dil = tuple(int(x) for x in rng.integers(1, dil_hi, size=H))
     if causal:
         gk = "none"
     else:

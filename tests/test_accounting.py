@@ -68,3 +68,15 @@ def test_encoder_flops_count_every_product_of_a_layer():
                  + 2 * tok * hid * 256            # FFN intermediate
                  + 2 * tok * 256 * hid)           # FFN output
     assert bench.encoder_flops(ew, [g]) == 3 * per_layer
+
+
+@pytest.mark.parametrize("wl", CASES, ids=[c.name for c in CASES])
+def test_row_block_flops_add_up(wl):
+    # Row blocks of every (batch, head) partition the whole count.
+    total = 0
+    for b in range(wl.B):
+        for h in range(wl.H):
+            cut = wl.n // 3
+            total += accounting.useful_flops_rows(wl, h, (0, cut), batch=b)
+            total += accounting.useful_flops_rows(wl, h, (cut, wl.n), batch=b)
+    assert total == accounting.useful_flops(wl)

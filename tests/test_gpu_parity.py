@@ -50,6 +50,12 @@ EDGE = [
              pad_tail=(300, 0)),
     Workload("dilated-globals", "f16", 1, 4, 900, 40, dilation=(1, 2, 3, 5),
              globals_kind="random:20", pad_tail=(77,), seed=9),
+    # (dilation, residue) classes 7 + 8 + 9 + 10 = 34: the last head does not
+    # fit the residue tensor maps and loads its rows one by one
+    Workload("residue-budget", "bf16", 2, 4, 1200, 48, dilation=(7, 8, 9, 10),
+             globals_kind="random:11", pad_tail=(0, 90), seed=15),
+    Workload("residue-budget-causal", "f16", 1, 3, 1500, 100, dilation=(11, 12, 13),
+             causal=True, seed=16),
     Workload("fp32-mixed", "f32", 2, 3, 600, 50, dilation=(1, 2, 4), globals_kind="random:9",
              pad_tail=(0, 41), seed=10),
     Workload("fp32-causal", "f32", 1, 2, 513, 33, dilation=(1, 3), causal=True, seed=11),
@@ -108,7 +114,9 @@ def test_full_size_workload(name):
     wl = WORKLOADS[name]
     x = make_inputs(wl)
     out = gpu_forward(x).float().cpu().numpy()
-    heads = sorted({0, wl.H // 2, wl.H - 1})
+    # Heads 0, H/2, H-1 and the first head of every distinct dilation.
+    dil = list(x["dilation"])
+    heads = sorted({0, wl.H // 2, wl.H - 1} | {dil.index(d) for d in set(dil)})
     tol = TOL[wl.dtype]
     for h in heads:
         xs = dict(x)

@@ -37,16 +37,21 @@ def _run(wl):
     if gm is None:
         gm = torch.zeros((wl.B, wl.n), dtype=torch.uint8, device="cuda")
     gidx, counts = lf.global_index(gm)
-    mg = int(counts.max().item())
+    # The oracle takes its global index from the CPU oracle's compaction of
+    # the host mask, never from the CUDA path; the GPU compaction must agree.
+    ref_gidx, ref_counts = oracle.global_index(gm.cpu().numpy())
+    assert np.array_equal(gidx.cpu().numpy(), ref_gidx)
+    assert np.array_equal(counts.cpu().numpy(), ref_counts)
+    mg = int(ref_counts.max())
     sentinel = torch.full((wl.B, wl.H, wl.n, 64), 3.0, dtype=x["x"].dtype, device="cuda")
     out = lf.qkv_projection(d["x"], d["w"], d["bias"], d["wqg"], d["bqg"], gidx, counts,
                             H=wl.H, max_global=mg, out={"qg": sentinel.clone()})
     torch.cuda.synchronize()
     f64 = lambda t: t.double().cpu().numpy()
     ref = projection_forward(f64(x["x"]), f64(x["w"]), f64(x["bias"]), f64(x["wqg"]),
-                             f64(x["bqg"]), gidx.cpu().numpy(), counts.cpu().numpy(), H=wl.H,
+                             f64(x["bqg"]), ref_gidx, ref_counts, H=wl.H,
                              qg_init=f64(sentinel))
-    return out, ref, gidx.cpu().numpy(), counts.cpu().numpy()
+    return out, ref, ref_gidx, ref_counts
 
 
 @pytest.mark.parametrize("wl", CASES, ids=[w.name for w in CASES])

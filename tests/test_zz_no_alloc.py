@@ -11,7 +11,7 @@ import torch
 import sparse_long_sequence_lf_b200 as lf
 from sparse_long_sequence_lf_b200._lib import STATIC_SCRATCH_BYTES
 from sparse_long_sequence_lf_b200.workloads import Workload, make_inputs
-from gpu_helpers import TOL, max_global_of, to_dev
+from gpu_helpers import TOL, assert_close, max_global_of, oracle_forward, to_dev
 
 CASES = [
     # globals anywhere, tail padding, per-head dilation
@@ -41,9 +41,12 @@ def test_static_scratch_matches_forward(wl):
     torch.cuda.synchronize()
     assert scratch[0] == scratch[1] != 0
     assert lf.scratch_status(scratch[1]) == 0
+    # The same kernels on the same inputs: the results must be identical, bit
+    # for bit; a scratch region that aliased another would show here.
     for out in outs:
-        err = (out.double() - ref.double()).abs().max().item()
-        assert err <= TOL[wl.dtype], err
+        assert torch.equal(out, ref)
+    # And the static path on its own against the fp64 oracle.
+    assert_close(outs[1], oracle_forward(x), TOL[wl.dtype], wl.name)
 
 
 def test_static_scratch_limit_is_refused():
@@ -57,3 +60,16 @@ def test_static_scratch_limit_is_refused():
         512, None, 0, None, None, None)
     assert rc == -8
     assert b"16 MiB" in _lib.lib().lf_status_string(rc)
+
+
+@pytest.mark.parametrize("sizes,code", [((0, 2, 256, 64, 1), -1), ((1, 2, 256, 64, 300), -1),
+                                        ((1, 2, 256, 32, 1), -2)])
+def test_static_invalid_sizes_are_refused_on_the_host(sizes, code):
+    # Sizes with no workspace are refused before anything touches a device
+    # (no GPU needed): zero batches, more global slots than tokens, d_head 32.
+    from sparse_long_sequence_lf_b200 import _lib
+    B, H, n, d, mg = sizes
+    rc = _lib.lib().lf_attention_forward_static(
+        _lib.LF_BF16, B, H, n, d, None, None, None, None, None, None, None, None, mg,
+        64, None, 0, None, None, None)
+    assert rc == code
