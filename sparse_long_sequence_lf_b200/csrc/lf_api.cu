@@ -13,7 +13,7 @@ int launch_prepare(const uint8_t *local_mask, const uint8_t *global_mask, int B,
                    int max_global, int32_t *gidx, int32_t *counts, int *flags, uint32_t *vbits,
                    uint32_t *gbits, int *status, int *counters, int counters_per_batch,
                    cudaStream_t stream);
-template <typename T> int launch_simt(const AttnArgs &a, cudaStream_t stream);
+int launch_f32(const AttnArgs &a, cudaStream_t stream);
 int launch_tc(lf_dtype dtype, const AttnArgs &a, cudaStream_t stream);
 int launch_projection(lf_dtype dtype, int B, int n, int H, const void *x, const void *w,
                       const void *bias, const void *wqg, const void *bqg, const int32_t *gidx,
@@ -191,7 +191,7 @@ int lf_attention_run(lf_dtype dtype, int B, int H, int n, int d_head, const void
     a.out = out;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (dtype) {
-        case LF_F32: return launch_simt<float>(a, s);
+        case LF_F32: return launch_f32(a, s);
         case LF_F16: return launch_tc(LF_F16, a, s);
         case LF_BF16: return launch_tc(LF_BF16, a, s);
     }

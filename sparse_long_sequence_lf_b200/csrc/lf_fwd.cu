@@ -138,7 +138,7 @@ struct ItemInfo {
     int g;          // global tokens of the batch (clamped to max_global)
     int chunk;
     int has_pad;
-    int pad_[1];
+    int res;        // band: residue tensor map of (head, r), -1: rows one by one
 };
 static_assert(sizeof(ItemInfo) == 64, "item record size");
 
@@ -164,6 +164,9 @@ struct __align__(1024) FwdSmem {
     uint64_t drain;
     int batch_count[kBatchCache];
     int batch_flags[kBatchCache];
+    int head_dil[kMaxHeads];            // per-head tables, copied from the kernel
+    int head_prefix[kMaxHeads + 1];     // arguments (indexed per item)
+    int head_res[kMaxHeads];
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -172,10 +175,11 @@ constexpr size_t kFwdSmemBytes = sizeof(FwdSmem) + 1024;
 static_assert(kFwdSmemBytes <= 232448, "shared memory per CTA");
 
 // ------------------------------------------------------------ small helpers
-__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                             int *status, uint64_t limit_ns)
+// The part of a bounded wait that runs only when the phase is not complete
+// at the first test; out of line to keep the roles' code small.
+__device__ __forceinline__ bool wait_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                       int *status, uint64_t limit_ns)
 {
-    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     uint32_t spins = 0;
     for (;;) {
@@ -196,7 +200,8 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
 __device__ __forceinline__ bool warp_wait(const FwdParams &p, FwdSmem &sm, uint64_t *bar,
                                           uint32_t parity)
 {
-    const bool ok = wait_bounded(bar, parity, &sm.abort_flag, p.a.ws.status, p.wait_ns);
+    const bool ok = mbar_try_wait(bar, parity) ||
+                    wait_slow(bar, parity, &sm.abort_flag, p.a.ws.status, p.wait_ns);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -236,17 +241,48 @@ __device__ __forceinline__ int batch_flags(const FwdSmem &sm, const AttnArgs &a,
     return b < kBatchCache ? sm.batch_flags[b] : a.ws.flags[b];
 }
 
+// Band item -> (batch, head, residue, tile of 128 rows): the heads' item
+// counts are prefix sums in shared memory (binary search), the residues of
+// a head are walked in order.
+__device__ __forceinline__ void band_item_s(const FwdSmem &sm, const AttnArgs &a, int item, int &b,
+                                            int &h, int &r, int &tile)
+{
+    b = item / a.band_items_per_batch;
+    int rem = item - b * a.band_items_per_batch;
+    int lo = 0, hi = a.H - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (sm.head_prefix[mid] <= rem)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    h = lo;
+    rem -= sm.head_prefix[h];
+    const int dil = sm.head_dil[h];
+    r = 0;
+    for (;;) {
+        const int n_r = (a.n - r + dil - 1) / dil;
+        const int t = (n_r + kRows - 1) / kRows;
+        if (rem < t || r + 1 >= dil) break;
+        rem -= t;
+        ++r;
+    }
+    tile = rem;
+}
+
 __device__ __forceinline__ ItemInfo decode_item(const FwdParams &p, const FwdSmem &sm, int item)
 {
     const AttnArgs &a = p.a;
     ItemInfo I;
-    I.pad_[0] = 0;
+    I.res = -1;
     if (item < p.band_items) {
         int tile;
-        band_item(a, item, I.b, I.h, I.r, tile);
+        band_item_s(sm, a, item, I.b, I.h, I.r, tile);
         I.kind = 1;
         I.bh = I.b * a.H + I.h;
-        I.dil = a.dil[I.h];
+        I.dil = sm.head_dil[I.h];
+        I.res = sm.head_res[I.h] >= 0 ? sm.head_res[I.h] + I.r : -1;
         I.n_r = (a.n - I.r + I.dil - 1) / I.dil;
         I.q0 = tile * kRows;
         const int rows_hi = min(I.q0 + kRows - 1, I.n_r - 1);
@@ -283,102 +319,123 @@ __device__ __forceinline__ ItemInfo decode_item(const FwdParams &p, const FwdSme
 }
 
 // ------------------------------------------------------------ producer
+// The producer keeps, per slot, two items ahead of the one whose tiles it is
+// loading: item records are written to the slot's ring as soon as they are
+// claimed, their Q tiles load as soon as a Q buffer frees, and the index of
+// the item after them is already being claimed (the atomic's round trip
+// overlaps the tile loads), so that an item change stalls neither slot.
 struct ProducerSlot {
-    ItemInfo I;
-    int t;          // next tile of the item
-    int k;          // items fetched so far (ring position of the next one)
-    int jt;         // tiles produced so far
-    bool active;
+    int kc;         // item whose tiles are being loaded (count within the slot)
+    int t;          // its next tile
+    int kw;         // item records written to the ring
+    int kq;         // items whose Q load was started (or that need none)
+    int claimed;    // index claimed for record kw (lane 0)
+    int jt;         // tiles loaded
+    bool ended;     // the "no more items" record has been written
 };
 
-// Fetches the next item of slot X from the device-wide counter, writes its
-// record to the slot's item ring and loads its Q tile.  Returns false on abort.
-__device__ __forceinline__ bool producer_fetch(const FwdParams &p, FwdSmem &sm, ProducerSlot &S, int X,
-                                            int lane, int *sched, int *finished, uint32_t &q_armed,
-                                            uint32_t &q_par)
+// Claims the next item index from the device-wide counter (lane 0 only; the
+// value is read when the record is written).
+__device__ __forceinline__ int claim_item(int *sched, int lane)
 {
-    const AttnArgs &a = p.a;
+    return lane == 0 ? atomicAdd(sched, 1) : 0;
+}
+
+// Decodes the claimed index into the slot's next ring record and claims the
+// one after.  Items without work (a tile of global rows past the batch's
+// count) are skipped.  The end of the items is written as a record of kind 0.
+__device__ __forceinline__ bool producer_write_next(const FwdParams &p, FwdSmem &sm, ProducerSlot &S,
+                                                    int X, int lane, int *sched)
+{
     ItemInfo I;
     I.kind = 0;
     for (;;) {
-        int idx = 0;
-        if (lane == 0) idx = atomicAdd(sched, 1);
-        idx = __shfl_sync(0xffffffffu, idx, 0);
+        const int idx = __shfl_sync(0xffffffffu, S.claimed, 0);
         if (idx >= p.total_items) {
-            // Every producer meets the end once per slot; the last one resets
-            // the counters for the next launch on this workspace.
-            if (lane == 0) {
-                __threadfence();
-                if (atomicAdd(finished, 1) == int(2 * gridDim.x) - 1) {
-                    atomicExch(sched, 0);
-                    atomicExch(finished, 0);
-                }
-            }
             I.kind = 0;
+            S.ended = true;
             break;
         }
         I = decode_item(p, sm, idx);
+        S.claimed = claim_item(sched, lane);
         if (I.ntiles > 0) break;
     }
-    const int k = S.k;
+    const int k = S.kw;
     const int rs = k % kRing;
     if (!warp_wait(p, sm, &sm.item_empty[X][rs], (uint32_t(k / kRing) & 1u) ^ 1u)) return false;
-    if (I.kind != 0) {
-        const int qb = k & 1;
-        const uint32_t use = uint32_t(k >> 1);
-        if (!warp_wait(p, sm, &sm.q_empty[X][qb], (use & 1u) ^ 1u)) return false;
-        uint8_t *qd = sm.q[X][qb];
-        uint64_t *qbar = &sm.q_full[X][qb];
-        const bool stall = p.stall_first_q && blockIdx.x == 0 && X == 0 && k == 0;
-        if (!stall) {
-            const int rb = I.kind == 1 ? p.res_base[I.h] : -1;
-            if (rb >= 0) {
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(qbar, kQBytes);
-                    tma_load_3d(qd, &p.res_q[rb + I.r], qbar, 0, I.q0, I.bh);
-                }
-            } else if (I.kind == 1) {
-                if (lane == 0) mbar_arrive_expect_tx(qbar, kQBytes);
-                __syncwarp();
-                for (int rr = lane; rr < kRows; rr += 32) {
-                    const int ir = I.q0 + rr;
-                    const int y = ir < I.n_r ? I.bh * a.n + ir * I.dil + I.r : p.oob_row;
-                    tma_load_2d(qd + rr * kRowBytes, &p.maps[kMapQRow], qbar, 0, y);
-                }
-            } else {
-                // Only the rows of real global tokens: a query row only feeds
-                // its own output row, and rows past the count are never stored.
-                const int rows = min(kRows, I.g - I.q0);
-                if (lane == 0) mbar_arrive_expect_tx(qbar, rows * kRowBytes);
-                __syncwarp();
-                for (int rr = lane; rr < rows; rr += 32) {
-                    const int y = I.bh * a.n + a.ws.gidx[size_t(I.b) * a.n + I.q0 + rr];
-                    tma_load_2d(qd + rr * kRowBytes, &p.maps[kMapQgRow], qbar, 0, y);
-                }
-            }
-            // Bit 2X + qb: a Q copy of that buffer was started; its parity.
-            const uint32_t bit = 1u << (2 * X + qb);
-            q_armed |= bit;
-            q_par = (use & 1u) ? (q_par | bit) : (q_par & ~bit);
-        }
-    }
     if (lane == 0) sm.items[X][rs] = I;
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.item_full[X][rs]);
-    S.I = I;
-    S.t = 0;
-    S.k = k + 1;
-    S.active = I.kind != 0;
+    ++S.kw;
     return true;
 }
 
-// Loads tile S.t of the slot's item into ring stage `stage` and writes its
-// column masks to the slot's tile-mask ring.
+// Starts the Q load of record S.kq when its buffer is free (or at once if
+// `block`); returns false on abort.
+__device__ __forceinline__ bool producer_q(const FwdParams &p, FwdSmem &sm, ProducerSlot &S, int X,
+                                           int lane, bool block, uint32_t &q_armed, uint32_t &q_par)
+{
+    const AttnArgs &a = p.a;
+    if (S.kq >= S.kw) return true;
+    const int k = S.kq;
+    const ItemInfo &I = sm.items[X][k % kRing];
+    if (I.kind == 0) {
+        ++S.kq;
+        return true;
+    }
+    const int qb = k & 1;
+    const uint32_t use = uint32_t(k >> 1);
+    const uint32_t want = (use & 1u) ^ 1u;
+    if (block) {
+        if (!warp_wait(p, sm, &sm.q_empty[X][qb], want)) return false;
+    } else if (!__all_sync(0xffffffffu, mbar_try_wait(&sm.q_empty[X][qb], want))) {
+        return true;
+    }
+    uint8_t *qd = sm.q[X][qb];
+    uint64_t *qbar = &sm.q_full[X][qb];
+    const bool stall = p.stall_first_q && blockIdx.x == 0 && X == 0 && k == 0;
+    if (!stall) {
+        if (I.kind == 1 && I.res >= 0) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(qbar, kQBytes);
+                tma_load_3d(qd, &p.res_q[I.res], qbar, 0, I.q0, I.bh);
+            }
+        } else if (I.kind == 1) {
+            if (lane == 0) mbar_arrive_expect_tx(qbar, kQBytes);
+            __syncwarp();
+            for (int rr = lane; rr < kRows; rr += 32) {
+                const int ir = I.q0 + rr;
+                const int y = ir < I.n_r ? I.bh * a.n + ir * I.dil + I.r : p.oob_row;
+                tma_load_2d(qd + rr * kRowBytes, &p.maps[kMapQRow], qbar, 0, y);
+            }
+        } else {
+            // Only the rows of real global tokens: a query row only feeds its
+            // own output row, and rows past the count are never stored.
+            const int rows = min(kRows, I.g - I.q0);
+            if (lane == 0) mbar_arrive_expect_tx(qbar, rows * kRowBytes);
+            __syncwarp();
+            for (int rr = lane; rr < rows; rr += 32) {
+                const int y = I.bh * a.n + a.ws.gidx[size_t(I.b) * a.n + I.q0 + rr];
+                tma_load_2d(qd + rr * kRowBytes, &p.maps[kMapQgRow], qbar, 0, y);
+            }
+        }
+        // Bit 2X + qb: a Q copy of that buffer was started; its parity.
+        const uint32_t bit = 1u << (2 * X + qb);
+        q_armed |= bit;
+        q_par = (use & 1u) ? (q_par | bit) : (q_par & ~bit);
+    }
+    __syncwarp();
+    ++S.kq;
+    return true;
+}
+
+// Loads tile S.t of the slot's current item into ring stage `stage` and
+// writes its column masks to the slot's tile-mask ring.
 __device__ __forceinline__ void producer_tile(const FwdParams &p, FwdSmem &sm, ProducerSlot &S,
                                               int X, int lane, int stage)
 {
     const AttnArgs &a = p.a;
-    const ItemInfo &I = S.I;
+    const ItemInfo I = sm.items[X][S.kc % kRing];
     const int t = S.t;
     uint8_t *kd = sm.k[stage];
     uint8_t *vd = sm.v[stage];
@@ -412,12 +469,11 @@ __device__ __forceinline__ void producer_tile(const FwdParams &p, FwdSmem &sm, P
         } else if (lane < 4) {
             tm.bits[lane] = 0xffffffffu;
         }
-        const int rb = p.res_base[I.h];
-        if (rb >= 0) {
+        if (I.res >= 0) {
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar, 2 * kKvBytes);
-                tma_load_3d(kd, &p.res_k[rb + I.r], bar, 0, k0, I.bh);
-                tma_load_3d(vd, &p.res_v[rb + I.r], bar, 0, k0, I.bh);
+                tma_load_3d(kd, &p.res_k[I.res], bar, 0, k0, I.bh);
+                tma_load_3d(vd, &p.res_v[I.res], bar, 0, k0, I.bh);
             }
         } else {
             if (lane == 0) mbar_arrive_expect_tx(bar, 2 * kKvBytes);
@@ -457,67 +513,99 @@ __device__ __forceinline__ void producer_tile(const FwdParams &p, FwdSmem &sm, P
     if (lane == 0) mbar_arrive(&sm.tm_full[X][S.jt % kRing]);
 }
 
+template <typename S> __device__ __forceinline__ void swap_state(S &a, S &b)
+{
+    const S t = a;
+    a = b;
+    b = t;
+}
+
+// The producer and the MMA issuer serve the two slots in turn, skipping a
+// slot that has no more work: slot X, then slot X^1, ...  Both loops keep the
+// state of the slot they serve in `A` and of the other one in `B` and swap
+// them every turn, so that the code of a turn exists once (the roles' code is
+// small enough to stay in the instruction caches next to the softmax's).
 __device__ __forceinline__ void producer_role(const FwdParams &p, FwdSmem &sm, int lane)
 {
     int *sched = p.a.ws.status + 16;
-    int *finished = p.a.ws.status + 32;
-    ProducerSlot S[kSlots];
+    ProducerSlot A, B;
     uint32_t kv_armed = 0, kv_par = 0;   // bit s: stage s was filled; its parity
     uint32_t qa = 0, qp = 0;             // bit 2X+b: Q buffer b of slot X was filled
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-#pragma unroll
-    for (int X = 0; X < kSlots; ++X) {
-        S[X].k = 0;
-        S[X].jt = 0;
-        S[X].active = false;
-        if (ok) ok = producer_fetch(p, sm, S[X], X, lane, sched, finished, qa, qp);
-    }
-    while (ok && (S[0].active || S[1].active)) {
-#pragma unroll
-        for (int X = 0; X < kSlots; ++X) {
-            if (!ok || !S[X].active) continue;
+    A.kc = A.t = A.kw = A.kq = A.jt = 0;
+    A.ended = false;
+    B = A;
+    A.claimed = claim_item(sched, lane);
+    B.claimed = claim_item(sched, lane);
+    int X = 0;
+#pragma unroll 1
+    for (;;) {
+        // Keep two records ahead of the current item.
+        if (!A.ended && A.kw < A.kc + 2) ok = producer_write_next(p, sm, A, X, lane, sched);
+        // The Q load of the oldest record without one: at once if it is the
+        // current item's, else only if its buffer is already free.
+        if (ok) ok = producer_q(p, sm, A, X, lane, A.kq == A.kc, qa, qp);
+        if (!ok) break;
+        const bool busy_a = A.kc < A.kw && sm.items[X][A.kc % kRing].kind != 0;
+        if (busy_a) {
             if (!warp_wait(p, sm, &sm.kv_empty[stage], phase ^ 1u)) {
                 ok = false;
                 break;
             }
-            producer_tile(p, sm, S[X], X, lane, stage);
+            producer_tile(p, sm, A, X, lane, stage);
             kv_armed |= 1u << stage;
             kv_par = phase ? (kv_par | (1u << stage)) : (kv_par & ~(1u << stage));
             advance_ring(stage, phase);
-            ++S[X].jt;
-            if (++S[X].t == S[X].I.ntiles)
-                ok = producer_fetch(p, sm, S[X], X, lane, sched, finished, qa, qp);
+            ++A.jt;
+            if (++A.t == sm.items[X][A.kc % kRing].ntiles) {
+                ++A.kc;
+                A.t = 0;
+            }
+        } else if (B.ended && B.kc == B.kw - 1) {
+            // Both slots are at their end records (this one is: a slot that is
+            // not at its end always has a record of a real item to load).
+            break;
         }
+        swap_state(A, B);
+        X ^= 1;
     }
     if (!ok || sm.abort_flag) {
         for (int s = 0; s < kStages; ++s)
             if ((kv_armed >> s) & 1u) drain_wait(&sm.kv_full[s], (kv_par >> s) & 1u, p.wait_ns);
-        for (int X = 0; X < kSlots; ++X)
-            for (int b = 0; b < 2; ++b)
-                if ((qa >> (2 * X + b)) & 1u)
-                    drain_wait(&sm.q_full[X][b], (qp >> (2 * X + b)) & 1u, p.wait_ns);
+        for (int q = 0; q < 2 * kSlots; ++q)
+            if ((qa >> q) & 1u) drain_wait(&sm.q_full[q >> 1][q & 1], (qp >> q) & 1u, p.wait_ns);
     }
 }
 
 // ------------------------------------------------------------ MMA issuer
 struct MmaSlot {
-    ItemInfo I;
-    int t, k, j;    // tile of the item, items taken, tiles issued
+    int k, t, j;    // items taken, tile of the current item, tiles issued
     int stage;      // ring stage of the tile whose S was issued last
-    bool active;
+    int kind, ntiles, nkv, g;   // of the current item (kind 0: no more items)
 };
+
+__device__ __forceinline__ int mma_tile_cols(const MmaSlot &S)
+{
+    if (S.kind != 1 || S.t < S.nkv) return kTileKeys;
+    const int left = min(kTileKeys, S.g - (S.t - S.nkv) * kTileKeys);
+    return (left + 15) & ~15;
+}
 
 __device__ __forceinline__ bool mma_next_item(const FwdParams &p, FwdSmem &sm, MmaSlot &S, int X)
 {
     const int rs = S.k % kRing;
     if (!warp_wait(p, sm, &sm.item_full[X][rs], uint32_t(S.k / kRing) & 1u)) return false;
-    S.I = sm.items[X][rs];
+    const ItemInfo &I = sm.items[X][rs];
+    S.kind = I.kind;
+    S.ntiles = I.ntiles;
+    S.nkv = I.nkv;
+    S.g = I.g;
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.item_empty[X][rs]);
-    S.active = S.I.kind != 0;
     S.t = 0;
+    ++S.k;
     return true;
 }
 
@@ -532,7 +620,7 @@ __device__ __forceinline__ bool mma_issue_s(const FwdParams &p, FwdSmem &sm, Mma
         return false;
     if (!warp_wait(p, sm, &sm.kv_full[stage], phase)) return false;
     tc_fence_after();
-    const int N = tile_cols(S.I, S.t);
+    const int N = mma_tile_cols(S);
     const uint32_t tS = tmem + X * kSlotCols;
     const uint64_t qdesc = make_sdesc(smem_u32(sm.q[X][kq & 1]), 16, 1024);
     const uint64_t kdesc = make_sdesc(smem_u32(sm.k[stage]), 16, 1024);
@@ -542,7 +630,7 @@ __device__ __forceinline__ bool mma_issue_s(const FwdParams &p, FwdSmem &sm, Mma
         mma_ss_elect(tS, qdesc + uint64_t((kk * 32) >> 4), kdesc + uint64_t((kk * 32) >> 4), idesc,
                      kk > 0 ? 1u : 0u);
     tc_commit_elect(&sm.s_full[X]);
-    if (S.t == S.I.ntiles - 1) tc_commit_elect(&sm.q_empty[X][kq & 1]);
+    if (S.t == S.ntiles - 1) tc_commit_elect(&sm.q_empty[X][kq & 1]);
     __syncwarp();
     S.stage = stage;
     advance_ring(stage, phase);
@@ -553,57 +641,53 @@ __device__ __forceinline__ void mma_role(const FwdParams &p, FwdSmem &sm, uint32
 {
     const uint32_t id_s = make_idesc(128, 0, bf16, false);
     const uint32_t id_pv = make_idesc(128, 64, bf16, true);
-    MmaSlot S[kSlots];
+    MmaSlot A, B;
+    A.k = A.j = A.t = A.ntiles = 0;
+    A.kind = 1;              // "needs its first item"
+    B = A;
+    bool pv_pending_a = false, pv_pending_b = false;
     int stage = 0;
     uint32_t phase = 0;
-#pragma unroll
-    for (int X = 0; X < kSlots; ++X) {
-        S[X].k = 0;
-        S[X].j = 0;
-        S[X].active = false;
-        if (!mma_next_item(p, sm, S[X], X)) return;
-        ++S[X].k;
-    }
-#pragma unroll
-    for (int X = 0; X < kSlots; ++X)
-        if (S[X].active && !mma_issue_s(p, sm, S[X], X, tmem, id_s, stage, phase)) return;
+    int X = 0;
+#pragma unroll 1
     for (;;) {
-        bool any = false;
-#pragma unroll
-        for (int X = 0; X < kSlots; ++X) {
-            MmaSlot &s = S[X];
-            if (!s.active) continue;
-            any = true;
-            const int kq = s.k - 1;
-            const int ob = kq & 1;
-            if (!warp_wait(p, sm, &sm.p_full[X], uint32_t(s.j) & 1u)) return;
-            // The first PV of an item overwrites its O buffer: the epilogue of
-            // the item two before must have read it.
-            if (s.t == 0 && kq >= 2 &&
-                !warp_wait(p, sm, &sm.o_empty[X][ob], uint32_t((kq >> 1) - 1) & 1u))
-                return;
-            tc_fence_after();
-            {
+        if (A.kind == 0 && B.kind == 0) break;
+        if (A.kind != 0) {
+            if (pv_pending_a) {
+                const int kq = A.k - 1;
+                const int ob = kq & 1;
+                if (!warp_wait(p, sm, &sm.p_full[X], uint32_t(A.j) & 1u)) return;
+                // The first PV of an item overwrites its O buffer: the epilogue
+                // of the item two before must have read it.
+                if (A.t == 0 && kq >= 2 &&
+                    !warp_wait(p, sm, &sm.o_empty[X][ob], uint32_t((kq >> 1) - 1) & 1u))
+                    return;
+                tc_fence_after();
                 const uint32_t tP = tmem + X * kSlotCols;
                 const uint32_t tO = tP + 128 + ob * 64;
-                const uint64_t vdesc = make_sdesc(smem_u32(sm.v[s.stage]), 16, 1024);
-                const int ksteps = tile_cols(s.I, s.t) >> 4;
+                const uint64_t vdesc = make_sdesc(smem_u32(sm.v[A.stage]), 16, 1024);
+                const int ksteps = mma_tile_cols(A) >> 4;
                 for (int kk = 0; kk < ksteps; ++kk)
                     mma_ts_elect(tO, tP + kk * 8, vdesc + uint64_t((kk * 2048) >> 4), id_pv,
-                                 (kk > 0 || s.t > 0) ? 1u : 0u);
-                tc_commit_elect(&sm.kv_empty[s.stage]);
-                if (s.t == s.I.ntiles - 1) tc_commit_elect(&sm.o_full[X][ob]);
+                                 (kk > 0 || A.t > 0) ? 1u : 0u);
+                tc_commit_elect(&sm.kv_empty[A.stage]);
+                if (A.t == A.ntiles - 1) tc_commit_elect(&sm.o_full[X][ob]);
+                __syncwarp();
+                ++A.j;
+                ++A.t;
+                pv_pending_a = false;
             }
-            __syncwarp();
-            ++s.j;
-            if (++s.t == s.I.ntiles) {
-                if (!mma_next_item(p, sm, s, X)) return;
-                ++s.k;
-                if (!s.active) continue;
+            if (A.t == A.ntiles && !mma_next_item(p, sm, A, X)) return;
+            if (A.kind != 0) {
+                if (!mma_issue_s(p, sm, A, X, tmem, id_s, stage, phase)) return;
+                pv_pending_a = true;
             }
-            if (!mma_issue_s(p, sm, s, X, tmem, id_s, stage, phase)) return;
         }
-        if (!any) break;
+        swap_state(A, B);
+        const bool tmp = pv_pending_a;
+        pv_pending_a = pv_pending_b;
+        pv_pending_b = tmp;
+        X ^= 1;
     }
 }
 
@@ -867,7 +951,7 @@ __device__ __forceinline__ void epilogue(const FwdParams &p, FwdSmem &sm, uint32
         if (kind == 1) {
             const int pos = ro.write ? row * I.dil + I.r : 0;
             T *dst = static_cast<T *>(a.out) + (size_t(bh) * a.n + pos) * kDHead;
-            const float inv = ro.valid ? 1.f / ro.l : 0.f;
+            const float inv = ro.valid ? __frcp_rn(ro.l) : 0.f;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float o[32];
@@ -982,7 +1066,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, ui
         if (I.kind == 0) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.item_empty[X][rs]);
-            break;
+            if (!pending) break;
         }
         const uint32_t tO = tS + 128 + (k & 1) * 64;
         const int row = I.q0 + tid;
@@ -1000,7 +1084,22 @@ __device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, ui
             ro.write = row_in && (!ro.valid || !bit_at(gb, i));
         }
         RowState st{-INFINITY, 0.f};
-        for (int t = 0; t < I.ntiles; ++t) {
+        // A record of kind 0 (no more items) runs no tile but still flushes
+        // the pending epilogue below.
+        const int ntiles = I.kind == 0 ? 0 : I.ntiles;
+        for (int t = 0; t <= ntiles; ++t) {
+            if (t == 1 || (t == 0 && ntiles == 0)) {
+                if (pending) {
+                    // The previous item's products are complete: every product
+                    // of this slot before this item's first S is.
+                    const int ke = k - 1;
+                    if (!warp_wait(p, sm, &sm.o_full[X][ke & 1], uint32_t(ke >> 1) & 1u)) return;
+                    tc_fence_after();
+                    epilogue<T>(p, sm, tmem_row, X, ke, pend, tid);
+                    pending = false;
+                }
+            }
+            if (t == ntiles) break;
             const int rt = jt % kRing;
             if (!warp_wait(p, sm, &sm.tm_full[X][rt], uint32_t(jt / kRing) & 1u)) return;
             uint32_t mw[4];
@@ -1012,26 +1111,13 @@ __device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, ui
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.p_full[X]);
             ++jt;
-            if (t == 0 && pending) {
-                // The previous item's products finished before this tile's S.
-                const int ke = k - 1;
-                if (!warp_wait(p, sm, &sm.o_full[X][ke & 1], uint32_t(ke >> 1) & 1u)) return;
-                tc_fence_after();
-                epilogue<T>(p, sm, tmem_row, X, ke, pend, tid);
-                pending = false;
-            }
         }
+        if (I.kind == 0) break;
         ro.m = st.m;
         ro.l = st.l;
         pend = ro;
         pending = true;
         ++k;
-    }
-    if (pending) {
-        const int ke = k - 1;
-        if (!warp_wait(p, sm, &sm.o_full[X][ke & 1], uint32_t(ke >> 1) & 1u)) return;
-        tc_fence_after();
-        epilogue<T>(p, sm, tmem_row, X, ke, pend, tid);
     }
 }
 
@@ -1084,6 +1170,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     // workspace it writes (compacted indices, bitmaps, counters) is read
     // only below.
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    for (int h = threadIdx.x; h < p.a.H; h += kThreads) {
+        sm.head_dil[h] = p.a.dil[h];
+        sm.head_prefix[h] = p.a.head_prefix[h];
+        sm.head_res[h] = p.res_base[h];
+    }
+    if (threadIdx.x == 0) sm.head_prefix[p.a.H] = p.a.head_prefix[p.a.H];
     for (int b = threadIdx.x; b < kBatchCache && b < p.a.B; b += kThreads) {
         sm.batch_count[b] = p.a.ws.counts[b];
         sm.batch_flags[b] = p.a.ws.flags[b];
@@ -1117,6 +1209,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+    }
+    // Every CTA counts itself out, also after an abort; the last one resets
+    // the item counter for the next launch on this workspace (no CTA claims
+    // items any more by then).
+    if (threadIdx.x == 0) {
+        int *sched = p.a.ws.status + 16;
+        int *finished = p.a.ws.status + 32;
+        __threadfence();
+        if (atomicAdd(finished, 1) == int(gridDim.x) - 1) {
+            atomicExch(sched, 0);
+            atomicExch(finished, 0);
+        }
     }
 }
 

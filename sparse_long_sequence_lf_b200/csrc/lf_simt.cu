@@ -1,353 +1,386 @@
-// CUDA-core kernels of the attention: the fp32 path.
+// CUDA-core attention for fp32 inputs.
 //
 // fp32 inputs are computed in fp32 on the FMA pipes end to end (the tensor
-// cores' tf32 mode keeps 10 mantissa bits, too few for fp32 parity):
+// cores' tf32 mode keeps 10 mantissa bits, too few for fp32 parity).  One
+// launch holds two kinds of CTAs, 128 threads each:
 //
-//   band kernel     one CTA per 32 query rows of one (batch, head, residue
-//                   class of the dilation), four threads per row; keys stream
-//                   through shared memory 32 at a time; an online softmax
-//                   covers the window taps and then the global-token columns.
-//                   Writes every row except valid global rows (zeros for
-//                   padding).
-//   global kernel   one CTA per (batch*head, chunk of 512 keys, group of 32
-//                   global rows); a warp owns 8 global rows, lanes split the
-//                   keys for the scores and the head dimension for Vg; writes
-//                   fp32 partials (max, sum, acc) and the last CTA of a group
-//                   merges the chunks (log-sum-exp) into the output rows.
+//   global CTAs   (batch*head, 512-key chunk, group of 32 global rows): each
+//                 of the four warps takes a quarter of the chunk's keys for
+//                 every row of the group (lane = key for the scores, lane =
+//                 two head dimensions for Vg), the four quarters are merged
+//                 in shared memory into the chunk's fp32 partials (max, sum,
+//                 unnormalised output), and the last CTA of a group merges
+//                 the chunks by log-sum-exp into the output rows.
+//   band CTAs     8 query rows of one (batch, head, residue class of the
+//                 dilation), 16 threads per row; each thread takes 4 of the
+//                 64 keys of a staged tile with the full 64-wide dot product
+//                 (no reduction per score), the row's threads share the
+//                 running maximum, and their partial sums and outputs are
+//                 added up once at the end.  Keys stream through shared
+//                 memory in 64-key tiles (cp.async, three stages): the
+//                 window taps, then the global-token columns that are not
+//                 taps.  Writes every row except valid global rows (zeros
+//                 for padding).
+//
+// Shared-memory rows of K/V are 68 floats apart, so 16-byte reads of
+// different rows at the same column fall in distinct banks.  The launch is
+// chained to the mask-preparation kernel by programmatic dependent launch.
 //
 // ("LongFormer: The Long-Document Transformer" notes, "Sliding Window",
 // "Dilated Sliding Window", "Global Attention"; FasterTransformer Longformer
 // Encoder guide, "compute flow": softmax of local rows over window + global
 // tokens, of global rows over the whole sequence, masked rows zeroed.)
 #include "lf_device.cuh"
-#include "lf_vec.cuh"
 
 namespace lf {
 
-constexpr int kSimtRows = 32;                     // query rows per band CTA
-constexpr int kSimtThreads = 4 * kSimtRows;       // four threads per row
-constexpr int kSimtParts = 128 / kSimtRows;       // band CTAs per 128-row band item
-constexpr int kSimtKeys = 32;
+constexpr int kF32Threads = 128;
+constexpr int kBandRows = 8;                      // query rows per band CTA
+constexpr int kTpr = 16;                          // threads per row
+constexpr int kBandParts = 128 / kBandRows;       // band CTAs per 128-row band item
+constexpr int kTileKeysF = 64;                    // keys per staged band tile
+constexpr int kKpt = kTileKeysF / kTpr;           // keys per thread and tile
+constexpr int kStride = 68;                       // floats between staged rows
+constexpr int kBandStages = 3;
+constexpr int kGWarps = 4;
+constexpr int kGKeys = 32;                        // keys per warp tile (lane = key)
+constexpr int kGQuarter = kChunkKeys / kGWarps;   // 128 keys of a chunk per warp
+constexpr float kRescaleF = 8.f;                  // lazy rescale (log2 units)
 
-// One staged tile of 32 keys: each thread holds 4 of the 512 four-element
-// pieces of K and of V (key c = tid/16 + 8u, dims 4*(tid%16) .. +3), loaded
-// into registers while the previous tile is being consumed.
-struct KvStage {
-    float4 k[4], v[4];
-    int pos[4];
+struct BandSmem {
+    float k[kBandStages][kTileKeysF][kStride];
+    float v[kBandStages][kTileKeysF][kStride];
+    int pos[kBandStages][kTileKeysF];             // sequence position, -1 = not a key
 };
 
-// One CTA per 32 query rows (a quarter of a 128-row band item); four threads
-// per row, each holding a quarter of the head dimension of q and of the
-// accumulator.  Scores are reduced over the four threads with two shuffles.
-template <typename T>
-__global__ void __launch_bounds__(kSimtThreads)
-band_simt_kernel(const AttnArgs a)
-{
-    __shared__ __align__(16) float ks[kSimtKeys][kDHead];
-    __shared__ __align__(16) float vs[kSimtKeys][kDHead];
-    __shared__ float ss[kSimtKeys][kSimtRows];   // scores, column = row of this CTA
-    __shared__ int kpos[kSimtKeys];    // sequence position of each staged key, -1 = not a key
+struct GlobSmem {
+    float q[kSlotGroup][kDHead];                  // Qg rows, scaled by log2(e)/sqrt(d)
+    float k[kGWarps][kGKeys][kStride];
+    float v[kGWarps][kGKeys][kDHead];
+    int ok[kGWarps][kGKeys];
+    float st[kGWarps][kSlotGroup][kPartialFloats];   // per warp and row: m, l, acc[64]
+};
 
+constexpr size_t kF32Smem = sizeof(BandSmem) > sizeof(GlobSmem) ? sizeof(BandSmem)
+                                                                 : sizeof(GlobSmem);
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid)
+{
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    const int n = valid ? 16 : 0;                  // 0: the 16 bytes are zero-filled
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(n)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ float dot64(const float (&q)[kDHead], const float *krow)
+{
+    float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+#pragma unroll
+    for (int x = 0; x < kDHead; x += 4) {
+        const float4 k4 = *reinterpret_cast<const float4 *>(krow + x);
+        d0 = fmaf(q[x], k4.x, d0);
+        d1 = fmaf(q[x + 1], k4.y, d1);
+        d2 = fmaf(q[x + 2], k4.z, d2);
+        d3 = fmaf(q[x + 3], k4.w, d3);
+    }
+    return (d0 + d1) + (d2 + d3);
+}
+
+// ------------------------------------------------------------------ band
+__device__ __forceinline__ void band_cta(const AttnArgs &a, int cta, uint8_t *smem_raw)
+{
+    BandSmem &sm = *reinterpret_cast<BandSmem *>(smem_raw);
     int b, h, r, tile;
-    band_item(a, blockIdx.x / kSimtParts, b, h, r, tile);
+    band_item(a, cta / kBandParts, b, h, r, tile);
     const int dil = a.dil[h];
     const int n = a.n;
     const int n_r = (n - r + dil - 1) / dil;
+    const int r0 = tile * 128 + (cta % kBandParts) * kBandRows;     // first residue-space row
+    if (r0 >= n_r) return;
     const int tid = threadIdx.x;
-    const int rl = tid >> 2;                        // row of this CTA
-    const int qd = tid & 3;                         // quarter of the head dimension
-    const int r0 = tile * 128 + (blockIdx.x % kSimtParts) * kSimtRows;   // first residue-space row
-    const int ir = r0 + rl;                         // row in residue space
+    const int rl = tid / kTpr, tl = tid % kTpr;
+    const int ir = r0 + rl;
     const bool row_in = ir < n_r;
-    const int i = ir * dil + r;                     // sequence position
+    const int i = ir * dil + r;
     const size_t bh = size_t(b) * a.H + h;
-    const T *Q = static_cast<const T *>(a.q) + bh * n * kDHead;
-    const T *K = static_cast<const T *>(a.k) + bh * n * kDHead;
-    const T *V = static_cast<const T *>(a.v) + bh * n * kDHead;
+    const float *Q = static_cast<const float *>(a.q) + bh * n * kDHead;
+    const float *K = static_cast<const float *>(a.k) + bh * n * kDHead;
+    const float *V = static_cast<const float *>(a.v) + bh * n * kDHead;
     const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
     const uint32_t *gb = a.ws.gbits + size_t(b) * a.L.nwords;
-    if (tid == 0 && blockIdx.x % kSimtParts == 0 && a.ws.counts[b] > a.max_global)
-        set_status(a.ws.status, kErrGlobalOverflow);
-    if (r0 >= n_r) return;                          // no rows in this quarter
+    const int g = min(a.ws.counts[b], a.max_global);
+    const int *gl = a.ws.gidx + size_t(b) * n;
 
-    constexpr int kQ = kDHead / 4;                  // 16 dimensions per thread
-    float q[kQ], acc[kQ];
+    const int rows_hi = min(r0 + kBandRows - 1, n_r - 1);
+    const int lo = max(a.causal ? r0 - (a.window - 1) : r0 - a.half, 0);
+    const int hi = min(a.causal ? rows_hi : rows_hi + a.half, n_r - 1);
+    const int nband = (hi - lo) / kTileKeysF + 1;
+    const int ntiles = nband + (g + kTileKeysF - 1) / kTileKeysF;
+
+    // Loads tile t into its stage: thread t handles key tid/2, half a row.
+    auto issue = [&](int t) {
+        if (t < ntiles) {
+            const int st = t % kBandStages;
+            const int c = tid >> 1;
+            int j;
+            if (t < nband) {
+                const int jr = lo + kTileKeysF * t + c;
+                j = jr <= hi ? jr * dil + r : -1;
+            } else {
+                const int slot = kTileKeysF * (t - nband) + c;
+                j = slot < g ? gl[slot] : -1;
+            }
+            const float *ks = K + size_t(j < 0 ? 0 : j) * kDHead;
+            const float *vs = V + size_t(j < 0 ? 0 : j) * kDHead;
+            const int f0 = (tid & 1) * 32;
 #pragma unroll
-    for (int x = 0; x < kQ; x += 4) {
-        const float4 t = row_in ? load4(Q + size_t(i) * kDHead + kQ * qd + x)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-        q[x] = t.x * a.scale_log2;
-        q[x + 1] = t.y * a.scale_log2;
-        q[x + 2] = t.z * a.scale_log2;
-        q[x + 3] = t.w * a.scale_log2;
+            for (int f = 0; f < 32; f += 4) {
+                cp_async16(&sm.k[st][c][f0 + f], ks + f0 + f, j >= 0);
+                cp_async16(&sm.v[st][c][f0 + f], vs + f0 + f, j >= 0);
+            }
+            if ((tid & 1) == 0) sm.pos[st][c] = (j >= 0 && bit_at(vb, j)) ? j : -1;
+        }
+        cp_async_commit();
+    };
+    for (int t = 0; t < kBandStages - 1; ++t) issue(t);
+
+    float q[kDHead], acc[kDHead];
+#pragma unroll
+    for (int x = 0; x < kDHead; x += 4) {
+        const float4 t4 = row_in ? __ldg(reinterpret_cast<const float4 *>(Q + size_t(i) * kDHead + x))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+        q[x] = t4.x * a.scale_log2;
+        q[x + 1] = t4.y * a.scale_log2;
+        q[x + 2] = t4.z * a.scale_log2;
+        q[x + 3] = t4.w * a.scale_log2;
         acc[x] = acc[x + 1] = acc[x + 2] = acc[x + 3] = 0.f;
     }
     float m = -INFINITY, l = 0.f;
 
-    // Residue-space key range covered by the rows of this CTA.
-    const int rows_hi = min(r0 + kSimtRows - 1, n_r - 1);
-    int lo, hi;
-    if (a.causal) {
-        lo = r0 - (a.window - 1);
-        hi = rows_hi;
-    } else {
-        lo = r0 - a.half;
-        hi = rows_hi + a.half;
-    }
-    lo = max(lo, 0);
-    hi = min(hi, n_r - 1);
-
-    // Pass 1 puts the scores of the staged keys in shared memory, pass 2
-    // takes the exponentials and accumulates P V.
-    auto consume = [&](int k0, bool band_tile) {
+    for (int t = 0; t < ntiles; ++t) {
+        issue(t + kBandStages - 1);
+        cp_async_wait<kBandStages - 1>();
+        __syncthreads();
+        const int st = t % kBandStages;
+        const bool band_tile = t < nband;
+        float s[kKpt];
         float tmax = -INFINITY;
-#pragma unroll 2
-        for (int c = 0; c < kSimtKeys; ++c) {
-            float d0 = 0.f, d1 = 0.f;
 #pragma unroll
-            for (int x = 0; x < kQ; x += 4) {
-                const float4 kv = *reinterpret_cast<const float4 *>(&ks[c][kQ * qd + x]);
-                d0 = fmaf(q[x], kv.x, d0);
-                d1 = fmaf(q[x + 1], kv.y, d1);
-                d0 = fmaf(q[x + 2], kv.z, d0);
-                d1 = fmaf(q[x + 3], kv.w, d1);
-            }
-            float dot = d0 + d1;
-            dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-            dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-            const int j = kpos[c];
+        for (int u = 0; u < kKpt; ++u) {
+            const int c = tl + kTpr * u;
+            const int j = sm.pos[st][c];
             bool ok = row_in && j >= 0;
             if (ok) {
                 if (band_tile) {
-                    const int jr = k0 + c;
+                    const int jr = lo + kTileKeysF * t + c;
                     ok = a.causal ? (jr <= ir && ir - jr <= a.window - 1)
                                   : (jr - ir <= a.half && ir - jr <= a.half);
                 } else {
                     ok = !is_tap(i, j, a.window, a.half, dil, a.causal);
                 }
             }
-            const float sc = ok ? dot : -INFINITY;
-            if (qd == 0) ss[c][rl] = sc;
-            tmax = fmaxf(tmax, sc);
+            s[u] = ok ? dot64(q, &sm.k[st][c][0]) : -INFINITY;
+            tmax = fmaxf(tmax, s[u]);
         }
-        __syncwarp();
-        const float mnew = fmaxf(m, tmax);
-        const float base = (mnew == -INFINITY) ? 0.f : mnew;
-        const float corr = exp2f(m - base);
-        l *= corr;
 #pragma unroll
-        for (int x = 0; x < kQ; ++x) acc[x] *= corr;
-#pragma unroll 2
-        for (int c = 0; c < kSimtKeys; ++c) {
-            const float p = exp2f(ss[c][rl] - base);
+        for (int o = 1; o < kTpr; o <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+        if (tmax > m + kRescaleF || (m == -INFINITY && tmax != -INFINITY)) {
+            const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - tmax);
+            m = tmax;
+            l *= alpha;
+#pragma unroll
+            for (int x = 0; x < kDHead; ++x) acc[x] *= alpha;
+        }
+        const float base = (m == -INFINITY) ? 0.f : m;
+#pragma unroll
+        for (int u = 0; u < kKpt; ++u) {
+            const float p = exp2f(s[u] - base);
             l += p;
+            const float *vrow = &sm.v[st][tl + kTpr * u][0];
 #pragma unroll
-            for (int x = 0; x < kQ; x += 4) {
-                const float4 vv = *reinterpret_cast<const float4 *>(&vs[c][kQ * qd + x]);
-                acc[x] = fmaf(p, vv.x, acc[x]);
-                acc[x + 1] = fmaf(p, vv.y, acc[x + 1]);
-                acc[x + 2] = fmaf(p, vv.z, acc[x + 2]);
-                acc[x + 3] = fmaf(p, vv.w, acc[x + 3]);
+            for (int x = 0; x < kDHead; x += 4) {
+                const float4 v4 = *reinterpret_cast<const float4 *>(vrow + x);
+                acc[x] = fmaf(p, v4.x, acc[x]);
+                acc[x + 1] = fmaf(p, v4.y, acc[x + 1]);
+                acc[x + 2] = fmaf(p, v4.z, acc[x + 2]);
+                acc[x + 3] = fmaf(p, v4.w, acc[x + 3]);
             }
         }
-        __syncwarp();
-        m = mnew;
-    };
-
-    // Key tiles: the window taps, 32 residue-space keys at a time, then the
-    // global-token columns (keys that are not already window taps), 32 slots
-    // at a time.  The next tile's loads are in flight during each consume.
-    int g = a.ws.counts[b];
-    g = min(g, a.max_global);
-    const int *gl = a.ws.gidx + size_t(b) * n;
-    const int nband = hi >= lo ? (hi - lo) / kSimtKeys + 1 : 0;
-    const int ntiles = nband + (g + kSimtKeys - 1) / kSimtKeys;
-    const int x4 = 4 * (tid & 15);
-    auto fetch = [&](int t, KvStage &st) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int c = (tid >> 4) + 8 * u;
-            int j;
-            if (t < nband) {
-                const int jr = lo + kSimtKeys * t + c;
-                j = (jr <= hi && jr * dil + r < n) ? jr * dil + r : -1;
-            } else {
-                const int slot = kSimtKeys * (t - nband) + c;
-                j = slot < g ? gl[slot] : -1;
-            }
-            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-            st.k[u] = j >= 0 ? load4(K + size_t(j) * kDHead + x4) : z;
-            st.v[u] = j >= 0 ? load4(V + size_t(j) * kDHead + x4) : z;
-            st.pos[u] = (j >= 0 && bit_at(vb, j)) ? j : -1;
-        }
-    };
-    KvStage st;
-    if (ntiles > 0) fetch(0, st);
-    for (int t = 0; t < ntiles; ++t) {
         __syncthreads();
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int c = (tid >> 4) + 8 * u;
-            *reinterpret_cast<float4 *>(&ks[c][x4]) = st.k[u];
-            *reinterpret_cast<float4 *>(&vs[c][x4]) = st.v[u];
-            if (x4 == 0) kpos[c] = st.pos[u];
-        }
-        __syncthreads();
-        if (t + 1 < ntiles) fetch(t + 1, st);
-        consume(lo + kSimtKeys * t, t < nband);
     }
+    cp_async_wait<0>();
 
-    if (!row_in) return;
-    T *O = static_cast<T *>(a.out) + bh * n * kDHead + size_t(i) * kDHead + kQ * qd;
-    if (!bit_at(vb, i)) {
+    // Sum over the row's 16 threads: l by shuffles, acc through shared memory
+    // (the staging area is free now); thread tl then owns dims 4tl .. 4tl+3.
 #pragma unroll
-        for (int x = 0; x < kQ; x += 4) store4(O + x, make_float4(0.f, 0.f, 0.f, 0.f));
+    for (int o = 1; o < kTpr; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    __syncthreads();
+    float *red = &sm.k[0][0][0];                  // [kBandRows][kTpr][kDHead + 4]
+    float *mine = red + (rl * kTpr + tl) * (kDHead + 4);
+#pragma unroll
+    for (int x = 0; x < kDHead; x += 4)
+        *reinterpret_cast<float4 *>(mine + x) = make_float4(acc[x], acc[x + 1], acc[x + 2], acc[x + 3]);
+    __syncthreads();
+    float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kTpr; ++w) {
+        const float4 p4 = *reinterpret_cast<const float4 *>(red + (rl * kTpr + w) * (kDHead + 4) + 4 * tl);
+        o4.x += p4.x;
+        o4.y += p4.y;
+        o4.z += p4.z;
+        o4.w += p4.w;
+    }
+    if (!row_in) return;
+    float *O = static_cast<float *>(a.out) + bh * n * kDHead + size_t(i) * kDHead + 4 * tl;
+    if (!bit_at(vb, i)) {
+        *reinterpret_cast<float4 *>(O) = make_float4(0.f, 0.f, 0.f, 0.f);
         return;
     }
-    if (bit_at(gb, i)) return;     // written by the global-row kernel
+    if (bit_at(gb, i)) return;     // written by the global rows
     const float inv = 1.f / l;
-#pragma unroll
-    for (int x = 0; x < kQ; x += 4)
-        store4(O + x, make_float4(acc[x] * inv, acc[x + 1] * inv, acc[x + 2] * inv, acc[x + 3] * inv));
+    *reinterpret_cast<float4 *>(O) = make_float4(o4.x * inv, o4.y * inv, o4.z * inv, o4.w * inv);
 }
 
-constexpr int kGlobWarps = 4;
-constexpr int kGlobSlotsPerWarp = kSlotGroup / kGlobWarps;   // 8
-constexpr int kGlobKeys = 64;
-
-template <typename T>
-__global__ void __launch_bounds__(kGlobWarps * 32)
-global_simt_kernel(const AttnArgs a)
+// ---------------------------------------------------------------- global
+__device__ __forceinline__ void global_cta(const AttnArgs &a, int cta, uint8_t *smem_raw)
 {
-    __shared__ __align__(16) float qs[kSlotGroup][kDHead];
-    __shared__ float ks[kGlobKeys][kDHead + 1];
-    __shared__ __align__(16) float vs[kGlobKeys][kDHead];
-    __shared__ int kok[kGlobKeys];
+    GlobSmem &sm = *reinterpret_cast<GlobSmem *>(smem_raw);
     __shared__ int s_last;
-
-    const int chunk = blockIdx.x;
-    const int bh = blockIdx.y;
-    const int group = blockIdx.z;
+    const int nch = a.L.nchunks;
+    const int per_bh = nch * a.L.ngroups;
+    const int bh = cta / per_bh;
+    const int rem = cta - bh * per_bh;
+    const int group = rem / nch;
+    const int chunk = rem - group * nch;
     const int b = bh / a.H;
     const int n = a.n;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    int g = min(a.ws.counts[b], a.max_global);
-    if (a.ws.counts[b] > a.max_global && tid == 0 && chunk == 0 && group == 0 && (bh % a.H) == 0)
-        set_status(a.ws.status, kErrGlobalOverflow);
+    const int g = min(a.ws.counts[b], a.max_global);
     const int slot0 = group * kSlotGroup;
     if (slot0 >= g) return;
+    const int rows = min(kSlotGroup, g - slot0);
     const int *gl = a.ws.gidx + size_t(b) * n;
     const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
-    const T *Qg = static_cast<const T *>(a.qg) + size_t(bh) * n * kDHead;
-    const T *Kg = static_cast<const T *>(a.kg) + size_t(bh) * n * kDHead;
-    const T *Vg = static_cast<const T *>(a.vg) + size_t(bh) * n * kDHead;
+    const float *Qg = static_cast<const float *>(a.qg) + size_t(bh) * n * kDHead;
+    const float *Kg = static_cast<const float *>(a.kg) + size_t(bh) * n * kDHead;
+    const float *Vg = static_cast<const float *>(a.vg) + size_t(bh) * n * kDHead;
 
-    const int x4 = 4 * (tid & 15);
-#pragma unroll
-    for (int u = 0; u < kSlotGroup / 8; ++u) {
-        const int s = (tid >> 4) + 8 * u;
-        const int slot = slot0 + s;
-        const float4 t = slot < g ? load4(Qg + size_t(gl[slot]) * kDHead + x4)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4 *>(&qs[s][x4]) =
-            make_float4(t.x * a.scale_log2, t.y * a.scale_log2, t.z * a.scale_log2,
-                        t.w * a.scale_log2);
+    for (int e = tid; e < kSlotGroup * (kDHead / 4); e += kF32Threads) {
+        const int s = e / (kDHead / 4), x = 4 * (e % (kDHead / 4));
+        float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (s < rows) t4 = __ldg(reinterpret_cast<const float4 *>(Qg + size_t(gl[slot0 + s]) * kDHead + x));
+        *reinterpret_cast<float4 *>(&sm.q[s][x]) =
+            make_float4(t4.x * a.scale_log2, t4.y * a.scale_log2, t4.z * a.scale_log2,
+                        t4.w * a.scale_log2);
     }
-
-    float m[kGlobSlotsPerWarp], l[kGlobSlotsPerWarp], acc0[kGlobSlotsPerWarp],
-        acc1[kGlobSlotsPerWarp];
-#pragma unroll
-    for (int t = 0; t < kGlobSlotsPerWarp; ++t) {
-        m[t] = -INFINITY;
-        l[t] = 0.f;
-        acc0[t] = 0.f;
-        acc1[t] = 0.f;
+    // Per-warp running state of every row: m, l, and lane's two dimensions.
+    float *stw = &sm.st[warp][0][0];
+    for (int s = lane; s < kSlotGroup; s += 32) {
+        stw[s * kPartialFloats] = -INFINITY;
+        stw[s * kPartialFloats + 1] = 0.f;
     }
+    for (int s = 0; s < kSlotGroup; ++s) {
+        stw[s * kPartialFloats + 2 + 2 * lane] = 0.f;
+        stw[s * kPartialFloats + 3 + 2 * lane] = 0.f;
+    }
+    __syncthreads();
 
-    // Key tiles of 64: each thread holds 8 of the 1024 four-element pieces of
-    // Kg and of Vg (key c = tid/16 + 8u), loaded while the previous tile is
-    // being consumed.
-    const int key_begin = chunk * kChunkKeys;
-    const int key_end = min(n, key_begin + kChunkKeys);
-    constexpr int kPieces = kGlobKeys / 8;
-    float4 kr[kPieces], vr[kPieces];
-    auto fetch = [&](int k0) {
+    const int key_end = min(n, (chunk + 1) * kChunkKeys);
+    const int kbeg = chunk * kChunkKeys + warp * kGQuarter;
+    const int kend = min(key_end, kbeg + kGQuarter);
+    for (int k0 = kbeg; k0 < kend; k0 += kGKeys) {
+        // This warp's tile: lane = key.
+        const int j = k0 + lane;
+        const bool in = j < kend;
+        const float *ks = Kg + size_t(in ? j : 0) * kDHead;
+        const float *vs = Vg + size_t(in ? j : 0) * kDHead;
 #pragma unroll
-        for (int u = 0; u < kPieces; ++u) {
-            const int j = k0 + (tid >> 4) + 8 * u;
-            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-            kr[u] = j < key_end ? load4(Kg + size_t(j) * kDHead + x4) : z;
-            vr[u] = j < key_end ? load4(Vg + size_t(j) * kDHead + x4) : z;
+        for (int f = 0; f < kDHead; f += 4) {
+            cp_async16(&sm.k[warp][lane][f], ks + f, in);
+            cp_async16(&sm.v[warp][lane][f], vs + f, in);
         }
-    };
-    fetch(key_begin);
-    for (int k0 = key_begin; k0 < key_end; k0 += kGlobKeys) {
-        __syncthreads();
+        cp_async_commit();
+        sm.ok[warp][lane] = in && bit_at(vb, j);
+        cp_async_wait<0>();
+        __syncwarp();
+        const bool ok = sm.ok[warp][lane];
+        for (int s = 0; s < rows; ++s) {
+            float qv[kDHead];
 #pragma unroll
-        for (int u = 0; u < kPieces; ++u) {
-            const int c = (tid >> 4) + 8 * u;
-            ks[c][x4] = kr[u].x;
-            ks[c][x4 + 1] = kr[u].y;
-            ks[c][x4 + 2] = kr[u].z;
-            ks[c][x4 + 3] = kr[u].w;
-            *reinterpret_cast<float4 *>(&vs[c][x4]) = vr[u];
-        }
-        if (tid < kGlobKeys) kok[tid] = k0 + tid < key_end && bit_at(vb, k0 + tid);
-        __syncthreads();
-        if (k0 + kGlobKeys < key_end) fetch(k0 + kGlobKeys);
-#pragma unroll
-        for (int t = 0; t < kGlobSlotsPerWarp; ++t) {
-            const int s = warp * kGlobSlotsPerWarp + t;
-            if (slot0 + s >= g) break;
-            float s0 = 0.f, s1 = 0.f;
-#pragma unroll 16
-            for (int x = 0; x < kDHead; ++x) {
-                s0 = fmaf(qs[s][x], ks[lane][x], s0);
-                s1 = fmaf(qs[s][x], ks[lane + 32][x], s1);
+            for (int x = 0; x < kDHead; x += 4) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(&sm.q[s][x]);
+                qv[x] = t4.x;
+                qv[x + 1] = t4.y;
+                qv[x + 2] = t4.z;
+                qv[x + 3] = t4.w;
             }
-            s0 = kok[lane] ? s0 : -INFINITY;
-            s1 = kok[lane + 32] ? s1 : -INFINITY;
-            float tmax = fmaxf(s0, s1);
+            const float sc = ok ? dot64(qv, &sm.k[warp][lane][0]) : -INFINITY;
+            float tmax = sc;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
-            const float mnew = fmaxf(m[t], tmax);
-            const float base = (mnew == -INFINITY) ? 0.f : mnew;
-            const float corr = exp2f(m[t] - base);
-            const float p0 = exp2f(s0 - base), p1 = exp2f(s1 - base);
-            float psum = p0 + p1;
+            float *row = stw + s * kPartialFloats;
+            float mr = row[0], lr = row[1];
+            float a0 = row[2 + 2 * lane], a1 = row[3 + 2 * lane];
+            if (tmax > mr + kRescaleF || (mr == -INFINITY && tmax != -INFINITY)) {
+                const float alpha = (mr == -INFINITY) ? 0.f : exp2f(mr - tmax);
+                mr = tmax;
+                lr *= alpha;
+                a0 *= alpha;
+                a1 *= alpha;
+            }
+            const float base = (mr == -INFINITY) ? 0.f : mr;
+            const float p = exp2f(sc - base);
+            float psum = p;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
-            l[t] = l[t] * corr + psum;
-            float a0 = acc0[t] * corr, a1 = acc1[t] * corr;
+            lr += psum;
 #pragma unroll 8
-            for (int c = 0; c < 32; ++c) {
-                const float pa = __shfl_sync(0xffffffffu, p0, c);
-                const float pb = __shfl_sync(0xffffffffu, p1, c);
-                a0 = fmaf(pa, vs[c][2 * lane], a0);
-                a1 = fmaf(pa, vs[c][2 * lane + 1], a1);
-                a0 = fmaf(pb, vs[c + 32][2 * lane], a0);
-                a1 = fmaf(pb, vs[c + 32][2 * lane + 1], a1);
+            for (int c = 0; c < kGKeys; ++c) {
+                const float pc = __shfl_sync(0xffffffffu, p, c);
+                const float2 v2 = *reinterpret_cast<const float2 *>(&sm.v[warp][c][2 * lane]);
+                a0 = fmaf(pc, v2.x, a0);
+                a1 = fmaf(pc, v2.y, a1);
             }
-            acc0[t] = a0;
-            acc1[t] = a1;
-            m[t] = mnew;
+            __syncwarp();
+            if (lane == 0) {
+                row[0] = mr;
+                row[1] = lr;
+            }
+            row[2 + 2 * lane] = a0;
+            row[3 + 2 * lane] = a1;
+            __syncwarp();
         }
     }
+    __syncthreads();
 
-    // Partials of this chunk.
+    // Merge the four quarters of the chunk into its partials: warp w takes
+    // rows w, w+4, ...; lane owns two dimensions.
+    const size_t mg = size_t(a.max_global);
+    for (int s = warp; s < rows; s += kGWarps) {
+        float M = -INFINITY;
 #pragma unroll
-    for (int t = 0; t < kGlobSlotsPerWarp; ++t) {
-        const int slot = slot0 + warp * kGlobSlotsPerWarp + t;
-        if (slot >= g) break;
-        float *P = partial_base(a, bh, chunk) + slot;
-        const size_t mg = size_t(a.max_global);
-        if (lane == 0) {
-            P[0] = m[t];
-            P[mg] = l[t];
+        for (int w = 0; w < kGWarps; ++w) M = fmaxf(M, sm.st[w][s][0]);
+        float L = 0.f, a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int w = 0; w < kGWarps; ++w) {
+            const float mw = sm.st[w][s][0];
+            const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+            L = fmaf(f, sm.st[w][s][1], L);
+            a0 = fmaf(f, sm.st[w][s][2 + 2 * lane], a0);
+            a1 = fmaf(f, sm.st[w][s][3 + 2 * lane], a1);
         }
-        P[(2 + 2 * lane) * mg] = acc0[t];
-        P[(3 + 2 * lane) * mg] = acc1[t];
+        float *P = partial_base(a, bh, chunk) + slot0 + s;
+        if (lane == 0) {
+            P[0] = M;
+            P[mg] = L;
+        }
+        P[(2 + 2 * lane) * mg] = a0;
+        P[(3 + 2 * lane) * mg] = a1;
     }
 
     // The last CTA of this (bh, group) to finish merges every chunk.
@@ -356,36 +389,61 @@ global_simt_kernel(const AttnArgs a)
     if (tid == 0) {
         int *ctr = a.ws.counters + size_t(bh) * (a.L.ngroups + 1) + group;
         const int prev = atomicAdd(ctr, 1);
-        s_last = (prev == int(gridDim.x) - 1);
+        s_last = (prev == nch - 1);
         if (s_last) *ctr = 0;
     }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    T *Out = static_cast<T *>(a.out) + size_t(bh) * n * kDHead;
-    for (int s = warp; s < kSlotGroup; s += kGlobWarps) {
+    float *Out = static_cast<float *>(a.out) + size_t(bh) * n * kDHead;
+    for (int s = warp; s < rows; s += kGWarps) {
         const int slot = slot0 + s;
-        if (slot >= g) break;
         const int p = gl[slot];
-        if (!bit_at(vb, p)) continue;   // padded global position: the band kernel wrote zeros
-        combine_row_partials<T>(a, bh, slot, gridDim.x, lane, Out + size_t(p) * kDHead);
+        if (!bit_at(vb, p)) continue;   // padded global position: the band CTAs wrote zeros
+        combine_row_partials<float>(a, bh, slot, nch, lane, Out + size_t(p) * kDHead);
     }
 }
 
-template <typename T>
-int launch_simt(const AttnArgs &a, cudaStream_t stream)
+__global__ void __launch_bounds__(kF32Threads) attn_f32_kernel(const AttnArgs a, int nglob)
 {
-    const int band_items = a.B * a.band_items_per_batch;
-    if (band_items > 0) band_simt_kernel<T><<<band_items * kSimtParts, kSimtThreads, 0, stream>>>(a);
-    if (a.max_global > 0) {
-        dim3 grid(a.L.nchunks, a.B * a.H, a.L.ngroups);
-        global_simt_kernel<T><<<grid, kGlobWarps * 32, 0, stream>>>(a);
+    extern __shared__ __align__(16) uint8_t f32_smem[];
+    // The compacted indices, counts and bitmaps come from the kernel before.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (blockIdx.x == 0)
+        for (int b = threadIdx.x; b < a.B; b += kF32Threads)
+            if (a.ws.counts[b] > a.max_global) set_status(a.ws.status, kErrGlobalOverflow);
+    if (int(blockIdx.x) < nglob)
+        global_cta(a, blockIdx.x, f32_smem);
+    else
+        band_cta(a, blockIdx.x - nglob, f32_smem);
+}
+
+int launch_f32(const AttnArgs &a, cudaStream_t stream)
+{
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(attn_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(kF32Smem)) != cudaSuccess)
+            return kErrCuda;
+        attr_set[dev] = true;
     }
+    // Global CTAs first: they hold the longest key ranges.
+    const int nglob = a.max_global > 0 ? a.B * a.H * a.L.nchunks * a.L.ngroups : 0;
+    const int nband = a.B * a.band_items_per_batch * kBandParts;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nglob + nband);
+    cfg.blockDim = dim3(kF32Threads);
+    cfg.dynamicSmemBytes = kF32Smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, attn_f32_kernel, a, nglob) != cudaSuccess) return kErrCuda;
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
-
-template int launch_simt<float>(const AttnArgs &, cudaStream_t);
-template int launch_simt<__half>(const AttnArgs &, cudaStream_t);
-template int launch_simt<__nv_bfloat16>(const AttnArgs &, cudaStream_t);
 
 }  // namespace lf
