@@ -767,13 +767,32 @@ struct RowState {
     float m, l;
 };
 
-// Online softmax of one 128-key score tile for this thread's row.  mw[c]
-// marks the keys of this row among columns [32c, 32c+32); a chunk that is
-// empty for every row of the warp is skipped (its probabilities are zero)
-// and a chunk that is full for every row is not masked.  Writes P =
-// 2^(S*scale*log2e - m) as 16-bit pairs over the first 64 columns of the tile
-// and adds the row sum.  O is rescaled in TMEM only when the running maximum
-// grows by more than 2^8; every PV before this tile has completed then.
+template <typename T> __device__ __forceinline__ void unpack2(uint32_t w, float &lo, float &hi);
+template <> __device__ __forceinline__ void unpack2<__nv_bfloat16>(uint32_t w, float &lo, float &hi)
+{
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w));
+    lo = f.x;
+    hi = f.y;
+}
+template <> __device__ __forceinline__ void unpack2<__half>(uint32_t w, float &lo, float &hi)
+{
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w));
+    lo = f.x;
+    hi = f.y;
+}
+
+// Online softmax of one 128-key score tile for this thread's row, 32 keys at
+// a time (one compact loop: the code stays small enough for the instruction
+// caches shared with the producer and MMA warps).  mw[c] marks the keys of
+// this row among columns [32c, 32c+32); a chunk that is empty for every row
+// of the warp is skipped (its probabilities are zero) and a chunk that is
+// full for every row is not masked.  P = 2^(S*scale*log2e - m) goes as 16-bit
+// pairs over the first 64 columns of the tile (chunk c to packed columns
+// [16c, 16c+16), which hold scores already read).  The running maximum m is
+// kept lazily: it moves only when a chunk's maximum exceeds it by more than
+// 2^8; then the row sum, the probabilities already written in this tile and,
+// at the end of the tile, O (every PV before this tile has completed) are
+// scaled by the same factor.
 template <typename T>
 __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, RowState &st, bool first,
                                              const uint32_t (&mw)[4], float sl2)
@@ -784,79 +803,84 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, RowState 
         any_m |= (__any_sync(0xffffffffu, mw[c] != 0u) ? 1u : 0u) << c;
         full_m |= (__all_sync(0xffffffffu, mw[c] == 0xffffffffu) ? 1u : 0u) << c;
     }
-    float s[128];
-    tmem_ld128(tS, s);
-    float mc[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        mc[c] = -INFINITY;
-        if ((any_m >> c) & 1u) {
-            if (!((full_m >> c) & 1u)) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    s[32 * c + i] = ((mw[c] >> i) & 1u) ? s[32 * c + i] : -INFINITY;
-            }
-            mc[c] = max32(&s[32 * c]);
-        }
-    }
-    const float mt = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])) * sl2;
-    float alpha = 1.f;
-    bool rescale = false;
     if (first) {
-        st.m = mt;
+        st.m = -INFINITY;
         st.l = 0.f;
-    } else if (mt > st.m + kRescaleLog2) {
-        alpha = ex2(st.m - mt);
-        st.m = mt;
-        rescale = true;
     }
-    const float nb = (st.m == -INFINITY) ? 0.f : -st.m;
-    float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
-    // Two halves of 64 keys: each half's 32 packed columns are stored as soon
-    // as they are ready, which bounds the registers held at once.
+    float m = st.m, l = st.l;
+    float alpha_o = 1.f;        // factor O must take for this tile's new maxima
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+        if ((any_m >> c) & 1u) {
+            float s[32];
+            tmem_ld32(tS + 32 * c, s);
+            if (!((full_m >> c) & 1u)) {
+                const uint32_t mc = c == 0 ? mw[0] : c == 1 ? mw[1] : c == 2 ? mw[2] : mw[3];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * h + cc;
-            if ((any_m >> c) & 1u) {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int q = 16 * c + i;
-                    float x0, x1, p0, p1;
-                    fma2(x0, x1, s[2 * q], s[2 * q + 1], sl2, sl2, nb, nb);
-                    if ((kPolyPairs >> (q & 7)) & 1u) {
-                        exp2_poly2(x0, x1, p0, p1);
-                    } else {
-                        p0 = ex2(x0);
-                        p1 = ex2(x1);
-                    }
-                    if (i & 1)
-                        add2(sb0, sb1, sb0, sb1, p0, p1);
-                    else
-                        add2(sa0, sa1, sa0, sa1, p0, p1);
-                    pk[16 * cc + i] = pack2<T>(p0, p1);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) pk[16 * cc + i] = 0u;
+                for (int i = 0; i < 32; ++i) s[i] = ((mc >> i) & 1u) ? s[i] : -INFINITY;
             }
-        }
-        tmem_st32(tS + 32 * h, pk);
-    }
-    if (__any_sync(0xffffffffu, rescale)) {
+            const float cmax = max32(s) * sl2;
+            const bool need = cmax > m + kRescaleLog2;
+            if (__any_sync(0xffffffffu, need)) {
+                const float a = !need ? 1.f : (m == -INFINITY ? 0.f : ex2(m - cmax));
+                if (need) m = cmax;
+                l *= a;
+                alpha_o *= a;
+                // Probabilities of earlier chunks of this tile were taken against
+                // the old maximum.
+                if (__any_sync(0xffffffffu, a != 1.f && a != 0.f)) {
+                    for (int c2 = 0; c2 < c; ++c2) {
+                        float w[16];
+                        tmem_ld16(tS + 16 * c2, w);
+                        uint32_t r[16];
 #pragma unroll
+                        for (int x = 0; x < 16; ++x) {
+                            float lo, hi;
+                            unpack2<T>(__float_as_uint(w[x]), lo, hi);
+                            r[x] = pack2<T>(lo * a, hi * a);
+                        }
+                        tmem_st16(tS + 16 * c2, r);
+                    }
+                }
+            }
+            const float nb = (m == -INFINITY) ? 0.f : -m;
+            float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float x0, x1, p0, p1;
+                fma2(x0, x1, s[2 * i], s[2 * i + 1], sl2, sl2, nb, nb);
+                if ((kPolyPairs >> (i & 7)) & 1u) {
+                    exp2_poly2(x0, x1, p0, p1);
+                } else {
+                    p0 = ex2(x0);
+                    p1 = ex2(x1);
+                }
+                if (i & 1)
+                    add2(sb0, sb1, sb0, sb1, p0, p1);
+                else
+                    add2(sa0, sa1, sa0, sa1, p0, p1);
+                pk[i] = pack2<T>(p0, p1);
+            }
+            l += (sa0 + sa1) + (sb0 + sb1);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = 0u;
+        }
+        tmem_st16(tS + 16 * c, pk);
+    }
+    if (!first && __any_sync(0xffffffffu, alpha_o != 1.f)) {
         for (int half = 0; half < 2; ++half) {
             float o[32];
             tmem_ld32(tO + half * 32, o);
             uint32_t ob[32];
 #pragma unroll
-            for (int x = 0; x < 32; ++x) ob[x] = __float_as_uint(o[x] * alpha);
+            for (int x = 0; x < 32; ++x) ob[x] = __float_as_uint(o[x] * alpha_o);
             tmem_st32(tO + half * 32, ob);
         }
     }
-    st.l = st.l * alpha + ((sa0 + sa1) + (sb0 + sb1));
+    st.m = m;
+    st.l = l;
     tmem_st_wait();
 }
 
@@ -895,7 +919,7 @@ __device__ __forceinline__ void store_row(T *dst, const float (&o)[64], float in
 // wrote the last chunk of the group; the partials of the other chunks come
 // from other CTAs, so they are read past L1.
 template <typename T>
-__device__ __noinline__ void merge_global_rows(const AttnArgs &a, int b, int bh, int g, int slot0,
+__device__ __forceinline__ void merge_global_rows(const AttnArgs &a, int b, int bh, int g, int slot0,
                                                int lane)
 {
     const int slot = slot0 + lane;
