@@ -71,7 +71,7 @@ using namespace sm100;
 
 constexpr int kRows = 128;                        // query rows per tile (M)
 constexpr int kTileKeys = 128;                    // keys per S tile (N) / K-V stage
-constexpr int kStages = 4;                        // K/V ring depth (shared by the slots)
+constexpr int kStages = 2;                        // K and V ring depth per slot
 constexpr int kSlots = 2;
 constexpr int kRing = 4;                          // item and tile-info rings per slot
 constexpr int kQBytes = kRows * kDHead * 2;       // 16 KB of 16-bit elements
@@ -79,7 +79,7 @@ constexpr int kKvBytes = kTileKeys * kDHead * 2;  // 16 KB
 constexpr int kRowBytes = kDHead * 2;             // 128 B
 constexpr int kThreads = 384;
 constexpr int kWarpProducer = 8;
-constexpr int kWarpMma = 9;
+constexpr int kWarpTmem = 9;                      // allocates and frees the tensor memory
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlotCols = 256;               // S (128) | O0 (64) | O1 (64)
 constexpr float kRescaleLog2 = 8.f;               // lazy rescale: P stays below 2^8
@@ -152,16 +152,17 @@ struct TileMask {
 
 struct __align__(1024) FwdSmem {
     uint8_t q[kSlots][2][kQBytes];
-    uint8_t k[kStages][kKvBytes];
-    uint8_t v[kStages][kKvBytes];
+    uint8_t k[kSlots][kStages][kKvBytes];
+    uint8_t v[kSlots][kStages][kKvBytes];
     TileMask tmask[kSlots][kRing];
     ItemInfo items[kSlots][kRing];
     uint64_t q_full[kSlots][2], q_empty[kSlots][2];
-    uint64_t kv_full[kStages], kv_empty[kStages];
+    uint64_t k_full[kSlots][kStages], k_empty[kSlots][kStages];
+    uint64_t v_full[kSlots][kStages], v_empty[kSlots][kStages];
     uint64_t item_full[kSlots][kRing], item_empty[kSlots][kRing];
     uint64_t tm_full[kSlots][kRing];
-    uint64_t s_full[kSlots], p_full[kSlots], o_full[kSlots][2], o_empty[kSlots][2];
-    uint64_t drain;
+    uint64_t s_full[kSlots], p_full[kSlots], o_full[kSlots][2];
+    uint64_t drain[kSlots];
     int batch_count[kBatchCache];
     int batch_flags[kBatchCache];
     int head_dil[kMaxHeads];            // per-head tables, copied from the kernel
@@ -211,14 +212,6 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, uint6
 {
     const uint64_t t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < limit_ns) {
-    }
-}
-
-__device__ __forceinline__ void advance_ring(int &stage, uint32_t &phase)
-{
-    if (++stage == kStages) {
-        stage = 0;
-        phase ^= 1u;
     }
 }
 
@@ -429,66 +422,44 @@ __device__ __forceinline__ bool producer_q(const FwdParams &p, FwdSmem &sm, Prod
     return true;
 }
 
-// Loads tile S.t of the slot's current item into ring stage `stage` and
-// writes its column masks to the slot's tile-mask ring.
-__device__ __forceinline__ void producer_tile(const FwdParams &p, FwdSmem &sm, ProducerSlot &S,
-                                              int X, int lane, int stage)
+// Loads tile S.t of the slot's current item: its K tile (with the tile's
+// column masks in the slot's tile-mask ring) into K stage jt % kStages, then
+// its V tile into V stage jt % kStages, each once the stage has been released
+// (the K stage by the tile's QK^T two tiles back, the V stage by its PV).
+// Returns false on abort; `armed` and `par` record the copies started (bit
+// 4X + 2*stage + {0: K, 1: V}) for the drain.
+__device__ __forceinline__ bool producer_tile(const FwdParams &p, FwdSmem &sm, ProducerSlot &S,
+                                              int X, int lane, uint32_t &armed, uint32_t &par)
 {
     const AttnArgs &a = p.a;
     const ItemInfo I = sm.items[X][S.kc % kRing];
     const int t = S.t;
-    uint8_t *kd = sm.k[stage];
-    uint8_t *vd = sm.v[stage];
-    uint64_t *bar = &sm.kv_full[stage];
+    const int stage = S.jt % kStages;
+    const uint32_t phase = uint32_t(S.jt / kStages) & 1u;
+    uint8_t *kd = sm.k[X][stage];
+    uint8_t *vd = sm.v[X][stage];
+    uint64_t *kbar = &sm.k_full[X][stage];
+    uint64_t *vbar = &sm.v_full[X][stage];
     TileMask &tm = sm.tmask[X][S.jt % kRing];
     const uint32_t *vb = a.ws.vbits + size_t(I.b) * a.L.nwords;
-    if (I.kind == 2) {
-        const int k0 = I.klo + t * kTileKeys;
+    const int kind = I.kind == 2 ? 2 : (t < I.nkv ? 1 : 3);   // 3: global-token columns
+    const int k0 = I.klo + t * kTileKeys;
+    const int s0 = (t - I.nkv) * kTileKeys;
+    const int rows = tile_cols(I, t);
+    if (!warp_wait(p, sm, &sm.k_empty[X][stage], phase ^ 1u)) return false;
+    // Column masks.
+    if (kind == 2 || (kind == 1 && I.has_pad)) {
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
             const int j = k0 + 32 * w + lane;
-            const bool ok = j < I.key_end && (!I.has_pad || bit_at(vb, j));
+            const bool ok = kind == 2 ? (j < I.key_end && (!I.has_pad || bit_at(vb, j)))
+                                      : (j < I.n_r && bit_at(vb, j * I.dil + I.r));
             const uint32_t bits = __ballot_sync(0xffffffffu, ok);
             if (lane == 0) tm.bits[w] = bits;
         }
-        if (lane == 0) {
-            mbar_arrive_expect_tx(bar, 2 * kKvBytes);
-            tma_load_3d(kd, &p.maps[kMapKgTile], bar, 0, k0, I.bh);
-            tma_load_3d(vd, &p.maps[kMapVgTile], bar, 0, k0, I.bh);
-        }
-    } else if (t < I.nkv) {
-        const int k0 = I.klo + t * kTileKeys;
-        if (I.has_pad) {
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const int jr = k0 + 32 * w + lane;
-                const bool ok = jr < I.n_r && bit_at(vb, jr * I.dil + I.r);
-                const uint32_t bits = __ballot_sync(0xffffffffu, ok);
-                if (lane == 0) tm.bits[w] = bits;
-            }
-        } else if (lane < 4) {
-            tm.bits[lane] = 0xffffffffu;
-        }
-        if (I.res >= 0) {
-            if (lane == 0) {
-                mbar_arrive_expect_tx(bar, 2 * kKvBytes);
-                tma_load_3d(kd, &p.res_k[I.res], bar, 0, k0, I.bh);
-                tma_load_3d(vd, &p.res_v[I.res], bar, 0, k0, I.bh);
-            }
-        } else {
-            if (lane == 0) mbar_arrive_expect_tx(bar, 2 * kKvBytes);
-            __syncwarp();
-            for (int rr = lane; rr < kTileKeys; rr += 32) {
-                const int jr = k0 + rr;
-                const int y = jr < I.n_r ? I.bh * a.n + jr * I.dil + I.r : p.oob_row;
-                tma_load_2d(kd + rr * kRowBytes, &p.maps[kMapKRow], bar, 0, y);
-                tma_load_2d(vd + rr * kRowBytes, &p.maps[kMapVRow], bar, 0, y);
-            }
-        }
+    } else if (kind == 1) {
+        if (lane < 4) tm.bits[lane] = 0xffffffffu;
     } else {
-        // Global-token columns: the K/V rows of the global tokens, gathered.
-        const int s0 = (t - I.nkv) * kTileKeys;
-        const int rows = tile_cols(I, t);
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
             const int c = 32 * w + lane;
@@ -499,18 +470,44 @@ __device__ __forceinline__ void producer_tile(const FwdParams &p, FwdSmem &sm, P
             const uint32_t bits = __ballot_sync(0xffffffffu, ok);
             if (lane == 0) tm.bits[w] = bits;
         }
-        if (lane == 0) mbar_arrive_expect_tx(bar, 2 * rows * kRowBytes);
-        __syncwarp();
-        for (int rr = lane; rr < rows; rr += 32) {
-            const int slot = s0 + rr;
-            const int y = slot < I.g ? I.bh * a.n + a.ws.gidx[size_t(I.b) * a.n + slot]
-                                     : p.oob_row;
-            tma_load_2d(kd + rr * kRowBytes, &p.maps[kMapKRow], bar, 0, y);
-            tma_load_2d(vd + rr * kRowBytes, &p.maps[kMapVRow], bar, 0, y);
-        }
     }
-    __syncwarp();
+    // K (or V when second): a whole tile by one TMA copy, or rows one by one.
+    auto load = [&](bool is_v, uint8_t *dst, uint64_t *bar) {
+        if (kind == 2 || (kind == 1 && I.res >= 0)) {
+            if (lane == 0) {
+                const CUtensorMap *m = kind == 2 ? &p.maps[is_v ? kMapVgTile : kMapKgTile]
+                                                 : (is_v ? &p.res_v[I.res] : &p.res_k[I.res]);
+                mbar_arrive_expect_tx(bar, kKvBytes);
+                tma_load_3d(dst, m, bar, 0, k0, I.bh);
+            }
+        } else {
+            const int n_rows = kind == 1 ? kTileKeys : rows;
+            if (lane == 0) mbar_arrive_expect_tx(bar, n_rows * kRowBytes);
+            __syncwarp();
+            const CUtensorMap *m = &p.maps[is_v ? kMapVRow : kMapKRow];
+            for (int rr = lane; rr < n_rows; rr += 32) {
+                int y = p.oob_row;
+                if (kind == 1) {
+                    const int jr = k0 + rr;
+                    if (jr < I.n_r) y = I.bh * a.n + jr * I.dil + I.r;
+                } else if (s0 + rr < I.g) {
+                    y = I.bh * a.n + a.ws.gidx[size_t(I.b) * a.n + s0 + rr];
+                }
+                tma_load_2d(dst + rr * kRowBytes, m, bar, 0, y);
+            }
+        }
+        __syncwarp();
+    };
+    load(false, kd, kbar);
     if (lane == 0) mbar_arrive(&sm.tm_full[X][S.jt % kRing]);
+    const uint32_t kb = 1u << (4 * X + 2 * stage);
+    armed |= kb;
+    par = phase ? (par | kb) : (par & ~kb);
+    if (!warp_wait(p, sm, &sm.v_empty[X][stage], phase ^ 1u)) return false;
+    load(true, vd, vbar);
+    armed |= kb << 1;
+    par = phase ? (par | (kb << 1)) : (par & ~(kb << 1));
+    return true;
 }
 
 template <typename S> __device__ __forceinline__ void swap_state(S &a, S &b)
@@ -529,10 +526,8 @@ __device__ __forceinline__ void producer_role(const FwdParams &p, FwdSmem &sm, i
 {
     int *sched = p.a.ws.status + 16;
     ProducerSlot A, B;
-    uint32_t kv_armed = 0, kv_par = 0;   // bit s: stage s was filled; its parity
+    uint32_t kv_armed = 0, kv_par = 0;   // K/V copies started (see producer_tile); parities
     uint32_t qa = 0, qp = 0;             // bit 2X+b: Q buffer b of slot X was filled
-    int stage = 0;
-    uint32_t phase = 0;
     bool ok = true;
     A.kc = A.t = A.kw = A.kq = A.jt = 0;
     A.ended = false;
@@ -550,14 +545,10 @@ __device__ __forceinline__ void producer_role(const FwdParams &p, FwdSmem &sm, i
         if (!ok) break;
         const bool busy_a = A.kc < A.kw && sm.items[X][A.kc % kRing].kind != 0;
         if (busy_a) {
-            if (!warp_wait(p, sm, &sm.kv_empty[stage], phase ^ 1u)) {
+            if (!producer_tile(p, sm, A, X, lane, kv_armed, kv_par)) {
                 ok = false;
                 break;
             }
-            producer_tile(p, sm, A, X, lane, stage);
-            kv_armed |= 1u << stage;
-            kv_par = phase ? (kv_par | (1u << stage)) : (kv_par & ~(1u << stage));
-            advance_ring(stage, phase);
             ++A.jt;
             if (++A.t == sm.items[X][A.kc % kRing].ntiles) {
                 ++A.kc;
@@ -572,122 +563,14 @@ __device__ __forceinline__ void producer_role(const FwdParams &p, FwdSmem &sm, i
         X ^= 1;
     }
     if (!ok || sm.abort_flag) {
-        for (int s = 0; s < kStages; ++s)
-            if ((kv_armed >> s) & 1u) drain_wait(&sm.kv_full[s], (kv_par >> s) & 1u, p.wait_ns);
+        for (int b = 0; b < 4 * kSlots; ++b) {
+            if (!((kv_armed >> b) & 1u)) continue;
+            const int x = b >> 2, st = (b >> 1) & 1;
+            uint64_t *bar = (b & 1) ? &sm.v_full[x][st] : &sm.k_full[x][st];
+            drain_wait(bar, (kv_par >> b) & 1u, p.wait_ns);
+        }
         for (int q = 0; q < 2 * kSlots; ++q)
             if ((qa >> q) & 1u) drain_wait(&sm.q_full[q >> 1][q & 1], (qp >> q) & 1u, p.wait_ns);
-    }
-}
-
-// ------------------------------------------------------------ MMA issuer
-struct MmaSlot {
-    int k, t, j;    // items taken, tile of the current item, tiles issued
-    int stage;      // ring stage of the tile whose S was issued last
-    int kind, ntiles, nkv, g;   // of the current item (kind 0: no more items)
-};
-
-__device__ __forceinline__ int mma_tile_cols(const MmaSlot &S)
-{
-    if (S.kind != 1 || S.t < S.nkv) return kTileKeys;
-    const int left = min(kTileKeys, S.g - (S.t - S.nkv) * kTileKeys);
-    return (left + 15) & ~15;
-}
-
-__device__ __forceinline__ bool mma_next_item(const FwdParams &p, FwdSmem &sm, MmaSlot &S, int X)
-{
-    const int rs = S.k % kRing;
-    if (!warp_wait(p, sm, &sm.item_full[X][rs], uint32_t(S.k / kRing) & 1u)) return false;
-    const ItemInfo &I = sm.items[X][rs];
-    S.kind = I.kind;
-    S.ntiles = I.ntiles;
-    S.nkv = I.nkv;
-    S.g = I.g;
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.item_empty[X][rs]);
-    S.t = 0;
-    ++S.k;
-    return true;
-}
-
-// Issues S = Q K^T of the slot's current tile; returns false on abort.
-__device__ __forceinline__ bool mma_issue_s(const FwdParams &p, FwdSmem &sm, MmaSlot &S, int X,
-                                            uint32_t tmem, uint32_t id_s, int &stage,
-                                            uint32_t &phase)
-{
-    const int kq = S.k - 1;   // index of the current item
-    if (S.t == 0 &&
-        !warp_wait(p, sm, &sm.q_full[X][kq & 1], uint32_t(kq >> 1) & 1u))
-        return false;
-    if (!warp_wait(p, sm, &sm.kv_full[stage], phase)) return false;
-    tc_fence_after();
-    const int N = mma_tile_cols(S);
-    const uint32_t tS = tmem + X * kSlotCols;
-    const uint64_t qdesc = make_sdesc(smem_u32(sm.q[X][kq & 1]), 16, 1024);
-    const uint64_t kdesc = make_sdesc(smem_u32(sm.k[stage]), 16, 1024);
-    const uint32_t idesc = id_s | (uint32_t(N >> 3) << 17);
-#pragma unroll
-    for (int kk = 0; kk < kDHead / 16; ++kk)
-        mma_ss_elect(tS, qdesc + uint64_t((kk * 32) >> 4), kdesc + uint64_t((kk * 32) >> 4), idesc,
-                     kk > 0 ? 1u : 0u);
-    tc_commit_elect(&sm.s_full[X]);
-    if (S.t == S.ntiles - 1) tc_commit_elect(&sm.q_empty[X][kq & 1]);
-    __syncwarp();
-    S.stage = stage;
-    advance_ring(stage, phase);
-    return true;
-}
-
-__device__ __forceinline__ void mma_role(const FwdParams &p, FwdSmem &sm, uint32_t tmem, bool bf16)
-{
-    const uint32_t id_s = make_idesc(128, 0, bf16, false);
-    const uint32_t id_pv = make_idesc(128, 64, bf16, true);
-    MmaSlot A, B;
-    A.k = A.j = A.t = A.ntiles = 0;
-    A.kind = 1;              // "needs its first item"
-    B = A;
-    bool pv_pending_a = false, pv_pending_b = false;
-    int stage = 0;
-    uint32_t phase = 0;
-    int X = 0;
-#pragma unroll 1
-    for (;;) {
-        if (A.kind == 0 && B.kind == 0) break;
-        if (A.kind != 0) {
-            if (pv_pending_a) {
-                const int kq = A.k - 1;
-                const int ob = kq & 1;
-                if (!warp_wait(p, sm, &sm.p_full[X], uint32_t(A.j) & 1u)) return;
-                // The first PV of an item overwrites its O buffer: the epilogue
-                // of the item two before must have read it.
-                if (A.t == 0 && kq >= 2 &&
-                    !warp_wait(p, sm, &sm.o_empty[X][ob], uint32_t((kq >> 1) - 1) & 1u))
-                    return;
-                tc_fence_after();
-                const uint32_t tP = tmem + X * kSlotCols;
-                const uint32_t tO = tP + 128 + ob * 64;
-                const uint64_t vdesc = make_sdesc(smem_u32(sm.v[A.stage]), 16, 1024);
-                const int ksteps = mma_tile_cols(A) >> 4;
-                for (int kk = 0; kk < ksteps; ++kk)
-                    mma_ts_elect(tO, tP + kk * 8, vdesc + uint64_t((kk * 2048) >> 4), id_pv,
-                                 (kk > 0 || A.t > 0) ? 1u : 0u);
-                tc_commit_elect(&sm.kv_empty[A.stage]);
-                if (A.t == A.ntiles - 1) tc_commit_elect(&sm.o_full[X][ob]);
-                __syncwarp();
-                ++A.j;
-                ++A.t;
-                pv_pending_a = false;
-            }
-            if (A.t == A.ntiles && !mma_next_item(p, sm, A, X)) return;
-            if (A.kind != 0) {
-                if (!mma_issue_s(p, sm, A, X, tmem, id_s, stage, phase)) return;
-                pv_pending_a = true;
-            }
-        }
-        swap_state(A, B);
-        const bool tmp = pv_pending_a;
-        pv_pending_a = pv_pending_b;
-        pv_pending_b = tmp;
-        X ^= 1;
     }
 }
 
@@ -1005,7 +888,6 @@ __device__ __forceinline__ void epilogue(const FwdParams &p, FwdSmem &sm, uint32
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.o_empty[X][ob]);
     if (kind == 2 && active && p.merge_in_kernel) {
         // The last chunk to finish this warp's group of 32 global rows merges
         // them and resets the group's arrival counter for the next call on the
@@ -1069,23 +951,85 @@ __device__ __forceinline__ void tile_row_mask(const AttnArgs &a, const ItemInfo 
     }
 }
 
+// Products of a slot, issued by one elected thread of warp 0 of the slot's
+// softmax warpgroup (the issuing code runs every tile and stays in the
+// instruction caches).  QK^T of tile t of item k (the slot's jt-th tile).
+__device__ __forceinline__ bool issue_s(const FwdParams &p, FwdSmem &sm, uint32_t tS, int X,
+                                        const ItemInfo &I, int t, int k, int jt, bool bf16)
+{
+    const int stage = jt % kStages;
+    if (t == 0 && !warp_wait(p, sm, &sm.q_full[X][k & 1], uint32_t(k >> 1) & 1u)) return false;
+    if (!warp_wait(p, sm, &sm.k_full[X][stage], uint32_t(jt / kStages) & 1u)) return false;
+    tc_fence_after();
+    const int N = tile_cols(I, t);
+    const uint64_t qdesc = make_sdesc(smem_u32(sm.q[X][k & 1]), 16, 1024);
+    const uint64_t kdesc = make_sdesc(smem_u32(sm.k[X][stage]), 16, 1024);
+    const uint32_t idesc = make_idesc(128, 0, bf16, false) | (uint32_t(N >> 3) << 17);
+#pragma unroll
+    for (int kk = 0; kk < kDHead / 16; ++kk)
+        mma_ss_elect(tS, qdesc + uint64_t((kk * 32) >> 4), kdesc + uint64_t((kk * 32) >> 4), idesc,
+                     kk > 0 ? 1u : 0u);
+    tc_commit_elect(&sm.k_empty[X][stage]);
+    tc_commit_elect(&sm.s_full[X]);
+    if (t == I.ntiles - 1) tc_commit_elect(&sm.q_empty[X][k & 1]);
+    __syncwarp();
+    return true;
+}
+
+// O += P V of tile t of item k (the slot's jt-th tile).
+__device__ __forceinline__ bool issue_pv(const FwdParams &p, FwdSmem &sm, uint32_t tS, int X,
+                                         const ItemInfo &I, int t, int k, int jt, bool bf16)
+{
+    const int stage = jt % kStages;
+    if (!warp_wait(p, sm, &sm.v_full[X][stage], uint32_t(jt / kStages) & 1u)) return false;
+    tc_fence_after();
+    const uint32_t tO = tS + 128 + (k & 1) * 64;
+    const uint64_t vdesc = make_sdesc(smem_u32(sm.v[X][stage]), 16, 1024);
+    const uint32_t idesc = make_idesc(128, 64, bf16, true);
+    const int ksteps = tile_cols(I, t) >> 4;
+    for (int kk = 0; kk < ksteps; ++kk)
+        mma_ts_elect(tO, tS + kk * 8, vdesc + uint64_t((kk * 2048) >> 4), idesc,
+                     (kk > 0 || t > 0) ? 1u : 0u);
+    tc_commit_elect(&sm.v_empty[X][stage]);
+    if (t == I.ntiles - 1) tc_commit_elect(&sm.o_full[X][k & 1]);
+    __syncwarp();
+    return true;
+}
+
+// The softmax warpgroup of slot X.  Per tile: masks, wait for S, softmax,
+// P to TMEM; then warp 0 waits for the four warps' P and issues PV of this
+// tile and QK^T of the next one (the slot's products run in that order, so
+// once S of a tile is complete so is every product before it).  The epilogue
+// of an item runs after the first tile of the next one.
 template <typename T>
 __device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, uint32_t tmem, int X,
                                              int tid)
 {
     const AttnArgs &a = p.a;
     const int warp = tid >> 5, lane = tid & 31;
+    const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
     const uint32_t tmem_row = tmem + (uint32_t(warp * 32) << 16);
     const uint32_t tS = tmem_row + X * kSlotCols;
+    const uint32_t tS0 = tmem + X * kSlotCols;      // lane 0 of the slot: MMA operand base
     const float sl2 = a.scale_log2;
     int k = 0;      // items taken
     int jt = 0;     // tiles taken
     RowOut pend;
     bool pending = false;
+    bool ok = true;
 
-    for (;;) {
+    // The first QK^T of the slot.
+    if (warp == 0) {
+        if (!warp_wait(p, sm, &sm.item_full[X][0], 0u)) {
+            ok = false;
+        } else {
+            const ItemInfo I0 = sm.items[X][0];
+            if (I0.kind != 0) ok = issue_s(p, sm, tS0, X, I0, 0, 0, 0, bf16);
+        }
+    }
+    while (ok) {
         const int rs = k % kRing;
-        if (!warp_wait(p, sm, &sm.item_full[X][rs], uint32_t(k / kRing) & 1u)) return;
+        if (!warp_wait(p, sm, &sm.item_full[X][rs], uint32_t(k / kRing) & 1u)) break;
         const ItemInfo I = sm.items[X][rs];
         if (I.kind == 0) {
             __syncwarp();
@@ -1114,10 +1058,12 @@ __device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, ui
         for (int t = 0; t <= ntiles; ++t) {
             if (t == 1 || (t == 0 && ntiles == 0)) {
                 if (pending) {
-                    // The previous item's products are complete: every product
-                    // of this slot before this item's first S is.
+                    // Every product of the previous item is complete.
                     const int ke = k - 1;
-                    if (!warp_wait(p, sm, &sm.o_full[X][ke & 1], uint32_t(ke >> 1) & 1u)) return;
+                    if (!warp_wait(p, sm, &sm.o_full[X][ke & 1], uint32_t(ke >> 1) & 1u)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     epilogue<T>(p, sm, tmem_row, X, ke, pend, tid);
                     pending = false;
@@ -1125,23 +1071,51 @@ __device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, ui
             }
             if (t == ntiles) break;
             const int rt = jt % kRing;
-            if (!warp_wait(p, sm, &sm.tm_full[X][rt], uint32_t(jt / kRing) & 1u)) return;
+            if (!warp_wait(p, sm, &sm.tm_full[X][rt], uint32_t(jt / kRing) & 1u)) {
+                ok = false;
+                break;
+            }
             uint32_t mw[4];
             if (active) tile_row_mask(a, I, sm.tmask[X][rt], t, row, lane, mw);
-            if (!warp_wait(p, sm, &sm.s_full[X], uint32_t(jt) & 1u)) return;
+            if (!warp_wait(p, sm, &sm.s_full[X], uint32_t(jt) & 1u)) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
             if (active) softmax_tile<T>(tS, tO, st, t == 0, mw, sl2);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.p_full[X]);
+            if (warp == 0) {
+                // Every warp's P is in TMEM: PV of this tile, then the next S.
+                ok = warp_wait(p, sm, &sm.p_full[X], uint32_t(jt) & 1u) &&
+                     issue_pv(p, sm, tS0, X, I, t, k, jt, bf16);
+                if (ok && t + 1 < ntiles) {
+                    ok = issue_s(p, sm, tS0, X, I, t + 1, k, jt + 1, bf16);
+                } else if (ok) {
+                    const int kn = k + 1;
+                    ok = warp_wait(p, sm, &sm.item_full[X][kn % kRing], uint32_t(kn / kRing) & 1u);
+                    if (ok) {
+                        const ItemInfo In = sm.items[X][kn % kRing];
+                        if (In.kind != 0) ok = issue_s(p, sm, tS0, X, In, 0, kn, jt + 1, bf16);
+                    }
+                }
+                if (!ok) break;
+            }
             ++jt;
         }
-        if (I.kind == 0) break;
+        if (!ok || I.kind == 0) break;
         ro.m = st.m;
         ro.l = st.l;
         pend = ro;
         pending = true;
         ++k;
+    }
+    if (warp == 0) {
+        // Every product this warp issued has completed once this commit lands.
+        tc_commit_elect(&sm.drain[X]);
+        __syncwarp();
+        drain_wait(&sm.drain[X], 0, p.wait_ns);
     }
 }
 
@@ -1159,22 +1133,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             for (int b = 0; b < 2; ++b) {
                 mbar_init(&sm.q_full[X][b], 1);
                 mbar_init(&sm.q_empty[X][b], 1);
-                mbar_init(&sm.o_empty[X][b], 4);      // one arrival per softmax warp
                 mbar_init(&sm.o_full[X][b], 1);
+            }
+            for (int st = 0; st < kStages; ++st) {
+                mbar_init(&sm.k_full[X][st], 1);
+                mbar_init(&sm.k_empty[X][st], 1);
+                mbar_init(&sm.v_full[X][st], 1);
+                mbar_init(&sm.v_empty[X][st], 1);
             }
             for (int r = 0; r < kRing; ++r) {
                 mbar_init(&sm.item_full[X][r], 1);
-                mbar_init(&sm.item_empty[X][r], 5);   // four softmax warps + the MMA warp
+                mbar_init(&sm.item_empty[X][r], 4);   // one arrival per softmax warp
                 mbar_init(&sm.tm_full[X][r], 1);
             }
             mbar_init(&sm.s_full[X], 1);
             mbar_init(&sm.p_full[X], 4);
+            mbar_init(&sm.drain[X], 1);
         }
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sm.kv_full[s], 1);
-            mbar_init(&sm.kv_empty[s], 1);
-        }
-        mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
         mbar_fence_init();
     }
@@ -1186,7 +1161,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             tma_prefetch_map(&p.res_v[m]);
         }
     }
-    if (warp == kWarpMma) {
+    if (warp == kWarpTmem) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -1218,19 +1193,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         softmax_role<T>(p, sm, tmem, warp >> 2, threadIdx.x & 127);
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
-        if (warp == kWarpProducer) {
-            producer_role(p, sm, lane);
-        } else if (warp == kWarpMma) {
-            mma_role(p, sm, tmem, std::is_same<T, __nv_bfloat16>::value);
-            // Every MMA this warp issued has completed once this commit lands.
-            tc_commit_elect(&sm.drain);
-            __syncwarp();
-            drain_wait(&sm.drain, 0, p.wait_ns);
-        }
+        if (warp == kWarpProducer) producer_role(p, sm, lane);
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == kWarpMma) {
+    if (warp == kWarpTmem) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
