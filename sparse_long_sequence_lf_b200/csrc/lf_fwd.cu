@@ -70,18 +70,26 @@ namespace lf {
 using namespace sm100;
 
 constexpr int kRows = 128;                        // query rows per tile (M)
-constexpr int kTileKeys = 128;                    // keys per S tile (N) / K-V stage
-constexpr int kStages = 2;                        // K and V ring depth per slot
+constexpr int kTileKeys = 96;                     // keys per S tile (N) / K-V stage
+constexpr int kChunks = kTileKeys / 32;           // 32-key chunks of a tile (softmax loop)
+constexpr int kStages = 3;                        // K and V ring depth per slot
 constexpr int kSlots = 2;
-constexpr int kRing = 4;                          // item and tile-info rings per slot
+constexpr int kRing = 4;                          // item records per slot
+// Tile masks per slot: the producer writes the mask of tile j once the K
+// stage of tile j-3 is free, i.e. once QK^T of tile j-3, PV of tile j-5 and
+// the softmax of tile j-5 are done; the softmax may still read the mask of
+// tile j-4, so the ring must hold at least five.
+constexpr int kMaskRing = 8;
 constexpr int kQBytes = kRows * kDHead * 2;       // 16 KB of 16-bit elements
-constexpr int kKvBytes = kTileKeys * kDHead * 2;  // 16 KB
+constexpr int kKvBytes = kTileKeys * kDHead * 2;  // 12 KB
 constexpr int kRowBytes = kDHead * 2;             // 128 B
 constexpr int kThreads = 384;
-constexpr int kWarpProducer = 8;
-constexpr int kWarpTmem = 9;                      // allocates and frees the tensor memory
+constexpr int kWarpProducer = 8;                  // warps 8, 9: TMA producers of slots 0, 1
+constexpr int kWarpMma = 10;                      // warps 10, 11: MMA issuers of slots 0, 1
+constexpr int kWarpTmem = 10;                     // allocates and frees the tensor memory
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSlotCols = 256;               // S (128) | O0 (64) | O1 (64)
+constexpr uint32_t kSlotCols = 256;               // S0 (96) | S1 (96) | O (64)
+constexpr uint32_t kColO = 2 * kTileKeys;         // O within a slot's columns
 constexpr float kRescaleLog2 = 8.f;               // lazy rescale: P stays below 2^8
 // Register split: the two softmax warpgroups take registers from the control
 // warpgroup: 256 * 208 + 128 * 80 = 63488 registers, which the launch (384
@@ -108,8 +116,8 @@ constexpr int kBatchCache = 64;                   // per-batch counts / flags ke
 struct FwdParams {
     CUtensorMap maps[kMapCount];              // first: 64-byte aligned
     CUtensorMap res_q[kMaxResidues];          // Q tiles of 128 rows
-    CUtensorMap res_k[kMaxResidues];          // K tiles of 128 rows
-    CUtensorMap res_v[kMaxResidues];          // V tiles of 128 rows
+    CUtensorMap res_k[kMaxResidues];          // K tiles of kTileKeys rows
+    CUtensorMap res_v[kMaxResidues];          // V tiles of kTileKeys rows
     AttnArgs a;
     int res_base[kMaxHeads];  // residue map of (head h, residue 0); -1: load rows one by one
     int band_items;       // B * band_items_per_batch, numbered first
@@ -154,14 +162,17 @@ struct __align__(1024) FwdSmem {
     uint8_t q[kSlots][2][kQBytes];
     uint8_t k[kSlots][kStages][kKvBytes];
     uint8_t v[kSlots][kStages][kKvBytes];
-    TileMask tmask[kSlots][kRing];
+    TileMask tmask[kSlots][kMaskRing];
     ItemInfo items[kSlots][kRing];
     uint64_t q_full[kSlots][2], q_empty[kSlots][2];
     uint64_t k_full[kSlots][kStages], k_empty[kSlots][kStages];
     uint64_t v_full[kSlots][kStages], v_empty[kSlots][kStages];
     uint64_t item_full[kSlots][kRing], item_empty[kSlots][kRing];
-    uint64_t tm_full[kSlots][kRing];
-    uint64_t s_full[kSlots], p_full[kSlots], o_full[kSlots][2];
+    uint64_t tm_full[kSlots][kMaskRing];
+    // S / P buffer b of slot X: S(j) complete, P(j) stored, for the tiles j
+    // with j % 2 == b (the softmax can store P(j+1) before PV(j) is issued).
+    uint64_t s_full[kSlots][2], p_full[kSlots][2];
+    uint64_t pv_done[kSlots], o_full[kSlots], o_free[kSlots];
     uint64_t drain[kSlots];
     int batch_count[kBatchCache];
     int batch_flags[kBatchCache];
@@ -412,8 +423,8 @@ __device__ __forceinline__ bool producer_q(const FwdParams &p, FwdSmem &sm, Prod
                 tma_load_2d(qd + rr * kRowBytes, &p.maps[kMapQgRow], qbar, 0, y);
             }
         }
-        // Bit 2X + qb: a Q copy of that buffer was started; its parity.
-        const uint32_t bit = 1u << (2 * X + qb);
+        // Bit qb: a Q copy of that buffer was started; its parity.
+        const uint32_t bit = 1u << qb;
         q_armed |= bit;
         q_par = (use & 1u) ? (q_par | bit) : (q_par & ~bit);
     }
@@ -427,7 +438,7 @@ __device__ __forceinline__ bool producer_q(const FwdParams &p, FwdSmem &sm, Prod
 // its V tile into V stage jt % kStages, each once the stage has been released
 // (the K stage by the tile's QK^T two tiles back, the V stage by its PV).
 // Returns false on abort; `armed` and `par` record the copies started (bit
-// 4X + 2*stage + {0: K, 1: V}) for the drain.
+// 2*stage + {0: K, 1: V}) for the drain.
 __device__ __forceinline__ bool producer_tile(const FwdParams &p, FwdSmem &sm, ProducerSlot &S,
                                               int X, int lane, uint32_t &armed, uint32_t &par)
 {
@@ -440,7 +451,7 @@ __device__ __forceinline__ bool producer_tile(const FwdParams &p, FwdSmem &sm, P
     uint8_t *vd = sm.v[X][stage];
     uint64_t *kbar = &sm.k_full[X][stage];
     uint64_t *vbar = &sm.v_full[X][stage];
-    TileMask &tm = sm.tmask[X][S.jt % kRing];
+    TileMask &tm = sm.tmask[X][S.jt % kMaskRing];
     const uint32_t *vb = a.ws.vbits + size_t(I.b) * a.L.nwords;
     const int kind = I.kind == 2 ? 2 : (t < I.nkv ? 1 : 3);   // 3: global-token columns
     const int k0 = I.klo + t * kTileKeys;
@@ -450,7 +461,7 @@ __device__ __forceinline__ bool producer_tile(const FwdParams &p, FwdSmem &sm, P
     // Column masks.
     if (kind == 2 || (kind == 1 && I.has_pad)) {
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
+        for (int w = 0; w < kChunks; ++w) {
             const int j = k0 + 32 * w + lane;
             const bool ok = kind == 2 ? (j < I.key_end && (!I.has_pad || bit_at(vb, j)))
                                       : (j < I.n_r && bit_at(vb, j * I.dil + I.r));
@@ -458,10 +469,10 @@ __device__ __forceinline__ bool producer_tile(const FwdParams &p, FwdSmem &sm, P
             if (lane == 0) tm.bits[w] = bits;
         }
     } else if (kind == 1) {
-        if (lane < 4) tm.bits[lane] = 0xffffffffu;
+        if (lane < kChunks) tm.bits[lane] = 0xffffffffu;
     } else {
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
+        for (int w = 0; w < kChunks; ++w) {
             const int c = 32 * w + lane;
             const int slot = s0 + c;
             const int j = slot < I.g ? a.ws.gidx[size_t(I.b) * a.n + slot] : -1;
@@ -499,8 +510,8 @@ __device__ __forceinline__ bool producer_tile(const FwdParams &p, FwdSmem &sm, P
         __syncwarp();
     };
     load(false, kd, kbar);
-    if (lane == 0) mbar_arrive(&sm.tm_full[X][S.jt % kRing]);
-    const uint32_t kb = 1u << (4 * X + 2 * stage);
+    if (lane == 0) mbar_arrive(&sm.tm_full[X][S.jt % kMaskRing]);
+    const uint32_t kb = 1u << (2 * stage);
     armed |= kb;
     par = phase ? (par | kb) : (par & ~kb);
     if (!warp_wait(p, sm, &sm.v_empty[X][stage], phase ^ 1u)) return false;
@@ -510,31 +521,18 @@ __device__ __forceinline__ bool producer_tile(const FwdParams &p, FwdSmem &sm, P
     return true;
 }
 
-template <typename S> __device__ __forceinline__ void swap_state(S &a, S &b)
-{
-    const S t = a;
-    a = b;
-    b = t;
-}
-
-// The producer and the MMA issuer serve the two slots in turn, skipping a
-// slot that has no more work: slot X, then slot X^1, ...  Both loops keep the
-// state of the slot they serve in `A` and of the other one in `B` and swap
-// them every turn, so that the code of a turn exists once (the roles' code is
-// small enough to stay in the instruction caches next to the softmax's).
-__device__ __forceinline__ void producer_role(const FwdParams &p, FwdSmem &sm, int lane)
+// The producer of slot X: item records two ahead, Q tiles as soon as a Q
+// buffer frees, the K and V tiles of the current item.
+__device__ __forceinline__ void producer_role(const FwdParams &p, FwdSmem &sm, int X, int lane)
 {
     int *sched = p.a.ws.status + 16;
-    ProducerSlot A, B;
+    ProducerSlot A;
     uint32_t kv_armed = 0, kv_par = 0;   // K/V copies started (see producer_tile); parities
-    uint32_t qa = 0, qp = 0;             // bit 2X+b: Q buffer b of slot X was filled
+    uint32_t qa = 0, qp = 0;             // bit b: Q buffer b was filled; parity
     bool ok = true;
     A.kc = A.t = A.kw = A.kq = A.jt = 0;
     A.ended = false;
-    B = A;
     A.claimed = claim_item(sched, lane);
-    B.claimed = claim_item(sched, lane);
-    int X = 0;
 #pragma unroll 1
     for (;;) {
         // Keep two records ahead of the current item.
@@ -543,34 +541,126 @@ __device__ __forceinline__ void producer_role(const FwdParams &p, FwdSmem &sm, i
         // current item's, else only if its buffer is already free.
         if (ok) ok = producer_q(p, sm, A, X, lane, A.kq == A.kc, qa, qp);
         if (!ok) break;
-        const bool busy_a = A.kc < A.kw && sm.items[X][A.kc % kRing].kind != 0;
-        if (busy_a) {
-            if (!producer_tile(p, sm, A, X, lane, kv_armed, kv_par)) {
-                ok = false;
-                break;
-            }
-            ++A.jt;
-            if (++A.t == sm.items[X][A.kc % kRing].ntiles) {
-                ++A.kc;
-                A.t = 0;
-            }
-        } else if (B.ended && B.kc == B.kw - 1) {
-            // Both slots are at their end records (this one is: a slot that is
-            // not at its end always has a record of a real item to load).
+        // A slot that is not at its end always has the record of a real item.
+        if (sm.items[X][A.kc % kRing].kind == 0) break;
+        if (!producer_tile(p, sm, A, X, lane, kv_armed, kv_par)) {
+            ok = false;
             break;
         }
-        swap_state(A, B);
-        X ^= 1;
+        ++A.jt;
+        if (++A.t == sm.items[X][A.kc % kRing].ntiles) {
+            ++A.kc;
+            A.t = 0;
+        }
     }
     if (!ok || sm.abort_flag) {
-        for (int b = 0; b < 4 * kSlots; ++b) {
+        for (int b = 0; b < 2 * kStages; ++b) {
             if (!((kv_armed >> b) & 1u)) continue;
-            const int x = b >> 2, st = (b >> 1) & 1;
-            uint64_t *bar = (b & 1) ? &sm.v_full[x][st] : &sm.k_full[x][st];
+            uint64_t *bar = (b & 1) ? &sm.v_full[X][b >> 1] : &sm.k_full[X][b >> 1];
             drain_wait(bar, (kv_par >> b) & 1u, p.wait_ns);
         }
-        for (int q = 0; q < 2 * kSlots; ++q)
-            if ((qa >> q) & 1u) drain_wait(&sm.q_full[q >> 1][q & 1], (qp >> q) & 1u, p.wait_ns);
+        for (int b = 0; b < 2; ++b)
+            if ((qa >> b) & 1u) drain_wait(&sm.q_full[X][b], (qp >> b) & 1u, p.wait_ns);
+    }
+}
+
+// ------------------------------------------------------------ MMA issuer
+// The MMA issuer of slot X (one elected thread).  S is double-buffered: QK^T
+// of tile j+2 goes to the buffer of tile j right after PV of tile j (which
+// reads P(j) there), so while the softmax works on tile j+1 the tensor core
+// has already computed its scores.  Per slot the products run in issue order.
+struct MmaCursor {
+    int k;          // item
+    int t;          // tile within the item
+    int j;          // tile within the slot
+    int kind, ntiles;
+};
+
+// Moves a cursor to its next tile; reads the next item's record from the
+// ring when the item ends.  Returns false on abort.
+__device__ __forceinline__ bool mma_advance(const FwdParams &p, FwdSmem &sm, MmaCursor &c, int X)
+{
+    ++c.j;
+    if (++c.t < c.ntiles) return true;
+    ++c.k;
+    c.t = 0;
+    const int rs = c.k % kRing;
+    if (!warp_wait(p, sm, &sm.item_full[X][rs], uint32_t(c.k / kRing) & 1u)) return false;
+    c.kind = sm.items[X][rs].kind;
+    c.ntiles = sm.items[X][rs].ntiles;
+    return true;
+}
+
+__device__ __forceinline__ bool mma_issue_s(const FwdParams &p, FwdSmem &sm, uint32_t tS0, int X,
+                                            const MmaCursor &c, bool bf16)
+{
+    const ItemInfo &I = sm.items[X][c.k % kRing];
+    const int stage = c.j % kStages;
+    if (c.t == 0 && !warp_wait(p, sm, &sm.q_full[X][c.k & 1], uint32_t(c.k >> 1) & 1u)) return false;
+    if (!warp_wait(p, sm, &sm.k_full[X][stage], uint32_t(c.j / kStages) & 1u)) return false;
+    tc_fence_after();
+    const int N = tile_cols(I, c.t);
+    const uint64_t qdesc = make_sdesc(smem_u32(sm.q[X][c.k & 1]), 16, 1024);
+    const uint64_t kdesc = make_sdesc(smem_u32(sm.k[X][stage]), 16, 1024);
+    const uint32_t idesc = make_idesc(128, 0, bf16, false) | (uint32_t(N >> 3) << 17);
+    const uint32_t tS = tS0 + (c.j & 1) * kTileKeys;
+#pragma unroll
+    for (int kk = 0; kk < kDHead / 16; ++kk)
+        mma_ss_elect(tS, qdesc + uint64_t((kk * 32) >> 4), kdesc + uint64_t((kk * 32) >> 4), idesc,
+                     kk > 0 ? 1u : 0u);
+    tc_commit_elect(&sm.k_empty[X][stage]);
+    tc_commit_elect(&sm.s_full[X][c.j & 1]);
+    if (c.t == c.ntiles - 1) tc_commit_elect(&sm.q_empty[X][c.k & 1]);
+    __syncwarp();
+    return true;
+}
+
+__device__ __forceinline__ void mma_role(const FwdParams &p, FwdSmem &sm, uint32_t tmem, int X,
+                                         bool bf16)
+{
+    const uint32_t tS0 = tmem + X * kSlotCols;
+    const uint32_t tO = tS0 + kColO;
+    const uint32_t id_pv = make_idesc(128, 64, bf16, true);
+    // cs: the next QK^T to issue; cp: the next PV.
+    MmaCursor cs, cp;
+    cs.k = cs.t = cs.j = 0;
+    if (!warp_wait(p, sm, &sm.item_full[X][0], 0u)) return;
+    cs.kind = sm.items[X][0].kind;
+    cs.ntiles = sm.items[X][0].ntiles;
+    cp = cs;
+    // The first two QK^T of the slot.
+    for (int i = 0; i < 2 && cs.kind != 0; ++i) {
+        if (!mma_issue_s(p, sm, tS0, X, cs, bf16) || !mma_advance(p, sm, cs, X)) return;
+    }
+#pragma unroll 1
+    while (cp.kind != 0) {
+        const ItemInfo &I = sm.items[X][cp.k % kRing];
+        const int stage = cp.j % kStages;
+        if (!warp_wait(p, sm, &sm.p_full[X][cp.j & 1], uint32_t(cp.j >> 1) & 1u)) return;
+        // The first PV of an item overwrites O: the epilogue of the item
+        // before must have read it.
+        if (cp.t == 0 && cp.k > 0 &&
+            !warp_wait(p, sm, &sm.o_free[X], uint32_t(cp.k - 1) & 1u))
+            return;
+        if (!warp_wait(p, sm, &sm.v_full[X][stage], uint32_t(cp.j / kStages) & 1u)) return;
+        tc_fence_after();
+        const uint64_t vdesc = make_sdesc(smem_u32(sm.v[X][stage]), 16, 1024);
+        const uint32_t tP = tS0 + (cp.j & 1) * kTileKeys;
+        const int ksteps = tile_cols(I, cp.t) >> 4;
+        for (int kk = 0; kk < ksteps; ++kk)
+            mma_ts_elect(tO, tP + kk * 8, vdesc + uint64_t((kk * 2048) >> 4), id_pv,
+                         (kk > 0 || cp.t > 0) ? 1u : 0u);
+        tc_commit_elect(&sm.v_empty[X][stage]);
+        tc_commit_elect(&sm.pv_done[X]);
+        const bool last = cp.t == cp.ntiles - 1;
+        if (last) tc_commit_elect(&sm.o_full[X]);
+        __syncwarp();
+        if (last && (threadIdx.x & 31) == 0) mbar_arrive(&sm.item_empty[X][cp.k % kRing]);
+        if (!mma_advance(p, sm, cp, X)) return;
+        // QK^T two tiles ahead, into the buffer P(j) has just been read from.
+        if (cs.kind != 0) {
+            if (!mma_issue_s(p, sm, tS0, X, cs, bf16) || !mma_advance(p, sm, cs, X)) return;
+        }
     }
 }
 
@@ -677,12 +767,14 @@ template <> __device__ __forceinline__ void unpack2<__half>(uint32_t w, float &l
 // at the end of the tile, O (every PV before this tile has completed) are
 // scaled by the same factor.
 template <typename T>
-__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, RowState &st, bool first,
-                                             const uint32_t (&mw)[4], float sl2)
+__device__ __forceinline__ bool softmax_tile(const FwdParams &p, FwdSmem &sm, uint32_t tS,
+                                             uint32_t tO, RowState &st, bool first,
+                                             const uint32_t (&mw)[4], float sl2, uint64_t *pv_bar,
+                                             uint32_t pv_parity)
 {
     uint32_t any_m = 0, full_m = 0;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < kChunks; ++c) {
         any_m |= (__any_sync(0xffffffffu, mw[c] != 0u) ? 1u : 0u) << c;
         full_m |= (__all_sync(0xffffffffu, mw[c] == 0xffffffffu) ? 1u : 0u) << c;
     }
@@ -693,7 +785,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, RowState 
     float m = st.m, l = st.l;
     float alpha_o = 1.f;        // factor O must take for this tile's new maxima
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < kChunks; ++c) {
         uint32_t pk[16];
         if ((any_m >> c) & 1u) {
             float s[32];
@@ -753,6 +845,9 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, RowState 
         tmem_st16(tS + 16 * c, pk);
     }
     if (!first && __any_sync(0xffffffffu, alpha_o != 1.f)) {
+        // O must hold every PV before this tile (the previous one may run).
+        if (!warp_wait(p, sm, pv_bar, pv_parity)) return false;
+        tc_fence_after();
         for (int half = 0; half < 2; ++half) {
             float o[32];
             tmem_ld32(tO + half * 32, o);
@@ -765,6 +860,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, RowState 
     st.m = m;
     st.l = l;
     tmem_st_wait();
+    return true;
 }
 
 template <typename T>
@@ -850,8 +946,7 @@ __device__ __forceinline__ void epilogue(const FwdParams &p, FwdSmem &sm, uint32
     const int warp = tid >> 5, lane = tid & 31;
     const ItemInfo &I = sm.items[X][ke % kRing];
     const int kind = I.kind, bh = I.bh, q0 = I.q0;
-    const int ob = ke & 1;
-    const uint32_t tO = tmem_row + X * kSlotCols + 128 + ob * 64;
+    const uint32_t tO = tmem_row + X * kSlotCols + kColO;
     const int row = q0 + tid;
     const bool active = kind == 2 ? q0 + warp * 32 < I.g : q0 + warp * 32 < I.n_r;
     if (active) {
@@ -888,6 +983,7 @@ __device__ __forceinline__ void epilogue(const FwdParams &p, FwdSmem &sm, uint32
     }
     tc_fence_before();
     __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.o_free[X]);
     if (kind == 2 && active && p.merge_in_kernel) {
         // The last chunk to finish this warp's group of 32 global rows merges
         // them and resets the group's arrival counter for the next call on the
@@ -918,13 +1014,13 @@ __device__ __forceinline__ void tile_row_mask(const AttnArgs &a, const ItemInfo 
 {
     if (I.kind == 2) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) mw[c] = tm.bits[c];
+        for (int c = 0; c < 4; ++c) mw[c] = c < kChunks ? tm.bits[c] : 0u;
     } else if (t < I.nkv) {
         const int k0 = I.klo + t * kTileKeys;
         const int lo = max(row - (a.causal ? a.window - 1 : a.half), 0);
         const int hi = min(row + (a.causal ? 0 : a.half), I.n_r - 1);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) mw[c] = range_bits(c, lo - k0, hi - k0) & tm.bits[c];
+        for (int c = 0; c < 4; ++c) mw[c] = c < kChunks ? range_bits(c, lo - k0, hi - k0) & tm.bits[c] : 0u;
     } else {
         // Global-token columns: real, unpadded tokens that are not already
         // window taps of this row.  A tap shares the row's residue class and
@@ -936,6 +1032,10 @@ __device__ __forceinline__ void tile_row_mask(const AttnArgs &a, const ItemInfo 
         const int i_hi = __shfl_sync(0xffffffffu, i, 31) + span;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
+            if (c >= kChunks) {
+                mw[c] = 0u;
+                continue;
+            }
             uint32_t m = tm.bits[c];
             const int jl = tm.jpos[32 * c + lane];
             const bool near = jl >= i_lo && jl <= i_hi && (jl % I.dil) == I.r;
@@ -951,66 +1051,18 @@ __device__ __forceinline__ void tile_row_mask(const AttnArgs &a, const ItemInfo 
     }
 }
 
-// Products of a slot, issued by one elected thread of warp 0 of the slot's
-// softmax warpgroup (the issuing code runs every tile and stays in the
-// instruction caches).  QK^T of tile t of item k (the slot's jt-th tile).
-__device__ __forceinline__ bool issue_s(const FwdParams &p, FwdSmem &sm, uint32_t tS, int X,
-                                        const ItemInfo &I, int t, int k, int jt, bool bf16)
-{
-    const int stage = jt % kStages;
-    if (t == 0 && !warp_wait(p, sm, &sm.q_full[X][k & 1], uint32_t(k >> 1) & 1u)) return false;
-    if (!warp_wait(p, sm, &sm.k_full[X][stage], uint32_t(jt / kStages) & 1u)) return false;
-    tc_fence_after();
-    const int N = tile_cols(I, t);
-    const uint64_t qdesc = make_sdesc(smem_u32(sm.q[X][k & 1]), 16, 1024);
-    const uint64_t kdesc = make_sdesc(smem_u32(sm.k[X][stage]), 16, 1024);
-    const uint32_t idesc = make_idesc(128, 0, bf16, false) | (uint32_t(N >> 3) << 17);
-#pragma unroll
-    for (int kk = 0; kk < kDHead / 16; ++kk)
-        mma_ss_elect(tS, qdesc + uint64_t((kk * 32) >> 4), kdesc + uint64_t((kk * 32) >> 4), idesc,
-                     kk > 0 ? 1u : 0u);
-    tc_commit_elect(&sm.k_empty[X][stage]);
-    tc_commit_elect(&sm.s_full[X]);
-    if (t == I.ntiles - 1) tc_commit_elect(&sm.q_empty[X][k & 1]);
-    __syncwarp();
-    return true;
-}
-
-// O += P V of tile t of item k (the slot's jt-th tile).
-__device__ __forceinline__ bool issue_pv(const FwdParams &p, FwdSmem &sm, uint32_t tS, int X,
-                                         const ItemInfo &I, int t, int k, int jt, bool bf16)
-{
-    const int stage = jt % kStages;
-    if (!warp_wait(p, sm, &sm.v_full[X][stage], uint32_t(jt / kStages) & 1u)) return false;
-    tc_fence_after();
-    const uint32_t tO = tS + 128 + (k & 1) * 64;
-    const uint64_t vdesc = make_sdesc(smem_u32(sm.v[X][stage]), 16, 1024);
-    const uint32_t idesc = make_idesc(128, 64, bf16, true);
-    const int ksteps = tile_cols(I, t) >> 4;
-    for (int kk = 0; kk < ksteps; ++kk)
-        mma_ts_elect(tO, tS + kk * 8, vdesc + uint64_t((kk * 2048) >> 4), idesc,
-                     (kk > 0 || t > 0) ? 1u : 0u);
-    tc_commit_elect(&sm.v_empty[X][stage]);
-    if (t == I.ntiles - 1) tc_commit_elect(&sm.o_full[X][k & 1]);
-    __syncwarp();
-    return true;
-}
-
 // The softmax warpgroup of slot X.  Per tile: masks, wait for S, softmax,
-// P to TMEM; then warp 0 waits for the four warps' P and issues PV of this
-// tile and QK^T of the next one (the slot's products run in that order, so
-// once S of a tile is complete so is every product before it).  The epilogue
-// of an item runs after the first tile of the next one.
+// P to TMEM, arrive.  The epilogue of an item runs after the first tile of
+// the next one (the issuer waits for it before that item's first PV).
 template <typename T>
 __device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, uint32_t tmem, int X,
                                              int tid)
 {
     const AttnArgs &a = p.a;
     const int warp = tid >> 5, lane = tid & 31;
-    const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
     const uint32_t tmem_row = tmem + (uint32_t(warp * 32) << 16);
-    const uint32_t tS = tmem_row + X * kSlotCols;
-    const uint32_t tS0 = tmem + X * kSlotCols;      // lane 0 of the slot: MMA operand base
+    const uint32_t tSlot = tmem_row + X * kSlotCols;
+    const uint32_t tO = tSlot + kColO;
     const float sl2 = a.scale_log2;
     int k = 0;      // items taken
     int jt = 0;     // tiles taken
@@ -1018,15 +1070,6 @@ __device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, ui
     bool pending = false;
     bool ok = true;
 
-    // The first QK^T of the slot.
-    if (warp == 0) {
-        if (!warp_wait(p, sm, &sm.item_full[X][0], 0u)) {
-            ok = false;
-        } else {
-            const ItemInfo I0 = sm.items[X][0];
-            if (I0.kind != 0) ok = issue_s(p, sm, tS0, X, I0, 0, 0, 0, bf16);
-        }
-    }
     while (ok) {
         const int rs = k % kRing;
         if (!warp_wait(p, sm, &sm.item_full[X][rs], uint32_t(k / kRing) & 1u)) break;
@@ -1036,7 +1079,6 @@ __device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, ui
             if (lane == 0) mbar_arrive(&sm.item_empty[X][rs]);
             if (!pending) break;
         }
-        const uint32_t tO = tS + 128 + (k & 1) * 64;
         const int row = I.q0 + tid;
         const int wrow0 = I.q0 + warp * 32;
         const bool active = I.kind == 2 ? wrow0 < I.g : wrow0 < I.n_r;
@@ -1060,7 +1102,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, ui
                 if (pending) {
                     // Every product of the previous item is complete.
                     const int ke = k - 1;
-                    if (!warp_wait(p, sm, &sm.o_full[X][ke & 1], uint32_t(ke >> 1) & 1u)) {
+                    if (!warp_wait(p, sm, &sm.o_full[X], uint32_t(ke) & 1u)) {
                         ok = false;
                         break;
                     }
@@ -1070,38 +1112,26 @@ __device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, ui
                 }
             }
             if (t == ntiles) break;
-            const int rt = jt % kRing;
-            if (!warp_wait(p, sm, &sm.tm_full[X][rt], uint32_t(jt / kRing) & 1u)) {
+            const int rt = jt % kMaskRing;
+            if (!warp_wait(p, sm, &sm.tm_full[X][rt], uint32_t(jt / kMaskRing) & 1u)) {
                 ok = false;
                 break;
             }
             uint32_t mw[4];
             if (active) tile_row_mask(a, I, sm.tmask[X][rt], t, row, lane, mw);
-            if (!warp_wait(p, sm, &sm.s_full[X], uint32_t(jt) & 1u)) {
+            if (!warp_wait(p, sm, &sm.s_full[X][jt & 1], uint32_t(jt >> 1) & 1u)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            if (active) softmax_tile<T>(tS, tO, st, t == 0, mw, sl2);
+            if (active && !softmax_tile<T>(p, sm, tSlot + (jt & 1) * kTileKeys, tO, st, t == 0, mw,
+                                           sl2, &sm.pv_done[X], uint32_t(jt - 1) & 1u)) {
+                ok = false;
+                break;
+            }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.p_full[X]);
-            if (warp == 0) {
-                // Every warp's P is in TMEM: PV of this tile, then the next S.
-                ok = warp_wait(p, sm, &sm.p_full[X], uint32_t(jt) & 1u) &&
-                     issue_pv(p, sm, tS0, X, I, t, k, jt, bf16);
-                if (ok && t + 1 < ntiles) {
-                    ok = issue_s(p, sm, tS0, X, I, t + 1, k, jt + 1, bf16);
-                } else if (ok) {
-                    const int kn = k + 1;
-                    ok = warp_wait(p, sm, &sm.item_full[X][kn % kRing], uint32_t(kn / kRing) & 1u);
-                    if (ok) {
-                        const ItemInfo In = sm.items[X][kn % kRing];
-                        if (In.kind != 0) ok = issue_s(p, sm, tS0, X, In, 0, kn, jt + 1, bf16);
-                    }
-                }
-                if (!ok) break;
-            }
+            if (lane == 0) mbar_arrive(&sm.p_full[X][jt & 1]);
             ++jt;
         }
         if (!ok || I.kind == 0) break;
@@ -1110,12 +1140,6 @@ __device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, ui
         pend = ro;
         pending = true;
         ++k;
-    }
-    if (warp == 0) {
-        // Every product this warp issued has completed once this commit lands.
-        tc_commit_elect(&sm.drain[X]);
-        __syncwarp();
-        drain_wait(&sm.drain[X], 0, p.wait_ns);
     }
 }
 
@@ -1133,7 +1157,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             for (int b = 0; b < 2; ++b) {
                 mbar_init(&sm.q_full[X][b], 1);
                 mbar_init(&sm.q_empty[X][b], 1);
-                mbar_init(&sm.o_full[X][b], 1);
+                mbar_init(&sm.s_full[X][b], 1);
+                mbar_init(&sm.p_full[X][b], 4);           // one arrival per softmax warp
             }
             for (int st = 0; st < kStages; ++st) {
                 mbar_init(&sm.k_full[X][st], 1);
@@ -1143,11 +1168,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             }
             for (int r = 0; r < kRing; ++r) {
                 mbar_init(&sm.item_full[X][r], 1);
-                mbar_init(&sm.item_empty[X][r], 4);   // one arrival per softmax warp
-                mbar_init(&sm.tm_full[X][r], 1);
+                mbar_init(&sm.item_empty[X][r], 5);   // four softmax warps + the MMA warp
             }
-            mbar_init(&sm.s_full[X], 1);
-            mbar_init(&sm.p_full[X], 4);
+            for (int r = 0; r < kMaskRing; ++r) mbar_init(&sm.tm_full[X][r], 1);
+            mbar_init(&sm.pv_done[X], 1);
+            mbar_init(&sm.o_full[X], 1);
+            mbar_init(&sm.o_free[X], 4);
             mbar_init(&sm.drain[X], 1);
         }
         sm.abort_flag = 0;
@@ -1193,7 +1219,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         softmax_role<T>(p, sm, tmem, warp >> 2, threadIdx.x & 127);
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
-        if (warp == kWarpProducer) producer_role(p, sm, lane);
+        if (warp < kWarpMma) {
+            producer_role(p, sm, warp - kWarpProducer, lane);
+        } else {
+            const int X = warp - kWarpMma;
+            mma_role(p, sm, tmem, X, std::is_same<T, __nv_bfloat16>::value);
+            // Every MMA this warp issued has completed once this commit lands.
+            tc_commit_elect(&sm.drain[X]);
+            __syncwarp();
+            drain_wait(&sm.drain[X], 0, p.wait_ns);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -1281,10 +1316,10 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder()
     return fn;
 }
 
-// Whole tiles of 128 rows of the residue class r of dilation dil of each
-// (batch*head) slice: rows r, r+dil, ... ; dims {64, ceil((n-r)/dil), B*H}.
+// Whole tiles of box_rows rows of the residue class r of dilation dil of
+// each (batch*head) slice: rows r, r+dil, ... ; dims {64, ceil((n-r)/dil), B*H}.
 bool encode_tile_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int n, int BH,
-                     int dil, int r)
+                     int box_rows, int dil, int r)
 {
     auto enc = get_encoder();
     if (!enc) return false;
@@ -1292,7 +1327,7 @@ bool encode_tile_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, i
     base = static_cast<const char *>(base) + size_t(r) * kRowBytes;
     cuuint64_t dims[3] = {cuuint64_t(kDHead), cuuint64_t(n_r), cuuint64_t(BH)};
     cuuint64_t strides[2] = {cuuint64_t(dil) * kRowBytes, cuuint64_t(n) * kRowBytes};
-    cuuint32_t box[3] = {kDHead, cuuint32_t(kRows), 1};
+    cuuint32_t box[3] = {kDHead, cuuint32_t(box_rows), 1};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1323,7 +1358,8 @@ struct MapCacheEntry {
 };
 
 // Encoded tensor maps, reused while the same buffer and shape come back.
-// kind: 0 = tiles of 128 rows, 1 = single rows.
+// kind: 0 = tiles of kRows rows (Q), 1 = single rows, 2 = tiles of kTileKeys
+// rows (K, V, Kg, Vg).
 bool cached_map(CUtensorMap *out, int kind, const void *base, CUtensorMapDataType dt, int n, int BH,
                 int dil = 1, int r = 0)
 {
@@ -1340,7 +1376,8 @@ bool cached_map(CUtensorMap *out, int kind, const void *base, CUtensorMapDataTyp
         }
     CUtensorMap m;
     const bool ok = kind == 1 ? encode_row_map(&m, base, dt, long(n) * BH)
-                              : encode_tile_map(&m, base, dt, n, BH, dil, r);
+                              : encode_tile_map(&m, base, dt, n, BH, kind == 0 ? kRows : kTileKeys,
+                                                dil, r);
     if (!ok) return false;
     MapCacheEntry &e = cache[next++ % kCache];
     e = MapCacheEntry{base, kind, int(dt), n, BH, dil, r, m, true};
@@ -1375,15 +1412,15 @@ int launch_typed(const AttnArgs &a, CUtensorMapDataType dt, cudaStream_t stream)
         const int base = p.n_res;
         for (int r = 0; r < nres && ok; ++r) {
             ok = ok && cached_map(&p.res_q[base + r], 0, a.q, dt, a.n, BH, dil, r);
-            ok = ok && cached_map(&p.res_k[base + r], 0, a.k, dt, a.n, BH, dil, r);
-            ok = ok && cached_map(&p.res_v[base + r], 0, a.v, dt, a.n, BH, dil, r);
+            ok = ok && cached_map(&p.res_k[base + r], 2, a.k, dt, a.n, BH, dil, r);
+            ok = ok && cached_map(&p.res_v[base + r], 2, a.v, dt, a.n, BH, dil, r);
         }
         p.n_res += nres;
         for (int h2 = h; h2 < a.H; ++h2)
             if (a.dil[h2] == dil) p.res_base[h2] = base;
     }
-    ok = ok && cached_map(&p.maps[kMapKgTile], 0, a.kg, dt, a.n, BH);
-    ok = ok && cached_map(&p.maps[kMapVgTile], 0, a.vg, dt, a.n, BH);
+    ok = ok && cached_map(&p.maps[kMapKgTile], 2, a.kg, dt, a.n, BH);
+    ok = ok && cached_map(&p.maps[kMapVgTile], 2, a.vg, dt, a.n, BH);
     ok = ok && cached_map(&p.maps[kMapQRow], 1, a.q, dt, a.n, BH);
     ok = ok && cached_map(&p.maps[kMapKRow], 1, a.k, dt, a.n, BH);
     ok = ok && cached_map(&p.maps[kMapVRow], 1, a.v, dt, a.n, BH);
