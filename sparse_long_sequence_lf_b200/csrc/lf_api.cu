@@ -12,7 +12,7 @@ namespace lf {
 int launch_prepare(const uint8_t *local_mask, const uint8_t *global_mask, int B, int n,
                    int max_global, int32_t *gidx, int32_t *counts, int *flags, uint32_t *vbits,
                    uint32_t *gbits, int *status, int *counters, int counters_per_batch,
-                   cudaStream_t stream);
+                   int fill_tail, cudaStream_t stream);
 int launch_f32(const AttnArgs &a, cudaStream_t stream);
 int launch_tc(lf_dtype dtype, const AttnArgs &a, cudaStream_t stream);
 int launch_projection(lf_dtype dtype, int B, int n, int H, const void *x, const void *w,
@@ -154,7 +154,7 @@ int lf_global_index(const uint8_t *global_mask, int B, int n, int32_t *global_id
     if (B < 1 || n < 1 || !global_mask || !global_idx || !counts) return LF_ERR_INVALID_ARG;
     if (int rc = device_ok()) return rc;
     return launch_prepare(nullptr, global_mask, B, n, n, global_idx, counts, nullptr, nullptr,
-                          nullptr, nullptr, nullptr, 0, static_cast<cudaStream_t>(stream));
+                          nullptr, nullptr, nullptr, 0, 1, static_cast<cudaStream_t>(stream));
 }
 
 size_t lf_workspace_size(int B, int H, int n, int d_head, int max_global)
@@ -174,7 +174,7 @@ int lf_attention_prepare(int B, int H, int n, int d_head, const uint8_t *local_m
     if (int rc = device_ok()) return rc;
     WsPtrs p = ws_ptrs(workspace, L);
     return launch_prepare(local_mask, global_mask, B, n, max_global, p.gidx, p.counts, p.flags,
-                          p.vbits, p.gbits, p.status, p.counters, H * (L.ngroups + 1),
+                          p.vbits, p.gbits, p.status, p.counters, H * (L.ngroups + 1), 0,
                           static_cast<cudaStream_t>(stream));
 }
 

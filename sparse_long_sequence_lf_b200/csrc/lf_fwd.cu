@@ -92,10 +92,10 @@ constexpr uint32_t kSlotCols = 256;               // S0 (96) | S1 (96) | O (64)
 constexpr uint32_t kColO = 2 * kTileKeys;         // O within a slot's columns
 constexpr float kRescaleLog2 = 8.f;               // lazy rescale: P stays below 2^8
 // Register split: the two softmax warpgroups take registers from the control
-// warpgroup: 256 * 208 + 128 * 80 = 63488 registers, which the launch (384
+// warpgroup: 256 * 208 + 128 * 88 = 64512 registers, which the launch (384
 // threads at the compiled count) must hold (checked on the host).
 constexpr int kRegsSoftmax = 208;
-constexpr int kRegsControl = 80;
+constexpr int kRegsControl = 88;
 constexpr int kRegsNeeded = 2 * 128 * kRegsSoftmax + 128 * kRegsControl;
 // Of every 8 column pairs of a score tile, the pairs whose bit is set here
 // take 2^x from a cubic on the FMA pipe, the others from the SFU; the two
@@ -339,10 +339,12 @@ struct ProducerSlot {
 };
 
 // Claims the next item index from the device-wide counter (lane 0 only; the
-// value is read when the record is written).
+// value is read when the record is written).  The first item of every slot
+// is fixed (slot X of CTA c takes item kSlots * c + X), so the counter hands
+// out the items after those and no atomic sits on the start of the kernel.
 __device__ __forceinline__ int claim_item(int *sched, int lane)
 {
-    return lane == 0 ? atomicAdd(sched, 1) : 0;
+    return lane == 0 ? atomicAdd(sched, 1) + int(gridDim.x) * kSlots : 0;
 }
 
 // Decodes the claimed index into the slot's next ring record and claims the
@@ -532,7 +534,7 @@ __device__ __forceinline__ void producer_role(const FwdParams &p, FwdSmem &sm, i
     bool ok = true;
     A.kc = A.t = A.kw = A.kq = A.jt = 0;
     A.ended = false;
-    A.claimed = claim_item(sched, lane);
+    A.claimed = int(blockIdx.x) * kSlots + X;
 #pragma unroll 1
     for (;;) {
         // Keep two records ahead of the current item.
@@ -565,16 +567,49 @@ __device__ __forceinline__ void producer_role(const FwdParams &p, FwdSmem &sm, i
 }
 
 // ------------------------------------------------------------ MMA issuer
-// The MMA issuer of slot X (one elected thread).  S is double-buffered: QK^T
-// of tile j+2 goes to the buffer of tile j right after PV of tile j (which
-// reads P(j) there), so while the softmax works on tile j+1 the tensor core
-// has already computed its scores.  Per slot the products run in issue order.
+// The MMA issuer of slot X is one thread (lane 0 of the slot's MMA warp): it
+// waits on the barriers itself and issues every tcgen05.mma and commit of the
+// slot, so no instruction of the loop is a warp vote or an election.  S is
+// double-buffered: QK^T of tile j+2 goes to the buffer of tile j right after
+// PV of tile j (which reads P(j) there), so while the softmax works on tile
+// j+1 the tensor core has already computed its scores.  Per slot the products
+// run in issue order.
 struct MmaCursor {
     int k;          // item
     int t;          // tile within the item
     int j;          // tile within the slot
     int kind, ntiles;
+    int nkv, g;     // key tiles before the global-column tiles; global tokens
 };
+
+// Bounded wait of a single thread.
+__device__ __forceinline__ bool thread_wait(const FwdParams &p, FwdSmem &sm, uint64_t *bar,
+                                            uint32_t parity)
+{
+    return mbar_try_wait(bar, parity) ||
+           wait_slow(bar, parity, &sm.abort_flag, p.a.ws.status, p.wait_ns);
+}
+
+// Keys of tile t of the cursor's item (see tile_cols).
+__device__ __forceinline__ int cursor_cols(const MmaCursor &c, int t)
+{
+    if (c.kind != 1 || t < c.nkv) return kTileKeys;
+    const int left = min(kTileKeys, c.g - (t - c.nkv) * kTileKeys);
+    return (left + 15) & ~15;
+}
+
+// Reads the fields of ring record k the issuer needs.  Returns false on abort.
+__device__ __forceinline__ bool mma_load_item(const FwdParams &p, FwdSmem &sm, MmaCursor &c, int X)
+{
+    const int rs = c.k % kRing;
+    if (!thread_wait(p, sm, &sm.item_full[X][rs], uint32_t(c.k / kRing) & 1u)) return false;
+    const ItemInfo &I = sm.items[X][rs];
+    c.kind = I.kind;
+    c.ntiles = I.ntiles;
+    c.nkv = I.nkv;
+    c.g = I.g;
+    return true;
+}
 
 // Moves a cursor to its next tile; reads the next item's record from the
 // ring when the item ends.  Returns false on abort.
@@ -584,34 +619,33 @@ __device__ __forceinline__ bool mma_advance(const FwdParams &p, FwdSmem &sm, Mma
     if (++c.t < c.ntiles) return true;
     ++c.k;
     c.t = 0;
-    const int rs = c.k % kRing;
-    if (!warp_wait(p, sm, &sm.item_full[X][rs], uint32_t(c.k / kRing) & 1u)) return false;
-    c.kind = sm.items[X][rs].kind;
-    c.ntiles = sm.items[X][rs].ntiles;
-    return true;
+    return mma_load_item(p, sm, c, X);
 }
 
 __device__ __forceinline__ bool mma_issue_s(const FwdParams &p, FwdSmem &sm, uint32_t tS0, int X,
-                                            const MmaCursor &c, bool bf16)
+                                            const MmaCursor &c, int &stage, uint32_t &phase,
+                                            bool bf16)
 {
-    const ItemInfo &I = sm.items[X][c.k % kRing];
-    const int stage = c.j % kStages;
-    if (c.t == 0 && !warp_wait(p, sm, &sm.q_full[X][c.k & 1], uint32_t(c.k >> 1) & 1u)) return false;
-    if (!warp_wait(p, sm, &sm.k_full[X][stage], uint32_t(c.j / kStages) & 1u)) return false;
+    if (c.t == 0 && !thread_wait(p, sm, &sm.q_full[X][c.k & 1], uint32_t(c.k >> 1) & 1u))
+        return false;
+    if (!thread_wait(p, sm, &sm.k_full[X][stage], phase)) return false;
     tc_fence_after();
-    const int N = tile_cols(I, c.t);
+    const int N = cursor_cols(c, c.t);
     const uint64_t qdesc = make_sdesc(smem_u32(sm.q[X][c.k & 1]), 16, 1024);
     const uint64_t kdesc = make_sdesc(smem_u32(sm.k[X][stage]), 16, 1024);
     const uint32_t idesc = make_idesc(128, 0, bf16, false) | (uint32_t(N >> 3) << 17);
     const uint32_t tS = tS0 + (c.j & 1) * kTileKeys;
 #pragma unroll
     for (int kk = 0; kk < kDHead / 16; ++kk)
-        mma_ss_elect(tS, qdesc + uint64_t((kk * 32) >> 4), kdesc + uint64_t((kk * 32) >> 4), idesc,
-                     kk > 0 ? 1u : 0u);
-    tc_commit_elect(&sm.k_empty[X][stage]);
-    tc_commit_elect(&sm.s_full[X][c.j & 1]);
-    if (c.t == c.ntiles - 1) tc_commit_elect(&sm.q_empty[X][c.k & 1]);
-    __syncwarp();
+        mma_ss(tS, qdesc + uint64_t((kk * 32) >> 4), kdesc + uint64_t((kk * 32) >> 4), idesc,
+               kk > 0 ? 1u : 0u);
+    tc_commit(&sm.k_empty[X][stage]);
+    tc_commit(&sm.s_full[X][c.j & 1]);
+    if (c.t == c.ntiles - 1) tc_commit(&sm.q_empty[X][c.k & 1]);
+    if (++stage == kStages) {
+        stage = 0;
+        phase ^= 1u;
+    }
     return true;
 }
 
@@ -621,45 +655,49 @@ __device__ __forceinline__ void mma_role(const FwdParams &p, FwdSmem &sm, uint32
     const uint32_t tS0 = tmem + X * kSlotCols;
     const uint32_t tO = tS0 + kColO;
     const uint32_t id_pv = make_idesc(128, 64, bf16, true);
-    // cs: the next QK^T to issue; cp: the next PV.
+    // cs: the next QK^T to issue; cp: the next PV.  Each walks the K (V)
+    // stages in order: stage index and phase parity.
     MmaCursor cs, cp;
+    int ks = 0, vs = 0;
+    uint32_t kph = 0, vph = 0;
     cs.k = cs.t = cs.j = 0;
-    if (!warp_wait(p, sm, &sm.item_full[X][0], 0u)) return;
-    cs.kind = sm.items[X][0].kind;
-    cs.ntiles = sm.items[X][0].ntiles;
+    if (!mma_load_item(p, sm, cs, X)) return;
     cp = cs;
     // The first two QK^T of the slot.
     for (int i = 0; i < 2 && cs.kind != 0; ++i) {
-        if (!mma_issue_s(p, sm, tS0, X, cs, bf16) || !mma_advance(p, sm, cs, X)) return;
+        if (!mma_issue_s(p, sm, tS0, X, cs, ks, kph, bf16) || !mma_advance(p, sm, cs, X)) return;
     }
 #pragma unroll 1
     while (cp.kind != 0) {
-        const ItemInfo &I = sm.items[X][cp.k % kRing];
-        const int stage = cp.j % kStages;
-        if (!warp_wait(p, sm, &sm.p_full[X][cp.j & 1], uint32_t(cp.j >> 1) & 1u)) return;
+        if (!thread_wait(p, sm, &sm.p_full[X][cp.j & 1], uint32_t(cp.j >> 1) & 1u)) return;
         // The first PV of an item overwrites O: the epilogue of the item
         // before must have read it.
-        if (cp.t == 0 && cp.k > 0 &&
-            !warp_wait(p, sm, &sm.o_free[X], uint32_t(cp.k - 1) & 1u))
+        if (cp.t == 0 && cp.k > 0 && !thread_wait(p, sm, &sm.o_free[X], uint32_t(cp.k - 1) & 1u))
             return;
-        if (!warp_wait(p, sm, &sm.v_full[X][stage], uint32_t(cp.j / kStages) & 1u)) return;
+        if (!thread_wait(p, sm, &sm.v_full[X][vs], vph)) return;
         tc_fence_after();
-        const uint64_t vdesc = make_sdesc(smem_u32(sm.v[X][stage]), 16, 1024);
+        const uint64_t vdesc = make_sdesc(smem_u32(sm.v[X][vs]), 16, 1024);
         const uint32_t tP = tS0 + (cp.j & 1) * kTileKeys;
-        const int ksteps = tile_cols(I, cp.t) >> 4;
-        for (int kk = 0; kk < ksteps; ++kk)
-            mma_ts_elect(tO, tP + kk * 8, vdesc + uint64_t((kk * 2048) >> 4), id_pv,
-                         (kk > 0 || cp.t > 0) ? 1u : 0u);
-        tc_commit_elect(&sm.v_empty[X][stage]);
-        tc_commit_elect(&sm.pv_done[X]);
-        const bool last = cp.t == cp.ntiles - 1;
-        if (last) tc_commit_elect(&sm.o_full[X]);
-        __syncwarp();
-        if (last && (threadIdx.x & 31) == 0) mbar_arrive(&sm.item_empty[X][cp.k % kRing]);
+        const int ksteps = cursor_cols(cp, cp.t) >> 4;
+#pragma unroll
+        for (int kk = 0; kk < kTileKeys / 16; ++kk)
+            if (kk < ksteps)
+                mma_ts(tO, tP + kk * 8, vdesc + uint64_t((kk * 2048) >> 4), id_pv,
+                       (kk > 0 || cp.t > 0) ? 1u : 0u);
+        tc_commit(&sm.v_empty[X][vs]);
+        tc_commit(&sm.pv_done[X]);
+        if (++vs == kStages) {
+            vs = 0;
+            vph ^= 1u;
+        }
+        if (cp.t == cp.ntiles - 1) {
+            tc_commit(&sm.o_full[X]);
+            mbar_arrive(&sm.item_empty[X][cp.k % kRing]);
+        }
         if (!mma_advance(p, sm, cp, X)) return;
         // QK^T two tiles ahead, into the buffer P(j) has just been read from.
         if (cs.kind != 0) {
-            if (!mma_issue_s(p, sm, tS0, X, cs, bf16) || !mma_advance(p, sm, cs, X)) return;
+            if (!mma_issue_s(p, sm, tS0, X, cs, ks, kph, bf16) || !mma_advance(p, sm, cs, X)) return;
         }
     }
 }
@@ -1223,11 +1261,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             producer_role(p, sm, warp - kWarpProducer, lane);
         } else {
             const int X = warp - kWarpMma;
-            mma_role(p, sm, tmem, X, std::is_same<T, __nv_bfloat16>::value);
-            // Every MMA this warp issued has completed once this commit lands.
-            tc_commit_elect(&sm.drain[X]);
+            if (lane == 0) {
+                mma_role(p, sm, tmem, X, std::is_same<T, __nv_bfloat16>::value);
+                // Every MMA this thread issued has completed once this commit lands.
+                tc_commit(&sm.drain[X]);
+                drain_wait(&sm.drain[X], 0, p.wait_ns);
+            }
             __syncwarp();
-            drain_wait(&sm.drain[X], 0, p.wait_ns);
         }
     }
     tc_fence_before();
@@ -1250,47 +1290,70 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
 }
 
-// Merges the chunk partials of every global row into its output row: one
-// warp per (batch*head, global slot); lane l handles dimensions 2l, 2l+1.
-// Launched after the attention kernel (programmatic dependent launch: its
-// prologue overlaps the attention kernel's tail, the wait below orders it).
+// Merges the chunk partials of every global row into its output row.  A
+// block takes 32 global slots of one (batch*head), lane = slot, so that every
+// load is one 128-byte run of a field over the 32 slots; warp w owns the
+// output dimensions [4w, 4w + 4).  One pass over the chunks keeps a running
+// maximum (log-sum-exp: m in log2 units, the row sum l and the unnormalised
+// output are rescaled when it grows).  Launched after the attention kernel
+// (programmatic dependent launch: the wait below orders it).
+constexpr int kCombineWarps = kDHead / 4;
+
 template <typename T>
-__global__ void __launch_bounds__(128) combine_kernel(const AttnArgs a)
+__global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const AttnArgs a)
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int lane = threadIdx.x & 31;
+    const int d0 = 4 * (threadIdx.x >> 5);
     const int bh = blockIdx.x;
-    const int slot = blockIdx.y * 4 + (threadIdx.x >> 5);
+    const int slot = blockIdx.y * 32 + lane;
     const int b = bh / a.H;
     const int g = min(a.ws.counts[b], a.max_global);
+    if (int(blockIdx.y) * 32 >= g) return;
+    const size_t mg = size_t(a.max_global);
+    const size_t cstride = kPartialFloats * mg;
+    const float *P = partial_base(a, bh, 0) + min(slot, a.max_global - 1);
+    float M = -INFINITY, L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    // Eight chunks per round: all their loads are issued before any is used,
+    // so the round costs one memory latency.
+    constexpr int kPerRound = 8;
+    for (int c0 = 0; c0 < a.L.nchunks; c0 += kPerRound) {
+        float mc[kPerRound], lc[kPerRound], oc[kPerRound][4];
+#pragma unroll
+        for (int u = 0; u < kPerRound; ++u) {
+            const bool in = c0 + u < a.L.nchunks;
+            const float *pc = P + size_t(in ? c0 + u : 0) * cstride;
+            mc[u] = in ? __ldcg(pc) : -INFINITY;
+            lc[u] = __ldcg(pc + mg);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) oc[u][x] = __ldcg(pc + (2 + d0 + x) * mg);
+        }
+        float mr = M;
+#pragma unroll
+        for (int u = 0; u < kPerRound; ++u) mr = fmaxf(mr, mc[u]);
+        if (mr == -INFINITY) continue;      // no key for this row so far
+        const float fo = exp2f(M - mr);     // 0 while M is still -inf
+        L *= fo;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) acc[x] *= fo;
+#pragma unroll
+        for (int u = 0; u < kPerRound; ++u) {
+            const float f = exp2f(mc[u] - mr);   // 0 for a chunk without keys
+            L = fmaf(f, lc[u], L);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) acc[x] = fmaf(f, oc[u][x], acc[x]);
+        }
+        M = mr;
+    }
     if (slot >= g) return;
     const int pos = a.ws.gidx[size_t(b) * a.n + slot];
     if (!bit_at(a.ws.vbits + size_t(b) * a.L.nwords, pos)) return;   // padded: zeros elsewhere
-    const int nch = a.L.nchunks;
-    const size_t mg = size_t(a.max_global);
-    const size_t cstride = kPartialFloats * mg;
-    const float *P = partial_base(a, bh, 0) + slot;
-    float M = -INFINITY;
-    for (int c = lane; c < nch; c += 32) M = fmaxf(M, P[c * cstride]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f, a0 = 0.f, a1 = 0.f;
-#pragma unroll 4
-    for (int c = 0; c < nch; ++c) {
-        const float *pc = P + c * cstride;
-        const float mc = pc[0];
-        const float f = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
-        L = fmaf(f, pc[mg], L);
-        a0 = fmaf(f, pc[(2 + 2 * lane) * mg], a0);
-        a1 = fmaf(f, pc[(3 + 2 * lane) * mg], a1);
-    }
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    T *dst = static_cast<T *>(a.out) + (size_t(bh) * a.n + pos) * kDHead;
-    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-        reinterpret_cast<__nv_bfloat162 *>(dst)[lane] = __floats2bfloat162_rn(a0 * inv, a1 * inv);
-    } else {
-        reinterpret_cast<__half2 *>(dst)[lane] = __floats2half2_rn(a0 * inv, a1 * inv);
-    }
+    T *dst = static_cast<T *>(a.out) + (size_t(bh) * a.n + pos) * kDHead + d0;
+    uint2 v;
+    v.x = pack2<T>(acc[0] * inv, acc[1] * inv);
+    v.y = pack2<T>(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2 *>(dst) = v;
 }
 
 // ------------------------------------------------------------------ host
@@ -1467,8 +1530,8 @@ int launch_typed(const AttnArgs &a, CUtensorMapDataType dt, cudaStream_t stream)
     if (cudaLaunchKernelEx(&cfg, attn_fwd_kernel<T>, p) != cudaSuccess) return kErrCuda;
     if (a.max_global > 0 && !p.merge_in_kernel) {
         cudaLaunchConfig_t cc = {};
-        cc.gridDim = dim3(a.B * a.H, (a.max_global + 3) / 4);
-        cc.blockDim = dim3(128);
+        cc.gridDim = dim3(a.B * a.H, (a.max_global + 31) / 32);
+        cc.blockDim = dim3(32 * kCombineWarps);
         cc.stream = stream;
         cc.attrs = attr;
         cc.numAttrs = 1;

@@ -43,11 +43,14 @@ __device__ __forceinline__ uint32_t word_bits(const uint8_t *m, int p0, int n, b
     return w;
 }
 
-// One CTA per batch.  Any output pointer may be NULL (not written).
+// One CTA per batch.  Any output pointer may be NULL (not written).  The
+// entries of gidx past the count are set to -1 only with fill_tail (the
+// attention kernels read the first count entries alone).
 __global__ void __launch_bounds__(kPrepThreads)
 prepare_kernel(const uint8_t *__restrict__ local_mask, const uint8_t *__restrict__ global_mask,
                int B, int n, int max_global, int32_t *gidx, int32_t *counts, int *flags,
-               uint32_t *vbits, uint32_t *gbits, int *status, int *counters, int counters_per_batch)
+               uint32_t *vbits, uint32_t *gbits, int *status, int *counters, int counters_per_batch,
+               int fill_tail)
 {
     // The attention kernel may start its prologue now; it waits for this
     // grid's results before reading them.
@@ -120,7 +123,8 @@ prepare_kernel(const uint8_t *__restrict__ local_mask, const uint8_t *__restrict
                 gidx[size_t(b) * n + off++] = 32 * (w0 + k) + i;
             }
         }
-        for (int p = total + tid; p < n; p += kPrepThreads) gidx[size_t(b) * n + p] = -1;
+        if (fill_tail)
+            for (int p = total + tid; p < n; p += kPrepThreads) gidx[size_t(b) * n + p] = -1;
     }
     if (tid == 0) {
         if (counts) counts[b] = total;
@@ -132,12 +136,12 @@ prepare_kernel(const uint8_t *__restrict__ local_mask, const uint8_t *__restrict
 int launch_prepare(const uint8_t *local_mask, const uint8_t *global_mask, int B, int n,
                    int max_global, int32_t *gidx, int32_t *counts, int *flags, uint32_t *vbits,
                    uint32_t *gbits, int *status, int *counters, int counters_per_batch,
-                   cudaStream_t stream)
+                   int fill_tail, cudaStream_t stream)
 {
     if ((n + 31) / 32 > kPrepThreads * kPrepMaxWordsPerThread) return kErrUnsupported;
     prepare_kernel<<<B, kPrepThreads, 0, stream>>>(local_mask, global_mask, B, n, max_global, gidx,
                                                    counts, flags, vbits, gbits, status, counters,
-                                                   counters_per_batch);
+                                                   counters_per_batch, fill_tail);
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 
