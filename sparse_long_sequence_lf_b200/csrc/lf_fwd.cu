@@ -1302,6 +1302,8 @@ constexpr int kCombineWarps = kDHead / 4;
 template <typename T>
 __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const AttnArgs a)
 {
+    // The next kernel in the stream may launch now; it waits for this grid.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int lane = threadIdx.x & 31;
     const int d0 = 4 * (threadIdx.x >> 5);

@@ -68,6 +68,28 @@ prepare_kernel(const uint8_t *__restrict__ local_mask, const uint8_t *__restrict
     const int wpt = (nwords + kPrepThreads - 1) / kPrepThreads;   // words per thread (<= 8)
     const int w0 = tid * wpt;
 
+    // The mask words first, into registers: the masks are inputs of this
+    // call, read while the kernel ahead in the stream (launched with
+    // programmatic serialization, so this grid may start before it ends)
+    // may still read the workspace written below.
+    uint32_t gw[kPrepMaxWordsPerThread], vw[kPrepMaxWordsPerThread];
+    int mine = 0, pad = 0;
+#pragma unroll
+    for (int k = 0; k < kPrepMaxWordsPerThread; ++k) {
+        gw[k] = 0u;
+        vw[k] = 0u;
+        const int w = w0 + k;
+        if (k < wpt && w < nwords) {
+            gw[k] = word_bits(gm, 32 * w, n, gm != nullptr, false);
+            vw[k] = word_bits(lm, 32 * w, n, lm != nullptr, true);
+            mine += __popc(gw[k]);
+            const int left = n - 32 * w;
+            const uint32_t inrange = left >= 32 ? 0xffffffffu : ((1u << left) - 1u);
+            pad |= (vw[k] != inrange);
+        }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
     // The status word, and the attention kernel's item counter and finished
     // count (words 16 and 32 of the status region), start at zero.
     if (tid == 0 && b == 0 && status) {
@@ -78,23 +100,12 @@ prepare_kernel(const uint8_t *__restrict__ local_mask, const uint8_t *__restrict
     if (counters)
         for (int c = tid; c < counters_per_batch; c += kPrepThreads)
             counters[size_t(b) * counters_per_batch + c] = 0;
-
-    uint32_t gw[kPrepMaxWordsPerThread];
-    int mine = 0, pad = 0;
 #pragma unroll
     for (int k = 0; k < kPrepMaxWordsPerThread; ++k) {
-        gw[k] = 0u;
         const int w = w0 + k;
         if (k < wpt && w < nwords) {
-            const uint32_t g = word_bits(gm, 32 * w, n, gm != nullptr, false);
-            const uint32_t v = word_bits(lm, 32 * w, n, lm != nullptr, true);
-            gw[k] = g;
-            mine += __popc(g);
-            const int left = n - 32 * w;
-            const uint32_t inrange = left >= 32 ? 0xffffffffu : ((1u << left) - 1u);
-            pad |= (v != inrange);
-            if (vbits) vbits[size_t(b) * nwords + w] = v;
-            if (gbits) gbits[size_t(b) * nwords + w] = g;
+            if (vbits) vbits[size_t(b) * nwords + w] = vw[k];
+            if (gbits) gbits[size_t(b) * nwords + w] = gw[k];
         }
     }
     // Block-wide exclusive scan of the per-thread global counts.
@@ -139,9 +150,21 @@ int launch_prepare(const uint8_t *local_mask, const uint8_t *global_mask, int B,
                    int fill_tail, cudaStream_t stream)
 {
     if ((n + 31) / 32 > kPrepThreads * kPrepMaxWordsPerThread) return kErrUnsupported;
-    prepare_kernel<<<B, kPrepThreads, 0, stream>>>(local_mask, global_mask, B, n, max_global, gidx,
-                                                   counts, flags, vbits, gbits, status, counters,
-                                                   counters_per_batch, fill_tail);
+    // Programmatic dependent launch: the mask loads overlap the tail of the
+    // kernel ahead in the stream; the writes wait for it (griddepcontrol.wait).
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(B);
+    cfg.blockDim = dim3(kPrepThreads);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, prepare_kernel, local_mask, global_mask, B, n, max_global, gidx,
+                           counts, flags, vbits, gbits, status, counters, counters_per_batch,
+                           fill_tail) != cudaSuccess)
+        return kErrCuda;
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 
