@@ -53,7 +53,7 @@ def load_peaks():
 # Kernel sources whose change invalidates a stored DRAM-traffic figure.
 TRAFFIC_SOURCES = {
     "attn_fwd_kernel": ("lf_fwd.cu", "lf_sm100.cuh", "lf_device.cuh"),
-    "band_simt_kernel": ("lf_simt.cu", "lf_device.cuh"),
+    "attn_f32_kernel": ("lf_simt.cu", "lf_device.cuh"),
     "proj_kernel": ("lf_proj.cu", "lf_sm100.cuh", "lf_device.cuh"),
 }
 
@@ -253,7 +253,8 @@ def run_gpu_arm(args, wl, world, rank, local):
         raise RuntimeError(f"device status {status} after warm-up")
 
     chunk = nsets * max(1, 64 // nsets)
-    g_chunk = capture(step, min(chunk, args.steps))
+    n_chunk = min(chunk, args.steps)           # steps in one replay of g_chunk
+    g_chunk = capture(step, n_chunk)
     full, rem = divmod(args.steps, chunk) if args.steps >= chunk else (0, args.steps)
     g_rem = capture(step, rem) if (rem and full) else None
     if full == 0:
@@ -301,7 +302,7 @@ def run_gpu_arm(args, wl, world, rank, local):
 
     # Distribution of the step time: every replay of the graph timed on its
     # own (events on the launching stream), at least 50 replays.
-    step_dist = replay_distribution(replay, g_chunk, chunk, stream, device, samples=50)
+    step_dist = replay_distribution(replay, g_chunk, n_chunk, stream, device, samples=50)
 
     status = lf.workspace_status(ws, stream)
     if status != 0:
@@ -331,7 +332,7 @@ def run_gpu_arm(args, wl, world, rank, local):
     peaks, peak_kind = load_peaks()
     achieved_gbs = bytes_ / (kernel_ms * 1e-3) / 1e9
     kernel_tflops = flops / (kernel_ms * 1e-3) / 1e12
-    kname = "attn_fwd_kernel" if wl.dtype != "f32" else "band_simt_kernel"
+    kname = "attn_fwd_kernel" if wl.dtype != "f32" else "attn_f32_kernel"
     roofline = {
         "kernel": kname,
         "bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],

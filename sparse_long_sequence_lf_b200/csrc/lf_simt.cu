@@ -2,26 +2,29 @@
 //
 // fp32 inputs are computed in fp32 on the FMA pipes end to end (the tensor
 // cores' tf32 mode keeps 10 mantissa bits, too few for fp32 parity).  One
-// launch holds two kinds of CTAs, 128 threads each:
+// launch holds two kinds of CTAs, 256 threads (eight warps) each, so that
+// every SM sub-partition has two warps to switch between:
 //
 //   global CTAs   (batch*head, 512-key chunk, group of 32 global rows): each
-//                 of the four warps takes a quarter of the chunk's keys for
+//                 of the eight warps takes an eighth of the chunk's keys for
 //                 every row of the group (lane = key for the scores, lane =
-//                 two head dimensions for Vg), the four quarters are merged
-//                 in shared memory into the chunk's fp32 partials (max, sum,
+//                 two head dimensions for Vg), the eight parts are merged in
+//                 shared memory into the chunk's fp32 partials (max, sum,
 //                 unnormalised output), and the last CTA of a group merges
 //                 the chunks by log-sum-exp into the output rows.
 //   band CTAs     8 query rows of one (batch, head, residue class of the
-//                 dilation), 16 threads per row; each thread takes 4 of the
-//                 64 keys of a staged tile with the full 64-wide dot product
-//                 (no reduction per score), the row's threads share the
-//                 running maximum, and their partial sums and outputs are
-//                 added up once at the end.  Keys stream through shared
-//                 memory in 64-key tiles (cp.async, three stages): the
-//                 window taps, then the global-token columns that are not
-//                 taps.  Writes every row except valid global rows (zeros
-//                 for padding).
+//                 dilation), one warp per row; each lane takes 2 of the 64
+//                 keys of a staged tile with the full 64-wide dot product
+//                 (no reduction per score), the row's lanes share the running
+//                 maximum, and their partial sums and outputs are added up
+//                 once at the end.  Keys stream through shared memory in
+//                 64-key tiles (cp.async, three stages): the window taps,
+//                 then the global-token columns that are not taps.  Writes
+//                 every row except valid global rows (zeros for padding).
 //
+// Before waiting for the kernel ahead in the stream, each CTA asks L2 for the
+// key and value rows it will read (their addresses follow from the kernel
+// arguments alone).
 // Shared-memory rows of K/V are 68 floats apart, so 16-byte reads of
 // different rows at the same column fall in distinct banks.  The launch is
 // chained to the mask-preparation kernel by programmatic dependent launch.
@@ -34,17 +37,17 @@
 
 namespace lf {
 
-constexpr int kF32Threads = 128;
+constexpr int kF32Threads = 256;
 constexpr int kBandRows = 8;                      // query rows per band CTA
-constexpr int kTpr = 16;                          // threads per row
+constexpr int kTpr = 32;                          // threads per row (one warp)
 constexpr int kBandParts = 128 / kBandRows;       // band CTAs per 128-row band item
 constexpr int kTileKeysF = 64;                    // keys per staged band tile
 constexpr int kKpt = kTileKeysF / kTpr;           // keys per thread and tile
 constexpr int kStride = 68;                       // floats between staged rows
 constexpr int kBandStages = 3;
-constexpr int kGWarps = 4;
+constexpr int kGWarps = kF32Threads / 32;
 constexpr int kGKeys = 32;                        // keys per warp tile (lane = key)
-constexpr int kGQuarter = kChunkKeys / kGWarps;   // 128 keys of a chunk per warp
+constexpr int kGQuarter = kChunkKeys / kGWarps;   // 64 keys of a chunk per warp
 constexpr float kRescaleF = 8.f;                  // lazy rescale (log2 units)
 
 struct BandSmem {
@@ -122,28 +125,29 @@ __device__ __forceinline__ void band_cta(const AttnArgs &a, int cta, uint8_t *sm
     const int nband = (hi - lo) / kTileKeysF + 1;
     const int ntiles = nband + (g + kTileKeysF - 1) / kTileKeysF;
 
-    // Loads tile t into its stage: thread t handles key tid/2, half a row.
+    // Loads tile t into its stage.  Sixteen consecutive threads copy one
+    // 256-byte row (16 bytes each), so a warp's copy covers two whole rows;
+    // thread tid takes rows tid/16 + 16u, u < 4.
     auto issue = [&](int t) {
         if (t < ntiles) {
             const int st = t % kBandStages;
-            const int c = tid >> 1;
-            int j;
-            if (t < nband) {
-                const int jr = lo + kTileKeysF * t + c;
-                j = jr <= hi ? jr * dil + r : -1;
-            } else {
-                const int slot = kTileKeysF * (t - nband) + c;
-                j = slot < g ? gl[slot] : -1;
-            }
-            const float *ks = K + size_t(j < 0 ? 0 : j) * kDHead;
-            const float *vs = V + size_t(j < 0 ? 0 : j) * kDHead;
-            const int f0 = (tid & 1) * 32;
+            const int part = (tid & 15) * 4;
 #pragma unroll
-            for (int f = 0; f < 32; f += 4) {
-                cp_async16(&sm.k[st][c][f0 + f], ks + f0 + f, j >= 0);
-                cp_async16(&sm.v[st][c][f0 + f], vs + f0 + f, j >= 0);
+            for (int u = 0; u < kTileKeysF / 16; ++u) {
+                const int c = (tid >> 4) + 16 * u;
+                int j;
+                if (t < nband) {
+                    const int jr = lo + kTileKeysF * t + c;
+                    j = jr <= hi ? jr * dil + r : -1;
+                } else {
+                    const int slot = kTileKeysF * (t - nband) + c;
+                    j = slot < g ? gl[slot] : -1;
+                }
+                const size_t row = size_t(j < 0 ? 0 : j) * kDHead + part;
+                cp_async16(&sm.k[st][c][part], K + row, j >= 0);
+                cp_async16(&sm.v[st][c][part], V + row, j >= 0);
+                if (part == 0) sm.pos[st][c] = (j >= 0 && bit_at(vb, j)) ? j : -1;
             }
-            if ((tid & 1) == 0) sm.pos[st][c] = (j >= 0 && bit_at(vb, j)) ? j : -1;
         }
         cp_async_commit();
     };
@@ -215,35 +219,37 @@ __device__ __forceinline__ void band_cta(const AttnArgs &a, int cta, uint8_t *sm
     }
     cp_async_wait<0>();
 
-    // Sum over the row's 16 threads: l by shuffles, acc through shared memory
-    // (the staging area is free now); thread tl then owns dims 4tl .. 4tl+3.
+    // Sum over the row's 32 threads: l by shuffles, acc through shared memory
+    // (the K and V staging areas, contiguous, are free now); thread tl then
+    // owns dims 2tl and 2tl+1.
 #pragma unroll
     for (int o = 1; o < kTpr; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
     __syncthreads();
+    static_assert(sizeof(float) * kBandRows * kTpr * (kDHead + 4) <=
+                      sizeof(BandSmem::k) + sizeof(BandSmem::v),
+                  "row-sum buffer exceeds the staging area");
     float *red = &sm.k[0][0][0];                  // [kBandRows][kTpr][kDHead + 4]
     float *mine = red + (rl * kTpr + tl) * (kDHead + 4);
 #pragma unroll
     for (int x = 0; x < kDHead; x += 4)
         *reinterpret_cast<float4 *>(mine + x) = make_float4(acc[x], acc[x + 1], acc[x + 2], acc[x + 3]);
     __syncthreads();
-    float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
+    float2 o2 = make_float2(0.f, 0.f);
+#pragma unroll 8
     for (int w = 0; w < kTpr; ++w) {
-        const float4 p4 = *reinterpret_cast<const float4 *>(red + (rl * kTpr + w) * (kDHead + 4) + 4 * tl);
-        o4.x += p4.x;
-        o4.y += p4.y;
-        o4.z += p4.z;
-        o4.w += p4.w;
+        const float2 p2 = *reinterpret_cast<const float2 *>(red + (rl * kTpr + w) * (kDHead + 4) + 2 * tl);
+        o2.x += p2.x;
+        o2.y += p2.y;
     }
     if (!row_in) return;
-    float *O = static_cast<float *>(a.out) + bh * n * kDHead + size_t(i) * kDHead + 4 * tl;
+    float *O = static_cast<float *>(a.out) + bh * n * kDHead + size_t(i) * kDHead + 2 * tl;
     if (!bit_at(vb, i)) {
-        *reinterpret_cast<float4 *>(O) = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float2 *>(O) = make_float2(0.f, 0.f);
         return;
     }
     if (bit_at(gb, i)) return;     // written by the global rows
     const float inv = 1.f / l;
-    *reinterpret_cast<float4 *>(O) = make_float4(o4.x * inv, o4.y * inv, o4.z * inv, o4.w * inv);
+    *reinterpret_cast<float2 *>(O) = make_float2(o2.x * inv, o2.y * inv);
 }
 
 // ---------------------------------------------------------------- global
@@ -294,17 +300,23 @@ __device__ __forceinline__ void global_cta(const AttnArgs &a, int cta, uint8_t *
     const int kbeg = chunk * kChunkKeys + warp * kGQuarter;
     const int kend = min(key_end, kbeg + kGQuarter);
     for (int k0 = kbeg; k0 < kend; k0 += kGKeys) {
-        // This warp's tile: lane = key.
-        const int j = k0 + lane;
-        const bool in = j < kend;
-        const float *ks = Kg + size_t(in ? j : 0) * kDHead;
-        const float *vs = Vg + size_t(in ? j : 0) * kDHead;
+        // This warp's tile (lane = key in the arithmetic below).  The copy
+        // goes by rows: 16 consecutive lanes take one 256-byte row.
+        {
+            const int part = (lane & 15) * 4;
 #pragma unroll
-        for (int f = 0; f < kDHead; f += 4) {
-            cp_async16(&sm.k[warp][lane][f], ks + f, in);
-            cp_async16(&sm.v[warp][lane][f], vs + f, in);
+            for (int u = 0; u < kGKeys / 2; ++u) {
+                const int c = (lane >> 4) + 2 * u;
+                const int jc = k0 + c;
+                const bool inc = jc < kend;
+                const size_t row = size_t(inc ? jc : 0) * kDHead + part;
+                cp_async16(&sm.k[warp][c][part], Kg + row, inc);
+                cp_async16(&sm.v[warp][c][part], Vg + row, inc);
+            }
         }
         cp_async_commit();
+        const int j = k0 + lane;
+        const bool in = j < kend;
         sm.ok[warp][lane] = in && bit_at(vb, j);
         cp_async_wait<0>();
         __syncwarp();
@@ -358,8 +370,8 @@ __device__ __forceinline__ void global_cta(const AttnArgs &a, int cta, uint8_t *
     }
     __syncthreads();
 
-    // Merge the four quarters of the chunk into its partials: warp w takes
-    // rows w, w+4, ...; lane owns two dimensions.
+    // Merge the eight parts of the chunk into its partials: warp w takes
+    // rows w, w+8, ...; lane owns two dimensions.
     const size_t mg = size_t(a.max_global);
     for (int s = warp; s < rows; s += kGWarps) {
         float M = -INFINITY;
@@ -404,9 +416,54 @@ __device__ __forceinline__ void global_cta(const AttnArgs &a, int cta, uint8_t *
     }
 }
 
+// Brings `bytes` (a multiple of 16) from 16-byte aligned global memory into L2.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes)
+{
+    if (bytes == 0) return;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// The key and value rows a CTA will read, into L2, from the kernel arguments
+// alone (no workspace value): a global CTA's chunk of Kg and Vg, a band CTA's
+// query rows and the contiguous span of sequence positions its window taps
+// fall in.  Issued before the wait for the kernel ahead in the stream; L2 is
+// the point of coherence, so nothing it holds goes stale.
+__device__ __forceinline__ void prefetch_inputs(const AttnArgs &a, int cta, int nglob)
+{
+    const int n = a.n;
+    constexpr uint32_t kRow = kDHead * sizeof(float);
+    if (cta < nglob) {
+        const int per_bh = a.L.nchunks * a.L.ngroups;
+        const int bh = cta / per_bh;
+        const int chunk = (cta - bh * per_bh) % a.L.nchunks;
+        const int k0 = chunk * kChunkKeys, k1 = min(n, k0 + kChunkKeys);
+        const size_t off = (size_t(bh) * n + k0) * kDHead;
+        prefetch_l2(static_cast<const float *>(a.kg) + off, uint32_t(k1 - k0) * kRow);
+        prefetch_l2(static_cast<const float *>(a.vg) + off, uint32_t(k1 - k0) * kRow);
+        return;
+    }
+    cta -= nglob;
+    int b, h, r, tile;
+    band_item(a, cta / kBandParts, b, h, r, tile);
+    const int dil = a.dil[h];
+    const int n_r = (n - r + dil - 1) / dil;
+    const int r0 = tile * 128 + (cta % kBandParts) * kBandRows;
+    if (r0 >= n_r) return;
+    const int rows_hi = min(r0 + kBandRows - 1, n_r - 1);
+    const int lo = max(a.causal ? r0 - (a.window - 1) : r0 - a.half, 0);
+    const int hi = min(a.causal ? rows_hi : rows_hi + a.half, n_r - 1);
+    const size_t base = size_t(b * a.H + h) * n * kDHead;
+    const size_t q0 = size_t(r0 * dil + r) * kDHead, q1 = size_t(rows_hi * dil + r + 1) * kDHead;
+    const size_t j0 = size_t(lo * dil + r) * kDHead, j1 = size_t(hi * dil + r + 1) * kDHead;
+    prefetch_l2(static_cast<const float *>(a.q) + base + q0, uint32_t((q1 - q0) * sizeof(float)));
+    prefetch_l2(static_cast<const float *>(a.k) + base + j0, uint32_t((j1 - j0) * sizeof(float)));
+    prefetch_l2(static_cast<const float *>(a.v) + base + j0, uint32_t((j1 - j0) * sizeof(float)));
+}
+
 __global__ void __launch_bounds__(kF32Threads) attn_f32_kernel(const AttnArgs a, int nglob)
 {
     extern __shared__ __align__(16) uint8_t f32_smem[];
+    if (threadIdx.x == 0) prefetch_inputs(a, blockIdx.x, nglob);
     // The compacted indices, counts and bitmaps come from the kernel before.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (blockIdx.x == 0)
