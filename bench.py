@@ -1163,13 +1163,16 @@ def run_oracle_heads(oracle, x, wl, heads):
 def run_cpu_baseline(wl, budget_s=10.0):
     import oracle
     x, heads, reps, flops = oracle_sample_plan(wl, budget_s)
+    # The thread count of the OpenMP run, read before the single-thread run
+    # below sets the OpenMP default to one thread.
+    cores = oracle.default().max_threads()
     t0 = time.perf_counter()
     for _ in range(reps):
         run_oracle_heads(oracle, x, wl, heads)
     dt = time.perf_counter() - t0
     single = run_cpu_single_thread(wl, x, budget_s=max(1.0, budget_s / 4))
     return {"value": round(flops * reps / dt / 1e12, 6), "unit": UNIT,
-            "cores": oracle.default().max_threads(), "kind": "oracle",
+            "cores": cores, "kind": "oracle",
             "sample": f"{heads} of {wl.H} heads x {wl.B} batches, {reps} repetition(s), "
                       f"{dt:.1f} s, fp64 C oracle with OpenMP",
             "seconds": round(dt, 2), "single_thread": single}
