@@ -10,7 +10,7 @@
 //   band items    128 query rows of one (batch, head, residue class of the
 //                 head's dilation).  A dilated head is a plain band over each
 //                 residue subsequence x[r::dil], so the same tile loop serves
-//                 every dilation.  The keys stream as 128-key tiles over the
+//                 every dilation.  The keys stream as 96-key tiles over the
 //                 band's diagonals, then as tiles of the (deduplicated) global
 //                 tokens; an online softmax runs over all of them.
 //   global items  up to 128 global rows of one (batch, head) against one
@@ -22,38 +22,38 @@
 //
 // Schedule.  A persistent grid, one CTA per SM.  Items are handed out by a
 // device-wide atomic counter (band items first, the cheaper global items
-// last), so CTAs that finish early take more work.  Each CTA runs two item
-// "slots" at once; their softmax warpgroups alternate with the tensor core:
-// while slot 0 turns its scores into probabilities, the tensor core runs
-// slot 1's PV and next QK^T, and the other way round.
+// last), so CTAs that finish early take more work; the first item of every
+// slot is fixed by its CTA index.  Each CTA runs two item "slots" at once;
+// their softmax warpgroups share the tensor core and the exponential units.
 //
-// Layout of one CTA (384 threads = 3 warpgroups):
+// Layout of one CTA (384 threads):
 //   warps 0-3    softmax warpgroup of slot 0 (thread t owns query row t)
 //   warps 4-7    softmax warpgroup of slot 1
-//   warp  8      TMA producer of both slots: fetches items, decodes them,
-//                loads Q, K, V tiles, and precomputes each key tile's column
-//                masks (padding bits, global-token positions) in shared memory
-//   warp  9      MMA issuer of both slots (one elected thread), owns TMEM
-//   warps 10-11  idle (registers go to the softmax warpgroups)
+//   warps 8, 9   TMA producers of slots 0 and 1: item records two ahead, Q,
+//                K and V tiles, and each key tile's column masks (padding
+//                bits, global-token positions) in shared memory
+//   warps 10, 11 MMA issuers of slots 0 and 1 (lane 0 only: one thread waits
+//                on the barriers and issues every MMA and commit); warp 10
+//                allocates and frees the tensor memory
 //
-// TMEM (512 columns, slot X uses [256X, 256X+256)): the 128-key score tile S
-// (fp32; the 16-bit probabilities P overwrite its first 64 columns as pairs)
-// and two 64-column output accumulators O, used by alternate items so that
-// the epilogue of item k (done by the softmax warps after the first tile of
-// item k+1) overlaps item k+1's products.
+// TMEM (512 columns, slot X uses [256X, 256X+256)): two 96-column score
+// buffers S0, S1 (fp32; the 16-bit probabilities P overwrite the first 48
+// columns of a buffer as pairs) and a 64-column output accumulator O.
 //   S = Q K^T      tcgen05.mma kind::f16, A = Q (smem, K-major),
-//                  B = K tile (smem, K-major), 128x128 fp32 in TMEM
+//                  B = K tile (smem, K-major), 128x96 fp32 in TMEM
 //   O += P V       tcgen05.mma kind::f16, A = P (TMEM), B = V tile
 //                  (smem, MN-major), 128x64 fp32 in TMEM
-// Per slot and tile the MMA warp issues PV(j) then S(j+1): when the softmax
-// sees S(j+1) ready, every product before it (PV(j) included) is complete.
+// Per slot and tile the issuer puts PV(j) then S(j+2) into the buffer P(j)
+// was read from, so the softmax of tile j+1 finds its scores ready.  The
+// epilogue of item k (done by the softmax warps after the first tile of item
+// k+1) reads O before the first PV of item k+1 overwrites it.
 // Shared-memory tiles have 128-byte rows with the 128-byte swizzle, written
 // by TMA: whole tiles from residue-class tensor maps (rows r, r+dil, ...),
 // single-row loads for global tokens, gathered Qg rows and heads beyond the
-// residue-map budget.  K/V tiles run through a 4-stage ring shared by the two
-// slots (filled and drained in the same alternating order).  Every wait on an
-// mbarrier is bounded; on expiry the kernel records LF_ERR_DEVICE_TIMEOUT,
-// drains its own copies and MMAs, frees its TMEM and returns.
+// residue-map budget.  Each slot has two Q buffers and three K and three V
+// stages.  Every wait on an mbarrier is bounded; on expiry the kernel records
+// LF_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs, frees its TMEM and
+// returns.
 #include <algorithm>
 #include <atomic>
 #include <cstring>
