@@ -841,8 +841,10 @@ __device__ __forceinline__ bool softmax_tile(const FwdParams &p, FwdSmem &sm, ui
                 l *= a;
                 alpha_o *= a;
                 // Probabilities of earlier chunks of this tile were taken against
-                // the old maximum.
+                // the old maximum.  Their stores must land before they are
+                // read back.
                 if (__any_sync(0xffffffffu, a != 1.f && a != 0.f)) {
+                    if (c > 0) tmem_st_wait();
                     for (int c2 = 0; c2 < c; ++c2) {
                         float w[16];
                         tmem_ld16(tS + 16 * c2, w);
@@ -966,10 +968,21 @@ __device__ __forceinline__ void merge_global_rows(const AttnArgs &a, int b, int 
 
 // Per-row results an item's epilogue needs after the softmax has moved on;
 // the item's record stays in the slot's item ring until the epilogue is done.
+// The row's words of the valid-key and global-token bitmaps are loaded when
+// the item starts and decoded only in the epilogue, so their latency hides
+// behind the item's tiles.
 struct RowOut {
     float m, l;
-    bool write;     // band: the row exists and is not a valid global row
-    bool valid;     // band: the row is not padding
+    uint32_t vword, gword;  // band: bitmap words holding the row's position
+    int bit;                // band: the row's bit in them
+    bool row_in;            // band: the row exists
+    __device__ __forceinline__ bool valid() const { return row_in && ((vword >> bit) & 1u); }
+    // The row exists and is not a valid global row (those come from the
+    // global items).
+    __device__ __forceinline__ bool write() const
+    {
+        return row_in && (!valid() || !((gword >> bit) & 1u));
+    }
 };
 
 // Writes the output of item `ke` of slot X: band rows O / l (zeros for padded
@@ -989,14 +1002,15 @@ __device__ __forceinline__ void epilogue(const FwdParams &p, FwdSmem &sm, uint32
     const bool active = kind == 2 ? q0 + warp * 32 < I.g : q0 + warp * 32 < I.n_r;
     if (active) {
         if (kind == 1) {
-            const int pos = ro.write ? row * I.dil + I.r : 0;
+            const bool write = ro.write();
+            const int pos = write ? row * I.dil + I.r : 0;
             T *dst = static_cast<T *>(a.out) + (size_t(bh) * a.n + pos) * kDHead;
-            const float inv = ro.valid ? __frcp_rn(ro.l) : 0.f;
+            const float inv = ro.valid() ? __frcp_rn(ro.l) : 0.f;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float o[32];
                 tmem_ld32(tO + half * 32, o);
-                if (ro.write) store_half_row<T>(dst + half * 32, o, inv);
+                if (write) store_half_row<T>(dst + half * 32, o, inv);
             }
         } else {
             const int slot = row;
@@ -1121,15 +1135,17 @@ __device__ __forceinline__ void softmax_role(const FwdParams &p, FwdSmem &sm, ui
         const int wrow0 = I.q0 + warp * 32;
         const bool active = I.kind == 2 ? wrow0 < I.g : wrow0 < I.n_r;
         RowOut ro;
-        ro.write = false;
-        ro.valid = false;
+        ro.vword = ro.gword = 0u;
+        ro.bit = 0;
+        ro.row_in = false;
         if (I.kind == 1 && active) {
-            const bool row_in = row < I.n_r;
+            ro.row_in = row < I.n_r;
             const int i = row * I.dil + I.r;
-            const uint32_t *vb = a.ws.vbits + size_t(I.b) * a.L.nwords;
-            const uint32_t *gb = a.ws.gbits + size_t(I.b) * a.L.nwords;
-            ro.valid = row_in && bit_at(vb, i);
-            ro.write = row_in && (!ro.valid || !bit_at(gb, i));
+            ro.bit = i & 31;
+            if (ro.row_in) {
+                ro.vword = a.ws.vbits[size_t(I.b) * a.L.nwords + (i >> 5)];
+                ro.gword = a.ws.gbits[size_t(I.b) * a.L.nwords + (i >> 5)];
+            }
         }
         RowState st{-INFINITY, 0.f};
         // A record of kind 0 (no more items) runs no tile but still flushes
