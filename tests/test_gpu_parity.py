@@ -66,6 +66,13 @@ EDGE = [
     # ... and by the separate merge kernel (9 chunks)
     Workload("merge-9-chunks", "f16", 1, 2, 4097, 16, globals_kind="random:40",
              pad_tail=(5,), seed=14),
+    # More band items than a full grid holds at once (296 item slots on a
+    # B200), so slots take second items from the counter: dilations, global
+    # tokens and padding ...
+    Workload("items-beyond-grid", "bf16", 1, 8, 6000, 512, dilation=(1, 1, 1, 1, 2, 2, 3, 3),
+             globals_kind="random:3", pad_tail=(40,), seed=15),
+    # ... and 384 items of a single key tile each over three batches.
+    Workload("single-tile-items", "f16", 3, 64, 192, 8, dilation=(2,) * 64, seed=16),
 ]
 
 
