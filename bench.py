@@ -182,12 +182,17 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- GPU arm
-def make_device_sets(wl, nsets, device):
+def make_device_sets(wl, nsets, device, heads=None):
+    """`nsets` input sets of the workload on the device; with heads=(h0, h1)
+    only those heads of each full set (one problem split by heads)."""
     import torch
+    from sparse_long_sequence_lf_b200.sharding import shard_inputs
     from sparse_long_sequence_lf_b200.workloads import make_inputs
     sets = []
     for s in range(nsets):
         x = make_inputs(wl, seed=wl.seed + 7919 * s)
+        if heads is not None:
+            x = shard_inputs(x, *heads)
         sets.append({k: (v.to(device) if torch.is_tensor(v) else v) for k, v in x.items()})
     return sets
 
@@ -212,11 +217,20 @@ def run_gpu_arm(args, wl, world, rank, local):
     torch.cuda.set_device(device)
     dist = init_dist(world, "nccl")
 
-    x0 = make_device_sets(wl, 1, device)[0]
+    # --shard heads: the ranks split one problem by heads (strong scaling);
+    # otherwise every rank runs the whole workload (weak scaling).
+    wl_full, heads, ranges = wl, None, None
+    if args.shard == "heads" and world > 1:
+        from sparse_long_sequence_lf_b200.sharding import head_ranges
+        ranges = head_ranges(wl.H, world)
+        heads = ranges[rank]
+        wl = wl.with_(H=heads[1] - heads[0],
+                      dilation=tuple(wl.dilation_list()[heads[0]:heads[1]]))
+    x0 = make_device_sets(wl_full, 1, device, heads)[0]
     per_set = sum(t.numel() * t.element_size() for t in x0.values() if torch.is_tensor(t))
     per_set += x0["q"].numel() * x0["q"].element_size()          # output
     nsets = max(2, -(-2 * L2_BYTES // per_set))
-    sets = [x0] + make_device_sets(wl.with_(seed=wl.seed + 1), nsets - 1, device)
+    sets = [x0] + make_device_sets(wl_full.with_(seed=wl_full.seed + 1), nsets - 1, device, heads)
     outs = [torch.empty_like(s["q"]) for s in sets]
     max_global = max(int((s["global_mask"] != 0).sum(1).max()) if s["global_mask"] is not None
                      else 0 for s in sets)
@@ -326,8 +340,17 @@ def run_gpu_arm(args, wl, world, rank, local):
     flops = accounting.useful_flops(wl)
     bytes_ = accounting.algorithmic_bytes(wl)
     ms_per_step = max_ms / args.steps
-    value = whole_job_rate(flops, args.steps, world, max_ms) / 1e12
-    tokens_per_s = whole_job_rate(accounting.tokens(wl), args.steps, world, max_ms)
+    if heads is None:
+        value = whole_job_rate(flops, args.steps, world, max_ms) / 1e12
+        tokens_per_s = whole_job_rate(accounting.tokens(wl), args.steps, world, max_ms)
+    else:
+        # One problem over all ranks: its units over the slowest rank's time.
+        value = accounting.useful_flops(wl_full) * args.steps / (max_ms * 1e-3) / 1e12
+        tokens_per_s = accounting.tokens(wl_full) * args.steps / (max_ms * 1e-3)
+    shard_check = None
+    if heads is not None:
+        shard_check = check_head_shards(wl_full, sets[0], outs[0], ranges, max_global, ws,
+                                        stream, device, rank, step)
 
     peaks, peak_kind = load_peaks()
     achieved_gbs = bytes_ / (kernel_ms * 1e-3) / 1e9
@@ -337,7 +360,8 @@ def run_gpu_arm(args, wl, world, rank, local):
         "kernel": kname,
         "bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
         "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
-        "traffic": stored_traffic(kname, wl.name), "peak_source": peak_kind,
+        "traffic": stored_traffic(kname, wl.name) if heads is None else None,
+        "peak_source": peak_kind,
         "kernel_us": round(kernel_ms * 1e3, 3), "algorithmic_bytes": bytes_,
         "useful_tflops": round(kernel_tflops, 1),
         "tensor_frac_of_measured_bf16": round(kernel_tflops / peaks["bf16_tflops"], 4),
@@ -349,7 +373,8 @@ def run_gpu_arm(args, wl, world, rank, local):
         dist.barrier()
     e2e = run_e2e(args, wl, device, stream, max_global)
     e2e_max_ms = reduce_max(e2e["ms_per_step"], device)
-    e2e["value"] = round(whole_job_rate(flops, 1, world, e2e_max_ms) / 1e12, 4)
+    e2e["value"] = round((whole_job_rate(flops, 1, world, e2e_max_ms) if heads is None else
+                          accounting.useful_flops(wl_full) / (e2e_max_ms * 1e-3)) / 1e12, 4)
     e2e["ms_per_step"] = round(e2e_max_ms, 4)
 
     cpu = None
@@ -359,10 +384,10 @@ def run_gpu_arm(args, wl, world, rank, local):
     result = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": wl.dtype, "data": "synthetic",
+        "higher_is_better": True, "scaling": "weak" if heads is None else "strong",
+        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
         "tokens_per_s": round(tokens_per_s, 1),
-        "config": workload_config(wl, world),
+        "config": workload_config(wl_full, world, heads_split=heads is not None),
         "timing": {"l2": f"{nsets} rotating input sets, {nsets * per_set / 2**20:.0f} MiB > 2x L2",
                    "launch": "CUDA graph of C-ABI calls",
                    "useful_gflop_per_step": round(flops / 1e9, 4),
@@ -374,6 +399,8 @@ def run_gpu_arm(args, wl, world, rank, local):
         "gpu_launches": launches_per_step(wl, max_global) * args.steps,
         "clocks": clocks,
     }
+    if shard_check is not None:
+        result["shard_check"] = shard_check
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -1200,13 +1227,47 @@ def run_cpu_single_thread(wl, x, budget_s=2.5):
             "sample": f"rows 0..{rows} of batch 0 head 0, best of 3 ({best:.2f} s)"}
 
 
-def workload_config(wl, world):
+def workload_config(wl, world, heads_split=False):
     """The workload part of a bench line's config (both arms)."""
+    if world == 1:
+        par = "single GPU"
+    elif heads_split:
+        par = f"one problem, heads split over {world} GPUs"
+    else:
+        par = f"independent replicas x{world}"
     return {"workload": wl.name, "B": wl.B, "H": wl.H, "n": wl.n, "d_head": wl.d,
             "window": wl.window, "dilation": wl.dilation_list(), "causal": wl.causal,
             "globals": wl.globals_kind, "pad_tail": list(wl.pad_tail),
-            "global_batch": wl.B * world, "seq_len": wl.n,
-            "parallelism": f"independent replicas x{world}" if world > 1 else "single GPU"}
+            "global_batch": wl.B * (1 if heads_split else world), "seq_len": wl.n,
+            "parallelism": par}
+
+
+def check_head_shards(wl_full, set0, out0, ranges, max_global, ws, stream, device, rank, step):
+    """After the timed region of a head-split run: every rank recomputes its
+    heads of input set 0, the slices are all-gathered, and rank 0 compares
+    them with the whole problem run on its own GPU.  The heads are
+    independent, so the two must agree bit for bit."""
+    import torch
+    import sparse_long_sequence_lf_b200 as lf
+    from sparse_long_sequence_lf_b200.sharding import gather_heads
+    from sparse_long_sequence_lf_b200.workloads import make_inputs
+    with torch.cuda.stream(stream):
+        step(0)
+    stream.synchronize()
+    full = gather_heads(out0, ranges)
+    verdict = None
+    if rank == 0:
+        x = {k: (v.to(device) if torch.is_tensor(v) else v) for k, v in make_inputs(wl_full).items()}
+        ws_full = lf.new_workspace(wl_full.B, wl_full.H, wl_full.n, max_global, device)
+        ref = lf.attention_forward(x["q"], x["k"], x["v"], x["qg"], x["kg"], x["vg"],
+                                   x["local_mask"], x["global_mask"], window=wl_full.window,
+                                   dilation=x["dilation"], causal=wl_full.causal,
+                                   max_global=max_global, workspace=ws_full)
+        torch.cuda.synchronize(device)
+        if not torch.equal(ref, full):
+            raise RuntimeError("head-split output differs from the single-GPU output")
+        verdict = f"gathered heads equal the single-GPU forward bit for bit ({len(ranges)} ranks)"
+    return verdict
 
 
 def run_reference_arm(args, wl, world, rank):
@@ -1251,6 +1312,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="under torchrun: every rank runs the whole workload (replicas, weak "
+                         "scaling) or the ranks split one problem by heads (strong scaling)")
     ap.add_argument("--encoder", default=None,
                     help="encoder stack of --op encoder (default: the 24-layer fp16 model)")
     ap.add_argument("--op", choices=["attention", "projection", "output", "backward", "encoder"],
@@ -1267,6 +1331,10 @@ def main(argv=None):
         if world == 1 and args.gpus > 1:
             ap.error("--gpus N > 1 needs torchrun with N processes")
     wl = WORKLOADS[args.workload]
+    if args.shard == "heads" and world > wl.H:
+        ap.error("--shard heads needs at most H ranks")
+    if args.shard == "heads" and args.op != "attention":
+        ap.error("--shard heads applies to the attention op")
     if args.impl == "reference":
         run_reference_arm(args, wl, world, rank)
         return
