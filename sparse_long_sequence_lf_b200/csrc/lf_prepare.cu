@@ -88,6 +88,23 @@ prepare_kernel(const uint8_t *__restrict__ local_mask, const uint8_t *__restrict
             pad |= (vw[k] != inrange);
         }
     }
+    // Block-wide exclusive scan of the per-thread global counts (registers
+    // and shared memory only, so it also runs before the wait).
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    const int any_pad = __syncthreads_or(pad);
+    int before = 0, total = 0;
+    for (int w = 0; w < kPrepWarps; ++w) {
+        const int t = warp_sum[w];
+        before += (w < warp) ? t : 0;
+        total += t;
+    }
+    int off = before + incl - mine;
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // The status word, and the attention kernel's item counter and finished
@@ -108,22 +125,6 @@ prepare_kernel(const uint8_t *__restrict__ local_mask, const uint8_t *__restrict
             if (gbits) gbits[size_t(b) * nwords + w] = gw[k];
         }
     }
-    // Block-wide exclusive scan of the per-thread global counts.
-    int incl = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-    }
-    if (lane == 31) warp_sum[warp] = incl;
-    const int any_pad = __syncthreads_or(pad);
-    int before = 0, total = 0;
-    for (int w = 0; w < kPrepWarps; ++w) {
-        const int t = warp_sum[w];
-        before += (w < warp) ? t : 0;
-        total += t;
-    }
-    int off = before + incl - mine;
     if (gidx) {
 #pragma unroll
         for (int k = 0; k < kPrepMaxWordsPerThread; ++k) {
