@@ -804,9 +804,13 @@ def run_backward_arm(args, wl, world, rank, local):
             d["ws"] = lf.new_workspace(wl.B, wl.H, wl.n, mg, device)
             kw = dict(window=wl.window, dilation=xs["dilation"], causal=wl.causal,
                       max_global=mg)
+            # bf16 / fp16: the forward also keeps each row's log-sum-exp, which
+            # the backward reads instead of recomputing (the training pair).
+            d["lse"] = (torch.empty((wl.B, wl.H, wl.n), dtype=torch.float32, device=device)
+                        if wl.dtype != "f32" and not args.no_lse else None)
             d["out"] = lf.attention_forward(*[d[nm] for nm in names], d["local_mask"],
                                             d["global_mask"], workspace=d["ws"], stream=stream,
-                                            **kw)
+                                            lse=d["lse"], **kw)
             d["dout"] = make_output_grad(wl, seed=wl.seed + 7919 * s_).to(device)
             d["grads"] = {nm: torch.empty_like(d["q"]) for nm in names}
             d["kw"] = kw
@@ -822,7 +826,7 @@ def run_backward_arm(args, wl, world, rank, local):
         d = sets[i % nsets]
         lf.attention_backward(*[d[nm] for nm in names], d["out"], d["dout"],
                               workspace=d["ws"], grads=d["grads"], scratch=scratch,
-                              stream=stream, **d["kw"])
+                              lse=d["lse"], stream=stream, **d["kw"])
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
@@ -947,6 +951,7 @@ def run_backward_arm(args, wl, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic",
         "config": {**workload_config(wl, world), "op": "backward",
+                   "lse": "from the forward" if sets[0]["lse"] is not None else "recomputed",
                    "l2": f"{nsets} rotating input sets, {nsets * per_set / 2**20:.0f} MiB > 2x L2",
                    "launch": "CUDA graph of C-ABI calls",
                    "useful_gflop_per_step": round(flops / 1e9, 4)},
@@ -1312,6 +1317,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-lse", action="store_true",
+                    help="--op backward: recompute the rows' log-sum-exp instead of taking it "
+                         "from the forward")
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="under torchrun: every rank runs the whole workload (replicas, weak "
                          "scaling) or the ranks split one problem by heads (strong scaling)")

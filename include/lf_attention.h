@@ -161,6 +161,25 @@ LF_API int lf_attention_forward(lf_dtype dtype, int B, int H, int n, int d_head,
                          lf_stream_t stream);
 
 /*
+ * lf_attention_forward for training (bf16 / fp16): also writes, for every
+ * valid non-global row, its log-sum-exp over its key set in log2 units,
+ *   lse[b, h, i] = log2( sum_j 2^(s_ij * log2(e) / sqrt(d_head)) ),
+ * where s_ij = <q_i, k_j> (the scores of the row's softmax).  The entries of
+ * padded rows and of global rows are left as they were.
+ *
+ *   lse          device fp32 [B, H, n], 4-byte aligned; NULL is refused.
+ * lf_attention_backward_lse reads it instead of recomputing it.  fp32 inputs
+ * return LF_ERR_UNSUPPORTED.  Other arguments and errors as lf_attention_forward.
+ */
+LF_API int lf_attention_forward_lse(lf_dtype dtype, int B, int H, int n, int d_head,
+                             const void *q, const void *k, const void *v,
+                             const void *qg, const void *kg, const void *vg,
+                             const uint8_t *local_mask, const uint8_t *global_mask,
+                             int max_global, int window, const int32_t *dilation, int causal,
+                             void *out, float *lse, void *workspace, size_t workspace_bytes,
+                             lf_stream_t stream);
+
+/*
  * The whole forward from HOST buffers: copies the six projections and the
  * masks from host memory (pinned memory makes the copies asynchronous) into
  * caller-provided device staging buffers, runs lf_attention_forward, copies
@@ -388,6 +407,25 @@ LF_API int lf_attention_backward(lf_dtype dtype, int B, int H, int n, int d_head
                          void *dq, void *dk, void *dv, void *dqg, void *dkg, void *dvg,
                          const void *workspace, size_t workspace_bytes,
                          void *scratch, size_t scratch_bytes, lf_stream_t stream);
+
+/*
+ * lf_attention_backward (bf16 / fp16) with the band rows' log-sum-exp taken
+ * from lf_attention_forward_lse on the same inputs, instead of a first pass
+ * over the keys that recomputes it.
+ *
+ *   lse          device fp32 [B, H, n] as lf_attention_forward_lse wrote it
+ *                for these inputs, 4-byte aligned; NULL is refused.
+ * fp32 inputs return LF_ERR_UNSUPPORTED.  Other arguments and errors as
+ * lf_attention_backward (the CUDA-core fallback recomputes the values).
+ */
+LF_API int lf_attention_backward_lse(lf_dtype dtype, int B, int H, int n, int d_head,
+                              const void *q, const void *k, const void *v,
+                              const void *qg, const void *kg, const void *vg,
+                              const void *out, const void *dout, const float *lse,
+                              int max_global, int window, const int32_t *dilation, int causal,
+                              void *dq, void *dk, void *dv, void *dqg, void *dkg, void *dvg,
+                              const void *workspace, size_t workspace_bytes, void *scratch,
+                              size_t scratch_bytes, lf_stream_t stream);
 
 /*
  * Feed-forward block of an encoder layer (FasterTransformer Longformer

@@ -85,6 +85,10 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         "lf_backward_scratch_size": (Z, [I, I, I, I, I]),
         "lf_attention_backward": (I, [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P, I, P, P, P,
                                       P, P, P, P, Z, P, Z, P]),
+        "lf_attention_forward_lse": (I, [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P, I, P, P,
+                                         P, Z, P]),
+        "lf_attention_backward_lse": (I, [I, I, I, I, I, P, P, P, P, P, P, P, P, P, I, I, P, I, P,
+                                          P, P, P, P, P, P, Z, P, Z, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -133,11 +133,13 @@ def attention_run(q, k, v, qg, kg, vg, *, window, dilation=None, causal=False, m
 
 def attention_forward(q, k, v, qg, kg, vg, local_mask=None, global_mask=None, *, window,
                       dilation=None, causal=False, max_global=None, out=None, workspace=None,
-                      stream=None):
+                      lse=None, stream=None):
     """Longformer attention forward; returns out [B, H, n, 64] in the input dtype.
 
     max_global: host upper bound on the global tokens of any batch; when None
     it is read from global_mask (one device-to-host sync).
+    lse: optional fp32 [B, H, n] tensor (bf16 / fp16 only): receives each
+    valid non-global row's log-sum-exp (log2 units) for attention_backward.
     """
     dt, (B, H, n, _) = _check_projections([q, k, v, qg, kg, vg])
     lm = _mask(local_mask, B, n, "local_mask")
@@ -150,12 +152,26 @@ def attention_forward(q, k, v, qg, kg, vg, local_mask=None, global_mask=None, *,
         out = torch.empty_like(q)
     _check_projections([q, out])
     _dev(workspace, "workspace")
+    if lse is not None:
+        _check_lse(lse, B, H, n, q.device)
+        _lib.check(_lib.lib().lf_attention_forward_lse(
+            dt, B, H, n, D_HEAD, _ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg), _ptr(vg),
+            _ptr(lm), _ptr(gm), int(max_global), int(window), _dilation(dilation, H),
+            int(bool(causal)), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+            _stream_ptr(stream)), "lf_attention_forward_lse")
+        return out
     _lib.check(_lib.lib().lf_attention_forward(
         dt, B, H, n, D_HEAD, _ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg), _ptr(vg), _ptr(lm),
         _ptr(gm), int(max_global), int(window), _dilation(dilation, H), int(bool(causal)),
         _ptr(out), _ptr(workspace), workspace.numel(), _stream_ptr(stream)),
         "lf_attention_forward")
     return out
+
+
+def _check_lse(lse, B, H, n, device):
+    if (not isinstance(lse, torch.Tensor) or lse.dtype != torch.float32
+            or tuple(lse.shape) != (B, H, n) or not lse.is_contiguous() or lse.device != device):
+        raise ValueError("lse must be a contiguous fp32 [B, H, n] tensor on the inputs' device")
 
 
 def host_staging_size(dtype: torch.dtype, B: int, H: int, n: int) -> int:
@@ -308,13 +324,15 @@ def backward_scratch_size(B: int, H: int, n: int, max_global: int) -> int:
 
 
 def attention_backward(q, k, v, qg, kg, vg, out, dout, *, window, dilation=None, causal=False,
-                       max_global, workspace, grads=None, scratch=None, stream=None):
+                       max_global, workspace, grads=None, scratch=None, lse=None, stream=None):
     """``lf_attention_backward``: gradients of the attention with respect to
     q, k, v, qg, kg, vg given the forward output ``out`` and dLoss/dout.
 
     ``workspace`` is the forward's prepared workspace (same masks and
-    max_global).  Returns a dict of the six gradients (``grads`` may supply
-    them, keyed q, k, v, qg, kg, vg).
+    max_global).  ``lse``: the log-sum-exp attention_forward(lse=...) wrote
+    for these inputs (bf16 / fp16), read instead of recomputed.  Returns a
+    dict of the six gradients (``grads`` may supply them, keyed q, k, v, qg,
+    kg, vg).
     """
     dt, (B, H, n, _) = _check_projections([q, k, v, qg, kg, vg])
     _check_projections([q, out, dout])
@@ -327,6 +345,15 @@ def attention_backward(q, k, v, qg, kg, vg, out, dout, *, window, dilation=None,
                               device=q.device)
     _dev(workspace, "workspace")
     _dev(scratch, "scratch")
+    if lse is not None:
+        _check_lse(lse, B, H, n, q.device)
+        _lib.check(_lib.lib().lf_attention_backward_lse(
+            dt, B, H, n, D_HEAD, _ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg), _ptr(vg),
+            _ptr(out), _ptr(dout), _ptr(lse), int(max_global), int(window),
+            _dilation(dilation, H), int(bool(causal)), *[_ptr(grads[nm]) for nm in names],
+            _ptr(workspace), workspace.numel(), _ptr(scratch), scratch.numel(),
+            _stream_ptr(stream)), "lf_attention_backward_lse")
+        return grads
     _lib.check(_lib.lib().lf_attention_backward(
         dt, B, H, n, D_HEAD, _ptr(q), _ptr(k), _ptr(v), _ptr(qg), _ptr(kg), _ptr(vg), _ptr(out),
         _ptr(dout), int(max_global), int(window), _dilation(dilation, H), int(bool(causal)),

@@ -178,17 +178,20 @@ int lf_attention_prepare(int B, int H, int n, int d_head, const uint8_t *local_m
                           static_cast<cudaStream_t>(stream));
 }
 
-int lf_attention_run(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
-                     const void *k, const void *v, const void *qg, const void *kg, const void *vg,
-                     int max_global, int window, const int32_t *dilation, int causal, void *out,
-                     void *workspace, size_t workspace_bytes, lf_stream_t stream)
+namespace {
+int attention_run(lf_dtype dtype, int B, int H, int n, int d_head, const void *q, const void *k,
+                  const void *v, const void *qg, const void *kg, const void *vg, int max_global,
+                  int window, const int32_t *dilation, int causal, void *out, void *workspace,
+                  size_t workspace_bytes, float *lse, lf_stream_t stream)
 {
     AttnArgs a;
     if (int rc = make_args(dtype, B, H, n, d_head, q, k, v, qg, kg, vg, max_global, window,
                            dilation, causal, workspace, workspace_bytes, {out}, a))
         return rc;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LF_ERR_INVALID_ARG;
     if (int rc = device_ok()) return rc;
     a.out = out;
+    a.lse_out = lse;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (dtype) {
         case LF_F32: return launch_f32(a, s);
@@ -198,11 +201,11 @@ int lf_attention_run(lf_dtype dtype, int B, int H, int n, int d_head, const void
     return LF_ERR_INVALID_ARG;
 }
 
-int lf_attention_forward(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
-                         const void *k, const void *v, const void *qg, const void *kg,
-                         const void *vg, const uint8_t *local_mask, const uint8_t *global_mask,
-                         int max_global, int window, const int32_t *dilation, int causal,
-                         void *out, void *workspace, size_t workspace_bytes, lf_stream_t stream)
+int attention_forward(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
+                      const void *k, const void *v, const void *qg, const void *kg,
+                      const void *vg, const uint8_t *local_mask, const uint8_t *global_mask,
+                      int max_global, int window, const int32_t *dilation, int causal, void *out,
+                      void *workspace, size_t workspace_bytes, float *lse, lf_stream_t stream)
 {
     // Argument checks of the run come first so nothing is launched on error.
     if (d_head != kDHead) return LF_ERR_UNSUPPORTED;
@@ -210,8 +213,43 @@ int lf_attention_forward(lf_dtype dtype, int B, int H, int n, int d_head, const 
     int rc = lf_attention_prepare(B, H, n, d_head, local_mask, global_mask, max_global,
                                   workspace, workspace_bytes, stream);
     if (rc != LF_OK) return rc;
-    return lf_attention_run(dtype, B, H, n, d_head, q, k, v, qg, kg, vg, max_global, window,
-                            dilation, causal, out, workspace, workspace_bytes, stream);
+    return attention_run(dtype, B, H, n, d_head, q, k, v, qg, kg, vg, max_global, window,
+                         dilation, causal, out, workspace, workspace_bytes, lse, stream);
+}
+}  // namespace
+
+int lf_attention_run(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
+                     const void *k, const void *v, const void *qg, const void *kg, const void *vg,
+                     int max_global, int window, const int32_t *dilation, int causal, void *out,
+                     void *workspace, size_t workspace_bytes, lf_stream_t stream)
+{
+    return attention_run(dtype, B, H, n, d_head, q, k, v, qg, kg, vg, max_global, window,
+                         dilation, causal, out, workspace, workspace_bytes, nullptr, stream);
+}
+
+int lf_attention_forward(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
+                         const void *k, const void *v, const void *qg, const void *kg,
+                         const void *vg, const uint8_t *local_mask, const uint8_t *global_mask,
+                         int max_global, int window, const int32_t *dilation, int causal,
+                         void *out, void *workspace, size_t workspace_bytes, lf_stream_t stream)
+{
+    return attention_forward(dtype, B, H, n, d_head, q, k, v, qg, kg, vg, local_mask,
+                             global_mask, max_global, window, dilation, causal, out, workspace,
+                             workspace_bytes, nullptr, stream);
+}
+
+int lf_attention_forward_lse(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
+                             const void *k, const void *v, const void *qg, const void *kg,
+                             const void *vg, const uint8_t *local_mask,
+                             const uint8_t *global_mask, int max_global, int window,
+                             const int32_t *dilation, int causal, void *out, float *lse,
+                             void *workspace, size_t workspace_bytes, lf_stream_t stream)
+{
+    if (!lse) return LF_ERR_INVALID_ARG;
+    if (dtype != LF_BF16 && dtype != LF_F16) return LF_ERR_UNSUPPORTED;
+    return attention_forward(dtype, B, H, n, d_head, q, k, v, qg, kg, vg, local_mask,
+                             global_mask, max_global, window, dilation, causal, out, workspace,
+                             workspace_bytes, lse, stream);
 }
 
 size_t lf_host_staging_size(lf_dtype dtype, int B, int H, int n, int d_head)
@@ -338,13 +376,14 @@ size_t lf_backward_scratch_size(int B, int H, int n, int d_head, int max_global)
     return backward_scratch_bytes(B, H, n, max_global);
 }
 
-int lf_attention_backward(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
-                          const void *k, const void *v, const void *qg, const void *kg,
-                          const void *vg, const void *out, const void *dout, int max_global,
-                          int window, const int32_t *dilation, int causal, void *dq, void *dk,
-                          void *dv, void *dqg, void *dkg, void *dvg, const void *workspace,
-                          size_t workspace_bytes, void *scratch, size_t scratch_bytes,
-                          lf_stream_t stream)
+namespace {
+int attention_backward(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
+                       const void *k, const void *v, const void *qg, const void *kg,
+                       const void *vg, const void *out, const void *dout, int max_global,
+                       int window, const int32_t *dilation, int causal, void *dq, void *dk,
+                       void *dv, void *dqg, void *dkg, void *dvg, const void *workspace,
+                       size_t workspace_bytes, void *scratch, size_t scratch_bytes,
+                       const float *lse, lf_stream_t stream)
 {
     BwdArgs A;
     if (int rc = make_args(dtype, B, H, n, d_head, q, k, v, qg, kg, vg, max_global, window,
@@ -355,10 +394,12 @@ int lf_attention_backward(lf_dtype dtype, int B, int H, int n, int d_head, const
     if (!scratch || scratch_bytes < need || reinterpret_cast<uintptr_t>(scratch) % 256)
         return LF_ERR_WORKSPACE;
     if (int rc = device_ok()) return rc;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LF_ERR_INVALID_ARG;
     A.out = out;
     A.dout = dout;
     A.dq = dq; A.dk = dk; A.dv = dv; A.dqg = dqg; A.dkg = dkg; A.dvg = dvg;
     backward_scratch_ptrs(A, scratch, B, H, n, max_global);
+    A.lse_in = lse;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (dtype) {
         case LF_F32: return launch_backward_simt<float>(A, 4, s);
@@ -371,6 +412,36 @@ int lf_attention_backward(lf_dtype dtype, int B, int H, int n, int d_head, const
         }
     }
     return LF_ERR_INVALID_ARG;
+}
+}  // namespace
+
+int lf_attention_backward(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
+                          const void *k, const void *v, const void *qg, const void *kg,
+                          const void *vg, const void *out, const void *dout, int max_global,
+                          int window, const int32_t *dilation, int causal, void *dq, void *dk,
+                          void *dv, void *dqg, void *dkg, void *dvg, const void *workspace,
+                          size_t workspace_bytes, void *scratch, size_t scratch_bytes,
+                          lf_stream_t stream)
+{
+    return attention_backward(dtype, B, H, n, d_head, q, k, v, qg, kg, vg, out, dout,
+                              max_global, window, dilation, causal, dq, dk, dv, dqg, dkg, dvg,
+                              workspace, workspace_bytes, scratch, scratch_bytes, nullptr, stream);
+}
+
+int lf_attention_backward_lse(lf_dtype dtype, int B, int H, int n, int d_head, const void *q,
+                              const void *k, const void *v, const void *qg, const void *kg,
+                              const void *vg, const void *out, const void *dout,
+                              const float *lse, int max_global, int window,
+                              const int32_t *dilation, int causal, void *dq, void *dk, void *dv,
+                              void *dqg, void *dkg, void *dvg, const void *workspace,
+                              size_t workspace_bytes, void *scratch, size_t scratch_bytes,
+                              lf_stream_t stream)
+{
+    if (!lse) return LF_ERR_INVALID_ARG;
+    if (dtype != LF_BF16 && dtype != LF_F16) return LF_ERR_UNSUPPORTED;
+    return attention_backward(dtype, B, H, n, d_head, q, k, v, qg, kg, vg, out, dout,
+                              max_global, window, dilation, causal, dq, dk, dv, dqg, dkg, dvg,
+                              workspace, workspace_bytes, scratch, scratch_bytes, lse, stream);
 }
 
 size_t lf_ffn_workspace_size(int B, int n, int hidden, int inter)

@@ -13,6 +13,7 @@ struct BwdArgs {
     const void *out, *dout;     // forward output O and its gradient dO
     void *dq, *dk, *dv, *dqg, *dkg, *dvg;
     float *lse, *dsum;          // [B*H*n] per band row: log2-domain lse, D
+    const float *lse_in;        // optional: the forward's lse of the band rows
     float *lse_g, *dsum_g;      // [B*H*max_global] per global slot
     // Global tokens as keys of the rows that do not reach them through the
     // window: [B*H*max_global][dk (64, unscaled) | dv (64)] fp32 sums.

@@ -204,7 +204,10 @@ __device__ __forceinline__ void producer_role(const Params &p, Smem &sm, const I
                         it.s0 + hf * kN, it.bh);
         }
     }
-    const int total = (kKeys ? 1 : 2) * it.ntiles;
+    // The rows side streams the tiles twice unless the forward's log-sum-exp
+    // of the rows is given (pass 1 only).
+    const bool one_pass = kKeys || p.A.lse_in != nullptr;
+    const int total = (one_pass ? 1 : 2) * it.ntiles;
     bool armed[kStages] = {};
     uint32_t armed_ph[kStages] = {};
     bool ok = true;
@@ -215,7 +218,7 @@ __device__ __forceinline__ void producer_role(const Params &p, Smem &sm, const I
             ok = false;
             break;
         }
-        const int pass = u / it.ntiles, t = u - pass * it.ntiles;
+        const int pass = one_pass ? 1 : u / it.ntiles, t = one_pass ? u : u - it.ntiles * pass;
         const bool need_b2 = kKeys || pass == 1;
         const uint32_t bytes = kTileBytes * (need_b2 ? 2u : 1u);
         if (t < it.nband) {
@@ -264,12 +267,13 @@ __device__ __forceinline__ void mma_role(const Params &p, Smem &sm, const Item &
     tc_fence_after();
     const uint64_t a1d = make_sdesc(smem_u32(sm.a1), 16, 1024);
     const uint64_t a2d = make_sdesc(smem_u32(sm.a2), 16, 1024);
-    const int total = (kKeys ? 1 : 2) * it.ntiles;
+    const bool one_pass = kKeys || p.A.lse_in != nullptr;
+    const int total = (one_pass ? 1 : 2) * it.ntiles;
     bool first_acc = true;
     for (int u = 0; u < total; ++u) {
         const int st = u % kStages;
         const uint32_t ph = uint32_t(u / kStages) & 1u;
-        const bool grad = kKeys || u >= it.ntiles;
+        const bool grad = one_pass || u >= it.ntiles;
         if (!warp_wait(&sm.full[st], ph, &sm.abort_flag, a.ws.status)) return;
         tc_fence_after();
         const uint64_t b1d = make_sdesc(smem_u32(sm.b1[st]), 16, 1024);
@@ -375,9 +379,11 @@ __device__ __forceinline__ void rows_softmax(const Params &p, Smem &sm, const It
     const int tlo = row - (a.causal ? a.window - 1 : a.half);
     const int thi = row + (a.causal ? 0 : a.half);
     float m = -INFINITY, l = 0.f, lse = INFINITY;
+    const bool one_pass = A.lse_in != nullptr;
+    if (one_pass && active) lse = A.lse_in[size_t(it.bh) * n + i];
 
-    for (int u = 0; u < 2 * it.ntiles; ++u) {
-        const int pass = u / it.ntiles, t = u - pass * it.ntiles;
+    for (int u = 0; u < (one_pass ? 1 : 2) * it.ntiles; ++u) {
+        const int pass = one_pass ? 1 : u / it.ntiles, t = one_pass ? u : u - it.ntiles * pass;
         uint32_t mw[2];
         rows_mask(a, it, t, lane, i, active, tlo, thi, mw);
         if (!warp_wait(&sm.s_full, uint32_t(u) & 1u, &sm.abort_flag, a.ws.status)) return;

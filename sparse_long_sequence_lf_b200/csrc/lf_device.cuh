@@ -104,6 +104,7 @@ __host__ __device__ inline WsPtrs ws_ptrs(void *ws, const WsLayout &L)
 struct AttnArgs {
     const void *q, *k, *v, *qg, *kg, *vg;
     void *out;
+    float *lse_out;   // optional [B*H*n]: log-sum-exp (log2 units) of the band rows
     WsPtrs ws;
     WsLayout L;
     int B, H, n;

@@ -1006,6 +1006,8 @@ __device__ __forceinline__ void epilogue(const FwdParams &p, FwdSmem &sm, uint32
             const int pos = write ? row * I.dil + I.r : 0;
             T *dst = static_cast<T *>(a.out) + (size_t(bh) * a.n + pos) * kDHead;
             const float inv = ro.valid() ? __frcp_rn(ro.l) : 0.f;
+            if (a.lse_out && write && ro.valid())
+                a.lse_out[size_t(bh) * a.n + pos] = ro.m + log2f(ro.l);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float o[32];

@@ -150,3 +150,68 @@ def test_backward_full_size_sampled_heads(name):
             worst = np.unravel_index(int(np.argmax(excess)), excess.shape)
             assert excess.max() <= tol, (f"{name} head {h} d{nm}: err "
                                          f"{abs(got[worst] - want[worst]):.3e} at {worst}")
+
+
+# ------------------------------------------------- log-sum-exp from the forward
+LSE_CASES = [c for c in CASES if c.dtype != "f32" and c.name != "n1"] + [
+    Workload("lse-dil-causal", "bf16", 1, 3, 700, 48, dilation=(1, 2, 3), causal=True, seed=15),
+]
+
+
+def _lse_want(x, wl):
+    """log2 of each valid non-global row's softmax denominator, from the
+    oracle's key sets (fp64): log2 sum_j exp(<q_i, k_j> / 8)."""
+    local, _ = obw.key_masks(x["local_mask"], x["global_mask"], B=wl.B, H=wl.H, n=wl.n,
+                             window=wl.window, dilation=x["dilation"], causal=wl.causal)
+    q = x["q"].double()
+    k = x["k"].double()
+    s = torch.einsum("bhid,bhjd->bhij", q, k) / 8.0
+    m = torch.from_numpy(local)
+    s = s.masked_fill(~m, float("-inf"))
+    rows = m.any(dim=-1)
+    return (torch.logsumexp(s, dim=-1) / np.log(2.0)).numpy(), rows.numpy()
+
+
+@pytest.mark.parametrize("wl", LSE_CASES, ids=[w.name for w in LSE_CASES])
+def test_backward_with_forward_lse(wl):
+    # The forward writes each valid non-global row's log-sum-exp (log2 units);
+    # the backward given it skips its first pass.  Both against fp64.
+    x = make_inputs(wl)
+    dout = make_output_grad(wl)
+    g = to_dev(x)
+    mg = max_global_of(x)
+    ws = lf.new_workspace(wl.B, wl.H, wl.n, mg, "cuda")
+    kw = dict(window=wl.window, dilation=x["dilation"], causal=wl.causal, max_global=mg)
+    lse = torch.full((wl.B, wl.H, wl.n), float("nan"), dtype=torch.float32, device="cuda")
+    out = lf.attention_forward(g["q"], g["k"], g["v"], g["qg"], g["kg"], g["vg"],
+                               g["local_mask"], g["global_mask"], workspace=ws, lse=lse, **kw)
+    grads = lf.attention_backward(g["q"], g["k"], g["v"], g["qg"], g["kg"], g["vg"], out,
+                                  dout.cuda(), workspace=ws, lse=lse, **kw)
+    torch.cuda.synchronize()
+    assert lf.workspace_status(ws) == 0
+    want, rows = _lse_want(x, wl)
+    got = lse.cpu().numpy().astype(np.float64)
+    isg = (np.zeros((wl.B, wl.n), bool) if x["global_mask"] is None
+           else x["global_mask"].numpy().astype(bool))
+    band = rows & ~isg[:, None, :]
+    # The forward's sum uses its 2^x (relative error below 7.5e-5).
+    assert np.all(np.abs(got[band] - want[band]) <= 1e-3), wl.name
+    ref = obw.backward(x["q"], x["k"], x["v"], x["qg"], x["kg"], x["vg"], x["local_mask"],
+                       x["global_mask"], dout, window=wl.window, dilation=x["dilation"],
+                       causal=wl.causal)
+    tol = TOL[wl.dtype]
+    for nm in NAMES:
+        got_g = grads[nm].float().cpu().numpy().astype(np.float64)
+        err = np.abs(got_g - ref[nm]) - tol * np.abs(ref[nm])
+        assert err.max() <= tol, f"{wl.name} d{nm}: {err.max():.3e}"
+
+
+def test_lse_entry_points_refuse_fp32_and_null():
+    from sparse_long_sequence_lf_b200 import _lib
+    L = _lib.lib()
+    rc = L.lf_attention_forward_lse(_lib.LF_F32, 1, 1, 64, 64, *([None] * 8), 0, 8, None, 0,
+                                    None, None, None, 0, None)
+    assert rc in (-1, -2)
+    rc = L.lf_attention_backward_lse(_lib.LF_BF16, 1, 1, 64, 64, *([None] * 9), 0, 8, None, 0,
+                                     *([None] * 6), None, 0, None, 0, None)
+    assert rc == -1
