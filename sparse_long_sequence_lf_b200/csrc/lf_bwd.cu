@@ -385,6 +385,16 @@ __device__ __forceinline__ SlotGroups slot_groups(int gv, int rl)
     return q;
 }
 
+// Sums v over the quads of this warp that share its slot (quads whose index
+// differs by a multiple of G2); afterwards every such quad holds the warp's
+// sum, and only the first of them (lane / 4 < G2) adds it to shared memory,
+// so a shared sum takes one atomic add per warp instead of one per quad.
+__device__ __forceinline__ float warp_slot_sum(float v, int G2)
+{
+    for (int off = 4 * G2; off < 32; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
 // ------------------------------------------------- global tokens as keys
 // Contributions of the rows that reach a global token only as a global key
 // (valid non-global rows that are not its window taps): one CTA per
@@ -467,7 +477,12 @@ __global__ void __launch_bounds__(kThreads) gcols_kernel(const BwdArgs A)
         }
     }
     // Groups of the same slot meet in shared memory; one global add per value.
-    if (kvalid) {
+#pragma unroll
+    for (int x = 0; x < kQ; ++x) {
+        dk[x] = warp_slot_sum(dk[x], sg.G2);
+        dv[x] = warp_slot_sum(dv[x], sg.G2);
+    }
+    if (kvalid && ((tid & 31) >> 2) < sg.G2) {
 #pragma unroll
         for (int x = 0; x < kQ; ++x) {
             atomicAdd(&red[sg.sl][kQ * qd + x], dk[x]);
@@ -610,7 +625,9 @@ __global__ void __launch_bounds__(kThreads) grows_chunk_kernel(const BwdArgs A)
         A.lse_g[size_t(bh) * mg + slot] = lse;
         A.dsum_g[size_t(bh) * mg + slot] = D;
     }
-    if (active) {
+#pragma unroll
+    for (int x = 0; x < kQ; ++x) dq[x] = warp_slot_sum(dq[x], sg.G2);
+    if (active && ((tid & 31) >> 2) < sg.G2) {
 #pragma unroll
         for (int x = 0; x < kQ; ++x) atomicAdd(&red[sg.sl][kQ * qd + x], dq[x]);
     }
