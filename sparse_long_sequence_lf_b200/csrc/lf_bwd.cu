@@ -23,7 +23,8 @@
 //                  token) the sums gcols_kernel left in the scratch.
 //   gcols_kernel   a global token as the key of the valid non-global rows that
 //                  do not reach it through the window: chunks of 128 rows,
-//                  fp32 atomic sums per slot.
+//                  fp32 atomic sums per slot (gcols_small_kernel: the same
+//                  for at most 8 tokens, one warp per row, streamed).
 //   grows_chunk_kernel  global rows (Qg) against 128-key chunks of Kg, Vg:
 //                  pass 1 the chunk's (max, sum), pass 2 the merged
 //                  log-sum-exp and the chunk's dqg terms (fp32 atomics);
@@ -497,6 +498,130 @@ __global__ void __launch_bounds__(kThreads) gcols_kernel(const BwdArgs A)
     }
 }
 
+// The same sums for at most G global tokens (G = 1, 2, 4 or 8: the loops
+// over tokens and rows are unrolled, so the code grows with G), streamed:
+// one warp per row at a time, lane l holding dimensions 2l and 2l+1, the
+// tokens' K and V rows and their dk, dv sums in registers; a warp takes
+// kColRowsPerWarp rows, col_batch(G) at a time with all their loads (which
+// do not depend on one another) issued first.  The warps of a CTA add their
+// sums in shared memory, then once to A.gkv.
+constexpr int kSmallG = 8;
+constexpr int kColWarps = 8;
+constexpr int kColRowsPerWarp = 16;
+__host__ __device__ constexpr int col_batch(int) { return 4; }
+constexpr int kColRows = kColWarps * kColRowsPerWarp;   // rows per CTA
+
+template <typename T> __device__ __forceinline__ float2 load2(const T *p);
+template <> __device__ __forceinline__ float2 load2<float>(const float *p)
+{
+    return *reinterpret_cast<const float2 *>(p);
+}
+template <> __device__ __forceinline__ float2 load2<__half>(const __half *p)
+{
+    return __half22float2(*reinterpret_cast<const __half2 *>(p));
+}
+template <> __device__ __forceinline__ float2 load2<__nv_bfloat16>(const __nv_bfloat16 *p)
+{
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+}
+
+__device__ __forceinline__ float warp_sum(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+template <typename T, int G>
+__global__ void __launch_bounds__(32 * kColWarps) gcols_small_kernel(const BwdArgs A)
+{
+    const AttnArgs &a = A.a;
+    __shared__ __align__(16) float red[kColWarps][G][2 * kDHead];
+    const int n = a.n;
+    const int rchunks = (n + kColRows - 1) / kColRows;
+    const int bh = blockIdx.x / rchunks;
+    const int i0 = (blockIdx.x % rchunks) * kColRows;
+    const int b = bh / a.H, h = bh - b * a.H;
+    const int g = min(a.ws.counts[b], min(a.max_global, G));
+    if (g == 0) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
+    const uint32_t *gb = a.ws.gbits + size_t(b) * a.L.nwords;
+    const int dil = a.dil[h];
+    const size_t base = size_t(bh) * n * kDHead + 2 * lane;
+    const T *Q = static_cast<const T *>(a.q) + base;
+    const T *dO = static_cast<const T *>(A.dout) + base;
+    const float *lse = A.lse + size_t(bh) * n;
+    const float *dsum = A.dsum + size_t(bh) * n;
+
+    int js[G];
+    float2 kk[G], vv[G], dk[G], dv[G];
+#pragma unroll
+    for (int s = 0; s < G; ++s) {
+        js[s] = -1;
+        kk[s] = vv[s] = dk[s] = dv[s] = make_float2(0.f, 0.f);
+        if (s < g) {
+            const int j = a.ws.gidx[size_t(b) * n + s];
+            if (bit_at(vb, j)) {
+                js[s] = j;
+                const float2 kf = load2(static_cast<const T *>(a.k) + base + size_t(j) * kDHead);
+                kk[s] = make_float2(kf.x * a.scale_log2, kf.y * a.scale_log2);
+                vv[s] = load2(static_cast<const T *>(a.v) + base + size_t(j) * kDHead);
+            }
+        }
+    }
+    constexpr int kB = col_batch(G);
+    const int r0 = i0 + warp * kColRowsPerWarp;
+#pragma unroll 1
+    for (int rb = r0; rb < min(r0 + kColRowsPerWarp, n); rb += kB) {
+        float2 qv[kB], ov[kB];
+        float lv[kB], dvv[kB];
+        uint32_t vw[kB], gw[kB];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+            const int ii = min(rb + u, n - 1);
+            vw[u] = vb[ii >> 5];
+            gw[u] = gb[ii >> 5];
+            qv[u] = load2(Q + size_t(ii) * kDHead);
+            ov[u] = load2(dO + size_t(ii) * kDHead);
+            lv[u] = lse[ii];
+            dvv[u] = dsum[ii];
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+            const int i = rb + u;
+            if (i >= n || !((vw[u] >> (i & 31)) & 1u) || ((gw[u] >> (i & 31)) & 1u)) continue;
+#pragma unroll
+            for (int s = 0; s < G; ++s) {
+                if (s >= g || js[s] < 0 || is_tap(i, js[s], a.window, a.half, dil, a.causal)) continue;
+                const float sc = warp_sum(fmaf(qv[u].x, kk[s].x, qv[u].y * kk[s].y));
+                const float dp = warp_sum(fmaf(ov[u].x, vv[s].x, ov[u].y * vv[s].y));
+                const float pr = exp2f(sc - lv[u]);
+                const float ds = pr * (dp - dvv[u]);
+                dv[s].x = fmaf(pr, ov[u].x, dv[s].x);
+                dv[s].y = fmaf(pr, ov[u].y, dv[s].y);
+                dk[s].x = fmaf(ds, qv[u].x, dk[s].x);
+                dk[s].y = fmaf(ds, qv[u].y, dk[s].y);
+            }
+        }
+    }
+#pragma unroll
+    for (int s = 0; s < G; ++s) {
+        if (s >= g) break;
+        *reinterpret_cast<float2 *>(&red[warp][s][2 * lane]) = dk[s];
+        *reinterpret_cast<float2 *>(&red[warp][s][kDHead + 2 * lane]) = dv[s];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < g * 2 * kDHead; e += 32 * kColWarps) {
+        const int s = e / (2 * kDHead), x = e - s * (2 * kDHead);
+        if (!bit_at(vb, a.ws.gidx[size_t(b) * n + s])) continue;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kColWarps; ++w) acc += red[w][s][x];
+        atomicAdd(A.gkv + (size_t(bh) * a.max_global + s) * (2 * kDHead) + x, acc);
+    }
+}
+
 // ------------------------------------------------------------ global rows
 // Global rows against every valid key through Qg, Kg, Vg, split into chunks
 // of kGChunk keys: gstats_kernel writes each chunk's (max, sum) of the row's
@@ -776,7 +901,17 @@ int launch_global_cols(const BwdArgs &A, cudaStream_t stream)
     const size_t mg = size_t(a.max_global);
     if (cudaMemsetAsync(A.gkv, 0, sizeof(float) * bh * mg * 2 * kDHead, stream) != cudaSuccess)
         return kErrCuda;
-    gcols_kernel<T><<<bh * sparts * ((a.n + kGChunk - 1) / kGChunk), kThreads, 0, stream>>>(A);
+    const int cgrid = bh * ((a.n + kColRows - 1) / kColRows);
+    if (a.max_global <= 1)
+        gcols_small_kernel<T, 1><<<cgrid, 32 * kColWarps, 0, stream>>>(A);
+    else if (a.max_global <= 2)
+        gcols_small_kernel<T, 2><<<cgrid, 32 * kColWarps, 0, stream>>>(A);
+    else if (a.max_global <= 4)
+        gcols_small_kernel<T, 4><<<cgrid, 32 * kColWarps, 0, stream>>>(A);
+    else if (a.max_global <= kSmallG)
+        gcols_small_kernel<T, kSmallG><<<cgrid, 32 * kColWarps, 0, stream>>>(A);
+    else
+        gcols_kernel<T><<<bh * sparts * ((a.n + kGChunk - 1) / kGChunk), kThreads, 0, stream>>>(A);
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 

@@ -46,6 +46,12 @@ CASES = [
     # maps: the whole call takes the CUDA-core kernels
     Workload("residue-budget", "bf16", 1, 4, 300, 8, dilation=(7, 8, 9, 10),
              globals_kind="random:3", seed=14),
+    # At most 8 global tokens: the streamed global-column sums (8 exactly,
+    # dilations, padding; and the fp32 path with 3)
+    Workload("g8-dilated", "f16", 1, 3, 777, 40, dilation=(1, 2, 3), globals_kind="random:8",
+             pad_tail=(33,), seed=21),
+    Workload("fp32-g3", "f32", 1, 2, 400, 24, dilation=(1, 2), globals_kind="random:3",
+             seed=22),
 ]
 
 

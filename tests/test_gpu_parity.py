@@ -60,6 +60,11 @@ EDGE = [
              pad_tail=(0, 41), seed=10),
     Workload("fp32-causal", "f32", 1, 2, 513, 33, dilation=(1, 3), causal=True, seed=11),
     Workload("fp16-w2", "f16", 1, 2, 257, 2, globals_kind="first:3", seed=12),
+    # Global tokens in the free columns of the last window tile: from column 32
+    # (window 80: the last tile holds 16 keys), 60 tokens over two chunks,
+    # with dilations and padding; the edge items keep tiles of their own.
+    Workload("globals-share-last-tile", "bf16", 1, 3, 1000, 80, dilation=(1, 2, 3),
+             globals_kind="random:60", pad_tail=(50,), seed=17),
     # global rows merged by the last chunk (8 chunks of 512 keys) ...
     Workload("merge-8-chunks", "bf16", 1, 2, 4096, 16, globals_kind="random:40",
              pad_tail=(5,), seed=13),
