@@ -622,6 +622,45 @@ __global__ void __launch_bounds__(32 * kColWarps) gcols_small_kernel(const BwdAr
     }
 }
 
+// ------------------------------------------------------------ row statistics
+// lse and D = <dO_i, O_i> of every position i of every (batch, head) as the
+// band kernels leave them: the forward's lse and D for a valid non-global
+// row, +inf and 0 otherwise.  Eight threads per row, eight dimensions each.
+template <typename T>
+__global__ void __launch_bounds__(256) row_stats_kernel(const BwdArgs A)
+{
+    const AttnArgs &a = A.a;
+    const size_t rows = size_t(a.B) * a.H * a.n;
+    const size_t r = size_t(blockIdx.x) * 32 + (threadIdx.x >> 3);
+    const int part = threadIdx.x & 7;
+    if (r >= rows) return;      // whole groups of 8 lanes leave together
+    const int i = int(r % size_t(a.n));
+    const int b = int(r / (size_t(a.n) * a.H));
+    const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
+    const uint32_t *gb = a.ws.gbits + size_t(b) * a.L.nwords;
+    const bool active = bit_at(vb, i) && !bit_at(gb, i);
+    const float4 o0 = load4(static_cast<const T *>(A.out) + r * kDHead + 8 * part);
+    const float4 o1 = load4(static_cast<const T *>(A.out) + r * kDHead + 8 * part + 4);
+    const float4 d0 = load4(static_cast<const T *>(A.dout) + r * kDHead + 8 * part);
+    const float4 d1 = load4(static_cast<const T *>(A.dout) + r * kDHead + 8 * part + 4);
+    float s = d0.x * o0.x;
+    s = fmaf(d0.y, o0.y, s);
+    s = fmaf(d0.z, o0.z, s);
+    s = fmaf(d0.w, o0.w, s);
+    s = fmaf(d1.x, o1.x, s);
+    s = fmaf(d1.y, o1.y, s);
+    s = fmaf(d1.z, o1.z, s);
+    s = fmaf(d1.w, o1.w, s);
+    const unsigned grp = 0xffu << (threadIdx.x & 24);
+    s += __shfl_xor_sync(grp, s, 1);
+    s += __shfl_xor_sync(grp, s, 2);
+    s += __shfl_xor_sync(grp, s, 4);
+    if (part == 0) {
+        A.lse[r] = active ? A.lse_in[r] : INFINITY;
+        A.dsum[r] = active ? s : 0.f;
+    }
+}
+
 // ------------------------------------------------------------ global rows
 // Global rows against every valid key through Qg, Kg, Vg, split into chunks
 // of kGChunk keys: gstats_kernel writes each chunk's (max, sum) of the row's
@@ -862,6 +901,15 @@ __global__ void __launch_bounds__(kThreads) gkeys_kernel(const BwdArgs A)
 
 }  // namespace bwd
 
+template <typename T>
+int launch_row_stats(const BwdArgs &A, cudaStream_t stream)
+{
+    const size_t rows = size_t(A.a.B) * A.a.H * A.a.n;
+    if (rows == 0) return kOk;
+    bwd::row_stats_kernel<T><<<unsigned((rows + 31) / 32), 256, 0, stream>>>(A);
+    return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+}
+
 // Global rows (Qg against Kg, Vg) and the Kg/Vg keys: needs only the inputs
 // and the prepared workspace, so it runs beside the band rows.
 template <typename T>
@@ -927,8 +975,11 @@ std::unique_lock<std::mutex> side_stream(SideStream *&out)
     if (!made[dev]) {
         SideStream &s = side[dev];
         if (cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&s.stream2, cudaStreamNonBlocking) != cudaSuccess ||
             cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess)
+            cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&s.fork2, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&s.join2, cudaEventDisableTiming) != cudaSuccess)
             return lock;
         made[dev] = true;
     }
@@ -943,14 +994,15 @@ int launch_backward_simt(const BwdArgs &A, size_t elem, cudaStream_t stream)
     const int band_ctas = A.a.B * A.a.band_items_per_batch * kParts;
     return backward_schedule<T>(
         A, elem, stream,
-        [&]() {
-            if (band_ctas > 0) rows_kernel<T><<<band_ctas, kThreads, 0, stream>>>(A);
+        [&](cudaStream_t st) {
+            if (band_ctas > 0) rows_kernel<T><<<band_ctas, kThreads, 0, st>>>(A);
             return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
         },
-        [&]() {
-            if (band_ctas > 0) keys_kernel<T><<<band_ctas, kThreads, 0, stream>>>(A);
+        [&](cudaStream_t st) {
+            if (band_ctas > 0) keys_kernel<T><<<band_ctas, kThreads, 0, st>>>(A);
             return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
-        });
+        },
+        false);
 }
 
 template int launch_global_rows<__half>(const BwdArgs &, size_t, cudaStream_t);
@@ -959,6 +1011,8 @@ template int launch_global_rows<float>(const BwdArgs &, size_t, cudaStream_t);
 template int launch_global_cols<__half>(const BwdArgs &, cudaStream_t);
 template int launch_global_cols<__nv_bfloat16>(const BwdArgs &, cudaStream_t);
 template int launch_global_cols<float>(const BwdArgs &, cudaStream_t);
+template int launch_row_stats<__half>(const BwdArgs &, cudaStream_t);
+template int launch_row_stats<__nv_bfloat16>(const BwdArgs &, cudaStream_t);
 template int launch_backward_simt<float>(const BwdArgs &, size_t, cudaStream_t);
 template int launch_backward_simt<__half>(const BwdArgs &, size_t, cudaStream_t);
 template int launch_backward_simt<__nv_bfloat16>(const BwdArgs &, size_t, cudaStream_t);

@@ -66,13 +66,16 @@ template <typename T> int launch_backward_simt(const BwdArgs &A, size_t elem, cu
 // keys).
 template <typename T> int launch_global_rows(const BwdArgs &A, size_t elem, cudaStream_t stream);
 template <typename T> int launch_global_cols(const BwdArgs &A, cudaStream_t stream);
+// lse (from A.lse_in) and D of every band row into A.lse and A.dsum, for the
+// schedule in which the band rows and keys run side by side.
+template <typename T> int launch_row_stats(const BwdArgs &A, cudaStream_t stream);
 
 // A second stream of the current device, with the events that fork work onto
 // it and join it back; the returned lock serialises its use across host
 // threads (out = nullptr when it cannot be created).
 struct SideStream {
-    cudaStream_t stream;
-    cudaEvent_t fork, join;
+    cudaStream_t stream, stream2;
+    cudaEvent_t fork, join, fork2, join2;
 };
 std::unique_lock<std::mutex> side_stream(SideStream *&out);
 
@@ -81,7 +84,7 @@ std::unique_lock<std::mutex> side_stream(SideStream *&out);
 // under stream capture (the side stream joins and leaves with the events).
 template <typename T, typename RowsFn, typename KeysFn>
 int backward_schedule(const BwdArgs &A, size_t elem, cudaStream_t stream, RowsFn &&band_rows,
-                      KeysFn &&band_keys)
+                      KeysFn &&band_keys, bool side_by_side)
 {
     const size_t bytes = size_t(A.a.B) * A.a.H * A.a.n * kDHead * elem;
     // Qg gets gradient rows only at global positions.
@@ -94,9 +97,29 @@ int backward_schedule(const BwdArgs &A, size_t elem, cudaStream_t stream, RowsFn
         return kErrCuda;
     int rc = launch_global_rows<T>(A, elem, side->stream);
     const bool joined = cudaEventRecord(side->join, side->stream) == cudaSuccess;
-    if (rc == kOk) rc = band_rows();
-    if (rc == kOk) rc = launch_global_cols<T>(A, stream);
-    if (rc == kOk) rc = band_keys();
+    if (!side_by_side) {
+        if (rc == kOk) rc = band_rows(stream);
+        if (rc == kOk) rc = launch_global_cols<T>(A, stream);
+        if (rc == kOk) rc = band_keys(stream);
+    } else {
+        // The rows' lse comes from the forward (side_by_side, set by the
+        // tensor-core path when A.lse_in is given): with D computed first,
+        // the band rows (dq) and the global-token columns + band keys (dk,
+        // dv) need nothing from one another and run on two streams at once,
+        // so each fills the other's last partial wave of CTAs.
+        if (rc == kOk) rc = launch_row_stats<T>(A, stream);
+        bool joined2 = false;
+        if (rc == kOk && cudaEventRecord(side->fork2, stream) == cudaSuccess &&
+            cudaStreamWaitEvent(side->stream2, side->fork2, 0) == cudaSuccess) {
+            rc = launch_global_cols<T>(A, side->stream2);
+            if (rc == kOk) rc = band_keys(side->stream2);
+            joined2 = cudaEventRecord(side->join2, side->stream2) == cudaSuccess;
+            if (rc == kOk) rc = band_rows(stream);
+            if (!joined2 || cudaStreamWaitEvent(stream, side->join2, 0) != cudaSuccess) rc = kErrCuda;
+        } else if (rc == kOk) {
+            rc = kErrCuda;
+        }
+    }
     // Joined on every path, so a capture of `stream` stays well formed.
     if (!joined || cudaStreamWaitEvent(stream, side->join, 0) != cudaSuccess) return kErrCuda;
     return rc;

@@ -373,13 +373,16 @@ __device__ __forceinline__ void rows_softmax(const Params &p, Smem &sm, const It
     const uint32_t *gb = a.ws.gbits + size_t(it.b) * a.L.nwords;
     const bool active = row_in && bit_at(vb, i) && !bit_at(gb, i);
     const size_t rowoff = (size_t(it.bh) * n + (row_in ? i : 0)) * kDHead;
-    const float D = active ? row_dot(static_cast<const T *>(A.dout) + rowoff,
-                                     static_cast<const T *>(A.out) + rowoff)
-                           : 0.f;
+    // With the forward's lse, the row statistics (lse, D) are already in
+    // A.lse / A.dsum and the keys side may be reading them.
+    const bool one_pass = A.lse_in != nullptr;
+    const float D = one_pass ? A.dsum[size_t(it.bh) * n + (row_in ? i : 0)]
+                    : active ? row_dot(static_cast<const T *>(A.dout) + rowoff,
+                                       static_cast<const T *>(A.out) + rowoff)
+                             : 0.f;
     const int tlo = row - (a.causal ? a.window - 1 : a.half);
     const int thi = row + (a.causal ? 0 : a.half);
     float m = -INFINITY, l = 0.f, lse = INFINITY;
-    const bool one_pass = A.lse_in != nullptr;
     if (one_pass && active) lse = A.lse_in[size_t(it.bh) * n + i];
 
     for (int u = 0; u < (one_pass ? 1 : 2) * it.ntiles; ++u) {
@@ -442,7 +445,7 @@ __device__ __forceinline__ void rows_softmax(const Params &p, Smem &sm, const It
         tmem_ld32(tA1 + 32 * hf, acc);
         if (row_in) store_half_row<T>(static_cast<T *>(A.dq) + rowoff + 32 * hf, acc, inv_sqrt_d);
     }
-    if (row_in) {
+    if (row_in && !one_pass) {
         A.lse[size_t(it.bh) * n + i] = active ? lse : INFINITY;
         A.dsum[size_t(it.bh) * n + i] = D;
     }
@@ -735,9 +738,9 @@ int launch_typed(const BwdArgs &A, CUtensorMapDataType dt, cudaStream_t stream)
     if (!cached(&p.krow, a.k, dt, a.n, BH, false) || !cached(&p.vrow, a.v, dt, a.n, BH, false))
         return kErrCuda;
     p.oob_row = BH * a.n;
-    return backward_schedule<T>(A, sizeof(T), stream,
-                                [&]() { return launch_side<T, false>(p, stream); },
-                                [&]() { return launch_side<T, true>(p, stream); });
+    return backward_schedule<T>(
+        A, sizeof(T), stream, [&](cudaStream_t st) { return launch_side<T, false>(p, st); },
+        [&](cudaStream_t st) { return launch_side<T, true>(p, st); }, A.lse_in != nullptr);
 }
 
 }  // namespace bwdtc
