@@ -910,19 +910,14 @@ int launch_row_stats(const BwdArgs &A, cudaStream_t stream)
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 
-// Global rows (Qg against Kg, Vg) and the Kg/Vg keys: needs only the inputs
-// and the prepared workspace, so it runs beside the band rows.
+// Global rows (Qg against Kg, Vg): needs only the inputs and the prepared
+// workspace, so it runs beside the band rows.
 template <typename T>
-int launch_global_rows(const BwdArgs &A, size_t elem, cudaStream_t stream)
+int launch_global_rows(const BwdArgs &A, cudaStream_t stream)
 {
     using namespace bwd;
     const AttnArgs &a = A.a;
-    const size_t bytes = size_t(a.B) * a.H * a.n * kDHead * elem;
-    if (a.max_global == 0) {
-        if (cudaMemsetAsync(A.dkg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
-        if (cudaMemsetAsync(A.dvg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
-        return kOk;
-    }
+    if (a.max_global == 0) return kOk;
     const int bh = a.B * a.H;
     const int sparts = (a.max_global + kRows - 1) / kRows;
     const size_t mg = size_t(a.max_global);
@@ -932,7 +927,23 @@ int launch_global_rows(const BwdArgs &A, size_t elem, cudaStream_t stream)
     grows_chunk_kernel<T, true><<<bh * sparts * A.nchg, kThreads, 0, stream>>>(A);
     const size_t nfin = size_t(bh) * mg * (kDHead / 4);
     gfinal_kernel<T><<<unsigned((nfin + 255) / 256), 256, 0, stream>>>(A);
-    gkeys_kernel<T><<<bh * ((a.n + kRows - 1) / kRows), kThreads, 0, stream>>>(A);
+    return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+}
+
+// dkg, dvg of every key over the global rows (after launch_global_rows, which
+// leaves the global rows' lse and D); zeros without global tokens.
+template <typename T>
+int launch_global_keys(const BwdArgs &A, size_t elem, cudaStream_t stream)
+{
+    using namespace bwd;
+    const AttnArgs &a = A.a;
+    if (a.max_global == 0) {
+        const size_t bytes = size_t(a.B) * a.H * a.n * kDHead * elem;
+        if (cudaMemsetAsync(A.dkg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
+        if (cudaMemsetAsync(A.dvg, 0, bytes, stream) != cudaSuccess) return kErrCuda;
+        return kOk;
+    }
+    gkeys_kernel<T><<<a.B * a.H * ((a.n + kRows - 1) / kRows), kThreads, 0, stream>>>(A);
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 
@@ -1002,12 +1013,16 @@ int launch_backward_simt(const BwdArgs &A, size_t elem, cudaStream_t stream)
             if (band_ctas > 0) keys_kernel<T><<<band_ctas, kThreads, 0, st>>>(A);
             return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
         },
-        false);
+        [&](cudaStream_t st) { return launch_global_cols<T>(A, st); },
+        [&](cudaStream_t st) { return launch_global_keys<T>(A, elem, st); }, false);
 }
 
-template int launch_global_rows<__half>(const BwdArgs &, size_t, cudaStream_t);
-template int launch_global_rows<__nv_bfloat16>(const BwdArgs &, size_t, cudaStream_t);
-template int launch_global_rows<float>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_global_rows<__half>(const BwdArgs &, cudaStream_t);
+template int launch_global_rows<__nv_bfloat16>(const BwdArgs &, cudaStream_t);
+template int launch_global_rows<float>(const BwdArgs &, cudaStream_t);
+template int launch_global_keys<__half>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_global_keys<__nv_bfloat16>(const BwdArgs &, size_t, cudaStream_t);
+template int launch_global_keys<float>(const BwdArgs &, size_t, cudaStream_t);
 template int launch_global_cols<__half>(const BwdArgs &, cudaStream_t);
 template int launch_global_cols<__nv_bfloat16>(const BwdArgs &, cudaStream_t);
 template int launch_global_cols<float>(const BwdArgs &, cudaStream_t);

@@ -61,10 +61,11 @@ inline void backward_scratch_ptrs(BwdArgs &A, void *scratch, int B, int H, int n
 
 // CUDA-core path: every dtype, any dilations.
 template <typename T> int launch_backward_simt(const BwdArgs &A, size_t elem, cudaStream_t stream);
-// Global rows and Kg/Vg keys (independent of the band), and global tokens as
-// keys of the rows outside their window (after the band rows, before the band
-// keys).
-template <typename T> int launch_global_rows(const BwdArgs &A, size_t elem, cudaStream_t stream);
+// Global rows (independent of the band) and then the Kg/Vg keys over them,
+// and global tokens as keys of the rows outside their window (after the rows'
+// lse and D, before the band keys), on the CUDA cores.
+template <typename T> int launch_global_rows(const BwdArgs &A, cudaStream_t stream);
+template <typename T> int launch_global_keys(const BwdArgs &A, size_t elem, cudaStream_t stream);
 template <typename T> int launch_global_cols(const BwdArgs &A, cudaStream_t stream);
 // lse (from A.lse_in) and D of every band row into A.lse and A.dsum, for the
 // schedule in which the band rows and keys run side by side.
@@ -82,9 +83,10 @@ std::unique_lock<std::mutex> side_stream(SideStream *&out);
 // The backward's order on `stream`: zero dqg; fork the global-row chain onto
 // the side stream; band rows; global-token columns; band keys; join.  Works
 // under stream capture (the side stream joins and leaves with the events).
-template <typename T, typename RowsFn, typename KeysFn>
+template <typename T, typename RowsFn, typename KeysFn, typename GColsFn, typename GKeysFn>
 int backward_schedule(const BwdArgs &A, size_t elem, cudaStream_t stream, RowsFn &&band_rows,
-                      KeysFn &&band_keys, bool side_by_side)
+                      KeysFn &&band_keys, GColsFn &&global_cols, GKeysFn &&global_keys,
+                      bool side_by_side)
 {
     const size_t bytes = size_t(A.a.B) * A.a.H * A.a.n * kDHead * elem;
     // Qg gets gradient rows only at global positions.
@@ -95,11 +97,12 @@ int backward_schedule(const BwdArgs &A, size_t elem, cudaStream_t stream, RowsFn
     if (cudaEventRecord(side->fork, stream) != cudaSuccess ||
         cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess)
         return kErrCuda;
-    int rc = launch_global_rows<T>(A, elem, side->stream);
+    int rc = launch_global_rows<T>(A, side->stream);
+    if (rc == kOk) rc = global_keys(side->stream);
     const bool joined = cudaEventRecord(side->join, side->stream) == cudaSuccess;
     if (!side_by_side) {
         if (rc == kOk) rc = band_rows(stream);
-        if (rc == kOk) rc = launch_global_cols<T>(A, stream);
+        if (rc == kOk) rc = global_cols(stream);
         if (rc == kOk) rc = band_keys(stream);
     } else {
         // The rows' lse comes from the forward (side_by_side, set by the
@@ -111,7 +114,7 @@ int backward_schedule(const BwdArgs &A, size_t elem, cudaStream_t stream, RowsFn
         bool joined2 = false;
         if (rc == kOk && cudaEventRecord(side->fork2, stream) == cudaSuccess &&
             cudaStreamWaitEvent(side->stream2, side->fork2, 0) == cudaSuccess) {
-            rc = launch_global_cols<T>(A, side->stream2);
+            rc = global_cols(side->stream2);
             if (rc == kOk) rc = band_keys(side->stream2);
             joined2 = cudaEventRecord(side->join2, side->stream2) == cudaSuccess;
             if (rc == kOk) rc = band_rows(stream);

@@ -17,9 +17,19 @@
 //              queries that reach them through the window stream past once:
 //              S^T = K Q^T, dP^T = V dO^T, P^T and dS^T from the rows' lse
 //              and D, then dV += P^T dO and dK += dS^T Q.  A global token's
-//              sums over the rows that reach it only as a global key come
-//              from the CUDA-core kernels (A.gkv) and are added at the end.
-// Global rows (Qg, Kg, Vg) run on the CUDA cores (lf_bwd.cu).
+//              sums over the rows that reach it only as a global key (A.gkv)
+//              are added at the end.
+// Two more kinds of item run the keys side's products:
+//   global keys    128 keys of Kg, Vg (every position) stationary; the
+//                  global rows (Qg and dO rows at the global positions)
+//                  stream past: dkg, dvg.  Needs the global rows' lse and D
+//                  (more than 8 tokens; fewer take the CUDA-core kernel).
+//   global columns up to 128 global tokens' K, V rows stationary; a chunk of
+//                  the sequence's Q / dO rows streams past, masked to the
+//                  valid non-global rows that do not reach the token through
+//                  the window; the fp32 sums go atomically into A.gkv (more
+//                  than 8 tokens; fewer take the CUDA-core kernel).
+// The global rows themselves (dqg) run on the CUDA cores (lf_bwd.cu).
 //
 // Every product is kind::f16 with fp32 accumulation in TMEM and the operand
 // forms of the forward kernel: S-type products with both operands K-major in
@@ -60,10 +70,16 @@ constexpr int kWarpMma = 5;
 constexpr uint32_t kTmemCols = 256;
 constexpr int kMaxResidues = 24;
 enum { kTQ = 0, kTK = 1, kTV = 2, kTdO = 3 };
+// Item kinds (template argument of the kernel).
+enum Mode { kRowsMode = 0, kKeysMode = 1, kGKeysMode = 2, kGColsMode = 3 };
+constexpr int kGColRows = 512;           // rows a global-columns item streams
 
 struct Params {
     CUtensorMap res[4][kMaxResidues];   // 64-row tiles of the residue classes of Q, K, V, dO
     CUtensorMap krow, vrow;             // single rows of K and V (global-token columns)
+    CUtensorMap kgt, vgt;               // 64-row tiles of Kg, Vg (global keys items)
+    CUtensorMap qgrow, dorow;           // single rows of Qg, dO (global keys items)
+    CUtensorMap qt, dot;                // 64-row tiles of Q, dO (global columns items)
     BwdArgs A;
     int res_base[kMaxHeads];            // first residue map of head h
     int oob_row;                        // a row past the end of the row maps (reads zeros)
@@ -90,10 +106,42 @@ struct Item {
     int g;        // global tokens of the batch (clamped to max_global)
 };
 
-template <bool kKeys>
+template <int kMode>
 __device__ __forceinline__ Item decode(const AttnArgs &a)
 {
+    constexpr bool kKeys = kMode != kRowsMode;
     Item it;
+    if (kMode == kGKeysMode || kMode == kGColsMode) {
+        const int n = a.n;
+        int rem;
+        if (kMode == kGKeysMode) {
+            const int nkb = (n + kM - 1) / kM;
+            it.bh = blockIdx.x / nkb;
+            rem = blockIdx.x - it.bh * nkb;
+            it.s0 = rem * kM;
+            it.lo = 0;
+        } else {
+            const int sblocks = (a.max_global + kM - 1) / kM;
+            const int chunks = (n + kGColRows - 1) / kGColRows;
+            it.bh = blockIdx.x / (sblocks * chunks);
+            rem = blockIdx.x - it.bh * sblocks * chunks;
+            it.s0 = (rem / chunks) * kM;
+            it.lo = (rem % chunks) * kGColRows;
+        }
+        it.b = it.bh / a.H;
+        it.h = it.bh - it.b * a.H;
+        // Kg / Vg keys are plain positions; the global columns test window
+        // taps with the head's dilation.
+        it.dil = kMode == kGKeysMode ? 1 : a.dil[it.h];
+        it.r = 0;
+        it.n_r = n;
+        it.g = min(a.ws.counts[it.b], a.max_global);
+        it.nband = kMode == kGKeysMode ? (it.g + kN - 1) / kN
+                                       : (min(kGColRows, n - it.lo) + kN - 1) / kN;
+        it.ngc = 0;
+        it.ntiles = it.nband;
+        return it;
+    }
     int tile;
     band_item(a, blockIdx.x, it.b, it.h, it.r, tile);
     it.bh = it.b * a.H + it.h;
@@ -187,21 +235,40 @@ __device__ __forceinline__ void store_half_row(T *dst, const float (&v)[32], flo
 }
 
 // ---------------------------------------------------------------- producer
-template <bool kKeys>
-__device__ __forceinline__ void producer_role(const Params &p, Smem &sm, const Item &it, int lane)
+// Row of the flattened [B*H*n, 64] tensors holding global slot `slot` of
+// the item's (batch, head), or a row past the end (reads zeros).
+__device__ __forceinline__ int global_row(const Params &p, const Item &it, int slot)
 {
     const AttnArgs &a = p.A.a;
-    const int rb = p.res_base[it.h] + it.r;
+    return slot < it.g ? it.bh * a.n + a.ws.gidx[size_t(it.b) * a.n + slot] : p.oob_row;
+}
+
+template <int kMode>
+__device__ __forceinline__ void producer_role(const Params &p, Smem &sm, const Item &it, int lane)
+{
+    constexpr bool kKeys = kMode != kRowsMode;
+    const AttnArgs &a = p.A.a;
+    const int rb = kMode == kRowsMode || kMode == kKeysMode ? p.res_base[it.h] + it.r : 0;
     const int ta1 = kKeys ? kTK : kTQ, ta2 = kKeys ? kTV : kTdO;
     const int tb1 = kKeys ? kTQ : kTK, tb2 = kKeys ? kTdO : kTV;
-    if (lane == 0) {
+    if (kMode == kGColsMode) {
+        // The global tokens' K and V rows, gathered.
+        if (lane == 0) mbar_arrive_expect_tx(&sm.stat_full, 2 * kStatBytes);
+        __syncwarp();
+        for (int rr = lane; rr < kM; rr += 32) {
+            const int y = global_row(p, it, it.s0 + rr);
+            tma_load_2d(sm.a1 + rr * kRowBytes, &p.krow, &sm.stat_full, 0, y);
+            tma_load_2d(sm.a2 + rr * kRowBytes, &p.vrow, &sm.stat_full, 0, y);
+        }
+        __syncwarp();
+    } else if (lane == 0) {
+        const CUtensorMap *m1 = kMode == kGKeysMode ? &p.kgt : &p.res[ta1][rb];
+        const CUtensorMap *m2 = kMode == kGKeysMode ? &p.vgt : &p.res[ta2][rb];
         mbar_arrive_expect_tx(&sm.stat_full, 2 * kStatBytes);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-            tma_load_3d(sm.a1 + hf * kTileBytes, &p.res[ta1][rb], &sm.stat_full, 0,
-                        it.s0 + hf * kN, it.bh);
-            tma_load_3d(sm.a2 + hf * kTileBytes, &p.res[ta2][rb], &sm.stat_full, 0,
-                        it.s0 + hf * kN, it.bh);
+            tma_load_3d(sm.a1 + hf * kTileBytes, m1, &sm.stat_full, 0, it.s0 + hf * kN, it.bh);
+            tma_load_3d(sm.a2 + hf * kTileBytes, m2, &sm.stat_full, 0, it.s0 + hf * kN, it.bh);
         }
     }
     // The rows side streams the tiles twice unless the forward's log-sum-exp
@@ -221,7 +288,22 @@ __device__ __forceinline__ void producer_role(const Params &p, Smem &sm, const I
         const int pass = one_pass ? 1 : u / it.ntiles, t = one_pass ? u : u - it.ntiles * pass;
         const bool need_b2 = kKeys || pass == 1;
         const uint32_t bytes = kTileBytes * (need_b2 ? 2u : 1u);
-        if (t < it.nband) {
+        if (kMode == kGKeysMode) {
+            // The global rows: Qg and dO rows at the global positions.
+            if (lane == 0) mbar_arrive_expect_tx(&sm.full[st], bytes);
+            __syncwarp();
+            for (int rr = lane; rr < kN; rr += 32) {
+                const int y = global_row(p, it, t * kN + rr);
+                tma_load_2d(sm.b1[st] + rr * kRowBytes, &p.qgrow, &sm.full[st], 0, y);
+                tma_load_2d(sm.b2[st] + rr * kRowBytes, &p.dorow, &sm.full[st], 0, y);
+            }
+        } else if (kMode == kGColsMode) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.full[st], bytes);
+                tma_load_3d(sm.b1[st], &p.qt, &sm.full[st], 0, it.lo + t * kN, it.bh);
+                tma_load_3d(sm.b2[st], &p.dot, &sm.full[st], 0, it.lo + t * kN, it.bh);
+            }
+        } else if (t < it.nband) {
             if (lane == 0) {
                 const int y = it.lo + t * kN;
                 mbar_arrive_expect_tx(&sm.full[st], bytes);
@@ -255,10 +337,11 @@ __device__ __forceinline__ void producer_role(const Params &p, Smem &sm, const I
 }
 
 // --------------------------------------------------------------------- MMA
-template <bool kKeys>
+template <int kMode>
 __device__ __forceinline__ void mma_role(const Params &p, Smem &sm, const Item &it, uint32_t tmem,
                                          bool bf16)
 {
+    constexpr bool kKeys = kMode != kRowsMode;
     const AttnArgs &a = p.A.a;
     const uint32_t id_s = make_idesc(kM, kN, bf16, false);
     const uint32_t id_acc = make_idesc(kM, kDHead, bf16, true);
@@ -464,7 +547,7 @@ __device__ __forceinline__ int global_slot(const AttnArgs &a, int b, int j)
     return (hi >= 0 && gl[lo] == j) ? lo : -1;
 }
 
-template <typename T>
+template <typename T, int kMode>
 __device__ __forceinline__ void keys_softmax(const Params &p, Smem &sm, const Item &it,
                                              uint32_t tmem, int tid)
 {
@@ -475,17 +558,25 @@ __device__ __forceinline__ void keys_softmax(const Params &p, Smem &sm, const It
     const uint32_t tT2 = tT1 + 64, tA1 = tT1 + 128, tA2 = tT1 + 192;
     const float sl2 = a.scale_log2;
     const int n = a.n;
+    const size_t mg = size_t(a.max_global);
+    // This thread's key: band keys in residue space, every position of Kg /
+    // Vg, or the global token of slot s0 + tid.
     const int key = it.s0 + tid;
-    const bool key_in = key < it.n_r;
-    const int j = key * it.dil + it.r;
+    const bool key_in = kMode == kGColsMode ? key < it.g : key < it.n_r;
+    const int j = kMode == kGColsMode ? (key_in ? a.ws.gidx[size_t(it.b) * n + key] : 0)
+                                      : key * it.dil + it.r;
     const uint32_t *vb = a.ws.vbits + size_t(it.b) * a.L.nwords;
     const uint32_t *gb = a.ws.gbits + size_t(it.b) * a.L.nwords;
     const bool kvalid = key_in && bit_at(vb, j);
-    // Rows (residue space) that take this key as a window tap.
+    // Band keys: the rows (residue space) that take this key as a window tap.
     const int rlo = a.causal ? key : key - a.half;
     const int rhi = key + (a.causal ? a.window - 1 : a.half);
-    const float *lse = A.lse + size_t(it.bh) * n;
-    const float *dsum = A.dsum + size_t(it.bh) * n;
+    // Global columns: the positions that take token j as a window tap.
+    const int tlo = j - (a.causal ? 0 : a.half * it.dil);
+    const int thi = j + (a.causal ? (a.window - 1) * it.dil : a.half * it.dil);
+    const float *lse = kMode == kGKeysMode ? A.lse_g + size_t(it.bh) * mg : A.lse + size_t(it.bh) * n;
+    const float *dsum = kMode == kGKeysMode ? A.dsum_g + size_t(it.bh) * mg
+                                            : A.dsum + size_t(it.bh) * n;
 
     for (int u = 0; u < it.ntiles; ++u) {
         const int ir0 = it.lo + u * kN;
@@ -496,12 +587,39 @@ __device__ __forceinline__ void keys_softmax(const Params &p, Smem &sm, const It
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
             const int ir = ir0 + 32 * w + lane;
-            const int ii = ir * it.dil + it.r;
-            const bool act = ir < it.n_r && bit_at(vb, ii) && !bit_at(gb, ii);
-            const uint32_t ab = __ballot_sync(0xffffffffu, act);
-            mw[w] = kvalid ? (range_bits(w, rlo - ir0, rhi - ir0) & ab) : 0u;
-            cl[w] = act ? lse[ii] : INFINITY;
-            cd[w] = act ? dsum[ii] : 0.f;
+            if (kMode == kGKeysMode) {
+                // Streamed row = global slot ir: a valid global row takes every
+                // valid key.
+                const bool act = ir < it.g && bit_at(vb, a.ws.gidx[size_t(it.b) * n + ir]);
+                const uint32_t ab = __ballot_sync(0xffffffffu, act);
+                mw[w] = kvalid ? ab : 0u;
+                cl[w] = act ? lse[ir] : INFINITY;
+                cd[w] = act ? dsum[ir] : 0.f;
+            } else if (kMode == kGColsMode) {
+                // Streamed row = position ir: valid non-global rows that are
+                // not window taps of token j (same residue class within the
+                // dilated span).
+                const bool act = ir < n && bit_at(vb, ir) && !bit_at(gb, ir);
+                const uint32_t ab = __ballot_sync(0xffffffffu, act);
+                const int c0 = ir0 + 32 * w;
+                uint32_t taps = range_bits(0, tlo - c0, thi - c0);
+                if (it.dil > 1 && taps) {
+                    uint32_t pat = 0u;
+                    for (int c = ((j - c0) % it.dil + it.dil) % it.dil; c < 32; c += it.dil)
+                        pat |= 1u << c;
+                    taps &= pat;
+                }
+                mw[w] = kvalid ? (ab & ~taps) : 0u;
+                cl[w] = act ? lse[ir] : INFINITY;
+                cd[w] = act ? dsum[ir] : 0.f;
+            } else {
+                const int ii = ir * it.dil + it.r;
+                const bool act = ir < it.n_r && bit_at(vb, ii) && !bit_at(gb, ii);
+                const uint32_t ab = __ballot_sync(0xffffffffu, act);
+                mw[w] = kvalid ? (range_bits(w, rlo - ir0, rhi - ir0) & ab) : 0u;
+                cl[w] = act ? lse[ii] : INFINITY;
+                cd[w] = act ? dsum[ii] : 0.f;
+            }
         }
         if (!warp_wait(&sm.s_full, uint32_t(u) & 1u, &sm.abort_flag, a.ws.status)) return;
         tc_fence_after();
@@ -534,6 +652,39 @@ __device__ __forceinline__ void keys_softmax(const Params &p, Smem &sm, const It
     }
     if (!warp_wait(&sm.acc_full, 0, &sm.abort_flag, a.ws.status)) return;
     tc_fence_after();
+    if (kMode == kGColsMode) {
+        // Sums over this chunk's rows, unscaled dk then dv, into A.gkv.
+        float *dst = A.gkv + (size_t(it.bh) * mg + (key_in ? key : 0)) * (2 * kDHead);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            float dk[32], dv[32];
+            tmem_ld32(tA1 + 32 * hf, dk);
+            tmem_ld32(tA2 + 32 * hf, dv);
+            if (kvalid) {
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    atomicAdd(dst + 32 * hf + x, dk[x]);
+                    atomicAdd(dst + kDHead + 32 * hf + x, dv[x]);
+                }
+            }
+        }
+        return;
+    }
+    if (kMode == kGKeysMode) {
+        const float inv_sqrt_d = sl2 * 0.69314718055994531f;
+        const size_t keyoff = (size_t(it.bh) * n + (key_in ? key : 0)) * kDHead;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            float dk[32], dv[32];
+            tmem_ld32(tA1 + 32 * hf, dk);
+            tmem_ld32(tA2 + 32 * hf, dv);
+            if (key_in) {
+                store_half_row<T>(static_cast<T *>(A.dkg) + keyoff + 32 * hf, dk, inv_sqrt_d);
+                store_half_row<T>(static_cast<T *>(A.dvg) + keyoff + 32 * hf, dv, 1.f);
+            }
+        }
+        return;
+    }
     const int slot = (kvalid && bit_at(gb, j)) ? global_slot(a, it.b, j) : -1;
     const float *gsum = slot >= 0 ? A.gkv + (size_t(it.bh) * a.max_global + slot) * (2 * kDHead)
                                   : nullptr;
@@ -559,13 +710,33 @@ __device__ __forceinline__ void keys_softmax(const Params &p, Smem &sm, const It
 }
 
 // ------------------------------------------------------------------ kernel
-template <typename T, bool kKeys>
+template <typename T, int kMode>
 __global__ void __launch_bounds__(kThreads) bwd_tc_kernel(const __grid_constant__ Params p)
 {
     extern __shared__ uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                          ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Item it = decode<kMode>(p.A.a);
+    // Items without work leave before any barrier or tensor memory is set up:
+    // global columns past the batch's tokens; global keys of a batch without
+    // global tokens store zero gradients.
+    if (kMode == kGColsMode && (it.s0 >= it.g || it.ntiles <= 0)) return;
+    if (kMode == kGKeysMode && it.g == 0) {
+        const int key = it.s0 + int(threadIdx.x);
+        if (threadIdx.x < kM && key < it.n_r) {
+            const size_t off = (size_t(it.bh) * it.n_r + key) * kDHead;
+            float z[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) z[x] = 0.f;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                store_half_row<T>(static_cast<T *>(p.A.dkg) + off + 32 * hf, z, 1.f);
+                store_half_row<T>(static_cast<T *>(p.A.dvg) + off + 32 * hf, z, 1.f);
+            }
+        }
+        return;
+    }
     if (threadIdx.x == 0) {
         mbar_init(&sm.stat_full, 1);
         for (int s = 0; s < kStages; ++s) {
@@ -587,17 +758,16 @@ __global__ void __launch_bounds__(kThreads) bwd_tc_kernel(const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const Item it = decode<kKeys>(p.A.a);
 
     if (warp < 4) {
-        if (kKeys)
-            keys_softmax<T>(p, sm, it, tmem, threadIdx.x);
+        if (kMode != kRowsMode)
+            keys_softmax<T, kMode>(p, sm, it, tmem, threadIdx.x);
         else
             rows_softmax<T>(p, sm, it, tmem, threadIdx.x);
     } else if (warp == kWarpProducer) {
-        producer_role<kKeys>(p, sm, it, lane);
+        producer_role<kMode>(p, sm, it, lane);
     } else {
-        mma_role<kKeys>(p, sm, it, tmem, std::is_same<T, __nv_bfloat16>::value);
+        mma_role<kMode>(p, sm, it, tmem, std::is_same<T, __nv_bfloat16>::value);
         // Every MMA this warp issued has completed once this commit lands.
         tc_commit_elect(&sm.drain);
         __syncwarp();
@@ -684,23 +854,50 @@ bool cached(CUtensorMap *out, const void *base, CUtensorMapDataType dt, int n, i
     return true;
 }
 
-template <typename T, bool kKeys>
+template <typename T, int kMode>
 int launch_side(const Params &p, cudaStream_t stream)
 {
+    const AttnArgs &a = p.A.a;
     const size_t smem = sizeof(Smem) + 1024;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(bwd_tc_kernel<T, kKeys>,
+        if (cudaFuncSetAttribute(bwd_tc_kernel<T, kMode>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(smem)) != cudaSuccess)
             return kErrCuda;
         attr_set[dev] = true;
     }
-    const int grid = p.A.a.B * p.A.a.band_items_per_batch;
-    if (grid > 0) bwd_tc_kernel<T, kKeys><<<grid, kThreads, smem, stream>>>(p);
+    const int BH = a.B * a.H;
+    const int grid =
+        kMode == kGKeysMode   ? BH * ((a.n + kM - 1) / kM)
+        : kMode == kGColsMode ? BH * ((a.max_global + kM - 1) / kM) * ((a.n + kGColRows - 1) / kGColRows)
+                              : a.B * a.band_items_per_batch;
+    if (grid > 0) bwd_tc_kernel<T, kMode><<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+}
+
+// Global tokens as keys of the rows outside their window: the streamed
+// CUDA-core kernel for at most 8 tokens, else the tensor-core items.
+template <typename T>
+int launch_global_cols_tc(const Params &p, cudaStream_t stream)
+{
+    const AttnArgs &a = p.A.a;
+    if (a.max_global <= 8) return launch_global_cols<T>(p.A, stream);
+    const size_t bytes = sizeof(float) * size_t(a.B) * a.H * a.max_global * 2 * kDHead;
+    if (cudaMemsetAsync(p.A.gkv, 0, bytes, stream) != cudaSuccess) return kErrCuda;
+    return launch_side<T, kGColsMode>(p, stream);
+}
+
+// dkg, dvg on the tensor cores for more than 8 global tokens; the CUDA-core
+// kernel (zeros without global tokens) below that, where one 64-row tile of
+// a few real rows per item costs more than it saves.
+template <typename T>
+int launch_global_keys_tc(const Params &p, cudaStream_t stream)
+{
+    if (p.A.a.max_global <= 8) return launch_global_keys<T>(p.A, sizeof(T), stream);
+    return launch_side<T, kGKeysMode>(p, stream);
 }
 
 template <typename T>
@@ -737,10 +934,18 @@ int launch_typed(const BwdArgs &A, CUtensorMapDataType dt, cudaStream_t stream)
     }
     if (!cached(&p.krow, a.k, dt, a.n, BH, false) || !cached(&p.vrow, a.v, dt, a.n, BH, false))
         return kErrCuda;
+    if (a.max_global > 0 &&
+        (!cached(&p.kgt, a.kg, dt, a.n, BH, true) || !cached(&p.vgt, a.vg, dt, a.n, BH, true) ||
+         !cached(&p.qgrow, a.qg, dt, a.n, BH, false) ||
+         !cached(&p.dorow, A.dout, dt, a.n, BH, false) ||
+         !cached(&p.qt, a.q, dt, a.n, BH, true) || !cached(&p.dot, A.dout, dt, a.n, BH, true)))
+        return kErrCuda;
     p.oob_row = BH * a.n;
     return backward_schedule<T>(
-        A, sizeof(T), stream, [&](cudaStream_t st) { return launch_side<T, false>(p, st); },
-        [&](cudaStream_t st) { return launch_side<T, true>(p, st); }, A.lse_in != nullptr);
+        A, sizeof(T), stream, [&](cudaStream_t st) { return launch_side<T, kRowsMode>(p, st); },
+        [&](cudaStream_t st) { return launch_side<T, kKeysMode>(p, st); },
+        [&](cudaStream_t st) { return launch_global_cols_tc<T>(p, st); },
+        [&](cudaStream_t st) { return launch_global_keys_tc<T>(p, st); }, A.lse_in != nullptr);
 }
 
 }  // namespace bwdtc
