@@ -162,10 +162,11 @@ LF_API int lf_attention_forward(lf_dtype dtype, int B, int H, int n, int d_head,
 
 /*
  * lf_attention_forward for training (bf16 / fp16): also writes, for every
- * valid non-global row, its log-sum-exp over its key set in log2 units,
+ * valid row, its log-sum-exp over its key set in log2 units,
  *   lse[b, h, i] = log2( sum_j 2^(s_ij * log2(e) / sqrt(d_head)) ),
- * where s_ij = <q_i, k_j> (the scores of the row's softmax).  The entries of
- * padded rows and of global rows are left as they were.
+ * where s_ij = <q_i, k_j> for a non-global row (window taps and global
+ * tokens) and <qg_i, kg_j> for a global row (every valid key): the scores
+ * of the row's softmax.  The entries of padded rows are left as they were.
  *
  *   lse          device fp32 [B, H, n], 4-byte aligned; NULL is refused.
  * lf_attention_backward_lse reads it instead of recomputing it.  fp32 inputs
@@ -409,9 +410,9 @@ LF_API int lf_attention_backward(lf_dtype dtype, int B, int H, int n, int d_head
                          void *scratch, size_t scratch_bytes, lf_stream_t stream);
 
 /*
- * lf_attention_backward (bf16 / fp16) with the band rows' log-sum-exp taken
- * from lf_attention_forward_lse on the same inputs, instead of a first pass
- * over the keys that recomputes it.
+ * lf_attention_backward (bf16 / fp16) with the rows' log-sum-exp taken from
+ * lf_attention_forward_lse on the same inputs, instead of first passes over
+ * the keys that recompute it (band rows and global rows).
  *
  *   lse          device fp32 [B, H, n] as lf_attention_forward_lse wrote it
  *                for these inputs, 4-byte aligned; NULL is refused.

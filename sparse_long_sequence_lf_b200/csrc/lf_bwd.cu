@@ -661,6 +661,32 @@ __global__ void __launch_bounds__(256) row_stats_kernel(const BwdArgs A)
     }
 }
 
+// The same for the global rows, per (batch*head, global slot): the forward's
+// lse and D into A.lse_g, A.dsum_g (+inf and 0 past the count or padded).
+// One warp per slot, two dimensions per lane.
+template <typename T>
+__global__ void __launch_bounds__(256) global_stats_kernel(const BwdArgs A)
+{
+    const AttnArgs &a = A.a;
+    const size_t mg = size_t(a.max_global);
+    const size_t w = size_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (w >= size_t(a.B) * a.H * mg) return;    // whole warps leave together
+    const int bh = int(w / mg), slot = int(w % mg);
+    const int b = bh / a.H;
+    const int g = min(a.ws.counts[b], a.max_global);
+    const int pos = slot < g ? a.ws.gidx[size_t(b) * a.n + slot] : 0;
+    const bool active = slot < g && bit_at(a.ws.vbits + size_t(b) * a.L.nwords, pos);
+    const size_t off = (size_t(bh) * a.n + pos) * kDHead + 2 * lane;
+    const float2 o = load2(static_cast<const T *>(A.out) + off);
+    const float2 d = load2(static_cast<const T *>(A.dout) + off);
+    const float s = warp_sum(fmaf(d.x, o.x, d.y * o.y));
+    if (lane == 0) {
+        A.lse_g[w] = active ? A.lse_in[size_t(bh) * a.n + pos] : INFINITY;
+        A.dsum_g[w] = active ? s : 0.f;
+    }
+}
+
 // ------------------------------------------------------------ global rows
 // Global rows against every valid key through Qg, Kg, Vg, split into chunks
 // of kGChunk keys: gstats_kernel writes each chunk's (max, sum) of the row's
@@ -723,8 +749,14 @@ __global__ void __launch_bounds__(kThreads) grows_chunk_kernel(const BwdArgs A)
 #pragma unroll
         for (int x = 0; x < kQ; ++x) d = fmaf(dO[x], o[x], d);
         D = quad_sum(d);
-        // Merge the chunks' (max, sum) into the row's log-sum-exp.
-        if (active) {
+        if (A.lse_in) {
+            // The forward's lse and D, as global_stats_kernel left them.
+            if (active) {
+                lse = A.lse_g[size_t(bh) * mg + slot];
+                D = A.dsum_g[size_t(bh) * mg + slot];
+            }
+        } else if (active) {
+            // Merge the chunks' (max, sum) into the row's log-sum-exp.
             float M = -INFINITY;
             for (int c = 0; c < nch; ++c) M = fmaxf(M, part[c * mg + slot].x);
             float L = 0.f;
@@ -785,7 +817,7 @@ __global__ void __launch_bounds__(kThreads) grows_chunk_kernel(const BwdArgs A)
         }
         return;
     }
-    if (chunk == 0 && sg.grp == 0 && qd == 0 && sg.sl < gv) {
+    if (!A.lse_in && chunk == 0 && sg.grp == 0 && qd == 0 && sg.sl < gv) {
         A.lse_g[size_t(bh) * mg + slot] = lse;
         A.dsum_g[size_t(bh) * mg + slot] = D;
     }
@@ -907,6 +939,8 @@ int launch_row_stats(const BwdArgs &A, cudaStream_t stream)
     const size_t rows = size_t(A.a.B) * A.a.H * A.a.n;
     if (rows == 0) return kOk;
     bwd::row_stats_kernel<T><<<unsigned((rows + 31) / 32), 256, 0, stream>>>(A);
+    const size_t slots = size_t(A.a.B) * A.a.H * A.a.max_global;
+    if (slots > 0) bwd::global_stats_kernel<T><<<unsigned((slots + 7) / 8), 256, 0, stream>>>(A);
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 
@@ -923,10 +957,23 @@ int launch_global_rows(const BwdArgs &A, cudaStream_t stream)
     const size_t mg = size_t(a.max_global);
     if (cudaMemsetAsync(A.dqg_acc, 0, sizeof(float) * bh * mg * kDHead, stream) != cudaSuccess)
         return kErrCuda;
-    grows_chunk_kernel<T, false><<<bh * sparts * A.nchg, kThreads, 0, stream>>>(A);
+    // With the forward's lse (A.lse_in: global_stats_kernel has run) the
+    // first pass is not needed.
+    if (!A.lse_in) grows_chunk_kernel<T, false><<<bh * sparts * A.nchg, kThreads, 0, stream>>>(A);
     grows_chunk_kernel<T, true><<<bh * sparts * A.nchg, kThreads, 0, stream>>>(A);
     const size_t nfin = size_t(bh) * mg * (kDHead / 4);
     gfinal_kernel<T><<<unsigned((nfin + 255) / 256), 256, 0, stream>>>(A);
+    return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+}
+
+// dqg of the valid global rows from the fp32 sums in A.dqg_acc.
+template <typename T>
+int launch_global_final(const BwdArgs &A, cudaStream_t stream)
+{
+    using namespace bwd;
+    const AttnArgs &a = A.a;
+    const size_t nfin = size_t(a.B) * a.H * a.max_global * (kDHead / 4);
+    if (nfin > 0) gfinal_kernel<T><<<unsigned((nfin + 255) / 256), 256, 0, stream>>>(A);
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 
@@ -999,9 +1046,12 @@ std::unique_lock<std::mutex> side_stream(SideStream *&out)
 }
 
 template <typename T>
-int launch_backward_simt(const BwdArgs &A, size_t elem, cudaStream_t stream)
+int launch_backward_simt(const BwdArgs &A_in, size_t elem, cudaStream_t stream)
 {
     using namespace bwd;
+    // The CUDA-core path recomputes every log-sum-exp itself.
+    BwdArgs A = A_in;
+    A.lse_in = nullptr;
     const int band_ctas = A.a.B * A.a.band_items_per_batch * kParts;
     return backward_schedule<T>(
         A, elem, stream,
@@ -1013,6 +1063,7 @@ int launch_backward_simt(const BwdArgs &A, size_t elem, cudaStream_t stream)
             if (band_ctas > 0) keys_kernel<T><<<band_ctas, kThreads, 0, st>>>(A);
             return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
         },
+        [&](cudaStream_t st) { return launch_global_rows<T>(A, st); },
         [&](cudaStream_t st) { return launch_global_cols<T>(A, st); },
         [&](cudaStream_t st) { return launch_global_keys<T>(A, elem, st); }, false);
 }
@@ -1020,6 +1071,8 @@ int launch_backward_simt(const BwdArgs &A, size_t elem, cudaStream_t stream)
 template int launch_global_rows<__half>(const BwdArgs &, cudaStream_t);
 template int launch_global_rows<__nv_bfloat16>(const BwdArgs &, cudaStream_t);
 template int launch_global_rows<float>(const BwdArgs &, cudaStream_t);
+template int launch_global_final<__half>(const BwdArgs &, cudaStream_t);
+template int launch_global_final<__nv_bfloat16>(const BwdArgs &, cudaStream_t);
 template int launch_global_keys<__half>(const BwdArgs &, size_t, cudaStream_t);
 template int launch_global_keys<__nv_bfloat16>(const BwdArgs &, size_t, cudaStream_t);
 template int launch_global_keys<float>(const BwdArgs &, size_t, cudaStream_t);

@@ -66,9 +66,12 @@ template <typename T> int launch_backward_simt(const BwdArgs &A, size_t elem, cu
 // lse and D, before the band keys), on the CUDA cores.
 template <typename T> int launch_global_rows(const BwdArgs &A, cudaStream_t stream);
 template <typename T> int launch_global_keys(const BwdArgs &A, size_t elem, cudaStream_t stream);
+// dqg from the fp32 sums in A.dqg_acc (the last step of the global rows).
+template <typename T> int launch_global_final(const BwdArgs &A, cudaStream_t stream);
 template <typename T> int launch_global_cols(const BwdArgs &A, cudaStream_t stream);
-// lse (from A.lse_in) and D of every band row into A.lse and A.dsum, for the
-// schedule in which the band rows and keys run side by side.
+// lse (from A.lse_in) and D of every band row into A.lse and A.dsum, and of
+// every global slot into A.lse_g and A.dsum_g, for the schedule in which the
+// band rows and keys run side by side.
 template <typename T> int launch_row_stats(const BwdArgs &A, cudaStream_t stream);
 
 // A second stream of the current device, with the events that fork work onto
@@ -80,13 +83,18 @@ struct SideStream {
 };
 std::unique_lock<std::mutex> side_stream(SideStream *&out);
 
-// The backward's order on `stream`: zero dqg; fork the global-row chain onto
-// the side stream; band rows; global-token columns; band keys; join.  Works
-// under stream capture (the side stream joins and leaves with the events).
-template <typename T, typename RowsFn, typename KeysFn, typename GColsFn, typename GKeysFn>
+// The backward's order on `stream`: zero dqg; fork the global rows and then
+// the Kg/Vg keys onto the side stream; band rows; global-token columns; band
+// keys; join.  With side_by_side (the tensor-core path given the forward's
+// lse), every row's lse and D are written first (launch_row_stats), the side
+// stream forks after them, and the global-token columns + band keys run on a
+// third stream beside the band rows.  Works under stream capture (the side
+// streams join and leave with the events).
+template <typename T, typename RowsFn, typename KeysFn, typename GRowsFn, typename GColsFn,
+          typename GKeysFn>
 int backward_schedule(const BwdArgs &A, size_t elem, cudaStream_t stream, RowsFn &&band_rows,
-                      KeysFn &&band_keys, GColsFn &&global_cols, GKeysFn &&global_keys,
-                      bool side_by_side)
+                      KeysFn &&band_keys, GRowsFn &&global_rows, GColsFn &&global_cols,
+                      GKeysFn &&global_keys, bool side_by_side)
 {
     const size_t bytes = size_t(A.a.B) * A.a.H * A.a.n * kDHead * elem;
     // Qg gets gradient rows only at global positions.
@@ -94,32 +102,31 @@ int backward_schedule(const BwdArgs &A, size_t elem, cudaStream_t stream, RowsFn
     SideStream *side = nullptr;
     auto lock = side_stream(side);
     if (!side) return kErrCuda;
+    int rc = side_by_side ? launch_row_stats<T>(A, stream) : kOk;
     if (cudaEventRecord(side->fork, stream) != cudaSuccess ||
         cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess)
         return kErrCuda;
-    int rc = launch_global_rows<T>(A, side->stream);
+    if (rc == kOk) rc = global_rows(side->stream);
     if (rc == kOk) rc = global_keys(side->stream);
     const bool joined = cudaEventRecord(side->join, side->stream) == cudaSuccess;
     if (!side_by_side) {
         if (rc == kOk) rc = band_rows(stream);
         if (rc == kOk) rc = global_cols(stream);
         if (rc == kOk) rc = band_keys(stream);
-    } else {
-        // The rows' lse comes from the forward (side_by_side, set by the
-        // tensor-core path when A.lse_in is given): with D computed first,
-        // the band rows (dq) and the global-token columns + band keys (dk,
-        // dv) need nothing from one another and run on two streams at once,
-        // so each fills the other's last partial wave of CTAs.
-        if (rc == kOk) rc = launch_row_stats<T>(A, stream);
+    } else if (rc == kOk) {
+        // The band rows (dq) and the global-token columns + band keys (dk,
+        // dv) need nothing from one another once lse and D are written, so
+        // they run on two streams at once and each fills the other's last
+        // partial wave of CTAs.
         bool joined2 = false;
-        if (rc == kOk && cudaEventRecord(side->fork2, stream) == cudaSuccess &&
+        if (cudaEventRecord(side->fork2, stream) == cudaSuccess &&
             cudaStreamWaitEvent(side->stream2, side->fork2, 0) == cudaSuccess) {
             rc = global_cols(side->stream2);
             if (rc == kOk) rc = band_keys(side->stream2);
             joined2 = cudaEventRecord(side->join2, side->stream2) == cudaSuccess;
             if (rc == kOk) rc = band_rows(stream);
             if (!joined2 || cudaStreamWaitEvent(stream, side->join2, 0) != cudaSuccess) rc = kErrCuda;
-        } else if (rc == kOk) {
+        } else {
             rc = kErrCuda;
         }
     }

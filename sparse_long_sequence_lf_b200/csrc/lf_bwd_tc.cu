@@ -29,7 +29,10 @@
 //                  valid non-global rows that do not reach the token through
 //                  the window; the fp32 sums go atomically into A.gkv (more
 //                  than 8 tokens; fewer take the CUDA-core kernel).
-// The global rows themselves (dqg) run on the CUDA cores (lf_bwd.cu).
+//   global rows    up to 128 global rows' Qg, dO stationary; a chunk of Kg,
+//                  Vg tiles streams past once (the forward's lse): dqg sums
+//                  into A.dqg_acc (more than 8 tokens and the forward's lse;
+//                  otherwise the CUDA-core kernels of lf_bwd.cu).
 //
 // Every product is kind::f16 with fp32 accumulation in TMEM and the operand
 // forms of the forward kernel: S-type products with both operands K-major in
@@ -71,8 +74,19 @@ constexpr uint32_t kTmemCols = 256;
 constexpr int kMaxResidues = 24;
 enum { kTQ = 0, kTK = 1, kTV = 2, kTdO = 3 };
 // Item kinds (template argument of the kernel).
-enum Mode { kRowsMode = 0, kKeysMode = 1, kGKeysMode = 2, kGColsMode = 3 };
+enum Mode { kRowsMode = 0, kKeysMode = 1, kGKeysMode = 2, kGColsMode = 3, kGRowsMode = 4 };
 constexpr int kGColRows = 512;           // rows a global-columns item streams
+constexpr int kGRowKeys = 512;           // keys a global-rows item streams
+// Items whose stationary rows are keys (dK, dV products) ...
+__host__ __device__ constexpr bool keys_side(int mode)
+{
+    return mode == kKeysMode || mode == kGKeysMode || mode == kGColsMode;
+}
+// ... and items that stream their tiles once (the rows' lse is known).
+__device__ __forceinline__ bool single_pass(int mode, const BwdArgs &A)
+{
+    return mode != kRowsMode || A.lse_in != nullptr;
+}
 
 struct Params {
     CUtensorMap res[4][kMaxResidues];   // 64-row tiles of the residue classes of Q, K, V, dO
@@ -109,9 +123,9 @@ struct Item {
 template <int kMode>
 __device__ __forceinline__ Item decode(const AttnArgs &a)
 {
-    constexpr bool kKeys = kMode != kRowsMode;
+    constexpr bool kKeys = keys_side(kMode);
     Item it;
-    if (kMode == kGKeysMode || kMode == kGColsMode) {
+    if (kMode == kGKeysMode || kMode == kGColsMode || kMode == kGRowsMode) {
         const int n = a.n;
         int rem;
         if (kMode == kGKeysMode) {
@@ -121,23 +135,27 @@ __device__ __forceinline__ Item decode(const AttnArgs &a)
             it.s0 = rem * kM;
             it.lo = 0;
         } else {
+            // A block of 128 global slots against a chunk of rows (global
+            // columns) or of Kg / Vg keys (global rows).
+            const int span = kMode == kGColsMode ? kGColRows : kGRowKeys;
             const int sblocks = (a.max_global + kM - 1) / kM;
-            const int chunks = (n + kGColRows - 1) / kGColRows;
+            const int chunks = (n + span - 1) / span;
             it.bh = blockIdx.x / (sblocks * chunks);
             rem = blockIdx.x - it.bh * sblocks * chunks;
             it.s0 = (rem / chunks) * kM;
-            it.lo = (rem % chunks) * kGColRows;
+            it.lo = (rem % chunks) * span;
         }
         it.b = it.bh / a.H;
         it.h = it.bh - it.b * a.H;
         // Kg / Vg keys are plain positions; the global columns test window
         // taps with the head's dilation.
-        it.dil = kMode == kGKeysMode ? 1 : a.dil[it.h];
+        it.dil = kMode == kGColsMode ? a.dil[it.h] : 1;
         it.r = 0;
         it.n_r = n;
         it.g = min(a.ws.counts[it.b], a.max_global);
-        it.nband = kMode == kGKeysMode ? (it.g + kN - 1) / kN
-                                       : (min(kGColRows, n - it.lo) + kN - 1) / kN;
+        it.nband = kMode == kGKeysMode   ? (it.g + kN - 1) / kN
+                   : kMode == kGColsMode ? (min(kGColRows, n - it.lo) + kN - 1) / kN
+                                         : (min(kGRowKeys, n - it.lo) + kN - 1) / kN;
         it.ngc = 0;
         it.ntiles = it.nband;
         return it;
@@ -246,19 +264,22 @@ __device__ __forceinline__ int global_row(const Params &p, const Item &it, int s
 template <int kMode>
 __device__ __forceinline__ void producer_role(const Params &p, Smem &sm, const Item &it, int lane)
 {
-    constexpr bool kKeys = kMode != kRowsMode;
+    constexpr bool kKeys = keys_side(kMode);
     const AttnArgs &a = p.A.a;
     const int rb = kMode == kRowsMode || kMode == kKeysMode ? p.res_base[it.h] + it.r : 0;
     const int ta1 = kKeys ? kTK : kTQ, ta2 = kKeys ? kTV : kTdO;
     const int tb1 = kKeys ? kTQ : kTK, tb2 = kKeys ? kTdO : kTV;
-    if (kMode == kGColsMode) {
-        // The global tokens' K and V rows, gathered.
+    if (kMode == kGColsMode || kMode == kGRowsMode) {
+        // The global tokens' K and V rows, or the global rows' Qg and dO
+        // rows, gathered.
+        const CUtensorMap *m1 = kMode == kGColsMode ? &p.krow : &p.qgrow;
+        const CUtensorMap *m2 = kMode == kGColsMode ? &p.vrow : &p.dorow;
         if (lane == 0) mbar_arrive_expect_tx(&sm.stat_full, 2 * kStatBytes);
         __syncwarp();
         for (int rr = lane; rr < kM; rr += 32) {
             const int y = global_row(p, it, it.s0 + rr);
-            tma_load_2d(sm.a1 + rr * kRowBytes, &p.krow, &sm.stat_full, 0, y);
-            tma_load_2d(sm.a2 + rr * kRowBytes, &p.vrow, &sm.stat_full, 0, y);
+            tma_load_2d(sm.a1 + rr * kRowBytes, m1, &sm.stat_full, 0, y);
+            tma_load_2d(sm.a2 + rr * kRowBytes, m2, &sm.stat_full, 0, y);
         }
         __syncwarp();
     } else if (lane == 0) {
@@ -273,7 +294,7 @@ __device__ __forceinline__ void producer_role(const Params &p, Smem &sm, const I
     }
     // The rows side streams the tiles twice unless the forward's log-sum-exp
     // of the rows is given (pass 1 only).
-    const bool one_pass = kKeys || p.A.lse_in != nullptr;
+    const bool one_pass = single_pass(kMode, p.A);
     const int total = (one_pass ? 1 : 2) * it.ntiles;
     bool armed[kStages] = {};
     uint32_t armed_ph[kStages] = {};
@@ -297,11 +318,14 @@ __device__ __forceinline__ void producer_role(const Params &p, Smem &sm, const I
                 tma_load_2d(sm.b1[st] + rr * kRowBytes, &p.qgrow, &sm.full[st], 0, y);
                 tma_load_2d(sm.b2[st] + rr * kRowBytes, &p.dorow, &sm.full[st], 0, y);
             }
-        } else if (kMode == kGColsMode) {
+        } else if (kMode == kGColsMode || kMode == kGRowsMode) {
+            // Q / dO tiles of the sequence, or Kg / Vg tiles.
             if (lane == 0) {
                 mbar_arrive_expect_tx(&sm.full[st], bytes);
-                tma_load_3d(sm.b1[st], &p.qt, &sm.full[st], 0, it.lo + t * kN, it.bh);
-                tma_load_3d(sm.b2[st], &p.dot, &sm.full[st], 0, it.lo + t * kN, it.bh);
+                tma_load_3d(sm.b1[st], kMode == kGColsMode ? &p.qt : &p.kgt, &sm.full[st], 0,
+                            it.lo + t * kN, it.bh);
+                tma_load_3d(sm.b2[st], kMode == kGColsMode ? &p.dot : &p.vgt, &sm.full[st], 0,
+                            it.lo + t * kN, it.bh);
             }
         } else if (t < it.nband) {
             if (lane == 0) {
@@ -341,7 +365,7 @@ template <int kMode>
 __device__ __forceinline__ void mma_role(const Params &p, Smem &sm, const Item &it, uint32_t tmem,
                                          bool bf16)
 {
-    constexpr bool kKeys = kMode != kRowsMode;
+    constexpr bool kKeys = keys_side(kMode);
     const AttnArgs &a = p.A.a;
     const uint32_t id_s = make_idesc(kM, kN, bf16, false);
     const uint32_t id_acc = make_idesc(kM, kDHead, bf16, true);
@@ -350,7 +374,7 @@ __device__ __forceinline__ void mma_role(const Params &p, Smem &sm, const Item &
     tc_fence_after();
     const uint64_t a1d = make_sdesc(smem_u32(sm.a1), 16, 1024);
     const uint64_t a2d = make_sdesc(smem_u32(sm.a2), 16, 1024);
-    const bool one_pass = kKeys || p.A.lse_in != nullptr;
+    const bool one_pass = single_pass(kMode, p.A);
     const int total = (one_pass ? 1 : 2) * it.ntiles;
     bool first_acc = true;
     for (int u = 0; u < total; ++u) {
@@ -531,6 +555,74 @@ __device__ __forceinline__ void rows_softmax(const Params &p, Smem &sm, const It
     if (row_in && !one_pass) {
         A.lse[size_t(it.bh) * n + i] = active ? lse : INFINITY;
         A.dsum[size_t(it.bh) * n + i] = D;
+    }
+}
+
+// ------------------------------------------------------------- global rows
+// Thread = global slot s0 + tid (its Qg and dO rows stationary); the chunk's
+// Kg / Vg tiles stream past once with the rows' lse and D from
+// global_stats_kernel.  Every valid key of the chunk counts.  dq sums (fp32,
+// unscaled) go atomically into A.dqg_acc; gfinal_kernel scales and stores.
+template <typename T>
+__device__ __forceinline__ void grows_softmax(const Params &p, Smem &sm, const Item &it,
+                                              uint32_t tmem, int tid)
+{
+    const BwdArgs &A = p.A;
+    const AttnArgs &a = A.a;
+    const int warp = tid >> 5, lane = tid & 31;
+    const uint32_t tT1 = tmem + (uint32_t(warp * 32) << 16);
+    const uint32_t tT2 = tT1 + 64, tA1 = tT1 + 128;
+    const float sl2 = a.scale_log2;
+    const int n = a.n;
+    const size_t mg = size_t(a.max_global);
+    const int slot = it.s0 + tid;
+    const uint32_t *vb = a.ws.vbits + size_t(it.b) * a.L.nwords;
+    const bool active = slot < it.g && bit_at(vb, a.ws.gidx[size_t(it.b) * n + slot]);
+    const float lse = active ? A.lse_g[size_t(it.bh) * mg + slot] : INFINITY;
+    const float D = active ? A.dsum_g[size_t(it.bh) * mg + slot] : 0.f;
+
+    for (int u = 0; u < it.ntiles; ++u) {
+        uint32_t mw[2];
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            const int k = it.lo + u * kN + 32 * w + lane;
+            const uint32_t cb = __ballot_sync(0xffffffffu, k < n && bit_at(vb, k));
+            mw[w] = active ? cb : 0u;
+        }
+        if (!warp_wait(&sm.s_full, uint32_t(u) & 1u, &sm.abort_flag, a.ws.status)) return;
+        tc_fence_after();
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            float s[32], dp[32];
+            tmem_ld32(tT1 + 32 * hf, s);
+            tmem_ld32(tT2 + 32 * hf, dp);
+            const uint32_t bits = mw[hf];
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const float p0 = ((bits >> (2 * c)) & 1u) ? ex2(fmaf(s[2 * c], sl2, -lse)) : 0.f;
+                const float p1 =
+                    ((bits >> (2 * c + 1)) & 1u) ? ex2(fmaf(s[2 * c + 1], sl2, -lse)) : 0.f;
+                pk[c] = pack2<T>(p0 * (dp[2 * c] - D), p1 * (dp[2 * c + 1] - D));
+            }
+            tmem_st16(tT2 + 16 * hf, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_full);
+    }
+    if (!warp_wait(&sm.acc_full, 0, &sm.abort_flag, a.ws.status)) return;
+    tc_fence_after();
+    float *dst = A.dqg_acc + (size_t(it.bh) * mg + (active ? slot : 0)) * kDHead;
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        float acc[32];
+        tmem_ld32(tA1 + 32 * hf, acc);
+        if (active) {
+#pragma unroll
+            for (int x = 0; x < 32; ++x) atomicAdd(dst + 32 * hf + x, acc[x]);
+        }
     }
 }
 
@@ -721,7 +813,7 @@ __global__ void __launch_bounds__(kThreads) bwd_tc_kernel(const __grid_constant_
     // Items without work leave before any barrier or tensor memory is set up:
     // global columns past the batch's tokens; global keys of a batch without
     // global tokens store zero gradients.
-    if (kMode == kGColsMode && (it.s0 >= it.g || it.ntiles <= 0)) return;
+    if ((kMode == kGColsMode || kMode == kGRowsMode) && (it.s0 >= it.g || it.ntiles <= 0)) return;
     if (kMode == kGKeysMode && it.g == 0) {
         const int key = it.s0 + int(threadIdx.x);
         if (threadIdx.x < kM && key < it.n_r) {
@@ -760,8 +852,10 @@ __global__ void __launch_bounds__(kThreads) bwd_tc_kernel(const __grid_constant_
     const uint32_t tmem = sm.tmem_base;
 
     if (warp < 4) {
-        if (kMode != kRowsMode)
+        if (keys_side(kMode))
             keys_softmax<T, kMode>(p, sm, it, tmem, threadIdx.x);
+        else if (kMode == kGRowsMode)
+            grows_softmax<T>(p, sm, it, tmem, threadIdx.x);
         else
             rows_softmax<T>(p, sm, it, tmem, threadIdx.x);
     } else if (warp == kWarpProducer) {
@@ -870,9 +964,11 @@ int launch_side(const Params &p, cudaStream_t stream)
         attr_set[dev] = true;
     }
     const int BH = a.B * a.H;
+    const int sblocks = (a.max_global + kM - 1) / kM;
     const int grid =
         kMode == kGKeysMode   ? BH * ((a.n + kM - 1) / kM)
-        : kMode == kGColsMode ? BH * ((a.max_global + kM - 1) / kM) * ((a.n + kGColRows - 1) / kGColRows)
+        : kMode == kGColsMode ? BH * sblocks * ((a.n + kGColRows - 1) / kGColRows)
+        : kMode == kGRowsMode ? BH * sblocks * ((a.n + kGRowKeys - 1) / kGRowKeys)
                               : a.B * a.band_items_per_batch;
     if (grid > 0) bwd_tc_kernel<T, kMode><<<grid, kThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
@@ -888,6 +984,22 @@ int launch_global_cols_tc(const Params &p, cudaStream_t stream)
     const size_t bytes = sizeof(float) * size_t(a.B) * a.H * a.max_global * 2 * kDHead;
     if (cudaMemsetAsync(p.A.gkv, 0, bytes, stream) != cudaSuccess) return kErrCuda;
     return launch_side<T, kGColsMode>(p, stream);
+}
+
+// dqg of the global rows: with the forward's lse and more than 8 global
+// tokens the tensor-core items (one pass, fp32 sums, then gfinal_kernel);
+// otherwise the CUDA-core kernels (which skip their first pass given it).
+template <typename T>
+int launch_global_rows_tc(const Params &p, cudaStream_t stream)
+{
+    const AttnArgs &a = p.A.a;
+    if (a.max_global <= 8 || p.A.lse_in == nullptr) return launch_global_rows<T>(p.A, stream);
+    const size_t mg = size_t(a.max_global), bh = size_t(a.B) * a.H;
+    if (cudaMemsetAsync(p.A.dqg_acc, 0, sizeof(float) * bh * mg * kDHead, stream) != cudaSuccess)
+        return kErrCuda;
+    const int rc = launch_side<T, kGRowsMode>(p, stream);
+    if (rc != kOk) return rc;
+    return launch_global_final<T>(p.A, stream);
 }
 
 // dkg, dvg on the tensor cores for more than 8 global tokens; the CUDA-core
@@ -944,6 +1056,7 @@ int launch_typed(const BwdArgs &A, CUtensorMapDataType dt, cudaStream_t stream)
     return backward_schedule<T>(
         A, sizeof(T), stream, [&](cudaStream_t st) { return launch_side<T, kRowsMode>(p, st); },
         [&](cudaStream_t st) { return launch_side<T, kKeysMode>(p, st); },
+        [&](cudaStream_t st) { return launch_global_rows_tc<T>(p, st); },
         [&](cudaStream_t st) { return launch_global_cols_tc<T>(p, st); },
         [&](cudaStream_t st) { return launch_global_keys_tc<T>(p, st); }, A.lse_in != nullptr);
 }

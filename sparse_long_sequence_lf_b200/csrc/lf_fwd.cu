@@ -964,6 +964,7 @@ __device__ __forceinline__ void merge_global_rows(const AttnArgs &a, int b, int 
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
     store_row<T>(static_cast<T *>(a.out) + (size_t(bh) * a.n + pos) * kDHead, acc, inv);
+    if (a.lse_out && L > 0.f) a.lse_out[size_t(bh) * a.n + pos] = M + log2f(L);
 }
 
 // Per-row results an item's epilogue needs after the softmax has moved on;
@@ -1369,6 +1370,7 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const AttnA
     const int pos = a.ws.gidx[size_t(b) * a.n + slot];
     if (!bit_at(a.ws.vbits + size_t(b) * a.L.nwords, pos)) return;   // padded: zeros elsewhere
     const float inv = L > 0.f ? 1.f / L : 0.f;
+    if (a.lse_out && d0 == 0 && L > 0.f) a.lse_out[size_t(bh) * a.n + pos] = M + log2f(L);
     T *dst = static_cast<T *>(a.out) + (size_t(bh) * a.n + pos) * kDHead + d0;
     uint2 v;
     v.x = pack2<T>(acc[0] * inv, acc[1] * inv);

@@ -165,23 +165,25 @@ LSE_CASES = [c for c in CASES if c.dtype != "f32" and c.name != "n1"] + [
 
 
 def _lse_want(x, wl):
-    """log2 of each valid non-global row's softmax denominator, from the
-    oracle's key sets (fp64): log2 sum_j exp(<q_i, k_j> / 8)."""
-    local, _ = obw.key_masks(x["local_mask"], x["global_mask"], B=wl.B, H=wl.H, n=wl.n,
-                             window=wl.window, dilation=x["dilation"], causal=wl.causal)
-    q = x["q"].double()
-    k = x["k"].double()
-    s = torch.einsum("bhid,bhjd->bhij", q, k) / 8.0
-    m = torch.from_numpy(local)
-    s = s.masked_fill(~m, float("-inf"))
-    rows = m.any(dim=-1)
-    return (torch.logsumexp(s, dim=-1) / np.log(2.0)).numpy(), rows.numpy()
+    """log2 of each valid row's softmax denominator, from the oracle's key
+    sets (fp64): log2 sum_j exp(<q_i, k_j> / 8) for a non-global row and
+    log2 sum_j exp(<qg_i, kg_j> / 8) for a global row."""
+    local, glob = obw.key_masks(x["local_mask"], x["global_mask"], B=wl.B, H=wl.H, n=wl.n,
+                                window=wl.window, dilation=x["dilation"], causal=wl.causal)
+    out, rows = [], []
+    for qn, kn, mk in (("q", "k", local), ("qg", "kg", glob)):
+        s = torch.einsum("bhid,bhjd->bhij", x[qn].double(), x[kn].double()) / 8.0
+        m = torch.from_numpy(mk)
+        out.append((torch.logsumexp(s.masked_fill(~m, float("-inf")), dim=-1)
+                    / np.log(2.0)).numpy())
+        rows.append(m.any(dim=-1).numpy())
+    return out, rows
 
 
 @pytest.mark.parametrize("wl", LSE_CASES, ids=[w.name for w in LSE_CASES])
 def test_backward_with_forward_lse(wl):
-    # The forward writes each valid non-global row's log-sum-exp (log2 units);
-    # the backward given it skips its first pass.  Both against fp64.
+    # The forward writes each valid row's log-sum-exp (log2 units); the
+    # backward given it skips its first passes.  Both against fp64.
     x = make_inputs(wl)
     dout = make_output_grad(wl)
     g = to_dev(x)
@@ -195,13 +197,15 @@ def test_backward_with_forward_lse(wl):
                                   dout.cuda(), workspace=ws, lse=lse, **kw)
     torch.cuda.synchronize()
     assert lf.workspace_status(ws) == 0
-    want, rows = _lse_want(x, wl)
+    (want_b, want_g), (rows_b, rows_g) = _lse_want(x, wl)
     got = lse.cpu().numpy().astype(np.float64)
     isg = (np.zeros((wl.B, wl.n), bool) if x["global_mask"] is None
            else x["global_mask"].numpy().astype(bool))
-    band = rows & ~isg[:, None, :]
-    # The forward's sum uses its 2^x (relative error below 7.5e-5).
-    assert np.all(np.abs(got[band] - want[band]) <= 1e-3), wl.name
+    band = rows_b & ~isg[:, None, :]
+    glob = rows_g & isg[:, None, :]
+    # The forward's sums use its 2^x (relative error below 7.5e-5).
+    assert np.all(np.abs(got[band] - want_b[band]) <= 1e-3), wl.name
+    assert np.all(np.abs(got[glob] - want_g[glob]) <= 1e-3), wl.name + " (global rows)"
     ref = obw.backward(x["q"], x["k"], x["v"], x["qg"], x["kg"], x["vg"], x["local_mask"],
                        x["global_mask"], dout, window=wl.window, dilation=x["dilation"],
                        causal=wl.causal)
