@@ -626,10 +626,19 @@ __global__ void __launch_bounds__(32 * kColWarps) gcols_small_kernel(const BwdAr
 // lse and D = <dO_i, O_i> of every position i of every (batch, head) as the
 // band kernels leave them: the forward's lse and D for a valid non-global
 // row, +inf and 0 otherwise.  Eight threads per row, eight dimensions each.
+template <typename T> __device__ void global_stats(const BwdArgs &A, size_t w, int lane);
+
+// Blocks past the rows' take the global slots (global_stats), so that one
+// launch leaves every statistic.
 template <typename T>
-__global__ void __launch_bounds__(256) row_stats_kernel(const BwdArgs A)
+__global__ void __launch_bounds__(256) row_stats_kernel(const BwdArgs A, unsigned row_blocks)
 {
     const AttnArgs &a = A.a;
+    if (blockIdx.x >= row_blocks) {
+        global_stats<T>(A, size_t(blockIdx.x - row_blocks) * 8 + (threadIdx.x >> 5),
+                        threadIdx.x & 31);
+        return;
+    }
     const size_t rows = size_t(a.B) * a.H * a.n;
     const size_t r = size_t(blockIdx.x) * 32 + (threadIdx.x >> 3);
     const int part = threadIdx.x & 7;
@@ -661,16 +670,14 @@ __global__ void __launch_bounds__(256) row_stats_kernel(const BwdArgs A)
     }
 }
 
-// The same for the global rows, per (batch*head, global slot): the forward's
-// lse and D into A.lse_g, A.dsum_g (+inf and 0 past the count or padded).
-// One warp per slot, two dimensions per lane.
+// The same for the global rows, per (batch*head, global slot) w: the
+// forward's lse and D into A.lse_g, A.dsum_g (+inf and 0 past the count or
+// padded).  One warp per slot, two dimensions per lane.
 template <typename T>
-__global__ void __launch_bounds__(256) global_stats_kernel(const BwdArgs A)
+__device__ void global_stats(const BwdArgs &A, size_t w, int lane)
 {
     const AttnArgs &a = A.a;
     const size_t mg = size_t(a.max_global);
-    const size_t w = size_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
     if (w >= size_t(a.B) * a.H * mg) return;    // whole warps leave together
     const int bh = int(w / mg), slot = int(w % mg);
     const int b = bh / a.H;
@@ -938,9 +945,9 @@ int launch_row_stats(const BwdArgs &A, cudaStream_t stream)
 {
     const size_t rows = size_t(A.a.B) * A.a.H * A.a.n;
     if (rows == 0) return kOk;
-    bwd::row_stats_kernel<T><<<unsigned((rows + 31) / 32), 256, 0, stream>>>(A);
+    const unsigned row_blocks = unsigned((rows + 31) / 32);
     const size_t slots = size_t(A.a.B) * A.a.H * A.a.max_global;
-    if (slots > 0) bwd::global_stats_kernel<T><<<unsigned((slots + 7) / 8), 256, 0, stream>>>(A);
+    bwd::row_stats_kernel<T><<<row_blocks + unsigned((slots + 7) / 8), 256, 0, stream>>>(A, row_blocks);
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 

@@ -618,6 +618,7 @@ __device__ __forceinline__ void grows_softmax(const Params &p, Smem &sm, const I
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
         float acc[32];
+        __syncwarp();
         tmem_ld32(tA1 + 32 * hf, acc);
         if (active) {
 #pragma unroll
@@ -750,6 +751,7 @@ __device__ __forceinline__ void keys_softmax(const Params &p, Smem &sm, const It
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             float dk[32], dv[32];
+            __syncwarp();
             tmem_ld32(tA1 + 32 * hf, dk);
             tmem_ld32(tA2 + 32 * hf, dv);
             if (kvalid) {
@@ -768,6 +770,7 @@ __device__ __forceinline__ void keys_softmax(const Params &p, Smem &sm, const It
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             float dk[32], dv[32];
+            __syncwarp();
             tmem_ld32(tA1 + 32 * hf, dk);
             tmem_ld32(tA2 + 32 * hf, dv);
             if (key_in) {
