@@ -622,6 +622,105 @@ __global__ void __launch_bounds__(32 * kColWarps) gcols_small_kernel(const BwdAr
     }
 }
 
+// Global rows and Kg / Vg keys together for at most G global tokens, given
+// their lse and D (A.lse_g, A.dsum_g from the forward): one pass over the
+// keys computes, per key j and global row s, p = 2^(<qg_s, kg_j> log2e/8 -
+// lse_s) and dS = p (<dO_s, vg_j> - D_s); it stores dkg_j = sum_s dS q_s / 8
+// and dvg_j = sum_s p dO_s, and sums dq_s += dS kg_j into A.dqg_acc (fp32,
+// atomically once per CTA and slot).  One warp per key at a time, lane l
+// holding dimensions 2l, 2l+1; the global rows in registers.
+template <typename T, int G>
+__global__ void __launch_bounds__(32 * kColWarps) gglobal_small_kernel(const BwdArgs A)
+{
+    const AttnArgs &a = A.a;
+    __shared__ __align__(16) float red[kColWarps][G][kDHead];
+    const int n = a.n;
+    const size_t mg = size_t(a.max_global);
+    const int kchunks = (n + kColRows - 1) / kColRows;
+    const int bh = blockIdx.x / kchunks;
+    const int j0 = (blockIdx.x % kchunks) * kColRows;
+    const int b = bh / a.H;
+    const int g = min(a.ws.counts[b], min(a.max_global, G));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
+    const size_t base = size_t(bh) * n * kDHead + 2 * lane;
+    bool act[G];
+    float2 qv[G], ov[G], dq[G];
+    float ls[G], ds[G];
+#pragma unroll
+    for (int s = 0; s < G; ++s) {
+        act[s] = false;
+        qv[s] = ov[s] = dq[s] = make_float2(0.f, 0.f);
+        ls[s] = INFINITY;
+        ds[s] = 0.f;
+        if (s < g) {
+            const int pos = a.ws.gidx[size_t(b) * n + s];
+            if (bit_at(vb, pos)) {
+                act[s] = true;
+                qv[s] = load2(static_cast<const T *>(a.qg) + base + size_t(pos) * kDHead);
+                ov[s] = load2(static_cast<const T *>(A.dout) + base + size_t(pos) * kDHead);
+                ls[s] = A.lse_g[size_t(bh) * mg + s];
+                ds[s] = A.dsum_g[size_t(bh) * mg + s];
+            }
+        }
+    }
+    const float sl2 = a.scale_log2;
+    const float inv_sqrt_d = sl2 * 0.69314718055994531f;
+    const int r0 = j0 + warp * kColRowsPerWarp;
+#pragma unroll 1
+    for (int jb = r0; jb < min(r0 + kColRowsPerWarp, n); jb += 4) {
+        float2 kv[4], vv[4];
+        uint32_t vw[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int jj = min(jb + u, n - 1);
+            vw[u] = vb[jj >> 5];
+            kv[u] = load2(static_cast<const T *>(a.kg) + base + size_t(jj) * kDHead);
+            vv[u] = load2(static_cast<const T *>(a.vg) + base + size_t(jj) * kDHead);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = jb + u;
+            if (j >= n) continue;
+            const bool kvalid = (vw[u] >> (j & 31)) & 1u;
+            float2 dk = make_float2(0.f, 0.f), dv = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int s = 0; s < G; ++s) {
+                if (!act[s] || !kvalid) continue;
+                const float sc = warp_sum(fmaf(qv[s].x, kv[u].x, qv[s].y * kv[u].y));
+                const float dp = warp_sum(fmaf(ov[s].x, vv[u].x, ov[s].y * vv[u].y));
+                const float pr = exp2f(fmaf(sc, sl2, -ls[s]));
+                const float dsc = pr * (dp - ds[s]);
+                dk.x = fmaf(dsc, qv[s].x, dk.x);
+                dk.y = fmaf(dsc, qv[s].y, dk.y);
+                dv.x = fmaf(pr, ov[s].x, dv.x);
+                dv.y = fmaf(pr, ov[s].y, dv.y);
+                dq[s].x = fmaf(dsc, kv[u].x, dq[s].x);
+                dq[s].y = fmaf(dsc, kv[u].y, dq[s].y);
+            }
+            T *dkg = static_cast<T *>(A.dkg) + base + size_t(j) * kDHead;
+            T *dvg = static_cast<T *>(A.dvg) + base + size_t(j) * kDHead;
+            dkg[0] = from_f32<T>(dk.x * inv_sqrt_d);
+            dkg[1] = from_f32<T>(dk.y * inv_sqrt_d);
+            dvg[0] = from_f32<T>(dv.x);
+            dvg[1] = from_f32<T>(dv.y);
+        }
+    }
+#pragma unroll
+    for (int s = 0; s < G; ++s)
+        *reinterpret_cast<float2 *>(&red[warp][s][2 * lane]) = dq[s];
+    __syncthreads();
+    for (int e = threadIdx.x; e < G * kDHead; e += 32 * kColWarps) {
+        const int s = e / kDHead, x = e - s * kDHead;
+        if (s >= g) continue;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kColWarps; ++w) acc += red[w][s][x];
+        if (s < g && bit_at(vb, a.ws.gidx[size_t(b) * n + s]))
+            atomicAdd(A.dqg_acc + (size_t(bh) * mg + s) * kDHead + x, acc);
+    }
+}
+
 // ------------------------------------------------------------ row statistics
 // lse and D = <dO_i, O_i> of every position i of every (batch, head) as the
 // band kernels leave them: the forward's lse and D for a valid non-global
@@ -973,6 +1072,30 @@ int launch_global_rows(const BwdArgs &A, cudaStream_t stream)
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 
+// Global rows and Kg / Vg keys in one streamed pass for at most 8 global
+// tokens, given their lse and D (A.lse_in set: global_stats has run), then
+// dqg from the sums.
+template <typename T>
+int launch_global_small(const BwdArgs &A, cudaStream_t stream)
+{
+    using namespace bwd;
+    const AttnArgs &a = A.a;
+    const size_t bh = size_t(a.B) * a.H, mg = size_t(a.max_global);
+    if (cudaMemsetAsync(A.dqg_acc, 0, sizeof(float) * bh * mg * kDHead, stream) != cudaSuccess)
+        return kErrCuda;
+    const int grid = int(bh) * ((a.n + kColRows - 1) / kColRows);
+    if (a.max_global <= 1)
+        gglobal_small_kernel<T, 1><<<grid, 32 * kColWarps, 0, stream>>>(A);
+    else if (a.max_global <= 2)
+        gglobal_small_kernel<T, 2><<<grid, 32 * kColWarps, 0, stream>>>(A);
+    else if (a.max_global <= 4)
+        gglobal_small_kernel<T, 4><<<grid, 32 * kColWarps, 0, stream>>>(A);
+    else
+        gglobal_small_kernel<T, kSmallG><<<grid, 32 * kColWarps, 0, stream>>>(A);
+    if (cudaGetLastError() != cudaSuccess) return kErrCuda;
+    return launch_global_final<T>(A, stream);
+}
+
 // dqg of the valid global rows from the fp32 sums in A.dqg_acc.
 template <typename T>
 int launch_global_final(const BwdArgs &A, cudaStream_t stream)
@@ -1078,6 +1201,8 @@ int launch_backward_simt(const BwdArgs &A_in, size_t elem, cudaStream_t stream)
 template int launch_global_rows<__half>(const BwdArgs &, cudaStream_t);
 template int launch_global_rows<__nv_bfloat16>(const BwdArgs &, cudaStream_t);
 template int launch_global_rows<float>(const BwdArgs &, cudaStream_t);
+template int launch_global_small<__half>(const BwdArgs &, cudaStream_t);
+template int launch_global_small<__nv_bfloat16>(const BwdArgs &, cudaStream_t);
 template int launch_global_final<__half>(const BwdArgs &, cudaStream_t);
 template int launch_global_final<__nv_bfloat16>(const BwdArgs &, cudaStream_t);
 template int launch_global_keys<__half>(const BwdArgs &, size_t, cudaStream_t);

@@ -68,6 +68,9 @@ template <typename T> int launch_global_rows(const BwdArgs &A, cudaStream_t stre
 template <typename T> int launch_global_keys(const BwdArgs &A, size_t elem, cudaStream_t stream);
 // dqg from the fp32 sums in A.dqg_acc (the last step of the global rows).
 template <typename T> int launch_global_final(const BwdArgs &A, cudaStream_t stream);
+// Global rows and Kg / Vg keys in one streamed pass (at most 8 global
+// tokens, given the forward's lse: after launch_row_stats).
+template <typename T> int launch_global_small(const BwdArgs &A, cudaStream_t stream);
 template <typename T> int launch_global_cols(const BwdArgs &A, cudaStream_t stream);
 // lse (from A.lse_in) and D of every band row into A.lse and A.dsum, and of
 // every global slot into A.lse_g and A.dsum_g, for the schedule in which the

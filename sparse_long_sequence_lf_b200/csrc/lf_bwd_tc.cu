@@ -989,14 +989,17 @@ int launch_global_cols_tc(const Params &p, cudaStream_t stream)
     return launch_side<T, kGColsMode>(p, stream);
 }
 
-// dqg of the global rows: with the forward's lse and more than 8 global
-// tokens the tensor-core items (one pass, fp32 sums, then gfinal_kernel);
-// otherwise the CUDA-core kernels (which skip their first pass given it).
+// dqg of the global rows: with the forward's lse, the tensor-core items for
+// more than 8 global tokens (one pass, fp32 sums, then gfinal_kernel) and
+// the streamed CUDA-core pass over the keys for fewer (which also leaves
+// dkg, dvg); without it the CUDA-core kernels.
 template <typename T>
 int launch_global_rows_tc(const Params &p, cudaStream_t stream)
 {
     const AttnArgs &a = p.A.a;
-    if (a.max_global <= 8 || p.A.lse_in == nullptr) return launch_global_rows<T>(p.A, stream);
+    if (a.max_global == 0) return kOk;
+    if (p.A.lse_in == nullptr) return launch_global_rows<T>(p.A, stream);
+    if (a.max_global <= 8) return launch_global_small<T>(p.A, stream);   // dkg, dvg too
     const size_t mg = size_t(a.max_global), bh = size_t(a.B) * a.H;
     if (cudaMemsetAsync(p.A.dqg_acc, 0, sizeof(float) * bh * mg * kDHead, stream) != cudaSuccess)
         return kErrCuda;
@@ -1011,7 +1014,9 @@ int launch_global_rows_tc(const Params &p, cudaStream_t stream)
 template <typename T>
 int launch_global_keys_tc(const Params &p, cudaStream_t stream)
 {
-    if (p.A.a.max_global <= 8) return launch_global_keys<T>(p.A, sizeof(T), stream);
+    const int mg = p.A.a.max_global;
+    if (mg > 0 && mg <= 8 && p.A.lse_in) return kOk;    // done by launch_global_small
+    if (mg <= 8) return launch_global_keys<T>(p.A, sizeof(T), stream);
     return launch_side<T, kGKeysMode>(p, stream);
 }
 

@@ -123,11 +123,13 @@ def test_backward_rejects_bad_scratch():
                               window=8, max_global=0, workspace=ws, scratch=small)
 
 
+@pytest.mark.parametrize("use_lse", [False, True], ids=["recomputed-lse", "forward-lse"])
 @pytest.mark.parametrize("name", ["bf16-b1h12-n4096-w512-g1", "fp16-b2h16-n4096-w512-g64-pad300"])
-def test_backward_full_size_sampled_heads(name):
-    # The benchmark's workloads at full size through the same call; heads are
-    # independent, so the oracle checks heads 0 and H-1 of every batch element
-    # by element (a few seconds of fp64 each).
+def test_backward_full_size_sampled_heads(name, use_lse):
+    # The benchmark's workloads at full size through the same calls (with the
+    # forward's log-sum-exp, as the benchmark times it, and without); heads
+    # are independent, so the oracle checks heads 0 and H-1 of every batch
+    # element by element (a few seconds of fp64 each).
     from sparse_long_sequence_lf_b200.workloads import WORKLOADS
     wl = WORKLOADS[name]
     x = make_inputs(wl)
@@ -136,10 +138,12 @@ def test_backward_full_size_sampled_heads(name):
     mg = max_global_of(x)
     ws = lf.new_workspace(wl.B, wl.H, wl.n, mg, "cuda")
     kw = dict(window=wl.window, dilation=x["dilation"], causal=wl.causal, max_global=mg)
+    lse = (torch.empty((wl.B, wl.H, wl.n), dtype=torch.float32, device="cuda") if use_lse
+           else None)
     out = lf.attention_forward(g["q"], g["k"], g["v"], g["qg"], g["kg"], g["vg"],
-                               g["local_mask"], g["global_mask"], workspace=ws, **kw)
+                               g["local_mask"], g["global_mask"], workspace=ws, lse=lse, **kw)
     grads = lf.attention_backward(g["q"], g["k"], g["v"], g["qg"], g["kg"], g["vg"], out,
-                                  dout.cuda(), workspace=ws, **kw)
+                                  dout.cuda(), workspace=ws, lse=lse, **kw)
     torch.cuda.synchronize()
     assert lf.workspace_status(ws) == 0
     tol = TOL[wl.dtype]
