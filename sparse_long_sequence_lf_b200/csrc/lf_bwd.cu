@@ -856,7 +856,7 @@ __global__ void __launch_bounds__(kThreads) grows_chunk_kernel(const BwdArgs A)
         for (int x = 0; x < kQ; ++x) d = fmaf(dO[x], o[x], d);
         D = quad_sum(d);
         if (A.lse_in) {
-            // The forward's lse and D, as global_stats_kernel left them.
+            // The forward's lse and D, as row_stats_kernel left them.
             if (active) {
                 lse = A.lse_g[size_t(bh) * mg + slot];
                 D = A.dsum_g[size_t(bh) * mg + slot];
@@ -1063,7 +1063,7 @@ int launch_global_rows(const BwdArgs &A, cudaStream_t stream)
     const size_t mg = size_t(a.max_global);
     if (cudaMemsetAsync(A.dqg_acc, 0, sizeof(float) * bh * mg * kDHead, stream) != cudaSuccess)
         return kErrCuda;
-    // With the forward's lse (A.lse_in: global_stats_kernel has run) the
+    // With the forward's lse (A.lse_in: row_stats_kernel has run) the
     // first pass is not needed.
     if (!A.lse_in) grows_chunk_kernel<T, false><<<bh * sparts * A.nchg, kThreads, 0, stream>>>(A);
     grows_chunk_kernel<T, true><<<bh * sparts * A.nchg, kThreads, 0, stream>>>(A);

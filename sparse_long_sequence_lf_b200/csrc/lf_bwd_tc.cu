@@ -561,7 +561,7 @@ __device__ __forceinline__ void rows_softmax(const Params &p, Smem &sm, const It
 // ------------------------------------------------------------- global rows
 // Thread = global slot s0 + tid (its Qg and dO rows stationary); the chunk's
 // Kg / Vg tiles stream past once with the rows' lse and D from
-// global_stats_kernel.  Every valid key of the chunk counts.  dq sums (fp32,
+// row_stats_kernel.  Every valid key of the chunk counts.  dq sums (fp32,
 // unscaled) go atomically into A.dqg_acc; gfinal_kernel scales and stores.
 template <typename T>
 __device__ __forceinline__ void grows_softmax(const Params &p, Smem &sm, const Item &it,
