@@ -458,7 +458,10 @@ def run_e2e(args, wl, device, stream, max_global):
     e.record(stream)
     torch.cuda.synchronize(device)
     ms = s.elapsed_time(e) / steps
-    h2d = sum(t.numel() * t.element_size() for t in pin.values() if torch.is_tensor(t))
+    # The bytes the call copies in: Q, K, V, the masks, and Kg, Vg and the
+    # global rows of Qg when there are global tokens (lf_host_copy_bytes).
+    h2d = lf.host_copy_bytes(pin["q"].dtype, wl.B, wl.H, wl.n, pin["local_mask"],
+                             pin["global_mask"])
     d2h = out.numel() * out.element_size()
     return {"value": round(accounting.useful_flops(wl) / (ms * 1e-3) / 1e12, 4), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),

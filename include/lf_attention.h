@@ -181,10 +181,12 @@ LF_API int lf_attention_forward_lse(lf_dtype dtype, int B, int H, int n, int d_h
                              lf_stream_t stream);
 
 /*
- * The whole forward from HOST buffers: copies the six projections and the
- * masks from host memory (pinned memory makes the copies asynchronous) into
+ * The whole forward from HOST buffers: copies the projections and the masks
+ * from host memory (pinned memory makes the copies asynchronous) into
  * caller-provided device staging buffers, runs lf_attention_forward, copies
- * the output back to host memory and synchronises the stream.
+ * the output back to host memory and synchronises the stream.  Qg, Kg and Vg
+ * are copied only when the global mask has a global position (the kernels
+ * read them only then).  lf_host_copy_bytes returns the bytes copied in.
  *
  *   h_q ... h_vg    host [B, H, n, d_head] of dtype.
  *   h_local_mask, h_global_mask   host uint8 [B, n] or NULL.
@@ -197,6 +199,11 @@ LF_API int lf_attention_forward_lse(lf_dtype dtype, int B, int H, int n, int d_h
  * word of the workspace.
  */
 LF_API size_t lf_host_staging_size(lf_dtype dtype, int B, int H, int n, int d_head);
+/* Host-to-device bytes lf_attention_forward_host copies for these arguments
+ * (h_local_mask, h_global_mask: the host masks it will be given, or NULL);
+ * 0 for unsupported sizes.  Reads the global mask on the host. */
+LF_API size_t lf_host_copy_bytes(lf_dtype dtype, int B, int H, int n, int d_head,
+                                 const uint8_t *h_local_mask, const uint8_t *h_global_mask);
 LF_API int lf_attention_forward_host(lf_dtype dtype, int B, int H, int n, int d_head,
                               const void *h_q, const void *h_k, const void *h_v,
                               const void *h_qg, const void *h_kg, const void *h_vg,

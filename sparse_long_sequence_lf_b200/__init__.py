@@ -9,14 +9,15 @@ is missing.
 from .api import (attention_backward, attention_forward, attention_forward_host,
                   attention_forward_static, attention_prepare, attention_run,
                   backward_scratch_size, encoder_forward, encoder_workspace_size, ffn_block,
-                  ffn_workspace_size, global_index, host_staging_size, new_workspace,
-                  output_layer, output_workspace_size, qkv_projection, scratch_status,
+                  ffn_workspace_size, global_index, host_copy_bytes, host_staging_size,
+                  new_workspace, output_layer, output_workspace_size, qkv_projection, scratch_status,
                   workspace_size, workspace_status)
 from ._lib import LfError
 
 __all__ = ["attention_backward", "attention_forward", "attention_forward_host",
            "attention_forward_static", "attention_prepare", "attention_run",
            "backward_scratch_size", "encoder_forward", "encoder_workspace_size", "ffn_block",
-           "ffn_workspace_size", "global_index", "host_staging_size", "new_workspace",
+           "ffn_workspace_size", "global_index", "host_copy_bytes", "host_staging_size",
+           "new_workspace",
            "output_layer", "output_workspace_size", "qkv_projection", "scratch_status",
            "workspace_size", "workspace_status", "LfError"]

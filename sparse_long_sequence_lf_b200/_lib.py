@@ -67,6 +67,7 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         "lf_attention_forward": (I, [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P, I, P, P,
                                      Z, P]),
         "lf_host_staging_size": (Z, [I, I, I, I, I]),
+        "lf_host_copy_bytes": (Z, [I, I, I, I, I, P, P]),
         "lf_attention_forward_host": (I, [I, I, I, I, I, P, P, P, P, P, P, P, P, I, I, P, I, P,
                                           P, Z, P, Z, P]),
         "lf_workspace_status": (I, [P, P]),

@@ -178,6 +178,18 @@ def host_staging_size(dtype: torch.dtype, B: int, H: int, n: int) -> int:
     return int(_lib.lib().lf_host_staging_size(_DTYPES[dtype], B, H, n, D_HEAD))
 
 
+def host_copy_bytes(dtype: torch.dtype, B: int, H: int, n: int, local_mask=None,
+                    global_mask=None) -> int:
+    """Host-to-device bytes attention_forward_host copies for these host masks
+    (only what the kernels read; see lf_host_copy_bytes)."""
+    for m in (local_mask, global_mask):
+        if m is not None and (m.is_cuda or m.dtype not in (torch.uint8, torch.bool)
+                              or tuple(m.shape) != (B, n) or not m.is_contiguous()):
+            raise ValueError("host masks must be contiguous uint8 CPU tensors of shape [B, n]")
+    return int(_lib.lib().lf_host_copy_bytes(_DTYPES[dtype], B, H, n, D_HEAD, _ptr(local_mask),
+                                             _ptr(global_mask)))
+
+
 def attention_forward_host(q, k, v, qg, kg, vg, local_mask=None, global_mask=None, *, window,
                            dilation=None, causal=False, max_global, out, staging, workspace,
                            stream=None):

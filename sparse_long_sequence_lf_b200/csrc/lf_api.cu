@@ -260,6 +260,31 @@ size_t lf_host_staging_size(lf_dtype dtype, int B, int H, int n, int d_head)
     return 7 * t + 2 * m;
 }
 
+namespace {
+
+// What lf_attention_forward_host copies from the host: Q, K, V in full, and
+// Qg, Kg, Vg in full when the global mask has a global position (the kernels
+// read them only then).  Copying only Qg's global rows was measured slower:
+// small strided copies from host memory cost more than the bytes they save.
+bool has_global_token(const uint8_t *h_global_mask, int B, int n)
+{
+    if (!h_global_mask) return false;
+    for (size_t i = 0; i < size_t(B) * n; ++i)
+        if (h_global_mask[i]) return true;
+    return false;
+}
+
+}  // namespace
+
+size_t lf_host_copy_bytes(lf_dtype dtype, int B, int H, int n, int d_head,
+                          const uint8_t *h_local_mask, const uint8_t *h_global_mask)
+{
+    if (lf_host_staging_size(dtype, B, H, n, d_head) == 0) return 0;
+    const size_t tb = size_t(B) * H * n * kDHead * elem_size(dtype);
+    const size_t masks = (h_local_mask ? size_t(B) * n : 0) + (h_global_mask ? size_t(B) * n : 0);
+    return (has_global_token(h_global_mask, B, n) ? 6 : 3) * tb + masks;
+}
+
 int lf_attention_forward_host(lf_dtype dtype, int B, int H, int n, int d_head, const void *h_q,
                               const void *h_k, const void *h_v, const void *h_qg,
                               const void *h_kg, const void *h_vg, const uint8_t *h_local_mask,
@@ -279,8 +304,10 @@ int lf_attention_forward_host(lf_dtype dtype, int B, int H, int n, int d_head, c
     const size_t mb = size_t(B) * n;
     const size_t m = lf_align256(mb);
     char *base = static_cast<char *>(d_staging);
+    // Without a global token the kernels read no Qg, Kg, Vg.
+    const int ntensors = has_global_token(h_global_mask, B, n) ? 6 : 3;
     const void *src[6] = {h_q, h_k, h_v, h_qg, h_kg, h_vg};
-    for (int i = 0; i < 6; ++i)
+    for (int i = 0; i < ntensors; ++i)
         if (cudaMemcpyAsync(base + i * t, src[i], tb, cudaMemcpyHostToDevice, s) != cudaSuccess)
             return LF_ERR_CUDA;
     uint8_t *d_lm = nullptr, *d_gm = nullptr;

@@ -169,3 +169,18 @@ def test_ffn_and_encoder_argument_checks(L):
     assert enc(wsb=16) == -3
     if not torch.cuda.is_available():
         assert enc() == -7
+
+
+def test_host_copy_bytes_counts_only_what_the_kernels_read():
+    # Q, K, V always; Qg, Kg, Vg only when the global mask has a global token.
+    import torch
+    from sparse_long_sequence_lf_b200 import host_copy_bytes
+    B, H, n = 2, 3, 500
+    tb = B * H * n * 64 * 2
+    assert host_copy_bytes(torch.bfloat16, B, H, n) == 3 * tb
+    lm = torch.ones(B, n, dtype=torch.uint8)
+    gm = torch.zeros(B, n, dtype=torch.uint8)
+    assert host_copy_bytes(torch.bfloat16, B, H, n, lm, gm) == 3 * tb + 2 * B * n
+    gm[1, 499] = 1
+    assert host_copy_bytes(torch.bfloat16, B, H, n, lm, gm) == 6 * tb + 2 * B * n
+    assert host_copy_bytes(torch.float32, B, H, n, None, gm) == 12 * tb + B * n

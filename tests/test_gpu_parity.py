@@ -206,18 +206,23 @@ def test_global_overflow_is_reported():
     torch.cuda.synchronize()
 
 
-def test_host_entry_matches_device_entry():
-    wl = Workload("host", "bf16", 1, 2, 1500, 256, globals_kind="first:3", pad_tail=(10,),
+@pytest.mark.parametrize("globals_kind", ["first:3", "random:20", "random:150", "none"])
+def test_host_entry_matches_device_entry(globals_kind):
+    # The host path copies Qg, Kg, Vg only with global tokens; the staging
+    # buffer starts as 0xFF bytes (NaN for bf16), so a read of anything not
+    # copied shows in the output.
+    wl = Workload("host", "bf16", 2, 2, 1500, 256, globals_kind=globals_kind, pad_tail=(10, 0),
                   seed=8)
     x = make_inputs(wl)
     dev_out = gpu_forward(x).cpu()
+    mg = max_global_of(x)
     pin = {k: (v.pin_memory() if torch.is_tensor(v) else v) for k, v in x.items()}
     host_out = torch.empty_like(pin["q"]).pin_memory()
-    staging = torch.empty(lf.host_staging_size(torch.bfloat16, 1, 2, 1500), dtype=torch.uint8,
-                          device="cuda")
-    ws = lf.new_workspace(1, 2, 1500, 3)
+    staging = torch.full((lf.host_staging_size(torch.bfloat16, 2, 2, 1500),), 0xFF,
+                         dtype=torch.uint8, device="cuda")
+    ws = lf.new_workspace(2, 2, 1500, mg)
     lf.attention_forward_host(pin["q"], pin["k"], pin["v"], pin["qg"], pin["kg"], pin["vg"],
-                              pin["local_mask"], pin["global_mask"], window=256, max_global=3,
+                              pin["local_mask"], pin["global_mask"], window=256, max_global=mg,
                               out=host_out, staging=staging, workspace=ws)
     assert torch.equal(host_out, dev_out)
 
