@@ -532,18 +532,30 @@ __device__ __forceinline__ float warp_sum(float x)
     return x;
 }
 
-template <typename T, int G>
+template <typename T> __device__ void global_stats(const BwdArgs &A, size_t w, int lane);
+
+// kStats (the rows' lse from the forward): the same pass also writes every
+// row's lse and D = <dO_i, O_i> into A.lse, A.dsum (+inf and 0 for padded
+// and global rows), reading the lse from A.lse_in, and the blocks past the
+// rows' write the global slots' statistics (global_stats): one pass leaves
+// everything the band keys and the global parts need.
+template <typename T, int G, bool kStats>
 __global__ void __launch_bounds__(32 * kColWarps) gcols_small_kernel(const BwdArgs A)
 {
     const AttnArgs &a = A.a;
     __shared__ __align__(16) float red[kColWarps][G][2 * kDHead];
     const int n = a.n;
     const int rchunks = (n + kColRows - 1) / kColRows;
+    if (kStats && blockIdx.x >= unsigned(a.B * a.H * rchunks)) {
+        global_stats<T>(A, size_t(blockIdx.x - a.B * a.H * rchunks) * 8 + (threadIdx.x >> 5),
+                        threadIdx.x & 31);
+        return;
+    }
     const int bh = blockIdx.x / rchunks;
     const int i0 = (blockIdx.x % rchunks) * kColRows;
     const int b = bh / a.H, h = bh - b * a.H;
     const int g = min(a.ws.counts[b], min(a.max_global, G));
-    if (g == 0) return;
+    if (!kStats && g == 0) return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t *vb = a.ws.vbits + size_t(b) * a.L.nwords;
     const uint32_t *gb = a.ws.gbits + size_t(b) * a.L.nwords;
@@ -551,7 +563,8 @@ __global__ void __launch_bounds__(32 * kColWarps) gcols_small_kernel(const BwdAr
     const size_t base = size_t(bh) * n * kDHead + 2 * lane;
     const T *Q = static_cast<const T *>(a.q) + base;
     const T *dO = static_cast<const T *>(A.dout) + base;
-    const float *lse = A.lse + size_t(bh) * n;
+    const T *O = static_cast<const T *>(A.out) + base;
+    const float *lse = (kStats ? A.lse_in : A.lse) + size_t(bh) * n;
     const float *dsum = A.dsum + size_t(bh) * n;
 
     int js[G];
@@ -574,7 +587,7 @@ __global__ void __launch_bounds__(32 * kColWarps) gcols_small_kernel(const BwdAr
     const int r0 = i0 + warp * kColRowsPerWarp;
 #pragma unroll 1
     for (int rb = r0; rb < min(r0 + kColRowsPerWarp, n); rb += kB) {
-        float2 qv[kB], ov[kB];
+        float2 qv[kB], ov[kB], oo[kB];
         float lv[kB], dvv[kB];
         uint32_t vw[kB], gw[kB];
 #pragma unroll
@@ -584,13 +597,24 @@ __global__ void __launch_bounds__(32 * kColWarps) gcols_small_kernel(const BwdAr
             gw[u] = gb[ii >> 5];
             qv[u] = load2(Q + size_t(ii) * kDHead);
             ov[u] = load2(dO + size_t(ii) * kDHead);
+            if (kStats) oo[u] = load2(O + size_t(ii) * kDHead);
             lv[u] = lse[ii];
-            dvv[u] = dsum[ii];
+            dvv[u] = kStats ? 0.f : dsum[ii];
         }
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
             const int i = rb + u;
-            if (i >= n || !((vw[u] >> (i & 31)) & 1u) || ((gw[u] >> (i & 31)) & 1u)) continue;
+            if (i >= n) continue;
+            const bool act = ((vw[u] >> (i & 31)) & 1u) && !((gw[u] >> (i & 31)) & 1u);
+            if (kStats) {
+                const float D = warp_sum(fmaf(ov[u].x, oo[u].x, ov[u].y * oo[u].y));
+                dvv[u] = act ? D : 0.f;
+                if (lane == 0) {
+                    A.lse[size_t(bh) * n + i] = act ? lv[u] : INFINITY;
+                    A.dsum[size_t(bh) * n + i] = dvv[u];
+                }
+            }
+            if (!act) continue;
 #pragma unroll
             for (int s = 0; s < G; ++s) {
                 if (s >= g || js[s] < 0 || is_tap(i, js[s], a.window, a.half, dil, a.causal)) continue;
@@ -1042,11 +1066,31 @@ __global__ void __launch_bounds__(kThreads) gkeys_kernel(const BwdArgs A)
 template <typename T>
 int launch_row_stats(const BwdArgs &A, cudaStream_t stream)
 {
-    const size_t rows = size_t(A.a.B) * A.a.H * A.a.n;
+    using namespace bwd;
+    const AttnArgs &a = A.a;
+    const size_t rows = size_t(a.B) * a.H * a.n;
     if (rows == 0) return kOk;
+    const size_t slots = size_t(a.B) * a.H * a.max_global;
+    const unsigned slot_blocks = unsigned((slots + 7) / 8);
+    if (a.max_global > 0 && a.max_global <= kSmallG) {
+        // At most 8 global tokens: the statistics pass also sums the global
+        // columns (gcols_small_kernel<..., true>), so no separate pass
+        // stands between it and the band keys.
+        if (cudaMemsetAsync(A.gkv, 0, sizeof(float) * slots * 2 * kDHead, stream) != cudaSuccess)
+            return kErrCuda;
+        const unsigned grid = unsigned(a.B * a.H * ((a.n + kColRows - 1) / kColRows)) + slot_blocks;
+        if (a.max_global <= 1)
+            gcols_small_kernel<T, 1, true><<<grid, 32 * kColWarps, 0, stream>>>(A);
+        else if (a.max_global <= 2)
+            gcols_small_kernel<T, 2, true><<<grid, 32 * kColWarps, 0, stream>>>(A);
+        else if (a.max_global <= 4)
+            gcols_small_kernel<T, 4, true><<<grid, 32 * kColWarps, 0, stream>>>(A);
+        else
+            gcols_small_kernel<T, kSmallG, true><<<grid, 32 * kColWarps, 0, stream>>>(A);
+        return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
+    }
     const unsigned row_blocks = unsigned((rows + 31) / 32);
-    const size_t slots = size_t(A.a.B) * A.a.H * A.a.max_global;
-    bwd::row_stats_kernel<T><<<row_blocks + unsigned((slots + 7) / 8), 256, 0, stream>>>(A, row_blocks);
+    row_stats_kernel<T><<<row_blocks + slot_blocks, 256, 0, stream>>>(A, row_blocks);
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;
 }
 
@@ -1139,13 +1183,13 @@ int launch_global_cols(const BwdArgs &A, cudaStream_t stream)
         return kErrCuda;
     const int cgrid = bh * ((a.n + kColRows - 1) / kColRows);
     if (a.max_global <= 1)
-        gcols_small_kernel<T, 1><<<cgrid, 32 * kColWarps, 0, stream>>>(A);
+        gcols_small_kernel<T, 1, false><<<cgrid, 32 * kColWarps, 0, stream>>>(A);
     else if (a.max_global <= 2)
-        gcols_small_kernel<T, 2><<<cgrid, 32 * kColWarps, 0, stream>>>(A);
+        gcols_small_kernel<T, 2, false><<<cgrid, 32 * kColWarps, 0, stream>>>(A);
     else if (a.max_global <= 4)
-        gcols_small_kernel<T, 4><<<cgrid, 32 * kColWarps, 0, stream>>>(A);
+        gcols_small_kernel<T, 4, false><<<cgrid, 32 * kColWarps, 0, stream>>>(A);
     else if (a.max_global <= kSmallG)
-        gcols_small_kernel<T, kSmallG><<<cgrid, 32 * kColWarps, 0, stream>>>(A);
+        gcols_small_kernel<T, kSmallG, false><<<cgrid, 32 * kColWarps, 0, stream>>>(A);
     else
         gcols_kernel<T><<<bh * sparts * ((a.n + kGChunk - 1) / kGChunk), kThreads, 0, stream>>>(A);
     return cudaGetLastError() == cudaSuccess ? kOk : kErrCuda;

@@ -983,7 +983,9 @@ template <typename T>
 int launch_global_cols_tc(const Params &p, cudaStream_t stream)
 {
     const AttnArgs &a = p.A.a;
-    if (a.max_global <= 8) return launch_global_cols<T>(p.A, stream);
+    // With the forward's lse and at most 8 tokens the statistics pass has
+    // already summed them (launch_row_stats).
+    if (a.max_global <= 8) return p.A.lse_in ? kOk : launch_global_cols<T>(p.A, stream);
     const size_t bytes = sizeof(float) * size_t(a.B) * a.H * a.max_global * 2 * kDHead;
     if (cudaMemsetAsync(p.A.gkv, 0, bytes, stream) != cudaSuccess) return kErrCuda;
     return launch_side<T, kGColsMode>(p, stream);
